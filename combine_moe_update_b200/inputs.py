@@ -1,0 +1,241 @@
+"""Seeded synthetic workloads for the MoE update-expert / dispatch / combine path.
+
+This module only draws inputs: it holds none of the operators' arithmetic,
+and both the CUDA path and the CPU oracle are fed from it.  Every array is
+numpy; bf16 tensors are returned as ``uint16`` bit patterns (fp32 draws
+rounded to nearest even), everything else in its natural dtype.
+
+Workloads follow the shapes and limits of the operator pages
+(aclnnMoeUpdateExpert, aclnnMoeDistributeDispatchV2,
+aclnnMoeDistributeCombineAddRmsNorm): Bs <= 512, H in [1024, 8192],
+K <= 16, at most 1024 experts / instances.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+
+
+def bf16_bits(a) -> np.ndarray:
+    """fp32 -> bf16 bit patterns, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def bf16_to_f32(b) -> np.ndarray:
+    """bf16 bit patterns -> fp32 values (exact)."""
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+@dataclass
+class Workload:
+    """One MoE layer's inputs.  Shapes: x/residual/shared [bs, H] bf16 bits;
+    expert_ids [bs, K] logical ids; table [num_logical, F]; expert_scales
+    [bs, K] f32; smooth [num_instances, H] f32 or None; expert_out
+    [bs*K, H] bf16 bits (the stand-in for the expert FFN's output rows)."""
+    name: str
+    bs: int
+    hidden: int
+    top_k: int
+    num_logical: int
+    num_instances: int
+    ep_world_size: int
+    quant_mode: int
+    x: np.ndarray
+    expert_ids: np.ndarray
+    expert_scales: np.ndarray
+    table: np.ndarray
+    residual: np.ndarray
+    gamma: np.ndarray
+    norm_eps: float
+    prune_threshold: float = 0.0
+    active_mask: Optional[np.ndarray] = None
+    smooth: Optional[np.ndarray] = None
+    shared_x: Optional[np.ndarray] = None
+    expert_out: Optional[np.ndarray] = None
+    meta: dict = field(default_factory=dict)
+
+
+def identity_table(num_experts: int, ep_world_size: int) -> np.ndarray:
+    """One instance per logical expert, expert e on rank e // L: the mapping
+    is then the identity (instance id == logical id)."""
+    L = num_experts // ep_world_size
+    t = np.empty((num_experts, 2), np.int32)
+    t[:, 0] = 1
+    t[:, 1] = np.arange(num_experts) // L
+    return t
+
+
+def replicated_table(rng, num_logical, replicas, ep_world_size):
+    """Table with ``replicas[e]`` instances of expert e, placed on ranks by a
+    seeded permutation of the rank slots, re-drawn until no two instances of
+    one expert share a rank.  Columns past n_e are padded with -1."""
+    replicas = np.asarray(replicas, np.int64)
+    total = int(replicas.sum())
+    assert total % ep_world_size == 0
+    L = total // ep_world_size
+    F = int(replicas.max()) + 1
+    owners = np.repeat(np.arange(num_logical), replicas)
+    for _ in range(10000):
+        slot_rank = rng.permutation(total) // L
+        ok = True
+        for e in np.nonzero(replicas > 1)[0]:
+            r = slot_rank[owners == e]
+            if len(np.unique(r)) != len(r):
+                ok = False
+                break
+        if ok:
+            break
+    else:  # pragma: no cover
+        raise RuntimeError("could not place replicas")
+    t = np.full((num_logical, F), -1, np.int32)
+    t[:, 0] = replicas
+    fill = np.zeros(num_logical, np.int64)
+    for s in range(total):
+        e = owners[s]
+        t[e, 1 + fill[e]] = slot_rank[s]
+        fill[e] += 1
+    return t
+
+
+def topk_uniform(rng, bs, num_experts, k):
+    """K distinct expert ids per token, uniform without replacement."""
+    return np.argsort(rng.random((bs, num_experts)), axis=1)[:, :k].astype(np.int32)
+
+
+def topk_weighted(rng, bs, popularity, k):
+    """K distinct ids per token drawn one after another without replacement
+    with probabilities proportional to ``popularity`` (Gumbel-top-k)."""
+    logp = np.log(np.asarray(popularity, np.float64))
+    g = rng.gumbel(size=(bs, len(logp)))
+    return np.argsort(-(logp[None, :] + g), axis=1)[:, :k].astype(np.int32)
+
+
+def softmax_scales(rng, bs, k, sigma=1.0):
+    """expertScales: fp32 softmax over K logits drawn ~ N(0, sigma^2)."""
+    z = rng.normal(0.0, sigma, size=(bs, k))
+    z = np.exp(z - z.max(axis=1, keepdims=True))
+    return (z / z.sum(axis=1, keepdims=True)).astype(np.float32)
+
+
+def _common(rng, bs, hidden, top_k, rows):
+    return dict(
+        residual=bf16_bits(rng.standard_normal((bs, hidden), np.float32)),
+        gamma=bf16_bits(rng.uniform(0.5, 1.5, size=hidden).astype(np.float32)),
+        expert_out=bf16_bits(rng.standard_normal((rows, hidden), np.float32)),
+    )
+
+
+def make(name: str, seed: Optional[int] = None, bs: Optional[int] = None) -> Workload:
+    """Build one named workload.  ``seed`` / ``bs`` override the defaults."""
+    spec = dict(WORKLOADS[name])
+    if seed is not None:
+        spec["seed"] = seed
+    if bs is not None:
+        spec["bs"] = bs
+    return spec.pop("builder")(name, **spec)
+
+
+def _uniform_layer(name, seed, bs, hidden, num_experts, top_k, ep_world_size, quant_mode,
+                   smooth=False, shared=False, prune_threshold=0.0, logit_sigma=1.0):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = bf16_bits(rng.standard_normal((bs, hidden), np.float32))
+    ids = topk_uniform(rng, bs, num_experts, top_k)
+    scales = softmax_scales(rng, bs, top_k, logit_sigma)
+    w = Workload(name=name, bs=bs, hidden=hidden, top_k=top_k, num_logical=num_experts,
+                 num_instances=num_experts, ep_world_size=ep_world_size, quant_mode=quant_mode,
+                 x=x, expert_ids=ids, expert_scales=scales,
+                 table=identity_table(num_experts, ep_world_size), norm_eps=1e-6,
+                 prune_threshold=prune_threshold, **_common(rng, bs, hidden, top_k, bs * top_k))
+    if smooth:
+        w.smooth = rng.uniform(0.5, 2.0, size=(num_experts, hidden)).astype(np.float32)
+    if shared:
+        w.shared_x = bf16_bits(rng.standard_normal((bs, hidden), np.float32))
+    return w
+
+
+def _skewed_eplb(name, seed, bs, hidden=4096, num_logical=128, top_k=8, ep_world_size=16,
+                 hot=16, hot_replicas=3, zipf_s=1.2, outlier_p=0.01, outlier_scale=20.0):
+    """Zipf expert popularity (hot = low ids), the hot experts replicated so
+    the instance count divides evenly over the ranks, X with rare outliers,
+    mxfp8 dispatch."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    xf = rng.standard_normal((bs, hidden), np.float32)
+    out = rng.random((bs, hidden)) < outlier_p
+    xf[out] *= np.float32(outlier_scale)
+    pop = (np.arange(num_logical) + 1.0) ** (-zipf_s)
+    ids = topk_weighted(rng, bs, pop, top_k)
+    scales = softmax_scales(rng, bs, top_k)
+    replicas = np.ones(num_logical, np.int64)
+    replicas[:hot] = hot_replicas
+    table = replicated_table(rng, num_logical, replicas, ep_world_size)
+    return Workload(name=name, bs=bs, hidden=hidden, top_k=top_k, num_logical=num_logical,
+                    num_instances=int(replicas.sum()), ep_world_size=ep_world_size, quant_mode=4,
+                    x=bf16_bits(xf), expert_ids=ids, expert_scales=scales, table=table,
+                    norm_eps=1e-6, **_common(rng, bs, hidden, top_k, bs * top_k))
+
+
+WORKLOADS = {
+    # Bs 8, H 1024, 8 experts, K 2, 4 simulated ranks, no quantization.
+    "tiny": dict(builder=_uniform_layer, seed=0, bs=8, hidden=1024, num_experts=8, top_k=2,
+                 ep_world_size=4, quant_mode=0),
+    # Decode batch of a DeepSeek-like layer: 256 experts, K 8, 32 ranks, per-token
+    # int8 with per-expert smooth scales, one shared expert.
+    "deepseek_decode": dict(builder=_uniform_layer, seed=1, bs=256, hidden=7168, num_experts=256,
+                            top_k=8, ep_world_size=32, quant_mode=2, smooth=True, shared=True),
+    # The same layer at the largest batch the pages allow (Bs 512).
+    "deepseek_decode_bs512": dict(builder=_uniform_layer, seed=1, bs=512, hidden=7168,
+                                  num_experts=256, top_k=8, ep_world_size=32, quant_mode=2,
+                                  smooth=True, shared=True),
+    # ... and its unquantized variant (bf16 rows, no smooth, no shared expert).
+    "deepseek_decode_bs512_bf16": dict(builder=_uniform_layer, seed=1, bs=512, hidden=7168,
+                                       num_experts=256, top_k=8, ep_world_size=32, quant_mode=0),
+    # Zipf(1.2) routing over 128 experts, 160 instances on 16 ranks, mxfp8.
+    "skewed_eplb": dict(builder=_skewed_eplb, seed=2, bs=512),
+    # Largest shapes: H 8192, 1024 experts, K 16, 256 ranks, per-128-tile int8,
+    # threshold pruning at 0.05 on softmax weights of N(0, 2) logits.
+    "max_shape": dict(builder=_uniform_layer, seed=3, bs=512, hidden=8192, num_experts=1024,
+                      top_k=16, ep_world_size=256, quant_mode=3, prune_threshold=0.05,
+                      logit_sigma=float(np.sqrt(2.0))),
+}
+
+
+@dataclass
+class LayerStack:
+    """Inputs of L chained MoE layers: X_0, residual_0, and per layer the
+    routing (ids, scales) and gamma.  Layer l+1 takes X = y_l and
+    residual = x_out_l; the expert is the identity (combine reads the rows
+    dispatch wrote)."""
+    bs: int
+    hidden: int
+    top_k: int
+    num_experts: int
+    ep_world_size: int
+    layers: int
+    x0: np.ndarray
+    residual0: np.ndarray
+    expert_ids: list
+    expert_scales: list
+    gammas: list
+    table: np.ndarray
+    norm_eps: float = 1e-6
+
+
+def make_layer_stack(seed=4, layers=32, bs=128, hidden=2048, num_experts=64, top_k=6,
+                     ep_world_size=8) -> LayerStack:
+    rng0 = np.random.Generator(np.random.PCG64([seed, 1000]))
+    x0 = bf16_bits(rng0.standard_normal((bs, hidden), np.float32))
+    r0 = bf16_bits(rng0.standard_normal((bs, hidden), np.float32))
+    ids, scs, gs = [], [], []
+    for l in range(layers):
+        rng = np.random.Generator(np.random.PCG64([seed, l]))
+        ids.append(topk_uniform(rng, bs, num_experts, top_k))
+        scs.append(softmax_scales(rng, bs, top_k))
+        gs.append(bf16_bits(rng.uniform(0.5, 1.5, size=hidden).astype(np.float32)))
+    return LayerStack(bs=bs, hidden=hidden, top_k=top_k, num_experts=num_experts,
+                      ep_world_size=ep_world_size, layers=layers, x0=x0, residual0=r0,
+                      expert_ids=ids, expert_scales=scs, gammas=gs,
+                      table=identity_table(num_experts, ep_world_size))

@@ -1,0 +1,78 @@
+/*
+ * moe_oracle.h -- plain, slow, obviously-correct CPU oracle for the MoE
+ * update-expert / dispatch / combine+Add+RMSNorm path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library includes,
+ * links or calls this code; only the test-suite, the smoke check and the
+ * CPU-baseline leg of the benchmark do.  It shares no code, header, table
+ * or helper with the CUDA path.
+ *
+ * Sources (the operator pages this follows):
+ *   [UE]  aclnnMoeUpdateExpert -- description (load balancing, expert
+ *         pruning) and "Restriction on the shape format" (mapping table).
+ *   [DV2] aclnnMoeDistributeDispatchV2 -- 计算公式 (formulas), cases 1..5
+ *         (quantMode 0..4), and the quantMode constraints section.
+ *   [CAR] aclnnMoeDistributeCombineAddRmsNorm -- 计算公式 (formula) and
+ *         约束说明 item 4 (shape variables).
+ *
+ * Conventions: all arrays are row-major, host memory, caller-owned.
+ * bf16 values travel as their raw 16-bit patterns (uint16_t).
+ * Return values are bit masks of ORC_ERR_* (0 = clean).
+ */
+#ifndef MOE_ORACLE_H
+#define MOE_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ORC_ERR_BAD_ID    1u  /* an expert / instance id outside its range: item dropped */
+#define ORC_ERR_BAD_TABLE 2u  /* mapping table violates its restrictions: every item dropped */
+
+/* Largest fp8 e4m3 finite value and the exponent of its leading bit
+ * (448 = 1.75 * 2^8), used by quantMode 4. */
+#define ORC_E4M3_EMAX 8
+
+/* Step 1: logical expert -> deployed instance, plus pruning.  [UE]
+ * expert_scales and active_mask may be NULL.  prune_threshold <= 0 (or
+ * expert_scales == NULL) disables threshold pruning. */
+uint32_t orc_update_expert(int32_t bs, int32_t top_k, int32_t num_logical,
+                           int32_t table_cols, int32_t ep_world_size,
+                           const int32_t *expert_ids, const float *expert_scales,
+                           const uint8_t *active_mask, float prune_threshold,
+                           const int32_t *table,
+                           int32_t *balanced_ids, uint8_t *balanced_mask);
+
+/* Step 2: order the active (token, k) copies by destination instance and
+ * quantize / copy them into the expert-major receive buffer.  [DV2]
+ * quant_mode: 0 none (bf16 copy), 2 per-token int8, 3 per-128-tile int8,
+ * 4 mxfp8 (e4m3, 32-element blocks, E8M0 scale bytes).
+ * mask, smooth may be NULL.  dyn_scales is ignored for mode 0. */
+uint32_t orc_dispatch(int32_t bs, int32_t hidden, int32_t top_k,
+                      int32_t num_instances, int32_t quant_mode,
+                      const uint16_t *x_bf16, const int32_t *instance_ids,
+                      const uint8_t *mask, const float *smooth,
+                      void *expand_x, void *dyn_scales,
+                      int32_t *expand_idx, int32_t *src_of_row,
+                      int32_t *expert_counts, int32_t *expert_offsets);
+
+/* Step 3: gather, weighted top-K sum plus shared-expert term, residual add
+ * and RMSNorm, all in double.  [CAR]
+ * shared_x, y_bf16, x_out_bf16, rstd, y_f64, x_f64 may be NULL. */
+void orc_combine_add_rmsnorm(int32_t bs, int32_t hidden, int32_t top_k,
+                             const uint16_t *expand_x_bf16, const int32_t *expand_idx,
+                             const float *expert_scales, const uint16_t *shared_x,
+                             const uint16_t *residual_x, const uint16_t *gamma,
+                             double norm_eps,
+                             uint16_t *y_bf16, uint16_t *x_out_bf16, float *rstd,
+                             double *y_f64, double *x_f64);
+
+/* Exposed pieces, so the tests can pin them on their own. */
+uint8_t orc_e4m3_encode(float v);   /* round-to-nearest-even, saturating */
+uint16_t orc_bf16_from_double(double v); /* round-to-nearest-even */
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,162 @@
+"""Python front of the CPU oracle (oracle/moe_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import this module.  It builds
+the C oracle with gcc (``-O2 -fno-fast-math -ffp-contract=off``), loads it
+with ctypes and marshals numpy arrays; all arithmetic lives in the C file.
+It never imports the product package and the product never imports it.
+
+bf16 arrays are numpy ``uint16`` bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_HDR = os.path.join(_HERE, "moe_oracle.h")
+_OUT_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_OUT_DIR, "libmoe_oracle.so")
+CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared"]
+
+ERR_BAD_ID = 1
+ERR_BAD_TABLE = 2
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/_build/libmoe_oracle.so`` if stale."""
+    os.makedirs(_OUT_DIR, exist_ok=True)
+    newest_src = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest_src:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            vp, i32, f32, f64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_double
+            L.orc_update_expert.restype = ctypes.c_uint32
+            L.orc_update_expert.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, f32, vp, vp, vp]
+            L.orc_dispatch.restype = ctypes.c_uint32
+            L.orc_dispatch.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.orc_combine_add_rmsnorm.restype = None
+            L.orc_combine_add_rmsnorm.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, f64,
+                                                  vp, vp, vp, vp, vp]
+            L.orc_e4m3_encode.restype = ctypes.c_uint8
+            L.orc_e4m3_encode.argtypes = [f32]
+            L.orc_bf16_from_double.restype = ctypes.c_uint16
+            L.orc_bf16_from_double.argtypes = [f64]
+            _lib = L
+    return _lib
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def update_expert(expert_ids, table, ep_world_size, expert_scales=None, active_mask=None,
+                  prune_threshold=0.0):
+    """aclnnMoeUpdateExpert: returns (balanced_ids [bs,K] int32, balanced_mask [bs,K] uint8, err)."""
+    ids = _c(expert_ids, np.int32)
+    tab = _c(table, np.int32)
+    bs, k = ids.shape
+    sc = _c(expert_scales, np.float32)
+    am = _c(active_mask, np.uint8)
+    bal = np.empty((bs, k), np.int32)
+    bm = np.empty((bs, k), np.uint8)
+    err = lib().orc_update_expert(bs, k, tab.shape[0], tab.shape[1], int(ep_world_size),
+                                  _p(ids), _p(sc), _p(am), float(prune_threshold), _p(tab),
+                                  _p(bal), _p(bm))
+    return bal, bm, int(err)
+
+
+def dispatch(x_bf16, instance_ids, num_instances, quant_mode, mask=None, smooth=None):
+    """aclnnMoeDistributeDispatchV2 on one simulated source rank.
+
+    Returns a dict: expand_x [bs*K, H] (uint16 bf16 bits for mode 0, int8 for
+    modes 2/3, uint8 e4m3 codes for mode 4), dyn_scales (None for mode 0;
+    [rows] f32, [rows, ceil(H/128)] f32, or [rows, H/32] uint8 E8M0),
+    expand_idx [bs,K], src_of_row [n], counts [E], offsets [E+1], n, err.
+    """
+    x = _c(x_bf16, np.uint16)
+    ids = _c(instance_ids, np.int32)
+    bs, H = x.shape
+    k = ids.shape[1]
+    rows = bs * k
+    m = _c(mask, np.uint8)
+    sm = _c(smooth, np.float32)
+    if quant_mode == 0:
+        ex = np.zeros((rows, H), np.uint16)
+        ds = None
+    elif quant_mode == 2:
+        ex = np.zeros((rows, H), np.int8)
+        ds = np.zeros((rows,), np.float32)
+    elif quant_mode == 3:
+        ex = np.zeros((rows, H), np.int8)
+        ds = np.zeros((rows, (H + 127) // 128), np.float32)
+    elif quant_mode == 4:
+        ex = np.zeros((rows, H), np.uint8)
+        ds = np.zeros((rows, H // 32), np.uint8)
+    else:
+        raise ValueError(f"oracle has no quant_mode {quant_mode}")
+    idx = np.empty((bs, k), np.int32)
+    src = np.full((rows,), -1, np.int32)
+    cnt = np.empty((num_instances,), np.int32)
+    off = np.empty((num_instances + 1,), np.int32)
+    err = lib().orc_dispatch(bs, H, k, int(num_instances), int(quant_mode), _p(x), _p(ids), _p(m),
+                             _p(sm), _p(ex), _p(ds), _p(idx), _p(src), _p(cnt), _p(off))
+    n = int(off[-1])
+    return dict(expand_x=ex, dyn_scales=ds, expand_idx=idx, src_of_row=src[:n], counts=cnt,
+                offsets=off, n=n, err=int(err))
+
+
+def combine_add_rmsnorm(expand_x_bf16, expand_idx, expert_scales, residual_x, gamma, norm_eps,
+                        shared_x=None):
+    """aclnnMoeDistributeCombineAddRmsNorm.  Returns a dict with y / x_out as
+    bf16 bits, their unrounded float64 values, and rstd (float32)."""
+    ex = _c(expand_x_bf16, np.uint16)
+    idx = _c(expand_idx, np.int32)
+    sc = _c(expert_scales, np.float32)
+    res = _c(residual_x, np.uint16)
+    g = _c(gamma, np.uint16)
+    sh = _c(shared_x, np.uint16)
+    bs, k = idx.shape
+    H = res.shape[1]
+    y = np.empty((bs, H), np.uint16)
+    xo = np.empty((bs, H), np.uint16)
+    rstd = np.empty((bs,), np.float32)
+    y64 = np.empty((bs, H), np.float64)
+    x64 = np.empty((bs, H), np.float64)
+    lib().orc_combine_add_rmsnorm(bs, H, k, _p(ex), _p(idx), _p(sc), _p(sh), _p(res), _p(g),
+                                  float(norm_eps), _p(y), _p(xo), _p(rstd), _p(y64), _p(x64))
+    return dict(y=y, x_out=xo, rstd=rstd, y_f64=y64, x_f64=x64)
+
+
+def e4m3_encode(values):
+    """Element-wise oracle e4m3 encoder (slow: one ctypes call per value)."""
+    f = lib().orc_e4m3_encode
+    v = np.asarray(values, np.float32).ravel()
+    return np.array([f(float(t)) for t in v], np.uint8).reshape(np.shape(values))
+
+
+def bf16_from_double(values):
+    f = lib().orc_bf16_from_double
+    v = np.asarray(values, np.float64).ravel()
+    return np.array([f(float(t)) for t in v], np.uint16).reshape(np.shape(values))

@@ -1,0 +1,492 @@
+"""Pins for the CPU oracle, against things other than itself.
+
+Every check here is a hand-derived worked example (tests/golden/), a brute
+force on tiny inputs, a closed form, an invariant the pages imply, or a
+library routine that the special case reduces to.  None of them re-types the
+oracle's own formula.  CPU only.
+"""
+import json
+import math
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+from combine_moe_update_b200 import inputs as gen
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")))
+
+
+def bits(vals):
+    return gen.bf16_bits(np.asarray(vals, np.float32))
+
+
+# --------------------------------------------------------------------------
+# update_expert (aclnnMoeUpdateExpert)
+# --------------------------------------------------------------------------
+
+def test_update_expert_worked_example(orc):
+    g = GOLDEN["update_expert_small"]
+    for case in g["cases"]:
+        am = None if case["active_mask"] is None else np.array(case["active_mask"], np.uint8)
+        bal, bm, err = orc.update_expert(np.array(g["expert_ids"]), np.array(g["table"]),
+                                         g["ep_world_size"],
+                                         expert_scales=np.array(g["expert_scales"], np.float32),
+                                         active_mask=am, prune_threshold=case["prune_threshold"])
+        assert err == 0
+        np.testing.assert_array_equal(bal, g["balanced_ids"])
+        np.testing.assert_array_equal(bm, case["balanced_mask"])
+
+
+@pytest.mark.parametrize("E,ws", [(8, 4), (256, 32), (1024, 256), (64, 8), (12, 3)])
+def test_update_expert_identity_table_is_identity(orc, E, ws):
+    rng = np.random.default_rng(E)
+    ids = gen.topk_uniform(rng, 40, E, min(8, E))
+    bal, bm, err = orc.update_expert(ids, gen.identity_table(E, ws), ws)
+    assert err == 0
+    np.testing.assert_array_equal(bal, ids)
+    assert bm.all()
+
+
+def test_update_expert_replicated_table_invariants(orc):
+    w = gen.make("skewed_eplb")
+    bal, bm, err = orc.update_expert(w.expert_ids, w.table, w.ep_world_size)
+    assert err == 0 and bm.all()
+    N, ws = w.num_instances, w.ep_world_size
+    L = N // ws
+    # the map (e, j) -> instance is a bijection onto [0, N) with L instances per rank
+    seen = {}
+    for e in range(w.num_logical):
+        n = w.table[e, 0]
+        for j in range(n):
+            ids = np.full((1, 1), e, np.int32)
+            # token index i = j routes to replica j (i mod n_e)
+            b, _, _ = orc.update_expert(np.repeat(ids, j + 1, axis=0), w.table, ws)
+            inst = int(b[j, 0])
+            assert inst // L == w.table[e, 1 + j], "instance must live on the table's rank"
+            seen[(e, j)] = inst
+    assert sorted(seen.values()) == list(range(N))
+    # every copy lands on the rank the table names for replica i mod n_e
+    i = np.arange(w.bs)[:, None]
+    n_e = w.table[w.expert_ids, 0]
+    want_rank = w.table[w.expert_ids, 1 + (i % n_e)]
+    np.testing.assert_array_equal(bal // L, want_rank)
+    # instances of one rank are ordered by (logical id, replica)
+    for r in range(ws):
+        pairs = sorted([p for p, v in seen.items() if v // L == r])
+        assert [seen[p] for p in pairs] == list(range(r * L, (r + 1) * L))
+
+
+@pytest.mark.parametrize("bad", ["zero_count", "rank_out_of_range", "uneven", "too_many_cols"])
+def test_update_expert_bad_table_drops_everything(orc, bad):
+    t = gen.identity_table(8, 4).copy()
+    if bad == "zero_count":
+        t[3, 0] = 0
+    elif bad == "rank_out_of_range":
+        t[5, 1] = 4
+    elif bad == "uneven":
+        t[0, 1] = 1           # rank 0 now has 1 instance, rank 1 has 3
+    elif bad == "too_many_cols":
+        t[2, 0] = 2           # n_e must be <= F - 1 = 1
+    ids = np.array([[0, 1], [2, 3]], np.int32)
+    bal, bm, err = orc.update_expert(ids, t, 4)
+    assert err & orc.ERR_BAD_TABLE
+    assert (bal == -1).all() and (bm == 0).all()
+
+
+def test_update_expert_bad_id_drops_only_that_copy(orc):
+    ids = np.array([[0, 9], [-1, 3]], np.int32)
+    bal, bm, err = orc.update_expert(ids, gen.identity_table(8, 4), 4)
+    assert err == orc.ERR_BAD_ID
+    np.testing.assert_array_equal(bal, [[0, -1], [-1, 3]])
+    np.testing.assert_array_equal(bm, [[1, 0], [0, 1]])
+
+
+def test_update_expert_pruning_fraction_max_shape(orc):
+    """Pruned exactly where the weight is strictly below the threshold."""
+    w = gen.make("max_shape")
+    _, bm, err = orc.update_expert(w.expert_ids, w.table, w.ep_world_size,
+                                   expert_scales=w.expert_scales, prune_threshold=w.prune_threshold)
+    assert err == 0
+    np.testing.assert_array_equal(bm == 0, w.expert_scales < np.float32(w.prune_threshold))
+    assert 0.3 < (bm == 0).mean() < 0.7
+
+
+# --------------------------------------------------------------------------
+# dispatch: routing / index part (aclnnMoeDistributeDispatchV2)
+# --------------------------------------------------------------------------
+
+def test_dispatch_index_worked_example(orc):
+    g = GOLDEN["dispatch_index_small"]
+    x = np.zeros((3, 8), np.uint16)
+    for case in g["cases"]:
+        m = None if case["mask"] is None else np.array(case["mask"], np.uint8)
+        out = orc.dispatch(x, np.array(g["instance_ids"]), g["num_instances"], 0, mask=m)
+        assert out["err"] == 0
+        np.testing.assert_array_equal(out["expand_idx"], case["expand_idx"])
+        np.testing.assert_array_equal(out["src_of_row"], case["src_of_row"])
+        np.testing.assert_array_equal(out["counts"], case["counts"])
+        np.testing.assert_array_equal(out["offsets"], case["offsets"])
+
+
+def _brute_rows(ids, mask):
+    """Row of an active copy = number of active copies with a smaller
+    (instance, token, k) key; O(n^2), no sorting."""
+    bs, K = ids.shape
+    i, k = np.meshgrid(np.arange(bs), np.arange(K), indexing="ij")
+    key = np.stack([ids.ravel(), i.ravel(), k.ravel()], 1).astype(np.int64)
+    act = mask.ravel().astype(bool)
+    a, b = key[:, None, :], key[None, :, :]
+    less = (b[..., 0] < a[..., 0]) | ((b[..., 0] == a[..., 0]) & (
+        (b[..., 1] < a[..., 1]) | ((b[..., 1] == a[..., 1]) & (b[..., 2] < a[..., 2]))))
+    rows = (less & act[None, :]).sum(1)
+    return np.where(act, rows, -1).reshape(bs, K)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_dispatch_index_brute_force(orc, seed):
+    rng = np.random.default_rng(100 + seed)
+    bs, K = int(rng.integers(1, 24)), int(rng.integers(1, 5))
+    E = int(rng.integers(K, 17))
+    ids = rng.integers(0, E, size=(bs, K)).astype(np.int32)   # duplicates allowed
+    mask = (rng.random((bs, K)) < 0.7).astype(np.uint8)
+    out = orc.dispatch(np.zeros((bs, 8), np.uint16), ids, E, 0, mask=mask)
+    np.testing.assert_array_equal(out["expand_idx"], _brute_rows(ids, mask))
+    np.testing.assert_array_equal(out["counts"], np.bincount(ids[mask == 1], minlength=E))
+
+
+@pytest.mark.parametrize("name", ["tiny", "deepseek_decode", "skewed_eplb", "max_shape"])
+def test_dispatch_index_invariants(orc, name):
+    w = gen.make(name)
+    bal, bm, err = orc.update_expert(w.expert_ids, w.table, w.ep_world_size,
+                                     expert_scales=w.expert_scales, prune_threshold=w.prune_threshold)
+    out = orc.dispatch(w.x[:, :8].copy(), bal, w.num_instances, 0, mask=bm)
+    idx, src, cnt, off, n = out["expand_idx"], out["src_of_row"], out["counts"], out["offsets"], out["n"]
+    assert n == int(bm.sum()) == int(cnt.sum())
+    if w.prune_threshold == 0:
+        assert n == w.bs * w.top_k
+    assert off[0] == 0 and off[-1] == n and (np.diff(off) == cnt).all()
+    act = np.nonzero(bm.ravel())[0]
+    np.testing.assert_array_equal(np.sort(idx.ravel()[act]), np.arange(n))
+    np.testing.assert_array_equal(src[idx.ravel()[act]], act)
+    assert (idx.ravel()[bm.ravel() == 0] == -1).all()
+    # every bucket holds its instance's copies in increasing (token, k) order
+    for e in range(w.num_instances):
+        seg = src[off[e]:off[e + 1]]
+        assert (np.diff(seg) > 0).all()
+        assert (bal.ravel()[seg] == e).all()
+    # rank r's region is the contiguous rows of instances [r L, (r+1) L)
+    L = w.num_instances // w.ep_world_size
+    rank_of_row = bal.ravel()[src] // L
+    assert (np.diff(rank_of_row) >= 0).all()
+
+
+def test_dispatch_bad_instance_id_dropped(orc):
+    ids = np.array([[0, 5], [2, 3]], np.int32)
+    out = orc.dispatch(np.zeros((2, 8), np.uint16), ids, 4, 0)
+    assert out["err"] == orc.ERR_BAD_ID
+    np.testing.assert_array_equal(out["expand_idx"], [[0, -1], [1, 2]])
+    np.testing.assert_array_equal(out["counts"], [1, 0, 1, 1])
+
+
+def test_dispatch_mode0_copies_rows(orc):
+    w = gen.make("tiny")
+    out = orc.dispatch(w.x, w.expert_ids, w.num_instances, 0)
+    src = out["src_of_row"]
+    np.testing.assert_array_equal(out["expand_x"][: out["n"]], w.x[src // w.top_k])
+
+
+# --------------------------------------------------------------------------
+# dispatch: int8 quantization (quantMode 2 / 3)
+# --------------------------------------------------------------------------
+
+def test_int8_worked_rows(orc):
+    for row in GOLDEN["quant_int8_rows"]["rows"]:
+        x = bits([row["x"]])
+        sm = None if row["smooth"] is None else np.array([row["smooth"]], np.float32)
+        out = orc.dispatch(x, np.zeros((1, 1), np.int32), 1, 2, smooth=sm)
+        np.testing.assert_array_equal(out["expand_x"][0], row["q"])
+        assert out["dyn_scales"][0] == np.float32(row["scale"])
+        if "scale_bits" in row:
+            assert int(out["dyn_scales"][:1].view(np.uint32)[0]) == int(row["scale_bits"], 16)
+
+
+def test_int8_per_tile_worked(orc):
+    """Tile t of a per-tile row behaves like a per-token row on its own
+    128 elements: tile 0 = first worked row, tile 1 = second, last tile
+    partial (H = 264 -> tiles of 128, 128, 8)."""
+    rows = GOLDEN["quant_int8_rows"]["rows"]
+    H = 264
+    x = np.zeros(H, np.float32)
+    x[0:8] = rows[0]["x"]
+    x[128:136] = rows[1]["x"]
+    x[256:264] = rows[2]["x"]
+    out = orc.dispatch(bits([x]), np.zeros((1, 1), np.int32), 1, 3)
+    q, s = out["expand_x"][0], out["dyn_scales"][0]
+    assert s.shape == (3,)
+    np.testing.assert_array_equal(q[0:8], rows[0]["q"])
+    np.testing.assert_array_equal(q[128:136], rows[1]["q"])
+    assert s[0] == 1.0 and s[1] == 2.0
+    # third tile: amax 127 with no smooth -> codes = x rounded, scale 1
+    np.testing.assert_array_equal(q[256:264], np.rint(np.array(rows[2]["x"], np.float64)))
+    assert s[2] == 1.0
+    assert not q[8:128].any() and not q[136:256].any()
+
+
+def _f32(xbits):
+    return gen.bf16_to_f32(xbits).astype(np.float32)
+
+
+@pytest.mark.parametrize("mode", [2, 3])
+def test_int8_error_bound_and_extremes(orc, mode):
+    """Spec bound: |q * scale - xFp32| <= amax / 254 (half a step);
+    the largest element maps to +-127; codes in [-127, 127]; codes are
+    monotone in xFp32."""
+    w = gen.make("deepseek_decode", bs=24)
+    w.x[3] = 0   # one all-zero token
+    out = orc.dispatch(w.x, w.expert_ids, w.num_instances, mode, smooth=w.smooth)
+    q = out["expand_x"].astype(np.float64)
+    src = out["src_of_row"]
+    inst = w.expert_ids.ravel()[src]
+    xf = (_f32(w.x)[src // w.top_k] * w.smooth[inst]).astype(np.float64)  # exact product in f64
+    n, H = len(src), w.hidden
+    seg = H if mode == 2 else 128
+    nt = (H + seg - 1) // seg
+    sc = out["dyn_scales"].reshape(n, nt).astype(np.float64)
+    assert (np.abs(q[:n]) <= 127).all()
+    for t in range(nt):
+        xs, qs = xf[:, t * seg:(t + 1) * seg], q[:n, t * seg:(t + 1) * seg]
+        # the fp32 product differs from the f64 one by at most half an ulp
+        amax = np.abs(xs).max(1)
+        err = np.abs(qs * sc[:, t:t + 1] - xs).max(1)
+        assert (err <= amax / 254 * (1 + 2 ** -16) + 1e-30).all()
+        nz = amax > 0
+        j = np.abs(xs).argmax(1)
+        np.testing.assert_array_equal(np.abs(qs[np.arange(n), j])[nz], 127)
+        assert (qs[~nz] == 0).all() and (sc[~nz, t] == 0).all()
+        o = np.argsort(xs, axis=1)
+        assert (np.diff(np.take_along_axis(qs, o, 1), axis=1) >= 0).all()
+
+
+def test_int8_smooth_power_of_two_scales_only_the_scale(orc):
+    """A power-of-two smooth row 2^p (one per instance) leaves every code as
+    it is and multiplies the sent scale by exactly 2^p; this pins that the
+    smooth row is picked by the destination instance (reading R9)."""
+    w = gen.make("deepseek_decode", bs=16)
+    p = (np.arange(w.num_instances) % 7) - 3
+    smooth = np.repeat((2.0 ** p)[:, None], w.hidden, 1).astype(np.float32)
+    base = orc.dispatch(w.x, w.expert_ids, w.num_instances, 2)
+    sm = orc.dispatch(w.x, w.expert_ids, w.num_instances, 2, smooth=smooth)
+    np.testing.assert_array_equal(base["expand_x"], sm["expand_x"])
+    inst = w.expert_ids.ravel()[base["src_of_row"]]
+    np.testing.assert_array_equal(sm["dyn_scales"][: base["n"]],
+                                  base["dyn_scales"][: base["n"]] * (2.0 ** p[inst]).astype(np.float32))
+    ones = orc.dispatch(w.x, w.expert_ids, w.num_instances, 3, smooth=np.ones_like(smooth))
+    none = orc.dispatch(w.x, w.expert_ids, w.num_instances, 3)
+    np.testing.assert_array_equal(ones["expand_x"], none["expand_x"])
+    np.testing.assert_array_equal(ones["dyn_scales"], none["dyn_scales"])
+
+
+def test_int8_single_tile_equals_per_token(orc):
+    w = gen.make("deepseek_decode", bs=8)
+    x = w.x[:, :128].copy()
+    a = orc.dispatch(x, w.expert_ids, w.num_instances, 2, smooth=w.smooth[:, :128].copy())
+    b = orc.dispatch(x, w.expert_ids, w.num_instances, 3, smooth=w.smooth[:, :128].copy())
+    np.testing.assert_array_equal(a["expand_x"], b["expand_x"])
+    np.testing.assert_array_equal(a["dyn_scales"], b["dyn_scales"][:, 0])
+
+
+# --------------------------------------------------------------------------
+# dispatch: mxfp8 (quantMode 4) and the e4m3 encoder
+# --------------------------------------------------------------------------
+
+def e4m3_decode(c):
+    """OCP FP8 E4M3 decode from the format definition (bias 7, no inf,
+    S.1111.111 = NaN)."""
+    c = int(c)
+    s = -1.0 if c & 0x80 else 1.0
+    e, m = (c >> 3) & 0xF, c & 7
+    if e == 15 and m == 7:
+        return math.nan
+    if e == 0:
+        return s * m * 2.0 ** -9
+    return s * (1 + m / 8) * 2.0 ** (e - 7)
+
+
+DEC = np.array([e4m3_decode(c) for c in range(256)])
+
+
+def test_e4m3_roundtrip_all_codes(orc):
+    for c in range(256):
+        v = DEC[c]
+        if math.isnan(v):
+            continue
+        assert orc.e4m3_encode(np.float32(v)) == c, hex(c)
+
+
+def test_e4m3_against_library_all_bf16(orc):
+    """All 65536 bf16 values: below 464 the result equals ml_dtypes' and
+    torch's float8_e4m3fn cast (round to nearest even); at or above it, the
+    oracle saturates to +-448 where those libraries give NaN."""
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    v = gen.bf16_to_f32(b)
+    fin = np.isfinite(v)
+    got = orc.e4m3_encode(v[fin])
+    lib = v[fin].astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    tch = torch.from_numpy(v[fin].copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    small = np.abs(v[fin]) < 464
+    np.testing.assert_array_equal(got[small], lib[small])
+    np.testing.assert_array_equal(got[small], tch[small])
+    big = ~small
+    np.testing.assert_array_equal(got[big], np.where(np.signbit(v[fin][big]), 0xFE, 0x7E))
+
+
+def test_e4m3_brute_force_nearest(orc):
+    """Random fp32 values and every exact midpoint between neighbouring
+    codes: the code is the nearest finite value, ties to the even code."""
+    rng = np.random.default_rng(7)
+    mag = 2.0 ** rng.uniform(-13, 9.2, 3000)
+    vals = (mag * rng.choice([-1, 1], 3000)).astype(np.float32)
+    pos = np.sort(DEC[np.isfinite(DEC) & (DEC >= 0)])
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(np.float32)
+    vals = np.concatenate([vals, mids, -mids])
+    got = orc.e4m3_encode(vals)
+    finite_codes = np.array([c for c in range(256) if not math.isnan(DEC[c])])
+    for v, g in zip(vals, got):
+        if abs(v) >= 448:
+            assert DEC[g] == math.copysign(448.0, v)
+            continue
+        d = np.abs(DEC[finite_codes] - float(v))
+        best = finite_codes[d == d.min()]
+        if len(best) > 1:   # a tie: the code with an even mantissa (for 0: the sign of v)
+            best = [c for c in best if (c & 1) == 0 and (DEC[c] != 0 or (c >> 7) == np.signbit(v))]
+        assert g == best[0], (v, g, best)
+
+
+def test_mxfp8_worked_blocks(orc):
+    for blk in GOLDEN["quant_mxfp8_blocks"]["blocks"]:
+        x = np.zeros(32, np.float32)
+        x[: len(blk["x_head"])] = blk["x_head"]
+        out = orc.dispatch(bits([x]), np.zeros((1, 1), np.int32), 1, 4)
+        assert out["dyn_scales"][0, 0] == blk["scale_byte"]
+        np.testing.assert_array_equal(out["expand_x"][0, : len(blk["q_head"])], blk["q_head"])
+
+
+def test_mxfp8_block_invariants(orc):
+    w = gen.make("skewed_eplb", bs=32)
+    out = orc.dispatch(w.x, w.expert_ids, w.num_instances, 4)
+    n, H = out["n"], w.hidden
+    x = gen.bf16_to_f32(w.x)[out["src_of_row"] // w.top_k].astype(np.float64).reshape(n, H // 32, 32)
+    se = out["dyn_scales"][:n].astype(np.int64) - 127
+    amax = np.abs(x).max(2)
+    r = amax * 2.0 ** (-se)
+    assert ((r >= 256) & (r < 512)).all()      # floor(log2 amax) - 8 exactly
+    deq = DEC[out["expand_x"][:n].reshape(n, H // 32, 32)] * 2.0 ** se[..., None]
+    v = np.abs(x) * 2.0 ** (-se[..., None])
+    sat = v >= 448
+    np.testing.assert_array_equal(np.abs(deq[sat]), (448 * 2.0 ** se[..., None] * np.ones_like(x))[sat])
+    norm = (v >= 2 ** -6) & ~sat
+    assert (np.abs(deq[norm] - x[norm]) <= np.abs(x[norm]) * 2 ** -4).all()
+    sub = v < 2 ** -6
+    assert (np.abs(deq - x)[sub] <= (2.0 ** -10 * 2.0 ** se[..., None] * np.ones_like(x))[sub]).all()
+    assert sat.any()   # the x20 outliers do saturate somewhere
+
+
+# --------------------------------------------------------------------------
+# combine + Add + RMSNorm (aclnnMoeDistributeCombineAddRmsNorm)
+# --------------------------------------------------------------------------
+
+def test_bf16_rounding_against_library(orc):
+    rng = np.random.default_rng(3)
+    f = (rng.standard_normal(20000) * 2.0 ** rng.integers(-30, 30, 20000)).astype(np.float32)
+    np.testing.assert_array_equal(orc.bf16_from_double(f.astype(np.float64)),
+                                  f.astype(ml_dtypes.bfloat16).view(np.uint16))
+    # exact midpoints go to the even neighbour; a hair above goes up
+    lo = np.array([1.0, 1.0078125, 3.0, -5.0], np.float64)      # bf16 values; ulp 2^-7 * 2^e
+    ulp = np.array([2 ** -7, 2 ** -7, 2 ** -6, 2 ** -5])
+    mid = lo + np.sign(lo) * ulp / 2
+    up = gen.bf16_bits((lo + np.sign(lo) * ulp).astype(np.float32))
+    lob = gen.bf16_bits(lo.astype(np.float32))
+    even = np.where((lob & 1) == 0, lob, up)
+    np.testing.assert_array_equal(orc.bf16_from_double(mid), even)
+    np.testing.assert_array_equal(orc.bf16_from_double(mid + np.sign(lo) * ulp * 2 ** -30), up)
+
+
+def test_combine_constant_row_closed_form(orc):
+    g = GOLDEN["combine_constant_row"]
+    H = g["hidden"]
+    ex = bits(np.full((1, H), g["expert_value"]))
+    res = bits(np.full((1, H), g["residual_value"]))
+    gam = bits(np.full(H, g["gamma_value"]))
+    out = orc.combine_add_rmsnorm(ex, np.zeros((1, 1), np.int32), np.ones((1, 1), np.float32),
+                                  res, gam, g["norm_eps"])
+    c = g["expert_value"] + g["residual_value"]
+    want = c / math.sqrt(c * c + g["norm_eps"]) * g["gamma_value"]
+    np.testing.assert_allclose(out["y_f64"], want, rtol=1e-14)
+    assert out["rstd"][0] == np.float32(1 / math.sqrt(c * c + g["norm_eps"]))
+
+
+def _rms_norm_lib(x, gamma, eps):
+    t = torch.from_numpy(np.asarray(x, np.float64))
+    return torch.nn.functional.rms_norm(t, (t.shape[-1],), torch.from_numpy(gamma), eps).numpy()
+
+
+def test_combine_single_expert_is_rmsnorm(orc):
+    """K = 1, weight 1, zero residual, no shared expert: y = RMSNorm(row)."""
+    w = gen.make("deepseek_decode", bs=6)
+    rows = w.expert_out[:6]
+    idx = np.arange(6, dtype=np.int32)[:, None]
+    out = orc.combine_add_rmsnorm(rows, idx, np.ones((6, 1), np.float32), np.zeros_like(w.residual),
+                                  w.gamma, 1e-6)
+    g = gen.bf16_to_f32(w.gamma).astype(np.float64)
+    np.testing.assert_allclose(out["y_f64"], _rms_norm_lib(gen.bf16_to_f32(rows), g, 1e-6),
+                               rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", ["tiny", "deepseek_decode_bs512_bf16"])
+def test_identity_expert_invariant(orc, name):
+    """quantMode 0, identity experts, weights summing to 1, no shared
+    expert: dispatch then combine returns RMSNorm(x + residual)."""
+    w = gen.make(name, bs=16)
+    d = orc.dispatch(w.x, w.expert_ids, w.num_instances, 0)
+    out = orc.combine_add_rmsnorm(d["expand_x"], d["expand_idx"], w.expert_scales, w.residual,
+                                  w.gamma, w.norm_eps)
+    x = gen.bf16_to_f32(w.x).astype(np.float64) + gen.bf16_to_f32(w.residual)
+    want = _rms_norm_lib(x, gen.bf16_to_f32(w.gamma).astype(np.float64), w.norm_eps)
+    np.testing.assert_allclose(out["y_f64"], want, rtol=0, atol=1e-5)
+
+
+def test_combine_linear_in_scales_and_prune_skips(orc):
+    w = gen.make("deepseek_decode", bs=8)
+    d = orc.dispatch(w.x, w.expert_ids, w.num_instances, 0)
+    zero = np.zeros_like(w.residual)
+    s1 = (np.round(w.expert_scales * 64) / 64).astype(np.float32)  # dyadic: s1 + s2 is exact
+    s2 = np.roll(s1, 1, axis=1)
+    run = lambda s, idx=d["expand_idx"], sh=None: orc.combine_add_rmsnorm(
+        d["expand_x"], idx, s, zero, w.gamma, 1e-6, shared_x=sh)["x_f64"]
+    np.testing.assert_allclose(run(2 * s1), 2 * run(s1), rtol=1e-15)
+    np.testing.assert_allclose(run(s1 + s2), run(s1) + run(s2), rtol=1e-12, atol=1e-12)
+    # a pruned copy (row -1) contributes exactly what a zero weight does
+    idx = d["expand_idx"].copy()
+    idx[:, 3] = -1
+    s0 = s1.copy()
+    s0[:, 3] = 0
+    np.testing.assert_array_equal(run(s1, idx), run(s0))
+
+
+def test_combine_shared_expert_weighting(orc):
+    """Reading R5: Sum_k(s_k * ata_k + s_k * shared) weights the shared row by
+    the sum of the kept weights (1 when no copy is pruned)."""
+    w = gen.make("deepseek_decode", bs=4)
+    K = w.top_k
+    zero_rows = np.zeros((4 * K, w.hidden), np.uint16)
+    idx = np.arange(4 * K, dtype=np.int32).reshape(4, K)
+    idx[1, :3] = -1
+    s = np.full((4, K), 0.125, np.float32)
+    out = orc.combine_add_rmsnorm(zero_rows, idx, s, np.zeros_like(w.residual), w.gamma, 1e-6,
+                                  shared_x=w.shared_x)
+    sh = gen.bf16_to_f32(w.shared_x).astype(np.float64)
+    np.testing.assert_array_equal(out["x_f64"][0], sh[0])            # 8 * 0.125 = 1
+    np.testing.assert_array_equal(out["x_f64"][1], sh[1] * 0.625)    # 5 kept copies
