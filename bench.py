@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""MoE dispatch+combine throughput on B200: tokens/s and achieved HBM GB/s.
+
+One step = one MoE layer's hot path on one batch of seeded synthetic input:
+moe_update_expert -> moe_dispatch -> moe_combine_add_rmsnorm (the expert FFN
+between dispatch and combine is stood in for by a resident buffer of bf16
+expert-output rows).  Every timed step starts with a cold L2 (a 512 MiB
+buffer is overwritten before it, outside the timed events).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
+
+With N > 1 it runs under torch.distributed.run, one process per GPU; the
+path has no exchange step on one GPU, so every rank runs an independent
+replica on its own batch (weak scaling, no data-path collective) and the
+reported value is the tokens of all ranks over the slowest rank's time.
+`--impl reference` times the plain CPU oracle on this host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "deepseek_decode_bs512"
+METRIC = "MoE dispatch+combine tokens/s (1 B200; HBM GB/s vs peak in roofline)"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------
+# algorithmic bytes: what each operation must move at minimum
+# --------------------------------------------------------------------------
+
+def algorithmic_bytes(w, n, x_out=False, rstd=False):
+    """Bytes each op must read + write for workload `w` with `n` kept copies.
+    Pruned copies are not counted (the method skips them)."""
+    bs, H, K, E = w.bs, w.hidden, w.top_k, w.num_instances
+    items = bs * K
+    upd = items * (4 + 4 + 4 + 1) + (4 if w.prune_threshold > 0 else 0) + 2 * 4 * w.num_logical
+    code = 2 if w.quant_mode == 0 else 1
+    sc = {0: 0, 2: 4, 3: 4 * ((H + 127) // 128), 4: H // 32}[w.quant_mode]
+    smooth_rows = 0
+    if w.smooth is not None:
+        smooth_rows = len(set(map(int, w.meta.get("distinct_instances", []))))
+    disp = (2 * bs * H                      # x
+            + 4 * H * smooth_rows           # smooth rows of the instances hit
+            + n * (H * code + sc)           # codes + scales of every kept copy
+            + items * (4 + 1)               # instance ids + mask
+            + items * 4 + n * 4             # expand_idx + src_of_row
+            + 4 * E + 4 * (E + 1))          # counts + offsets
+    comb = (n * 2 * H                       # expert rows gathered back
+            + 2 * bs * H                    # residual
+            + (2 * bs * H if w.shared_x is not None else 0)
+            + 2 * H                         # gamma
+            + 2 * bs * H                    # y
+            + (2 * bs * H if x_out else 0) + (4 * bs if rstd else 0)
+            + items * (4 + 4))              # expand_idx + scales
+    return dict(update=upd, dispatch=disp, combine=comb)
+
+
+def source_hash():
+    """Hash of the CUDA sources, to tell whether stored ncu counters still
+    describe the kernels being timed."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "combine_moe_update_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(p))[f"{kernel}@{workload}"]
+    except (OSError, KeyError, ValueError):
+        return None
+    return rec.get("dram_bytes_per_launch") if rec.get("source_hash") == source_hash() else None
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(p))["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region (read-only NVML queries)
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index, period_s=0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no samples
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (host side; covered by gloo tests)
+# --------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def reduce_over_ranks(values, op):
+    """Element-wise max / sum of a list of floats over all ranks (identity
+    when torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op={"max": dist.ReduceOp.MAX, "sum": dist.ReduceOp.SUM}[op])
+    return t.cpu().tolist()
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# the B200 arm
+# --------------------------------------------------------------------------
+
+def run_b200(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    from combine_moe_update_b200 import binding as B
+    from combine_moe_update_b200 import inputs as gen
+
+    torch.cuda.set_device(local_rank)
+    w = gen.make(args.workload, seed=None if rank == 0 else 1000 + rank)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    bf = lambda a: dev(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16)
+
+    # resident parameters of the layer
+    table = dev(w.table)
+    smooth = None if w.smooth is None else dev(w.smooth)
+    gamma = bf(w.gamma)
+    # this batch's activations
+    ids, scales = dev(w.expert_ids), dev(w.expert_scales)
+    x, residual, expert_out = bf(w.x), bf(w.residual), bf(w.expert_out)
+    shared = None if w.shared_x is None else bf(w.shared_x)
+    ws = B.new_workspace()
+    bal = torch.empty_like(ids)
+    bm = torch.empty(ids.shape, dtype=torch.uint8, device="cuda")
+    d = B.alloc_dispatch_outputs(w.bs, w.hidden, w.top_k, w.num_instances, w.quant_mode)
+    c = dict(y=torch.empty_like(x), x_out=None, rstd=None)
+
+    def step(xx=x, ii=ids, ss=scales, rr=residual, ee=expert_out, sh=shared):
+        B.update_expert(ii, table, w.ep_world_size, expert_scales=ss, prune_threshold=w.prune_threshold,
+                        workspace=ws, out=(bal, bm))
+        B.dispatch(xx, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
+                   workspace=ws, out=d)
+        B.combine_add_rmsnorm(ee, d["expand_idx"], ss, rr, gamma, w.norm_eps, shared_x=sh, workspace=ws, out=c)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert B.read_device_error(ws) == 0, "device error during warm-up"
+    n = int(d["offsets"][-1].item())
+    w.meta["distinct_instances"] = torch.unique(bal[bm.bool()]).cpu().tolist() if smooth is not None else []
+    alg = algorithmic_bytes(w, n)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for s in range(K):
+            flush.zero_()
+            e = ev[s]
+            e[0].record()
+            B.update_expert(ids, table, w.ep_world_size, expert_scales=scales, prune_threshold=w.prune_threshold,
+                            workspace=ws, out=(bal, bm))
+            e[1].record()
+            B.dispatch(x, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
+                       workspace=ws, out=d)
+            e[2].record()
+            B.combine_add_rmsnorm(expert_out, d["expand_idx"], scales, residual, gamma, w.norm_eps,
+                                  shared_x=shared, workspace=ws, out=c)
+            e[3].record()
+        torch.cuda.synchronize()
+    barrier()
+    assert B.read_device_error(ws) == 0, "device error during the timed steps"
+    ms = lambda a, b: sum(ev[s][a].elapsed_time(ev[s][b]) for s in range(K)) / K
+    t_step, t_upd, t_disp, t_comb = ms(0, 3), ms(0, 1), ms(1, 2), ms(2, 3)
+    t_step, t_upd, t_disp, t_comb = reduce_over_ranks([t_step, t_upd, t_disp, t_comb], "max")
+    value = world * w.bs / (t_step * 1e-3)
+    dc_value = world * w.bs / ((t_disp + t_comb) * 1e-3)
+
+    # ---- end to end through the public API with host buffers ----
+    pin = lambda t: t.cpu().pin_memory()
+    h_in = dict(x=pin(x), ids=pin(ids), scales=pin(scales), residual=pin(residual), expert_out=pin(expert_out))
+    if shared is not None:
+        h_in["shared"] = pin(shared)
+    d_in = dict(x=torch.empty_like(x), ids=torch.empty_like(ids), scales=torch.empty_like(scales),
+                residual=torch.empty_like(residual), expert_out=torch.empty_like(expert_out),
+                shared=None if shared is None else torch.empty_like(shared))
+    h_y = torch.empty(c["y"].shape, dtype=c["y"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = h_y.numel() * h_y.element_size()
+
+    def e2e_step():
+        for k_, t in h_in.items():
+            d_in[k_].copy_(t, non_blocking=True)
+        step(d_in["x"], d_in["ids"], d_in["scales"], d_in["residual"], d_in["expert_out"], d_in["shared"])
+        h_y.copy_(c["y"], non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ke = max(10, min(K, 200))
+    e0.record()
+    for _ in range(ke):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    (t_e2e,) = reduce_over_ranks([e0.elapsed_time(e1) / ke], "max")
+
+    peak, peak_kind = measured_peak()
+    achieved = alg["combine"] / (t_comb * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "combine_kernel", "achieved": round(achieved, 1),
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "traffic": stored_traffic("combine_kernel", args.workload),
+                "algorithmic_bytes": alg["combine"]}
+    disp_gbs = alg["dispatch"] / (t_disp * 1e-3) / 1e9
+    step_gbs = (alg["update"] + alg["dispatch"] + alg["combine"]) / (t_step * 1e-3) / 1e9
+    dc_gbs = (alg["dispatch"] + alg["combine"]) / ((t_disp + t_comb) * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {0: "bf16", 2: "int8", 3: "int8", 4: "fp8e4m3"}[w.quant_mode] + "+fp32",
+        "data": "synthetic (seeded; pages' shapes)",
+        "config": {"workload": args.workload, "bs": w.bs, "hidden": w.hidden, "top_k": w.top_k,
+                   "num_instances": w.num_instances, "ep_world_size_simulated": w.ep_world_size,
+                   "quant_mode": w.quant_mode, "smooth_scales": w.smooth is not None,
+                   "shared_expert": w.shared_x is not None, "kept_copies": n,
+                   "l2": "flushed (512 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
+        "breakdown_us": {"update_expert": round(t_upd * 1e3, 2), "dispatch": round(t_disp * 1e3, 2),
+                         "combine": round(t_comb * 1e3, 2)},
+        "dispatch_plus_combine": {"tokens_per_s": round(dc_value, 1), "hbm_gbs": round(dc_gbs, 1),
+                                  "frac_of_peak": round(dc_gbs / peak, 4),
+                                  "algorithmic_bytes": alg["dispatch"] + alg["combine"]},
+        "achieved_gbs": {"step": round(step_gbs, 1), "dispatch": round(disp_gbs, 1), "combine": round(achieved, 1)},
+        "roofline": roofline,
+        "e2e": {"value": round(world * w.bs / (t_e2e * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "pinned host activations -> device, the three calls, y -> host; layer parameters resident"},
+        "gpu_launches": 4 * K,
+        "clocks": clk.summary(),
+    }
+    return out, w
+
+
+# --------------------------------------------------------------------------
+# the CPU oracle, as a reported baseline and as the reference arm
+# --------------------------------------------------------------------------
+
+def oracle_step(orc, w):
+    bal, bm, _ = orc.update_expert(w.expert_ids, w.table, w.ep_world_size, expert_scales=w.expert_scales,
+                                   prune_threshold=w.prune_threshold)
+    d = orc.dispatch(w.x, bal, w.num_instances, w.quant_mode, mask=bm, smooth=w.smooth)
+    orc.combine_add_rmsnorm(w.expert_out, d["expand_idx"], w.expert_scales, w.residual, w.gamma, w.norm_eps,
+                            shared_x=w.shared_x)
+
+
+def subsample(w, tokens):
+    """The first `tokens` tokens of the workload (same parameters)."""
+    import copy
+    s = copy.copy(w)
+    s.bs = tokens
+    for k in ("x", "expert_ids", "expert_scales", "residual", "shared_x", "active_mask"):
+        v = getattr(w, k)
+        if v is not None:
+            setattr(s, k, v[:tokens].copy())
+    s.expert_out = w.expert_out[: tokens * w.top_k].copy()
+    return s
+
+
+def cpu_baseline(w, budget_s=10.0):
+    from oracle import oracle as orc
+    oracle_step(orc, subsample(w, 8))  # build + warm
+    t0 = time.perf_counter()
+    steps = 0
+    while True:
+        oracle_step(orc, w)
+        steps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(steps * w.bs / dt, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{steps} full steps of {w.bs} tokens ({dt:.1f} s, single-threaded C oracle)"}
+
+
+def run_reference(args, rank):
+    """Reference arm: the plain CPU oracle on this host's cores."""
+    if rank != 0:
+        return None
+    from combine_moe_update_b200 import inputs as gen
+    from oracle import oracle as orc
+    w = gen.make(args.workload)
+    orc.build()
+    # calibrate: seconds per token, then size each step so the run stays within ~2 minutes
+    t0 = time.perf_counter()
+    oracle_step(orc, subsample(w, 16))
+    per_tok = (time.perf_counter() - t0) / 16
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    tokens = int(max(1, min(w.bs, budget / max(per_tok, 1e-9))))
+    sample = subsample(w, tokens)
+    for _ in range(args.warmup):
+        oracle_step(orc, sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(orc, sample)
+    dt = time.perf_counter() - t0
+    value = args.steps * tokens / dt
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quant / f64 combine",
+        "data": "synthetic (seeded; pages' shapes)",
+        "config": {"workload": args.workload, "bs": w.bs, "hidden": w.hidden, "top_k": w.top_k,
+                   "num_instances": w.num_instances, "quant_mode": w.quant_mode, "tokens_per_step": tokens},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{tokens} of {w.bs} tokens per step, {args.steps} steps"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local_rank = dist_env()
+
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    import datetime
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out, w = run_b200(args, rank, world, local_rank)
+        if rank == 0:
+            out["cpu_baseline"] = cpu_baseline(w, args.cpu_baseline_seconds) if world == 1 else None
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,232 @@
+"""Thin ctypes binding of libmoe_b200.so (include/moe_b200.h).
+
+Argument marshalling only: tensors are checked for device, dtype and
+contiguity, outputs are allocated with torch when the caller passes none,
+and raw pointers plus the current CUDA stream go to the C ABI.  Every step
+of the computation runs in the library's CUDA kernels; there is no CPU or
+PyTorch fallback, and a missing or unloadable library raises at import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
+DEV_BAD_ID, DEV_BAD_TABLE = 1, 2
+WORKSPACE_BYTES = 256
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {_status_name(status)}")
+
+
+class UpdateParams(ctypes.Structure):
+    _fields_ = [("bs", ctypes.c_int32), ("top_k", ctypes.c_int32), ("num_logical", ctypes.c_int32),
+                ("table_cols", ctypes.c_int32), ("ep_world_size", ctypes.c_int32),
+                ("prune_threshold", ctypes.c_float)]
+
+
+class DispatchParams(ctypes.Structure):
+    _fields_ = [("bs", ctypes.c_int32), ("hidden", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("ep_world_size", ctypes.c_int32), ("num_instances", ctypes.c_int32),
+                ("quant_mode", ctypes.c_int32)]
+
+
+class CombineParams(ctypes.Structure):
+    _fields_ = [("bs", ctypes.c_int32), ("hidden", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("expand_rows", ctypes.c_int32), ("norm_eps", ctypes.c_float)]
+
+
+EXPORTS = (
+    "moe_workspace_init", "moe_read_device_error", "moe_clear_device_error", "moe_status_string",
+    "moe_update_expert_workspace_size", "moe_update_expert",
+    "moe_dispatch_workspace_size", "moe_dispatch",
+    "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm",
+)
+
+
+def _load():
+    path = _build.LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"libmoe_b200.so is not built ({path}); run combine_moe_update_b200.build")
+    L = ctypes.CDLL(path)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    P = ctypes.POINTER
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [ctypes.c_int]
+    L.moe_workspace_init.argtypes = [vp, sz, vp]
+    L.moe_read_device_error.argtypes = [vp, P(ctypes.c_uint32), vp]
+    L.moe_clear_device_error.argtypes = [vp, vp]
+    L.moe_update_expert_workspace_size.argtypes = [P(UpdateParams), P(sz)]
+    L.moe_update_expert.argtypes = [P(UpdateParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_dispatch_workspace_size.argtypes = [P(DispatchParams), P(sz)]
+    L.moe_dispatch.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_combine_add_rmsnorm_workspace_size.argtypes = [P(CombineParams), P(sz)]
+    L.moe_combine_add_rmsnorm.argtypes = [P(CombineParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    for name in EXPORTS:
+        if name != "moe_status_string":
+            getattr(L, name).restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def _status_name(s):
+    return lib.moe_status_string(int(s)).decode()
+
+
+def _check(fn, status):
+    if status != MOE_OK:
+        raise MoeError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _req(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _opt(t, name, dtype, shape=None):
+    return None if t is None else _req(t, name, dtype, shape)
+
+
+# --------------------------------------------------------------------------
+# workspace / device errors
+# --------------------------------------------------------------------------
+
+def new_workspace(device=None, stream=None) -> torch.Tensor:
+    """A zeroed workspace (holds the sticky device error word)."""
+    ws = torch.empty(WORKSPACE_BYTES, dtype=torch.uint8, device=device or "cuda")
+    _check("moe_workspace_init", lib.moe_workspace_init(_ptr(ws), WORKSPACE_BYTES, _stream(stream)))
+    return ws
+
+
+def read_device_error(workspace: torch.Tensor, stream=None) -> int:
+    bits = ctypes.c_uint32(0)
+    _check("moe_read_device_error", lib.moe_read_device_error(_ptr(workspace), ctypes.byref(bits), _stream(stream)))
+    return int(bits.value)
+
+
+def clear_device_error(workspace: torch.Tensor, stream=None) -> None:
+    _check("moe_clear_device_error", lib.moe_clear_device_error(_ptr(workspace), _stream(stream)))
+
+
+# --------------------------------------------------------------------------
+# the three operations
+# --------------------------------------------------------------------------
+
+def update_expert(expert_ids, table, ep_world_size, expert_scales=None, active_mask=None,
+                  prune_threshold=0.0, workspace=None, out=None, stream=None):
+    """moe_update_expert.  Returns (balanced_ids int32 [bs,K], balanced_mask uint8 [bs,K])."""
+    _req(expert_ids, "expert_ids", torch.int32)
+    bs, k = expert_ids.shape
+    _req(table, "table", torch.int32)
+    _opt(expert_scales, "expert_scales", torch.float32, (bs, k))
+    _opt(active_mask, "active_mask", torch.uint8, (bs,))
+    p = UpdateParams(bs, k, table.shape[0], table.shape[1], int(ep_world_size), float(prune_threshold))
+    if out is None:
+        out = (torch.empty((bs, k), dtype=torch.int32, device=expert_ids.device),
+               torch.empty((bs, k), dtype=torch.uint8, device=expert_ids.device))
+    bal, bm = out
+    _req(bal, "balanced_ids", torch.int32, (bs, k))
+    _req(bm, "balanced_mask", torch.uint8, (bs, k))
+    ws = workspace if workspace is not None else new_workspace(expert_ids.device, stream)
+    _check("moe_update_expert", lib.moe_update_expert(
+        ctypes.byref(p), _ptr(expert_ids), _ptr(expert_scales), _ptr(active_mask), _ptr(table),
+        _ptr(bal), _ptr(bm), _ptr(ws), ws.numel(), _stream(stream)))
+    return bal, bm
+
+
+def expand_dtype(quant_mode):
+    return {0: torch.bfloat16, 2: torch.int8, 3: torch.int8, 4: torch.uint8}[quant_mode]
+
+
+def scales_shape(quant_mode, rows, hidden):
+    return {0: None, 2: ((rows,), torch.float32), 3: ((rows, (hidden + 127) // 128), torch.float32),
+            4: ((rows, hidden // 32), torch.uint8)}[quant_mode]
+
+
+def alloc_dispatch_outputs(bs, hidden, top_k, num_instances, quant_mode, device="cuda"):
+    rows = bs * top_k
+    ss = scales_shape(quant_mode, rows, hidden)
+    return dict(
+        expand_x=torch.empty((rows, hidden), dtype=expand_dtype(quant_mode), device=device),
+        dyn_scales=None if ss is None else torch.empty(ss[0], dtype=ss[1], device=device),
+        expand_idx=torch.empty((bs, top_k), dtype=torch.int32, device=device),
+        src_of_row=torch.empty((rows,), dtype=torch.int32, device=device),
+        counts=torch.empty((num_instances,), dtype=torch.int32, device=device),
+        offsets=torch.empty((num_instances + 1,), dtype=torch.int32, device=device),
+    )
+
+
+def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=None, smooth=None,
+             workspace=None, out=None, stream=None):
+    """moe_dispatch.  Returns a dict with expand_x, dyn_scales, expand_idx,
+    src_of_row, counts and offsets (see include/moe_b200.h for layouts)."""
+    _req(x, "x", torch.bfloat16)
+    bs, H = x.shape
+    _req(instance_ids, "instance_ids", torch.int32)
+    k = instance_ids.shape[1]
+    _req(instance_ids, "instance_ids", torch.int32, (bs, k))
+    _opt(mask, "mask", torch.uint8, (bs, k))
+    _opt(smooth, "smooth", torch.float32, (num_instances, H))
+    if out is None:
+        out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
+    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode))
+    ws = workspace if workspace is not None else new_workspace(x.device, stream)
+    _check("moe_dispatch", lib.moe_dispatch(
+        ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
+        _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
+        _ptr(out["offsets"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, norm_eps,
+                        shared_x=None, want_x_out=False, want_rstd=False, workspace=None, out=None,
+                        stream=None):
+    """moe_combine_add_rmsnorm.  Returns a dict with y (and x_out / rstd when asked)."""
+    _req(expand_x, "expand_x", torch.bfloat16)
+    rows, H = expand_x.shape
+    _req(expand_idx, "expand_idx", torch.int32)
+    bs, k = expand_idx.shape
+    _req(expert_scales, "expert_scales", torch.float32, (bs, k))
+    _req(residual_x, "residual_x", torch.bfloat16, (bs, H))
+    _req(gamma, "gamma", torch.bfloat16, (H,))
+    _opt(shared_x, "shared_x", torch.bfloat16, (bs, H))
+    if out is None:
+        dev = expand_x.device
+        out = dict(y=torch.empty((bs, H), dtype=torch.bfloat16, device=dev),
+                   x_out=torch.empty((bs, H), dtype=torch.bfloat16, device=dev) if want_x_out else None,
+                   rstd=torch.empty((bs,), dtype=torch.float32, device=dev) if want_rstd else None)
+    p = CombineParams(bs, H, k, rows, float(norm_eps))
+    ws = workspace if workspace is not None else new_workspace(expand_x.device, stream)
+    _check("moe_combine_add_rmsnorm", lib.moe_combine_add_rmsnorm(
+        ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x),
+        _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")), _ptr(out.get("rstd")),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out

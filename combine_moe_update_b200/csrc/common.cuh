@@ -1,0 +1,125 @@
+// common.cuh -- small device helpers shared by the MoE kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+constexpr uint32_t kDevBadId = 1u;     // id or row index out of range: item dropped
+constexpr uint32_t kDevBadTable = 2u;  // mapping table broke its restrictions
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ void raise_error(uint32_t *err, uint32_t bits) { atomicOr(err, bits); }
+
+// Programmatic dependent launch (PTX griddepcontrol, sm_90 and later).  A
+// kernel launched with the programmatic-serialization attribute may start
+// while its predecessor runs; it must call pdl_wait() before it touches
+// anything the predecessor writes.  Without the attribute both are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// 16-byte load through the non-coherent path without L1 allocation: for
+// rows that are read once per kernel.
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte read-only load that may be cached in L1 (rows reused by a block).
+__device__ __forceinline__ uint4 ld_cached(const void *p) {
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+__device__ __forceinline__ void st_v4(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+
+// bf16 pair (one 32-bit word, element 0 in the low half) -> two floats, exact.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Eight bf16 in a uint4 -> eight floats.
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+    f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+    f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+// Two floats -> bf16 pair, round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Inclusive prefix sum over a block of up to 1024 threads (blockDim.x a
+// multiple of 32).  s_warp must hold 32 ints.  Contains two barriers and
+// leaves s_warp in use: put a barrier before reusing it.
+__device__ __forceinline__ int block_inclusive_scan(int v, int *s_warp) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) s_warp[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        int s = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(kFull, s, o);
+            if (lane >= o) s += y;
+        }
+        s_warp[lane] = s;
+    }
+    __syncthreads();
+    if (w > 0) v += s_warp[w - 1];
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+// Block-wide max / sum.  s_red holds one float per warp.  Two barriers, so
+// the buffer can be reused by the next call.
+template <int NWARPS>
+__device__ __forceinline__ float block_max(float v, float *s_red) {
+    v = warp_max(v);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = s_red[0];
+#pragma unroll
+    for (int w = 1; w < NWARPS; ++w) r = fmaxf(r, s_red[w]);
+    __syncthreads();
+    return r;
+}
+
+template <int NWARPS>
+__device__ __forceinline__ float block_sum(float v, float *s_red) {
+    v = warp_sum(v);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w) r += s_red[w];  // fixed order: deterministic
+    __syncthreads();
+    return r;
+}
+
+}  // namespace moe

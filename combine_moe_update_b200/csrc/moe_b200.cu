@@ -1,0 +1,300 @@
+// moe_b200.cu -- the C ABI of include/moe_b200.h: host-side validation,
+// workspace sizing and kernel launches.  All compute is in the kernels of
+// update_expert.cuh, rank.cuh, dispatch.cuh and combine.cuh.
+#include "moe_b200.h"
+
+#include <cstdint>
+#include <cstring>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "rank.cuh"
+#include "update_expert.cuh"
+
+namespace {
+
+// The workspace holds the sticky device error word (4 bytes), padded to 256.
+constexpr size_t kWorkspaceBytes = 256;
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline moe_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool check_workspace(const void *ws, size_t bytes) {
+    return ws != nullptr && aligned(ws, 16) && bytes >= kWorkspaceBytes;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory on the current
+// device (cached per device and kernel).
+template <typename Kernel>
+bool ensure_smem(Kernel k, size_t bytes, int slot) {
+    static int done[64][4];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (bytes <= 48 * 1024) return true;
+    if (done[dev][slot] >= (int)bytes) return true;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+    done[dev][slot] = (int)bytes;
+    return true;
+}
+
+// --- parameter checks: the limits of each page's shape-variable section ---
+
+bool valid_update(const moe_update_params &p) {
+    if (p.bs < 1 || p.bs > MOE_MAX_BS) return false;
+    if (p.num_logical < 1 || p.num_logical > MOE_MAX_EXPERTS) return false;
+    if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K || p.top_k > p.num_logical) return false;
+    if (p.ep_world_size < MOE_MIN_EP_WORLD || p.ep_world_size > MOE_MAX_EP_WORLD) return false;
+    if (p.table_cols < 2 || p.table_cols > p.ep_world_size + 1) return false;
+    if (!(p.prune_threshold == p.prune_threshold)) return false;  // NaN
+    return true;
+}
+
+moe_status valid_dispatch(const moe_dispatch_params &p) {
+    if (p.bs < 1 || p.bs > MOE_MAX_BS) return MOE_ERR_INVALID_ARG;
+    if (p.hidden < MOE_MIN_HIDDEN || p.hidden > MOE_MAX_HIDDEN || p.hidden % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (p.num_instances < 1 || p.num_instances > MOE_MAX_EXPERTS) return MOE_ERR_INVALID_ARG;
+    if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K || p.top_k > p.num_instances) return MOE_ERR_INVALID_ARG;
+    if (p.ep_world_size < MOE_MIN_EP_WORLD || p.ep_world_size > MOE_MAX_EP_WORLD) return MOE_ERR_INVALID_ARG;
+    if (p.num_instances % p.ep_world_size != 0) return MOE_ERR_INVALID_ARG;  // equal instances per rank
+    if (p.quant_mode == 1) return MOE_ERR_UNSUPPORTED;                     // static quantization
+    if (p.quant_mode != 0 && p.quant_mode != 2 && p.quant_mode != 3 && p.quant_mode != 4)
+        return MOE_ERR_INVALID_ARG;
+    if (p.quant_mode == 4 && p.hidden % 32 != 0) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+bool valid_combine(const moe_combine_params &p) {
+    if (p.bs < 1 || p.bs > MOE_MAX_BS) return false;
+    if (p.hidden < MOE_MIN_HIDDEN || p.hidden > MOE_MAX_HIDDEN || p.hidden % 16 != 0) return false;
+    if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K) return false;
+    if (p.expand_rows < 1) return false;
+    if (!(p.norm_eps >= 0.0f) || p.norm_eps > 3.0e38f) return false;  // rejects NaN and inf
+    return true;
+}
+
+template <typename Args>
+cudaError_t launch_pdl(void (*kernel)(Args), dim3 grid, dim3 block, size_t smem, cudaStream_t s, const Args &args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
+template <int MODE, bool SMOOTH>
+cudaError_t launch_dispatch(const moe::DispatchArgs &a, cudaStream_t s) {
+    return launch_pdl(moe::dispatch_kernel<MODE, SMOOTH>, dim3(a.bs), dim3(moe::kDpThreads), 0, s, a);
+}
+
+template <int KMAX>
+void launch_combine(const moe::CombineArgs &a, cudaStream_t s) {
+    if (a.shared_x)
+        moe::combine_kernel<KMAX, true><<<a.bs, moe::kCbThreads, 0, s>>>(a);
+    else
+        moe::combine_kernel<KMAX, false><<<a.bs, moe::kCbThreads, 0, s>>>(a);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+moe_status moe_workspace_init(void *workspace, size_t bytes, void *cuda_stream) {
+    if (!check_workspace(workspace, bytes)) return MOE_ERR_WORKSPACE;
+    return cudaMemsetAsync(workspace, 0, bytes, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_clear_device_error(void *workspace, void *cuda_stream) {
+    if (workspace == nullptr || !aligned(workspace, 16)) return MOE_ERR_WORKSPACE;
+    return cudaMemsetAsync(workspace, 0, sizeof(uint32_t), as_stream(cuda_stream)) == cudaSuccess ? MOE_OK
+                                                                                                   : MOE_ERR_CUDA;
+}
+
+moe_status moe_read_device_error(const void *workspace, uint32_t *bits, void *cuda_stream) {
+    if (workspace == nullptr || !aligned(workspace, 16)) return MOE_ERR_WORKSPACE;
+    if (bits == nullptr) return MOE_ERR_INVALID_ARG;
+    uint32_t v = 0;
+    cudaStream_t s = as_stream(cuda_stream);
+    if (cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    *bits = v;
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------- update ---
+
+moe_status moe_update_expert_workspace_size(const moe_update_params *p, size_t *bytes) {
+    if (p == nullptr || bytes == nullptr || !valid_update(*p)) return MOE_ERR_INVALID_ARG;
+    *bytes = kWorkspaceBytes;
+    return MOE_OK;
+}
+
+moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_ids, const float *expert_scales,
+                             const uint8_t *active_mask, const int32_t *table, int32_t *balanced_ids,
+                             uint8_t *balanced_mask, void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr || !valid_update(*p)) return MOE_ERR_INVALID_ARG;
+    if (!expert_ids || !table || !balanced_ids || !balanced_mask) return MOE_ERR_INVALID_ARG;
+    if (!aligned(expert_ids, 4) || !aligned(table, 4) || !aligned(balanced_ids, 4) ||
+        (expert_scales && !aligned(expert_scales, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
+
+    moe::UpdateArgs a;
+    a.bs = p->bs;
+    a.top_k = p->top_k;
+    a.num_logical = p->num_logical;
+    a.table_cols = p->table_cols;
+    a.ep_world_size = p->ep_world_size;
+    a.prune_threshold = p->prune_threshold;
+    a.expert_ids = expert_ids;
+    a.expert_scales = expert_scales;
+    a.active_mask = active_mask;
+    a.table = table;
+    a.balanced_ids = balanced_ids;
+    a.balanced_mask = balanced_mask;
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    const size_t smem = moe::update_expert_smem_bytes(p->ep_world_size);
+    if (!ensure_smem(moe::update_expert_kernel, smem, 0)) return MOE_ERR_CUDA;
+    moe::update_expert_kernel<<<1, moe::kUeThreads, smem, as_stream(cuda_stream)>>>(a);
+    return launch_status();
+}
+
+// -------------------------------------------------------------- dispatch ---
+
+moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, size_t *bytes) {
+    if (p == nullptr || bytes == nullptr) return MOE_ERR_INVALID_ARG;
+    moe_status st = valid_dispatch(*p);
+    if (st != MOE_OK) return st;
+    *bytes = kWorkspaceBytes;
+    return MOE_OK;
+}
+
+moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32_t *instance_ids,
+                        const uint8_t *mask, const float *smooth_scales, void *expand_x, void *dyn_scales,
+                        int32_t *expand_idx, int32_t *src_of_row, int32_t *expert_counts, int32_t *expert_offsets,
+                        void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr) return MOE_ERR_INVALID_ARG;
+    moe_status st = valid_dispatch(*p);
+    if (st != MOE_OK) return st;
+    const int mode = p->quant_mode;
+    if (!x || !instance_ids || !expand_x || !expand_idx || !src_of_row || !expert_counts || !expert_offsets)
+        return MOE_ERR_INVALID_ARG;
+    if ((mode == 0) != (dyn_scales == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (smooth_scales && (mode == 0 || mode == 4)) return MOE_ERR_INVALID_ARG;  // the page: scales must be null
+    if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(instance_ids, 4) || !aligned(expand_idx, 4) ||
+        !aligned(src_of_row, 4) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
+        (smooth_scales && !aligned(smooth_scales, 16)) || ((mode == 2 || mode == 3) && !aligned(dyn_scales, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(cuda_stream);
+    uint32_t *err = reinterpret_cast<uint32_t *>(workspace);
+
+    moe::RankArgs r;
+    r.items = p->bs * p->top_k;
+    r.num_instances = p->num_instances;
+    r.ids = instance_ids;
+    r.mask = mask;
+    r.expand_idx = expand_idx;
+    r.src_of_row = src_of_row;
+    r.counts = expert_counts;
+    r.offsets = expert_offsets;
+    r.err = err;
+    const size_t smem = moe::rank_smem_bytes(p->num_instances);
+    if (!ensure_smem(moe::rank_kernel, smem, 1)) return MOE_ERR_CUDA;
+    moe::rank_kernel<<<1, moe::kRkThreads, smem, s>>>(r);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+    moe::DispatchArgs a;
+    a.bs = p->bs;
+    a.hidden = p->hidden;
+    a.top_k = p->top_k;
+    a.tiles = (p->hidden + 127) / 128;
+    a.x = reinterpret_cast<const uint16_t *>(x);
+    a.ids = instance_ids;
+    a.smooth = smooth_scales;
+    a.expand_x = expand_x;
+    a.dyn_scales = dyn_scales;
+    a.expand_idx = expand_idx;
+    a.err = err;
+    cudaError_t e = cudaSuccess;
+    const bool sm = smooth_scales != nullptr;
+    switch (mode) {
+        case 0: e = launch_dispatch<0, false>(a, s); break;
+        case 2: e = sm ? launch_dispatch<2, true>(a, s) : launch_dispatch<2, false>(a, s); break;
+        case 3: e = sm ? launch_dispatch<3, true>(a, s) : launch_dispatch<3, false>(a, s); break;
+        case 4: e = launch_dispatch<4, false>(a, s); break;
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+// --------------------------------------------------------------- combine ---
+
+moe_status moe_combine_add_rmsnorm_workspace_size(const moe_combine_params *p, size_t *bytes) {
+    if (p == nullptr || bytes == nullptr || !valid_combine(*p)) return MOE_ERR_INVALID_ARG;
+    *bytes = kWorkspaceBytes;
+    return MOE_OK;
+}
+
+moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expand_x, const int32_t *expand_idx,
+                                   const float *expert_scales, const void *shared_x, const void *residual_x,
+                                   const void *gamma, void *y, void *x_out, float *rstd_out, void *workspace,
+                                   size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr || !valid_combine(*p)) return MOE_ERR_INVALID_ARG;
+    if (!expand_x || !expand_idx || !expert_scales || !residual_x || !gamma || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned(expand_x, 16) || !aligned(residual_x, 16) || !aligned(gamma, 16) || !aligned(y, 16) ||
+        (shared_x && !aligned(shared_x, 16)) || (x_out && !aligned(x_out, 16)) || !aligned(expand_idx, 4) ||
+        !aligned(expert_scales, 4) || (rstd_out && !aligned(rstd_out, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
+
+    moe::CombineArgs a;
+    a.bs = p->bs;
+    a.hidden = p->hidden;
+    a.top_k = p->top_k;
+    a.expand_rows = p->expand_rows;
+    a.norm_eps = p->norm_eps;
+    a.expand_x = reinterpret_cast<const uint16_t *>(expand_x);
+    a.expand_idx = expand_idx;
+    a.scales = expert_scales;
+    a.shared_x = reinterpret_cast<const uint16_t *>(shared_x);
+    a.residual = reinterpret_cast<const uint16_t *>(residual_x);
+    a.gamma = reinterpret_cast<const uint16_t *>(gamma);
+    a.y = reinterpret_cast<uint16_t *>(y);
+    a.x_out = reinterpret_cast<uint16_t *>(x_out);
+    a.rstd_out = rstd_out;
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    cudaStream_t s = as_stream(cuda_stream);
+    if (p->top_k <= 4) launch_combine<4>(a, s);
+    else if (p->top_k <= 8) launch_combine<8>(a, s);
+    else launch_combine<16>(a, s);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,152 @@
+// update_expert.cuh -- logical expert -> deployed instance, plus pruning.
+//
+// Follows aclnnMoeUpdateExpert (description: "Load balancing", "Expert
+// pruning"; "Restriction on the shape format" for the mapping table).  One
+// block of 1024 threads does everything: it is a few kilobytes of work and
+// a single block keeps the table bookkeeping in shared memory.
+//
+//   1. Read n_e (column 0) for every logical expert, check 1 <= n_e <= F-1,
+//      and prefix-sum it: instance (e, j) gets position first[e] + j.
+//   2. Thread p owns position p (<= 1024 positions): it finds its expert by
+//      binary search and reads the hosting rank from the table.
+//   3. Stable ranking of the positions by rank gives each instance its slot
+//      on that rank (earlier positions first), and checks that every rank
+//      hosts exactly L = total / ws instances.  inst = rank * L + slot.
+//   4. Every (token i, k) copy takes replica i mod n_e of its expert; the
+//      keep bit is mask[i] and "not (scale < threshold)".
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+struct UpdateArgs {
+    int bs, top_k, num_logical, table_cols, ep_world_size;
+    float prune_threshold;
+    const int32_t *expert_ids;
+    const float *expert_scales;  // may be null
+    const uint8_t *active_mask;  // may be null
+    const int32_t *table;
+    int32_t *balanced_ids;
+    uint8_t *balanced_mask;
+    uint32_t *err;
+};
+
+constexpr int kUeThreads = 1024;
+
+// Dynamic shared memory: n[1024], first[1024], inst[1024] ints, then one
+// uint16 counter per (warp, rank).
+inline size_t update_expert_smem_bytes(int ep_world_size) {
+    return 3 * 1024 * sizeof(int) + 32 * (size_t)ep_world_size * sizeof(uint16_t);
+}
+
+__device__ __forceinline__ void update_expert_drop_all(const UpdateArgs &a) {
+    const int n = a.bs * a.top_k;
+    for (int it = threadIdx.x; it < n; it += blockDim.x) {
+        a.balanced_ids[it] = -1;
+        a.balanced_mask[it] = 0;
+    }
+    if (threadIdx.x == 0) raise_error(a.err, kDevBadTable);
+}
+
+__global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    int *s_n = reinterpret_cast<int *>(smem);
+    int *s_first = s_n + 1024;
+    int *s_inst = s_first + 1024;
+    uint16_t *s_wc = reinterpret_cast<uint16_t *>(s_inst + 1024);  // [32][ws]
+    __shared__ int s_warp[32];
+    __shared__ int s_bad, s_total;
+
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int F = a.table_cols, ws = a.ep_world_size, E = a.num_logical;
+
+    if (t == 0) s_bad = 0;
+    for (int q = t; q < 32 * ws; q += kUeThreads) s_wc[q] = 0;
+    __syncthreads();
+
+    // 1. instance counts and their prefix sum
+    int n = 0;
+    if (t < E) {
+        n = a.table[(size_t)t * F];
+        if (n < 1 || n > F - 1) {
+            s_bad = 1;
+            n = 0;
+        }
+    }
+    const int incl = block_inclusive_scan(n, s_warp);
+    if (t < E) {
+        s_n[t] = n;
+        s_first[t] = incl - n;
+    }
+    if (t == kUeThreads - 1) s_total = incl;
+    __syncthreads();
+    const int total = s_total;
+    if (t == 0 && (total < 1 || total > 1024 || total % ws != 0)) s_bad = 1;
+    __syncthreads();
+    if (s_bad) {
+        update_expert_drop_all(a);
+        return;
+    }
+    const int L = total / ws;
+
+    // 2. the rank of instance position t
+    int r = -1;
+    if (t < total) {
+        int lo = 0, hi = E - 1;  // largest e with first[e] <= t (first is strictly increasing)
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (s_first[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        r = a.table[(size_t)lo * F + 1 + (t - s_first[lo])];
+        if (r < 0 || r >= ws) {
+            s_bad = 1;
+            r = -1;
+        }
+    }
+
+    // 3. stable rank by r: lanes of one warp first, then warps in order
+    const unsigned peers = __match_any_sync(kFull, r);
+    const int intra = __popc(peers & ((1u << lane) - 1u));
+    if (r >= 0 && lane == __ffs(peers) - 1) s_wc[w * ws + r] = (uint16_t)__popc(peers);
+    __syncthreads();
+    if (s_bad) {
+        update_expert_drop_all(a);
+        return;
+    }
+    for (int rr = t; rr < ws; rr += kUeThreads) {
+        int run = 0;
+        for (int ww = 0; ww < 32; ++ww) {
+            int c = s_wc[ww * ws + rr];
+            s_wc[ww * ws + rr] = (uint16_t)run;
+            run += c;
+        }
+        if (run != L) s_bad = 1;  // every rank hosts the same number of instances
+    }
+    __syncthreads();
+    if (s_bad) {
+        update_expert_drop_all(a);
+        return;
+    }
+    if (t < total) s_inst[t] = r * L + s_wc[w * ws + r] + intra;
+    __syncthreads();
+
+    // 4. every (token, k) copy
+    const int items = a.bs * a.top_k;
+    for (int it = t; it < items; it += kUeThreads) {
+        const int i = it / a.top_k;
+        const int e = a.expert_ids[it];
+        if (e < 0 || e >= E) {
+            raise_error(a.err, kDevBadId);
+            a.balanced_ids[it] = -1;
+            a.balanced_mask[it] = 0;
+            continue;
+        }
+        a.balanced_ids[it] = s_inst[s_first[e] + i % s_n[e]];
+        bool keep = a.active_mask ? (a.active_mask[i] != 0) : true;
+        if (a.expert_scales && a.prune_threshold > 0.0f && a.expert_scales[it] < a.prune_threshold)
+            keep = false;
+        a.balanced_mask[it] = keep ? 1 : 0;
+    }
+}
+
+}  // namespace moe

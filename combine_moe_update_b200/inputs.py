@@ -139,7 +139,7 @@ def make(name: str, seed: Optional[int] = None, bs: Optional[int] = None) -> Wor
     return spec.pop("builder")(name, **spec)
 
 
-def _uniform_layer(name, seed, bs, hidden, num_experts, top_k, ep_world_size, quant_mode,
+def uniform_layer(name, seed, bs, hidden, num_experts, top_k, ep_world_size, quant_mode,
                    smooth=False, shared=False, prune_threshold=0.0, logit_sigma=1.0):
     rng = np.random.Generator(np.random.PCG64(seed))
     x = bf16_bits(rng.standard_normal((bs, hidden), np.float32))
@@ -180,24 +180,24 @@ def _skewed_eplb(name, seed, bs, hidden=4096, num_logical=128, top_k=8, ep_world
 
 WORKLOADS = {
     # Bs 8, H 1024, 8 experts, K 2, 4 simulated ranks, no quantization.
-    "tiny": dict(builder=_uniform_layer, seed=0, bs=8, hidden=1024, num_experts=8, top_k=2,
+    "tiny": dict(builder=uniform_layer, seed=0, bs=8, hidden=1024, num_experts=8, top_k=2,
                  ep_world_size=4, quant_mode=0),
     # Decode batch of a DeepSeek-like layer: 256 experts, K 8, 32 ranks, per-token
     # int8 with per-expert smooth scales, one shared expert.
-    "deepseek_decode": dict(builder=_uniform_layer, seed=1, bs=256, hidden=7168, num_experts=256,
+    "deepseek_decode": dict(builder=uniform_layer, seed=1, bs=256, hidden=7168, num_experts=256,
                             top_k=8, ep_world_size=32, quant_mode=2, smooth=True, shared=True),
     # The same layer at the largest batch the pages allow (Bs 512).
-    "deepseek_decode_bs512": dict(builder=_uniform_layer, seed=1, bs=512, hidden=7168,
+    "deepseek_decode_bs512": dict(builder=uniform_layer, seed=1, bs=512, hidden=7168,
                                   num_experts=256, top_k=8, ep_world_size=32, quant_mode=2,
                                   smooth=True, shared=True),
     # ... and its unquantized variant (bf16 rows, no smooth, no shared expert).
-    "deepseek_decode_bs512_bf16": dict(builder=_uniform_layer, seed=1, bs=512, hidden=7168,
+    "deepseek_decode_bs512_bf16": dict(builder=uniform_layer, seed=1, bs=512, hidden=7168,
                                        num_experts=256, top_k=8, ep_world_size=32, quant_mode=0),
     # Zipf(1.2) routing over 128 experts, 160 instances on 16 ranks, mxfp8.
     "skewed_eplb": dict(builder=_skewed_eplb, seed=2, bs=512),
     # Largest shapes: H 8192, 1024 experts, K 16, 256 ranks, per-128-tile int8,
     # threshold pruning at 0.05 on softmax weights of N(0, 2) logits.
-    "max_shape": dict(builder=_uniform_layer, seed=3, bs=512, hidden=8192, num_experts=1024,
+    "max_shape": dict(builder=uniform_layer, seed=3, bs=512, hidden=8192, num_experts=1024,
                       top_k=16, ep_world_size=256, quant_mode=3, prune_threshold=0.05,
                       logit_sigma=float(np.sqrt(2.0))),
 }

@@ -1,0 +1,239 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) MoE update-expert / dispatch /
+ * combine+Add+RMSNorm library (libmoe_b200.so).
+ *
+ * The three operations follow three operator pages:
+ *   aclnnMoeUpdateExpert                  -> moe_update_expert
+ *   aclnnMoeDistributeDispatchV2          -> moe_dispatch
+ *   aclnnMoeDistributeCombineAddRmsNorm   -> moe_combine_add_rmsnorm
+ * and, like them, come in two phases: *_workspace_size() checks the
+ * parameters and sizes the workspace, then the call itself runs on a CUDA
+ * stream ("函数原型" / "Parameters" / "Returns" sections of each page).
+ *
+ * Expert parallelism on one GPU.  The pages' epWorldSize ranks are simulated
+ * as partitions of one rank-major receive buffer in this GPU's memory: the
+ * EP AllToAllV of dispatch is a permutation of rows into that buffer, and
+ * the AllToAllV of combine is a gather back out of it.  No collective and no
+ * inter-GPU traffic is involved.  One source rank of `bs` tokens feeds the
+ * exchange.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device pointers are CUDA device (or managed) memory
+ *     owned by the caller; the library never allocates, frees or keeps them.
+ *     Arrays are dense and row-major.  bf16 arrays and the int8 / e4m3 rows of
+ *     expand_x must start on a 16-byte boundary; int32 / f32 arrays on 4 bytes.
+ *   - `cuda_stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work: they neither allocate nor synchronize
+ *     (except moe_read_device_error), so they may be captured in CUDA graphs.
+ *   - Errors the host can see (bad sizes, NULL / misaligned pointers, a
+ *     workspace that is too small) return a non-zero moe_status and enqueue
+ *     nothing.  Errors only the device can see (an id out of range, a bad
+ *     mapping table) never trap: the offending item is dropped and a sticky
+ *     bit is OR-ed into the error word at the start of the workspace, which
+ *     moe_read_device_error returns.
+ *   - Every output is a pure function of the inputs: runs are bitwise
+ *     reproducible ("确定性计算" / "Deterministic computation" on each page).
+ *   - The workspace must be zeroed once (moe_workspace_init) before its first
+ *     use; the error word then accumulates until moe_clear_device_error.
+ *     Calls that share a workspace share its error word.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported from libmoe_b200.so; everything else in the library is hidden. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* a size outside the pages' limits, a NULL or misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2,  /* a legal value this library does not implement */
+    MOE_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than *_workspace_size reported */
+    MOE_ERR_CUDA = 4          /* the CUDA runtime refused a launch or a copy */
+} moe_status;
+
+/* Bits of the device error word (first 4 bytes of the workspace). */
+#define MOE_DEV_BAD_ID    1u  /* an expert / instance id or an expand_idx row out of range */
+#define MOE_DEV_BAD_TABLE 2u  /* mapping table broke its restrictions; every copy was dropped */
+
+/* Limits taken from the pages (shape-variable constraints of each page). */
+#define MOE_MAX_BS        512   /* Bs in (0, 512] */
+#define MOE_MIN_HIDDEN    1024  /* H in [1024, 8192] */
+#define MOE_MAX_HIDDEN    8192
+#define MOE_MAX_TOP_K     16    /* K in (0, 16], K <= expert count */
+#define MOE_MAX_EXPERTS   1024  /* logical experts and deployed instances each <= 1024 */
+#define MOE_MIN_EP_WORLD  2     /* epWorldSize in [2, 768] */
+#define MOE_MAX_EP_WORLD  768
+
+/* ------------------------------------------------------------------------ */
+/* Workspace and the device error word                                       */
+/* ------------------------------------------------------------------------ */
+
+/* Zero `bytes` of a workspace on `cuda_stream` (cudaMemsetAsync). */
+MOE_API moe_status moe_workspace_init(void *workspace, size_t bytes, void *cuda_stream);
+
+/* Synchronize `cuda_stream`, then copy the error word of `workspace` into
+ * *bits (a host pointer).  The only call in this library that blocks. */
+MOE_API moe_status moe_read_device_error(const void *workspace, uint32_t *bits, void *cuda_stream);
+
+/* Zero the error word of `workspace` on `cuda_stream`. */
+MOE_API moe_status moe_clear_device_error(void *workspace, void *cuda_stream);
+
+/* Human-readable name of a status code (static storage). */
+MOE_API const char *moe_status_string(moe_status status);
+
+/* ------------------------------------------------------------------------ */
+/* moe_update_expert -- aclnnMoeUpdateExpert (load balancing + pruning)      */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t bs;             /* tokens, (0, 512] */
+    int32_t top_k;          /* K, (0, 16] and <= num_logical */
+    int32_t num_logical;    /* logical experts = rows of the table, (0, 1024] */
+    int32_t table_cols;     /* F, [2, ep_world_size + 1] */
+    int32_t ep_world_size;  /* simulated ranks, [2, 768] */
+    float prune_threshold;  /* copies whose expert_scales entry is strictly below this are
+                               pruned; <= 0 (or expert_scales == NULL) disables */
+} moe_update_params;
+
+MOE_API moe_status moe_update_expert_workspace_size(const moe_update_params *p, size_t *bytes);
+
+/*
+ * Maps each token's K logical expert ids to deployed instance ids and
+ * computes the keep mask (aclnnMoeUpdateExpert, description: "Load
+ * balancing", "Expert pruning"; "Restriction on the shape format").
+ *
+ *   expert_ids    [bs, K] int32  device, logical ids in [0, num_logical)
+ *   expert_scales [bs, K] f32    device, optional (NULL = no threshold pruning)
+ *   active_mask   [bs]    uint8  device, optional; 0 prunes every copy of a token
+ *                                (the (BS,) mask broadcast to (BS,K))
+ *   table         [num_logical, F] int32 device: column 0 = n_e instances of
+ *                                expert e (>= 1, <= F-1), columns 1..n_e = the
+ *                                rank hosting each instance.  All instances
+ *                                together <= 1024, every rank hosting the same
+ *                                number L of them.
+ *   balanced_ids  [bs, K] int32  device, out: instance id = rank * L + slot,
+ *                                slots numbered per rank in (expert, replica)
+ *                                order; token i uses replica i mod n_e.  So the
+ *                                rank is balanced_ids / L.
+ *   balanced_mask [bs, K] uint8  device, out: 1 = keep, 0 = pruned
+ *
+ * Device errors: a bad table sets MOE_DEV_BAD_TABLE and writes -1 / 0 for
+ * every copy; an id outside [0, num_logical) sets MOE_DEV_BAD_ID and writes
+ * -1 / 0 for that copy.  (The page's own load-balancing formula did not
+ * survive extraction; the replica rule above is this library's reading.)
+ */
+MOE_API moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_ids,
+                             const float *expert_scales, const uint8_t *active_mask,
+                             const int32_t *table, int32_t *balanced_ids,
+                             uint8_t *balanced_mask, void *workspace, size_t workspace_bytes,
+                             void *cuda_stream);
+
+/* ------------------------------------------------------------------------ */
+/* moe_dispatch -- aclnnMoeDistributeDispatchV2 (quantize + EP AllToAllV)    */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t bs;             /* tokens, (0, 512] */
+    int32_t hidden;         /* H, [1024, 8192]; this library needs H % 16 == 0 (H % 32 == 0 in mode 4) */
+    int32_t top_k;          /* K, (0, 16] and <= num_instances */
+    int32_t ep_world_size;  /* simulated ranks, [2, 768]; must divide num_instances */
+    int32_t num_instances;  /* deployed expert instances E, (0, 1024] */
+    int32_t quant_mode;     /* 0 none, 2 per-token int8, 3 per-128-tile int8, 4 mxfp8 (1: unsupported) */
+} moe_dispatch_params;
+
+MOE_API moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, size_t *bytes);
+
+/*
+ * Orders the active (token, k) copies by destination instance and writes each
+ * one, quantized per quant_mode, into the expert-major receive buffer
+ * (aclnnMoeDistributeDispatchV2, "计算公式" cases 1, 3, 4, 5).  Rows are
+ * sorted by (instance, token, k); instance ids are rank-major, so simulated
+ * rank r receives rows [expert_offsets[r*L], expert_offsets[(r+1)*L]).
+ *
+ *   x             [bs, H] bf16   device
+ *   instance_ids  [bs, K] int32  device, in [0, num_instances) (moe_update_expert's output)
+ *   mask          [bs, K] uint8  device, optional; 0 = copy not sent
+ *   smooth_scales [num_instances, H] f32 device, optional, modes 2 and 3 only:
+ *                                xFp32 = x * smooth_scales[instance]
+ *   expand_x      [bs*K, H]      device, out: bf16 (mode 0), int8 (2, 3) or e4m3 (4).
+ *                                Rows >= expert_offsets[E] are left untouched.
+ *   dyn_scales    device, out, NULL in mode 0:
+ *                   mode 2: [bs*K] f32 = 1 / (127 / max|xFp32|)        (0 for an all-zero row)
+ *                   mode 3: [bs*K, ceil(H/128)] f32, the same per 128-element tile
+ *                   mode 4: [bs*K, H/32] uint8 E8M0 byte = sharedExp + 127, the
+ *                           dequantization factor 2^sharedExp of each 32-block,
+ *                           sharedExp = floor(log2 max|x|) - 8 clamped to >= -127
+ *   expand_idx    [bs, K] int32  device, out: row of copy (i, k), -1 if not sent
+ *   src_of_row    [bs*K]  int32  device, out: i*K + k of each row < expert_offsets[E]
+ *   expert_counts [E]     int32  device, out: rows received by each instance
+ *   expert_offsets[E+1]   int32  device, out: exclusive prefix sum, [E] = rows used
+ *
+ * int8 codes round half to even and clamp to [-127, 127]; e4m3 codes round
+ * half to even and saturate at +-448.  All quantization arithmetic is IEEE
+ * binary32, so codes and scales are bit-exact against any IEEE evaluation of
+ * the same formulas.  Device errors: an instance id out of range sets
+ * MOE_DEV_BAD_ID and the copy is not sent.
+ */
+MOE_API moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32_t *instance_ids,
+                        const uint8_t *mask, const float *smooth_scales, void *expand_x,
+                        void *dyn_scales, int32_t *expand_idx, int32_t *src_of_row,
+                        int32_t *expert_counts, int32_t *expert_offsets, void *workspace,
+                        size_t workspace_bytes, void *cuda_stream);
+
+/* ------------------------------------------------------------------------ */
+/* moe_combine_add_rmsnorm -- aclnnMoeDistributeCombineAddRmsNorm            */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t bs;           /* tokens, (0, 512] */
+    int32_t hidden;       /* H, [1024, 8192], H % 16 == 0 */
+    int32_t top_k;        /* K, (0, 16] */
+    int32_t expand_rows;  /* rows of expand_x (>= every non-negative expand_idx + 1), > 0 */
+    float norm_eps;       /* normEps, finite and >= 0 */
+} moe_combine_params;
+
+MOE_API moe_status moe_combine_add_rmsnorm_workspace_size(const moe_combine_params *p, size_t *bytes);
+
+/*
+ * For each token i (aclnnMoeDistributeCombineAddRmsNorm, "计算公式"):
+ *   combineOut = sum over kept k of (s_ik * expand_x[expand_idx[i,k]] + s_ik * shared_x[i])
+ *   x          = combineOut + residual_x[i]
+ *   y          = x / sqrt(mean_h(x^2) + norm_eps) * gamma
+ * accumulated in fp32.  A copy with expand_idx == -1 (pruned) contributes
+ * nothing, its weight included.
+ *
+ *   expand_x      [expand_rows, H] bf16 device (the expert outputs, rows as dispatch laid them out)
+ *   expand_idx    [bs, K] int32  device (dispatch's output)
+ *   expert_scales [bs, K] f32    device
+ *   shared_x      [bs, H] bf16   device, optional (shared-expert output)
+ *   residual_x    [bs, H] bf16   device
+ *   gamma         [H]     bf16   device
+ *   y             [bs, H] bf16   device, out
+ *   x_out         [bs, H] bf16   device, optional out: x before the norm
+ *   rstd_out      [bs]    f32    device, optional out: 1 / sqrt(mean(x^2) + eps)
+ *
+ * Device errors: an expand_idx entry >= expand_rows (or < -1) sets
+ * MOE_DEV_BAD_ID and that copy is skipped.
+ */
+MOE_API moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expand_x,
+                                   const int32_t *expand_idx, const float *expert_scales,
+                                   const void *shared_x, const void *residual_x, const void *gamma,
+                                   void *y, void *x_out, float *rstd_out, void *workspace,
+                                   size_t workspace_bytes, void *cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

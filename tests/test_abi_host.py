@@ -1,0 +1,175 @@
+"""Host-side checks of the C ABI; no GPU needed.
+
+The library must load without a GPU, export every function the header
+declares, size workspaces, and reject out-of-contract arguments with the
+documented status before it would launch anything.  Only argument sets that
+fail validation are passed to the launching entry points here, so nothing
+below can reach a kernel.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+# The negative cases below hand fake (never dereferenced) pointers to calls
+# that must reject their arguments first.  Should validation ever regress, a
+# launch on such pointers must not be able to reach a real GPU.
+pytestmark = pytest.mark.skipif(torch.cuda.is_available(),
+                                reason="fake-pointer validation checks run only where no GPU is visible")
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from combine_moe_update_b200 import build
+    build.build()
+    from combine_moe_update_b200 import binding
+    return binding
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_page_operations():
+    names = declared_functions()
+    for n in ("moe_update_expert", "moe_dispatch", "moe_combine_add_rmsnorm",
+              "moe_update_expert_workspace_size", "moe_dispatch_workspace_size",
+              "moe_combine_add_rmsnorm_workspace_size", "moe_read_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from combine_moe_update_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\S+)$", out, flags=re.M))
+    for n in declared_functions():
+        assert n in exported, n
+        assert getattr(L.lib, n) is not None
+    # nothing beyond the ABI leaks out
+    assert {e for e in exported if e.startswith("moe_")} == set(declared_functions())
+
+
+def test_status_strings(L):
+    assert L.lib.moe_status_string(0) == b"MOE_OK"
+    assert L.lib.moe_status_string(3) == b"MOE_ERR_WORKSPACE"
+
+
+def ws_size(L, fn, params):
+    n = ctypes.c_size_t(0)
+    st = getattr(L.lib, fn)(ctypes.byref(params), ctypes.byref(n))
+    return st, n.value
+
+
+def test_workspace_sizes_for_valid_params(L):
+    assert ws_size(L, "moe_update_expert_workspace_size", L.UpdateParams(512, 16, 1024, 257, 256, 0.05)) == (0, 256)
+    assert ws_size(L, "moe_dispatch_workspace_size", L.DispatchParams(512, 7168, 8, 32, 256, 2)) == (0, 256)
+    assert ws_size(L, "moe_combine_add_rmsnorm_workspace_size", L.CombineParams(512, 8192, 16, 8192, 1e-6)) == (0, 256)
+
+
+UPDATE_BAD = [
+    dict(bs=0), dict(bs=513), dict(top_k=0), dict(top_k=17), dict(num_logical=0), dict(num_logical=1025),
+    dict(top_k=9, num_logical=8), dict(ep_world_size=1), dict(ep_world_size=769), dict(table_cols=1),
+    dict(table_cols=34), dict(prune_threshold=float("nan")),
+]
+
+
+@pytest.mark.parametrize("bad", UPDATE_BAD)
+def test_update_expert_rejects(L, bad):
+    base = dict(bs=8, top_k=2, num_logical=8, table_cols=2, ep_world_size=32, prune_threshold=0.0)
+    base.update(bad)
+    p = L.UpdateParams(*base.values())
+    assert ws_size(L, "moe_update_expert_workspace_size", p)[0] == L.MOE_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(0x10000)
+    st = L.lib.moe_update_expert(ctypes.byref(p), fake, None, None, fake, fake, fake, fake, 256, None)
+    assert st == L.MOE_ERR_INVALID_ARG
+
+
+DISPATCH_BAD = [
+    (dict(bs=0), 1), (dict(bs=513), 1), (dict(hidden=1008), 1), (dict(hidden=8208), 1), (dict(hidden=1032), 1),
+    (dict(top_k=0), 1), (dict(top_k=17), 1), (dict(num_instances=1025), 1), (dict(num_instances=0), 1),
+    (dict(ep_world_size=1), 1), (dict(ep_world_size=769), 1), (dict(ep_world_size=24), 1),
+    (dict(quant_mode=5), 1), (dict(quant_mode=-1), 1), (dict(quant_mode=1), 2),
+    (dict(quant_mode=4, hidden=1040), 1),
+]
+
+
+@pytest.mark.parametrize("bad,status", DISPATCH_BAD)
+def test_dispatch_rejects(L, bad, status):
+    base = dict(bs=8, hidden=1024, top_k=2, ep_world_size=4, num_instances=8, quant_mode=0)
+    base.update(bad)
+    p = L.DispatchParams(*base.values())
+    assert ws_size(L, "moe_dispatch_workspace_size", p)[0] == status
+    f = ctypes.c_void_p(0x10000)
+    st = L.lib.moe_dispatch(ctypes.byref(p), f, f, None, None, f, f if base["quant_mode"] else None,
+                            f, f, f, f, f, 256, None)
+    assert st == status
+
+
+def _dispatch_call(L, mode=2, **ptrs):
+    p = L.DispatchParams(8, 1024, 2, 4, 8, mode)
+    f = ctypes.c_void_p(0x10000)
+    args = dict(x=f, ids=f, mask=None, smooth=None, ex=f, ds=f if mode else None, idx=f, src=f, cnt=f,
+                off=f, ws=f, wsb=256)
+    args.update(ptrs)
+    return L.lib.moe_dispatch(ctypes.byref(p), args["x"], args["ids"], args["mask"], args["smooth"],
+                              args["ex"], args["ds"], args["idx"], args["src"], args["cnt"], args["off"],
+                              args["ws"], args["wsb"], None)
+
+
+def test_dispatch_pointer_rules(L):
+    f8 = ctypes.c_void_p(0x10008)  # 8-byte aligned only
+    assert _dispatch_call(L, x=None) == L.MOE_ERR_INVALID_ARG
+    assert _dispatch_call(L, x=f8) == L.MOE_ERR_INVALID_ARG          # bf16 rows need 16 bytes
+    assert _dispatch_call(L, ex=f8) == L.MOE_ERR_INVALID_ARG
+    assert _dispatch_call(L, mode=2, ds=None) == L.MOE_ERR_INVALID_ARG   # mode 2 needs scales out
+    assert _dispatch_call(L, mode=0, ds=ctypes.c_void_p(0x10000)) == L.MOE_ERR_INVALID_ARG
+    assert _dispatch_call(L, mode=4, smooth=ctypes.c_void_p(0x10000)) == L.MOE_ERR_INVALID_ARG
+    assert _dispatch_call(L, mode=0, smooth=ctypes.c_void_p(0x10000)) == L.MOE_ERR_INVALID_ARG
+    assert _dispatch_call(L, ws=None) == L.MOE_ERR_WORKSPACE
+    assert _dispatch_call(L, wsb=255) == L.MOE_ERR_WORKSPACE
+
+
+COMBINE_BAD = [dict(bs=0), dict(bs=513), dict(hidden=1000), dict(hidden=9000), dict(top_k=0), dict(top_k=17),
+               dict(expand_rows=0), dict(norm_eps=-1.0), dict(norm_eps=float("nan")), dict(norm_eps=float("inf"))]
+
+
+@pytest.mark.parametrize("bad", COMBINE_BAD)
+def test_combine_rejects(L, bad):
+    base = dict(bs=8, hidden=1024, top_k=2, expand_rows=16, norm_eps=1e-6)
+    base.update(bad)
+    p = L.CombineParams(*base.values())
+    assert ws_size(L, "moe_combine_add_rmsnorm_workspace_size", p)[0] == L.MOE_ERR_INVALID_ARG
+    f = ctypes.c_void_p(0x10000)
+    st = L.lib.moe_combine_add_rmsnorm(ctypes.byref(p), f, f, f, None, f, f, f, None, None, f, 256, None)
+    assert st == L.MOE_ERR_INVALID_ARG
+
+
+def test_combine_pointer_rules(L):
+    p = L.CombineParams(8, 1024, 2, 16, 1e-6)
+    f, f8 = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10008)
+    call = lambda ex=f, res=f, y=f, sh=None, ws=f: L.lib.moe_combine_add_rmsnorm(
+        ctypes.byref(p), ex, f, f, sh, res, f, y, None, None, ws, 256, None)
+    assert call(ex=None) == L.MOE_ERR_INVALID_ARG
+    assert call(res=f8) == L.MOE_ERR_INVALID_ARG
+    assert call(y=f8) == L.MOE_ERR_INVALID_ARG
+    assert call(sh=f8) == L.MOE_ERR_INVALID_ARG
+    assert call(ws=None) == L.MOE_ERR_WORKSPACE
+
+
+def test_no_cpu_fallback_in_product():
+    """The product package never reaches the oracle."""
+    pkg = os.path.join(ROOT, "combine_moe_update_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b|moe_oracle|orc_", src, re.M), fn

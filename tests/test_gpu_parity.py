@@ -1,0 +1,350 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.  Bit-exact for routing, indices, counts, int8 / e4m3
+codes and scales; within 1e-2 relative (rms floor) for the bf16 combine
+outputs.  Outputs are poisoned before each call so that unwritten or
+overwritten rows show up."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from combine_moe_update_b200 import inputs as gen
+from oracle import oracle as orc
+
+from gpu_harness import (POISON, assert_close_bf16, assert_parity, dev, dev_bf16, host, poison_, run_gpu,
+                         run_oracle)
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")))
+
+
+@pytest.fixture(scope="module")
+def B():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from combine_moe_update_b200 import binding
+    return binding
+
+
+# ---------------------------------------------------------------- workloads
+
+@pytest.mark.parametrize("name", ["tiny", "deepseek_decode", "deepseek_decode_bs512",
+                                  "deepseek_decode_bs512_bf16", "skewed_eplb", "max_shape"])
+def test_parity_workloads(B, name):
+    w = gen.make(name)
+    assert_parity(w, run_gpu(w, B), run_oracle(w))
+
+
+@pytest.mark.parametrize("mode,H,smooth", [(0, 1040, False), (2, 1040, True), (2, 1040, False),
+                                           (3, 1040, False), (3, 1168, True), (4, 1056, False),
+                                           (2, 8192, True), (3, 8192, False), (4, 8192, False),
+                                           (0, 8192, False), (4, 2080, False)])
+def test_parity_ragged_hidden(B, mode, H, smooth):
+    """H not a multiple of 128 (a partial last tile), and the largest H."""
+    w = gen.uniform_layer(f"ragged{mode}_{H}", seed=11 + H, bs=37, hidden=H, num_experts=24, top_k=5,
+                          ep_world_size=6, quant_mode=mode, smooth=smooth, shared=(mode == 2))
+    assert_parity(w, run_gpu(w, B), run_oracle(w))
+
+
+@pytest.mark.parametrize("bs,K,E,ws,mode", [(1, 1, 2, 2, 0), (1, 16, 16, 2, 2), (3, 16, 16, 8, 4),
+                                            (512, 16, 1024, 256, 0), (5, 4, 768, 768, 3),
+                                            (511, 3, 9, 3, 2), (2, 2, 1024, 2, 4)])
+def test_parity_shape_extremes(B, bs, K, E, ws, mode):
+    w = gen.uniform_layer("extreme", seed=bs * 1000 + K, bs=bs, hidden=1024, num_experts=E, top_k=K,
+                          ep_world_size=ws, quant_mode=mode, smooth=(mode in (2, 3)))
+    assert_parity(w, run_gpu(w, B), run_oracle(w))
+
+
+def test_parity_everything_pruned(B):
+    """Threshold above every weight: no copy is sent, combine is residual-only."""
+    w = gen.make("deepseek_decode", bs=16)
+    w.prune_threshold = 2.0
+    g, o = run_gpu(w, B), run_oracle(w)
+    assert o["dispatch"]["n"] == 0
+    assert_parity(w, g, o)
+
+
+def test_parity_active_mask(B):
+    w = gen.make("max_shape", bs=64)
+    w.active_mask = (np.random.default_rng(5).random(64) < 0.6).astype(np.uint8)
+    assert_parity(w, run_gpu(w, B), run_oracle(w))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_parity_random_replicated_tables(B, seed):
+    rng = np.random.default_rng(seed)
+    ws = int(rng.choice([2, 3, 16, 64, 768]))
+    L = int(rng.integers(1, max(2, 1024 // ws) + 1))
+    total = ws * L
+    nl = int(rng.integers(max(1, total // ws), total + 1))
+    nl = min(nl, total)
+    reps = np.ones(nl, np.int64)
+    extra = total - nl
+    while extra:
+        e = int(rng.integers(0, nl))
+        if reps[e] < ws:
+            reps[e] += 1
+            extra -= 1
+    # any placement with L instances on every rank is legal (replicas may share a rank)
+    rank_of = rng.permutation(np.repeat(np.arange(ws), L))
+    F = int(rng.integers(int(reps.max()) + 1, ws + 2))
+    table = np.full((nl, F), -1, np.int32)
+    table[:, 0] = reps
+    pos = 0
+    for e in range(nl):
+        table[e, 1:1 + reps[e]] = rank_of[pos:pos + reps[e]]
+        pos += reps[e]
+    K = int(min(16, nl, rng.integers(1, 17)))
+    w = gen.uniform_layer("rep", seed=seed, bs=int(rng.integers(1, 513)), hidden=1024, num_experts=2 * K,
+                          top_k=K, ep_world_size=2, quant_mode=0)
+    w.num_logical, w.num_instances, w.ep_world_size, w.table = nl, total, ws, table
+    w.expert_ids = gen.topk_uniform(rng, w.bs, nl, K)
+    assert_parity(w, run_gpu(w, B), run_oracle(w))
+
+
+# ------------------------------------------------------------ rank / dispatch
+
+def run_dispatch_gpu(B, x_bits, ids, E, ws, mode, mask=None, smooth=None):
+    bs, K = ids.shape
+    d = B.alloc_dispatch_outputs(bs, x_bits.shape[1], K, E, mode)
+    for v in d.values():
+        if v is not None:
+            poison_(v)
+    wsp = B.new_workspace()
+    B.dispatch(dev_bf16(x_bits), dev(ids), E, ws, mode, mask=None if mask is None else dev(mask),
+               smooth=None if smooth is None else dev(smooth), workspace=wsp, out=d)
+    out = {k: (None if v is None else host(v)) for k, v in d.items()}
+    out["err"] = B.read_device_error(wsp)
+    return out
+
+
+def assert_dispatch_equal(g, o, mode):
+    n = o["n"]
+    np.testing.assert_array_equal(g["expand_idx"], o["expand_idx"])
+    np.testing.assert_array_equal(g["counts"], o["counts"])
+    np.testing.assert_array_equal(g["offsets"], o["offsets"])
+    np.testing.assert_array_equal(g["src_of_row"][:n], o["src_of_row"])
+    ge = g["expand_x"].view(np.uint8).reshape(g["expand_x"].shape[0], -1)
+    np.testing.assert_array_equal(ge[:n], o["expand_x"].view(np.uint8).reshape(ge.shape[0], -1)[:n])
+    assert (ge[n:] == POISON).all()
+    if mode:
+        gs = g["dyn_scales"].view(np.uint8).reshape(g["dyn_scales"].shape[0], -1)
+        np.testing.assert_array_equal(gs[:n], o["dyn_scales"].view(np.uint8).reshape(gs.shape[0], -1)[:n])
+    assert g["err"] == o["err"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_rank_random_ids_with_duplicates(B, seed):
+    """Ids drawn with replacement (duplicates inside a token), random masks,
+    up to 8192 copies over up to 1024 instances."""
+    rng = np.random.default_rng(50 + seed)
+    bs, K = int(rng.integers(1, 513)), int(rng.integers(1, 17))
+    ws = int(rng.choice([2, 4, 8, 32, 256]))
+    E = ws * int(rng.integers(1, 1024 // ws + 1))
+    K = min(K, E)
+    ids = rng.integers(0, E, size=(bs, K)).astype(np.int32)
+    if seed % 2:
+        ids = np.minimum(ids, E // 7)   # heavy skew into few buckets
+    mask = (rng.random((bs, K)) < rng.uniform(0.2, 1.0)).astype(np.uint8)
+    x = gen.bf16_bits(rng.standard_normal((bs, 1024), np.float32))
+    g = run_dispatch_gpu(B, x, ids, E, ws, 0, mask=mask)
+    o = orc.dispatch(x, ids, E, 0, mask=mask)
+    assert_dispatch_equal(g, o, 0)
+
+
+def edge_rows(H, rng):
+    """Rows that stress the quantizers: all zero, one huge outlier, tiny
+    (subnormal) values, signed zeros, exact powers of two, mixed scales."""
+    rows = [np.zeros(H), rng.standard_normal(H) * 1e-3, rng.standard_normal(H)]
+    r = rng.standard_normal(H)
+    r[H // 3] = 3.0e4
+    rows.append(r)
+    rows.append(np.full(H, -0.0))
+    rows.append(rng.standard_normal(H) * 1e-39)          # bf16 subnormals
+    rows.append(np.where(rng.random(H) < 0.5, 1.0, -2.0) * 2.0 ** rng.integers(-20, 20, H))
+    r = rng.standard_normal(H)
+    r[::32] = 0.0
+    r[5::64] = 1e-38
+    rows.append(r)
+    rows.append(np.tile(np.array([1.875, 1.5, -0.25, 1e-40] + [0.0] * 28), H // 32))
+    return gen.bf16_bits(np.array(rows, np.float32))
+
+
+@pytest.mark.parametrize("mode", [2, 3, 4])
+def test_quant_edge_rows(B, mode):
+    rng = np.random.default_rng(mode)
+    H = 1024
+    x = edge_rows(H, rng)
+    bs = x.shape[0]
+    ids = np.arange(bs * 2, dtype=np.int32).reshape(bs, 2) % 8
+    smooth = rng.uniform(0.5, 2.0, (8, H)).astype(np.float32) if mode != 4 else None
+    g = run_dispatch_gpu(B, x, ids, 8, 2, mode, smooth=smooth)
+    o = orc.dispatch(x, ids, 8, mode, smooth=smooth)
+    assert_dispatch_equal(g, o, mode)
+
+
+def test_e4m3_every_bf16_value_through_mxfp8(B):
+    """Every finite bf16 value passes the e4m3 encoder of the mxfp8 path once
+    with scale 2^0 (block max 256) and once with scale 2^-8 (block max 1.875,
+    so values beyond 448 saturate): codes and scale bytes match the oracle."""
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    v = gen.bf16_to_f32(allb)
+    for head, lim in ((256.0, 256.0), (1.875, 1.875)):
+        vals = v[np.isfinite(v) & (np.abs(v) < lim)]
+        nblk = -(-len(vals) // 31)
+        blocks = np.zeros((nblk, 32), np.float32)
+        blocks[:, 0] = head
+        flat = blocks[:, 1:].reshape(-1)
+        flat[: len(vals)] = vals
+        blocks[:, 1:] = flat.reshape(nblk, 31)
+        H = 4096
+        rows = -(-nblk * 32 // H)
+        x = np.zeros(rows * H, np.float32)
+        x[: nblk * 32] = blocks.reshape(-1)
+        x = gen.bf16_bits(x.reshape(rows, H))
+        ids = np.zeros((rows, 1), np.int32)
+        g = run_dispatch_gpu(B, x, ids, 2, 2, 4)
+        o = orc.dispatch(x, ids, 2, 4)
+        assert_dispatch_equal(g, o, 4)
+
+
+def test_worked_examples_on_gpu(B):
+    """The hand-derived rows of tests/golden, padded with zeros to H = 1024."""
+    H = 1024
+    for row in GOLDEN["quant_int8_rows"]["rows"]:
+        x = np.zeros((1, H), np.float32)
+        x[0, :8] = row["x"]
+        sm = None
+        if row["smooth"] is not None:
+            sm = np.ones((2, H), np.float32)
+            sm[0, :8] = row["smooth"]
+        g = run_dispatch_gpu(B, gen.bf16_bits(x), np.zeros((1, 1), np.int32), 2, 2, 2, smooth=sm)
+        np.testing.assert_array_equal(g["expand_x"][0, :8], row["q"])
+        assert not g["expand_x"][0, 8:].any()
+        assert g["dyn_scales"][0] == np.float32(row["scale"])
+        if "scale_bits" in row:
+            assert int(g["dyn_scales"][:1].view(np.uint32)[0]) == int(row["scale_bits"], 16)
+    for blk in GOLDEN["quant_mxfp8_blocks"]["blocks"]:
+        x = np.zeros((1, H), np.float32)
+        x[0, : len(blk["x_head"])] = blk["x_head"]
+        g = run_dispatch_gpu(B, gen.bf16_bits(x), np.zeros((1, 1), np.int32), 2, 2, 4)
+        assert g["dyn_scales"][0, 0] == blk["scale_byte"]
+        np.testing.assert_array_equal(g["expand_x"][0, : len(blk["q_head"])], blk["q_head"])
+
+
+# ------------------------------------------------------------ device errors
+
+def test_bad_ids_are_dropped_and_flagged(B):
+    w = gen.make("tiny")
+    ids = w.expert_ids.copy()
+    ids[2, 1] = 8          # out of range
+    ids[5, 0] = -3
+    wsp = B.new_workspace()
+    bal, bm = B.update_expert(dev(ids), dev(w.table), w.ep_world_size, workspace=wsp)
+    assert B.read_device_error(wsp) == B.DEV_BAD_ID
+    ob, om, oe = orc.update_expert(ids, w.table, w.ep_world_size)
+    assert oe == orc.ERR_BAD_ID
+    np.testing.assert_array_equal(host(bal), ob)
+    np.testing.assert_array_equal(host(bm), om)
+    # dispatch on raw out-of-range instance ids (mask ignored)
+    g = run_dispatch_gpu(B, w.x, ids, w.num_instances, w.ep_world_size, 0)
+    o = orc.dispatch(w.x, ids, w.num_instances, 0)
+    assert o["err"] == orc.ERR_BAD_ID
+    assert_dispatch_equal(g, o, 0)
+    # combine with a row index past expand_rows
+    B.clear_device_error(wsp)
+    idx = np.array([[0, 1]] * w.bs, np.int32)
+    idx[3, 1] = 10 ** 6
+    res = B.combine_add_rmsnorm(dev_bf16(w.expert_out), dev(idx), dev(w.expert_scales), dev_bf16(w.residual),
+                                dev_bf16(w.gamma), w.norm_eps, workspace=wsp)
+    assert B.read_device_error(wsp) == B.DEV_BAD_ID
+    idx_o = idx.copy()
+    idx_o[3, 1] = -1
+    c = orc.combine_add_rmsnorm(w.expert_out, idx_o, w.expert_scales, w.residual, w.gamma, w.norm_eps)
+    assert_close_bf16(host(res["y"]), c["y_f64"])
+
+
+@pytest.mark.parametrize("bad", ["zero_count", "rank_out_of_range", "uneven"])
+def test_bad_table_flagged(B, bad):
+    w = gen.make("tiny")
+    t = w.table.copy()
+    if bad == "zero_count":
+        t[3, 0] = 0
+    elif bad == "rank_out_of_range":
+        t[5, 1] = 4
+    else:
+        t[0, 1] = 1
+    wsp = B.new_workspace()
+    bal, bm = B.update_expert(dev(w.expert_ids), dev(t), w.ep_world_size, workspace=wsp)
+    assert B.read_device_error(wsp) & B.DEV_BAD_TABLE
+    assert (host(bal) == -1).all() and (host(bm) == 0).all()
+
+
+# ------------------------------------------------------------ determinism
+
+def test_runs_are_bitwise_identical(B):
+    w = gen.make("skewed_eplb")
+    a, b = run_gpu(w, B), run_gpu(w, B)
+    for k in a:
+        if a[k] is not None and not isinstance(a[k], int):
+            np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+# ------------------------------------------------------------ layer stack
+
+def test_layer_stack_cuda_graph(B):
+    """32 chained layers (update -> dispatch -> identity expert -> combine),
+    captured in one CUDA graph, against 32 chained oracle layers."""
+    st = gen.make_layer_stack()
+    L, bs, H, K, E = st.layers, st.bs, st.hidden, st.top_k, st.num_experts
+    ids = [dev(a) for a in st.expert_ids]
+    scs = [dev(a) for a in st.expert_scales]
+    gms = [dev_bf16(a) for a in st.gammas]
+    table = dev(st.table)
+    x0, r0 = dev_bf16(st.x0), dev_bf16(st.residual0)
+    wsp = B.new_workspace()
+    bal = [torch.empty((bs, K), dtype=torch.int32, device="cuda") for _ in range(L)]
+    bm = [torch.empty((bs, K), dtype=torch.uint8, device="cuda") for _ in range(L)]
+    dsp = [B.alloc_dispatch_outputs(bs, H, K, E, 0) for _ in range(L)]
+    outs = [dict(y=torch.empty((bs, H), dtype=torch.bfloat16, device="cuda"),
+                 x_out=torch.empty((bs, H), dtype=torch.bfloat16, device="cuda"), rstd=None) for _ in range(L)]
+
+    def stack():
+        x, r = x0, r0
+        for l in range(L):
+            B.update_expert(ids[l], table, st.ep_world_size, expert_scales=scs[l], workspace=wsp,
+                            out=(bal[l], bm[l]))
+            B.dispatch(x, bal[l], E, st.ep_world_size, 0, mask=bm[l], workspace=wsp, out=dsp[l])
+            B.combine_add_rmsnorm(dsp[l]["expand_x"], dsp[l]["expand_idx"], scs[l], r, gms[l], st.norm_eps,
+                                  workspace=wsp, out=outs[l])
+            x, r = outs[l]["y"], outs[l]["x_out"]
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        stack()  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    for o in outs:
+        o["y"].zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        stack()
+    g.replay()
+    torch.cuda.synchronize()
+    assert B.read_device_error(wsp) == 0
+
+    x, r = st.x0, st.residual0
+    for l in range(L):
+        ob, om, _ = orc.update_expert(st.expert_ids[l], st.table, st.ep_world_size,
+                                      expert_scales=st.expert_scales[l])
+        d = orc.dispatch(x, ob, E, 0, mask=om)
+        c = orc.combine_add_rmsnorm(d["expand_x"], d["expand_idx"], st.expert_scales[l], r, st.gammas[l],
+                                    st.norm_eps)
+        if l in (0, L // 2, L - 1):
+            assert_close_bf16(host(outs[l]["y"]), c["y_f64"], what=f"y layer {l}")
+            assert_close_bf16(host(outs[l]["x_out"]), c["x_f64"], what=f"x_out layer {l}")
+        if l == 0:
+            np.testing.assert_array_equal(host(dsp[0]["expand_idx"]), d["expand_idx"])
+        x, r = c["y"], c["x_out"]
