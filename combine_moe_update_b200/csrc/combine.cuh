@@ -5,13 +5,13 @@
 //   x = combineOut + residualX
 //   y = x / sqrt(mean(x^2) + normEps) * gamma
 //
-// One block of 256 threads per token.  Thread t owns the 8-element vectors
-// p = t, t + 256, ... of the row (H <= 8192 -> at most 4).  For each vector
-// it issues the K expert-row loads (the AllToAllV back, as a gather through
-// expand_idx), the shared-expert and residual loads at once, accumulates in
-// fp32 and keeps x in registers; one block reduction gives sum(x^2), then y
-// is written.  Each input byte is read once and each output byte written
-// once.
+// One block of 256 threads per token.  For each 8-element vector of the row
+// a thread issues the K expert-row loads (the AllToAllV back: a gather
+// through expand_idx), the shared-expert and the residual load together,
+// accumulates in fp32 and parks x in shared memory (so registers stay low
+// and several blocks share an SM, keeping enough bytes in flight).  One
+// block reduction gives sum(x^2); a second sweep over shared memory writes y
+// (and x).  Every input byte is read once and every output byte written once.
 #pragma once
 #include "common.cuh"
 
@@ -33,10 +33,13 @@ struct CombineArgs {
 };
 
 constexpr int kCbThreads = 256;
-constexpr int kCbVecs = 4;  // 8-element vectors per thread (H / 8 <= 1024)
 
-template <int KMAX, bool SHARED>
+inline size_t combine_smem_bytes(int hidden) { return (size_t)hidden * sizeof(float); }
+
+// KB: expert rows whose loads are issued together (<= KMAX).
+template <int KMAX, int KB, bool SHARED>
 __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
+    extern __shared__ __align__(16) float s_x[];  // x of this token, fp32 [H]
     __shared__ int s_row[16];
     __shared__ float s_w[16];
     __shared__ float s_red[kCbThreads / 32];
@@ -45,7 +48,7 @@ __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
 
     if (t < K) {
         int row = a.expand_idx[i * K + t];
-        float w = a.scales[i * K + t];
+        const float w = a.scales[i * K + t];
         if (row < -1 || row >= a.expand_rows) {
             raise_error(a.err, kDevBadId);
             row = -1;
@@ -66,34 +69,29 @@ __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
     }
 
     const size_t tok = (size_t)i * H;
-    float xs[kCbVecs][8];
-    uint4 gv[kCbVecs];
     float ss = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kCbVecs; ++j) {
-        const int p = t + j * kCbThreads;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xs[j][e] = 0.0f;
-        if (p >= V) continue;
-        uint4 rv[KMAX];
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            if (row[k] >= 0) rv[k] = ld_stream(a.expand_x + (size_t)row[k] * H + p * 8);
+#pragma unroll 1
+    for (int p = t; p < V; p += kCbThreads) {
         const uint4 res = ld_stream(a.residual + tok + p * 8);
         uint4 sh = make_uint4(0, 0, 0, 0);
         if constexpr (SHARED) sh = ld_stream(a.shared_x + tok + p * 8);
-        gv[j] = ld_cached(a.gamma + p * 8);
-
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
 #pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            if (row[k] < 0) continue;
-            float f[8];
-            unpack8(rv[k], f);
+        for (int k0 = 0; k0 < KMAX; k0 += KB) {
+            uint4 rv[KB];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(wk[k], f[e], acc[e]);
+            for (int k = 0; k < KB; ++k)
+                if (row[k0 + k] >= 0) rv[k] = ld_stream(a.expand_x + (size_t)row[k0 + k] * H + p * 8);
+#pragma unroll
+            for (int k = 0; k < KB; ++k) {
+                if (row[k0 + k] < 0) continue;
+                float f[8];
+                unpack8(rv[k], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wk[k0 + k], f[e], acc[e]);
+            }
         }
         if constexpr (SHARED) {
             float f[8];
@@ -105,33 +103,37 @@ __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
         unpack8(res, r);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            xs[j][e] = acc[e] + r[e];
-            ss = fmaf(xs[j][e], xs[j][e], ss);
+            acc[e] += r[e];
+            ss = fmaf(acc[e], acc[e], ss);
         }
+        float4 *xs = reinterpret_cast<float4 *>(s_x + p * 8);
+        xs[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        xs[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 
-    ss = block_sum<kCbThreads / 32>(ss, s_red);
+    ss = block_sum<kCbThreads / 32>(ss, s_red);  // its barriers also publish s_x
     const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(ss, (float)H) + a.norm_eps));
     if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
 
-#pragma unroll
-    for (int j = 0; j < kCbVecs; ++j) {
-        const int p = t + j * kCbThreads;
-        if (p >= V) continue;
+#pragma unroll 1
+    for (int p = t; p < V; p += kCbThreads) {
+        const float4 *xs = reinterpret_cast<const float4 *>(s_x + p * 8);
+        const float4 x0 = xs[0], x1 = xs[1];
+        const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         float g[8];
-        unpack8(gv[j], g);
+        unpack8(ld_cached(a.gamma + p * 8), g);
         uint4 yo;
-        yo.x = pack_bf16x2(xs[j][0] * rstd * g[0], xs[j][1] * rstd * g[1]);
-        yo.y = pack_bf16x2(xs[j][2] * rstd * g[2], xs[j][3] * rstd * g[3]);
-        yo.z = pack_bf16x2(xs[j][4] * rstd * g[4], xs[j][5] * rstd * g[5]);
-        yo.w = pack_bf16x2(xs[j][6] * rstd * g[6], xs[j][7] * rstd * g[7]);
+        yo.x = pack_bf16x2(x[0] * rstd * g[0], x[1] * rstd * g[1]);
+        yo.y = pack_bf16x2(x[2] * rstd * g[2], x[3] * rstd * g[3]);
+        yo.z = pack_bf16x2(x[4] * rstd * g[4], x[5] * rstd * g[5]);
+        yo.w = pack_bf16x2(x[6] * rstd * g[6], x[7] * rstd * g[7]);
         st_v4(a.y + tok + p * 8, yo);
         if (a.x_out) {
             uint4 xo;
-            xo.x = pack_bf16x2(xs[j][0], xs[j][1]);
-            xo.y = pack_bf16x2(xs[j][2], xs[j][3]);
-            xo.z = pack_bf16x2(xs[j][4], xs[j][5]);
-            xo.w = pack_bf16x2(xs[j][6], xs[j][7]);
+            xo.x = pack_bf16x2(x[0], x[1]);
+            xo.y = pack_bf16x2(x[2], x[3]);
+            xo.z = pack_bf16x2(x[4], x[5]);
+            xo.w = pack_bf16x2(x[6], x[7]);
             st_v4(a.x_out + tok + p * 8, xo);
         }
     }

@@ -1,47 +1,72 @@
-// dispatch.cuh -- quantize each token and scatter its K copies into the
+// dispatch.cuh -- quantize the tokens and scatter their K copies into the
 // expert-major receive buffer (aclnnMoeDistributeDispatchV2, "计算公式").
 //
-// One block of 128 threads per token.  Thread t owns the 16-element chunks
-// c = t, t + 128, ... of the row (H <= 8192 -> at most 4 chunks): it loads
-// them once with 16-byte loads and keeps them in registers.  Then, per mode:
-//   0  (case 1)  copy: the bf16 row is written to every destination row;
-//   2  (case 3)  per-token int8: block-wide max |xFp32| via warp shuffles,
-//                dyn = 127 / amax, q = rint(xFp32 * dyn), scale = 1 / dyn;
-//   3  (case 4)  the same per 128-element tile: the 8 threads sharing a tile
-//                reduce with three xor-shuffles;
-//   4  (case 5)  mxfp8: per 32-element block (two threads, one shuffle)
-//                sharedExp = floor(log2 amax) - 8, read exactly from the
-//                exponent bits; q = e4m3_satfinite(x * 2^-sharedExp); the
-//                scale byte is sharedExp + 127 (E8M0).
-// Without smooth scales all K copies are identical, so the codes are made
-// once -- while the ranking kernel is still running (programmatic dependent
-// launch) -- and only the K row writes wait for it.  With per-instance smooth
-// scales (modes 2 and 3) every copy is quantized with its own instance's
-// smooth row.
+// The EP AllToAllV is, on one GPU, a permutation of the (token, k) copies
+// into rank-major rows; the page requires a deterministic result
+// ("确定性计算"), so a copy's row is its position in (instance, token, k)
+// order.  Each kernel below is the whole operation in one launch: every
+// block rebuilds what it needs of that order from the (at most 8192) copy
+// keys -- a warp-aggregated shared-memory histogram plus a scan -- while its
+// own row loads are in flight.  Counts decide nothing about order, so the
+// result is the same on every run.
 //
-// All quantization arithmetic is IEEE binary32 with explicit round-to-
-// nearest intrinsics, so no contraction or approximation can move a code.
+// dispatch_token_kernel<MODE>   one block per token, no smooth scales: the
+//   row is loaded once (16-byte loads kept in registers), quantized once
+//   (all K copies are identical) and written K times.
+// dispatch_instance_kernel<MODE> smooth scales (modes 2, 3): one block per
+//   (instance, slice of its rows).  The instance's smooth row is staged in
+//   shared memory by one TMA bulk copy; the block then streams its rows'
+//   tokens from L2, one row ahead, so every smooth row is read from memory
+//   once instead of once per copy.
+//
+// Quantization, per mode ("计算公式" cases 1, 3, 4, 5):
+//   0  copy the bf16 row;
+//   2  xFp32 = x * smooth; dyn = 127 / max|xFp32| over the row;
+//      q = rint(xFp32 * dyn) clamped to [-127, 127]; scale = 1 / dyn;
+//   3  the same per 128-element tile (reduced with xor-shuffles);
+//   4  mxfp8: per 32-element block sharedExp = floor(log2 max|x|) - 8 taken
+//      from the exponent bits; q = e4m3_satfinite(x * 2^-sharedExp); scale
+//      byte = sharedExp + 127.
+// All of it in IEEE binary32 with explicit round-to-nearest intrinsics, so no
+// contraction or approximation can move a code.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
 struct DispatchArgs {
-    int bs, hidden, top_k, tiles;  // tiles = ceil(H / 128) (mode 3)
-    const uint16_t *x;             // bf16 bits [bs, H]
-    const int32_t *ids;            // instance ids [bs, K]
-    const float *smooth;           // [E, H] or null
+    int bs, hidden, top_k, num_instances;
+    int tiles;   // ceil(H / 128) (mode 3)
+    int splits;  // blocks per instance (instance kernel)
+    const uint16_t *x;  // bf16 bits [bs, H]
+    const int32_t *ids;  // instance ids [bs, K]
+    const uint8_t *mask;  // [bs, K] or null
+    const float *smooth;  // [E, H] or null
     void *expand_x;
     void *dyn_scales;
-    const int32_t *expand_idx;  // written by rank_kernel
+    int32_t *expand_idx;
+    int32_t *src_of_row;
+    int32_t *counts;
+    int32_t *offsets;
     uint32_t *err;
 };
 
-constexpr int kDpThreads = 128;
-constexpr int kDpChunks = 4;  // 16-element chunks per thread (H / 16 <= 512)
+constexpr int kDpThreads = 256;
+constexpr int kDpWarps = kDpThreads / 32;
+constexpr int kKeyBatch = 8;  // copy keys loaded per thread before they are used
 
-// xFp32 of one 16-element chunk: bf16 -> f32 (exact), times the smooth row.
-__device__ __forceinline__ void chunk_xf(const uint4 (&xv)[2], const float *sm, float (&f)[16]) {
+// Key of copy j: its instance if it is sent, -1 if masked out, -2 if its id
+// is out of range (then it is dropped and reported).
+__device__ __forceinline__ int copy_key(const DispatchArgs &a, int j) {
+    if (a.mask && a.mask[j] == 0) return -1;
+    const int id = __ldg(a.ids + j);
+    return (id >= 0 && id < a.num_instances) ? id : -2;
+}
+
+// ------------------------------------------------------------ quantizers ---
+
+// 16 bf16 of a chunk -> floats (exact).
+__device__ __forceinline__ void chunk16(const uint4 (&xv)[2], float (&f)[16]) {
     float a[8], b[8];
     unpack8(xv[0], a);
     unpack8(xv[1], b);
@@ -50,46 +75,38 @@ __device__ __forceinline__ void chunk_xf(const uint4 (&xv)[2], const float *sm, 
         f[e] = a[e];
         f[8 + e] = b[e];
     }
-    if (sm) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 s = __ldg(reinterpret_cast<const float4 *>(sm) + q);
-            f[4 * q + 0] = __fmul_rn(f[4 * q + 0], s.x);
-            f[4 * q + 1] = __fmul_rn(f[4 * q + 1], s.y);
-            f[4 * q + 2] = __fmul_rn(f[4 * q + 2], s.z);
-            f[4 * q + 3] = __fmul_rn(f[4 * q + 3], s.w);
-        }
-    }
 }
 
-__device__ __forceinline__ float chunk_amax(const float (&f)[16]) {
+template <int N>
+__device__ __forceinline__ float abs_max(const float (&f)[N]) {
     float m = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(f[e]));
+    for (int e = 0; e < N; ++e) m = fmaxf(m, fabsf(f[e]));
     return m;
 }
 
-// int8 codes of a chunk: clamp(rint(xf * dyn), -127, 127); all zero when
-// the segment's amax is 0 (dyn would be +inf).
-__device__ __forceinline__ uint4 chunk_int8(const float (&f)[16], float dyn, bool zero) {
-    uint32_t w[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            int v = __float2int_rn(__fmul_rn(f[4 * q + e], dyn));
-            v = v > 127 ? 127 : (v < -127 ? -127 : v);
-            word |= (uint32_t)(v & 0xff) << (8 * e);
-        }
-        w[q] = zero ? 0u : word;
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
+// clamp(rint(v * dyn), -127, 127) as one byte.
+__device__ __forceinline__ uint32_t q8(float v, float dyn) {
+    int q = __float2int_rn(__fmul_rn(v, dyn));
+    q = q > 127 ? 127 : (q < -127 ? -127 : q);
+    return (uint32_t)(q & 0xff);
 }
 
-// sharedExp = floor(log2 amax) - 8 (emax of e4m3), clamped to >= -127;
-// -127 for an all-zero block.  floor(log2) comes from the exponent field
-// (or the leading mantissa bit of a subnormal), never from a log routine.
+// Four int8 codes per 32-bit word; all zero when the segment's amax is 0
+// (dyn would be +inf there).
+template <int NW>
+__device__ __forceinline__ void pack_int8(const float *f, float dyn, bool zero, uint32_t *w) {
+#pragma unroll
+    for (int q = 0; q < NW; ++q) {
+        const uint32_t word = q8(f[4 * q], dyn) | (q8(f[4 * q + 1], dyn) << 8) | (q8(f[4 * q + 2], dyn) << 16) |
+                              (q8(f[4 * q + 3], dyn) << 24);
+        w[q] = zero ? 0u : word;
+    }
+}
+
+// sharedExp = floor(log2 amax) - 8 (emax of e4m3), clamped to >= -127; -127
+// for an all-zero block.  floor(log2) comes from the exponent field (or the
+// leading mantissa bit of a subnormal), never from a logarithm routine.
 __device__ __forceinline__ int mx_shared_exp(float amax) {
     if (amax == 0.0f) return -127;
     const uint32_t b = __float_as_uint(amax);
@@ -99,10 +116,10 @@ __device__ __forceinline__ int mx_shared_exp(float amax) {
     return se < -127 ? -127 : se;
 }
 
-// e4m3 codes of a chunk: round to nearest even, saturate to +-448.  The
+// e4m3 codes of 16 values, round to nearest even, saturating at +-448.  The
 // multiply by the exact power of two 2^-se equals the page's X / 2^se.
-__device__ __forceinline__ uint4 chunk_e4m3(const float (&f)[16], int se) {
-    const float inv = __uint_as_float((uint32_t)(127 - se) << 23);  // 2^-se, normal for se in [-127, 119]
+__device__ __forceinline__ uint4 e4m3x16(const float (&f)[16], int se) {
+    const float inv = __uint_as_float((uint32_t)(127 - se) << 23);  // 2^-se; normal for se in [-127, 119]
     uint32_t w[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -115,112 +132,31 @@ __device__ __forceinline__ uint4 chunk_e4m3(const float (&f)[16], int se) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Quantized codes of this thread's chunks plus the scales it must write.
-struct QuantOut {
-    uint4 q[kDpChunks];
-    float seg_scale[kDpChunks];  // mode 3: scale of the chunk's tile
-    uint8_t e8[kDpChunks];       // mode 4: E8M0 byte of the chunk's block
-    float row_scale;             // mode 2
-};
+// --------------------------------------------------------- token kernel ---
+
+constexpr int kTkChunks = 2;  // 16-element chunks per thread: H / 16 <= 512 = 256 * 2
+
+inline size_t token_smem_bytes(int num_instances) { return 3 * (size_t)num_instances * sizeof(int); }
 
 template <int MODE>
-__device__ __forceinline__ void quantize_row(const uint4 (&xv)[kDpChunks][2], const float *sm_row,
-                                             int nchunk, float *s_red, QuantOut &o) {
-    const int t = threadIdx.x;
-    float amax[kDpChunks];
-#pragma unroll
-    for (int j = 0; j < kDpChunks; ++j) {
-        const int c = t + j * kDpThreads;
-        amax[j] = 0.0f;
-        if (c < nchunk) {
-            float f[16];
-            chunk_xf(xv[j], sm_row ? sm_row + c * 16 : nullptr, f);
-            amax[j] = chunk_amax(f);
-        }
-    }
-    if constexpr (MODE == 2) {
-        float m = 0.0f;
-#pragma unroll
-        for (int j = 0; j < kDpChunks; ++j) m = fmaxf(m, amax[j]);
-        m = block_max<kDpThreads / 32>(m, s_red);
-        const float dyn = __fdiv_rn(127.0f, m);  // +inf when m == 0
-        o.row_scale = __frcp_rn(dyn);           // 1 / dynamicScales (0 when m == 0)
-#pragma unroll
-        for (int j = 0; j < kDpChunks; ++j) {
-            const int c = t + j * kDpThreads;
-            if (c < nchunk) {
-                float f[16];
-                chunk_xf(xv[j], sm_row ? sm_row + c * 16 : nullptr, f);
-                o.q[j] = chunk_int8(f, dyn, m == 0.0f);
-            }
-        }
-    } else if constexpr (MODE == 3) {
-#pragma unroll
-        for (int j = 0; j < kDpChunks; ++j) {
-            float m = amax[j];  // the 8 lanes of one 128-element tile
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
-            const float dyn = __fdiv_rn(127.0f, m);
-            o.seg_scale[j] = __frcp_rn(dyn);
-            const int c = t + j * kDpThreads;
-            if (c < nchunk) {
-                float f[16];
-                chunk_xf(xv[j], sm_row ? sm_row + c * 16 : nullptr, f);
-                o.q[j] = chunk_int8(f, dyn, m == 0.0f);
-            }
-        }
-    } else if constexpr (MODE == 4) {
-#pragma unroll
-        for (int j = 0; j < kDpChunks; ++j) {
-            float m = amax[j];  // the 2 lanes of one 32-element block
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-            const int se = mx_shared_exp(m);
-            o.e8[j] = (uint8_t)(se + 127);
-            const int c = t + j * kDpThreads;
-            if (c < nchunk) {
-                float f[16];
-                chunk_xf(xv[j], nullptr, f);
-                o.q[j] = chunk_e4m3(f, se);
-            }
-        }
-    }
-}
+__global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs a) {
+    extern __shared__ __align__(16) int smem_i[];
+    const int E = a.num_instances;
+    int *hist = smem_i;       // sent copies per instance
+    int *pref = hist + E;     // ... among the copies of earlier tokens
+    int *off = pref + E;      // exclusive prefix of hist
+    __shared__ float s_red[kDpWarps];
+    __shared__ int s_warp[32];
+    __shared__ int s_key[16], s_row[16];
 
-template <int MODE>
-__device__ __forceinline__ void write_copy(const DispatchArgs &a, int row, int nchunk, const QuantOut &o) {
-    const int t = threadIdx.x, H = a.hidden;
-    uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
-#pragma unroll
-    for (int j = 0; j < kDpChunks; ++j) {
-        const int c = t + j * kDpThreads;
-        if (c < nchunk) {
-            st_v4(dst + c * 16, o.q[j]);
-            if constexpr (MODE == 3) {
-                if ((t & 7) == 0) reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (c >> 3)] = o.seg_scale[j];
-            }
-            if constexpr (MODE == 4) {
-                if ((t & 1) == 0) reinterpret_cast<uint8_t *>(a.dyn_scales)[(size_t)row * (H >> 5) + (c >> 1)] = o.e8[j];
-            }
-        }
-    }
-    if constexpr (MODE == 2) {
-        if (t == 0) reinterpret_cast<float *>(a.dyn_scales)[row] = o.row_scale;
-    }
-}
+    const int i = blockIdx.x, t = threadIdx.x, lane = t & 31;
+    const int H = a.hidden, nchunk = H >> 4, K = a.top_k, N = a.bs * K, mine = i * K;
 
-template <int MODE, bool SMOOTH>
-__global__ void __launch_bounds__(kDpThreads) dispatch_kernel(DispatchArgs a) {
-    __shared__ float s_red[kDpThreads / 32];
-    __shared__ int s_rows[16], s_inst[16];
-    const int i = blockIdx.x, t = threadIdx.x;
-    const int H = a.hidden, nchunk = H >> 4, K = a.top_k;
-
-    // The token's row: inputs of the call, safe to read before pdl_wait().
+    // 1. this token's row: issue the loads first, use them last
     const uint16_t *xrow = a.x + (size_t)i * H;
-    uint4 xv[kDpChunks][2];
+    uint4 xv[kTkChunks][2];
 #pragma unroll
-    for (int j = 0; j < kDpChunks; ++j) {
+    for (int j = 0; j < kTkChunks; ++j) {
         const int c = t + j * kDpThreads;
         if (c < nchunk) {
             xv[j][0] = ld_stream(xrow + c * 16);
@@ -230,46 +166,348 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_kernel(DispatchArgs a) {
         }
     }
 
-    if constexpr (MODE == 0) {
-        pdl_wait();  // expand_idx comes from rank_kernel
-        if (t < K) s_rows[t] = a.expand_idx[i * K + t];
-        __syncthreads();
-        for (int k = 0; k < K; ++k) {
-            const int row = s_rows[k];
-            if (row < 0) continue;
+    // 2. histogram of all sent copies and of those of earlier tokens
+    for (int q = t; q < 2 * E; q += kDpThreads) smem_i[q] = 0;
+    if (t < K) s_key[t] = copy_key(a, mine + t);
+    __syncthreads();
+    for (int j0 = 0; j0 < N; j0 += kDpThreads * kKeyBatch) {  // uniform trip count
+        int key[kKeyBatch];
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int j = j0 + u * kDpThreads + t;
+            key[u] = j < N ? copy_key(a, j) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int j = j0 + u * kDpThreads + t;
+            int k = key[u];
+            if (k == -2) {
+                if (i == 0) raise_error(a.err, kDevBadId);
+                k = -1;
+            }
+            const bool early = j < mine;
+            const unsigned peers = __match_any_sync(kFull, k < 0 ? -1 : (k << 1) | (early ? 1 : 0));
+            if (k >= 0 && lane == __ffs(peers) - 1) {
+                atomicAdd(&hist[k], __popc(peers));
+                if (early) atomicAdd(&pref[k], __popc(peers));
+            }
+        }
+    }
+    __syncthreads();
+
+    // 3. bucket offsets: 4 consecutive instances per thread (E <= 1024)
+    int v[4], sum = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int b = t * 4 + u;
+        v[u] = b < E ? hist[b] : 0;
+        sum += v[u];
+    }
+    const int incl = block_inclusive_scan(sum, s_warp);
+    const int total = s_warp[kDpWarps - 1];
+    int run = incl - sum;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int b = t * 4 + u;
+        if (b < E) {
+            off[b] = run;
+            if (i == 0) {
+                a.counts[b] = v[u];
+                a.offsets[b] = run;
+            }
+        }
+        run += v[u];
+    }
+    if (i == 0 && t == 0) a.offsets[E] = total;
+    __syncthreads();
+
+    // 4. rows of this token's copies
+    if (t < K) {
+        const int k = s_key[t];
+        int row = -1;
+        if (k >= 0) {
+            int same = 0;
+            for (int u = 0; u < t; ++u) same += (s_key[u] == k);
+            row = off[k] + pref[k] + same;
+            a.src_of_row[row] = mine + t;
+        }
+        a.expand_idx[mine + t] = row;
+        s_row[t] = row;
+    }
+    __syncthreads();
+
+    // 5. quantize once, write every copy
+    uint4 q[kTkChunks];
+    float seg[kTkChunks];
+    uint8_t e8[kTkChunks];
+    float row_scale = 0.0f;
+    if constexpr (MODE == 2) {
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kTkChunks; ++j) {
+            float f[16];
+            chunk16(xv[j], f);
+            m = fmaxf(m, abs_max(f));
+        }
+        m = block_max<kDpWarps>(m, s_red);
+        const float dyn = __fdiv_rn(127.0f, m);  // +inf when m == 0
+        row_scale = __frcp_rn(dyn);              // 1 / dynamicScales (0 when m == 0)
+#pragma unroll
+        for (int j = 0; j < kTkChunks; ++j) {
+            float f[16];
+            chunk16(xv[j], f);
+            uint32_t w[4];
+            pack_int8<4>(f, dyn, m == 0.0f, w);
+            q[j] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else if constexpr (MODE == 3) {
+#pragma unroll
+        for (int j = 0; j < kTkChunks; ++j) {
+            float f[16];
+            chunk16(xv[j], f);
+            float m = abs_max(f);  // the 8 lanes sharing a 128-element tile
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+            const float dyn = __fdiv_rn(127.0f, m);
+            seg[j] = __frcp_rn(dyn);
+            uint32_t w[4];
+            pack_int8<4>(f, dyn, m == 0.0f, w);
+            q[j] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else if constexpr (MODE == 4) {
+#pragma unroll
+        for (int j = 0; j < kTkChunks; ++j) {
+            float f[16];
+            chunk16(xv[j], f);
+            float m = abs_max(f);  // the 2 lanes sharing a 32-element block
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+            const int se = mx_shared_exp(m);
+            e8[j] = (uint8_t)(se + 127);
+            q[j] = e4m3x16(f, se);
+        }
+    }
+
+    for (int k = 0; k < K; ++k) {
+        const int row = s_row[k];
+        if (row < 0) continue;
+        if constexpr (MODE == 0) {
             uint16_t *dst = reinterpret_cast<uint16_t *>(a.expand_x) + (size_t)row * H;
 #pragma unroll
-            for (int j = 0; j < kDpChunks; ++j) {
+            for (int j = 0; j < kTkChunks; ++j) {
                 const int c = t + j * kDpThreads;
                 if (c < nchunk) {
                     st_v4(dst + c * 16, xv[j][0]);
                     st_v4(dst + c * 16 + 8, xv[j][1]);
                 }
             }
+        } else {
+            uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
+#pragma unroll
+            for (int j = 0; j < kTkChunks; ++j) {
+                const int c = t + j * kDpThreads;
+                if (c < nchunk) {
+                    st_v4(dst + c * 16, q[j]);
+                    if constexpr (MODE == 3) {
+                        if ((t & 7) == 0)
+                            reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (c >> 3)] = seg[j];
+                    }
+                    if constexpr (MODE == 4) {
+                        if ((t & 1) == 0)
+                            reinterpret_cast<uint8_t *>(a.dyn_scales)[(size_t)row * (H >> 5) + (c >> 1)] = e8[j];
+                    }
+                }
+            }
+            if constexpr (MODE == 2) {
+                if (t == 0) reinterpret_cast<float *>(a.dyn_scales)[row] = row_scale;
+            }
         }
-    } else if constexpr (!SMOOTH) {
-        QuantOut o;
-        quantize_row<MODE>(xv, nullptr, nchunk, s_red, o);
-        pdl_wait();
-        if (t < K) s_rows[t] = a.expand_idx[i * K + t];
-        __syncthreads();
-        for (int k = 0; k < K; ++k) {
-            const int row = s_rows[k];
-            if (row >= 0) write_copy<MODE>(a, row, nchunk, o);
+    }
+}
+
+// ------------------------------------------------------ instance kernel ---
+
+constexpr int kImVecs = 4;  // 8-element vectors per thread: H / 8 <= 1024 = 256 * 4
+
+// Copies per warp in the instance kernel's key scan (a multiple of 32).
+__host__ __device__ inline int im_per_warp(int copies) { return ((copies + kDpWarps - 1) / kDpWarps + 31) & ~31; }
+
+// Dynamic shared memory: the smooth row, then one copy list per warp.
+inline size_t instance_smem_bytes(int hidden, int copies) {
+    return (size_t)hidden * sizeof(float) + (size_t)kDpWarps * im_per_warp(copies) * sizeof(int);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_b[];
+    const int H = a.hidden, K = a.top_k, N = a.bs * K, E = a.num_instances, V = H >> 3;
+    float *s_sm = reinterpret_cast<float *>(smem_b);
+    int *s_list = reinterpret_cast<int *>(smem_b + (size_t)H * sizeof(float));
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ int s_wcnt[kDpWarps], s_wless[kDpWarps], s_ok;
+    __shared__ float s_red[kDpWarps];
+
+    const int e = blockIdx.x / a.splits, sp = blockIdx.x % a.splits;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+
+    // 1. the instance's smooth row -> shared memory, one bulk copy
+    if (t == 0) {
+        mbar_init(&s_bar, 1);
+        mbar_arrive_expect_tx(&s_bar, (uint32_t)H * sizeof(float));
+        bulk_copy_g2s(s_sm, a.smooth + (size_t)e * H, (uint32_t)H * sizeof(float), &s_bar);
+    }
+
+    // 2. the copies sent to instance e, in (token, k) order: warp w scans the
+    //    contiguous range [w * per_warp, (w + 1) * per_warp) of copies
+    const int per_warp = im_per_warp(N);
+    const unsigned lower = (1u << lane) - 1u;
+    int cnt = 0, less = 0;
+    for (int b0 = 0; b0 < per_warp; b0 += 32 * kKeyBatch) {  // uniform trip count
+        int key[kKeyBatch];
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int off = b0 + u * 32 + lane;
+            const int j = w * per_warp + off;
+            key[u] = (off < per_warp && j < N) ? copy_key(a, j) : -1;
         }
-    } else {
-        pdl_wait();
-        if (t < K) {
-            s_rows[t] = a.expand_idx[i * K + t];
-            s_inst[t] = a.ids[i * K + t];
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int off = b0 + u * 32 + lane;
+            const int j = w * per_warp + off;
+            int k = key[u];
+            if (k == -2 && blockIdx.x == 0) raise_error(a.err, kDevBadId);
+            if (blockIdx.x == 0 && k < 0 && off < per_warp && j < N) a.expand_idx[j] = -1;  // not sent
+            less += (k >= 0 && k < e) ? 1 : 0;
+            const unsigned hit = __ballot_sync(kFull, k == e);
+            if (k == e) s_list[w * per_warp + cnt + __popc(hit & lower)] = j;
+            cnt += __popc(hit);
         }
-        __syncthreads();
-        for (int k = 0; k < K; ++k) {
-            const int row = s_rows[k];  // same value in every thread: the branch is uniform
-            if (row < 0) continue;
-            QuantOut o;
-            quantize_row<MODE>(xv, a.smooth + (size_t)s_inst[k] * H, nchunk, s_red, o);
-            write_copy<MODE>(a, row, nchunk, o);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) less += __shfl_xor_sync(kFull, less, o);
+    if (lane == 0) {
+        s_wcnt[w] = cnt;
+        s_wless[w] = less;
+    }
+    __syncthreads();
+    int wpre[kDpWarps + 1];
+    wpre[0] = 0;
+    int start = 0;
+#pragma unroll
+    for (int u = 0; u < kDpWarps; ++u) {
+        wpre[u + 1] = wpre[u] + s_wcnt[u];
+        start += s_wless[u];
+    }
+    const int count = wpre[kDpWarps];
+    if (sp == 0 && t == 0) {
+        a.counts[e] = count;
+        a.offsets[e] = start;
+        if (e == E - 1) a.offsets[E] = start + count;
+    }
+    const int r0 = (int)((long long)count * sp / a.splits);
+    const int r1 = (int)((long long)count * (sp + 1) / a.splits);
+    auto copy_of = [&](int r) {  // r-th copy of the bucket: which warp's list holds it
+        int u = 0, base = 0;
+#pragma unroll
+        for (int q = 1; q < kDpWarps; ++q)
+            if (wpre[q] <= r) {
+                u = q;
+                base = wpre[q];
+            }
+        return s_list[u * per_warp + (r - base)];
+    };
+    for (int r = r0 + t; r < r1; r += kDpThreads) {
+        const int j = copy_of(r);
+        a.src_of_row[start + r] = j;
+        a.expand_idx[j] = start + r;
+    }
+
+    // 3. wait (bounded) for the smooth row
+    if (t == 0) s_ok = mbar_wait_bounded(&s_bar, 0) ? 1 : 0;
+    __syncthreads();
+    if (!s_ok) {
+        if (t == 0) {
+            raise_error(a.err, kDevTimeout);
+            mbar_wait_bounded(&s_bar, 0);  // a last bounded wait for the copy in flight
+        }
+        return;
+    }
+
+    // 4. quantize the rows, loading the next row's token while this one reduces
+    const float4 *sm4 = reinterpret_cast<const float4 *>(s_sm);
+    auto load_row = [&](int r, uint4 (&xv)[kImVecs]) {
+        const uint16_t *xr = a.x + (size_t)(copy_of(r) / K) * H;
+#pragma unroll
+        for (int q = 0; q < kImVecs; ++q) {
+            const int p = t + q * kDpThreads;
+            xv[q] = p < V ? ld_stream(xr + p * 8) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    auto xf_of = [&](const uint4 &xq, int p, float (&f)[8]) {
+        unpack8(xq, f);
+        const float4 s0 = sm4[2 * p], s1 = sm4[2 * p + 1];
+        f[0] = __fmul_rn(f[0], s0.x); f[1] = __fmul_rn(f[1], s0.y);
+        f[2] = __fmul_rn(f[2], s0.z); f[3] = __fmul_rn(f[3], s0.w);
+        f[4] = __fmul_rn(f[4], s1.x); f[5] = __fmul_rn(f[5], s1.y);
+        f[6] = __fmul_rn(f[6], s1.z); f[7] = __fmul_rn(f[7], s1.w);
+    };
+    uint4 xn[kImVecs];
+    if (r0 < r1) load_row(r0, xn);
+    for (int r = r0; r < r1; ++r) {  // uniform over the block
+        uint4 xc[kImVecs];
+#pragma unroll
+        for (int q = 0; q < kImVecs; ++q) xc[q] = xn[q];
+        if (r + 1 < r1) load_row(r + 1, xn);
+        const int row = start + r;
+        uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
+        if constexpr (MODE == 2) {
+            float m = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kImVecs; ++q) {
+                const int p = t + q * kDpThreads;
+                if (p < V) {
+                    float f[8];
+                    xf_of(xc[q], p, f);
+                    m = fmaxf(m, abs_max(f));
+                }
+            }
+            m = block_max<kDpWarps>(m, s_red);
+            const float dyn = __fdiv_rn(127.0f, m);
+#pragma unroll
+            for (int q = 0; q < kImVecs; ++q) {
+                const int p = t + q * kDpThreads;
+                if (p < V) {
+                    float f[8];
+                    xf_of(xc[q], p, f);
+                    uint32_t wd[2];
+                    pack_int8<2>(f, dyn, m == 0.0f, wd);
+                    *reinterpret_cast<uint2 *>(dst + p * 8) = make_uint2(wd[0], wd[1]);
+                }
+            }
+            if (t == 0) reinterpret_cast<float *>(a.dyn_scales)[row] = __frcp_rn(dyn);
+        } else {  // MODE 3: a 128-element tile is 16 vectors = 16 consecutive lanes
+#pragma unroll
+            for (int q = 0; q < kImVecs; ++q) {
+                const int p = t + q * kDpThreads;
+                float f[8];
+                float m = 0.0f;
+                if (p < V) {
+                    xf_of(xc[q], p, f);
+                    m = abs_max(f);
+                }
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
+                if (p < V) {
+                    const float dyn = __fdiv_rn(127.0f, m);
+                    uint32_t wd[2];
+                    pack_int8<2>(f, dyn, m == 0.0f, wd);
+                    *reinterpret_cast<uint2 *>(dst + p * 8) = make_uint2(wd[0], wd[1]);
+                    if ((t & 15) == 0)
+                        reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (p >> 4)] = __frcp_rn(dyn);
+                }
+            }
         }
     }
 }

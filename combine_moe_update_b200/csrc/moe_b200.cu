@@ -1,6 +1,6 @@
 // moe_b200.cu -- the C ABI of include/moe_b200.h: host-side validation,
 // workspace sizing and kernel launches.  All compute is in the kernels of
-// update_expert.cuh, rank.cuh, dispatch.cuh and combine.cuh.
+// update_expert.cuh, dispatch.cuh and combine.cuh.
 #include "moe_b200.h"
 
 #include <cstdint>
@@ -9,7 +9,6 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "dispatch.cuh"
-#include "rank.cuh"
 #include "update_expert.cuh"
 
 namespace {
@@ -33,7 +32,7 @@ bool check_workspace(const void *ws, size_t bytes) {
 // device (cached per device and kernel).
 template <typename Kernel>
 bool ensure_smem(Kernel k, size_t bytes, int slot) {
-    static int done[64][4];
+    static int done[64][16];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     if (bytes <= 48 * 1024) return true;
@@ -80,31 +79,37 @@ bool valid_combine(const moe_combine_params &p) {
 }
 
 template <typename Args>
-cudaError_t launch_pdl(void (*kernel)(Args), dim3 grid, dim3 block, size_t smem, cudaStream_t s, const Args &args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args);
+cudaError_t launch(void (*kernel)(Args), int grid, int block, size_t smem, cudaStream_t s, const Args &args) {
+    kernel<<<grid, block, smem, s>>>(args);
+    return cudaGetLastError();
 }
 
-template <int MODE, bool SMOOTH>
-cudaError_t launch_dispatch(const moe::DispatchArgs &a, cudaStream_t s) {
-    return launch_pdl(moe::dispatch_kernel<MODE, SMOOTH>, dim3(a.bs), dim3(moe::kDpThreads), 0, s, a);
+// Blocks per instance for the smooth-scale kernel: about four rows each.
+int dispatch_splits(int copies, int instances) {
+    const int avg = (copies + instances - 1) / instances;
+    int s = (avg + 3) / 4;
+    return s < 1 ? 1 : (s > 16 ? 16 : s);
 }
 
-template <int KMAX>
-void launch_combine(const moe::CombineArgs &a, cudaStream_t s) {
-    if (a.shared_x)
-        moe::combine_kernel<KMAX, true><<<a.bs, moe::kCbThreads, 0, s>>>(a);
-    else
-        moe::combine_kernel<KMAX, false><<<a.bs, moe::kCbThreads, 0, s>>>(a);
+template <int MODE>
+cudaError_t launch_dispatch_token(const moe::DispatchArgs &a, cudaStream_t s) {
+    const size_t smem = moe::token_smem_bytes(a.num_instances);
+    if (!ensure_smem(moe::dispatch_token_kernel<MODE>, smem, 1 + MODE)) return cudaErrorInvalidValue;
+    return launch(moe::dispatch_token_kernel<MODE>, a.bs, moe::kDpThreads, smem, s, a);
+}
+
+template <int MODE>
+cudaError_t launch_dispatch_instance(const moe::DispatchArgs &a, cudaStream_t s) {
+    const size_t smem = moe::instance_smem_bytes(a.hidden, a.bs * a.top_k);
+    if (!ensure_smem(moe::dispatch_instance_kernel<MODE>, smem, 6 + MODE)) return cudaErrorInvalidValue;
+    return launch(moe::dispatch_instance_kernel<MODE>, a.num_instances * a.splits, moe::kDpThreads, smem, s, a);
+}
+
+template <int KMAX, int KB>
+cudaError_t launch_combine(const moe::CombineArgs &a, cudaStream_t s) {
+    const size_t smem = moe::combine_smem_bytes(a.hidden);
+    if (a.shared_x) return launch(moe::combine_kernel<KMAX, KB, true>, a.bs, moe::kCbThreads, smem, s, a);
+    return launch(moe::combine_kernel<KMAX, KB, false>, a.bs, moe::kCbThreads, smem, s, a);
 }
 
 }  // namespace
@@ -209,49 +214,37 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
         (smooth_scales && !aligned(smooth_scales, 16)) || ((mode == 2 || mode == 3) && !aligned(dyn_scales, 4)))
         return MOE_ERR_INVALID_ARG;
     if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
-    cudaStream_t s = as_stream(cuda_stream);
-    uint32_t *err = reinterpret_cast<uint32_t *>(workspace);
-
-    moe::RankArgs r;
-    r.items = p->bs * p->top_k;
-    r.num_instances = p->num_instances;
-    r.ids = instance_ids;
-    r.mask = mask;
-    r.expand_idx = expand_idx;
-    r.src_of_row = src_of_row;
-    r.counts = expert_counts;
-    r.offsets = expert_offsets;
-    r.err = err;
-    const size_t smem = moe::rank_smem_bytes(p->num_instances);
-    if (!ensure_smem(moe::rank_kernel, smem, 1)) return MOE_ERR_CUDA;
-    moe::rank_kernel<<<1, moe::kRkThreads, smem, s>>>(r);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-
     moe::DispatchArgs a;
     a.bs = p->bs;
     a.hidden = p->hidden;
     a.top_k = p->top_k;
+    a.num_instances = p->num_instances;
     a.tiles = (p->hidden + 127) / 128;
+    a.splits = dispatch_splits(p->bs * p->top_k, p->num_instances);
     a.x = reinterpret_cast<const uint16_t *>(x);
     a.ids = instance_ids;
+    a.mask = mask;
     a.smooth = smooth_scales;
     a.expand_x = expand_x;
     a.dyn_scales = dyn_scales;
     a.expand_idx = expand_idx;
-    a.err = err;
+    a.src_of_row = src_of_row;
+    a.counts = expert_counts;
+    a.offsets = expert_offsets;
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    cudaStream_t s = as_stream(cuda_stream);
     cudaError_t e = cudaSuccess;
-    const bool sm = smooth_scales != nullptr;
-    switch (mode) {
-        case 0: e = launch_dispatch<0, false>(a, s); break;
-        case 2: e = sm ? launch_dispatch<2, true>(a, s) : launch_dispatch<2, false>(a, s); break;
-        case 3: e = sm ? launch_dispatch<3, true>(a, s) : launch_dispatch<3, false>(a, s); break;
-        case 4: e = launch_dispatch<4, false>(a, s); break;
+    if (smooth_scales) {
+        e = mode == 2 ? launch_dispatch_instance<2>(a, s) : launch_dispatch_instance<3>(a, s);
+    } else {
+        switch (mode) {
+            case 0: e = launch_dispatch_token<0>(a, s); break;
+            case 2: e = launch_dispatch_token<2>(a, s); break;
+            case 3: e = launch_dispatch_token<3>(a, s); break;
+            case 4: e = launch_dispatch_token<4>(a, s); break;
+        }
     }
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-    }
-    return launch_status();
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // --------------------------------------------------------------- combine ---
@@ -291,10 +284,11 @@ moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expa
     a.rstd_out = rstd_out;
     a.err = reinterpret_cast<uint32_t *>(workspace);
     cudaStream_t s = as_stream(cuda_stream);
-    if (p->top_k <= 4) launch_combine<4>(a, s);
-    else if (p->top_k <= 8) launch_combine<8>(a, s);
-    else launch_combine<16>(a, s);
-    return launch_status();
+    cudaError_t e;
+    if (p->top_k <= 4) e = launch_combine<4, 4>(a, s);
+    else if (p->top_k <= 8) e = launch_combine<8, 8>(a, s);
+    else e = launch_combine<16, 8>(a, s);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -32,6 +32,7 @@ struct UpdateArgs {
 };
 
 constexpr int kUeThreads = 1024;
+constexpr int kUeItems = 8;  // copies per thread: bs * K <= 8192 = 1024 * 8
 
 // Dynamic shared memory: n[1024], first[1024], inst[1024] ints, then one
 // uint16 counter per (warp, rank).
@@ -59,6 +60,25 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
 
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int F = a.table_cols, ws = a.ep_world_size, E = a.num_logical;
+
+    // The copies' inputs do not depend on the table: load them first so the
+    // loads overlap the table bookkeeping.
+    const int items = a.bs * a.top_k;
+    int pe[kUeItems];
+    float ps[kUeItems];
+    bool pa[kUeItems];
+#pragma unroll
+    for (int u = 0; u < kUeItems; ++u) {
+        const int it = t + u * kUeThreads;
+        pe[u] = -1;
+        ps[u] = 0.0f;
+        pa[u] = true;
+        if (it < items) {
+            pe[u] = a.expert_ids[it];
+            if (a.expert_scales) ps[u] = a.expert_scales[it];
+            if (a.active_mask) pa[u] = a.active_mask[it / a.top_k] != 0;
+        }
+    }
 
     if (t == 0) s_bad = 0;
     for (int q = t; q < 32 * ws; q += kUeThreads) s_wc[q] = 0;
@@ -131,10 +151,12 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     __syncthreads();
 
     // 4. every (token, k) copy
-    const int items = a.bs * a.top_k;
-    for (int it = t; it < items; it += kUeThreads) {
+#pragma unroll
+    for (int u = 0; u < kUeItems; ++u) {
+        const int it = t + u * kUeThreads;
+        if (it >= items) continue;
         const int i = it / a.top_k;
-        const int e = a.expert_ids[it];
+        const int e = pe[u];
         if (e < 0 || e >= E) {
             raise_error(a.err, kDevBadId);
             a.balanced_ids[it] = -1;
@@ -142,9 +164,8 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
             continue;
         }
         a.balanced_ids[it] = s_inst[s_first[e] + i % s_n[e]];
-        bool keep = a.active_mask ? (a.active_mask[i] != 0) : true;
-        if (a.expert_scales && a.prune_threshold > 0.0f && a.expert_scales[it] < a.prune_threshold)
-            keep = false;
+        bool keep = pa[u];
+        if (a.expert_scales && a.prune_threshold > 0.0f && ps[u] < a.prune_threshold) keep = false;
         a.balanced_mask[it] = keep ? 1 : 0;
     }
 }

@@ -65,6 +65,7 @@ typedef enum {
 /* Bits of the device error word (first 4 bytes of the workspace). */
 #define MOE_DEV_BAD_ID    1u  /* an expert / instance id or an expand_idx row out of range */
 #define MOE_DEV_BAD_TABLE 2u  /* mapping table broke its restrictions; every copy was dropped */
+#define MOE_DEV_TIMEOUT   4u  /* a bounded wait for an asynchronous copy gave up; outputs incomplete */
 
 /* Limits taken from the pages (shape-variable constraints of each page). */
 #define MOE_MAX_BS        512   /* Bs in (0, 512] */

@@ -76,7 +76,7 @@ def test_parity_active_mask(B):
 def test_parity_random_replicated_tables(B, seed):
     rng = np.random.default_rng(seed)
     ws = int(rng.choice([2, 3, 16, 64, 768]))
-    L = int(rng.integers(1, max(2, 1024 // ws) + 1))
+    L = int(rng.integers(1, 1024 // ws + 1))
     total = ws * L
     nl = int(rng.integers(max(1, total // ws), total + 1))
     nl = min(nl, total)
@@ -342,9 +342,19 @@ def test_layer_stack_cuda_graph(B):
         d = orc.dispatch(x, ob, E, 0, mask=om)
         c = orc.combine_add_rmsnorm(d["expand_x"], d["expand_idx"], st.expert_scales[l], r, st.gammas[l],
                                     st.norm_eps)
-        if l in (0, L // 2, L - 1):
-            assert_close_bf16(host(outs[l]["y"]), c["y_f64"], what=f"y layer {l}")
-            assert_close_bf16(host(outs[l]["x_out"]), c["x_f64"], what=f"x_out layer {l}")
+        np.testing.assert_array_equal(host(dsp[l]["expand_idx"]), d["expand_idx"])
         if l == 0:
-            np.testing.assert_array_equal(host(dsp[0]["expand_idx"]), d["expand_idx"])
+            assert_close_bf16(host(outs[l]["y"]), c["y_f64"], what="y layer 0")
+            assert_close_bf16(host(outs[l]["x_out"]), c["x_f64"], what="x_out layer 0")
+        else:
+            # Later layers take each side's own bf16 outputs as inputs.  With
+            # identity experts x = S * y + x_out, S = sum of the fp32 weights
+            # = 1 +- 1e-7, so sums of two bf16 values sit on bf16 rounding
+            # ties that the fp32 (GPU) and f64 (oracle) weight sums break
+            # differently; a flipped ulp then rides along into later layers.
+            # The chain is therefore held to a per-row relative L2 bound.
+            for got, want in ((host(outs[l]["y"]), c["y_f64"]), (host(outs[l]["x_out"]), c["x_f64"])):
+                g = gen.bf16_to_f32(got).astype(np.float64)
+                rel = np.linalg.norm(g - want, axis=1) / np.linalg.norm(want, axis=1)
+                assert rel.max() < 1e-2, (l, float(rel.max()))
         x, r = c["y"], c["x_out"]
