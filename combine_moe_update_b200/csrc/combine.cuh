@@ -5,13 +5,17 @@
 //   x = combineOut + residualX
 //   y = x / sqrt(mean(x^2) + normEps) * gamma
 //
-// One block of 256 threads per token.  For each 8-element vector of the row
-// a thread issues the K expert-row loads (the AllToAllV back: a gather
-// through expand_idx), the shared-expert and the residual load together,
-// accumulates in fp32 and parks x in shared memory (so registers stay low
-// and several blocks share an SM, keeping enough bytes in flight).  One
-// block reduction gives sum(x^2); a second sweep over shared memory writes y
-// (and x).  Every input byte is read once and every output byte written once.
+// A persistent kernel: each block owns tokens blockIdx.x, blockIdx.x + grid,
+// ... and streams them as a sequence of (token, H-chunk) units.  A unit is
+// the chunk of every kept expert row (the AllToAllV back: a gather through
+// expand_idx), of the shared-expert row and of the residual row -- each one
+// contiguous run of bytes, so one thread moves it into shared memory with a
+// single TMA bulk copy that completes on the unit's mbarrier.  kStages units
+// are in flight at once: while the block accumulates one unit (fp32, one
+// 8-element vector per thread) and, at a token's last chunk, reduces
+// sum(x^2) and writes y, the next units are already on their way.  x of the
+// current token stays in registers.  Every input byte is read from memory
+// once and every output byte written once.
 #pragma once
 #include "common.cuh"
 
@@ -33,108 +37,168 @@ struct CombineArgs {
 };
 
 constexpr int kCbThreads = 256;
+constexpr int kCbChunk = kCbThreads * 8;  // elements per unit: one 8-element vector per thread
+constexpr int kCbMaxChunks = 4;           // H <= 8192
+constexpr int kCbStages = 2;
+constexpr int kCbMaxTokens = 8;           // tokens per block (grid >= bs / 8)
 
-inline size_t combine_smem_bytes(int hidden) { return (size_t)hidden * sizeof(float); }
+// Rows per unit: K expert rows, the residual, and the shared-expert row.
+inline int combine_rows_per_unit(int top_k, bool shared) { return top_k + 1 + (shared ? 1 : 0); }
 
-// KB: expert rows whose loads are issued together (<= KMAX).
-template <int KMAX, int KB, bool SHARED>
+inline size_t combine_smem_bytes(int top_k, bool shared) {
+    return (size_t)kCbStages * combine_rows_per_unit(top_k, shared) * kCbChunk * sizeof(uint16_t);
+}
+
+template <int KMAX, bool SHARED>
 __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
-    extern __shared__ __align__(16) float s_x[];  // x of this token, fp32 [H]
-    __shared__ int s_row[16];
-    __shared__ float s_w[16];
+    extern __shared__ __align__(128) uint16_t s_stage[];  // [kStages][rows][kCbChunk]
+    __shared__ __align__(8) uint64_t s_full[kCbStages];
+    __shared__ int s_row[kCbMaxTokens][16];
+    __shared__ float s_w[kCbMaxTokens][16];
     __shared__ float s_red[kCbThreads / 32];
-    const int i = blockIdx.x, t = threadIdx.x;
-    const int H = a.hidden, V = H >> 3, K = a.top_k;
 
-    if (t < K) {
-        int row = a.expand_idx[i * K + t];
-        const float w = a.scales[i * K + t];
+    const int t = threadIdx.x, K = a.top_k, H = a.hidden;
+    const int R = K + 1 + (SHARED ? 1 : 0);  // rows per stage: K experts, residual, shared
+    const int n_chunks = (H + kCbChunk - 1) / kCbChunk;
+    const int n_tok = (a.bs - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // tokens of this block
+    const int n_units = n_tok * n_chunks;
+
+    // rows and weights of every token this block owns
+    for (int q = t; q < n_tok * K; q += kCbThreads) {
+        const int lt = q / K, k = q % K;
+        const int i = blockIdx.x + lt * gridDim.x;
+        int row = a.expand_idx[i * K + k];
+        const float w = a.scales[i * K + k];
         if (row < -1 || row >= a.expand_rows) {
             raise_error(a.err, kDevBadId);
             row = -1;
         }
-        s_row[t] = row;
-        s_w[t] = row >= 0 ? w : 0.0f;  // a pruned copy weighs nothing
+        s_row[lt][k] = row;
+        s_w[lt][k] = row >= 0 ? w : 0.0f;  // a pruned copy weighs nothing
+    }
+    if (t == 0) {
+        for (int s = 0; s < kCbStages; ++s) mbar_init(&s_full[s], 1);
     }
     __syncthreads();
 
-    int row[KMAX];
-    float wk[KMAX];
-    float wsum = 0.0f;  // sum of the kept weights, in k order
+    // Issue unit u into its stage (one thread).
+    auto issue = [&](int u) {
+        const int lt = u / n_chunks, c = u % n_chunks;
+        const int i = blockIdx.x + lt * gridDim.x;
+        const int h0 = c * kCbChunk;
+        const int len = (H - h0 < kCbChunk ? H - h0 : kCbChunk);
+        const uint32_t bytes = (uint32_t)len * sizeof(uint16_t);
+        const int st = u % kCbStages;
+        uint16_t *base = s_stage + (size_t)st * R * kCbChunk;
+        uint32_t total = bytes;  // residual
+        for (int k = 0; k < K; ++k) total += s_row[lt][k] >= 0 ? bytes : 0;
+        if (SHARED) total += bytes;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&s_full[st], total);
+        bulk_copy_g2s(base + (size_t)K * kCbChunk, a.residual + (size_t)i * H + h0, bytes, &s_full[st]);
+        if (SHARED) bulk_copy_g2s(base + (size_t)(K + 1) * kCbChunk, a.shared_x + (size_t)i * H + h0, bytes,
+                                  &s_full[st]);
+        for (int k = 0; k < K; ++k) {
+            const int row = s_row[lt][k];
+            if (row >= 0)
+                bulk_copy_g2s(base + (size_t)k * kCbChunk, a.expand_x + (size_t)row * H + h0, bytes, &s_full[st]);
+        }
+    };
+    if (t == 0)
+        for (int u = 0; u < kCbStages && u < n_units; ++u) issue(u);
+
+    // gamma of this thread's vectors, once
+    uint4 gv[kCbMaxChunks];
 #pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        row[k] = k < K ? s_row[k] : -1;
-        wk[k] = k < K ? s_w[k] : 0.0f;
-        wsum += wk[k];
+    for (int c = 0; c < kCbMaxChunks; ++c) {
+        const int h = c * kCbChunk + t * 8;
+        gv[c] = (c < n_chunks && h < H) ? ld_cached(a.gamma + h) : make_uint4(0, 0, 0, 0);
     }
 
-    const size_t tok = (size_t)i * H;
+    float xs[kCbMaxChunks][8];
     float ss = 0.0f;
-#pragma unroll 1
-    for (int p = t; p < V; p += kCbThreads) {
-        const uint4 res = ld_stream(a.residual + tok + p * 8);
-        uint4 sh = make_uint4(0, 0, 0, 0);
-        if constexpr (SHARED) sh = ld_stream(a.shared_x + tok + p * 8);
+    for (int u = 0; u < n_units; ++u) {
+        const int lt = u / n_chunks, c = u % n_chunks;
+        const int st = u % kCbStages;
+        const uint32_t phase = (uint32_t)(u / kCbStages) & 1u;
+        // every thread observes the unit's arrival itself; the verdict is block-uniform
+        if (!__syncthreads_and(mbar_wait_bounded(&s_full[st], phase))) {
+            // never leave with a bulk copy still in flight: one more bounded wait each
+            if (t == 0) {
+                raise_error(a.err, kDevTimeout);
+                for (int v = u; v < u + kCbStages && v < n_units; ++v)
+                    mbar_wait_bounded(&s_full[v % kCbStages], (uint32_t)(v / kCbStages) & 1u);
+            }
+            return;
+        }
+        const uint16_t *base = s_stage + (size_t)st * R * kCbChunk;
+        const int h = c * kCbChunk + t * 8;
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        if (h < H) {
+            float wsum = 0.0f;
 #pragma unroll
-        for (int k0 = 0; k0 < KMAX; k0 += KB) {
-            uint4 rv[KB];
-#pragma unroll
-            for (int k = 0; k < KB; ++k)
-                if (row[k0 + k] >= 0) rv[k] = ld_stream(a.expand_x + (size_t)row[k0 + k] * H + p * 8);
-#pragma unroll
-            for (int k = 0; k < KB; ++k) {
-                if (row[k0 + k] < 0) continue;
+            for (int k = 0; k < KMAX; ++k) {
+                if (k >= K) break;
+                const float w = s_w[lt][k];
+                wsum += w;
+                if (s_row[lt][k] < 0) continue;
                 float f[8];
-                unpack8(rv[k], f);
+                unpack8(*reinterpret_cast<const uint4 *>(base + (size_t)k * kCbChunk + t * 8), f);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wk[k0 + k], f[e], acc[e]);
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+            }
+            if constexpr (SHARED) {
+                float f[8];
+                unpack8(*reinterpret_cast<const uint4 *>(base + (size_t)(K + 1) * kCbChunk + t * 8), f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wsum, f[e], acc[e]);
+            }
+            float r[8];
+            unpack8(*reinterpret_cast<const uint4 *>(base + (size_t)K * kCbChunk + t * 8), r);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                acc[e] += r[e];
+                ss = fmaf(acc[e], acc[e], ss);
             }
         }
-        if constexpr (SHARED) {
-            float f[8];
-            unpack8(sh, f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(wsum, f[e], acc[e]);
-        }
-        float r[8];
-        unpack8(res, r);
+        for (int cc = 0; cc < kCbMaxChunks; ++cc)
+            if (cc == c) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            acc[e] += r[e];
-            ss = fmaf(acc[e], acc[e], ss);
-        }
-        float4 *xs = reinterpret_cast<float4 *>(s_x + p * 8);
-        xs[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        xs[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    }
+                for (int e = 0; e < 8; ++e) xs[cc][e] = acc[e];
+            }
+        __syncthreads();  // every thread is done with this stage
+        if (t == 0 && u + kCbStages < n_units) issue(u + kCbStages);
 
-    ss = block_sum<kCbThreads / 32>(ss, s_red);  // its barriers also publish s_x
-    const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(ss, (float)H) + a.norm_eps));
-    if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
-
-#pragma unroll 1
-    for (int p = t; p < V; p += kCbThreads) {
-        const float4 *xs = reinterpret_cast<const float4 *>(s_x + p * 8);
-        const float4 x0 = xs[0], x1 = xs[1];
-        const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        float g[8];
-        unpack8(ld_cached(a.gamma + p * 8), g);
-        uint4 yo;
-        yo.x = pack_bf16x2(x[0] * rstd * g[0], x[1] * rstd * g[1]);
-        yo.y = pack_bf16x2(x[2] * rstd * g[2], x[3] * rstd * g[3]);
-        yo.z = pack_bf16x2(x[4] * rstd * g[4], x[5] * rstd * g[5]);
-        yo.w = pack_bf16x2(x[6] * rstd * g[6], x[7] * rstd * g[7]);
-        st_v4(a.y + tok + p * 8, yo);
-        if (a.x_out) {
-            uint4 xo;
-            xo.x = pack_bf16x2(x[0], x[1]);
-            xo.y = pack_bf16x2(x[2], x[3]);
-            xo.z = pack_bf16x2(x[4], x[5]);
-            xo.w = pack_bf16x2(x[6], x[7]);
-            st_v4(a.x_out + tok + p * 8, xo);
+        if (c == n_chunks - 1) {  // the token is complete: normalize and write
+            const int i = blockIdx.x + lt * gridDim.x;
+            const float tot = block_sum<kCbThreads / 32>(ss, s_red);
+            ss = 0.0f;
+            const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));
+            if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
+#pragma unroll
+            for (int cc = 0; cc < kCbMaxChunks; ++cc) {
+                const int hh = cc * kCbChunk + t * 8;
+                if (cc >= n_chunks || hh >= H) continue;
+                float g[8];
+                unpack8(gv[cc], g);
+                uint4 yo;
+                yo.x = pack_bf16x2(xs[cc][0] * rstd * g[0], xs[cc][1] * rstd * g[1]);
+                yo.y = pack_bf16x2(xs[cc][2] * rstd * g[2], xs[cc][3] * rstd * g[3]);
+                yo.z = pack_bf16x2(xs[cc][4] * rstd * g[4], xs[cc][5] * rstd * g[5]);
+                yo.w = pack_bf16x2(xs[cc][6] * rstd * g[6], xs[cc][7] * rstd * g[7]);
+                st_v4(a.y + (size_t)i * H + hh, yo);
+                if (a.x_out) {
+                    uint4 xo;
+                    xo.x = pack_bf16x2(xs[cc][0], xs[cc][1]);
+                    xo.y = pack_bf16x2(xs[cc][2], xs[cc][3]);
+                    xo.z = pack_bf16x2(xs[cc][4], xs[cc][5]);
+                    xo.w = pack_bf16x2(xs[cc][6], xs[cc][7]);
+                    st_v4(a.x_out + (size_t)i * H + hh, xo);
+                }
+            }
         }
     }
 }

@@ -53,13 +53,14 @@ struct DispatchArgs {
 
 constexpr int kDpThreads = 256;
 constexpr int kDpWarps = kDpThreads / 32;
-constexpr int kKeyBatch = 8;  // copy keys loaded per thread before they are used
+constexpr int kKeyBatch = 16;  // copy keys loaded per thread before they are used
 
 // Key of copy j: its instance if it is sent, -1 if masked out, -2 if its id
 // is out of range (then it is dropped and reported).
 __device__ __forceinline__ int copy_key(const DispatchArgs &a, int j) {
-    if (a.mask && a.mask[j] == 0) return -1;
-    const int id = __ldg(a.ids + j);
+    const int id = __ldg(a.ids + j);  // both loads issue before either is used
+    const bool sent = a.mask ? __ldg(a.mask + j) != 0 : true;
+    if (!sent) return -1;
     return (id >= 0 && id < a.num_instances) ? id : -2;
 }
 
@@ -85,22 +86,26 @@ __device__ __forceinline__ float abs_max(const float (&f)[N]) {
     return m;
 }
 
-// clamp(rint(v * dyn), -127, 127) as one byte.
-__device__ __forceinline__ uint32_t q8(float v, float dyn) {
-    int q = __float2int_rn(__fmul_rn(v, dyn));
-    q = q > 127 ? 127 : (q < -127 ? -127 : q);
-    return (uint32_t)(q & 0xff);
+// rint(v * dyn) as the low byte of a float: adding 1.5 * 2^23 leaves
+// 1.5 * 2^23 + rint(v * dyn) (IEEE addition rounds half to even, and the
+// spacing there is 1), whose low byte is the code in two's complement.  Exact
+// while |v * dyn| < 2^22; here |v| <= amax and dyn = RN(127 / amax), so
+// |v * dyn| <= 127 (1 + 2^-24) and the code never leaves [-127, 127]: the
+// clamp to that range is never active.  Full-rate adds replace the slower
+// float-to-int conversion.
+__device__ __forceinline__ uint32_t q8_bits(float v, float dyn) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(v, dyn), 12582912.0f));
 }
 
-// Four int8 codes per 32-bit word; all zero when the segment's amax is 0
-// (dyn would be +inf there).
+// Four int8 codes per 32-bit word (element 0 in the low byte); all zero when
+// the segment's amax is 0 (dyn would be +inf there).
 template <int NW>
 __device__ __forceinline__ void pack_int8(const float *f, float dyn, bool zero, uint32_t *w) {
 #pragma unroll
     for (int q = 0; q < NW; ++q) {
-        const uint32_t word = q8(f[4 * q], dyn) | (q8(f[4 * q + 1], dyn) << 8) | (q8(f[4 * q + 2], dyn) << 16) |
-                              (q8(f[4 * q + 3], dyn) << 24);
-        w[q] = zero ? 0u : word;
+        const uint32_t lo = __byte_perm(q8_bits(f[4 * q], dyn), q8_bits(f[4 * q + 1], dyn), 0x0040);
+        const uint32_t hi = __byte_perm(q8_bits(f[4 * q + 2], dyn), q8_bits(f[4 * q + 3], dyn), 0x0040);
+        w[q] = zero ? 0u : __byte_perm(lo, hi, 0x5410);
     }
 }
 
@@ -344,7 +349,7 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
     float *s_sm = reinterpret_cast<float *>(smem_b);
     int *s_list = reinterpret_cast<int *>(smem_b + (size_t)H * sizeof(float));
     __shared__ __align__(8) uint64_t s_bar;
-    __shared__ int s_wcnt[kDpWarps], s_wless[kDpWarps], s_ok;
+    __shared__ int s_wcnt[kDpWarps], s_wless[kDpWarps];
     __shared__ float s_red[kDpWarps];
 
     const int e = blockIdx.x / a.splits, sp = blockIdx.x % a.splits;
@@ -422,10 +427,8 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
         a.expand_idx[j] = start + r;
     }
 
-    // 3. wait (bounded) for the smooth row
-    if (t == 0) s_ok = mbar_wait_bounded(&s_bar, 0) ? 1 : 0;
-    __syncthreads();
-    if (!s_ok) {
+    // 3. wait (bounded) for the smooth row; every thread observes it itself
+    if (!__syncthreads_and(mbar_wait_bounded(&s_bar, 0))) {
         if (t == 0) {
             raise_error(a.err, kDevTimeout);
             mbar_wait_bounded(&s_bar, 0);  // a last bounded wait for the copy in flight
@@ -433,8 +436,15 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
         return;
     }
 
-    // 4. quantize the rows, loading the next row's token while this one reduces
-    const float4 *sm4 = reinterpret_cast<const float4 *>(s_sm);
+    // 4. the smooth row into registers, then quantize the rows, loading the
+    //    next row's token while this one reduces
+    float sv[kImVecs][8];
+#pragma unroll
+    for (int q = 0; q < kImVecs; ++q) {
+        const int p = t + q * kDpThreads;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sv[q][e] = p < V ? s_sm[p * 8 + e] : 0.0f;
+    }
     auto load_row = [&](int r, uint4 (&xv)[kImVecs]) {
         const uint16_t *xr = a.x + (size_t)(copy_of(r) / K) * H;
 #pragma unroll
@@ -443,44 +453,31 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
             xv[q] = p < V ? ld_stream(xr + p * 8) : make_uint4(0, 0, 0, 0);
         }
     };
-    auto xf_of = [&](const uint4 &xq, int p, float (&f)[8]) {
-        unpack8(xq, f);
-        const float4 s0 = sm4[2 * p], s1 = sm4[2 * p + 1];
-        f[0] = __fmul_rn(f[0], s0.x); f[1] = __fmul_rn(f[1], s0.y);
-        f[2] = __fmul_rn(f[2], s0.z); f[3] = __fmul_rn(f[3], s0.w);
-        f[4] = __fmul_rn(f[4], s1.x); f[5] = __fmul_rn(f[5], s1.y);
-        f[6] = __fmul_rn(f[6], s1.z); f[7] = __fmul_rn(f[7], s1.w);
-    };
     uint4 xn[kImVecs];
     if (r0 < r1) load_row(r0, xn);
     for (int r = r0; r < r1; ++r) {  // uniform over the block
-        uint4 xc[kImVecs];
+        float xf[kImVecs][8];
 #pragma unroll
-        for (int q = 0; q < kImVecs; ++q) xc[q] = xn[q];
+        for (int q = 0; q < kImVecs; ++q) {
+            unpack8(xn[q], xf[q]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xf[q][e] = __fmul_rn(xf[q][e], sv[q][e]);  // xFp32 = x * smooth
+        }
         if (r + 1 < r1) load_row(r + 1, xn);
         const int row = start + r;
         uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
         if constexpr (MODE == 2) {
             float m = 0.0f;
 #pragma unroll
-            for (int q = 0; q < kImVecs; ++q) {
-                const int p = t + q * kDpThreads;
-                if (p < V) {
-                    float f[8];
-                    xf_of(xc[q], p, f);
-                    m = fmaxf(m, abs_max(f));
-                }
-            }
+            for (int q = 0; q < kImVecs; ++q) m = fmaxf(m, abs_max(xf[q]));
             m = block_max<kDpWarps>(m, s_red);
             const float dyn = __fdiv_rn(127.0f, m);
 #pragma unroll
             for (int q = 0; q < kImVecs; ++q) {
                 const int p = t + q * kDpThreads;
                 if (p < V) {
-                    float f[8];
-                    xf_of(xc[q], p, f);
                     uint32_t wd[2];
-                    pack_int8<2>(f, dyn, m == 0.0f, wd);
+                    pack_int8<2>(xf[q], dyn, m == 0.0f, wd);
                     *reinterpret_cast<uint2 *>(dst + p * 8) = make_uint2(wd[0], wd[1]);
                 }
             }
@@ -489,12 +486,7 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
 #pragma unroll
             for (int q = 0; q < kImVecs; ++q) {
                 const int p = t + q * kDpThreads;
-                float f[8];
-                float m = 0.0f;
-                if (p < V) {
-                    xf_of(xc[q], p, f);
-                    m = abs_max(f);
-                }
+                float m = abs_max(xf[q]);  // 0 for p >= V
                 m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
                 m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
                 m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
@@ -502,7 +494,7 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
                 if (p < V) {
                     const float dyn = __fdiv_rn(127.0f, m);
                     uint32_t wd[2];
-                    pack_int8<2>(f, dyn, m == 0.0f, wd);
+                    pack_int8<2>(xf[q], dyn, m == 0.0f, wd);
                     *reinterpret_cast<uint2 *>(dst + p * 8) = make_uint2(wd[0], wd[1]);
                     if ((t & 15) == 0)
                         reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (p >> 4)] = __frcp_rn(dyn);

@@ -32,7 +32,7 @@ bool check_workspace(const void *ws, size_t bytes) {
 // device (cached per device and kernel).
 template <typename Kernel>
 bool ensure_smem(Kernel k, size_t bytes, int slot) {
-    static int done[64][16];
+    static int done[64][32];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     if (bytes <= 48 * 1024) return true;
@@ -105,11 +105,28 @@ cudaError_t launch_dispatch_instance(const moe::DispatchArgs &a, cudaStream_t s)
     return launch(moe::dispatch_instance_kernel<MODE>, a.num_instances * a.splits, moe::kDpThreads, smem, s, a);
 }
 
-template <int KMAX, int KB>
+// Persistent combine: as many blocks as fit on the device at once (at least
+// one per 8 tokens), each walking its tokens' (token, chunk) units.
+template <int KMAX, bool SHARED>
+cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
+    auto kernel = moe::combine_kernel<KMAX, SHARED>;
+    const size_t smem = moe::combine_smem_bytes(a.top_k, SHARED);
+    if (!ensure_smem(kernel, smem, 10 + (KMAX / 8) * 2 + (SHARED ? 1 : 0))) return cudaErrorInvalidValue;
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cudaErrorUnknown;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, moe::kCbThreads, smem) != cudaSuccess)
+        return cudaErrorUnknown;
+    int grid = sms * (per_sm > 0 ? per_sm : 1);
+    const int min_grid = (a.bs + moe::kCbMaxTokens - 1) / moe::kCbMaxTokens;
+    if (grid < min_grid) grid = min_grid;
+    if (grid > a.bs) grid = a.bs;
+    return launch(kernel, grid, moe::kCbThreads, smem, s, a);
+}
+
+template <int KMAX>
 cudaError_t launch_combine(const moe::CombineArgs &a, cudaStream_t s) {
-    const size_t smem = moe::combine_smem_bytes(a.hidden);
-    if (a.shared_x) return launch(moe::combine_kernel<KMAX, KB, true>, a.bs, moe::kCbThreads, smem, s, a);
-    return launch(moe::combine_kernel<KMAX, KB, false>, a.bs, moe::kCbThreads, smem, s, a);
+    return a.shared_x ? launch_combine_t<KMAX, true>(a, s) : launch_combine_t<KMAX, false>(a, s);
 }
 
 }  // namespace
@@ -285,9 +302,9 @@ moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expa
     a.err = reinterpret_cast<uint32_t *>(workspace);
     cudaStream_t s = as_stream(cuda_stream);
     cudaError_t e;
-    if (p->top_k <= 4) e = launch_combine<4, 4>(a, s);
-    else if (p->top_k <= 8) e = launch_combine<8, 8>(a, s);
-    else e = launch_combine<16, 8>(a, s);
+    if (p->top_k <= 4) e = launch_combine<4>(a, s);
+    else if (p->top_k <= 8) e = launch_combine<8>(a, s);
+    else e = launch_combine<16>(a, s);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
