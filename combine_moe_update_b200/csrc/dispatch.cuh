@@ -97,15 +97,25 @@ __device__ __forceinline__ uint32_t q8_bits(float v, float dyn) {
     return __float_as_uint(__fadd_rn(__fmul_rn(v, dyn), 12582912.0f));
 }
 
-// Four int8 codes per 32-bit word (element 0 in the low byte); all zero when
-// the segment's amax is 0 (dyn would be +inf there).
+// The code when dyn = +inf (amax == 0, or 127 / amax overflows fp32): v * inf
+// is +-inf, which saturates to +-127, or NaN (v = 0), which casts to 0.
+__device__ __forceinline__ uint32_t q8_inf(float v) { return v > 0.0f ? 0x7fu : (v < 0.0f ? 0x81u : 0u); }
+
+// Four int8 codes per 32-bit word (element 0 in the low byte).
 template <int NW>
-__device__ __forceinline__ void pack_int8(const float *f, float dyn, bool zero, uint32_t *w) {
+__device__ __forceinline__ void pack_int8(const float *f, float dyn, uint32_t *w) {
+    if (isinf(dyn)) {  // uniform over the segment
+#pragma unroll
+        for (int q = 0; q < NW; ++q)
+            w[q] = q8_inf(f[4 * q]) | (q8_inf(f[4 * q + 1]) << 8) | (q8_inf(f[4 * q + 2]) << 16) |
+                   (q8_inf(f[4 * q + 3]) << 24);
+        return;
+    }
 #pragma unroll
     for (int q = 0; q < NW; ++q) {
         const uint32_t lo = __byte_perm(q8_bits(f[4 * q], dyn), q8_bits(f[4 * q + 1], dyn), 0x0040);
         const uint32_t hi = __byte_perm(q8_bits(f[4 * q + 2], dyn), q8_bits(f[4 * q + 3], dyn), 0x0040);
-        w[q] = zero ? 0u : __byte_perm(lo, hi, 0x5410);
+        w[q] = __byte_perm(lo, hi, 0x5410);
     }
 }
 
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs
             float f[16];
             chunk16(xv[j], f);
             uint32_t w[4];
-            pack_int8<4>(f, dyn, m == 0.0f, w);
+            pack_int8<4>(f, dyn, w);
             q[j] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     } else if constexpr (MODE == 3) {
@@ -277,7 +287,7 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs
             const float dyn = __fdiv_rn(127.0f, m);
             seg[j] = __frcp_rn(dyn);
             uint32_t w[4];
-            pack_int8<4>(f, dyn, m == 0.0f, w);
+            pack_int8<4>(f, dyn, w);
             q[j] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     } else if constexpr (MODE == 4) {
@@ -477,7 +487,7 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
                 const int p = t + q * kDpThreads;
                 if (p < V) {
                     uint32_t wd[2];
-                    pack_int8<2>(xf[q], dyn, m == 0.0f, wd);
+                    pack_int8<2>(xf[q], dyn, wd);
                     *reinterpret_cast<uint2 *>(dst + p * 8) = make_uint2(wd[0], wd[1]);
                 }
             }
@@ -494,7 +504,7 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchA
                 if (p < V) {
                     const float dyn = __fdiv_rn(127.0f, m);
                     uint32_t wd[2];
-                    pack_int8<2>(xf[q], dyn, m == 0.0f, wd);
+                    pack_int8<2>(xf[q], dyn, wd);
                     *reinterpret_cast<uint2 *>(dst + p * 8) = make_uint2(wd[0], wd[1]);
                     if ((t & 15) == 0)
                         reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (p >> 4)] = __frcp_rn(dyn);

@@ -191,7 +191,10 @@ static int orc_item_cmp(const void *pa, const void *pb) {
  *   sent scale = 1.0 / dynamicScales
  * READING R6: dstTypeMax = 127, CastToInt8 rounds half to even and clamps to
  * [-127, 127].  READING R7: the sent scale is the fp32 quotient 1 / dyn.
- * READING R13: an all-zero segment gives codes 0 and scale 1/inf = 0. */
+ * READING R13: an all-zero segment gives codes 0 and scale 1/inf = 0.
+ * READING R20: when 127 / amax overflows fp32 (amax < 127 / FLT_MAX) the
+ * formula runs on dyn = +inf: CastToInt8 saturates +-inf to +-127 and maps the
+ * NaN of 0 * inf to 0; the scale is again 1/inf = 0. */
 static void orc_quant_int8_segment(const uint16_t *x, const float *smooth, int len,
                                    int8_t *q, float *scale_out) {
     float amax = 0.0f;
@@ -208,6 +211,7 @@ static void orc_quant_int8_segment(const uint16_t *x, const float *smooth, int l
         float xf = bf16_to_float(x[h]);
         if (smooth) xf = xf * smooth[h];
         float r = rintf(xf * dyn);
+        if (isnan(r)) r = 0.0f;
         if (r > 127.0f) r = 127.0f;
         if (r < -127.0f) r = -127.0f;
         q[h] = (int8_t)r;
