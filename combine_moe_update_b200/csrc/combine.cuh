@@ -5,15 +5,15 @@
 //   x = combineOut + residualX
 //   y = x / sqrt(mean(x^2) + normEps) * gamma
 //
-// A persistent kernel: each block owns tokens blockIdx.x, blockIdx.x + grid,
-// ... and streams them as a sequence of (token, H-chunk) units.  A unit is
-// the chunk of every kept expert row (the AllToAllV back: a gather through
-// expand_idx), of the shared-expert row and of the residual row -- each one
-// contiguous run of bytes, so one thread moves it into shared memory with a
-// single TMA bulk copy that completes on the unit's mbarrier.  kStages units
-// are in flight at once: while the block accumulates one unit (fp32, one
-// 8-element vector per thread) and, at a token's last chunk, reduces
-// sum(x^2) and writes y, the next units are already on their way.  x of the
+// A persistent kernel, one block per SM: block b owns tokens b, b + grid, ...
+// Thread t owns the 8-element vectors p = t, t + 256, ... of every row.  A
+// "unit" is one such vector slot of one token: the slot of every kept expert
+// row (the AllToAllV back, a gather through expand_idx), of the residual row
+// and of the shared-expert row.  Each thread streams its own units through a
+// DEPTH-deep ring of private shared-memory slots with 16-byte cp.async, so
+// DEPTH - 1 units per thread are always in flight and no barrier sits on the
+// load path; only the per-token sum(x^2) needs the block.  Accumulation is
+// fp32 (packed fp32x2 FMAs, each lane an ordinary IEEE FMA) and x of the
 // current token stays in registers.  Every input byte is read from memory
 // once and every output byte written once.
 #pragma once
@@ -37,31 +37,25 @@ struct CombineArgs {
 };
 
 constexpr int kCbThreads = 256;
-constexpr int kCbChunk = kCbThreads * 8;  // elements per unit: one 8-element vector per thread
-constexpr int kCbMaxChunks = 4;           // H <= 8192
-constexpr int kCbStages = 2;
-constexpr int kCbMaxTokens = 8;           // tokens per block (grid >= bs / 8)
+constexpr int kCbVecs = 4;       // 8-element vectors per thread: H / 8 <= 1024
+constexpr int kCbMaxTokens = 8;  // tokens per block (grid >= bs / 8)
 
-// Rows per unit: K expert rows, the residual, and the shared-expert row.
-inline int combine_rows_per_unit(int top_k, bool shared) { return top_k + 1 + (shared ? 1 : 0); }
-
-inline size_t combine_smem_bytes(int top_k, bool shared) {
-    return (size_t)kCbStages * combine_rows_per_unit(top_k, shared) * kCbChunk * sizeof(uint16_t);
+// Ring slots: [depth][K experts + residual + shared][kCbThreads] x 16 bytes.
+inline size_t combine_smem_bytes(int depth, int top_k, bool shared) {
+    return (size_t)depth * (top_k + 1 + (shared ? 1 : 0)) * kCbThreads * sizeof(uint4);
 }
 
-template <int KMAX, bool SHARED>
+template <int KMAX, bool SHARED, int DEPTH>
 __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
-    extern __shared__ __align__(128) uint16_t s_stage[];  // [kStages][rows][kCbChunk]
-    __shared__ __align__(8) uint64_t s_full[kCbStages];
+    extern __shared__ __align__(16) uint4 s_buf[];
     __shared__ int s_row[kCbMaxTokens][16];
     __shared__ float s_w[kCbMaxTokens][16];
     __shared__ float s_red[kCbThreads / 32];
 
-    const int t = threadIdx.x, K = a.top_k, H = a.hidden;
-    const int R = K + 1 + (SHARED ? 1 : 0);  // rows per stage: K experts, residual, shared
-    const int n_chunks = (H + kCbChunk - 1) / kCbChunk;
-    const int n_tok = (a.bs - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // tokens of this block
-    const int n_units = n_tok * n_chunks;
+    const int t = threadIdx.x, K = a.top_k, H = a.hidden, V = H >> 3;
+    const int R = K + 1 + (SHARED ? 1 : 0);
+    const int J = (V + kCbThreads - 1) / kCbThreads;  // vector slots per thread (uniform)
+    const int n_tok = (a.bs - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
     // rows and weights of every token this block owns
     for (int q = t; q < n_tok * K; q += kCbThreads) {
@@ -76,131 +70,120 @@ __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
         s_row[lt][k] = row;
         s_w[lt][k] = row >= 0 ? w : 0.0f;  // a pruned copy weighs nothing
     }
-    if (t == 0) {
-        for (int s = 0; s < kCbStages; ++s) mbar_init(&s_full[s], 1);
-    }
     __syncthreads();
 
-    // Issue unit u into its stage (one thread).
-    auto issue = [&](int u) {
-        const int lt = u / n_chunks, c = u % n_chunks;
-        const int i = blockIdx.x + lt * gridDim.x;
-        const int h0 = c * kCbChunk;
-        const int len = (H - h0 < kCbChunk ? H - h0 : kCbChunk);
-        const uint32_t bytes = (uint32_t)len * sizeof(uint16_t);
-        const int st = u % kCbStages;
-        uint16_t *base = s_stage + (size_t)st * R * kCbChunk;
-        uint32_t total = bytes;  // residual
-        for (int k = 0; k < K; ++k) total += s_row[lt][k] >= 0 ? bytes : 0;
-        if (SHARED) total += bytes;
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&s_full[st], total);
-        bulk_copy_g2s(base + (size_t)K * kCbChunk, a.residual + (size_t)i * H + h0, bytes, &s_full[st]);
-        if (SHARED) bulk_copy_g2s(base + (size_t)(K + 1) * kCbChunk, a.shared_x + (size_t)i * H + h0, bytes,
-                                  &s_full[st]);
-        for (int k = 0; k < K; ++k) {
-            const int row = s_row[lt][k];
-            if (row >= 0)
-                bulk_copy_g2s(base + (size_t)k * kCbChunk, a.expand_x + (size_t)row * H + h0, bytes, &s_full[st]);
-        }
-    };
-    if (t == 0)
-        for (int u = 0; u < kCbStages && u < n_units; ++u) issue(u);
-
     // gamma of this thread's vectors, once
-    uint4 gv[kCbMaxChunks];
+    uint4 gv[kCbVecs];
 #pragma unroll
-    for (int c = 0; c < kCbMaxChunks; ++c) {
-        const int h = c * kCbChunk + t * 8;
-        gv[c] = (c < n_chunks && h < H) ? ld_cached(a.gamma + h) : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < kCbVecs; ++j) {
+        const int p = t + j * kCbThreads;
+        gv[j] = (j < J && p < V) ? ld_cached(a.gamma + p * 8) : make_uint4(0, 0, 0, 0);
     }
 
-    float xs[kCbMaxChunks][8];
-    float ss = 0.0f;
-    for (int u = 0; u < n_units; ++u) {
-        const int lt = u / n_chunks, c = u % n_chunks;
-        const int st = u % kCbStages;
-        const uint32_t phase = (uint32_t)(u / kCbStages) & 1u;
-        // every thread observes the unit's arrival itself; the verdict is block-uniform
-        if (!__syncthreads_and(mbar_wait_bounded(&s_full[st], phase))) {
-            // never leave with a bulk copy still in flight: one more bounded wait each
-            if (t == 0) {
-                raise_error(a.err, kDevTimeout);
-                for (int v = u; v < u + kCbStages && v < n_units; ++v)
-                    mbar_wait_bounded(&s_full[v % kCbStages], (uint32_t)(v / kCbStages) & 1u);
-            }
-            return;
-        }
-        const uint16_t *base = s_stage + (size_t)st * R * kCbChunk;
-        const int h = c * kCbChunk + t * 8;
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-        if (h < H) {
-            float wsum = 0.0f;
+    // Issue one unit (token n, slot j) into ring stage st; always commit a
+    // group, empty or not, so the group count stays uniform.
+    int in_n = 0, in_j = 0, in_st = 0;
+    auto issue_next = [&]() {
+        const int p = t + in_j * kCbThreads;
+        if (in_n < n_tok && p < V) {
+            const int i = blockIdx.x + in_n * gridDim.x;
+            uint4 *slot = s_buf + (size_t)in_st * R * kCbThreads + t;
 #pragma unroll
             for (int k = 0; k < KMAX; ++k) {
                 if (k >= K) break;
-                const float w = s_w[lt][k];
-                wsum += w;
-                if (s_row[lt][k] < 0) continue;
-                float f[8];
-                unpack8(*reinterpret_cast<const uint4 *>(base + (size_t)k * kCbChunk + t * 8), f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+                const int row = s_row[in_n][k];
+                if (row >= 0) cp_async16(slot + k * kCbThreads, a.expand_x + (size_t)row * H + p * 8);
             }
-            if constexpr (SHARED) {
-                float f[8];
-                unpack8(*reinterpret_cast<const uint4 *>(base + (size_t)(K + 1) * kCbChunk + t * 8), f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wsum, f[e], acc[e]);
-            }
-            float r[8];
-            unpack8(*reinterpret_cast<const uint4 *>(base + (size_t)K * kCbChunk + t * 8), r);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                acc[e] += r[e];
-                ss = fmaf(acc[e], acc[e], ss);
-            }
+            cp_async16(slot + K * kCbThreads, a.residual + (size_t)i * H + p * 8);
+            if (SHARED) cp_async16(slot + (K + 1) * kCbThreads, a.shared_x + (size_t)i * H + p * 8);
         }
+        cp_async_commit();
+        if (++in_j == J) {
+            in_j = 0;
+            ++in_n;
+        }
+        if (++in_st == DEPTH) in_st = 0;
+    };
 #pragma unroll
-        for (int cc = 0; cc < kCbMaxChunks; ++cc)
-            if (cc == c) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) xs[cc][e] = acc[e];
-            }
-        __syncthreads();  // every thread is done with this stage
-        if (t == 0 && u + kCbStages < n_units) issue(u + kCbStages);
+    for (int d = 0; d < DEPTH - 1; ++d) issue_next();
 
-        if (c == n_chunks - 1) {  // the token is complete: normalize and write
-            const int i = blockIdx.x + lt * gridDim.x;
-            const float tot = block_sum<kCbThreads / 32>(ss, s_red);
-            ss = 0.0f;
-            const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));
-            if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
+    int st = 0;
+    for (int n = 0; n < n_tok; ++n) {
+        const int i = blockIdx.x + n * gridDim.x;
+        uint64_t w2[KMAX];
+        bool live[KMAX];
+        float wsum = 0.0f;  // sum of the kept weights, in k order
 #pragma unroll
-            for (int cc = 0; cc < kCbMaxChunks; ++cc) {
-                const int hh = cc * kCbChunk + t * 8;
-                if (cc >= n_chunks || hh >= H) continue;
-                float g[8];
-                unpack8(gv[cc], g);
-                uint4 yo;
-                yo.x = pack_bf16x2(xs[cc][0] * rstd * g[0], xs[cc][1] * rstd * g[1]);
-                yo.y = pack_bf16x2(xs[cc][2] * rstd * g[2], xs[cc][3] * rstd * g[3]);
-                yo.z = pack_bf16x2(xs[cc][4] * rstd * g[4], xs[cc][5] * rstd * g[5]);
-                yo.w = pack_bf16x2(xs[cc][6] * rstd * g[6], xs[cc][7] * rstd * g[7]);
-                st_v4(a.y + (size_t)i * H + hh, yo);
-                if (a.x_out) {
-                    uint4 xo;
-                    xo.x = pack_bf16x2(xs[cc][0], xs[cc][1]);
-                    xo.y = pack_bf16x2(xs[cc][2], xs[cc][3]);
-                    xo.z = pack_bf16x2(xs[cc][4], xs[cc][5]);
-                    xo.w = pack_bf16x2(xs[cc][6], xs[cc][7]);
-                    st_v4(a.x_out + (size_t)i * H + hh, xo);
+        for (int k = 0; k < KMAX; ++k) {
+            const float w = k < K ? s_w[n][k] : 0.0f;
+            live[k] = k < K && s_row[n][k] >= 0;
+            w2[k] = f2_pack(w, w);
+            wsum += w;
+        }
+        const uint64_t ws2 = f2_pack(wsum, wsum);
+
+        uint64_t xs[kCbVecs][4];
+        uint64_t ss2 = 0ull;
+#pragma unroll
+        for (int j = 0; j < kCbVecs; ++j) {
+            if (j >= J) break;  // uniform
+            issue_next();
+            cp_async_wait<DEPTH - 1>();  // this thread's copies of the oldest unit have landed
+            const int p = t + j * kCbThreads;
+            const uint4 *slot = s_buf + (size_t)st * R * kCbThreads + t;
+            if (++st == DEPTH) st = 0;
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+            if (p < V) {
+#pragma unroll
+                for (int k = 0; k < KMAX; ++k) {
+                    if (!live[k]) continue;
+                    const uint4 v = slot[k * kCbThreads];
+                    acc[0] = f2_fma(w2[k], bf16x2_to_f2(v.x), acc[0]);
+                    acc[1] = f2_fma(w2[k], bf16x2_to_f2(v.y), acc[1]);
+                    acc[2] = f2_fma(w2[k], bf16x2_to_f2(v.z), acc[2]);
+                    acc[3] = f2_fma(w2[k], bf16x2_to_f2(v.w), acc[3]);
                 }
+                if constexpr (SHARED) {
+                    const uint4 v = slot[(K + 1) * kCbThreads];
+                    acc[0] = f2_fma(ws2, bf16x2_to_f2(v.x), acc[0]);
+                    acc[1] = f2_fma(ws2, bf16x2_to_f2(v.y), acc[1]);
+                    acc[2] = f2_fma(ws2, bf16x2_to_f2(v.z), acc[2]);
+                    acc[3] = f2_fma(ws2, bf16x2_to_f2(v.w), acc[3]);
+                }
+                const uint4 r = slot[K * kCbThreads];
+                acc[0] = f2_add(acc[0], bf16x2_to_f2(r.x));
+                acc[1] = f2_add(acc[1], bf16x2_to_f2(r.y));
+                acc[2] = f2_add(acc[2], bf16x2_to_f2(r.z));
+                acc[3] = f2_add(acc[3], bf16x2_to_f2(r.w));
+#pragma unroll
+                for (int h = 0; h < 4; ++h) ss2 = f2_fma(acc[h], acc[h], ss2);
             }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) xs[j][h] = acc[h];
+        }
+
+        // the token is complete: normalize and write
+        const float tot = block_sum<kCbThreads / 32>(f2_lo(ss2) + f2_hi(ss2), s_red);
+        const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));
+        if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
+        const uint64_t r2 = f2_pack(rstd, rstd);
+#pragma unroll
+        for (int j = 0; j < kCbVecs; ++j) {
+            const int p = t + j * kCbThreads;
+            if (j >= J || p >= V) continue;
+            const uint32_t gw[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
+            uint32_t yo[4], xo[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const uint64_t yv = f2_mul(f2_mul(xs[j][h], r2), bf16x2_to_f2(gw[h]));
+                yo[h] = pack_bf16x2(f2_lo(yv), f2_hi(yv));
+                xo[h] = pack_bf16x2(f2_lo(xs[j][h]), f2_hi(xs[j][h]));
+            }
+            st_v4(a.y + (size_t)i * H + p * 8, make_uint4(yo[0], yo[1], yo[2], yo[3]));
+            if (a.x_out) st_v4(a.x_out + (size_t)i * H + p * 8, make_uint4(xo[0], xo[1], xo[2], xo[3]));
         }
     }
+    cp_async_wait<0>();  // only empty groups can remain; leave nothing in flight
 }
 
 }  // namespace moe

@@ -34,12 +34,14 @@ template <typename Kernel>
 bool ensure_smem(Kernel k, size_t bytes, int slot) {
     static int done[64][32];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    if (bytes <= 48 * 1024) return true;
-    if (done[dev][slot] >= (int)bytes) return true;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 32) return false;
+    if (done[dev][slot] >= (int)bytes + 1) return true;
+    if (bytes > 48 * 1024 &&
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return false;
-    done[dev][slot] = (int)bytes;
+    // prefer the largest shared-memory carveout, so occupancy is not capped by it
+    if (cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return false;
+    done[dev][slot] = (int)bytes + 1;
     return true;
 }
 
@@ -100,28 +102,35 @@ cudaError_t launch_dispatch_token(const moe::DispatchArgs &a, cudaStream_t s) {
 
 template <int MODE>
 cudaError_t launch_dispatch_instance(const moe::DispatchArgs &a, cudaStream_t s) {
-    const size_t smem = moe::instance_smem_bytes(a.hidden, a.bs * a.top_k);
+    const size_t smem = moe::instance_smem_bytes(a.hidden, a.bs * a.top_k, a.splits);
     if (!ensure_smem(moe::dispatch_instance_kernel<MODE>, smem, 6 + MODE)) return cudaErrorInvalidValue;
     return launch(moe::dispatch_instance_kernel<MODE>, a.num_instances * a.splits, moe::kDpThreads, smem, s, a);
 }
 
-// Persistent combine: as many blocks as fit on the device at once (at least
-// one per 8 tokens), each walking its tokens' (token, chunk) units.
-template <int KMAX, bool SHARED>
-cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
-    auto kernel = moe::combine_kernel<KMAX, SHARED>;
-    const size_t smem = moe::combine_smem_bytes(a.top_k, SHARED);
-    if (!ensure_smem(kernel, smem, 10 + (KMAX / 8) * 2 + (SHARED ? 1 : 0))) return cudaErrorInvalidValue;
-    int dev = 0, sms = 0, per_sm = 0;
+// Persistent combine: one block per SM (at least one per 8 tokens); the ring
+// depth is the largest of 8 / 4 / 2 units whose slots fit in 200 KB.
+template <int KMAX, bool SHARED, int DEPTH>
+cudaError_t launch_combine_d(const moe::CombineArgs &a, cudaStream_t s, int slot) {
+    auto kernel = moe::combine_kernel<KMAX, SHARED, DEPTH>;
+    const size_t smem = moe::combine_smem_bytes(DEPTH, a.top_k, SHARED);
+    if (!ensure_smem(kernel, smem, slot)) return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cudaErrorUnknown;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, moe::kCbThreads, smem) != cudaSuccess)
-        return cudaErrorUnknown;
-    int grid = sms * (per_sm > 0 ? per_sm : 1);
+    int grid = sms;
     const int min_grid = (a.bs + moe::kCbMaxTokens - 1) / moe::kCbMaxTokens;
     if (grid < min_grid) grid = min_grid;
     if (grid > a.bs) grid = a.bs;
     return launch(kernel, grid, moe::kCbThreads, smem, s, a);
+}
+
+template <int KMAX, bool SHARED>
+cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
+    const size_t budget = 200 * 1024;
+    const int base = 10 + (KMAX / 8) * 6 + (SHARED ? 3 : 0);
+    if (moe::combine_smem_bytes(8, a.top_k, SHARED) <= budget) return launch_combine_d<KMAX, SHARED, 8>(a, s, base);
+    if (moe::combine_smem_bytes(4, a.top_k, SHARED) <= budget) return launch_combine_d<KMAX, SHARED, 4>(a, s, base + 1);
+    return launch_combine_d<KMAX, SHARED, 2>(a, s, base + 2);
 }
 
 template <int KMAX>
