@@ -95,7 +95,10 @@ __device__ __forceinline__ uint4 ld_cached(const void *p) {
 __device__ __forceinline__ void st_v4(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
 
 // --- packed fp32x2 arithmetic (sm_100): two independent IEEE binary32
-// operations, each rounded to nearest even, in one instruction ---
+// operations, each rounded to nearest even, in one instruction.  A packed
+// multiply whose result feeds a packed add may be contracted into a fused
+// multiply-add; where the product's own rounding matters, multiply with the
+// scalar __fmul_rn instead. ---
 
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
     return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);

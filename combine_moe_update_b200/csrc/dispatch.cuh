@@ -76,12 +76,19 @@ __device__ __forceinline__ int copy_key(const DispatchArgs &a, int j) {
 // 1.5 * 2^23 + rint(v * dyn), exact while |v * dyn| < 2^22.  Here |v| <=
 // amax and dyn = RN(127 / amax), so |v * dyn| <= 127 (1 + 2^-24): codes stay
 // in [-127, 127] and the clamp to that range is never active.
+//
+// The product must be rounded to fp32 on its own before the add (the page's
+// quantOut = CastToInt8(xFp32 * dynamicScales) rounds it).  A packed multiply
+// followed by a packed add may be contracted into one fused multiply-add,
+// which skips that rounding and breaks ties such as a product that rounds to
+// exactly 63.5; the scalar round-to-nearest multiply is never contracted.
 __device__ __forceinline__ uint2 int8x8(const uint64_t (&v)[4], float dyn) {
-    const uint64_t d2 = f2_pack(dyn, dyn), magic = f2_pack(12582912.0f, 12582912.0f);
+    const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
     uint32_t b[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const uint64_t r = f2_add(f2_mul(v[q], d2), magic);
+        const uint64_t prod = f2_pack(__fmul_rn(f2_lo(v[q]), dyn), __fmul_rn(f2_hi(v[q]), dyn));
+        const uint64_t r = f2_add(prod, magic);
         b[2 * q] = (uint32_t)r;
         b[2 * q + 1] = (uint32_t)(r >> 32);
     }
