@@ -5,17 +5,23 @@
 //   x = combineOut + residualX
 //   y = x / sqrt(mean(x^2) + normEps) * gamma
 //
-// A persistent kernel, one block per SM: block b owns tokens b, b + grid, ...
-// Thread t owns the 8-element vectors p = t, t + 256, ... of every row.  A
-// "unit" is one such vector slot of one token: the slot of every kept expert
-// row (the AllToAllV back, a gather through expand_idx), of the residual row
-// and of the shared-expert row.  Each thread streams its own units through a
-// DEPTH-deep ring of private shared-memory slots with 16-byte cp.async, so
-// DEPTH - 1 units per thread are always in flight and no barrier sits on the
-// load path; only the per-token sum(x^2) needs the block.  Accumulation is
-// fp32 (packed fp32x2 FMAs, each lane an ordinary IEEE FMA) and x of the
-// current token stays in registers.  Every input byte is read from memory
-// once and every output byte written once.
+// A persistent, warp-specialized kernel, one block per SM.  Block b owns
+// tokens b, b + grid, ...; each token is cut into units of 2048 elements.  A
+// unit is that slice of every kept expert row (the AllToAllV back: a gather
+// through expand_idx), of the residual row and of the shared-expert row --
+// each a contiguous run of bytes, moved into shared memory by one TMA bulk
+// copy.  One producer warp keeps a ring of STAGES units in flight (a "full"
+// mbarrier per stage counts the bytes in, an "empty" one counts the consumer
+// warps out); eight consumer warps each take one 8-element vector per row of
+// a unit, accumulate in fp32 (packed fp32x2 FMAs, each lane an ordinary IEEE
+// FMA) and keep x of the current token in registers.  Only the per-token
+// sum(x^2) needs the consumers together (a named barrier); nothing stops the
+// producer.  Every input byte is read from memory once, every output byte
+// written once.
+//
+// Every wait is bounded.  A wait that gives up records MOE_DEV_TIMEOUT and the
+// thread carries on (its outputs are then wrong, and flagged), so no thread
+// ever leaves a barrier short of one arrival.
 #pragma once
 #include "common.cuh"
 
@@ -36,26 +42,40 @@ struct CombineArgs {
     uint32_t *err;
 };
 
-constexpr int kCbThreads = 256;
-constexpr int kCbVecs = 4;       // 8-element vectors per thread: H / 8 <= 1024
-constexpr int kCbMaxTokens = 8;  // tokens per block (grid >= bs / 8)
+constexpr int kCbConsumers = 256;                   // 8 consumer warps
+constexpr int kCbThreads = kCbConsumers + 32;       // + 1 producer warp
+constexpr int kCbChunk = kCbConsumers * 8;          // elements per unit
+constexpr int kCbMaxChunks = 4;                     // H <= 8192
+constexpr int kCbMaxTokens = 8;                     // tokens per block (grid >= bs / 8)
 
-// Ring slots: [depth][K experts + residual + shared][kCbThreads] x 16 bytes.
-inline size_t combine_smem_bytes(int depth, int top_k, bool shared) {
-    return (size_t)depth * (top_k + 1 + (shared ? 1 : 0)) * kCbThreads * sizeof(uint4);
+// Rows per unit: K expert rows, the residual, and the shared-expert row.
+inline int combine_rows(int top_k, bool shared) { return top_k + 1 + (shared ? 1 : 0); }
+
+inline size_t combine_smem_bytes(int stages, int top_k, bool shared) {
+    return (size_t)stages * combine_rows(top_k, shared) * kCbChunk * sizeof(uint16_t);
 }
 
-template <int KMAX, bool SHARED, int DEPTH>
-__global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
-    extern __shared__ __align__(16) uint4 s_buf[];
+template <int KMAX, bool SHARED, int STAGES>
+__global__ void __launch_bounds__(kCbThreads, 1) combine_kernel(CombineArgs a) {
+    extern __shared__ __align__(128) uint16_t s_stage[];  // [STAGES][R][kCbChunk]
+    __shared__ __align__(8) uint64_t s_full[STAGES], s_empty[STAGES];
     __shared__ int s_row[kCbMaxTokens][16];
     __shared__ float s_w[kCbMaxTokens][16];
-    __shared__ float s_red[kCbThreads / 32];
+    __shared__ float s_red[kCbConsumers / 32];
 
-    const int t = threadIdx.x, K = a.top_k, H = a.hidden, V = H >> 3;
-    const int R = K + 1 + (SHARED ? 1 : 0);
-    const int J = (V + kCbThreads - 1) / kCbThreads;  // vector slots per thread (uniform)
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int K = a.top_k, H = a.hidden, R = K + 1 + (SHARED ? 1 : 0);
+    const int n_chunks = (H + kCbChunk - 1) / kCbChunk;
     const int n_tok = (a.bs - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int n_units = n_tok * n_chunks;
+
+    if (t == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], kCbConsumers / 32);
+        }
+    }
+    pdl_wait();  // expand_idx and the expert rows come from earlier kernels
 
     // rows and weights of every token this block owns
     for (int q = t; q < n_tok * K; q += kCbThreads) {
@@ -72,42 +92,47 @@ __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
     }
     __syncthreads();
 
-    // gamma of this thread's vectors, once
-    uint4 gv[kCbVecs];
-#pragma unroll
-    for (int j = 0; j < kCbVecs; ++j) {
-        const int p = t + j * kCbThreads;
-        gv[j] = (j < J && p < V) ? ld_cached(a.gamma + p * 8) : make_uint4(0, 0, 0, 0);
+    if (warp == kCbConsumers / 32) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            bool ok = true;
+            for (int u = 0; u < n_units; ++u) {
+                const int st = u % STAGES;
+                if (u >= STAGES) ok &= mbar_wait_bounded(&s_empty[st], (uint32_t)((u / STAGES) & 1) ^ 1u);
+                const int lt = u / n_chunks, c = u % n_chunks;
+                const int i = blockIdx.x + lt * gridDim.x;
+                const int h0 = c * kCbChunk;
+                const uint32_t bytes = (uint32_t)((H - h0 < kCbChunk ? H - h0 : kCbChunk) * sizeof(uint16_t));
+                uint16_t *base = s_stage + (size_t)st * R * kCbChunk;
+                uint32_t total = bytes * (1 + (SHARED ? 1 : 0));
+                for (int k = 0; k < K; ++k) total += s_row[lt][k] >= 0 ? bytes : 0;
+                mbar_arrive_expect_tx(&s_full[st], total);
+                bulk_copy_g2s(base + (size_t)K * kCbChunk, a.residual + (size_t)i * H + h0, bytes, &s_full[st]);
+                if (SHARED)
+                    bulk_copy_g2s(base + (size_t)(K + 1) * kCbChunk, a.shared_x + (size_t)i * H + h0, bytes,
+                                  &s_full[st]);
+                for (int k = 0; k < K; ++k) {
+                    const int row = s_row[lt][k];
+                    if (row >= 0)
+                        bulk_copy_g2s(base + (size_t)k * kCbChunk, a.expand_x + (size_t)row * H + h0, bytes,
+                                      &s_full[st]);
+                }
+            }
+            if (!ok) raise_error(a.err, kDevTimeout);
+        }
+        pdl_launch_dependents();
+        return;
     }
 
-    // Issue one unit (token n, slot j) into ring stage st; always commit a
-    // group, empty or not, so the group count stays uniform.
-    int in_n = 0, in_j = 0, in_st = 0;
-    auto issue_next = [&]() {
-        const int p = t + in_j * kCbThreads;
-        if (in_n < n_tok && p < V) {
-            const int i = blockIdx.x + in_n * gridDim.x;
-            uint4 *slot = s_buf + (size_t)in_st * R * kCbThreads + t;
+    // ----------------------------------------------------------- consumers
+    uint4 gv[kCbMaxChunks];
 #pragma unroll
-            for (int k = 0; k < KMAX; ++k) {
-                if (k >= K) break;
-                const int row = s_row[in_n][k];
-                if (row >= 0) cp_async16(slot + k * kCbThreads, a.expand_x + (size_t)row * H + p * 8);
-            }
-            cp_async16(slot + K * kCbThreads, a.residual + (size_t)i * H + p * 8);
-            if (SHARED) cp_async16(slot + (K + 1) * kCbThreads, a.shared_x + (size_t)i * H + p * 8);
-        }
-        cp_async_commit();
-        if (++in_j == J) {
-            in_j = 0;
-            ++in_n;
-        }
-        if (++in_st == DEPTH) in_st = 0;
-    };
-#pragma unroll
-    for (int d = 0; d < DEPTH - 1; ++d) issue_next();
-
-    int st = 0;
+    for (int c = 0; c < kCbMaxChunks; ++c) {
+        const int h = c * kCbChunk + t * 8;
+        gv[c] = (c < n_chunks && h < H) ? ld_cached(a.gamma + h) : make_uint4(0, 0, 0, 0);
+    }
+    bool ok = true;
+    int u = 0;
     for (int n = 0; n < n_tok; ++n) {
         const int i = blockIdx.x + n * gridDim.x;
         uint64_t w2[KMAX];
@@ -122,35 +147,34 @@ __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
         }
         const uint64_t ws2 = f2_pack(wsum, wsum);
 
-        uint64_t xs[kCbVecs][4];
+        uint64_t xs[kCbMaxChunks][4];
         uint64_t ss2 = 0ull;
 #pragma unroll
-        for (int j = 0; j < kCbVecs; ++j) {
-            if (j >= J) break;  // uniform
-            issue_next();
-            cp_async_wait<DEPTH - 1>();  // this thread's copies of the oldest unit have landed
-            const int p = t + j * kCbThreads;
-            const uint4 *slot = s_buf + (size_t)st * R * kCbThreads + t;
-            if (++st == DEPTH) st = 0;
+        for (int c = 0; c < kCbMaxChunks; ++c) {
+            if (c >= n_chunks) break;  // uniform
+            const int st = u % STAGES;
+            ok &= mbar_wait_bounded(&s_full[st], (uint32_t)((u / STAGES) & 1));
+            ++u;
+            const uint16_t *base = s_stage + (size_t)st * R * kCbChunk + t * 8;
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-            if (p < V) {
+            if (c * kCbChunk + t * 8 < H) {
 #pragma unroll
                 for (int k = 0; k < KMAX; ++k) {
                     if (!live[k]) continue;
-                    const uint4 v = slot[k * kCbThreads];
+                    const uint4 v = *reinterpret_cast<const uint4 *>(base + (size_t)k * kCbChunk);
                     acc[0] = f2_fma(w2[k], bf16x2_to_f2(v.x), acc[0]);
                     acc[1] = f2_fma(w2[k], bf16x2_to_f2(v.y), acc[1]);
                     acc[2] = f2_fma(w2[k], bf16x2_to_f2(v.z), acc[2]);
                     acc[3] = f2_fma(w2[k], bf16x2_to_f2(v.w), acc[3]);
                 }
                 if constexpr (SHARED) {
-                    const uint4 v = slot[(K + 1) * kCbThreads];
+                    const uint4 v = *reinterpret_cast<const uint4 *>(base + (size_t)(K + 1) * kCbChunk);
                     acc[0] = f2_fma(ws2, bf16x2_to_f2(v.x), acc[0]);
                     acc[1] = f2_fma(ws2, bf16x2_to_f2(v.y), acc[1]);
                     acc[2] = f2_fma(ws2, bf16x2_to_f2(v.z), acc[2]);
                     acc[3] = f2_fma(ws2, bf16x2_to_f2(v.w), acc[3]);
                 }
-                const uint4 r = slot[K * kCbThreads];
+                const uint4 r = *reinterpret_cast<const uint4 *>(base + (size_t)K * kCbChunk);
                 acc[0] = f2_add(acc[0], bf16x2_to_f2(r.x));
                 acc[1] = f2_add(acc[1], bf16x2_to_f2(r.y));
                 acc[2] = f2_add(acc[2], bf16x2_to_f2(r.z));
@@ -158,32 +182,41 @@ __global__ void __launch_bounds__(kCbThreads) combine_kernel(CombineArgs a) {
 #pragma unroll
                 for (int h = 0; h < 4; ++h) ss2 = f2_fma(acc[h], acc[h], ss2);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[st]);  // this warp is done with the stage
 #pragma unroll
-            for (int h = 0; h < 4; ++h) xs[j][h] = acc[h];
+            for (int h = 0; h < 4; ++h) xs[c][h] = acc[h];
         }
 
-        // the token is complete: normalize and write
-        const float tot = block_sum<kCbThreads / 32>(f2_lo(ss2) + f2_hi(ss2), s_red);
+        // the token is complete: sum(x^2) over the consumers, then y
+        float v = warp_sum(f2_lo(ss2) + f2_hi(ss2));
+        if (lane == 0) s_red[warp] = v;
+        named_barrier(1, kCbConsumers);
+        float tot = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kCbConsumers / 32; ++w) tot += s_red[w];  // fixed order: deterministic
+        named_barrier(1, kCbConsumers);
         const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));
         if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
         const uint64_t r2 = f2_pack(rstd, rstd);
 #pragma unroll
-        for (int j = 0; j < kCbVecs; ++j) {
-            const int p = t + j * kCbThreads;
-            if (j >= J || p >= V) continue;
-            const uint32_t gw[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
+        for (int c = 0; c < kCbMaxChunks; ++c) {
+            const int h = c * kCbChunk + t * 8;
+            if (c >= n_chunks || h >= H) continue;
+            const uint32_t gw[4] = {gv[c].x, gv[c].y, gv[c].z, gv[c].w};
             uint32_t yo[4], xo[4];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const uint64_t yv = f2_mul(f2_mul(xs[j][h], r2), bf16x2_to_f2(gw[h]));
-                yo[h] = pack_bf16x2(f2_lo(yv), f2_hi(yv));
-                xo[h] = pack_bf16x2(f2_lo(xs[j][h]), f2_hi(xs[j][h]));
+            for (int q = 0; q < 4; ++q) {
+                const uint64_t yv = f2_mul(f2_mul(xs[c][q], r2), bf16x2_to_f2(gw[q]));
+                yo[q] = pack_bf16x2(f2_lo(yv), f2_hi(yv));
+                xo[q] = pack_bf16x2(f2_lo(xs[c][q]), f2_hi(xs[c][q]));
             }
-            st_v4(a.y + (size_t)i * H + p * 8, make_uint4(yo[0], yo[1], yo[2], yo[3]));
-            if (a.x_out) st_v4(a.x_out + (size_t)i * H + p * 8, make_uint4(xo[0], xo[1], xo[2], xo[3]));
+            st_v4(a.y + (size_t)i * H + h, make_uint4(yo[0], yo[1], yo[2], yo[3]));
+            if (a.x_out) st_v4(a.x_out + (size_t)i * H + h, make_uint4(xo[0], xo[1], xo[2], xo[3]));
         }
     }
-    cp_async_wait<0>();  // only empty groups can remain; leave nothing in flight
+    if (!ok) raise_error(a.err, kDevTimeout);
+    pdl_launch_dependents();
 }
 
 }  // namespace moe

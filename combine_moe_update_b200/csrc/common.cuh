@@ -59,6 +59,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     return ok != 0;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier over the first `count` threads of the block (named barrier `id`,
+// 1..15; id 0 is __syncthreads).  count must be a multiple of 32.
+__device__ __forceinline__ void named_barrier(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Wait for phase `phase` of an mbarrier, giving up after a bounded number of
 // polls (each poll may itself suspend for a while).  Returns false on
 // timeout, so a copy that never lands cannot hang the GPU.

@@ -2,24 +2,23 @@
 // expert-major receive buffer (aclnnMoeDistributeDispatchV2, "计算公式").
 //
 // The EP AllToAllV is, on one GPU, a permutation of the (token, k) copies
-// into rank-major rows; the page requires a deterministic result
+// into rank-major rows.  The page requires a deterministic result
 // ("确定性计算"), so a copy's row is its position in (instance, token, k)
-// order.  Each kernel below is the whole operation in one launch: every
-// block derives what it needs of that order from the (at most 8192) copy
-// keys while its own row loads are in flight.  Only counts are accumulated
-// concurrently, and counts do not depend on order, so every run gives the
-// same bytes.
+// order: route_kernel computes that order once -- a stable counting sort in
+// one block -- and the quantize-and-scatter kernels only look their rows up.
 //
-// dispatch_token_kernel<MODE>   one block per token, no smooth scales: the
-//   row is loaded once, quantized once (all K copies are identical) and
-//   written K times.  A shared-memory histogram of all copies and of the
-//   copies of earlier tokens gives the K destination rows.
-// dispatch_instance_kernel<MODE> smooth scales (modes 2, 3): one block per
-//   (instance, slice of its rows).  The instance's smooth row is staged in
-//   shared memory by one TMA bulk copy and then held in registers; the block
-//   compacts the copies routed to its instance (ballots over the keys) and
-//   streams their tokens' rows from L2, one row ahead, so every smooth row is
-//   read from memory once instead of once per copy.
+// The scatter kernels are launched as programmatic dependents of the route
+// kernel: everything that depends only on the call's inputs (loading the
+// token row and the smooth row, the absmax reduction, the quantization
+// itself) runs while the route kernel is still sorting, and only the final
+// row writes wait for it.
+//
+// dispatch_token_kernel<MODE>   no smooth scales: one block per token; the
+//   row is loaded, quantized once (all K copies are identical) and written K
+//   times.
+// dispatch_copy_kernel<MODE>    smooth scales (modes 2, 3): one block per
+//   (token, k) copy, so 4096 independent blocks at Bs 512, K 8; each loads
+//   its token row and its instance's smooth row (both mostly from L2).
 //
 // Quantization, per mode ("计算公式" cases 1, 3, 4, 5):
 //   0  copy the bf16 row;
@@ -29,8 +28,7 @@
 //   4  mxfp8: per 32-element block sharedExp = floor(log2 max|x|) - 8 taken
 //      from the exponent bits; q = e4m3_satfinite(x * 2^-sharedExp); scale
 //      byte = sharedExp + 127.
-// All arithmetic is IEEE binary32 rounded to nearest (packed fp32x2
-// instructions are two such operations each), so no contraction or
+// All arithmetic is IEEE binary32 rounded to nearest, so no contraction or
 // approximation can move a code.
 #pragma once
 #include "common.cuh"
@@ -39,10 +37,9 @@ namespace moe {
 
 struct DispatchArgs {
     int bs, hidden, top_k, num_instances;
-    int tiles;   // ceil(H / 128) (mode 3)
-    int splits;  // blocks per instance (instance kernel)
-    const uint16_t *x;  // bf16 bits [bs, H]
-    const int32_t *ids;  // instance ids [bs, K]
+    int tiles;  // ceil(H / 128) (mode 3)
+    const uint16_t *x;    // bf16 bits [bs, H]
+    const int32_t *ids;   // instance ids [bs, K]
     const uint8_t *mask;  // [bs, K] or null
     const float *smooth;  // [E, H] or null
     void *expand_x;
@@ -54,11 +51,6 @@ struct DispatchArgs {
     uint32_t *err;
 };
 
-constexpr int kDpThreads = 256;
-constexpr int kDpWarps = kDpThreads / 32;
-constexpr int kDpVecs = 4;     // 8-element vectors per thread: H / 8 <= 1024 = 256 * 4
-constexpr int kKeyBatch = 16;  // copy keys a thread loads before using them
-
 // Key of copy j: its instance if it is sent, -1 if masked out, -2 if its id
 // is out of range (then it is dropped and reported).
 __device__ __forceinline__ int copy_key(const DispatchArgs &a, int j) {
@@ -68,7 +60,106 @@ __device__ __forceinline__ int copy_key(const DispatchArgs &a, int j) {
     return (id >= 0 && id < a.num_instances) ? id : -2;
 }
 
+// ---------------------------------------------------------- route kernel ---
+//
+// One block of 1024 threads, <= 8192 copies, <= 1024 instances.  Warp w owns
+// the contiguous copies [w * P, (w + 1) * P) and walks them 32 at a time;
+// __match_any_sync groups equal instances, so a copy's rank inside its warp
+// is (earlier rounds' count) + (lower lanes with the same instance).  A
+// per-instance prefix over the 32 warps, then a scan over the instances,
+// turns those into rows.  No atomics decide an order.
+
+constexpr int kRtThreads = 1024;
+constexpr int kRtRounds = 8;  // 8192 copies / 32 warps / 32 lanes
+
+inline size_t route_smem_bytes(int num_instances) {
+    return 32 * (size_t)num_instances * sizeof(uint16_t) + (size_t)num_instances * sizeof(int);
+}
+
+__global__ void __launch_bounds__(kRtThreads, 1) route_kernel(DispatchArgs a) {
+    pdl_wait();               // the instance ids may come from the previous kernel
+    pdl_launch_dependents();  // the scatter kernel may start its input-only work now
+
+    extern __shared__ __align__(16) unsigned char smem_r[];
+    const int E = a.num_instances, N = a.bs * a.top_k;
+    uint16_t *s_wc = reinterpret_cast<uint16_t *>(smem_r);               // [32][E]
+    int *s_off = reinterpret_cast<int *>(smem_r + 64 * (size_t)E);      // [E]
+    __shared__ int s_warp[32];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int P = (N + 31) / 32;  // copies per warp
+    const int rounds = (P + 31) / 32;
+
+    int key[kRtRounds];
+#pragma unroll
+    for (int j = 0; j < kRtRounds; ++j) {
+        const int off = j * 32 + lane, it = w * P + off;
+        key[j] = (j < rounds && off < P && it < N) ? copy_key(a, it) : -1;
+    }
+    uint32_t *wc32 = reinterpret_cast<uint32_t *>(s_wc);
+    for (int q = t; q < 16 * E; q += kRtThreads) wc32[q] = 0;
+    __syncthreads();
+
+    const unsigned lower = (1u << lane) - 1u;
+    int local[kRtRounds];
+#pragma unroll
+    for (int j = 0; j < kRtRounds; ++j) {
+        local[j] = 0;
+        if (j >= rounds) continue;  // uniform
+        int k = key[j];
+        if (k == -2) {
+            raise_error(a.err, kDevBadId);
+            k = key[j] = -1;
+        }
+        const unsigned peers = __match_any_sync(kFull, k);
+        int base = 0;
+        if (k >= 0) base = s_wc[w * E + k];
+        __syncwarp();
+        if (k >= 0 && lane == __ffs(peers) - 1) s_wc[w * E + k] = (uint16_t)(base + __popc(peers));
+        __syncwarp();
+        local[j] = base + __popc(peers & lower);
+    }
+    __syncthreads();
+
+    int total_b = 0;  // E <= 1024: thread t owns instance t
+    if (t < E) {
+        int run = 0;
+#pragma unroll 8
+        for (int ww = 0; ww < 32; ++ww) {
+            const int c = s_wc[ww * E + t];
+            s_wc[ww * E + t] = (uint16_t)run;
+            run += c;
+        }
+        total_b = run;
+    }
+    const int incl = block_inclusive_scan(total_b, s_warp);
+    if (t < E) {
+        s_off[t] = incl - total_b;
+        a.counts[t] = total_b;
+        a.offsets[t] = incl - total_b;
+    }
+    if (t == kRtThreads - 1) a.offsets[E] = incl;
+    __syncthreads();
+
+#pragma unroll
+    for (int j = 0; j < kRtRounds; ++j) {
+        const int off = j * 32 + lane, it = w * P + off;
+        if (j >= rounds || off >= P || it >= N) continue;
+        const int k = key[j];
+        if (k < 0) {
+            a.expand_idx[it] = -1;
+            continue;
+        }
+        const int row = s_off[k] + s_wc[w * E + k] + local[j];
+        a.expand_idx[it] = row;
+        a.src_of_row[row] = it;
+    }
+}
+
 // ------------------------------------------------------------ quantizers ---
+
+constexpr int kDpThreads = 256;
+constexpr int kDpWarps = kDpThreads / 32;
+constexpr int kDpVecs = 4;  // 8-element vectors per thread: H / 8 <= 1024 = 256 * 4
 
 // int8 codes of 8 values (4 fp32 pairs) for a finite multiplier dyn.
 // rint(v * dyn) is the low byte of v * dyn + 1.5 * 2^23: IEEE addition
@@ -172,25 +263,83 @@ __device__ __forceinline__ float2 block_dyn(float m, float *s_red, float *s_out)
     return make_float2(s_out[0], s_out[1]);
 }
 
-// --------------------------------------------------------- token kernel ---
+// Quantize this thread's vectors of one row (xf: fp32 pairs, x * smooth
+// already applied).  Fills the codes and the scales this thread writes.
+template <int MODE>
+__device__ __forceinline__ void quantize_vecs(const uint64_t (&xf)[kDpVecs][4], int V, float *s_red, float *s_out,
+                                              uint2 (&qv)[kDpVecs], float (&seg)[kDpVecs], float &row_scale) {
+    const int t = threadIdx.x;
+    if constexpr (MODE == 2) {
+        float m = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kDpVecs; ++q) m = fmaxf(m, abs_max8(xf[q]));
+        const float2 ds = block_dyn(m, s_red, s_out);
+        row_scale = ds.y;
+#pragma unroll
+        for (int q = 0; q < kDpVecs; ++q) qv[q] = int8x8_any(xf[q], ds.x);
+    } else if constexpr (MODE == 3) {
+#pragma unroll
+        for (int q = 0; q < kDpVecs; ++q) {  // a 128-element tile = 16 vectors = 16 consecutive lanes
+            float m = abs_max8(xf[q]);       // 0 past the row's end
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
+            const bool lead = (t & 15) == 0 && t + q * kDpThreads < V;
+            float dyn = 0.0f;
+            if (lead) dyn = __fdiv_rn(127.0f, m);  // one division per tile
+            dyn = __shfl_sync(kFull, dyn, (t & 31) & ~15);
+            if (lead) seg[q] = __frcp_rn(dyn);
+            qv[q] = int8x8_any(xf[q], dyn);
+        }
+    } else if constexpr (MODE == 4) {
+#pragma unroll
+        for (int q = 0; q < kDpVecs; ++q) {  // a 32-element block = 4 consecutive lanes
+            float m = abs_max8(xf[q]);
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+            const int se = mx_shared_exp(m);
+            seg[q] = __int_as_float(se + 127);
+            qv[q] = e4m3x8(xf[q], se);
+        }
+    }
+}
 
-inline size_t token_smem_bytes(int num_instances) { return 3 * (size_t)num_instances * sizeof(int); }
+// Write this thread's codes (and scales) of one row.
+template <int MODE>
+__device__ __forceinline__ void write_row(const DispatchArgs &a, int row, int V, const uint2 (&qv)[kDpVecs],
+                                          const float (&seg)[kDpVecs], float row_scale) {
+    const int t = threadIdx.x, H = a.hidden;
+    uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
+#pragma unroll
+    for (int q = 0; q < kDpVecs; ++q) {
+        const int p = t + q * kDpThreads;
+        if (p >= V) continue;
+        *reinterpret_cast<uint2 *>(dst + p * 8) = qv[q];
+        if constexpr (MODE == 3) {
+            if ((t & 15) == 0) reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (p >> 4)] = seg[q];
+        }
+        if constexpr (MODE == 4) {
+            if ((t & 3) == 0)
+                reinterpret_cast<uint8_t *>(a.dyn_scales)[(size_t)row * (H >> 5) + (p >> 2)] =
+                    (uint8_t)__float_as_int(seg[q]);
+        }
+    }
+    if constexpr (MODE == 2) {
+        if (t == 0) reinterpret_cast<float *>(a.dyn_scales)[row] = row_scale;
+    }
+}
+
+// --------------------------------------------------------- token kernel ---
 
 template <int MODE>
 __global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs a) {
-    extern __shared__ __align__(16) int smem_i[];
-    const int E = a.num_instances;
-    int *hist = smem_i;    // sent copies per instance
-    int *pref = hist + E;  // ... among the copies of earlier tokens
-    int *off = pref + E;   // exclusive prefix of hist
-    __shared__ float s_red[kDpWarps], s_dyn[2];
-    __shared__ int s_warp[32];
-    __shared__ int s_key[16], s_row[16];
-
+    __shared__ float s_red[kDpWarps], s_out[2];
+    __shared__ int s_row[16];
     const int i = blockIdx.x, t = threadIdx.x;
-    const int H = a.hidden, V = H >> 3, K = a.top_k, N = a.bs * K, mine = i * K;
+    const int H = a.hidden, V = H >> 3, K = a.top_k;
 
-    // 1. this token's row: issue the loads first, use them last
+    // inputs of the call only: safe before the route kernel is done
     const uint16_t *xrow = a.x + (size_t)i * H;
     uint4 xv[kDpVecs];
 #pragma unroll
@@ -198,121 +347,19 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs
         const int p = t + q * kDpThreads;
         xv[q] = p < V ? ld_stream(xrow + p * 8) : make_uint4(0, 0, 0, 0);
     }
-
-    // 2. histogram of all sent copies and of those of earlier tokens
-    for (int q = t; q < 2 * E; q += kDpThreads) smem_i[q] = 0;
-    if (t < K) s_key[t] = copy_key(a, mine + t);
-    __syncthreads();
-    for (int j0 = 0; j0 < N; j0 += kDpThreads * kKeyBatch) {
-        int key[kKeyBatch];
-#pragma unroll
-        for (int u = 0; u < kKeyBatch; ++u) {
-            const int j = j0 + u * kDpThreads + t;
-            key[u] = j < N ? copy_key(a, j) : -1;
-        }
-#pragma unroll
-        for (int u = 0; u < kKeyBatch; ++u) {
-            const int j = j0 + u * kDpThreads + t;
-            const int k = key[u];
-            if (k >= 0) {
-                atomicAdd(&hist[k], 1);
-                if (j < mine) atomicAdd(&pref[k], 1);
-            } else if (k == -2 && i == 0) {
-                raise_error(a.err, kDevBadId);
-            }
-        }
-    }
-    __syncthreads();
-
-    // 3. bucket offsets: 4 consecutive instances per thread (E <= 1024)
-    int v4[4], sum = 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int b = t * 4 + u;
-        v4[u] = b < E ? hist[b] : 0;
-        sum += v4[u];
-    }
-    const int incl = block_inclusive_scan(sum, s_warp);
-    const int total = s_warp[kDpWarps - 1];
-    int run = incl - sum;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int b = t * 4 + u;
-        if (b < E) {
-            off[b] = run;
-            if (i == 0) {
-                a.counts[b] = v4[u];
-                a.offsets[b] = run;
-            }
-        }
-        run += v4[u];
-    }
-    if (i == 0 && t == 0) a.offsets[E] = total;
-    __syncthreads();
-
-    // 4. rows of this token's copies
-    if (t < K) {
-        const int k = s_key[t];
-        int row = -1;
-        if (k >= 0) {
-            int same = 0;
-            for (int u = 0; u < t; ++u) same += (s_key[u] == k);
-            row = off[k] + pref[k] + same;
-            a.src_of_row[row] = mine + t;
-        }
-        a.expand_idx[mine + t] = row;
-        s_row[t] = row;
-    }
-    __syncthreads();
-
-    // 5. quantize once, then write every copy
     uint2 qv[kDpVecs];
-    float seg[kDpVecs];  // mode 3: scale of the slot's tile; mode 4: E8M0 byte of its block (as bits)
+    float seg[kDpVecs] = {0.0f, 0.0f, 0.0f, 0.0f};
     float row_scale = 0.0f;
-    if constexpr (MODE == 2) {
-        float m = 0.0f;
+    if constexpr (MODE != 0) {
+        uint64_t xf[kDpVecs][4];
 #pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {
-            uint64_t f[4];
-            vec_to_f2(xv[q], f);
-            m = fmaxf(m, abs_max8(f));
-        }
-        const float2 ds = block_dyn(m, s_red, s_dyn);
-        row_scale = ds.y;
-#pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {
-            uint64_t f[4];
-            vec_to_f2(xv[q], f);
-            qv[q] = int8x8_any(f, ds.x);
-        }
-    } else if constexpr (MODE == 3) {
-#pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {  // a 128-element tile = 16 vectors = 16 consecutive lanes
-            uint64_t f[4];
-            vec_to_f2(xv[q], f);
-            float m = abs_max8(f);
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
-            const float dyn = __fdiv_rn(127.0f, m);
-            seg[q] = __frcp_rn(dyn);
-            qv[q] = int8x8_any(f, dyn);
-        }
-    } else if constexpr (MODE == 4) {
-#pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {  // a 32-element block = 4 consecutive lanes
-            uint64_t f[4];
-            vec_to_f2(xv[q], f);
-            float m = abs_max8(f);
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
-            const int se = mx_shared_exp(m);
-            seg[q] = __int_as_float(se + 127);
-            qv[q] = e4m3x8(f, se);
-        }
+        for (int q = 0; q < kDpVecs; ++q) vec_to_f2(xv[q], xf[q]);
+        quantize_vecs<MODE>(xf, V, s_red, s_out, qv, seg, row_scale);
     }
 
+    pdl_wait();  // the rows come from route_kernel
+    if (t < K) s_row[t] = a.expand_idx[i * K + t];
+    __syncthreads();
     for (int k = 0; k < K; ++k) {
         const int row = s_row[k];
         if (row < 0) continue;
@@ -324,200 +371,50 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs
                 if (p < V) st_v4(dst + p * 8, xv[q]);
             }
         } else {
-            uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
-#pragma unroll
-            for (int q = 0; q < kDpVecs; ++q) {
-                const int p = t + q * kDpThreads;
-                if (p >= V) continue;
-                *reinterpret_cast<uint2 *>(dst + p * 8) = qv[q];
-                if constexpr (MODE == 3) {
-                    if ((t & 15) == 0)
-                        reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (p >> 4)] = seg[q];
-                }
-                if constexpr (MODE == 4) {
-                    if ((t & 3) == 0)
-                        reinterpret_cast<uint8_t *>(a.dyn_scales)[(size_t)row * (H >> 5) + (p >> 2)] =
-                            (uint8_t)__float_as_int(seg[q]);
-                }
-            }
-            if constexpr (MODE == 2) {
-                if (t == 0) reinterpret_cast<float *>(a.dyn_scales)[row] = row_scale;
-            }
+            write_row<MODE>(a, row, V, qv, seg, row_scale);
         }
     }
 }
 
-// ------------------------------------------------------ instance kernel ---
-
-constexpr int kImMaxKeys = 32;  // keys per lane in the scan: per warp <= 1024 copies
-
-// Copies per warp in the instance kernel's key scan (a multiple of 32).
-__host__ __device__ inline int im_per_warp(int copies) { return ((copies + kDpWarps - 1) / kDpWarps + 31) & ~31; }
-
-// Rows of one instance a block handles at most: ceil(copies / splits).
-__host__ __device__ inline int im_row_cap(int copies, int splits) { return (copies + splits - 1) / splits; }
-
-// Dynamic shared memory: the smooth row, then the token of each owned row.
-inline size_t instance_smem_bytes(int hidden, int copies, int splits) {
-    return (size_t)hidden * sizeof(float) + (size_t)im_row_cap(copies, splits) * sizeof(int);
-}
+// ---------------------------------------------------------- copy kernel ---
 
 template <int MODE>
-__global__ void __launch_bounds__(kDpThreads) dispatch_instance_kernel(DispatchArgs a) {
-    extern __shared__ __align__(128) unsigned char smem_b[];
-    const int H = a.hidden, K = a.top_k, N = a.bs * K, E = a.num_instances, V = H >> 3;
-    float *s_sm = reinterpret_cast<float *>(smem_b);
-    int *s_tok = reinterpret_cast<int *>(smem_b + (size_t)H * sizeof(float));  // [cap]
-    __shared__ __align__(8) uint64_t s_bar;
-    __shared__ int s_wcnt[kDpWarps], s_wless[kDpWarps];
-    __shared__ float s_red[kDpWarps], s_dyn[2];
+__global__ void __launch_bounds__(kDpThreads) dispatch_copy_kernel(DispatchArgs a) {
+    __shared__ float s_red[kDpWarps], s_out[2];
+    const int c = blockIdx.x, t = threadIdx.x;  // c = i * K + k
+    const int H = a.hidden, V = H >> 3, K = a.top_k;
 
-    const int e = blockIdx.x / a.splits, sp = blockIdx.x % a.splits;
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-
-    // 1. the instance's smooth row -> shared memory, one bulk copy
-    if (t == 0) {
-        mbar_init(&s_bar, 1);
-        mbar_arrive_expect_tx(&s_bar, (uint32_t)H * sizeof(float));
-        bulk_copy_g2s(s_sm, a.smooth + (size_t)e * H, (uint32_t)H * sizeof(float), &s_bar);
-    }
-
-    // 2. the copies sent to e, in (token, k) order: warp w scans the contiguous
-    //    copies [w * per_warp, (w + 1) * per_warp), 32 per round
-    const int per_warp = im_per_warp(N);
-    const int rounds = per_warp >> 5;
-    const unsigned lower = (1u << lane) - 1u;
-    int key[kImMaxKeys];
-    int cnt = 0, less = 0;
-#pragma unroll
-    for (int u = 0; u < kImMaxKeys; ++u) {
-        const int j = w * per_warp + u * 32 + lane;
-        key[u] = (u < rounds && j < N) ? copy_key(a, j) : -1;
-    }
-#pragma unroll
-    for (int u = 0; u < kImMaxKeys; ++u) {
-        if (u >= rounds) break;
-        const int k = key[u];
-        less += (k >= 0 && k < e) ? 1 : 0;
-        cnt += __popc(__ballot_sync(kFull, k == e));
-        if (blockIdx.x == 0 && k < 0) {
-            const int j = w * per_warp + u * 32 + lane;
-            if (j < N) {
-                a.expand_idx[j] = -1;  // not sent
-                if (k == -2) raise_error(a.err, kDevBadId);
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) less += __shfl_xor_sync(kFull, less, o);
-    if (lane == 0) {
-        s_wcnt[w] = cnt;
-        s_wless[w] = less;
-    }
-    __syncthreads();
-    int wbase = 0, count = 0, start = 0;
-#pragma unroll
-    for (int u = 0; u < kDpWarps; ++u) {
-        wbase += (u < w) ? s_wcnt[u] : 0;
-        count += s_wcnt[u];
-        start += s_wless[u];
-    }
-    const int r0 = (int)((long long)count * sp / a.splits);
-    const int r1 = (int)((long long)count * (sp + 1) / a.splits);
-    if (sp == 0 && t == 0) {
-        a.counts[e] = count;
-        a.offsets[e] = start;
-        if (e == E - 1) a.offsets[E] = start + count;
-    }
-    // second pass over the same keys: place this block's rows
-    int pos = wbase;
-#pragma unroll
-    for (int u = 0; u < kImMaxKeys; ++u) {
-        if (u >= rounds) break;
-        const int k = key[u];
-        const unsigned hit = __ballot_sync(kFull, k == e);
-        if (k == e) {
-            const int r = pos + __popc(hit & lower);
-            if (r >= r0 && r < r1) {
-                const int j = w * per_warp + u * 32 + lane;
-                s_tok[r - r0] = j / K;
-                a.src_of_row[start + r] = j;
-                a.expand_idx[j] = start + r;
-            }
-        }
-        pos += __popc(hit);
-    }
-
-    // 3. wait (bounded) for the smooth row; every thread observes it itself
-    if (!__syncthreads_and(mbar_wait_bounded(&s_bar, 0))) {
-        if (t == 0) {
-            raise_error(a.err, kDevTimeout);
-            mbar_wait_bounded(&s_bar, 0);  // a last bounded wait for the copy in flight
-        }
-        return;
-    }
-
-    // 4. smooth row -> registers (fp32 pairs), then quantize the rows, loading
-    //    the next row's token while this one reduces
-    uint64_t sv[kDpVecs][4];
+    // inputs of the call only: safe before the route kernel is done
+    const int e = copy_key(a, c);
+    if (e < 0) return;  // not sent (or a bad id, which route_kernel reports)
+    const uint16_t *xrow = a.x + (size_t)(c / K) * H;
+    const float *srow = a.smooth + (size_t)e * H;
+    uint64_t xf[kDpVecs][4];
 #pragma unroll
     for (int q = 0; q < kDpVecs; ++q) {
         const int p = t + q * kDpThreads;
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-            sv[q][h] = p < V ? *reinterpret_cast<const uint64_t *>(s_sm + p * 8 + 2 * h) : 0ull;
+        uint4 xv = make_uint4(0, 0, 0, 0);
+        float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+        if (p < V) {
+            xv = ld_stream(xrow + p * 8);
+            s0 = __ldg(reinterpret_cast<const float4 *>(srow + p * 8));
+            s1 = __ldg(reinterpret_cast<const float4 *>(srow + p * 8) + 1);
+        }
+        uint64_t f[4];
+        vec_to_f2(xv, f);
+        xf[q][0] = f2_mul(f[0], f2_pack(s0.x, s0.y));  // xFp32 = x * smooth
+        xf[q][1] = f2_mul(f[1], f2_pack(s0.z, s0.w));
+        xf[q][2] = f2_mul(f[2], f2_pack(s1.x, s1.y));
+        xf[q][3] = f2_mul(f[3], f2_pack(s1.z, s1.w));
     }
-    auto load_row = [&](int r, uint4 (&xv)[kDpVecs]) {
-        const uint16_t *xr = a.x + (size_t)s_tok[r - r0] * H;
-#pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {
-            const int p = t + q * kDpThreads;
-            xv[q] = p < V ? ld_stream(xr + p * 8) : make_uint4(0, 0, 0, 0);
-        }
-    };
-    uint4 xn[kDpVecs];
-    if (r0 < r1) load_row(r0, xn);
-    for (int r = r0; r < r1; ++r) {  // uniform over the block
-        uint64_t xf[kDpVecs][4];
-#pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {
-            uint64_t f[4];
-            vec_to_f2(xn[q], f);
-#pragma unroll
-            for (int h = 0; h < 4; ++h) xf[q][h] = f2_mul(f[h], sv[q][h]);  // xFp32 = x * smooth
-        }
-        if (r + 1 < r1) load_row(r + 1, xn);
-        const int row = start + r;
-        uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
-        if constexpr (MODE == 2) {
-            float m = 0.0f;
-#pragma unroll
-            for (int q = 0; q < kDpVecs; ++q) m = fmaxf(m, abs_max8(xf[q]));
-            const float2 ds = block_dyn(m, s_red, s_dyn);
-#pragma unroll
-            for (int q = 0; q < kDpVecs; ++q) {
-                const int p = t + q * kDpThreads;
-                if (p < V) *reinterpret_cast<uint2 *>(dst + p * 8) = int8x8_any(xf[q], ds.x);
-            }
-            if (t == 0) reinterpret_cast<float *>(a.dyn_scales)[row] = ds.y;
-        } else {  // MODE 3: a 128-element tile is 16 vectors = 16 consecutive lanes
-#pragma unroll
-            for (int q = 0; q < kDpVecs; ++q) {
-                const int p = t + q * kDpThreads;
-                float m = abs_max8(xf[q]);  // 0 for p >= V
-                m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-                m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
-                m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
-                m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
-                if (p < V) {
-                    const float dyn = __fdiv_rn(127.0f, m);
-                    *reinterpret_cast<uint2 *>(dst + p * 8) = int8x8_any(xf[q], dyn);
-                    if ((t & 15) == 0)
-                        reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (p >> 4)] = __frcp_rn(dyn);
-                }
-            }
-        }
-    }
+    uint2 qv[kDpVecs];
+    float seg[kDpVecs] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float row_scale = 0.0f;
+    quantize_vecs<MODE>(xf, V, s_red, s_out, qv, seg, row_scale);
+
+    pdl_wait();  // the row comes from route_kernel
+    const int row = a.expand_idx[c];
+    if (row >= 0) write_row<MODE>(a, row, V, qv, seg, row_scale);
 }
 
 }  // namespace moe

@@ -20,10 +20,6 @@ inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintp
 
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
-inline moe_status launch_status() {
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
-
 bool check_workspace(const void *ws, size_t bytes) {
     return ws != nullptr && aligned(ws, 16) && bytes >= kWorkspaceBytes;
 }
@@ -80,39 +76,46 @@ bool valid_combine(const moe_combine_params &p) {
     return true;
 }
 
+// Every kernel is launched as a programmatic dependent of whatever precedes it
+// on the stream: its blocks may be scheduled while the previous kernel drains,
+// and each kernel calls griddepcontrol.wait before it touches memory a
+// predecessor could still be writing or reading (the route -> scatter pair
+// inside moe_dispatch is the one edge where the dependent first works on the
+// call's own inputs; the route kernel only releases it after its own wait).
+// The attribute is harmless when the predecessor is not a kernel.
 template <typename Args>
 cudaError_t launch(void (*kernel)(Args), int grid, int block, size_t smem, cudaStream_t s, const Args &args) {
-    kernel<<<grid, block, smem, s>>>(args);
-    return cudaGetLastError();
-}
-
-// Blocks per instance for the smooth-scale kernel: about four rows each.
-int dispatch_splits(int copies, int instances) {
-    const int avg = (copies + instances - 1) / instances;
-    int s = (avg + 3) / 4;
-    return s < 1 ? 1 : (s > 16 ? 16 : s);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args);
 }
 
 template <int MODE>
 cudaError_t launch_dispatch_token(const moe::DispatchArgs &a, cudaStream_t s) {
-    const size_t smem = moe::token_smem_bytes(a.num_instances);
-    if (!ensure_smem(moe::dispatch_token_kernel<MODE>, smem, 1 + MODE)) return cudaErrorInvalidValue;
-    return launch(moe::dispatch_token_kernel<MODE>, a.bs, moe::kDpThreads, smem, s, a);
+    if (!ensure_smem(moe::dispatch_token_kernel<MODE>, 0, 1 + MODE)) return cudaErrorInvalidValue;
+    return launch(moe::dispatch_token_kernel<MODE>, a.bs, moe::kDpThreads, 0, s, a);
 }
 
 template <int MODE>
-cudaError_t launch_dispatch_instance(const moe::DispatchArgs &a, cudaStream_t s) {
-    const size_t smem = moe::instance_smem_bytes(a.hidden, a.bs * a.top_k, a.splits);
-    if (!ensure_smem(moe::dispatch_instance_kernel<MODE>, smem, 6 + MODE)) return cudaErrorInvalidValue;
-    return launch(moe::dispatch_instance_kernel<MODE>, a.num_instances * a.splits, moe::kDpThreads, smem, s, a);
+cudaError_t launch_dispatch_copy(const moe::DispatchArgs &a, cudaStream_t s) {
+    if (!ensure_smem(moe::dispatch_copy_kernel<MODE>, 0, 6 + MODE)) return cudaErrorInvalidValue;
+    return launch(moe::dispatch_copy_kernel<MODE>, a.bs * a.top_k, moe::kDpThreads, 0, s, a);
 }
 
 // Persistent combine: one block per SM (at least one per 8 tokens); the ring
-// depth is the largest of 8 / 4 / 2 units whose slots fit in 200 KB.
-template <int KMAX, bool SHARED, int DEPTH>
-cudaError_t launch_combine_d(const moe::CombineArgs &a, cudaStream_t s, int slot) {
-    auto kernel = moe::combine_kernel<KMAX, SHARED, DEPTH>;
-    const size_t smem = moe::combine_smem_bytes(DEPTH, a.top_k, SHARED);
+// holds the most stages (8, 4 or 2) whose units fit in 200 KB.
+template <int KMAX, bool SHARED, int STAGES>
+cudaError_t launch_combine_s(const moe::CombineArgs &a, cudaStream_t s, int slot) {
+    auto kernel = moe::combine_kernel<KMAX, SHARED, STAGES>;
+    const size_t smem = moe::combine_smem_bytes(STAGES, a.top_k, SHARED);
     if (!ensure_smem(kernel, smem, slot)) return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
@@ -127,10 +130,10 @@ cudaError_t launch_combine_d(const moe::CombineArgs &a, cudaStream_t s, int slot
 template <int KMAX, bool SHARED>
 cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
     const size_t budget = 200 * 1024;
-    const int base = 10 + (KMAX / 8) * 6 + (SHARED ? 3 : 0);
-    if (moe::combine_smem_bytes(8, a.top_k, SHARED) <= budget) return launch_combine_d<KMAX, SHARED, 8>(a, s, base);
-    if (moe::combine_smem_bytes(4, a.top_k, SHARED) <= budget) return launch_combine_d<KMAX, SHARED, 4>(a, s, base + 1);
-    return launch_combine_d<KMAX, SHARED, 2>(a, s, base + 2);
+    const int slot = 12 + (KMAX / 8) * 6 + (SHARED ? 3 : 0);
+    if (moe::combine_smem_bytes(8, a.top_k, SHARED) <= budget) return launch_combine_s<KMAX, SHARED, 8>(a, s, slot);
+    if (moe::combine_smem_bytes(4, a.top_k, SHARED) <= budget) return launch_combine_s<KMAX, SHARED, 4>(a, s, slot + 1);
+    return launch_combine_s<KMAX, SHARED, 2>(a, s, slot + 2);
 }
 
 template <int KMAX>
@@ -209,8 +212,9 @@ moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_i
     a.err = reinterpret_cast<uint32_t *>(workspace);
     const size_t smem = moe::update_expert_smem_bytes(p->ep_world_size);
     if (!ensure_smem(moe::update_expert_kernel, smem, 0)) return MOE_ERR_CUDA;
-    moe::update_expert_kernel<<<1, moe::kUeThreads, smem, as_stream(cuda_stream)>>>(a);
-    return launch_status();
+    return launch(moe::update_expert_kernel, 1, moe::kUeThreads, smem, as_stream(cuda_stream), a) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 // -------------------------------------------------------------- dispatch ---
@@ -246,7 +250,6 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     a.top_k = p->top_k;
     a.num_instances = p->num_instances;
     a.tiles = (p->hidden + 127) / 128;
-    a.splits = dispatch_splits(p->bs * p->top_k, p->num_instances);
     a.x = reinterpret_cast<const uint16_t *>(x);
     a.ids = instance_ids;
     a.mask = mask;
@@ -259,9 +262,13 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     a.offsets = expert_offsets;
     a.err = reinterpret_cast<uint32_t *>(workspace);
     cudaStream_t s = as_stream(cuda_stream);
+
+    const size_t rsmem = moe::route_smem_bytes(p->num_instances);
+    if (!ensure_smem(moe::route_kernel, rsmem, 11)) return MOE_ERR_CUDA;
+    if (launch(moe::route_kernel, 1, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     if (smooth_scales) {
-        e = mode == 2 ? launch_dispatch_instance<2>(a, s) : launch_dispatch_instance<3>(a, s);
+        e = mode == 2 ? launch_dispatch_copy<2>(a, s) : launch_dispatch_copy<3>(a, s);
     } else {
         switch (mode) {
             case 0: e = launch_dispatch_token<0>(a, s); break;

@@ -58,6 +58,9 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     __shared__ int s_warp[32];
     __shared__ int s_bad, s_total;
 
+    pdl_wait();               // the ids may come from the previous kernel
+    pdl_launch_dependents();  // the next kernel waits for this one before it reads anything
+
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int F = a.table_cols, ws = a.ep_world_size, E = a.num_logical;
 
