@@ -49,6 +49,7 @@ EXPORTS = (
     "moe_update_expert_workspace_size", "moe_update_expert",
     "moe_dispatch_workspace_size", "moe_dispatch",
     "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm",
+    "moe_dispatch_noalloc",
 )
 
 
@@ -70,6 +71,7 @@ def _load():
     L.moe_dispatch.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_combine_add_rmsnorm_workspace_size.argtypes = [P(CombineParams), P(sz)]
     L.moe_combine_add_rmsnorm.argtypes = [P(CombineParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_dispatch_noalloc.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         if name != "moe_status_string":
             getattr(L, name).restype = ctypes.c_int
@@ -230,3 +232,27 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
         _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")), _ptr(out.get("rstd")),
         _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def dispatch_noalloc(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=None, smooth=None,
+                     out=None, device_error=None, stream=None):
+    """moe_dispatch_noalloc: moe_dispatch with the library's own static scratch
+    instead of a workspace.  device_error: optional int32 CUDA tensor of one
+    element that receives the call's device error word."""
+    _req(x, "x", torch.bfloat16)
+    bs, H = x.shape
+    _req(instance_ids, "instance_ids", torch.int32)
+    k = instance_ids.shape[1]
+    _req(instance_ids, "instance_ids", torch.int32, (bs, k))
+    _opt(mask, "mask", torch.uint8, (bs, k))
+    _opt(smooth, "smooth", torch.float32, (num_instances, H))
+    _opt(device_error, "device_error", torch.int32, (1,))
+    if out is None:
+        out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
+    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode))
+    _check("moe_dispatch_noalloc", lib.moe_dispatch_noalloc(
+        ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
+        _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
+        _ptr(out["offsets"]), _ptr(device_error), _stream(stream)))
+    return out
+

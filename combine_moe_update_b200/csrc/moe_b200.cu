@@ -324,4 +324,53 @@ moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expa
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// ------------------------------------------------------- dispatch, no alloc ---
+
 }  // extern "C"
+
+namespace {
+
+// The workspace of moe_dispatch_noalloc: a fixed array in every GPU's memory,
+// so that callers who cannot allocate need not pass one.  Host code must not
+// use this name as an address; the device address is looked up per device.
+__device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+void *noalloc_scratch_address(int dev) {
+    static void *addr[64];  // per device, filled on first use
+    if (dev < 0 || dev >= 64) return nullptr;
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" moe_status moe_dispatch_noalloc(const moe_dispatch_params *p, const void *x,
+                                           const int32_t *instance_ids, const uint8_t *mask,
+                                           const float *smooth_scales, void *expand_x, void *dyn_scales,
+                                           int32_t *expand_idx, int32_t *src_of_row, int32_t *expert_counts,
+                                           int32_t *expert_offsets, uint32_t *device_error_out,
+                                           void *cuda_stream) {
+    size_t need = 0;
+    const moe_status st = moe_dispatch_workspace_size(p, &need);
+    if (st != MOE_OK) return st;
+    if (need > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+    if (device_error_out && !aligned(device_error_out, 4)) return MOE_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    void *ws = noalloc_scratch_address(dev);
+    if (ws == nullptr) return MOE_ERR_CUDA;
+    cudaStream_t s = as_stream(cuda_stream);
+    // the array keeps the previous call's error word: start this call from zero
+    if (cudaMemsetAsync(ws, 0, need, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const moe_status r = moe_dispatch(p, x, instance_ids, mask, smooth_scales, expand_x, dyn_scales, expand_idx,
+                                      src_of_row, expert_counts, expert_offsets, ws, need, cuda_stream);
+    if (r != MOE_OK) return r;
+    if (device_error_out &&
+        cudaMemcpyAsync(device_error_out, ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}

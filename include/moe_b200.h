@@ -233,6 +233,40 @@ MOE_API moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const vo
                                    void *y, void *x_out, float *rstd_out, void *workspace,
                                    size_t workspace_bytes, void *cuda_stream);
 
+/* ------------------------------------------------------------------------ */
+/* moe_dispatch_noalloc -- moe_dispatch without a caller-provided workspace  */
+/* ------------------------------------------------------------------------ */
+
+/* Largest workspace moe_dispatch_noalloc can stand in for (bytes). */
+#define MOE_NOALLOC_SCRATCH_BYTES 256
+
+/*
+ * The operator pages have no counterpart for this call; it exists for
+ * callers that cannot allocate device memory of their own: runtimes that
+ * hand a kernel only the tensors it reads and writes (no workspace), or that
+ * run under a fixed memory plan where a cudaMalloc after start-up is not
+ * allowed.  It does exactly what moe_dispatch does, with the same arguments
+ * and results, but the workspace lives in a static device array inside the
+ * library (MOE_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that loads
+ * the library until the process exits).  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *
+ *   device_error_out  optional device pointer (4 bytes, caller-owned): receives
+ *                     this call's device error word (MOE_DEV_* bits) at its end.
+ *
+ * The first call on a device looks the array's device address up (with that
+ * device current); make that first call before any stream capture.  Each call
+ * zeroes the error word first, and every call on a device shares the one
+ * array, so calls that overlap on the GPU (other streams, other threads) race
+ * on it.  Returns MOE_ERR_WORKSPACE if the call would need more scratch than
+ * the array holds; other errors as moe_dispatch.
+ */
+MOE_API moe_status moe_dispatch_noalloc(const moe_dispatch_params *p, const void *x, const int32_t *instance_ids,
+                                        const uint8_t *mask, const float *smooth_scales, void *expand_x,
+                                        void *dyn_scales, int32_t *expand_idx, int32_t *src_of_row,
+                                        int32_t *expert_counts, int32_t *expert_offsets, uint32_t *device_error_out,
+                                        void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
