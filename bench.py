@@ -4,8 +4,9 @@
 One step = one MoE layer's hot path on one batch of seeded synthetic input:
 moe_update_expert -> moe_dispatch -> moe_combine_add_rmsnorm (the expert FFN
 between dispatch and combine is stood in for by a resident buffer of bf16
-expert-output rows).  Every timed step starts with a cold L2 (a 512 MiB
-buffer is overwritten before it, outside the timed events).
+expert-output rows).  Every timed step starts with a cold, clean L2 (a
+512 MiB buffer is overwritten and a 256 MiB one read before it, outside the
+timed events).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
 
@@ -215,8 +216,16 @@ def run_b200(args, rank, world, local_rank):
         B.combine_add_rmsnorm(ee, d["expand_idx"], ss, rr, gamma, w.norm_eps, shared_x=sh, workspace=ws, out=c)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    for _ in range(args.warmup):
+    clean = torch.empty(L2_FLUSH_BYTES // 2, dtype=torch.uint8, device="cuda")
+
+    def flush_l2():
+        # overwrite 512 MiB, then read 256 MiB: L2 then holds neither the step's
+        # inputs nor dirty lines whose write-back would land in the timed step
         flush.zero_()
+        clean.sum(dtype=torch.int64)
+
+    for _ in range(args.warmup):
+        flush_l2()
         step()
     torch.cuda.synchronize()
     assert B.read_device_error(ws) == 0, "device error during warm-up"
@@ -235,7 +244,7 @@ def run_b200(args, rank, world, local_rank):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=cap):
         for s_ in range(G):
-            flush.zero_()
+            flush_l2()
             e = ev[s_]
             e[0].record()
             B.update_expert(ids, table, w.ep_world_size, expert_scales=scales, prune_threshold=w.prune_threshold,
@@ -317,7 +326,7 @@ def run_b200(args, rank, world, local_rank):
                    "num_instances": w.num_instances, "ep_world_size_simulated": w.ep_world_size,
                    "quant_mode": w.quant_mode, "smooth_scales": w.smooth is not None,
                    "shared_expert": w.shared_x is not None, "kept_copies": n,
-                   "l2": "flushed (512 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
+                   "l2": "flushed before every timed step: 512 MiB written, then 256 MiB read", "parallelism": f"replicas x{world}"},
         "breakdown_us": {"update_expert": round(t_upd * 1e3, 2), "dispatch": round(t_disp * 1e3, 2),
                          "combine": round(t_comb * 1e3, 2)},
         "dispatch_plus_combine": {"tokens_per_s": round(dc_value, 1), "hbm_gbs": round(dc_gbs, 1),

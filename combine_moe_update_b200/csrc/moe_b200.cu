@@ -28,9 +28,9 @@ bool check_workspace(const void *ws, size_t bytes) {
 // device (cached per device and kernel).
 template <typename Kernel>
 bool ensure_smem(Kernel k, size_t bytes, int slot) {
-    static int done[64][32];
+    static int done[64][48];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 32) return false;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 48) return false;
     if (done[dev][slot] >= (int)bytes + 1) return true;
     if (bytes > 48 * 1024 &&
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
@@ -110,30 +110,22 @@ cudaError_t launch_dispatch_copy(const moe::DispatchArgs &a, cudaStream_t s) {
     return launch(moe::dispatch_copy_kernel<MODE>, a.bs * a.top_k, moe::kDpThreads, 0, s, a);
 }
 
-// Persistent combine: one block per SM (at least one per 8 tokens); the ring
-// holds the most stages (8, 4 or 2) whose units fit in 200 KB.
-template <int KMAX, bool SHARED, int STAGES>
-cudaError_t launch_combine_s(const moe::CombineArgs &a, cudaStream_t s, int slot) {
-    auto kernel = moe::combine_kernel<KMAX, SHARED, STAGES>;
-    const size_t smem = moe::combine_smem_bytes(STAGES, a.top_k, SHARED);
-    if (!ensure_smem(kernel, smem, slot)) return cudaErrorInvalidValue;
-    int dev = 0, sms = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cudaErrorUnknown;
-    int grid = sms;
-    const int min_grid = (a.bs + moe::kCbMaxTokens - 1) / moe::kCbMaxTokens;
-    if (grid < min_grid) grid = min_grid;
-    if (grid > a.bs) grid = a.bs;
-    return launch(kernel, grid, moe::kCbThreads, smem, s, a);
+// combine: one 128-thread block per token; VECS = ceil(H / 1024) vectors per thread.
+template <int KMAX, bool SHARED, int VECS>
+cudaError_t launch_combine_v(const moe::CombineArgs &a, cudaStream_t s, int slot) {
+    auto kernel = moe::combine_kernel<KMAX, SHARED, VECS>;
+    if (!ensure_smem(kernel, 0, slot)) return cudaErrorInvalidValue;
+    return launch(kernel, a.bs, moe::kCbThreads, 0, s, a);
 }
 
 template <int KMAX, bool SHARED>
 cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
-    const size_t budget = 200 * 1024;
-    const int slot = 12 + (KMAX / 8) * 6 + (SHARED ? 3 : 0);
-    if (moe::combine_smem_bytes(8, a.top_k, SHARED) <= budget) return launch_combine_s<KMAX, SHARED, 8>(a, s, slot);
-    if (moe::combine_smem_bytes(4, a.top_k, SHARED) <= budget) return launch_combine_s<KMAX, SHARED, 4>(a, s, slot + 1);
-    return launch_combine_s<KMAX, SHARED, 2>(a, s, slot + 2);
+    const int vecs = (a.hidden / 8 + moe::kCbThreads - 1) / moe::kCbThreads;  // 1..8
+    const int slot = 12 + ((KMAX / 8) * 2 + (SHARED ? 1 : 0)) * 4;
+    if (vecs <= 2) return launch_combine_v<KMAX, SHARED, 2>(a, s, slot);
+    if (vecs <= 4) return launch_combine_v<KMAX, SHARED, 4>(a, s, slot + 1);
+    if (vecs <= 7) return launch_combine_v<KMAX, SHARED, 7>(a, s, slot + 2);
+    return launch_combine_v<KMAX, SHARED, 8>(a, s, slot + 3);
 }
 
 template <int KMAX>
