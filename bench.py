@@ -216,13 +216,13 @@ def run_b200(args, rank, world, local_rank):
         B.combine_add_rmsnorm(ee, d["expand_idx"], ss, rr, gamma, w.norm_eps, shared_x=sh, workspace=ws, out=c)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    clean = torch.empty(L2_FLUSH_BYTES // 2, dtype=torch.uint8, device="cuda")
+    clean = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.float32, device="cuda")  # 256 MiB
 
     def flush_l2():
         # overwrite 512 MiB, then read 256 MiB: L2 then holds neither the step's
         # inputs nor dirty lines whose write-back would land in the timed step
         flush.zero_()
-        clean.sum(dtype=torch.int64)
+        clean.sum()
 
     for _ in range(args.warmup):
         flush_l2()
@@ -337,7 +337,7 @@ def run_b200(args, rank, world, local_rank):
         "e2e": {"value": round(world * w.bs / (t_e2e * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "pinned host activations -> device, the three calls, y -> host; layer parameters resident"},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 4 * K,  # update_expert, route, quantize-and-scatter, combine
         "timing": f"CUDA graphs of {G} steps; per-op CUDA events recorded as graph nodes",
         "clocks": clk.summary(),
     }

@@ -18,7 +18,7 @@ from . import build as _build
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
 DEV_BAD_ID, DEV_BAD_TABLE = 1, 2
-WORKSPACE_BYTES = 256
+WORKSPACE_BYTES = 256  # MOE_MAX_WORKSPACE_BYTES: serves every call
 
 
 class MoeError(RuntimeError):

@@ -5,16 +5,20 @@
 //   x = combineOut + residualX
 //   y = x / sqrt(mean(x^2) + normEps) * gamma
 //
-// One block of 128 threads per token, small enough that every token of a
-// decode batch is resident at once (Bs 512 needs 4 blocks per SM): the whole
-// transfer -- K expert rows gathered through expand_idx (the AllToAllV back),
-// the shared-expert row and the residual row -- is in flight in a single wave
-// instead of trickling through a bounded pipeline.  Thread t owns the
-// 8-element vectors p = t, t + 128, ... of the row; it issues all of its
-// 16-byte loads first, then accumulates in fp32 and keeps x in registers.
-// One block reduction gives sum(x^2); then y (and x) are written.  Every
-// input byte is read once and every output byte written once.
+// Each token is handled by a cluster of two 128-thread blocks, one per half
+// of the row, small enough that every token of a decode batch is resident at
+// once (Bs 512 -> 1024 blocks, 7 per SM): the whole transfer -- K expert rows
+// gathered through expand_idx (the AllToAllV back), the shared-expert row and
+// the residual row -- is in flight in a single wave, and half-token blocks
+// spread evenly over the SMs.  Thread t owns 8-element vectors of its half;
+// it issues all of its 16-byte loads first, then accumulates in fp32 and
+// keeps x in registers.  The two halves' sum(x^2) meet through distributed
+// shared memory (added in a fixed order, so both blocks get the same bits);
+// then each block writes its half of y (and x).  Every input byte is read
+// once and every output byte written once.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace moe {
@@ -36,14 +40,19 @@ struct CombineArgs {
 
 constexpr int kCbThreads = 128;
 
-// VECS: 8-element vectors per thread (ceil(H / 8 / 128) <= 8).
+// VECS: 8-element vectors per thread (ceil(H / 16 / 128) <= 4).
 template <int KMAX, bool SHARED, int VECS>
-__global__ void __launch_bounds__(kCbThreads, 4) combine_kernel(CombineArgs a) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kCbThreads, 7) combine_kernel(CombineArgs a) {
+    namespace cg = cooperative_groups;
     __shared__ int s_row[16];
     __shared__ float s_w[16];
     __shared__ float s_red[kCbThreads / 32];
-    const int i = blockIdx.x, t = threadIdx.x;
+    __shared__ float s_part;
+    const cg::cluster_group cluster = cg::this_cluster();
+    const int half = (int)cluster.block_rank();  // 0: first half of the row, 1: second
+    const int i = blockIdx.x >> 1, t = threadIdx.x;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
+    const int v0 = half ? (V + 1) / 2 : 0, v1 = half ? V : (V + 1) / 2;  // this block's vectors
 
     pdl_wait();  // expand_idx and the expert rows come from earlier kernels
     if (t < K) {
@@ -72,10 +81,10 @@ __global__ void __launch_bounds__(kCbThreads, 4) combine_kernel(CombineArgs a) {
     float ss = 0.0f;
 #pragma unroll
     for (int j = 0; j < VECS; ++j) {
-        const int p = t + j * kCbThreads;
+        const int p = v0 + t + j * kCbThreads;
 #pragma unroll
         for (int e = 0; e < 8; ++e) xs[j][e] = 0.0f;
-        if (p >= V) continue;
+        if (p >= v1) continue;
         uint4 rv[KMAX];
 #pragma unroll
         for (int k = 0; k < KMAX; ++k)
@@ -110,12 +119,17 @@ __global__ void __launch_bounds__(kCbThreads, 4) combine_kernel(CombineArgs a) {
     }
 
     ss = block_sum<kCbThreads / 32>(ss, s_red);
-    const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(ss, (float)H) + a.norm_eps));
-    if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
+    if (t == 0) s_part = ss;
+    cluster.sync();  // both halves' partial sums are in place
+    const float other = *cluster.map_shared_rank(&s_part, half ^ 1);
+    const float tot = half ? other + ss : ss + other;  // first half + second half, in both blocks
+    cluster.sync();  // neither block leaves while the other may still read it
+    const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));
+    if (t == 0 && half == 0 && a.rstd_out) a.rstd_out[i] = rstd;
 #pragma unroll
     for (int j = 0; j < VECS; ++j) {
-        const int p = t + j * kCbThreads;
-        if (p >= V) continue;
+        const int p = v0 + t + j * kCbThreads;
+        if (p >= v1) continue;
         float g[8];
         unpack8(ld_cached(a.gamma + p * 8), g);
         uint4 yo;

@@ -110,11 +110,23 @@ __device__ __forceinline__ void st_v4(void *p, uint4 v) { *reinterpret_cast<uint
 // multiply-add; where the product's own rounding matters, multiply with the
 // scalar __fmul_rn instead. ---
 
+// Pairs are built and split with register-pair moves, which cost no
+// instruction once registers are allocated.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
 }
-__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ float f2_lo(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+__device__ __forceinline__ float f2_hi(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
 
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     uint64_t d;
@@ -134,7 +146,7 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 
 // A bf16 pair (one 32-bit word, element 0 in the low half) as an fp32 pair.
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
-    return (uint64_t)(w << 16) | ((uint64_t)(w & 0xffff0000u) << 32);
+    return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
 // cp.async (16 bytes, global -> shared, bypassing L1) and its group control.
@@ -186,6 +198,29 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int *s_warp) {
     }
     __syncthreads();
     if (w > 0) v += s_warp[w - 1];
+    return v;
+}
+
+// floor(n / d) for 0 <= n < 2^16 and 1 <= d <= 2^16, given magic = ceil(2^32 / d)
+// (from div_magic; 0 stands for d = 1, whose magic 2^32 does not fit).
+// Writing magic = (2^32 + r) / d with 0 <= r < d, the product
+// n * magic / 2^32 = n / d + n r / (d 2^32) and the second term is below 1/d,
+// so it never carries floor(n / d) past the next integer.
+__host__ __device__ inline uint32_t div_magic(uint32_t d) {
+    return d <= 1 ? 0u : (uint32_t)((0x100000000ull + d - 1) / d);
+}
+__device__ __forceinline__ uint32_t div_by_magic(uint32_t n, uint32_t magic) {
+    return magic ? __umulhi(n, magic) : n;
+}
+
+// Inclusive prefix sum across the 32 lanes of a warp.
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += y;
+    }
     return v;
 }
 

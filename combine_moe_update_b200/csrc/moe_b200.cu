@@ -20,6 +20,9 @@ inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintp
 
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// The dispatch workspace: the error-word area.
+size_t dispatch_workspace_bytes(const moe_dispatch_params &) { return kWorkspaceBytes; }
+
 bool check_workspace(const void *ws, size_t bytes) {
     return ws != nullptr && aligned(ws, 16) && bytes >= kWorkspaceBytes;
 }
@@ -83,8 +86,8 @@ bool valid_combine(const moe_combine_params &p) {
 // inside moe_dispatch is the one edge where the dependent first works on the
 // call's own inputs; the route kernel only releases it after its own wait).
 // The attribute is harmless when the predecessor is not a kernel.
-template <typename Args>
-cudaError_t launch(void (*kernel)(Args), int grid, int block, size_t smem, cudaStream_t s, const Args &args) {
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
@@ -95,37 +98,38 @@ cudaError_t launch(void (*kernel)(Args), int grid, int block, size_t smem, cudaS
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args);
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 template <int MODE>
 cudaError_t launch_dispatch_token(const moe::DispatchArgs &a, cudaStream_t s) {
     if (!ensure_smem(moe::dispatch_token_kernel<MODE>, 0, 1 + MODE)) return cudaErrorInvalidValue;
-    return launch(moe::dispatch_token_kernel<MODE>, a.bs, moe::kDpThreads, 0, s, a);
+    return launch(moe::dispatch_token_kernel<MODE>, a.bs, moe::dp_threads(a.hidden >> 3), 0, s, a);
 }
 
 template <int MODE>
-cudaError_t launch_dispatch_copy(const moe::DispatchArgs &a, cudaStream_t s) {
-    if (!ensure_smem(moe::dispatch_copy_kernel<MODE>, 0, 6 + MODE)) return cudaErrorInvalidValue;
-    return launch(moe::dispatch_copy_kernel<MODE>, a.bs * a.top_k, moe::kDpThreads, 0, s, a);
+cudaError_t launch_dispatch_token_smooth(const moe::DispatchArgs &a, cudaStream_t s) {
+    if (!ensure_smem(moe::dispatch_token_smooth_kernel<MODE>, 0, 8 + MODE)) return cudaErrorInvalidValue;
+    return launch(moe::dispatch_token_smooth_kernel<MODE>, a.bs, moe::dp_threads(a.hidden >> 3), 0, s, a);
 }
 
-// combine: one 128-thread block per token; VECS = ceil(H / 1024) vectors per thread.
+// combine: a cluster of two 128-thread blocks per token (one per half row);
+// VECS = ceil(H / 16 / 128) vectors per thread.
 template <int KMAX, bool SHARED, int VECS>
 cudaError_t launch_combine_v(const moe::CombineArgs &a, cudaStream_t s, int slot) {
     auto kernel = moe::combine_kernel<KMAX, SHARED, VECS>;
     if (!ensure_smem(kernel, 0, slot)) return cudaErrorInvalidValue;
-    return launch(kernel, a.bs, moe::kCbThreads, 0, s, a);
+    return launch(kernel, 2 * a.bs, moe::kCbThreads, 0, s, a);
 }
 
 template <int KMAX, bool SHARED>
 cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
-    const int vecs = (a.hidden / 8 + moe::kCbThreads - 1) / moe::kCbThreads;  // 1..8
+    const int vecs = ((a.hidden / 8 + 1) / 2 + moe::kCbThreads - 1) / moe::kCbThreads;  // 1..4
     const int slot = 12 + ((KMAX / 8) * 2 + (SHARED ? 1 : 0)) * 4;
-    if (vecs <= 2) return launch_combine_v<KMAX, SHARED, 2>(a, s, slot);
-    if (vecs <= 4) return launch_combine_v<KMAX, SHARED, 4>(a, s, slot + 1);
-    if (vecs <= 7) return launch_combine_v<KMAX, SHARED, 7>(a, s, slot + 2);
-    return launch_combine_v<KMAX, SHARED, 8>(a, s, slot + 3);
+    if (vecs <= 1) return launch_combine_v<KMAX, SHARED, 1>(a, s, slot);
+    if (vecs <= 2) return launch_combine_v<KMAX, SHARED, 2>(a, s, slot + 1);
+    if (vecs <= 3) return launch_combine_v<KMAX, SHARED, 3>(a, s, slot + 2);
+    return launch_combine_v<KMAX, SHARED, 4>(a, s, slot + 3);
 }
 
 template <int KMAX>
@@ -194,6 +198,7 @@ moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_i
     a.num_logical = p->num_logical;
     a.table_cols = p->table_cols;
     a.ep_world_size = p->ep_world_size;
+    a.k_magic = moe::div_magic((uint32_t)p->top_k);
     a.prune_threshold = p->prune_threshold;
     a.expert_ids = expert_ids;
     a.expert_scales = expert_scales;
@@ -215,7 +220,7 @@ moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, size_t *byt
     if (p == nullptr || bytes == nullptr) return MOE_ERR_INVALID_ARG;
     moe_status st = valid_dispatch(*p);
     if (st != MOE_OK) return st;
-    *bytes = kWorkspaceBytes;
+    *bytes = dispatch_workspace_bytes(*p);
     return MOE_OK;
 }
 
@@ -235,13 +240,15 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
         !aligned(src_of_row, 4) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
         (smooth_scales && !aligned(smooth_scales, 16)) || ((mode == 2 || mode == 3) && !aligned(dyn_scales, 4)))
         return MOE_ERR_INVALID_ARG;
-    if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
+    if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < dispatch_workspace_bytes(*p))
+        return MOE_ERR_WORKSPACE;
     moe::DispatchArgs a;
     a.bs = p->bs;
     a.hidden = p->hidden;
     a.top_k = p->top_k;
     a.num_instances = p->num_instances;
     a.tiles = (p->hidden + 127) / 128;
+    a.k_magic = moe::div_magic((uint32_t)p->top_k);
     a.x = reinterpret_cast<const uint16_t *>(x);
     a.ids = instance_ids;
     a.mask = mask;
@@ -255,12 +262,13 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     a.err = reinterpret_cast<uint32_t *>(workspace);
     cudaStream_t s = as_stream(cuda_stream);
 
+    const int slices = moe::route_slices(p->bs * p->top_k);
     const size_t rsmem = moe::route_smem_bytes(p->num_instances);
     if (!ensure_smem(moe::route_kernel, rsmem, 11)) return MOE_ERR_CUDA;
-    if (launch(moe::route_kernel, 1, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch(moe::route_kernel, slices, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     if (smooth_scales) {
-        e = mode == 2 ? launch_dispatch_copy<2>(a, s) : launch_dispatch_copy<3>(a, s);
+        e = mode == 2 ? launch_dispatch_token_smooth<2>(a, s) : launch_dispatch_token_smooth<3>(a, s);
     } else {
         switch (mode) {
             case 0: e = launch_dispatch_token<0>(a, s); break;
@@ -357,7 +365,8 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_dispatch_params *p, const v
     if (ws == nullptr) return MOE_ERR_CUDA;
     cudaStream_t s = as_stream(cuda_stream);
     // the array keeps the previous call's error word: start this call from zero
-    if (cudaMemsetAsync(ws, 0, need, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // (the rest of the scratch is written before it is read within the call)
+    if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
     const moe_status r = moe_dispatch(p, x, instance_ids, mask, smooth_scales, expand_x, dyn_scales, expand_idx,
                                       src_of_row, expert_counts, expert_offsets, ws, need, cuda_stream);
     if (r != MOE_OK) return r;

@@ -21,6 +21,7 @@ namespace moe {
 
 struct UpdateArgs {
     int bs, top_k, num_logical, table_cols, ep_world_size;
+    uint32_t k_magic;  // div_magic(top_k)
     float prune_threshold;
     const int32_t *expert_ids;
     const float *expert_scales;  // may be null
@@ -34,10 +35,10 @@ struct UpdateArgs {
 constexpr int kUeThreads = 1024;
 constexpr int kUeItems = 8;  // copies per thread: bs * K <= 8192 = 1024 * 8
 
-// Dynamic shared memory: n[1024], first[1024], inst[1024] ints, then one
-// uint16 counter per (warp, rank).
+// Dynamic shared memory: n[1024], first[1024], inst[1024], the division
+// magic of every n[e] (1024), then one uint16 counter per (rank, warp).
 inline size_t update_expert_smem_bytes(int ep_world_size) {
-    return 3 * 1024 * sizeof(int) + 32 * (size_t)ep_world_size * sizeof(uint16_t);
+    return 4 * 1024 * sizeof(int) + 32 * (size_t)ep_world_size * sizeof(uint16_t);
 }
 
 __device__ __forceinline__ void update_expert_drop_all(const UpdateArgs &a) {
@@ -54,7 +55,8 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     int *s_n = reinterpret_cast<int *>(smem);
     int *s_first = s_n + 1024;
     int *s_inst = s_first + 1024;
-    uint16_t *s_wc = reinterpret_cast<uint16_t *>(s_inst + 1024);  // [32][ws]
+    uint32_t *s_mag = reinterpret_cast<uint32_t *>(s_inst + 1024);  // div_magic(n[e])
+    uint16_t *s_wc = reinterpret_cast<uint16_t *>(s_mag + 1024);   // [ws][32]
     __shared__ int s_warp[32];
     __shared__ int s_bad, s_total;
 
@@ -67,21 +69,29 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     // The copies' inputs do not depend on the table: load them first so the
     // loads overlap the table bookkeeping.
     const int items = a.bs * a.top_k;
+    // Every load is unconditional (indices clamped into range), so all of
+    // them are in flight together; items past the end are discarded below.
     int pe[kUeItems];
     float ps[kUeItems];
     bool pa[kUeItems];
 #pragma unroll
-    for (int u = 0; u < kUeItems; ++u) {
-        const int it = t + u * kUeThreads;
-        pe[u] = -1;
-        ps[u] = 0.0f;
-        pa[u] = true;
-        if (it < items) {
-            pe[u] = a.expert_ids[it];
-            if (a.expert_scales) ps[u] = a.expert_scales[it];
-            if (a.active_mask) pa[u] = a.active_mask[it / a.top_k] != 0;
-        }
+    for (int u = 0; u < kUeItems; ++u) pe[u] = __ldg(a.expert_ids + min(t + u * kUeThreads, items - 1));
+#pragma unroll
+    for (int u = 0; u < kUeItems; ++u) ps[u] = 0.0f;
+    if (a.expert_scales) {
+#pragma unroll
+        for (int u = 0; u < kUeItems; ++u) ps[u] = __ldg(a.expert_scales + min(t + u * kUeThreads, items - 1));
     }
+#pragma unroll
+    for (int u = 0; u < kUeItems; ++u) pa[u] = true;
+    if (a.active_mask) {
+#pragma unroll
+        for (int u = 0; u < kUeItems; ++u)
+            pa[u] = __ldg(a.active_mask + div_by_magic((uint32_t)min(t + u * kUeThreads, items - 1), a.k_magic)) != 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kUeItems; ++u)
+        if (t + u * kUeThreads >= items) pe[u] = -1;
 
     if (t == 0) s_bad = 0;
     for (int q = t; q < 32 * ws; q += kUeThreads) s_wc[q] = 0;
@@ -100,6 +110,7 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     if (t < E) {
         s_n[t] = n;
         s_first[t] = incl - n;
+        s_mag[t] = div_magic((uint32_t)n);
     }
     if (t == kUeThreads - 1) s_total = incl;
     __syncthreads();
@@ -130,27 +141,26 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     // 3. stable rank by r: lanes of one warp first, then warps in order
     const unsigned peers = __match_any_sync(kFull, r);
     const int intra = __popc(peers & ((1u << lane) - 1u));
-    if (r >= 0 && lane == __ffs(peers) - 1) s_wc[w * ws + r] = (uint16_t)__popc(peers);
+    if (r >= 0 && lane == __ffs(peers) - 1) s_wc[r * 32 + w] = (uint16_t)__popc(peers);
     __syncthreads();
     if (s_bad) {
         update_expert_drop_all(a);
         return;
     }
-    for (int rr = t; rr < ws; rr += kUeThreads) {
-        int run = 0;
-        for (int ww = 0; ww < 32; ++ww) {
-            int c = s_wc[ww * ws + rr];
-            s_wc[ww * ws + rr] = (uint16_t)run;
-            run += c;
-        }
-        if (run != L) s_bad = 1;  // every rank hosts the same number of instances
+    // per-rank exclusive prefix over the 32 warps: one shuffle scan per rank
+#pragma unroll 4
+    for (int rr = w; rr < ws; rr += 32) {
+        const int c = s_wc[rr * 32 + lane];
+        const int inc = warp_inclusive_scan(c);
+        s_wc[rr * 32 + lane] = (uint16_t)(inc - c);
+        if (lane == 31 && inc != L) s_bad = 1;  // every rank hosts the same number of instances
     }
     __syncthreads();
     if (s_bad) {
         update_expert_drop_all(a);
         return;
     }
-    if (t < total) s_inst[t] = r * L + s_wc[w * ws + r] + intra;
+    if (t < total) s_inst[t] = r * L + s_wc[r * 32 + w] + intra;
     __syncthreads();
 
     // 4. every (token, k) copy
@@ -158,7 +168,7 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     for (int u = 0; u < kUeItems; ++u) {
         const int it = t + u * kUeThreads;
         if (it >= items) continue;
-        const int i = it / a.top_k;
+        const int i = (int)div_by_magic((uint32_t)it, a.k_magic);  // it / K
         const int e = pe[u];
         if (e < 0 || e >= E) {
             raise_error(a.err, kDevBadId);
@@ -166,7 +176,9 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
             a.balanced_mask[it] = 0;
             continue;
         }
-        a.balanced_ids[it] = s_inst[s_first[e] + i % s_n[e]];
+        const int ne = s_n[e];
+        const int j = i - ne * (int)div_by_magic((uint32_t)i, s_mag[e]);  // replica i mod n_e
+        a.balanced_ids[it] = s_inst[s_first[e] + j];
         bool keep = pa[u];
         if (a.expert_scales && a.prune_threshold > 0.0f && ps[u] < a.prune_threshold) keep = false;
         a.balanced_mask[it] = keep ? 1 : 0;

@@ -35,7 +35,8 @@
  *     reproducible ("确定性计算" / "Deterministic computation" on each page).
  *   - The workspace must be zeroed once (moe_workspace_init) before its first
  *     use; the error word then accumulates until moe_clear_device_error.
- *     Calls that share a workspace share its error word.
+ *     Calls that share a workspace share its error word.  A workspace of
+ *     MOE_MAX_WORKSPACE_BYTES serves every call.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -66,6 +67,10 @@ typedef enum {
 #define MOE_DEV_BAD_ID    1u  /* an expert / instance id or an expand_idx row out of range */
 #define MOE_DEV_BAD_TABLE 2u  /* mapping table broke its restrictions; every copy was dropped */
 #define MOE_DEV_TIMEOUT   4u  /* a bounded wait for an asynchronous copy gave up; outputs incomplete */
+
+/* The largest workspace any *_workspace_size call reports (bytes): the
+ * 256-byte area that holds the error word. */
+#define MOE_MAX_WORKSPACE_BYTES 256
 
 /* Limits taken from the pages (shape-variable constraints of each page). */
 #define MOE_MAX_BS        512   /* Bs in (0, 512] */
@@ -237,8 +242,9 @@ MOE_API moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const vo
 /* moe_dispatch_noalloc -- moe_dispatch without a caller-provided workspace  */
 /* ------------------------------------------------------------------------ */
 
-/* Largest workspace moe_dispatch_noalloc can stand in for (bytes). */
-#define MOE_NOALLOC_SCRATCH_BYTES 256
+/* Largest workspace moe_dispatch_noalloc can stand in for (bytes): enough for
+ * every moe_dispatch the limits allow. */
+#define MOE_NOALLOC_SCRATCH_BYTES MOE_MAX_WORKSPACE_BYTES
 
 /*
  * The operator pages have no counterpart for this call; it exists for

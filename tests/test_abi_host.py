@@ -72,6 +72,8 @@ def ws_size(L, fn, params):
 def test_workspace_sizes_for_valid_params(L):
     assert ws_size(L, "moe_update_expert_workspace_size", L.UpdateParams(512, 16, 1024, 257, 256, 0.05)) == (0, 256)
     assert ws_size(L, "moe_dispatch_workspace_size", L.DispatchParams(512, 7168, 8, 32, 256, 2)) == (0, 256)
+    assert ws_size(L, "moe_dispatch_workspace_size", L.DispatchParams(512, 8192, 16, 256, 1024, 3)) == (0, 256)
+    assert L.WORKSPACE_BYTES == 256  # the largest any call needs, and the binding's default
     assert ws_size(L, "moe_combine_add_rmsnorm_workspace_size", L.CombineParams(512, 8192, 16, 8192, 1e-6)) == (0, 256)
 
 
