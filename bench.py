@@ -234,29 +234,43 @@ def run_b200(args, rank, world, local_rank):
     alg = algorithmic_bytes(w, n)
 
     # Timed region: CUDA graphs of G steps each, every step = [L2 flush] then
-    # update_expert, dispatch, combine bracketed by timing events recorded as
-    # graph nodes; the flush sits outside the brackets.
+    # update_expert, dispatch and combine between two timing events recorded
+    # as graph nodes; the flush sits outside the bracket.  Nothing separates
+    # the three calls, so each kernel's launch overlaps its predecessor's
+    # tail (programmatic dependent launch), as in a real layer.
+    # A second graph brackets every call with its own events for the per-call
+    # breakdown and the combine kernel's roofline; an event between two calls
+    # ends that overlap, so the three call times add up to more than a step.
     K = args.steps
     G = max(g for g in range(1, 17) if K % g == 0)
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(G)]
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=cap):
-        for s_ in range(G):
-            flush_l2()
-            e = ev[s_]
-            e[0].record()
-            B.update_expert(ids, table, w.ep_world_size, expert_scales=scales, prune_threshold=w.prune_threshold,
-                            workspace=ws, out=(bal, bm))
-            e[1].record()
-            B.dispatch(x, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
-                       workspace=ws, out=d)
-            e[2].record()
-            B.combine_add_rmsnorm(expert_out, d["expand_idx"], scales, residual, gamma, w.norm_eps,
-                                  shared_x=shared, workspace=ws, out=c)
-            e[3].record()
-    graph.replay()  # one untimed replay after capture
+
+    def capture(per_call):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4 if per_call else 2)]
+               for _ in range(G)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for e in evs:
+                flush_l2()
+                e[0].record()
+                B.update_expert(ids, table, w.ep_world_size, expert_scales=scales,
+                                prune_threshold=w.prune_threshold, workspace=ws, out=(bal, bm))
+                if per_call:
+                    e[1].record()
+                B.dispatch(x, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
+                           workspace=ws, out=d)
+                if per_call:
+                    e[2].record()
+                B.combine_add_rmsnorm(expert_out, d["expand_idx"], scales, residual, gamma, w.norm_eps,
+                                      shared_x=shared, workspace=ws, out=c)
+                e[-1].record()
+        return g, evs
+
+    graph, ev_step = capture(False)
+    graph_ops, ev_ops = capture(True)
+    for g in (graph, graph_ops):
+        g.replay()  # one untimed replay after capture
     torch.cuda.synchronize()
     sums = [0.0, 0.0, 0.0, 0.0]
     barrier()
@@ -265,13 +279,19 @@ def run_b200(args, rank, world, local_rank):
         for _ in range(K // G):
             graph.replay()
             torch.cuda.synchronize()
-            for e in ev:
-                sums[0] += e[0].elapsed_time(e[3])
+            for e in ev_step:
+                sums[0] += e[0].elapsed_time(e[1])
+        barrier()
+        torch.cuda.synchronize()
+        for _ in range(K // G):
+            graph_ops.replay()
+            torch.cuda.synchronize()
+            for e in ev_ops:
                 sums[1] += e[0].elapsed_time(e[1])
                 sums[2] += e[1].elapsed_time(e[2])
                 sums[3] += e[2].elapsed_time(e[3])
     barrier()
-    del graph
+    del graph, graph_ops
     assert B.read_device_error(ws) == 0, "device error during the timed steps"
     t_step, t_upd, t_disp, t_comb = reduce_over_ranks([v / K for v in sums], "max")
     value = world * w.bs / (t_step * 1e-3)
@@ -338,7 +358,8 @@ def run_b200(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "pinned host activations -> device, the three calls, y -> host; layer parameters resident"},
         "gpu_launches": 4 * K,  # update_expert, route, quantize-and-scatter, combine
-        "timing": f"CUDA graphs of {G} steps; per-op CUDA events recorded as graph nodes",
+        "timing": (f"CUDA graphs of {G} steps, events at each step's ends; breakdown_us from a second graph "
+                   "with events between the calls (no launch overlap there, so its parts sum above a step)"),
         "clocks": clk.summary(),
     }
     return out, w

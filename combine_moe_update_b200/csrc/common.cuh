@@ -224,10 +224,12 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
     return v;
 }
 
+// Max over the 32 lanes of a full warp in one instruction (sm_100a's
+// floating-point redux; NaN inputs are ignored, as fmaxf ignores them).
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-    return v;
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -18,9 +18,9 @@
 //   row is loaded, quantized once (all K copies are identical) and written K
 //   times.
 // dispatch_token_smooth_kernel<MODE>  smooth scales (modes 2, 3): one block
-//   per token; the row and the K instance ids are loaded once and each
-//   copy's smooth row is loaded one copy ahead, so memory latency overlaps
-//   the per-copy reduction and quantization.
+//   per token; the row and the K instance ids are loaded once; each copy's
+//   smooth row arrives in shared memory by a bulk asynchronous copy, so
+//   four blocks fit on an SM and a decode batch runs in one wave.
 //
 // Quantization, per mode ("计算公式" cases 1, 3, 4, 5):
 //   0  copy the bf16 row;
@@ -197,17 +197,17 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
 
 // ------------------------------------------------------------ quantizers ---
 
-constexpr int kDpThreads = 256;  // the most threads a token block runs
-constexpr int kDpWarps = kDpThreads / 32;
 constexpr int kDpVecs = 4;  // 8-element vectors per thread: H / 8 <= 1024 = 256 * 4
 
-// Threads of a token block for rows of V 8-element vectors: the fewest whole
-// warps that cover the row with kDpVecs vectors each, so that every warp has
-// the same number of vectors when 32 * kDpVecs divides V (H = 7168: 224
-// threads of 4 vectors, none idle at the per-row barrier).
+// Threads of a token block for rows of V 8-element vectors: the fewest
+// threads, from a fixed set of block sizes, that cover the row with kDpVecs
+// vectors each.  H = 7168 (V = 896) takes 224 threads, every one with 4
+// vectors, so no warp idles at a per-row barrier.  The block size is a
+// template parameter of the kernels, which makes every vector's offset a
+// compile-time constant.
 __host__ __device__ inline int dp_threads(int V) {
-    const int per = (V + kDpVecs - 1) / kDpVecs;
-    return ((per + 31) / 32) * 32;
+    const int need = ((V + kDpVecs - 1) / kDpVecs + 31) / 32 * 32;
+    return need <= 64 ? 64 : need <= 128 ? 128 : need <= 192 ? 192 : need <= 224 ? 224 : 256;
 }
 
 // int8 codes of 8 values (4 fp32 pairs) for a finite multiplier dyn.
@@ -250,8 +250,7 @@ __device__ __forceinline__ uint2 int8x8_inf(const uint64_t (&v)[4]) {
 }
 
 // Codes of this thread's vectors for a multiplier dyn shared by the whole
-// block (or warp).  The rare dyn = +inf case is a separate branch over all
-// vectors, so the common case runs only int8x8 and never pays for both.
+// block.  The rare dyn = +inf case is a separate branch over all vectors.
 __device__ __forceinline__ void int8_vecs(const uint64_t (&v)[kDpVecs][4], float dyn, uint2 (&qv)[kDpVecs]) {
     if (__builtin_expect(isinf(dyn), 0)) {
 #pragma unroll
@@ -262,11 +261,18 @@ __device__ __forceinline__ void int8_vecs(const uint64_t (&v)[kDpVecs][4], float
     }
 }
 
+// max |v| of 8 values, as a balanced tree (3 dependent steps, not 8).
 __device__ __forceinline__ float abs_max8(const uint64_t (&v)[4]) {
-    float m = 0.0f;
+    float m[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) m = fmaxf(m, fmaxf(fabsf(f2_lo(v[q])), fabsf(f2_hi(v[q]))));
-    return m;
+    for (int q = 0; q < 4; ++q) m[q] = fmaxf(fabsf(f2_lo(v[q])), fabsf(f2_hi(v[q])));
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// max |v| over this thread's vectors (vectors past the row's end hold 0).
+__device__ __forceinline__ float abs_max_vecs(const uint64_t (&v)[kDpVecs][4]) {
+    static_assert(kDpVecs == 4, "the tree below covers four vectors");
+    return fmaxf(fmaxf(abs_max8(v[0]), abs_max8(v[1])), fmaxf(abs_max8(v[2]), abs_max8(v[3])));
 }
 
 // 8 bf16 -> 4 fp32 pairs (exact).
@@ -303,38 +309,36 @@ __device__ __forceinline__ uint2 e4m3x8(const uint64_t (&v)[4], int se) {
     return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
-// Block-wide max of m; thread 0 turns it into dyn = 127 / max and
-// scale = 1 / dyn, which every thread reads back.  Two barriers.
-__device__ __forceinline__ float2 block_dyn(float m, float *s_red, float *s_out) {
+// max over the NW per-warp partials in shared memory, as a tree.
+template <int NW>
+__device__ __forceinline__ float max_partials(const float *s_red) {
+    float v[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) v[w] = s_red[w];
+#pragma unroll
+    for (int span = 1; span < NW; span *= 2)
+#pragma unroll
+        for (int w = 0; w + span < NW; w += 2 * span) v[w] = fmaxf(v[w], v[w + span]);
+    return v[0];
+}
+
+// Block-wide max of m; every thread turns it into dyn = 127 / max.  One
+// barrier; s_red must not be reused before the next barrier.
+template <int NT>
+__device__ __forceinline__ float block_dyn(float m, float *s_red) {
     m = warp_max(m);
     if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        float r = s_red[0];
-#pragma unroll
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, s_red[w]);
-        const float dyn = __fdiv_rn(127.0f, r);  // +inf when r == 0 or 127 / r overflows
-        s_out[0] = dyn;
-        s_out[1] = __frcp_rn(dyn);               // 1 / dynamicScales
-    }
-    __syncthreads();
-    return make_float2(s_out[0], s_out[1]);
+    return __fdiv_rn(127.0f, max_partials<NT / 32>(s_red));  // +inf when the max is 0 or 127 / max overflows
 }
 
-// Quantize this thread's vectors of one row (xf: fp32 pairs, x * smooth
-// already applied).  Fills the codes and the scales this thread writes.
-template <int MODE>
-__device__ __forceinline__ void quantize_vecs(const uint64_t (&xf)[kDpVecs][4], int V, float *s_red, float *s_out,
-                                              uint2 (&qv)[kDpVecs], float (&seg)[kDpVecs], float &row_scale) {
+// Quantize this thread's vectors of one row for the modes without a
+// block-wide reduction (xf: fp32 pairs, x * smooth already applied).
+template <int MODE, int NT>
+__device__ __forceinline__ void quantize_local(const uint64_t (&xf)[kDpVecs][4], int V, uint2 (&qv)[kDpVecs],
+                                               float (&seg)[kDpVecs]) {
     const int t = threadIdx.x;
-    if constexpr (MODE == 2) {
-        float m = 0.0f;
-#pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) m = fmaxf(m, abs_max8(xf[q]));
-        const float2 ds = block_dyn(m, s_red, s_out);
-        row_scale = ds.y;
-        int8_vecs(xf, ds.x, qv);
-    } else if constexpr (MODE == 3) {
+    if constexpr (MODE == 3) {
         float dq[kDpVecs];
 #pragma unroll
         for (int q = 0; q < kDpVecs; ++q) {  // a 128-element tile = 16 vectors = 16 consecutive lanes
@@ -343,7 +347,7 @@ __device__ __forceinline__ void quantize_vecs(const uint64_t (&xf)[kDpVecs][4], 
             m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
             m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
             m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
-            const bool lead = (t & 15) == 0 && t + q * (int)blockDim.x < V;
+            const bool lead = (t & 15) == 0 && t + q * NT < V;
             float dyn = 0.0f;
             if (lead) dyn = __fdiv_rn(127.0f, m);  // one division per tile
             dyn = __shfl_sync(kFull, dyn, (t & 31) & ~15);
@@ -376,14 +380,14 @@ __device__ __forceinline__ void quantize_vecs(const uint64_t (&xf)[kDpVecs][4], 
 }
 
 // Write this thread's codes (and scales) of one row.
-template <int MODE>
+template <int MODE, int NT>
 __device__ __forceinline__ void write_row(const DispatchArgs &a, int row, int V, const uint2 (&qv)[kDpVecs],
                                           const float (&seg)[kDpVecs], float row_scale) {
-    const int t = threadIdx.x, H = a.hidden, nt = blockDim.x;
+    const int t = threadIdx.x, H = a.hidden;
     uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
 #pragma unroll
     for (int q = 0; q < kDpVecs; ++q) {
-        const int p = t + q * nt;
+        const int p = t + q * NT;
         if (p >= V) continue;
         *reinterpret_cast<uint2 *>(dst + p * 8) = qv[q];
         if constexpr (MODE == 3) {
@@ -400,23 +404,28 @@ __device__ __forceinline__ void write_row(const DispatchArgs &a, int row, int V,
     }
 }
 
+// This thread's vectors of a bf16 row (zeros past the row's end).
+template <int NT>
+__device__ __forceinline__ void load_row(const uint16_t *row, int V, uint4 (&xv)[kDpVecs]) {
+#pragma unroll
+    for (int q = 0; q < kDpVecs; ++q) {
+        const int p = threadIdx.x + q * NT;
+        xv[q] = p < V ? ld_stream(row + p * 8) : make_uint4(0, 0, 0, 0);
+    }
+}
+
 // --------------------------------------------------------- token kernel ---
 
-template <int MODE>
-__global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs a) {
-    __shared__ float s_red[kDpWarps], s_out[2];
+template <int MODE, int NT>
+__global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
+    __shared__ float s_red[NT / 32];
     __shared__ int s_row[16];
-    const int i = blockIdx.x, t = threadIdx.x, nt = blockDim.x;
+    const int i = blockIdx.x, t = threadIdx.x;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
 
     // inputs of the call only: safe before the route kernel is done
-    const uint16_t *xrow = a.x + (size_t)i * H;
     uint4 xv[kDpVecs];
-#pragma unroll
-    for (int q = 0; q < kDpVecs; ++q) {
-        const int p = t + q * nt;
-        xv[q] = p < V ? ld_stream(xrow + p * 8) : make_uint4(0, 0, 0, 0);
-    }
+    load_row<NT>(a.x + (size_t)i * H, V, xv);
     uint2 qv[kDpVecs];
     float seg[kDpVecs] = {0.0f, 0.0f, 0.0f, 0.0f};
     float row_scale = 0.0f;
@@ -424,7 +433,13 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs
         uint64_t xf[kDpVecs][4];
 #pragma unroll
         for (int q = 0; q < kDpVecs; ++q) vec_to_f2(xv[q], xf[q]);
-        quantize_vecs<MODE>(xf, V, s_red, s_out, qv, seg, row_scale);
+        if constexpr (MODE == 2) {
+            const float dyn = block_dyn<NT>(abs_max_vecs(xf), s_red);
+            row_scale = __frcp_rn(dyn);  // 1 / dynamicScales
+            int8_vecs(xf, dyn, qv);
+        } else {
+            quantize_local<MODE, NT>(xf, V, qv, seg);
+        }
     }
 
     pdl_wait();  // the rows come from route_kernel
@@ -437,109 +452,120 @@ __global__ void __launch_bounds__(kDpThreads) dispatch_token_kernel(DispatchArgs
             uint16_t *dst = reinterpret_cast<uint16_t *>(a.expand_x) + (size_t)row * H;
 #pragma unroll
             for (int q = 0; q < kDpVecs; ++q) {
-                const int p = t + q * nt;
+                const int p = t + q * NT;
                 if (p < V) st_v4(dst + p * 8, xv[q]);
             }
         } else {
-            write_row<MODE>(a, row, V, qv, seg, row_scale);
+            write_row<MODE, NT>(a, row, V, qv, seg, row_scale);
         }
     }
 }
 
 // -------------------------------------------------- token smooth kernel ---
 //
-// Smooth scales (modes 2, 3), one block per token: the token's row and its K
-// instance ids are loaded once; copy k's smooth row is loaded one copy ahead
-// (while copy k - 1 reduces and quantizes), so the per-copy memory latency
-// overlaps compute.  The block waits for the route only before its first
-// row write.
+// Smooth scales (modes 2, 3), one block per token.  The token's row stays in
+// registers; warp 0 lists the token's sent copies.  Each copy's smooth row
+// (H fp32) is brought into shared memory by one bulk asynchronous copy
+// issued as soon as every thread has read the previous row, so no registers
+// hold rows in flight: the block stays small enough (at most 72 registers a
+// thread at 224 threads) for four blocks per SM, so a 512-token batch runs
+// in a single wave with the other blocks covering each one's waits.
+//
+// Per copy: wait for the smooth row; xFp32 = x * smooth; mode 2 publishes
+// each warp's partial max and takes one barrier (which also frees the
+// shared row for the next copy's load), then every thread finishes the max,
+// dyn = 127 / max and the codes; mode 3's reductions stay within 16 lanes.
 
-template <int MODE>
-__global__ void __launch_bounds__(kDpThreads, 2) dispatch_token_smooth_kernel(DispatchArgs a) {
-    __shared__ float s_red[2][kDpWarps];
-    __shared__ int s_key[16], s_row[16];
-    const int i = blockIdx.x, t = threadIdx.x, nt = blockDim.x, nw = nt >> 5;
+inline size_t smooth_smem_bytes(int hidden) { return (size_t)hidden * sizeof(float); }
+
+template <int MODE, int NT>
+__global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_kernel(DispatchArgs a) {
+    constexpr int NW = NT / 32;
+    extern __shared__ __align__(128) float s_smooth[];  // [H]: the current copy's smooth row
+    __shared__ float s_red[2][NW];
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ int s_key[16], s_pos[16], s_row[16], s_ns;
+    const int i = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
+    const uint32_t row_bytes = (uint32_t)H * sizeof(float);  // a multiple of 16 (H % 16 == 0)
 
     // inputs of the call only: safe before the route kernel is done
-    const uint16_t *xrow = a.x + (size_t)i * H;
     uint4 xv[kDpVecs];
-#pragma unroll
-    for (int q = 0; q < kDpVecs; ++q) {
-        const int p = t + q * nt;
-        xv[q] = p < V ? ld_stream(xrow + p * 8) : make_uint4(0, 0, 0, 0);
-    }
-    if (t < K) s_key[t] = copy_key(a, i * K + t);
-    __syncthreads();
-
-    auto load_smooth = [&](int e, float4 (&sv)[kDpVecs][2]) {
-        const float *srow = a.smooth + (size_t)e * H;
-#pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {
-            const int p = t + q * nt;
-            if (p < V) {
-                sv[q][0] = __ldg(reinterpret_cast<const float4 *>(srow + p * 8));
-                sv[q][1] = __ldg(reinterpret_cast<const float4 *>(srow + p * 8) + 1);
-            } else {
-                sv[q][0] = sv[q][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+    load_row<NT>(a.x + (size_t)i * H, V, xv);
+    if (w == 0) {  // the sent copies, in k order: instance and position k
+        const int key = lane < K ? copy_key(a, i * K + lane) : -1;
+        const unsigned sent = __ballot_sync(kFull, key >= 0);
+        if (key >= 0) {
+            const int c = __popc(sent & ((1u << lane) - 1u));
+            s_key[c] = key;
+            s_pos[c] = lane;
         }
+        if (lane == 0) {
+            s_ns = __popc(sent);
+            mbar_init(&s_bar, 1);
+        }
+    }
+    __syncthreads();
+    const int ns = s_ns;
+    auto fetch_smooth = [&](int c) {  // thread 0 only
+        mbar_arrive_expect_tx(&s_bar, row_bytes);
+        bulk_copy_g2s(s_smooth, a.smooth + (size_t)s_key[c] * H, row_bytes, &s_bar);
     };
-    auto next_sent = [&](int k) {  // first copy >= k that is sent, or K
-        while (k < K && s_key[k] < 0) ++k;
-        return k;
-    };
+    if (t == 0 && ns > 0) fetch_smooth(0);
 
-    float4 sn[kDpVecs][2];
-    int k = next_sent(0);
-    if (k < K) load_smooth(s_key[k], sn);
-    bool waited = false;
-    int par = 0;
-    while (k < K) {  // uniform over the block
+    for (int c = 0; c < ns; ++c) {
+        const bool landed = mbar_wait_bounded(&s_bar, c & 1);
         uint64_t xf[kDpVecs][4];
-        float m = 0.0f;
 #pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) {
+        for (int q = 0; q < kDpVecs; ++q) {  // xFp32 = x * smooth (0 past the row's end)
+            const int p = t + q * NT;
             uint64_t f[4];
             vec_to_f2(xv[q], f);
-            xf[q][0] = f2_mul(f[0], f2_pack(sn[q][0].x, sn[q][0].y));  // xFp32 = x * smooth
-            xf[q][1] = f2_mul(f[1], f2_pack(sn[q][0].z, sn[q][0].w));
-            xf[q][2] = f2_mul(f[2], f2_pack(sn[q][1].x, sn[q][1].y));
-            xf[q][3] = f2_mul(f[3], f2_pack(sn[q][1].z, sn[q][1].w));
+            float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+            if (p < V) {
+                s0 = reinterpret_cast<const float4 *>(s_smooth + p * 8)[0];
+                s1 = reinterpret_cast<const float4 *>(s_smooth + p * 8)[1];
+            }
+            xf[q][0] = f2_mul(f[0], f2_pack(s0.x, s0.y));
+            xf[q][1] = f2_mul(f[1], f2_pack(s0.z, s0.w));
+            xf[q][2] = f2_mul(f[2], f2_pack(s1.x, s1.y));
+            xf[q][3] = f2_mul(f[3], f2_pack(s1.z, s1.w));
         }
-        const int kn = next_sent(k + 1);
-        if (kn < K) load_smooth(s_key[kn], sn);  // the next copy's smooth row, in flight during this one
-
         uint2 qv[kDpVecs];
         float seg[kDpVecs] = {0.0f, 0.0f, 0.0f, 0.0f};
         float row_scale = 0.0f;
         if constexpr (MODE == 2) {
-#pragma unroll
-            for (int q = 0; q < kDpVecs; ++q) m = fmaxf(m, abs_max8(xf[q]));
-            // one barrier per copy: partials in alternating buffers, every thread
-            // finishes the max and the division itself
-            m = warp_max(m);
-            if ((t & 31) == 0) s_red[par][t >> 5] = m;
-            __syncthreads();
-            float r = s_red[par][0];
-#pragma unroll
-            for (int w = 1; w < nw; ++w) r = fmaxf(r, s_red[par][w]);
-            par ^= 1;
-            const float dyn = __fdiv_rn(127.0f, r);  // +inf when r == 0 or 127 / r overflows
-            if (t == 0) row_scale = __frcp_rn(dyn);
+            const float m = warp_max(abs_max_vecs(xf));
+            if (lane == 0) s_red[c & 1][w] = m;
+        }
+        // every thread has read the smooth row (and published its partial):
+        // the buffer may be refilled.  A row that never landed stops the
+        // block (the same verdict in every thread) once a second bounded
+        // wait has given the copy in flight its chance to finish.
+        if (__syncthreads_or(!landed)) {
+            if (t == 0) {
+                raise_error(a.err, kDevTimeout);
+                mbar_wait_bounded(&s_bar, c & 1);
+            }
+            return;
+        }
+        if (t == 0 && c + 1 < ns) {
+            fence_proxy_async_smem();
+            fetch_smooth(c + 1);
+        }
+        if constexpr (MODE == 2) {
+            const float dyn = __fdiv_rn(127.0f, max_partials<NW>(s_red[c & 1]));  // +inf when the max is 0
+            row_scale = __frcp_rn(dyn);                                           // or 127 / max overflows
             int8_vecs(xf, dyn, qv);
         } else {
-            quantize_vecs<MODE>(xf, V, nullptr, nullptr, qv, seg, row_scale);
+            quantize_local<MODE, NT>(xf, V, qv, seg);
         }
-
-        if (!waited) {
+        if (c == 0) {
             pdl_wait();  // the rows come from the route kernel
             if (t < K) s_row[t] = a.expand_idx[i * K + t];
             __syncthreads();
-            waited = true;
         }
-        write_row<MODE>(a, s_row[k], V, qv, seg, row_scale);
-        k = kn;
+        write_row<MODE, NT>(a, s_row[s_pos[c]], V, qv, seg, row_scale);
     }
 }
 

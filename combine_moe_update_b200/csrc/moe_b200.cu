@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "combine.cuh"
 #include "common.cuh"
@@ -27,21 +28,34 @@ bool check_workspace(const void *ws, size_t bytes) {
     return ws != nullptr && aligned(ws, 16) && bytes >= kWorkspaceBytes;
 }
 
-// Opt a kernel into more than 48 KB of dynamic shared memory on the current
-// device (cached per device and kernel).
-template <typename Kernel>
-bool ensure_smem(Kernel k, size_t bytes, int slot) {
-    static int done[64][48];
+// Opt a kernel into more than 48 KB of dynamic shared memory and the largest
+// shared-memory carveout on the current device, once per (kernel, device).
+bool ensure_smem_fn(const void *fn, size_t bytes) {
+    struct Done {
+        const void *fn;
+        int dev;
+        size_t bytes;
+    };
+    static std::mutex mu;
+    static Done done[512];
+    static int n_done = 0;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 48) return false;
-    if (done[dev][slot] >= (int)bytes + 1) return true;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int j = 0; j < n_done; ++j)
+        if (done[j].fn == fn && done[j].dev == dev && done[j].bytes >= bytes) return true;
     if (bytes > 48 * 1024 &&
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return false;
     // prefer the largest shared-memory carveout, so occupancy is not capped by it
-    if (cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return false;
-    done[dev][slot] = (int)bytes + 1;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return false;
+    if (n_done < 512) done[n_done++] = Done{fn, dev, bytes};
     return true;
+}
+
+template <typename Kernel>
+bool ensure_smem(Kernel k, size_t bytes) {
+    return ensure_smem_fn(reinterpret_cast<const void *>(k), bytes);
 }
 
 // --- parameter checks: the limits of each page's shape-variable section ---
@@ -101,35 +115,64 @@ cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t smem, c
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Token kernels are compiled for a few block sizes (dp_threads); pick the
+// one for this row length.
+template <int MODE, template <int, int> class Sel>
+cudaError_t launch_by_threads(const moe::DispatchArgs &a, cudaStream_t s) {
+    switch (moe::dp_threads(a.hidden >> 3)) {
+        case 64: return Sel<MODE, 64>::go(a, s);
+        case 128: return Sel<MODE, 128>::go(a, s);
+        case 192: return Sel<MODE, 192>::go(a, s);
+        case 224: return Sel<MODE, 224>::go(a, s);
+        default: return Sel<MODE, 256>::go(a, s);
+    }
+}
+
+template <int MODE, int NT>
+struct TokenLaunch {
+    static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
+        auto kernel = moe::dispatch_token_kernel<MODE, NT>;
+        if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
+        return launch(kernel, a.bs, NT, 0, s, a);
+    }
+};
+
+template <int MODE, int NT>
+struct TokenSmoothLaunch {
+    static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
+        auto kernel = moe::dispatch_token_smooth_kernel<MODE, NT>;
+        const size_t smem = moe::smooth_smem_bytes(a.hidden);
+        if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
+        return launch(kernel, a.bs, NT, smem, s, a);
+    }
+};
+
 template <int MODE>
 cudaError_t launch_dispatch_token(const moe::DispatchArgs &a, cudaStream_t s) {
-    if (!ensure_smem(moe::dispatch_token_kernel<MODE>, 0, 1 + MODE)) return cudaErrorInvalidValue;
-    return launch(moe::dispatch_token_kernel<MODE>, a.bs, moe::dp_threads(a.hidden >> 3), 0, s, a);
+    return launch_by_threads<MODE, TokenLaunch>(a, s);
 }
 
 template <int MODE>
 cudaError_t launch_dispatch_token_smooth(const moe::DispatchArgs &a, cudaStream_t s) {
-    if (!ensure_smem(moe::dispatch_token_smooth_kernel<MODE>, 0, 8 + MODE)) return cudaErrorInvalidValue;
-    return launch(moe::dispatch_token_smooth_kernel<MODE>, a.bs, moe::dp_threads(a.hidden >> 3), 0, s, a);
+    return launch_by_threads<MODE, TokenSmoothLaunch>(a, s);
 }
 
 // combine: a cluster of two 128-thread blocks per token (one per half row);
 // VECS = ceil(H / 16 / 128) vectors per thread.
 template <int KMAX, bool SHARED, int VECS>
-cudaError_t launch_combine_v(const moe::CombineArgs &a, cudaStream_t s, int slot) {
+cudaError_t launch_combine_v(const moe::CombineArgs &a, cudaStream_t s) {
     auto kernel = moe::combine_kernel<KMAX, SHARED, VECS>;
-    if (!ensure_smem(kernel, 0, slot)) return cudaErrorInvalidValue;
+    if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
     return launch(kernel, 2 * a.bs, moe::kCbThreads, 0, s, a);
 }
 
 template <int KMAX, bool SHARED>
 cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
     const int vecs = ((a.hidden / 8 + 1) / 2 + moe::kCbThreads - 1) / moe::kCbThreads;  // 1..4
-    const int slot = 12 + ((KMAX / 8) * 2 + (SHARED ? 1 : 0)) * 4;
-    if (vecs <= 1) return launch_combine_v<KMAX, SHARED, 1>(a, s, slot);
-    if (vecs <= 2) return launch_combine_v<KMAX, SHARED, 2>(a, s, slot + 1);
-    if (vecs <= 3) return launch_combine_v<KMAX, SHARED, 3>(a, s, slot + 2);
-    return launch_combine_v<KMAX, SHARED, 4>(a, s, slot + 3);
+    if (vecs <= 1) return launch_combine_v<KMAX, SHARED, 1>(a, s);
+    if (vecs <= 2) return launch_combine_v<KMAX, SHARED, 2>(a, s);
+    if (vecs <= 3) return launch_combine_v<KMAX, SHARED, 3>(a, s);
+    return launch_combine_v<KMAX, SHARED, 4>(a, s);
 }
 
 template <int KMAX>
@@ -208,7 +251,7 @@ moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_i
     a.balanced_mask = balanced_mask;
     a.err = reinterpret_cast<uint32_t *>(workspace);
     const size_t smem = moe::update_expert_smem_bytes(p->ep_world_size);
-    if (!ensure_smem(moe::update_expert_kernel, smem, 0)) return MOE_ERR_CUDA;
+    if (!ensure_smem(moe::update_expert_kernel, smem)) return MOE_ERR_CUDA;
     return launch(moe::update_expert_kernel, 1, moe::kUeThreads, smem, as_stream(cuda_stream), a) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
@@ -264,7 +307,7 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
 
     const int slices = moe::route_slices(p->bs * p->top_k);
     const size_t rsmem = moe::route_smem_bytes(p->num_instances);
-    if (!ensure_smem(moe::route_kernel, rsmem, 11)) return MOE_ERR_CUDA;
+    if (!ensure_smem(moe::route_kernel, rsmem)) return MOE_ERR_CUDA;
     if (launch(moe::route_kernel, slices, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     if (smooth_scales) {
