@@ -90,8 +90,6 @@ inline size_t route_smem_bytes(int num_instances) {
 }
 
 __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
-    pdl_wait();               // the instance ids may come from the previous kernel
-    pdl_launch_dependents();  // the scatter kernel may start its input-only work now
     extern __shared__ __align__(16) unsigned char smem_r[];
     const int E = a.num_instances, N = a.bs * a.top_k, g = blockIdx.x;
     uint16_t *s_cnt = reinterpret_cast<uint16_t *>(smem_r);                                  // [E][16]
@@ -101,6 +99,14 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
     __shared__ int s_warp[32];
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int mine0 = g * kRtThreads;  // first copy of this slice
+
+    // shared-memory counters cleared while the previous kernel may still run
+    uint32_t *cnt32 = reinterpret_cast<uint32_t *>(s_cnt);
+    for (int q = t; q < 8 * E; q += kRtThreads) cnt32[q] = 0;  // E * 16 uint16
+    for (int q = t; q < 2 * E; q += kRtThreads) s_all[q] = 0;  // s_all and s_before
+    __syncthreads();
+    pdl_wait();               // the instance ids may come from the previous kernel
+    pdl_launch_dependents();  // the scatter kernel may start its input-only work now
 
     // every copy's key (for the histograms) and this thread's own copy; the
     // loads are unconditional (indices clamped into range) so that all of
@@ -130,10 +136,6 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
         raise_error(a.err, kDevBadId);
         k = -1;
     }
-    uint32_t *cnt32 = reinterpret_cast<uint32_t *>(s_cnt);
-    for (int q = t; q < 8 * E; q += kRtThreads) cnt32[q] = 0;  // E * 16 uint16
-    for (int q = t; q < 2 * E; q += kRtThreads) s_all[q] = 0;  // s_all and s_before
-    __syncthreads();
 
 #pragma unroll
     for (int u = 0; u < kRtKeys; ++u) {
@@ -218,19 +220,17 @@ __host__ __device__ inline int dp_threads(int V) {
 // in [-127, 127] and the clamp to that range is never active.
 //
 // The product must be rounded to fp32 on its own before the add (the page's
-// quantOut = CastToInt8(xFp32 * dynamicScales) rounds it).  A packed multiply
-// followed by a packed add may be contracted into one fused multiply-add,
-// which skips that rounding and breaks ties such as a product that rounds to
-// exactly 63.5; the scalar round-to-nearest multiply is never contracted.
+// quantOut = CastToInt8(xFp32 * dynamicScales) rounds it).  Scalar
+// round-to-nearest intrinsics are never contracted into a fused multiply-add
+// (which would skip that rounding and break ties such as a product that
+// rounds to exactly 63.5), and unlike packed pairs they need no register
+// pairing moves.
 __device__ __forceinline__ uint2 int8x8(const uint64_t (&v)[4], float dyn) {
-    const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
     uint32_t b[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const uint64_t prod = f2_pack(__fmul_rn(f2_lo(v[q]), dyn), __fmul_rn(f2_hi(v[q]), dyn));
-        const uint64_t r = f2_add(prod, magic);
-        b[2 * q] = __float_as_uint(f2_lo(r));
-        b[2 * q + 1] = __float_as_uint(f2_hi(r));
+        b[2 * q] = __float_as_uint(__fadd_rn(__fmul_rn(f2_lo(v[q]), dyn), 12582912.0f));
+        b[2 * q + 1] = __float_as_uint(__fadd_rn(__fmul_rn(f2_hi(v[q]), dyn), 12582912.0f));
     }
     const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
@@ -476,12 +476,18 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
 // shared row for the next copy's load), then every thread finishes the max,
 // dyn = 127 / max and the codes; mode 3's reductions stay within 16 lanes.
 
-inline size_t smooth_smem_bytes(int hidden) { return (size_t)hidden * sizeof(float); }
+// The shared smooth row, padded to the NT * kDpVecs vectors the threads
+// cover, so that every thread reads all its vectors without a bound check;
+// the padding is zeroed once and no copy writes it (x is 0 there too).
+template <int NT>
+__host__ __device__ inline int smooth_smem_floats(int hidden) {
+    return hidden > NT * kDpVecs * 8 ? hidden : NT * kDpVecs * 8;
+}
 
 template <int MODE, int NT>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_kernel(DispatchArgs a) {
     constexpr int NW = NT / 32;
-    extern __shared__ __align__(128) float s_smooth[];  // [H]: the current copy's smooth row
+    extern __shared__ __align__(128) float s_smooth[];  // the current copy's smooth row, then zeros
     __shared__ float s_red[2][NW];
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_key[16], s_pos[16], s_row[16], s_ns;
@@ -489,9 +495,20 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
     const int H = a.hidden, V = H >> 3, K = a.top_k;
     const uint32_t row_bytes = (uint32_t)H * sizeof(float);  // a multiple of 16 (H % 16 == 0)
 
+    // Shared-memory banks: a 16-byte read per lane at a 32-byte lane stride
+    // would put two lanes of each quarter-warp on the same banks.  Lanes
+    // with bit 2 set therefore hold their vectors' two 4-element halves
+    // swapped (x here, the smooth halves at the reads, the codes back at the
+    // writes), so each quarter-warp's reads cover all 32 banks once.
+    const bool swap = (lane >> 2) & 1;
     // inputs of the call only: safe before the route kernel is done
     uint4 xv[kDpVecs];
     load_row<NT>(a.x + (size_t)i * H, V, xv);
+#pragma unroll
+    for (int q = 0; q < kDpVecs; ++q)
+        if (swap) xv[q] = make_uint4(xv[q].z, xv[q].w, xv[q].x, xv[q].y);
+    const float *s_first = s_smooth + (swap ? 4 : 0), *s_second = s_smooth + (swap ? 0 : 4);
+    for (int e = H + t; e < smooth_smem_floats<NT>(H); e += NT) s_smooth[e] = 0.0f;
     if (w == 0) {  // the sent copies, in k order: instance and position k
         const int key = lane < K ? copy_key(a, i * K + lane) : -1;
         const unsigned sent = __ballot_sync(kFull, key >= 0);
@@ -521,11 +538,8 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
             const int p = t + q * NT;
             uint64_t f[4];
             vec_to_f2(xv[q], f);
-            float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
-            if (p < V) {
-                s0 = reinterpret_cast<const float4 *>(s_smooth + p * 8)[0];
-                s1 = reinterpret_cast<const float4 *>(s_smooth + p * 8)[1];
-            }
+            const float4 s0 = *reinterpret_cast<const float4 *>(s_first + p * 8);
+            const float4 s1 = *reinterpret_cast<const float4 *>(s_second + p * 8);
             xf[q][0] = f2_mul(f[0], f2_pack(s0.x, s0.y));
             xf[q][1] = f2_mul(f[1], f2_pack(s0.z, s0.w));
             xf[q][2] = f2_mul(f[2], f2_pack(s1.x, s1.y));
@@ -553,6 +567,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
             fence_proxy_async_smem();
             fetch_smooth(c + 1);
         }
+        if (c + 1 == ns) pdl_launch_dependents();  // the next kernel may be scheduled as blocks finish
         if constexpr (MODE == 2) {
             const float dyn = __fdiv_rn(127.0f, max_partials<NW>(s_red[c & 1]));  // +inf when the max is 0
             row_scale = __frcp_rn(dyn);                                           // or 127 / max overflows
@@ -565,6 +580,9 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
             if (t < K) s_row[t] = a.expand_idx[i * K + t];
             __syncthreads();
         }
+#pragma unroll
+        for (int q = 0; q < kDpVecs; ++q)
+            if (swap) qv[q] = make_uint2(qv[q].y, qv[q].x);
         write_row<MODE, NT>(a, s_row[s_pos[c]], V, qv, seg, row_scale);
     }
 }

@@ -28,8 +28,9 @@ bool check_workspace(const void *ws, size_t bytes) {
     return ws != nullptr && aligned(ws, 16) && bytes >= kWorkspaceBytes;
 }
 
-// Opt a kernel into more than 48 KB of dynamic shared memory and the largest
-// shared-memory carveout on the current device, once per (kernel, device).
+// Allow a kernel its dynamic shared memory (beyond 48 KB needs the opt-in)
+// and the largest shared-memory carveout on the current device, once per
+// (kernel, device).
 bool ensure_smem_fn(const void *fn, size_t bytes) {
     struct Done {
         const void *fn;
@@ -44,8 +45,7 @@ bool ensure_smem_fn(const void *fn, size_t bytes) {
     std::lock_guard<std::mutex> lock(mu);
     for (int j = 0; j < n_done; ++j)
         if (done[j].fn == fn && done[j].dev == dev && done[j].bytes >= bytes) return true;
-    if (bytes > 48 * 1024 &&
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+    if (bytes > 0 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return false;
     // prefer the largest shared-memory carveout, so occupancy is not capped by it
     if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return false;
@@ -141,7 +141,7 @@ template <int MODE, int NT>
 struct TokenSmoothLaunch {
     static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
         auto kernel = moe::dispatch_token_smooth_kernel<MODE, NT>;
-        const size_t smem = moe::smooth_smem_bytes(a.hidden);
+        const size_t smem = (size_t)moe::smooth_smem_floats<NT>(a.hidden) * sizeof(float);
         if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
         return launch(kernel, a.bs, NT, smem, s, a);
     }
