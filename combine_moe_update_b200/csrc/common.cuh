@@ -118,13 +118,13 @@ __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
     return d;
 }
 __device__ __forceinline__ float f2_lo(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    float lo;
+    asm("{\n\t.reg .f32 hi;\n\tmov.b64 {%0, hi}, %1;\n\t}" : "=f"(lo) : "l"(v));
     return lo;
 }
 __device__ __forceinline__ float f2_hi(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    float hi;
+    asm("{\n\t.reg .f32 lo;\n\tmov.b64 {lo, %0}, %1;\n\t}" : "=f"(hi) : "l"(v));
     return hi;
 }
 

@@ -175,9 +175,27 @@ cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
     return launch_combine_v<KMAX, SHARED, 4>(a, s);
 }
 
+template <int KMAX, bool SHARED, int NT>
+cudaError_t launch_combine_nt(const moe::CombineArgs &a, cudaStream_t s) {
+    auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT>;
+    if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
+    return launch(kernel, a.bs, NT, 0, s, a);
+}
+
+template <int KMAX, bool SHARED>
+cudaError_t launch_combine_tok(const moe::CombineArgs &a, cudaStream_t s) {
+    switch (moe::dp_threads(a.hidden >> 3)) {
+        case 64: return launch_combine_nt<KMAX, SHARED, 64>(a, s);
+        case 128: return launch_combine_nt<KMAX, SHARED, 128>(a, s);
+        case 192: return launch_combine_nt<KMAX, SHARED, 192>(a, s);
+        case 224: return launch_combine_nt<KMAX, SHARED, 224>(a, s);
+        default: return launch_combine_nt<KMAX, SHARED, 256>(a, s);
+    }
+}
+
 template <int KMAX>
 cudaError_t launch_combine(const moe::CombineArgs &a, cudaStream_t s) {
-    return a.shared_x ? launch_combine_t<KMAX, true>(a, s) : launch_combine_t<KMAX, false>(a, s);
+    return a.shared_x ? launch_combine_tok<KMAX, true>(a, s) : launch_combine_tok<KMAX, false>(a, s);
 }
 
 }  // namespace
@@ -247,10 +265,15 @@ moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_i
     a.expert_scales = expert_scales;
     a.active_mask = active_mask;
     a.table = table;
+    // stage the table in shared memory when it fits: by one bulk copy when its
+    // address and size allow one (16-byte multiples), else by plain loads
+    const size_t tab_bytes = (size_t)p->num_logical * p->table_cols * sizeof(int32_t);
+    a.table_mode = tab_bytes > moe::kUeTableSmemMax ? 0 : (aligned(table, 16) && tab_bytes % 16 == 0) ? 2 : 1;
     a.balanced_ids = balanced_ids;
     a.balanced_mask = balanced_mask;
     a.err = reinterpret_cast<uint32_t *>(workspace);
-    const size_t smem = moe::update_expert_smem_bytes(p->ep_world_size);
+    const size_t smem =
+        moe::update_expert_smem_bytes(p->ep_world_size, a.table_mode, p->num_logical, p->table_cols);
     if (!ensure_smem(moe::update_expert_kernel, smem)) return MOE_ERR_CUDA;
     return launch(moe::update_expert_kernel, 1, moe::kUeThreads, smem, as_stream(cuda_stream), a) == cudaSuccess
                ? MOE_OK

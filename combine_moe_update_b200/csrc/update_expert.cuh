@@ -27,6 +27,7 @@ struct UpdateArgs {
     const float *expert_scales;  // may be null
     const uint8_t *active_mask;  // may be null
     const int32_t *table;
+    int table_mode;  // 0: read from global memory; 1: staged in shared memory by loads; 2: by one bulk copy
     int32_t *balanced_ids;
     uint8_t *balanced_mask;
     uint32_t *err;
@@ -36,10 +37,19 @@ constexpr int kUeThreads = 1024;
 constexpr int kUeItems = 8;  // copies per thread: bs * K <= 8192 = 1024 * 8
 
 // Dynamic shared memory: n[1024], first[1024], inst[1024], the division
-// magic of every n[e] (1024), then one uint16 counter per (rank, warp).
-inline size_t update_expert_smem_bytes(int ep_world_size) {
-    return 4 * 1024 * sizeof(int) + 32 * (size_t)ep_world_size * sizeof(uint16_t);
+// magic of every n[e] (1024), one uint16 counter per (rank, warp), then (in
+// table modes 1 and 2) the whole [E, F] table, 16-byte aligned.
+__host__ __device__ inline size_t update_expert_counters_bytes(int ep_world_size) {
+    return ((32 * (size_t)ep_world_size * sizeof(uint16_t)) + 15) / 16 * 16;
 }
+inline size_t update_expert_smem_bytes(int ep_world_size, int table_mode, int num_logical, int table_cols) {
+    return 4 * 1024 * sizeof(int) + update_expert_counters_bytes(ep_world_size) +
+           (table_mode ? (size_t)num_logical * table_cols * sizeof(int32_t) : 0);
+}
+// Tables up to this size are staged in shared memory: both table reads of
+// the kernel (column 0, then one entry per instance) then cost no dependent
+// global-memory round trip.
+constexpr size_t kUeTableSmemMax = 160 * 1024;
 
 __device__ __forceinline__ void update_expert_drop_all(const UpdateArgs &a) {
     const int n = a.bs * a.top_k;
@@ -56,6 +66,9 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     int *s_first = s_n + 1024;
     int *s_inst = s_first + 1024;
     uint32_t *s_mag = reinterpret_cast<uint32_t *>(s_inst + 1024);  // div_magic(n[e])
+    const int32_t *s_tab = reinterpret_cast<const int32_t *>(
+        smem + 4 * 1024 * sizeof(int) + update_expert_counters_bytes(a.ep_world_size));
+    __shared__ __align__(8) uint64_t s_tab_bar;
     uint16_t *s_wc = reinterpret_cast<uint16_t *>(s_mag + 1024);   // [ws][32]
     __shared__ int s_warp[32];
     __shared__ int s_bad, s_total;
@@ -65,9 +78,17 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
 
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int F = a.table_cols, ws = a.ep_world_size, E = a.num_logical;
+    const uint32_t tab_bytes = (uint32_t)(E * F) * sizeof(int32_t);
 
-    // The copies' inputs do not depend on the table: load them first so the
-    // loads overlap the table bookkeeping.
+    // The table first (one bulk copy in mode 2), then the copies' inputs,
+    // which do not depend on it, so that all the loads are in flight together.
+    if (a.table_mode == 2 && t == 0) {
+        mbar_init(&s_tab_bar, 1);
+        mbar_arrive_expect_tx(&s_tab_bar, tab_bytes);
+        bulk_copy_g2s(const_cast<int32_t *>(s_tab), a.table, tab_bytes, &s_tab_bar);
+    }
+    if (a.table_mode == 1)
+        for (int q = t; q < E * F; q += kUeThreads) const_cast<int32_t *>(s_tab)[q] = __ldg(a.table + q);
     const int items = a.bs * a.top_k;
     // Every load is unconditional (indices clamped into range), so all of
     // them are in flight together; items past the end are discarded below.
@@ -95,12 +116,22 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
 
     if (t == 0) s_bad = 0;
     for (int q = t; q < 32 * ws; q += kUeThreads) s_wc[q] = 0;
-    __syncthreads();
+    __syncthreads();  // also publishes the mbarrier's initialisation (and a loaded table)
+    const bool tab_ok = a.table_mode != 2 || mbar_wait_bounded(&s_tab_bar, 0);
+    if (__syncthreads_or(!tab_ok)) {  // the table copy never landed: report, wait once more, drop all
+        if (t == 0) {
+            raise_error(a.err, kDevTimeout);
+            mbar_wait_bounded(&s_tab_bar, 0);
+        }
+        update_expert_drop_all(a);
+        return;
+    }
+    const int32_t *tab = a.table_mode ? s_tab : a.table;
 
     // 1. instance counts and their prefix sum
     int n = 0;
     if (t < E) {
-        n = a.table[(size_t)t * F];
+        n = tab[(size_t)t * F];
         if (n < 1 || n > F - 1) {
             s_bad = 1;
             n = 0;
@@ -131,7 +162,7 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
             int mid = (lo + hi + 1) >> 1;
             if (s_first[mid] <= t) lo = mid; else hi = mid - 1;
         }
-        r = a.table[(size_t)lo * F + 1 + (t - s_first[lo])];
+        r = tab[(size_t)lo * F + 1 + (t - s_first[lo])];
         if (r < 0 || r >= ws) {
             s_bad = 1;
             r = -1;

@@ -104,6 +104,46 @@ def test_parity_random_replicated_tables(B, seed):
     assert_parity(w, run_gpu(w, B), run_oracle(w))
 
 
+@pytest.mark.parametrize("case", ["bulk", "odd_size", "misaligned", "too_big"])
+def test_update_table_staging(B, case):
+    """The mapping table is staged in shared memory by one bulk copy (16-byte
+    aligned address and size), by plain loads (other sizes or addresses), or
+    read from global memory (tables over 160 KB); all agree with the oracle."""
+    rng = np.random.default_rng({"bulk": 1, "odd_size": 2, "misaligned": 3, "too_big": 4}[case])
+    nl, ws, F = {"bulk": (16, 4, 5), "odd_size": (7, 7, 3), "misaligned": (16, 4, 5), "too_big": (1024, 64, 65)}[case]
+    total = nl if case != "bulk" and case != "misaligned" else 32
+    reps = np.ones(nl, np.int64)
+    extra = total - nl
+    while extra:
+        e = int(rng.integers(0, nl))
+        if reps[e] < F - 1:
+            reps[e] += 1
+            extra -= 1
+    rank_of = rng.permutation(np.repeat(np.arange(ws), total // ws))
+    table = np.full((nl, F), -1, np.int32)
+    table[:, 0] = reps
+    pos = 0
+    for e in range(nl):
+        table[e, 1:1 + reps[e]] = rank_of[pos:pos + reps[e]]
+        pos += reps[e]
+    K = min(8, nl)
+    ids = gen.topk_uniform(rng, 96, nl, K)
+    t_dev = dev(table)
+    if case == "misaligned":  # the same table 4 bytes past a 16-byte boundary
+        buf = torch.zeros(table.size + 4, dtype=torch.int32, device="cuda")
+        buf[1:1 + table.size] = t_dev.reshape(-1)
+        t_dev = buf[1:1 + table.size].view(nl, F)
+        assert t_dev.data_ptr() % 16 == 4
+    wsp = B.new_workspace()
+    bal, bm = B.update_expert(dev(ids), t_dev, ws, workspace=wsp)
+    torch.cuda.synchronize()
+    assert B.read_device_error(wsp) == 0
+    ob, om, oe = orc.update_expert(ids, table, ws)
+    assert oe == 0
+    np.testing.assert_array_equal(host(bal), ob)
+    np.testing.assert_array_equal(host(bm), om)
+
+
 # ------------------------------------------------------------ rank / dispatch
 
 def run_dispatch_gpu(B, x_bits, ids, E, ws, mode, mask=None, smooth=None):
