@@ -275,7 +275,8 @@ moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_i
     const size_t smem =
         moe::update_expert_smem_bytes(p->ep_world_size, a.table_mode, p->num_logical, p->table_cols);
     if (!ensure_smem(moe::update_expert_kernel, smem)) return MOE_ERR_CUDA;
-    return launch(moe::update_expert_kernel, 1, moe::kUeThreads, smem, as_stream(cuda_stream), a) == cudaSuccess
+    return launch(moe::update_expert_kernel, moe::update_expert_blocks(p->bs * p->top_k), moe::kUeThreads, smem,
+                  as_stream(cuda_stream), a) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }

@@ -1,9 +1,10 @@
 // update_expert.cuh -- logical expert -> deployed instance, plus pruning.
 //
 // Follows aclnnMoeUpdateExpert (description: "Load balancing", "Expert
-// pruning"; "Restriction on the shape format" for the mapping table).  One
-// block of 1024 threads does everything: it is a few kilobytes of work and
-// a single block keeps the table bookkeeping in shared memory.
+// pruning"; "Restriction on the shape format" for the mapping table).  Each
+// block of 1024 threads stages the table in shared memory and does the table
+// bookkeeping (steps 1-3, at most 1024 instance positions) itself, then maps
+// its own slice of 1024 copies (step 4); the blocks run on different SMs.
 //
 //   1. Read n_e (column 0) for every logical expert, check 1 <= n_e <= F-1,
 //      and prefix-sum it: instance (e, j) gets position first[e] + j.
@@ -34,7 +35,14 @@ struct UpdateArgs {
 };
 
 constexpr int kUeThreads = 1024;
-constexpr int kUeItems = 8;  // copies per thread: bs * K <= 8192 = 1024 * 8
+constexpr int kUeItems = 1;  // copies per thread; a block maps kUeThreads * kUeItems copies
+
+// Blocks for `items` copies.  Every block repeats the table bookkeeping (a
+// few thousand shared-memory operations) and maps its own slice of copies,
+// so the slices run on different SMs at once.
+__host__ __device__ inline int update_expert_blocks(int items) {
+    return (items + kUeThreads * kUeItems - 1) / (kUeThreads * kUeItems);
+}
 
 // Dynamic shared memory: n[1024], first[1024], inst[1024], the division
 // magic of every n[e] (1024), one uint16 counter per (rank, warp), then (in
@@ -51,9 +59,10 @@ inline size_t update_expert_smem_bytes(int ep_world_size, int table_mode, int nu
 // global-memory round trip.
 constexpr size_t kUeTableSmemMax = 160 * 1024;
 
+// Drop this block's slice of copies (a bad table drops every copy).
 __device__ __forceinline__ void update_expert_drop_all(const UpdateArgs &a) {
-    const int n = a.bs * a.top_k;
-    for (int it = threadIdx.x; it < n; it += blockDim.x) {
+    const int n = min(a.bs * a.top_k, (int)(blockIdx.x + 1) * kUeThreads * kUeItems);
+    for (int it = blockIdx.x * kUeThreads * kUeItems + threadIdx.x; it < n; it += blockDim.x) {
         a.balanced_ids[it] = -1;
         a.balanced_mask[it] = 0;
     }
@@ -90,29 +99,32 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     if (a.table_mode == 1)
         for (int q = t; q < E * F; q += kUeThreads) const_cast<int32_t *>(s_tab)[q] = __ldg(a.table + q);
     const int items = a.bs * a.top_k;
+    const int base = blockIdx.x * kUeThreads * kUeItems;  // this block's first copy
     // Every load is unconditional (indices clamped into range), so all of
     // them are in flight together; items past the end are discarded below.
     int pe[kUeItems];
     float ps[kUeItems];
     bool pa[kUeItems];
 #pragma unroll
-    for (int u = 0; u < kUeItems; ++u) pe[u] = __ldg(a.expert_ids + min(t + u * kUeThreads, items - 1));
+    for (int u = 0; u < kUeItems; ++u) pe[u] = __ldg(a.expert_ids + min(base + t + u * kUeThreads, items - 1));
 #pragma unroll
     for (int u = 0; u < kUeItems; ++u) ps[u] = 0.0f;
     if (a.expert_scales) {
 #pragma unroll
-        for (int u = 0; u < kUeItems; ++u) ps[u] = __ldg(a.expert_scales + min(t + u * kUeThreads, items - 1));
+        for (int u = 0; u < kUeItems; ++u)
+            ps[u] = __ldg(a.expert_scales + min(base + t + u * kUeThreads, items - 1));
     }
 #pragma unroll
     for (int u = 0; u < kUeItems; ++u) pa[u] = true;
     if (a.active_mask) {
 #pragma unroll
         for (int u = 0; u < kUeItems; ++u)
-            pa[u] = __ldg(a.active_mask + div_by_magic((uint32_t)min(t + u * kUeThreads, items - 1), a.k_magic)) != 0;
+            pa[u] = __ldg(a.active_mask +
+                          div_by_magic((uint32_t)min(base + t + u * kUeThreads, items - 1), a.k_magic)) != 0;
     }
 #pragma unroll
     for (int u = 0; u < kUeItems; ++u)
-        if (t + u * kUeThreads >= items) pe[u] = -1;
+        if (base + t + u * kUeThreads >= items) pe[u] = -1;
 
     if (t == 0) s_bad = 0;
     for (int q = t; q < 32 * ws; q += kUeThreads) s_wc[q] = 0;
@@ -197,7 +209,7 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     // 4. every (token, k) copy
 #pragma unroll
     for (int u = 0; u < kUeItems; ++u) {
-        const int it = t + u * kUeThreads;
+        const int it = base + t + u * kUeThreads;
         if (it >= items) continue;
         const int i = (int)div_by_magic((uint32_t)it, a.k_magic);  // it / K
         const int e = pe[u];
