@@ -157,24 +157,7 @@ cudaError_t launch_dispatch_token_smooth(const moe::DispatchArgs &a, cudaStream_
     return launch_by_threads<MODE, TokenSmoothLaunch>(a, s);
 }
 
-// combine: a cluster of two 128-thread blocks per token (one per half row);
-// VECS = ceil(H / 16 / 128) vectors per thread.
-template <int KMAX, bool SHARED, int VECS>
-cudaError_t launch_combine_v(const moe::CombineArgs &a, cudaStream_t s) {
-    auto kernel = moe::combine_kernel<KMAX, SHARED, VECS>;
-    if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
-    return launch(kernel, 2 * a.bs, moe::kCbThreads, 0, s, a);
-}
-
-template <int KMAX, bool SHARED>
-cudaError_t launch_combine_t(const moe::CombineArgs &a, cudaStream_t s) {
-    const int vecs = ((a.hidden / 8 + 1) / 2 + moe::kCbThreads - 1) / moe::kCbThreads;  // 1..4
-    if (vecs <= 1) return launch_combine_v<KMAX, SHARED, 1>(a, s);
-    if (vecs <= 2) return launch_combine_v<KMAX, SHARED, 2>(a, s);
-    if (vecs <= 3) return launch_combine_v<KMAX, SHARED, 3>(a, s);
-    return launch_combine_v<KMAX, SHARED, 4>(a, s);
-}
-
+// combine: one block per token, block size from the row length.
 template <int KMAX, bool SHARED, int NT>
 cudaError_t launch_combine_nt(const moe::CombineArgs &a, cudaStream_t s) {
     auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT>;
