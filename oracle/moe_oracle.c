@@ -246,10 +246,25 @@ static void orc_quant_mxfp8_block(const uint16_t *x, int len, uint8_t *q, uint8_
         q[h] = orc_e4m3_encode(bf16_to_float(x[h]) / dyn);
 }
 
+/* Case 2 (quantMode 1, static quantization), one element:
+ *   xFp32 = CastToFp32(X) * scales
+ *   quantOut = Cast(xFp32, dstType)
+ * READING R21: dstType is int8 and Cast rounds half to even, then saturates
+ * to the int8 range [-128, 127]; a NaN product (0 * inf) casts to 0.  The
+ * scales are one coefficient (1,), one per column (H,), or one row per
+ * destination instance (E, H); nothing is sent besides the codes. */
+static int8_t orc_static_int8(float xf) {
+    float r = rintf(xf);
+    if (isnan(r)) return 0;
+    if (r > 127.0f) r = 127.0f;
+    if (r < -128.0f) r = -128.0f;
+    return (int8_t)r;
+}
+
 uint32_t orc_dispatch(int32_t bs, int32_t hidden, int32_t top_k,
                       int32_t num_instances, int32_t quant_mode,
                       const uint16_t *x_bf16, const int32_t *instance_ids,
-                      const uint8_t *mask, const float *smooth,
+                      const uint8_t *mask, const float *smooth, int64_t scales_len,
                       void *expand_x, void *dyn_scales,
                       int32_t *expand_idx, int32_t *src_of_row,
                       int32_t *expert_counts, int32_t *expert_offsets) {
@@ -290,6 +305,15 @@ uint32_t orc_dispatch(int32_t bs, int32_t hidden, int32_t top_k,
         const float *sm = smooth ? smooth + (size_t)items[r].id * H : NULL; /* READING R9 */
         if (quant_mode == 0) {
             memcpy((uint16_t *)expand_x + (size_t)r * H, xr, sizeof(uint16_t) * (size_t)H);
+        } else if (quant_mode == 1) {
+            int8_t *q = (int8_t *)expand_x + (size_t)r * H;
+            for (int h = 0; h < H; ++h) {
+                float s;
+                if (scales_len == 1) s = smooth[0];
+                else if (scales_len == H) s = smooth[h];
+                else s = smooth[(size_t)items[r].id * H + h];
+                q[h] = orc_static_int8(bf16_to_float(xr[h]) * s);
+            }
         } else if (quant_mode == 2) {
             orc_quant_int8_segment(xr, sm, H, (int8_t *)expand_x + (size_t)r * H,
                                    (float *)dyn_scales + r);

@@ -46,13 +46,15 @@ uint32_t orc_update_expert(int32_t bs, int32_t top_k, int32_t num_logical,
 
 /* Step 2: order the active (token, k) copies by destination instance and
  * quantize / copy them into the expert-major receive buffer.  [DV2]
- * quant_mode: 0 none (bf16 copy), 2 per-token int8, 3 per-128-tile int8,
- * 4 mxfp8 (e4m3, 32-element blocks, E8M0 scale bytes).
- * mask, smooth may be NULL.  dyn_scales is ignored for mode 0. */
+ * quant_mode: 0 none (bf16 copy), 1 static int8, 2 per-token int8,
+ * 3 per-128-tile int8, 4 mxfp8 (e4m3, 32-element blocks, E8M0 scale bytes).
+ * smooth holds scales_len floats: modes 2/3 the (E, H) smooth scales (or
+ * NULL); mode 1 the static scales, (1,), (H,) or (E, H).  mask may be NULL.
+ * dyn_scales is ignored for modes 0 and 1. */
 uint32_t orc_dispatch(int32_t bs, int32_t hidden, int32_t top_k,
                       int32_t num_instances, int32_t quant_mode,
                       const uint16_t *x_bf16, const int32_t *instance_ids,
-                      const uint8_t *mask, const float *smooth,
+                      const uint8_t *mask, const float *smooth, int64_t scales_len,
                       void *expand_x, void *dyn_scales,
                       int32_t *expand_idx, int32_t *src_of_row,
                       int32_t *expert_counts, int32_t *expert_offsets);

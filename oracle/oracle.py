@@ -55,7 +55,8 @@ def lib():
             L.orc_update_expert.restype = ctypes.c_uint32
             L.orc_update_expert.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, f32, vp, vp, vp]
             L.orc_dispatch.restype = ctypes.c_uint32
-            L.orc_dispatch.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.orc_dispatch.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp,
+                                       vp, vp]
             L.orc_combine_add_rmsnorm.restype = None
             L.orc_combine_add_rmsnorm.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, f64,
                                                   vp, vp, vp, vp, vp]
@@ -91,9 +92,11 @@ def dispatch(x_bf16, instance_ids, num_instances, quant_mode, mask=None, smooth=
     """aclnnMoeDistributeDispatchV2 on one simulated source rank.
 
     Returns a dict: expand_x [bs*K, H] (uint16 bf16 bits for mode 0, int8 for
-    modes 2/3, uint8 e4m3 codes for mode 4), dyn_scales (None for mode 0;
-    [rows] f32, [rows, ceil(H/128)] f32, or [rows, H/32] uint8 E8M0),
+    modes 1/2/3, uint8 e4m3 codes for mode 4), dyn_scales (None for modes 0
+    and 1; [rows] f32, [rows, ceil(H/128)] f32, or [rows, H/32] uint8 E8M0),
     expand_idx [bs,K], src_of_row [n], counts [E], offsets [E+1], n, err.
+    smooth: modes 2/3 the (E, H) smooth scales or None; mode 1 the static
+    scales, shape (1,), (H,) or (E, H).
     """
     x = _c(x_bf16, np.uint16)
     ids = _c(instance_ids, np.int32)
@@ -104,6 +107,11 @@ def dispatch(x_bf16, instance_ids, num_instances, quant_mode, mask=None, smooth=
     sm = _c(smooth, np.float32)
     if quant_mode == 0:
         ex = np.zeros((rows, H), np.uint16)
+        ds = None
+    elif quant_mode == 1:
+        if sm is None or sm.size not in (1, H, num_instances * H):
+            raise ValueError("static quantization needs scales of shape (1,), (H,) or (E, H)")
+        ex = np.zeros((rows, H), np.int8)
         ds = None
     elif quant_mode == 2:
         ex = np.zeros((rows, H), np.int8)
@@ -121,7 +129,8 @@ def dispatch(x_bf16, instance_ids, num_instances, quant_mode, mask=None, smooth=
     cnt = np.empty((num_instances,), np.int32)
     off = np.empty((num_instances + 1,), np.int32)
     err = lib().orc_dispatch(bs, H, k, int(num_instances), int(quant_mode), _p(x), _p(ids), _p(m),
-                             _p(sm), _p(ex), _p(ds), _p(idx), _p(src), _p(cnt), _p(off))
+                             _p(sm), ctypes.c_int64(0 if sm is None else sm.size), _p(ex), _p(ds), _p(idx),
+                             _p(src), _p(cnt), _p(off))
     n = int(off[-1])
     return dict(expand_x=ex, dyn_scales=ds, expand_idx=idx, src_of_row=src[:n], counts=cnt,
                 offsets=off, n=n, err=int(err))

@@ -213,6 +213,42 @@ def test_int8_worked_rows(orc):
             assert int(out["dyn_scales"][:1].view(np.uint32)[0]) == int(row["scale_bits"], 16)
 
 
+def test_static_int8_worked_rows(orc):
+    """quantMode 1 on hand-derived rows (scale (1,)): rounding half to even,
+    saturation to [-128, 127], and the NaN of 0 * inf casting to 0."""
+    for row in GOLDEN["quant_static_int8"]["rows"]:
+        scale = np.float32(np.inf) if row["scale"] == "inf" else np.float32(row["scale"])
+        out = orc.dispatch(bits([row["x"]]), np.zeros((1, 1), np.int32), 1, 1, smooth=np.array([scale]))
+        np.testing.assert_array_equal(out["expand_x"][0], row["q"])
+        assert out["dyn_scales"] is None
+
+
+@pytest.mark.parametrize("shape", ["one", "per_column", "per_instance"])
+def test_static_int8_matches_numpy_rint(orc, shape):
+    """Every scale shape against numpy's own round-half-to-even and clip on
+    the fp32 product, with the scale taken from the copy's destination
+    instance for (E, H) scales."""
+    rng = np.random.default_rng(21)
+    bs, H, K, E = 9, 1024, 3, 5
+    x = gen.bf16_bits(rng.standard_normal((bs, H), np.float32) * 40)
+    ids = gen.topk_uniform(rng, bs, E, K)
+    sc = {"one": np.array([1.7], np.float32), "per_column": rng.uniform(0.5, 3, H).astype(np.float32),
+          "per_instance": rng.uniform(0.5, 3, (E, H)).astype(np.float32)}[shape]
+    out = orc.dispatch(x, ids, E, 1, smooth=sc)
+    xf = gen.bf16_to_f32(x).astype(np.float32)
+    for r in range(out["n"]):
+        j = out["src_of_row"][r]
+        i, k = divmod(int(j), K)
+        s = sc if shape != "per_instance" else sc[ids[i, k]]
+        want = np.clip(np.rint((xf[i] * s).astype(np.float32)), -128, 127).astype(np.int8)
+        np.testing.assert_array_equal(out["expand_x"][r], want)
+
+
+def test_static_int8_needs_scales(orc):
+    with pytest.raises(ValueError):
+        orc.dispatch(bits([[1.0] * 1024]), np.zeros((1, 1), np.int32), 1, 1)
+
+
 def test_int8_per_tile_worked(orc):
     """Tile t of a per-tile row behaves like a per-token row on its own
     128 elements: tile 0 = first worked row, tile 1 = second, last tile
