@@ -49,12 +49,15 @@ def algorithmic_bytes(w, n, x_out=False, rstd=False):
     items = bs * K
     upd = items * (4 + 4 + 4 + 1) + (4 if w.prune_threshold > 0 else 0) + 2 * 4 * w.num_logical
     code = 2 if w.quant_mode == 0 else 1
-    sc = {0: 0, 2: 4, 3: 4 * ((H + 127) // 128), 4: H // 32}[w.quant_mode]
-    smooth_rows = 0
+    sc = {0: 0, 1: 0, 2: 4, 3: 4 * ((H + 127) // 128), 4: H // 32}[w.quant_mode]
+    scale_bytes = 0  # smooth rows of the instances hit, or the static scales
     if w.smooth is not None:
-        smooth_rows = len(set(map(int, w.meta.get("distinct_instances", []))))
+        if w.smooth.size in (1, H):
+            scale_bytes = 4 * w.smooth.size
+        else:
+            scale_bytes = 4 * H * len(set(map(int, w.meta.get("distinct_instances", []))))
     disp = (2 * bs * H                      # x
-            + 4 * H * smooth_rows           # smooth rows of the instances hit
+            + scale_bytes                   # smooth / static scales read
             + n * (H * code + sc)           # codes + scales of every kept copy
             + items * (4 + 1)               # instance ids + mask
             + items * 4 + n * 4             # expand_idx + src_of_row
@@ -418,7 +421,7 @@ def run_b200(args, rank, world, local_rank):
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": {0: "bf16", 2: "int8", 3: "int8", 4: "fp8e4m3"}[w.quant_mode] + "+fp32",
+        "vs_baseline": None, "dtype": {0: "bf16", 1: "int8", 2: "int8", 3: "int8", 4: "fp8e4m3"}[w.quant_mode] + "+fp32",
         "data": "synthetic (seeded; pages' shapes)",
         "config": {"workload": args.workload, "bs": w.bs, "hidden": w.hidden, "top_k": w.top_k,
                    "num_instances": w.num_instances, "ep_world_size_simulated": w.ep_world_size,

@@ -36,7 +36,7 @@ class UpdateParams(ctypes.Structure):
 class DispatchParams(ctypes.Structure):
     _fields_ = [("bs", ctypes.c_int32), ("hidden", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("ep_world_size", ctypes.c_int32), ("num_instances", ctypes.c_int32),
-                ("quant_mode", ctypes.c_int32)]
+                ("quant_mode", ctypes.c_int32), ("scales_len", ctypes.c_int32)]
 
 
 class CombineParams(ctypes.Structure):
@@ -165,12 +165,23 @@ def update_expert(expert_ids, table, ep_world_size, expert_scales=None, active_m
 
 
 def expand_dtype(quant_mode):
-    return {0: torch.bfloat16, 2: torch.int8, 3: torch.int8, 4: torch.uint8}[quant_mode]
+    return {0: torch.bfloat16, 1: torch.int8, 2: torch.int8, 3: torch.int8, 4: torch.uint8}[quant_mode]
 
 
 def scales_shape(quant_mode, rows, hidden):
-    return {0: None, 2: ((rows,), torch.float32), 3: ((rows, (hidden + 127) // 128), torch.float32),
+    return {0: None, 1: None, 2: ((rows,), torch.float32), 3: ((rows, (hidden + 127) // 128), torch.float32),
             4: ((rows, hidden // 32), torch.uint8)}[quant_mode]
+
+
+def _check_scales(smooth, quant_mode, num_instances, hidden):
+    """quant_mode 1: static scales of shape (1,), (H,) or (E, H); modes 2/3:
+    optional (E, H) smooth scales."""
+    if quant_mode == 1:
+        if smooth is None or smooth.dtype != torch.float32 or not smooth.is_contiguous() or \
+                smooth.numel() not in (1, hidden, int(num_instances) * hidden):
+            raise ValueError("quant_mode 1 needs float32 scales of shape (1,), (H,) or (num_instances, H)")
+    else:
+        _opt(smooth, "smooth", torch.float32, (num_instances, hidden))
 
 
 def alloc_dispatch_outputs(bs, hidden, top_k, num_instances, quant_mode, device="cuda"):
@@ -196,10 +207,11 @@ def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=Non
     k = instance_ids.shape[1]
     _req(instance_ids, "instance_ids", torch.int32, (bs, k))
     _opt(mask, "mask", torch.uint8, (bs, k))
-    _opt(smooth, "smooth", torch.float32, (num_instances, H))
+    _check_scales(smooth, quant_mode, num_instances, H)
     if out is None:
         out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
-    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode))
+    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode),
+                       0 if smooth is None else smooth.numel())
     ws = workspace if workspace is not None else new_workspace(x.device, stream)
     _check("moe_dispatch", lib.moe_dispatch(
         ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
@@ -245,11 +257,12 @@ def dispatch_noalloc(x, instance_ids, num_instances, ep_world_size, quant_mode, 
     k = instance_ids.shape[1]
     _req(instance_ids, "instance_ids", torch.int32, (bs, k))
     _opt(mask, "mask", torch.uint8, (bs, k))
-    _opt(smooth, "smooth", torch.float32, (num_instances, H))
+    _check_scales(smooth, quant_mode, num_instances, H)
     _opt(device_error, "device_error", torch.int32, (1,))
     if out is None:
         out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
-    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode))
+    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode),
+                       0 if smooth is None else smooth.numel())
     _check("moe_dispatch_noalloc", lib.moe_dispatch_noalloc(
         ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
         _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),

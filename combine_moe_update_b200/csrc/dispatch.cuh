@@ -22,8 +22,10 @@
 //   smooth row arrives in shared memory by a bulk asynchronous copy, so
 //   four blocks fit on an SM and a decode batch runs in one wave.
 //
-// Quantization, per mode ("计算公式" cases 1, 3, 4, 5):
+// Quantization, per mode ("计算公式" cases 1 to 5):
 //   0  copy the bf16 row;
+//   1  static: xFp32 = x * scales (one coefficient, per column, or the
+//      destination instance's row); q = Cast(xFp32, int8), saturating;
 //   2  xFp32 = x * smooth; dyn = 127 / max|xFp32| over the row;
 //      q = rint(xFp32 * dyn); scale = 1 / dyn;
 //   3  the same per 128-element tile;
@@ -44,7 +46,8 @@ struct DispatchArgs {
     const uint16_t *x;    // bf16 bits [bs, H]
     const int32_t *ids;   // instance ids [bs, K]
     const uint8_t *mask;  // [bs, K] or null
-    const float *smooth;  // [E, H] or null
+    const float *smooth;  // modes 2/3: [E, H] smooth scales or null; mode 1: static scales
+    int scales_len;       // floats in smooth: 0, 1 (one coefficient), H (per column) or E * H (per instance)
     void *expand_x;
     void *dyn_scales;
     int32_t *expand_idx;
@@ -237,6 +240,25 @@ __device__ __forceinline__ uint2 int8x8(const uint64_t (&v)[4], float dyn) {
     return make_uint2(lo, hi);
 }
 
+// Static int8 codes of 8 values (quantMode 1): Cast(v, int8) rounds half to
+// even and saturates to [-128, 127], a NaN giving 0.  Clamping before the
+// rounding gives the same codes (every value beyond the range rounds to a
+// saturated code either way) and keeps the magic-number add exact.
+__device__ __forceinline__ uint2 int8x8_static(const uint64_t (&v)[4]) {
+    uint32_t b[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float lo = f2_lo(v[q]), hi = f2_hi(v[q]);
+        const float cl = lo != lo ? 0.0f : fminf(fmaxf(lo, -128.0f), 127.0f);
+        const float ch = hi != hi ? 0.0f : fminf(fmaxf(hi, -128.0f), 127.0f);
+        b[2 * q] = __float_as_uint(__fadd_rn(cl, 12582912.0f));
+        b[2 * q + 1] = __float_as_uint(__fadd_rn(ch, 12582912.0f));
+    }
+    const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+    return make_uint2(lo, hi);
+}
+
 // The codes when dyn = +inf (amax == 0, or 127 / amax overflows fp32): v * inf
 // is +-inf, which saturates to +-127, or NaN (v = 0), which casts to 0.
 __device__ __forceinline__ uint32_t q8_inf(float v) { return v > 0.0f ? 0x7fu : (v < 0.0f ? 0x81u : 0u); }
@@ -338,7 +360,10 @@ template <int MODE, int NT>
 __device__ __forceinline__ void quantize_local(const uint64_t (&xf)[kDpVecs][4], int V, uint2 (&qv)[kDpVecs],
                                                float (&seg)[kDpVecs]) {
     const int t = threadIdx.x;
-    if constexpr (MODE == 3) {
+    if constexpr (MODE == 1) {
+#pragma unroll
+        for (int q = 0; q < kDpVecs; ++q) qv[q] = int8x8_static(xf[q]);
+    } else if constexpr (MODE == 3) {
         float dq[kDpVecs];
 #pragma unroll
         for (int q = 0; q < kDpVecs; ++q) {  // a 128-element tile = 16 vectors = 16 consecutive lanes
@@ -433,6 +458,28 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         uint64_t xf[kDpVecs][4];
 #pragma unroll
         for (int q = 0; q < kDpVecs; ++q) vec_to_f2(xv[q], xf[q]);
+        if constexpr (MODE == 1) {  // xFp32 = x * scales: one coefficient, or one per column
+            if (a.scales_len == 1) {
+                const float c = __ldg(a.smooth);
+                const uint64_t c2 = f2_pack(c, c);
+#pragma unroll
+                for (int q = 0; q < kDpVecs; ++q)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) xf[q][j] = f2_mul(xf[q][j], c2);
+            } else {
+#pragma unroll
+                for (int q = 0; q < kDpVecs; ++q) {
+                    const int p = t + q * NT;
+                    if (p >= V) continue;
+                    const float4 s0 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8));
+                    const float4 s1 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8) + 1);
+                    xf[q][0] = f2_mul(xf[q][0], f2_pack(s0.x, s0.y));
+                    xf[q][1] = f2_mul(xf[q][1], f2_pack(s0.z, s0.w));
+                    xf[q][2] = f2_mul(xf[q][2], f2_pack(s1.x, s1.y));
+                    xf[q][3] = f2_mul(xf[q][3], f2_pack(s1.z, s1.w));
+                }
+            }
+        }
         if constexpr (MODE == 2) {
             const float dyn = block_dyn<NT>(abs_max_vecs(xf), s_red);
             row_scale = __frcp_rn(dyn);  // 1 / dynamicScales

@@ -77,9 +77,13 @@ moe_status valid_dispatch(const moe_dispatch_params &p) {
     if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K || p.top_k > p.num_instances) return MOE_ERR_INVALID_ARG;
     if (p.ep_world_size < MOE_MIN_EP_WORLD || p.ep_world_size > MOE_MAX_EP_WORLD) return MOE_ERR_INVALID_ARG;
     if (p.num_instances % p.ep_world_size != 0) return MOE_ERR_INVALID_ARG;  // equal instances per rank
-    if (p.quant_mode == 1) return MOE_ERR_UNSUPPORTED;                     // static quantization
-    if (p.quant_mode != 0 && p.quant_mode != 2 && p.quant_mode != 3 && p.quant_mode != 4)
-        return MOE_ERR_INVALID_ARG;
+    if (p.quant_mode < 0 || p.quant_mode > 4) return MOE_ERR_INVALID_ARG;
+    const long long eh = (long long)p.num_instances * p.hidden;
+    if (p.quant_mode == 1 && p.scales_len != 1 && p.scales_len != p.hidden && p.scales_len != eh)
+        return MOE_ERR_INVALID_ARG;  // static scales: (1,), (H,) or (E, H)
+    if ((p.quant_mode == 2 || p.quant_mode == 3) && p.scales_len != 0 && p.scales_len != eh)
+        return MOE_ERR_INVALID_ARG;  // smooth scales: (E, H)
+    if ((p.quant_mode == 0 || p.quant_mode == 4) && p.scales_len != 0) return MOE_ERR_INVALID_ARG;
     if (p.quant_mode == 4 && p.hidden % 32 != 0) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
@@ -284,11 +288,12 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     const int mode = p->quant_mode;
     if (!x || !instance_ids || !expand_x || !expand_idx || !src_of_row || !expert_counts || !expert_offsets)
         return MOE_ERR_INVALID_ARG;
-    if ((mode == 0) != (dyn_scales == nullptr)) return MOE_ERR_INVALID_ARG;
-    if (smooth_scales && (mode == 0 || mode == 4)) return MOE_ERR_INVALID_ARG;  // the page: scales must be null
+    if ((mode == 0 || mode == 1) != (dyn_scales == nullptr)) return MOE_ERR_INVALID_ARG;  // no scales sent
+    if ((smooth_scales != nullptr) != (p->scales_len > 0)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(instance_ids, 4) || !aligned(expand_idx, 4) ||
         !aligned(src_of_row, 4) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
-        (smooth_scales && !aligned(smooth_scales, 16)) || ((mode == 2 || mode == 3) && !aligned(dyn_scales, 4)))
+        (smooth_scales && !aligned(smooth_scales, p->scales_len == 1 ? 4 : 16)) ||
+        ((mode == 2 || mode == 3) && !aligned(dyn_scales, 4)))
         return MOE_ERR_INVALID_ARG;
     if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < dispatch_workspace_bytes(*p))
         return MOE_ERR_WORKSPACE;
@@ -303,6 +308,7 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     a.ids = instance_ids;
     a.mask = mask;
     a.smooth = smooth_scales;
+    a.scales_len = p->scales_len;
     a.expand_x = expand_x;
     a.dyn_scales = dyn_scales;
     a.expand_idx = expand_idx;
@@ -317,11 +323,19 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     if (!ensure_smem(moe::route_kernel, rsmem)) return MOE_ERR_CUDA;
     if (launch(moe::route_kernel, slices, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
-    if (smooth_scales) {
-        e = mode == 2 ? launch_dispatch_token_smooth<2>(a, s) : launch_dispatch_token_smooth<3>(a, s);
+    // scales that depend on the destination instance (a row per instance) need
+    // the per-copy kernel; one coefficient or one per column is per token
+    const bool per_instance = smooth_scales && p->scales_len > p->hidden;
+    if (per_instance) {
+        switch (mode) {
+            case 1: e = launch_dispatch_token_smooth<1>(a, s); break;
+            case 2: e = launch_dispatch_token_smooth<2>(a, s); break;
+            case 3: e = launch_dispatch_token_smooth<3>(a, s); break;
+        }
     } else {
         switch (mode) {
             case 0: e = launch_dispatch_token<0>(a, s); break;
+            case 1: e = launch_dispatch_token<1>(a, s); break;
             case 2: e = launch_dispatch_token<2>(a, s); break;
             case 3: e = launch_dispatch_token<3>(a, s); break;
             case 4: e = launch_dispatch_token<4>(a, s); break;

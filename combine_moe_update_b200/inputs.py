@@ -178,6 +178,16 @@ def _skewed_eplb(name, seed, bs, hidden=4096, num_logical=128, top_k=8, ep_world
                     norm_eps=1e-6, **_common(rng, bs, hidden, top_k, bs * top_k))
 
 
+def _static_layer(name, seed, **kw):
+    """A uniform layer with static int8 quantization (quantMode 1): per-instance
+    static scales U(10, 40), so x ~ N(0, 1) fills much of the int8 range and
+    the tails saturate."""
+    w = uniform_layer(name, seed, quant_mode=1, **kw)
+    rng = np.random.Generator(np.random.PCG64([seed, 21]))
+    w.smooth = rng.uniform(10.0, 40.0, size=(w.num_instances, w.hidden)).astype(np.float32)
+    return w
+
+
 WORKLOADS = {
     # Bs 8, H 1024, 8 experts, K 2, 4 simulated ranks, no quantization.
     "tiny": dict(builder=uniform_layer, seed=0, bs=8, hidden=1024, num_experts=8, top_k=2,
@@ -193,6 +203,9 @@ WORKLOADS = {
     # ... and its unquantized variant (bf16 rows, no smooth, no shared expert).
     "deepseek_decode_bs512_bf16": dict(builder=uniform_layer, seed=1, bs=512, hidden=7168,
                                        num_experts=256, top_k=8, ep_world_size=32, quant_mode=0),
+    # The Bs 512 layer with static int8 quantization and per-instance scales.
+    "deepseek_decode_bs512_static": dict(builder=_static_layer, seed=1, bs=512, hidden=7168,
+                                         num_experts=256, top_k=8, ep_world_size=32, shared=True),
     # Zipf(1.2) routing over 128 experts, 160 instances on 16 ranks, mxfp8.
     "skewed_eplb": dict(builder=_skewed_eplb, seed=2, bs=512),
     # Largest shapes: H 8192, 1024 experts, K 16, 256 ranks, per-128-tile int8,

@@ -155,7 +155,9 @@ typedef struct {
     int32_t top_k;          /* K, (0, 16] and <= num_instances */
     int32_t ep_world_size;  /* simulated ranks, [2, 768]; must divide num_instances */
     int32_t num_instances;  /* deployed expert instances E, (0, 1024] */
-    int32_t quant_mode;     /* 0 none, 2 per-token int8, 3 per-128-tile int8, 4 mxfp8 (1: unsupported) */
+    int32_t quant_mode;     /* 0 none, 1 static int8, 2 per-token int8, 3 per-128-tile int8, 4 mxfp8 */
+    int32_t scales_len;     /* floats in smooth_scales: 0 when it is NULL; modes 2/3 num_instances * H;
+                               mode 1: 1, H or num_instances * H (the static scales' shape) */
 } moe_dispatch_params;
 
 MOE_API moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, size_t *bytes);
@@ -163,18 +165,23 @@ MOE_API moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, siz
 /*
  * Orders the active (token, k) copies by destination instance and writes each
  * one, quantized per quant_mode, into the expert-major receive buffer
- * (aclnnMoeDistributeDispatchV2, "计算公式" cases 1, 3, 4, 5).  Rows are
+ * (aclnnMoeDistributeDispatchV2, "计算公式" cases 1 to 5).  Rows are
  * sorted by (instance, token, k); instance ids are rank-major, so simulated
  * rank r receives rows [expert_offsets[r*L], expert_offsets[(r+1)*L]).
  *
  *   x             [bs, H] bf16   device
  *   instance_ids  [bs, K] int32  device, in [0, num_instances) (moe_update_expert's output)
  *   mask          [bs, K] uint8  device, optional; 0 = copy not sent
- *   smooth_scales [num_instances, H] f32 device, optional, modes 2 and 3 only:
- *                                xFp32 = x * smooth_scales[instance]
- *   expand_x      [bs*K, H]      device, out: bf16 (mode 0), int8 (2, 3) or e4m3 (4).
+ *   smooth_scales f32 device, p->scales_len floats:
+ *                   modes 2 and 3, optional: [num_instances, H] smooth scales,
+ *                     xFp32 = x * smooth_scales[instance];
+ *                   mode 1, required: the static scales, shape (1,), (H,) or
+ *                     [num_instances, H] (row of the copy's instance),
+ *                     xFp32 = x * scale, code = Cast(xFp32, int8);
+ *                   modes 0 and 4: NULL.
+ *   expand_x      [bs*K, H]      device, out: bf16 (mode 0), int8 (1, 2, 3) or e4m3 (4).
  *                                Rows >= expert_offsets[E] are left untouched.
- *   dyn_scales    device, out, NULL in mode 0:
+ *   dyn_scales    device, out, NULL in modes 0 and 1:
  *                   mode 2: [bs*K] f32 = 1 / (127 / max|xFp32|)        (0 for an all-zero row)
  *                   mode 3: [bs*K, ceil(H/128)] f32, the same per 128-element tile
  *                   mode 4: [bs*K, H/32] uint8 E8M0 byte = sharedExp + 127, the
@@ -185,8 +192,9 @@ MOE_API moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, siz
  *   expert_counts [E]     int32  device, out: rows received by each instance
  *   expert_offsets[E+1]   int32  device, out: exclusive prefix sum, [E] = rows used
  *
- * int8 codes round half to even and clamp to [-127, 127]; e4m3 codes round
- * half to even and saturate at +-448.  All quantization arithmetic is IEEE
+ * int8 codes round half to even and clamp to [-127, 127] (modes 2 and 3) or
+ * saturate to [-128, 127] with NaN giving 0 (mode 1, static); e4m3 codes
+ * round half to even and saturate at +-448.  All quantization arithmetic is IEEE
  * binary32, so codes and scales are bit-exact against any IEEE evaluation of
  * the same formulas.  Device errors: an instance id out of range sets
  * MOE_DEV_BAD_ID and the copy is not sent.

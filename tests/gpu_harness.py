@@ -101,7 +101,9 @@ def assert_parity(w: gen.Workload, g: dict, o: dict):
     np.testing.assert_array_equal(ge[:n], oe[:n])
     assert (ge[n:] == POISON).all(), "rows past the used region must stay untouched"
     assert (g["src_of_row"][n:].view(np.uint8) == POISON).all()
-    if w.quant_mode != 0:
+    if w.quant_mode in (0, 1):  # no scales are sent
+        assert g["dyn_scales"] is None and d["dyn_scales"] is None
+    else:
         gs = g["dyn_scales"].view(np.uint8).reshape(g["dyn_scales"].shape[0], -1)
         os_ = d["dyn_scales"].view(np.uint8).reshape(d["dyn_scales"].shape[0], -1)
         np.testing.assert_array_equal(gs[:n], os_[:n])

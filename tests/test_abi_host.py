@@ -69,6 +69,12 @@ def ws_size(L, fn, params):
     return st, n.value
 
 
+@pytest.mark.parametrize("scales_len", [1, 1024, 8 * 1024])
+def test_static_quant_params_accepted(L, scales_len):
+    """quantMode 1 with scales of shape (1,), (H,) or (E, H) passes validation."""
+    assert ws_size(L, "moe_dispatch_workspace_size", L.DispatchParams(8, 1024, 2, 4, 8, 1, scales_len)) == (0, 256)
+
+
 def test_workspace_sizes_for_valid_params(L):
     assert ws_size(L, "moe_update_expert_workspace_size", L.UpdateParams(512, 16, 1024, 257, 256, 0.05)) == (0, 256)
     assert ws_size(L, "moe_dispatch_workspace_size", L.DispatchParams(512, 7168, 8, 32, 256, 2)) == (0, 256)
@@ -99,14 +105,18 @@ DISPATCH_BAD = [
     (dict(bs=0), 1), (dict(bs=513), 1), (dict(hidden=1008), 1), (dict(hidden=8208), 1), (dict(hidden=1032), 1),
     (dict(top_k=0), 1), (dict(top_k=17), 1), (dict(num_instances=1025), 1), (dict(num_instances=0), 1),
     (dict(ep_world_size=1), 1), (dict(ep_world_size=769), 1), (dict(ep_world_size=24), 1),
-    (dict(quant_mode=5), 1), (dict(quant_mode=-1), 1), (dict(quant_mode=1), 2),
+    (dict(quant_mode=5), 1), (dict(quant_mode=-1), 1),
     (dict(quant_mode=4, hidden=1040), 1),
+    # scales_len must match the mode: static scales (1,), (H,) or (E, H); smooth (E, H); none in modes 0 and 4
+    (dict(quant_mode=1, scales_len=0), 1), (dict(quant_mode=1, scales_len=3), 1),
+    (dict(quant_mode=2, scales_len=1024), 1), (dict(quant_mode=3, scales_len=1), 1),
+    (dict(quant_mode=0, scales_len=1), 1), (dict(quant_mode=4, scales_len=8 * 1024), 1),
 ]
 
 
 @pytest.mark.parametrize("bad,status", DISPATCH_BAD)
 def test_dispatch_rejects(L, bad, status):
-    base = dict(bs=8, hidden=1024, top_k=2, ep_world_size=4, num_instances=8, quant_mode=0)
+    base = dict(bs=8, hidden=1024, top_k=2, ep_world_size=4, num_instances=8, quant_mode=0, scales_len=0)
     base.update(bad)
     p = L.DispatchParams(*base.values())
     assert ws_size(L, "moe_dispatch_workspace_size", p)[0] == status

@@ -104,6 +104,40 @@ def test_parity_random_replicated_tables(B, seed):
     assert_parity(w, run_gpu(w, B), run_oracle(w))
 
 
+@pytest.mark.parametrize("shape", ["one", "per_column", "per_instance"])
+@pytest.mark.parametrize("H", [1024, 1168, 7168])
+def test_parity_static_quant(B, shape, H):
+    """quantMode 1: static scales of every shape, with products large enough
+    that many codes saturate, on a full row, a ragged row and the gate's H."""
+    w = gen.uniform_layer(f"static_{shape}_{H}", seed=17 + H, bs=37, hidden=H, num_experts=24, top_k=5,
+                          ep_world_size=6, quant_mode=1, shared=True)
+    rng = np.random.default_rng(H)
+    w.smooth = {"one": np.array([37.5], np.float32),
+                "per_column": rng.uniform(0.5, 80.0, H).astype(np.float32),
+                "per_instance": rng.uniform(0.5, 80.0, (w.num_instances, H)).astype(np.float32)}[shape]
+    assert_parity(w, run_gpu(w, B), run_oracle(w))
+
+
+@pytest.mark.parametrize("shape", ["one", "per_column", "per_instance"])
+def test_static_quant_ties_and_specials(B, shape):
+    """Half-integer products (ties to even), values past +-128, and 0 * inf."""
+    w = gen.uniform_layer(f"static_edge_{shape}", seed=5, bs=6, hidden=1024, num_experts=8, top_k=2,
+                          ep_world_size=4, quant_mode=1)
+    vals = np.arange(-140, 140.5, 0.5, dtype=np.float32)  # every half-integer in [-140, 140]
+    xf = np.zeros((w.bs, 1024), np.float32)
+    xf[0, :vals.size] = vals
+    xf[1, :vals.size] = -vals
+    xf[2, :8] = [0, 1, -1, 0, 2, -2, 0, 0]
+    w.x = gen.bf16_bits(xf)
+    s = {"one": np.array([1.0], np.float32), "per_column": np.ones(1024, np.float32),
+         "per_instance": np.ones((w.num_instances, 1024), np.float32)}[shape]
+    s = s.copy()
+    if shape == "per_column":
+        s[:8] = np.inf  # row 2's first 8 columns: 0 * inf = NaN -> 0, +-inf saturates
+    w.smooth = s
+    assert_parity(w, run_gpu(w, B), run_oracle(w))
+
+
 @pytest.mark.parametrize("case", ["bulk", "odd_size", "misaligned", "too_big"])
 def test_update_table_staging(B, case):
     """The mapping table is staged in shared memory by one bulk copy (16-byte
