@@ -30,18 +30,18 @@ class MoeError(RuntimeError):
 class UpdateParams(ctypes.Structure):
     _fields_ = [("bs", ctypes.c_int32), ("top_k", ctypes.c_int32), ("num_logical", ctypes.c_int32),
                 ("table_cols", ctypes.c_int32), ("ep_world_size", ctypes.c_int32),
-                ("prune_threshold", ctypes.c_float)]
+                ("prune_threshold", ctypes.c_float), ("sources", ctypes.c_int32)]
 
 
 class DispatchParams(ctypes.Structure):
     _fields_ = [("bs", ctypes.c_int32), ("hidden", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("ep_world_size", ctypes.c_int32), ("num_instances", ctypes.c_int32),
-                ("quant_mode", ctypes.c_int32), ("scales_len", ctypes.c_int32)]
+                ("quant_mode", ctypes.c_int32), ("scales_len", ctypes.c_int32), ("sources", ctypes.c_int32)]
 
 
 class CombineParams(ctypes.Structure):
     _fields_ = [("bs", ctypes.c_int32), ("hidden", ctypes.c_int32), ("top_k", ctypes.c_int32),
-                ("expand_rows", ctypes.c_int32), ("norm_eps", ctypes.c_float)]
+                ("expand_rows", ctypes.c_int32), ("norm_eps", ctypes.c_float), ("sources", ctypes.c_int32)]
 
 
 EXPORTS = (
@@ -121,11 +121,29 @@ def _opt(t, name, dtype, shape=None):
 # workspace / device errors
 # --------------------------------------------------------------------------
 
-def new_workspace(device=None, stream=None) -> torch.Tensor:
-    """A zeroed workspace (holds the sticky device error word)."""
-    ws = torch.empty(WORKSPACE_BYTES, dtype=torch.uint8, device=device or "cuda")
-    _check("moe_workspace_init", lib.moe_workspace_init(_ptr(ws), WORKSPACE_BYTES, _stream(stream)))
+def new_workspace(device=None, stream=None, nbytes=WORKSPACE_BYTES) -> torch.Tensor:
+    """A zeroed workspace (holds the sticky device error word; dispatch with
+    several source ranks may need more than the default, see
+    dispatch_workspace_bytes)."""
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+    _check("moe_workspace_init", lib.moe_workspace_init(_ptr(ws), nbytes, _stream(stream)))
     return ws
+
+
+def _per_source(tokens, sources, what):
+    if sources < 1 or tokens % sources:
+        raise ValueError(f"{what}: {tokens} tokens do not split over {sources} source ranks")
+    return tokens // sources
+
+
+def dispatch_workspace_bytes(bs, hidden, top_k, ep_world_size, num_instances, quant_mode, scales_len=0,
+                             sources=1):
+    """Workspace bytes moe_dispatch needs (bs = tokens per source rank)."""
+    n = ctypes.c_size_t(0)
+    p = DispatchParams(bs, hidden, top_k, int(ep_world_size), int(num_instances), int(quant_mode),
+                       int(scales_len), int(sources))
+    _check("moe_dispatch_workspace_size", lib.moe_dispatch_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return max(int(n.value), WORKSPACE_BYTES)
 
 
 def read_device_error(workspace: torch.Tensor, stream=None) -> int:
@@ -143,14 +161,16 @@ def clear_device_error(workspace: torch.Tensor, stream=None) -> None:
 # --------------------------------------------------------------------------
 
 def update_expert(expert_ids, table, ep_world_size, expert_scales=None, active_mask=None,
-                  prune_threshold=0.0, workspace=None, out=None, stream=None):
-    """moe_update_expert.  Returns (balanced_ids int32 [bs,K], balanced_mask uint8 [bs,K])."""
+                  prune_threshold=0.0, workspace=None, out=None, stream=None, sources=1):
+    """moe_update_expert.  Returns (balanced_ids int32 [bs,K], balanced_mask uint8 [bs,K]).
+    With sources = S the arrays hold S source ranks' tokens, rank-major."""
     _req(expert_ids, "expert_ids", torch.int32)
     bs, k = expert_ids.shape
     _req(table, "table", torch.int32)
     _opt(expert_scales, "expert_scales", torch.float32, (bs, k))
     _opt(active_mask, "active_mask", torch.uint8, (bs,))
-    p = UpdateParams(bs, k, table.shape[0], table.shape[1], int(ep_world_size), float(prune_threshold))
+    p = UpdateParams(_per_source(bs, sources, "update_expert"), k, table.shape[0], table.shape[1],
+                     int(ep_world_size), float(prune_threshold), int(sources))
     if out is None:
         out = (torch.empty((bs, k), dtype=torch.int32, device=expert_ids.device),
                torch.empty((bs, k), dtype=torch.uint8, device=expert_ids.device))
@@ -198,7 +218,7 @@ def alloc_dispatch_outputs(bs, hidden, top_k, num_instances, quant_mode, device=
 
 
 def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=None, smooth=None,
-             workspace=None, out=None, stream=None):
+             workspace=None, out=None, stream=None, sources=1):
     """moe_dispatch.  Returns a dict with expand_x, dyn_scales, expand_idx,
     src_of_row, counts and offsets (see include/moe_b200.h for layouts)."""
     _req(x, "x", torch.bfloat16)
@@ -210,9 +230,11 @@ def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=Non
     _check_scales(smooth, quant_mode, num_instances, H)
     if out is None:
         out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
-    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode),
-                       0 if smooth is None else smooth.numel())
-    ws = workspace if workspace is not None else new_workspace(x.device, stream)
+    sl = 0 if smooth is None else smooth.numel()
+    p = DispatchParams(_per_source(bs, sources, "dispatch"), H, k, int(ep_world_size), int(num_instances),
+                       int(quant_mode), sl, int(sources))
+    ws = workspace if workspace is not None else new_workspace(
+        x.device, stream, dispatch_workspace_bytes(p.bs, H, k, ep_world_size, num_instances, quant_mode, sl, sources))
     _check("moe_dispatch", lib.moe_dispatch(
         ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
         _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
@@ -222,7 +244,7 @@ def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=Non
 
 def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, norm_eps,
                         shared_x=None, want_x_out=False, want_rstd=False, workspace=None, out=None,
-                        stream=None):
+                        stream=None, sources=1):
     """moe_combine_add_rmsnorm.  Returns a dict with y (and x_out / rstd when asked)."""
     _req(expand_x, "expand_x", torch.bfloat16)
     rows, H = expand_x.shape
@@ -237,7 +259,7 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
         out = dict(y=torch.empty((bs, H), dtype=torch.bfloat16, device=dev),
                    x_out=torch.empty((bs, H), dtype=torch.bfloat16, device=dev) if want_x_out else None,
                    rstd=torch.empty((bs,), dtype=torch.float32, device=dev) if want_rstd else None)
-    p = CombineParams(bs, H, k, rows, float(norm_eps))
+    p = CombineParams(_per_source(bs, sources, "combine_add_rmsnorm"), H, k, rows, float(norm_eps), int(sources))
     ws = workspace if workspace is not None else new_workspace(expand_x.device, stream)
     _check("moe_combine_add_rmsnorm", lib.moe_combine_add_rmsnorm(
         ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x),
@@ -247,7 +269,7 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
 
 
 def dispatch_noalloc(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=None, smooth=None,
-                     out=None, device_error=None, stream=None):
+                     out=None, device_error=None, stream=None, sources=1):
     """moe_dispatch_noalloc: moe_dispatch with the library's own static scratch
     instead of a workspace.  device_error: optional int32 CUDA tensor of one
     element that receives the call's device error word."""
@@ -261,8 +283,8 @@ def dispatch_noalloc(x, instance_ids, num_instances, ep_world_size, quant_mode, 
     _opt(device_error, "device_error", torch.int32, (1,))
     if out is None:
         out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
-    p = DispatchParams(bs, H, k, int(ep_world_size), int(num_instances), int(quant_mode),
-                       0 if smooth is None else smooth.numel())
+    p = DispatchParams(_per_source(bs, sources, "dispatch_noalloc"), H, k, int(ep_world_size),
+                       int(num_instances), int(quant_mode), 0 if smooth is None else smooth.numel(), int(sources))
     _check("moe_dispatch_noalloc", lib.moe_dispatch_noalloc(
         ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
         _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),

@@ -201,11 +201,13 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int *s_warp) {
     return v;
 }
 
-// floor(n / d) for 0 <= n < 2^16 and 1 <= d <= 2^16, given magic = ceil(2^32 / d)
-// (from div_magic; 0 stands for d = 1, whose magic 2^32 does not fit).
-// Writing magic = (2^32 + r) / d with 0 <= r < d, the product
-// n * magic / 2^32 = n / d + n r / (d 2^32) and the second term is below 1/d,
-// so it never carries floor(n / d) past the next integer.
+// floor(n / d) for n * (d - 1) < 2^32 and 1 <= d <= 2^16, given
+// magic = ceil(2^32 / d) (from div_magic; 0 stands for d = 1, whose magic
+// 2^32 does not fit).  Writing magic = (2^32 + r) / d with 0 <= r < d, the
+// product n * magic / 2^32 = n / d + n r / (d 2^32); the second term is below
+// 1/d while n r < 2^32, so it never carries floor(n / d) past the next
+// integer.  (The library divides copy indices < 2^23 by K <= 16 and token
+// indices < 2^19 by replica counts <= 768.)
 __host__ __device__ inline uint32_t div_magic(uint32_t d) {
     return d <= 1 ? 0u : (uint32_t)((0x100000000ull + d - 1) / d);
 }

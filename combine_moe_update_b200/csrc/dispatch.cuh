@@ -200,6 +200,174 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
     }
 }
 
+// ---------------------------------------------------- route, many copies ---
+//
+// Past 8192 copies (several source ranks), rebuilding the whole histogram in
+// every slice no longer pays, so the same order is built in three passes
+// over slices of kRlCopies = 4096 copies with a table in the workspace:
+//   route_hist_kernel   slice s counts its sent copies per instance: tab[s][e]
+//   route_scan_kernel   per instance, the exclusive prefix of tab[.][e] over
+//                       the slices (in place), and the total tot[e]
+//   route_place_kernel  slice s: bucket offsets from a block scan of tot,
+//                       then 8 rounds of 512 copies, each ranked as in
+//                       route_kernel (match_any + per-warp prefix) on top of
+//                       a running per-instance count of the earlier rounds.
+// row = offset[e] + tab[s][e] + earlier rounds + rank in the round: the same
+// (instance, token, k) order as route_kernel.
+
+constexpr int kRlRounds = 8;
+constexpr int kRlCopies = kRtThreads * kRlRounds;  // 4096 copies per slice
+
+__host__ __device__ inline int route_large_slices(int copies) { return (copies + kRlCopies - 1) / kRlCopies; }
+
+// The workspace table after the error area: tab [S][E], then tot [E].
+inline size_t route_large_bytes(int copies, int num_instances) {
+    return ((size_t)route_large_slices(copies) * num_instances + num_instances) * sizeof(int);
+}
+
+// Keys of this thread's copies in the rounds of slice s (unconditional,
+// clamped loads, so all are in flight together); -1 past the end.
+__device__ __forceinline__ void slice_keys(const DispatchArgs &a, int s, int (&key)[kRlRounds]) {
+    const int N = a.bs * a.top_k, E = a.num_instances, t = threadIdx.x;
+    uint32_t sent[kRlRounds];
+#pragma unroll
+    for (int u = 0; u < kRlRounds; ++u) key[u] = __ldg(a.ids + min(s * kRlCopies + u * kRtThreads + t, N - 1));
+    if (a.mask) {
+#pragma unroll
+        for (int u = 0; u < kRlRounds; ++u) sent[u] = __ldg(a.mask + min(s * kRlCopies + u * kRtThreads + t, N - 1));
+    } else {
+#pragma unroll
+        for (int u = 0; u < kRlRounds; ++u) sent[u] = 1;
+    }
+#pragma unroll
+    for (int u = 0; u < kRlRounds; ++u) {
+        const int id = key[u];
+        key[u] = (s * kRlCopies + u * kRtThreads + t < N && sent[u] != 0) ? ((id >= 0 && id < E) ? id : -2) : -1;
+    }
+}
+
+// Dynamic shared memory: E ints.
+__global__ void __launch_bounds__(kRtThreads) route_hist_kernel(DispatchArgs a, int *tab) {
+    extern __shared__ __align__(16) int s_h[];
+    const int E = a.num_instances, s = blockIdx.x, t = threadIdx.x;
+    for (int e = t; e < E; e += kRtThreads) s_h[e] = 0;
+    __syncthreads();
+    pdl_wait();  // the instance ids may come from the previous kernel
+    pdl_launch_dependents();
+    int key[kRlRounds];
+    slice_keys(a, s, key);
+#pragma unroll
+    for (int u = 0; u < kRlRounds; ++u) {
+        if (key[u] >= 0) atomicAdd(&s_h[key[u]], 1);
+        if (key[u] == -2) raise_error(a.err, kDevBadId);  // each copy is in exactly one slice
+    }
+    __syncthreads();
+    for (int e = t; e < E; e += kRtThreads) tab[(size_t)s * E + e] = s_h[e];
+}
+
+// One thread per instance: the exclusive prefix of its column over the S
+// slices (loads batched by the unrolled loop) and its total.
+__global__ void __launch_bounds__(1024) route_scan_kernel(DispatchArgs a, int *tab, int *tot, int S) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int E = a.num_instances, e = blockIdx.x * 1024 + threadIdx.x;
+    if (e >= E) return;
+    int run = 0;
+#pragma unroll 8
+    for (int s = 0; s < S; ++s) {
+        const int v = tab[(size_t)s * E + e];
+        tab[(size_t)s * E + e] = run;
+        run += v;
+    }
+    tot[e] = run;
+}
+
+// Dynamic shared memory: per-(instance, warp) uint16 counters, then four
+// int arrays over the instances (offset, slice base, running count, round total).
+inline size_t route_place_smem_bytes(int num_instances) {
+    return (size_t)num_instances * kRtWarps * sizeof(uint16_t) + 4 * (size_t)num_instances * sizeof(int);
+}
+
+__global__ void __launch_bounds__(kRtThreads) route_place_kernel(DispatchArgs a, const int *tab, const int *tot) {
+    extern __shared__ __align__(16) unsigned char smem_p[];
+    const int E = a.num_instances, N = a.bs * a.top_k, s = blockIdx.x;
+    uint16_t *s_cnt = reinterpret_cast<uint16_t *>(smem_p);                                  // [E][16]
+    int *s_off = reinterpret_cast<int *>(smem_p + (size_t)E * kRtWarps * sizeof(uint16_t));  // [E]
+    int *s_base = s_off + E;                                                                // [E]
+    int *s_run = s_base + E;                                                                // [E]
+    int *s_rtot = s_run + E;                                                                // [E]
+    __shared__ int s_warp[32];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    for (int e = t; e < E; e += kRtThreads) {
+        s_run[e] = 0;
+        s_rtot[e] = 0;
+    }
+    pdl_wait();  // the table and the totals come from the previous kernels
+    pdl_launch_dependents();
+
+    int key[kRlRounds];
+    slice_keys(a, s, key);
+    // bucket offsets: exclusive scan of the totals, 2 consecutive instances per thread (E <= 1024)
+    int v2[2], sum = 0;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int b = t * 2 + u;
+        v2[u] = b < E ? __ldg(tot + b) : 0;
+        sum += v2[u];
+    }
+    const int incl = block_inclusive_scan(sum, s_warp);
+    const int total = s_warp[kRtWarps - 1];
+    int run = incl - sum;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int b = t * 2 + u;
+        if (b < E) {
+            s_off[b] = run;
+            if (s == 0) {
+                a.counts[b] = v2[u];
+                a.offsets[b] = run;
+            }
+        }
+        run += v2[u];
+    }
+    if (s == 0 && t == 0) a.offsets[E] = total;
+    for (int e = t; e < E; e += kRtThreads) s_base[e] = __ldg(tab + (size_t)s * E + e);
+
+    uint32_t *cnt32 = reinterpret_cast<uint32_t *>(s_cnt);
+    for (int u = 0; u < kRlRounds; ++u) {
+        for (int q = t; q < 8 * E; q += kRtThreads) cnt32[q] = 0;  // E * 16 uint16
+        __syncthreads();  // counters clear; the previous round's readers are done
+        const int k = key[u];
+        const unsigned peers = __match_any_sync(kFull, k);
+        if (k >= 0 && lane == __ffs(peers) - 1) s_cnt[k * kRtWarps + w] = (uint16_t)__popc(peers);
+        const int local = __popc(peers & ((1u << lane) - 1u));
+        __syncthreads();
+        for (int b = t; b < E; b += kRtThreads) {  // per-instance prefix over the 16 warps
+            s_run[b] += s_rtot[b];                 // the previous round's copies of b
+            int r = 0;
+#pragma unroll
+            for (int q = 0; q < kRtWarps; ++q) {
+                const int c = s_cnt[b * kRtWarps + q];
+                s_cnt[b * kRtWarps + q] = (uint16_t)r;
+                r += c;
+            }
+            s_rtot[b] = r;
+        }
+        __syncthreads();
+        const int j = s * kRlCopies + u * kRtThreads + t;
+        if (j < N) {
+            if (k < 0) {
+                a.expand_idx[j] = -1;
+            } else {
+                const int row = s_off[k] + s_base[k] + s_run[k] + s_cnt[k * kRtWarps + w] + local;
+                a.expand_idx[j] = row;
+                a.src_of_row[row] = j;
+            }
+        }
+        __syncthreads();  // every thread has read this round's counters
+    }
+}
+
 // ------------------------------------------------------------ quantizers ---
 
 constexpr int kDpVecs = 4;  // 8-element vectors per thread: H / 8 <= 1024 = 256 * 4

@@ -17,12 +17,24 @@ namespace {
 // The workspace holds the sticky device error word (4 bytes), padded to 256.
 constexpr size_t kWorkspaceBytes = 256;
 
+// Tokens of a call: bs per source rank times the source ranks (0 means 1).
+inline int total_tokens(int bs, int sources) { return bs * (sources > 1 ? sources : 1); }
+
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
-// The dispatch workspace: the error-word area.
-size_t dispatch_workspace_bytes(const moe_dispatch_params &) { return kWorkspaceBytes; }
+// Copies up to which the single-pass route runs (it rebuilds the whole
+// histogram in every slice); beyond, the three-pass route and its table.
+constexpr int kRouteSinglePassMax = moe::kRtThreads * moe::kRtKeys;  // 8192
+
+// The dispatch workspace: the error-word area, then (past 8192 copies) the
+// route's slice table.
+size_t dispatch_workspace_bytes(const moe_dispatch_params &p) {
+    const int copies = total_tokens(p.bs, p.sources) * p.top_k;
+    if (copies <= kRouteSinglePassMax) return kWorkspaceBytes;
+    return kWorkspaceBytes + (moe::route_large_bytes(copies, p.num_instances) + 15) / 16 * 16;
+}
 
 bool check_workspace(const void *ws, size_t bytes) {
     return ws != nullptr && aligned(ws, 16) && bytes >= kWorkspaceBytes;
@@ -67,8 +79,10 @@ bool valid_update(const moe_update_params &p) {
     if (p.ep_world_size < MOE_MIN_EP_WORLD || p.ep_world_size > MOE_MAX_EP_WORLD) return false;
     if (p.table_cols < 2 || p.table_cols > p.ep_world_size + 1) return false;
     if (!(p.prune_threshold == p.prune_threshold)) return false;  // NaN
+    if (p.sources < 0 || p.sources > p.ep_world_size) return false;
     return true;
 }
+
 
 moe_status valid_dispatch(const moe_dispatch_params &p) {
     if (p.bs < 1 || p.bs > MOE_MAX_BS) return MOE_ERR_INVALID_ARG;
@@ -77,6 +91,7 @@ moe_status valid_dispatch(const moe_dispatch_params &p) {
     if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K || p.top_k > p.num_instances) return MOE_ERR_INVALID_ARG;
     if (p.ep_world_size < MOE_MIN_EP_WORLD || p.ep_world_size > MOE_MAX_EP_WORLD) return MOE_ERR_INVALID_ARG;
     if (p.num_instances % p.ep_world_size != 0) return MOE_ERR_INVALID_ARG;  // equal instances per rank
+    if (p.sources < 0 || p.sources > p.ep_world_size) return MOE_ERR_INVALID_ARG;
     if (p.quant_mode < 0 || p.quant_mode > 4) return MOE_ERR_INVALID_ARG;
     const long long eh = (long long)p.num_instances * p.hidden;
     if (p.quant_mode == 1 && p.scales_len != 1 && p.scales_len != p.hidden && p.scales_len != eh)
@@ -94,6 +109,7 @@ bool valid_combine(const moe_combine_params &p) {
     if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K) return false;
     if (p.expand_rows < 1) return false;
     if (!(p.norm_eps >= 0.0f) || p.norm_eps > 3.0e38f) return false;  // rejects NaN and inf
+    if (p.sources < 0 || p.sources > MOE_MAX_EP_WORLD) return false;
     return true;
 }
 
@@ -241,7 +257,7 @@ moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_i
     if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
 
     moe::UpdateArgs a;
-    a.bs = p->bs;
+    a.bs = total_tokens(p->bs, p->sources);  // every source rank's tokens; token t picks replica t mod n_e
     a.top_k = p->top_k;
     a.num_logical = p->num_logical;
     a.table_cols = p->table_cols;
@@ -262,7 +278,7 @@ moe_status moe_update_expert(const moe_update_params *p, const int32_t *expert_i
     const size_t smem =
         moe::update_expert_smem_bytes(p->ep_world_size, a.table_mode, p->num_logical, p->table_cols);
     if (!ensure_smem(moe::update_expert_kernel, smem)) return MOE_ERR_CUDA;
-    return launch(moe::update_expert_kernel, moe::update_expert_blocks(p->bs * p->top_k), moe::kUeThreads, smem,
+    return launch(moe::update_expert_kernel, moe::update_expert_blocks(a.bs * p->top_k), moe::kUeThreads, smem,
                   as_stream(cuda_stream), a) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
@@ -298,7 +314,7 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < dispatch_workspace_bytes(*p))
         return MOE_ERR_WORKSPACE;
     moe::DispatchArgs a;
-    a.bs = p->bs;
+    a.bs = total_tokens(p->bs, p->sources);  // the kernels see every source rank's tokens
     a.hidden = p->hidden;
     a.top_k = p->top_k;
     a.num_instances = p->num_instances;
@@ -318,10 +334,25 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     a.err = reinterpret_cast<uint32_t *>(workspace);
     cudaStream_t s = as_stream(cuda_stream);
 
-    const int slices = moe::route_slices(p->bs * p->top_k);
-    const size_t rsmem = moe::route_smem_bytes(p->num_instances);
-    if (!ensure_smem(moe::route_kernel, rsmem)) return MOE_ERR_CUDA;
-    if (launch(moe::route_kernel, slices, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
+    const int copies = a.bs * p->top_k;
+    if (copies <= kRouteSinglePassMax) {
+        const int slices = moe::route_slices(copies);
+        const size_t rsmem = moe::route_smem_bytes(p->num_instances);
+        if (!ensure_smem(moe::route_kernel, rsmem)) return MOE_ERR_CUDA;
+        if (launch(moe::route_kernel, slices, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+        const int S = moe::route_large_slices(copies), E = p->num_instances;
+        int *tab = reinterpret_cast<int *>(reinterpret_cast<unsigned char *>(workspace) + kWorkspaceBytes);
+        int *tot = tab + (size_t)S * E;
+        const size_t hsmem = (size_t)E * sizeof(int), psmem = moe::route_place_smem_bytes(E);
+        if (!ensure_smem(moe::route_hist_kernel, hsmem) || !ensure_smem(moe::route_place_kernel, psmem))
+            return MOE_ERR_CUDA;
+        if (launch(moe::route_hist_kernel, S, moe::kRtThreads, hsmem, s, a, tab) != cudaSuccess ||
+            launch(moe::route_scan_kernel, (E + 1023) / 1024, 1024, 0, s, a, tab, tot, S) != cudaSuccess ||
+            launch(moe::route_place_kernel, S, moe::kRtThreads, psmem, s, a, (const int *)tab, (const int *)tot) !=
+                cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
     cudaError_t e = cudaSuccess;
     // scales that depend on the destination instance (a row per instance) need
     // the per-copy kernel; one coefficient or one per column is per token
@@ -365,7 +396,7 @@ moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expa
     if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
 
     moe::CombineArgs a;
-    a.bs = p->bs;
+    a.bs = total_tokens(p->bs, p->sources);
     a.hidden = p->hidden;
     a.top_k = p->top_k;
     a.expand_rows = p->expand_rows;

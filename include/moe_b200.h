@@ -36,7 +36,14 @@
  *   - The workspace must be zeroed once (moe_workspace_init) before its first
  *     use; the error word then accumulates until moe_clear_device_error.
  *     Calls that share a workspace share its error word.  A workspace of
- *     MOE_MAX_WORKSPACE_BYTES serves every call.
+ *     MOE_MAX_WORKSPACE_BYTES serves every call with one source rank (and
+ *     any call of at most 8192 copies); dispatch with several source ranks
+ *     may need more, as moe_dispatch_workspace_size reports.
+ *   - Several source ranks (the "sources" field): the pages' AllToAllV has
+ *     every EP rank send Bs tokens.  With sources = S, the calls take
+ *     T = S * bs tokens, rank-major (token t = r * bs + i of source rank r);
+ *     rows are ordered by (instance, r, i, k), the same as (instance, t, k).
+ *     0 means 1.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -68,8 +75,8 @@ typedef enum {
 #define MOE_DEV_BAD_TABLE 2u  /* mapping table broke its restrictions; every copy was dropped */
 #define MOE_DEV_TIMEOUT   4u  /* a bounded wait for an asynchronous copy gave up; outputs incomplete */
 
-/* The largest workspace any *_workspace_size call reports (bytes): the
- * 256-byte area that holds the error word. */
+/* The largest workspace any *_workspace_size call reports for one source
+ * rank (bytes): the 256-byte area that holds the error word. */
 #define MOE_MAX_WORKSPACE_BYTES 256
 
 /* Limits taken from the pages (shape-variable constraints of each page). */
@@ -110,6 +117,7 @@ typedef struct {
     int32_t ep_world_size;  /* simulated ranks, [2, 768] */
     float prune_threshold;  /* copies whose expert_scales entry is strictly below this are
                                pruned; <= 0 (or expert_scales == NULL) disables */
+    int32_t sources;        /* source ranks S, [0, ep_world_size] (0 = 1): arrays hold S * bs tokens */
 } moe_update_params;
 
 MOE_API moe_status moe_update_expert_workspace_size(const moe_update_params *p, size_t *bytes);
@@ -158,6 +166,8 @@ typedef struct {
     int32_t quant_mode;     /* 0 none, 1 static int8, 2 per-token int8, 3 per-128-tile int8, 4 mxfp8 */
     int32_t scales_len;     /* floats in smooth_scales: 0 when it is NULL; modes 2/3 num_instances * H;
                                mode 1: 1, H or num_instances * H (the static scales' shape) */
+    int32_t sources;        /* source ranks S, [0, ep_world_size] (0 = 1): x and the routing hold
+                               S * bs tokens, expand_x S * bs * K rows */
 } moe_dispatch_params;
 
 MOE_API moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, size_t *bytes);
@@ -215,6 +225,7 @@ typedef struct {
     int32_t top_k;        /* K, (0, 16] */
     int32_t expand_rows;  /* rows of expand_x (>= every non-negative expand_idx + 1), > 0 */
     float norm_eps;       /* normEps, finite and >= 0 */
+    int32_t sources;      /* source ranks S, [0, 768] (0 = 1): the token arrays hold S * bs tokens */
 } moe_combine_params;
 
 MOE_API moe_status moe_combine_add_rmsnorm_workspace_size(const moe_combine_params *p, size_t *bytes);

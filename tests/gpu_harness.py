@@ -43,29 +43,33 @@ def assert_close_bf16(got_bits, want_f64, rtol=1e-2, what="y"):
                            f"{np.argwhere(bad)[0].tolist()}: got {got[bad][0]}, want {want[bad][0]}")
 
 
-def run_gpu(w: gen.Workload, B, workspace=None, combine_rows=None, want_x_out=True):
+def run_gpu(w: gen.Workload, B, workspace=None, combine_rows=None, want_x_out=True, sources=1):
     """update_expert -> dispatch -> combine on the GPU.  Outputs are poisoned
     first.  combine reads `combine_rows` (bf16 bits) or the workload's
-    synthetic expert outputs."""
-    ws = workspace if workspace is not None else B.new_workspace()
+    synthetic expert outputs.  sources: the workload's w.bs tokens are that
+    many source ranks' tokens, rank-major."""
+    sl = 0 if w.smooth is None else w.smooth.size
+    ws = workspace if workspace is not None else B.new_workspace(nbytes=B.dispatch_workspace_bytes(
+        w.bs // sources, w.hidden, w.top_k, w.ep_world_size, w.num_instances, w.quant_mode, sl, sources))
     ids, table, sc = dev(w.expert_ids), dev(w.table), dev(w.expert_scales)
     am = None if w.active_mask is None else dev(w.active_mask)
     bal = poison_(torch.empty_like(ids))
     bm = poison_(torch.empty(ids.shape, dtype=torch.uint8, device="cuda"))
     B.update_expert(ids, table, w.ep_world_size, expert_scales=sc, active_mask=am,
-                    prune_threshold=w.prune_threshold, workspace=ws, out=(bal, bm))
+                    prune_threshold=w.prune_threshold, workspace=ws, out=(bal, bm), sources=sources)
     d = B.alloc_dispatch_outputs(w.bs, w.hidden, w.top_k, w.num_instances, w.quant_mode)
     for v in d.values():
         if v is not None:
             poison_(v)
     x = dev_bf16(w.x)
     sm = None if w.smooth is None else dev(w.smooth)
-    B.dispatch(x, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=sm, workspace=ws, out=d)
+    B.dispatch(x, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=sm, workspace=ws, out=d,
+               sources=sources)
     rows = combine_rows if combine_rows is not None else w.expert_out
     ex = dev_bf16(rows)
     sh = None if w.shared_x is None else dev_bf16(w.shared_x)
     c = B.combine_add_rmsnorm(ex, d["expand_idx"], sc, dev_bf16(w.residual), dev_bf16(w.gamma), w.norm_eps,
-                              shared_x=sh, want_x_out=want_x_out, want_rstd=True, workspace=ws)
+                              shared_x=sh, want_x_out=want_x_out, want_rstd=True, workspace=ws, sources=sources)
     torch.cuda.synchronize()
     out = dict(balanced_ids=host(bal), balanced_mask=host(bm), err=B.read_device_error(ws))
     for k, v in d.items():

@@ -104,6 +104,35 @@ def test_parity_random_replicated_tables(B, seed):
     assert_parity(w, run_gpu(w, B), run_oracle(w))
 
 
+@pytest.mark.parametrize("bs,S,E,K,H,ws,mode,smooth", [
+    (100, 3, 24, 5, 1168, 6, 3, True),        # 1500 copies: the single-pass route over three sources
+    (512, 3, 64, 6, 1024, 8, 2, True),        # 9216 copies: the three-pass route, a ragged last slice
+    (256, 32, 256, 8, 1024, 32, 2, True),     # 65536 copies: the gate's routing with all 32 ranks sending
+    (200, 7, 1024, 16, 1024, 256, 0, False),  # 22400 copies over 1024 instances, K 16
+])
+def test_parity_multi_source(B, bs, S, E, K, H, ws, mode, smooth):
+    """Every simulated rank sends its own Bs tokens (S source ranks, S * Bs
+    tokens rank-major): routing, rows, codes and combine against the oracle
+    on the same S * Bs tokens."""
+    w = gen.uniform_layer(f"src{S}_{bs}", seed=31 + S, bs=bs * S, hidden=H, num_experts=E, top_k=K,
+                          ep_world_size=ws, quant_mode=mode, smooth=smooth, shared=True)
+    assert_parity(w, run_gpu(w, B, sources=S), run_oracle(w))
+
+
+def test_multi_source_needs_its_workspace(B):
+    """Past 8192 copies the route needs its slice table: a workspace of the
+    default size is refused before anything runs."""
+    w = gen.uniform_layer("src_ws", seed=3, bs=512 * 3, hidden=1024, num_experts=64, top_k=6, ep_world_size=8,
+                          quant_mode=0)
+    need = B.dispatch_workspace_bytes(512, 1024, 6, 8, 64, 0, 0, 3)
+    assert need > B.WORKSPACE_BYTES
+    x = dev_bf16(w.x)
+    ids = dev(w.expert_ids)
+    with pytest.raises(B.MoeError) as e:
+        B.dispatch(x, ids, 64, 8, 0, workspace=B.new_workspace(), sources=3)
+    assert e.value.status == B.MOE_ERR_WORKSPACE
+
+
 @pytest.mark.parametrize("shape", ["one", "per_column", "per_instance"])
 @pytest.mark.parametrize("H", [1024, 1168, 7168])
 def test_parity_static_quant(B, shape, H):

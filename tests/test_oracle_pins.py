@@ -213,6 +213,33 @@ def test_int8_worked_rows(orc):
             assert int(out["dyn_scales"][:1].view(np.uint32)[0]) == int(row["scale_bits"], 16)
 
 
+def test_sources_order_and_additivity(orc):
+    """Several source ranks (READING R22): S * Bs tokens, rank-major.  Counts
+    are the sums of each rank's own counts (dispatching every rank alone),
+    and within each instance's rows the source rank, then the token, then k
+    never decrease."""
+    rng = np.random.default_rng(22)
+    S, bs, K, E, H = 4, 6, 3, 8, 1024
+    x = gen.bf16_bits(rng.standard_normal((S * bs, H), np.float32))
+    ids = gen.topk_uniform(rng, S * bs, E, K)
+    full = orc.dispatch(x, ids, E, 0)
+    parts = [orc.dispatch(x[r * bs:(r + 1) * bs], ids[r * bs:(r + 1) * bs], E, 0) for r in range(S)]
+    np.testing.assert_array_equal(full["counts"], sum(p["counts"] for p in parts))
+    src = full["src_of_row"]
+    for e in range(E):
+        seg = src[full["offsets"][e]:full["offsets"][e + 1]]
+        key = [(int(j) // K // bs, int(j) // K % bs, int(j) % K) for j in seg]
+        assert key == sorted(key)
+        assert all(ids[j // K, j % K] == e for j in seg)
+    # each rank's rows of instance e are its own dispatch's rows of e, in order
+    for e in range(E):
+        seg = src[full["offsets"][e]:full["offsets"][e + 1]]
+        for r in range(S):
+            mine = [int(j) - r * bs * K for j in seg if int(j) // K // bs == r]
+            p = parts[r]
+            np.testing.assert_array_equal(mine, p["src_of_row"][p["offsets"][e]:p["offsets"][e + 1]])
+
+
 def test_static_int8_worked_rows(orc):
     """quantMode 1 on hand-derived rows (scale (1,)): rounding half to even,
     saturation to [-128, 127], and the NaN of 0 * inf casting to 0."""
