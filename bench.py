@@ -19,6 +19,7 @@ reported value is the tokens of all ranks over the slowest rank's time.
 from __future__ import annotations
 
 import argparse
+import functools
 import hashlib
 import json
 import os
@@ -206,18 +207,25 @@ def run_b200(args, rank, world, local_rank):
     ids, scales = dev(w.expert_ids), dev(w.expert_scales)
     x, residual, expert_out = bf(w.x), bf(w.residual), bf(w.expert_out)
     shared = None if w.shared_x is None else bf(w.shared_x)
-    ws = B.new_workspace()
+    # several source ranks (every simulated rank sends its own tokens)
+    S = int(w.meta.get("sources", 1))
+    upd = functools.partial(B.update_expert, sources=S)
+    disp = functools.partial(B.dispatch, sources=S)
+    comb = functools.partial(B.combine_add_rmsnorm, sources=S)
+    ws = B.new_workspace(nbytes=B.dispatch_workspace_bytes(
+        w.bs // S, w.hidden, w.top_k, w.ep_world_size, w.num_instances, w.quant_mode,
+        0 if w.smooth is None else w.smooth.size, S))
     bal = torch.empty_like(ids)
     bm = torch.empty(ids.shape, dtype=torch.uint8, device="cuda")
     d = B.alloc_dispatch_outputs(w.bs, w.hidden, w.top_k, w.num_instances, w.quant_mode)
     c = dict(y=torch.empty_like(x), x_out=None, rstd=None)
 
     def step(xx=x, ii=ids, ss=scales, rr=residual, ee=expert_out, sh=shared):
-        B.update_expert(ii, table, w.ep_world_size, expert_scales=ss, prune_threshold=w.prune_threshold,
+        upd(ii, table, w.ep_world_size, expert_scales=ss, prune_threshold=w.prune_threshold,
                         workspace=ws, out=(bal, bm))
-        B.dispatch(xx, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
+        disp(xx, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
                    workspace=ws, out=d)
-        B.combine_add_rmsnorm(ee, d["expand_idx"], ss, rr, gamma, w.norm_eps, shared_x=sh, workspace=ws, out=c)
+        comb(ee, d["expand_idx"], ss, rr, gamma, w.norm_eps, shared_x=sh, workspace=ws, out=c)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     clean = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.float32, device="cuda")  # 256 MiB
@@ -258,15 +266,15 @@ def run_b200(args, rank, world, local_rank):
             for e in evs:
                 flush_l2()
                 e[0].record()
-                B.update_expert(ids, table, w.ep_world_size, expert_scales=scales,
+                upd(ids, table, w.ep_world_size, expert_scales=scales,
                                 prune_threshold=w.prune_threshold, workspace=ws, out=(bal, bm))
                 if per_call:
                     e[1].record()
-                B.dispatch(x, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
+                disp(x, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth,
                            workspace=ws, out=d)
                 if per_call:
                     e[2].record()
-                B.combine_add_rmsnorm(expert_out, d["expand_idx"], scales, residual, gamma, w.norm_eps,
+                comb(expert_out, d["expand_idx"], scales, residual, gamma, w.norm_eps,
                                       shared_x=shared, workspace=ws, out=c)
                 e[-1].record()
         return g, evs
@@ -289,11 +297,11 @@ def run_b200(args, rank, world, local_rank):
             ev_cold[0].record()
             for s_ in range(G):
                 xx, ii, ss, rr, ee, sh, tb, sm, gm = sets[s_ % R]
-                B.update_expert(ii, tb, w.ep_world_size, expert_scales=ss, prune_threshold=w.prune_threshold,
+                upd(ii, tb, w.ep_world_size, expert_scales=ss, prune_threshold=w.prune_threshold,
                                 workspace=ws, out=(bal, bm))
-                B.dispatch(xx, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=sm,
+                disp(xx, bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, smooth=sm,
                            workspace=ws, out=d)
-                B.combine_add_rmsnorm(ee, d["expand_idx"], ss, rr, gm, w.norm_eps, shared_x=sh, workspace=ws,
+                comb(ee, d["expand_idx"], ss, rr, gm, w.norm_eps, shared_x=sh, workspace=ws,
                                       out=c)
             ev_cold[1].record()
         l2_note = (f"not flushed: {R} input sets of {per_set / 2**20:.0f} MiB (activations and layer parameters) "
@@ -351,7 +359,7 @@ def run_b200(args, rank, world, local_rank):
             eb[0].record()
             for _ in range(M):
                 for st in sets:
-                    B.combine_add_rmsnorm(st["ee"], d["expand_idx"], scales, st["rr"], gamma, w.norm_eps,
+                    comb(st["ee"], d["expand_idx"], scales, st["rr"], gamma, w.norm_eps,
                                           shared_x=st["sh"], workspace=ws, out=c)
             eb[1].record()
         graph_c.replay()

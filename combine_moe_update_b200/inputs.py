@@ -178,6 +178,15 @@ def _skewed_eplb(name, seed, bs, hidden=4096, num_logical=128, top_k=8, ep_world
                     norm_eps=1e-6, **_common(rng, bs, hidden, top_k, bs * top_k))
 
 
+def _all_ranks_layer(name, seed, bs, sources, **kw):
+    """Every one of `sources` simulated ranks sends its own Bs tokens: a
+    uniform layer of sources * bs tokens, rank-major, tagged with the number
+    of source ranks."""
+    w = uniform_layer(name, seed, bs=bs * sources, **kw)
+    w.meta["sources"] = sources
+    return w
+
+
 def _static_layer(name, seed, **kw):
     """A uniform layer with static int8 quantization (quantMode 1): per-instance
     static scales U(10, 40), so x ~ N(0, 1) fills much of the int8 range and
@@ -206,6 +215,12 @@ WORKLOADS = {
     # The Bs 512 layer with static int8 quantization and per-instance scales.
     "deepseek_decode_bs512_static": dict(builder=_static_layer, seed=1, bs=512, hidden=7168,
                                          num_experts=256, top_k=8, ep_world_size=32, shared=True),
+    # All ranks as sources: the DeepSeek-like layer on 8 simulated ranks (32
+    # experts each), every rank sending its own Bs = 512 tokens (4096 tokens,
+    # 32768 copies).
+    "deepseek_ep8_all_ranks": dict(builder=_all_ranks_layer, seed=1, bs=512, sources=8, hidden=7168,
+                                   num_experts=256, top_k=8, ep_world_size=8, quant_mode=2, smooth=True,
+                                   shared=True),
     # Zipf(1.2) routing over 128 experts, 160 instances on 16 ranks, mxfp8.
     "skewed_eplb": dict(builder=_skewed_eplb, seed=2, bs=512),
     # Largest shapes: H 8192, 1024 experts, K 16, 256 ranks, per-128-tile int8,
