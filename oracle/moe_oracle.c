@@ -385,3 +385,30 @@ void orc_combine_add_rmsnorm(int32_t bs, int32_t hidden, int32_t top_k,
     }
     free(x);
 }
+
+/* The plain combine paired with the dispatch (the CombineV2 series named on
+ * the dispatch page; READING R23): the first line of the formula above and
+ * nothing after it,
+ *   combineOut = Sum_k(expertScales * ataOut + expertScales * sharedExpertX),
+ * rounded to bf16 once. */
+void orc_combine(int32_t bs, int32_t hidden, int32_t top_k,
+                 const uint16_t *expand_x_bf16, const int32_t *expand_idx,
+                 const float *expert_scales, const uint16_t *shared_x,
+                 uint16_t *out_bf16, double *out_f64) {
+    const int H = hidden;
+    for (int i = 0; i < bs; ++i) {
+        for (int h = 0; h < H; ++h) {
+            double c = 0.0;
+            for (int k = 0; k < top_k; ++k) {
+                int row = expand_idx[(size_t)i * top_k + k];
+                if (row < 0) continue;
+                double s = (double)expert_scales[(size_t)i * top_k + k];
+                double ata = (double)bf16_to_float(expand_x_bf16[(size_t)row * H + h]);
+                double sh = shared_x ? (double)bf16_to_float(shared_x[(size_t)i * H + h]) : 0.0;
+                c += s * ata + s * sh;
+            }
+            if (out_bf16) out_bf16[(size_t)i * H + h] = orc_bf16_from_double(c);
+            if (out_f64) out_f64[(size_t)i * H + h] = c;
+        }
+    }
+}

@@ -74,6 +74,13 @@ void orc_combine_add_rmsnorm(int32_t bs, int32_t hidden, int32_t top_k,
 uint8_t orc_e4m3_encode(float v);   /* round-to-nearest-even, saturating */
 uint16_t orc_bf16_from_double(double v); /* round-to-nearest-even */
 
+/* The plain combine (CombineV2 series): combineOut only, no residual and no
+ * RMSNorm.  out_bf16 / out_f64 may be NULL. */
+void orc_combine(int32_t bs, int32_t hidden, int32_t top_k,
+                 const uint16_t *expand_x_bf16, const int32_t *expand_idx,
+                 const float *expert_scales, const uint16_t *shared_x,
+                 uint16_t *out_bf16, double *out_f64);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,6 +60,8 @@ def lib():
             L.orc_combine_add_rmsnorm.restype = None
             L.orc_combine_add_rmsnorm.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, f64,
                                                   vp, vp, vp, vp, vp]
+            L.orc_combine.restype = None
+            L.orc_combine.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
             L.orc_e4m3_encode.restype = ctypes.c_uint8
             L.orc_e4m3_encode.argtypes = [f32]
             L.orc_bf16_from_double.restype = ctypes.c_uint16
@@ -156,6 +158,22 @@ def combine_add_rmsnorm(expand_x_bf16, expand_idx, expert_scales, residual_x, ga
     lib().orc_combine_add_rmsnorm(bs, H, k, _p(ex), _p(idx), _p(sc), _p(sh), _p(res), _p(g),
                                   float(norm_eps), _p(y), _p(xo), _p(rstd), _p(y64), _p(x64))
     return dict(y=y, x_out=xo, rstd=rstd, y_f64=y64, x_f64=x64)
+
+
+def combine(expand_x_bf16, expand_idx, expert_scales, shared_x=None):
+    """The plain combine (CombineV2 series): combineOut = sum_k (s_k * row_k +
+    s_k * shared) per token, no residual, no RMSNorm.  Returns out (bf16
+    bits) and out_f64."""
+    ex = _c(expand_x_bf16, np.uint16)
+    idx = _c(expand_idx, np.int32)
+    sc = _c(expert_scales, np.float32)
+    sh = _c(shared_x, np.uint16)
+    bs, k = idx.shape
+    H = ex.shape[1]
+    out = np.empty((bs, H), np.uint16)
+    o64 = np.empty((bs, H), np.float64)
+    lib().orc_combine(bs, H, k, _p(ex), _p(idx), _p(sc), _p(sh), _p(out), _p(o64))
+    return dict(out=out, out_f64=o64)
 
 
 def e4m3_encode(values):

@@ -240,6 +240,28 @@ def test_sources_order_and_additivity(orc):
             np.testing.assert_array_equal(mine, p["src_of_row"][p["offsets"][e]:p["offsets"][e + 1]])
 
 
+def test_plain_combine_closed_form(orc):
+    """The plain combine (READING R23) on rows with closed forms: expert row k
+    is the constant c_k, the shared row the constant d, so every element is
+    sum_k w_k (c_k + d); a pruned copy (-1) adds nothing; and it equals the
+    Add+RMSNorm combine's x minus the residual."""
+    H, K = 1024, 3
+    c = [1.5, -2.0, 0.25]
+    d = 0.5
+    ex = np.stack([np.full(H, v, np.float32) for v in c])
+    idx = np.array([[0, 1, 2], [2, -1, 0]], np.int32)
+    w = np.array([[0.5, 0.25, 0.25], [0.125, 0.5, 0.375]], np.float32)
+    sh = np.full((2, H), d, np.float32)
+    out = orc.combine(bits(ex), idx, w, shared_x=bits(sh))
+    want = [0.5 * (1.5 + d) + 0.25 * (-2.0 + d) + 0.25 * (0.25 + d), 0.125 * (0.25 + d) + 0.375 * (1.5 + d)]
+    for i in range(2):
+        assert np.all(out["out_f64"][i] == want[i])
+    res = np.zeros((2, H), np.float32)
+    full = orc.combine_add_rmsnorm(bits(ex), idx, w, bits(res), bits(np.ones(H, np.float32)), 1e-6,
+                                   shared_x=bits(sh))
+    np.testing.assert_array_equal(out["out_f64"], full["x_f64"])
+
+
 def test_static_int8_worked_rows(orc):
     """quantMode 1 on hand-derived rows (scale (1,)): rounding half to even,
     saturation to [-128, 127], and the NaN of 0 * inf casting to 0."""
