@@ -48,7 +48,7 @@ EXPORTS = (
     "moe_workspace_init", "moe_read_device_error", "moe_clear_device_error", "moe_status_string",
     "moe_update_expert_workspace_size", "moe_update_expert",
     "moe_dispatch_workspace_size", "moe_dispatch",
-    "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm",
+    "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm", "moe_combine",
     "moe_dispatch_noalloc",
 )
 
@@ -264,6 +264,25 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
     _check("moe_combine_add_rmsnorm", lib.moe_combine_add_rmsnorm(
         ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x),
         _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")), _ptr(out.get("rstd")),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def combine(expand_x, expand_idx, expert_scales, shared_x=None, workspace=None, out=None, stream=None, sources=1):
+    """moe_combine (the plain CombineV2-series combine): combineOut [bs, H] bf16."""
+    _req(expand_x, "expand_x", torch.bfloat16)
+    rows, H = expand_x.shape
+    _req(expand_idx, "expand_idx", torch.int32)
+    bs, k = expand_idx.shape
+    _req(expert_scales, "expert_scales", torch.float32, (bs, k))
+    _opt(shared_x, "shared_x", torch.bfloat16, (bs, H))
+    if out is None:
+        out = torch.empty((bs, H), dtype=torch.bfloat16, device=expand_x.device)
+    _req(out, "out", torch.bfloat16, (bs, H))
+    p = CombineParams(_per_source(bs, sources, "combine"), H, k, rows, 0.0, int(sources))
+    ws = workspace if workspace is not None else new_workspace(expand_x.device, stream)
+    _check("moe_combine", lib.moe_combine(
+        ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x), _ptr(out),
         _ptr(ws), ws.numel(), _stream(stream)))
     return out
 

@@ -38,7 +38,8 @@ struct CombineArgs {
 // thread owns exactly kCbVecs = 4 vectors when 32 * 4 divides H / 8.
 constexpr int kCbVecs = 4;
 
-template <int KMAX, bool SHARED, int NT>
+// NORM false: the plain combine (combineOut to y; no residual, no norm).
+template <int KMAX, bool SHARED, int NT, bool NORM>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(CombineArgs a) {
     __shared__ int s_row[16];
     __shared__ float s_w[16];
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
 #pragma unroll
         for (int k = 0; k < KMAX; ++k)
             if (row[k] >= 0) rv[k] = ld_stream(a.expand_x + (size_t)row[k] * H + p * 8);
-        const uint4 res = ld_stream(a.residual + tok + p * 8);
+        uint4 res = make_uint4(0, 0, 0, 0);
+        if constexpr (NORM) res = ld_stream(a.residual + tok + p * 8);
         uint4 sh = make_uint4(0, 0, 0, 0);
         if constexpr (SHARED) sh = ld_stream(a.shared_x + tok + p * 8);
         float acc[8];
@@ -110,6 +112,21 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
         }
     }
 
+    if constexpr (!NORM) {  // the plain combine: combineOut, rounded to bf16 once
+        pdl_launch_dependents();
+#pragma unroll
+        for (int j = 0; j < kCbVecs; ++j) {
+            const int p = t + j * NT;
+            if (p >= V) continue;
+            uint4 o;
+            o.x = pack_bf16x2(xs[j][0], xs[j][1]);
+            o.y = pack_bf16x2(xs[j][2], xs[j][3]);
+            o.z = pack_bf16x2(xs[j][4], xs[j][5]);
+            o.w = pack_bf16x2(xs[j][6], xs[j][7]);
+            st_v4(a.y + tok + p * 8, o);
+        }
+        return;
+    }
     const float tot = block_sum<NT / 32>(ss, s_red);
     pdl_launch_dependents();
     const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));

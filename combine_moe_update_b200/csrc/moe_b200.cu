@@ -178,27 +178,34 @@ cudaError_t launch_dispatch_token_smooth(const moe::DispatchArgs &a, cudaStream_
 }
 
 // combine: one block per token, block size from the row length.
-template <int KMAX, bool SHARED, int NT>
+template <int KMAX, bool SHARED, int NT, bool NORM>
 cudaError_t launch_combine_nt(const moe::CombineArgs &a, cudaStream_t s) {
-    auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT>;
+    auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, NORM>;
     if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
     return launch(kernel, a.bs, NT, 0, s, a);
 }
 
-template <int KMAX, bool SHARED>
+template <int KMAX, bool SHARED, bool NORM>
 cudaError_t launch_combine_tok(const moe::CombineArgs &a, cudaStream_t s) {
     switch (moe::dp_threads(a.hidden >> 3)) {
-        case 64: return launch_combine_nt<KMAX, SHARED, 64>(a, s);
-        case 128: return launch_combine_nt<KMAX, SHARED, 128>(a, s);
-        case 192: return launch_combine_nt<KMAX, SHARED, 192>(a, s);
-        case 224: return launch_combine_nt<KMAX, SHARED, 224>(a, s);
-        default: return launch_combine_nt<KMAX, SHARED, 256>(a, s);
+        case 64: return launch_combine_nt<KMAX, SHARED, 64, NORM>(a, s);
+        case 128: return launch_combine_nt<KMAX, SHARED, 128, NORM>(a, s);
+        case 192: return launch_combine_nt<KMAX, SHARED, 192, NORM>(a, s);
+        case 224: return launch_combine_nt<KMAX, SHARED, 224, NORM>(a, s);
+        default: return launch_combine_nt<KMAX, SHARED, 256, NORM>(a, s);
     }
 }
 
-template <int KMAX>
+template <int KMAX, bool NORM>
 cudaError_t launch_combine(const moe::CombineArgs &a, cudaStream_t s) {
-    return a.shared_x ? launch_combine_tok<KMAX, true>(a, s) : launch_combine_tok<KMAX, false>(a, s);
+    return a.shared_x ? launch_combine_tok<KMAX, true, NORM>(a, s) : launch_combine_tok<KMAX, false, NORM>(a, s);
+}
+
+template <bool NORM>
+cudaError_t launch_combine_k(const moe::CombineArgs &a, int top_k, cudaStream_t s) {
+    if (top_k <= 4) return launch_combine<4, NORM>(a, s);
+    if (top_k <= 8) return launch_combine<8, NORM>(a, s);
+    return launch_combine<16, NORM>(a, s);
 }
 
 }  // namespace
@@ -411,12 +418,31 @@ moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expa
     a.x_out = reinterpret_cast<uint16_t *>(x_out);
     a.rstd_out = rstd_out;
     a.err = reinterpret_cast<uint32_t *>(workspace);
-    cudaStream_t s = as_stream(cuda_stream);
-    cudaError_t e;
-    if (p->top_k <= 4) e = launch_combine<4>(a, s);
-    else if (p->top_k <= 8) e = launch_combine<8>(a, s);
-    else e = launch_combine<16>(a, s);
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_combine_k<true>(a, p->top_k, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// The plain combine (CombineV2 series): combineOut only.
+moe_status moe_combine(const moe_combine_params *p, const void *expand_x, const int32_t *expand_idx,
+                       const float *expert_scales, const void *shared_x, void *out, void *workspace,
+                       size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr || !valid_combine(*p)) return MOE_ERR_INVALID_ARG;
+    if (!expand_x || !expand_idx || !expert_scales || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(expand_x, 16) || !aligned(out, 16) || (shared_x && !aligned(shared_x, 16)) ||
+        !aligned(expand_idx, 4) || !aligned(expert_scales, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
+    moe::CombineArgs a = {};
+    a.bs = total_tokens(p->bs, p->sources);
+    a.hidden = p->hidden;
+    a.top_k = p->top_k;
+    a.expand_rows = p->expand_rows;
+    a.expand_x = reinterpret_cast<const uint16_t *>(expand_x);
+    a.expand_idx = expand_idx;
+    a.scales = expert_scales;
+    a.shared_x = reinterpret_cast<const uint16_t *>(shared_x);
+    a.y = reinterpret_cast<uint16_t *>(out);
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    return launch_combine_k<false>(a, p->top_k, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // ------------------------------------------------------- dispatch, no alloc ---

@@ -6,7 +6,8 @@
  *   aclnnMoeUpdateExpert                  -> moe_update_expert
  *   aclnnMoeDistributeDispatchV2          -> moe_dispatch
  *   aclnnMoeDistributeCombineAddRmsNorm   -> moe_combine_add_rmsnorm
- * and, like them, come in two phases: *_workspace_size() checks the
+ * (with moe_combine, the plain CombineV2-series combine that the dispatch
+ * page pairs it with) and, like them, come in two phases: *_workspace_size() checks the
  * parameters and sizes the workspace, then the call itself runs on a CUDA
  * stream ("函数原型" / "Parameters" / "Returns" sections of each page).
  *
@@ -256,6 +257,18 @@ MOE_API moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const vo
                                    const void *shared_x, const void *residual_x, const void *gamma,
                                    void *y, void *x_out, float *rstd_out, void *workspace,
                                    size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * The plain combine of the CombineV2 series, which the dispatch page names as
+ * its pairing (aclnnMoeDistributeDispatchV2, constraints; the formula is the
+ * first line of the one above, with no residual and no norm):
+ *   out[i] = sum over kept k of (s_ik * expand_x[expand_idx[i,k]] + s_ik * shared_x[i])
+ * accumulated in fp32 and rounded to bf16 once.  Parameters as for
+ * moe_combine_add_rmsnorm (norm_eps is not used); out is [bs, H] bf16.
+ */
+MOE_API moe_status moe_combine(const moe_combine_params *p, const void *expand_x, const int32_t *expand_idx,
+                               const float *expert_scales, const void *shared_x, void *out, void *workspace,
+                               size_t workspace_bytes, void *cuda_stream);
 
 /* ------------------------------------------------------------------------ */
 /* moe_dispatch_noalloc -- moe_dispatch without a caller-provided workspace  */

@@ -104,6 +104,22 @@ def test_parity_random_replicated_tables(B, seed):
     assert_parity(w, run_gpu(w, B), run_oracle(w))
 
 
+@pytest.mark.parametrize("name,shared", [("deepseek_decode", True), ("max_shape", False), ("tiny", False)])
+def test_plain_combine(B, name, shared):
+    """moe_combine (the plain CombineV2-series combine): combineOut only,
+    against the oracle on the rows dispatch produced."""
+    w = gen.make(name, bs=64 if name != "tiny" else None)
+    g = run_gpu(w, B)
+    ex = dev_bf16(w.expert_out)
+    sc = dev(w.expert_scales)
+    sh = dev_bf16(w.shared_x) if (shared and w.shared_x is not None) else None
+    out = B.combine(ex, dev(g["expand_idx"]), sc, shared_x=sh)
+    torch.cuda.synchronize()
+    o = orc.combine(w.expert_out, g["expand_idx"], w.expert_scales,
+                    shared_x=w.shared_x if sh is not None else None)
+    assert_close_bf16(host(out), o["out_f64"], what="combineOut")
+
+
 @pytest.mark.parametrize("bs,S,E,K,H,ws,mode,smooth", [
     (100, 3, 24, 5, 1168, 6, 3, True),        # 1500 copies: the single-pass route over three sources
     (512, 3, 64, 6, 1024, 8, 2, True),        # 9216 copies: the three-pass route, a ragged last slice
