@@ -59,15 +59,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     return ok != 0;
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
-// Barrier over the first `count` threads of the block (named barrier `id`,
-// 1..15; id 0 is __syncthreads).  count must be a multiple of 32.
-__device__ __forceinline__ void named_barrier(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 // Wait for phase `phase` of an mbarrier, giving up after a bounded number of
 // polls (each poll may itself suspend for a while).  Returns false on
@@ -133,29 +125,12 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
 
 // A bf16 pair (one 32-bit word, element 0 in the low half) as an fp32 pair.
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
     return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-// cp.async (16 bytes, global -> shared, bypassing L1) and its group control.
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // bf16 pair (one 32-bit word, element 0 in the low half) -> two floats, exact.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -240,20 +215,9 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Block-wide max / sum.  s_red holds one float per warp.  Two barriers, so
-// the buffer can be reused by the next call.
-template <int NWARPS>
-__device__ __forceinline__ float block_max(float v, float *s_red) {
-    v = warp_max(v);
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float r = s_red[0];
-#pragma unroll
-    for (int w = 1; w < NWARPS; ++w) r = fmaxf(r, s_red[w]);
-    __syncthreads();
-    return r;
-}
-
+// Block-wide sum.  s_red holds one float per warp; the warp sums are added
+// in a fixed order, so the result is the same on every run.  Two barriers,
+// so the buffer can be reused by the next call.
 template <int NWARPS>
 __device__ __forceinline__ float block_sum(float v, float *s_red) {
     v = warp_sum(v);
