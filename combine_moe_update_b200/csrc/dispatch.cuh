@@ -200,6 +200,110 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
     }
 }
 
+// ----------------------------------------------------------- block route ---
+//
+// For a small call (at most kFusedRouteMax copies) every token block
+// computes the rows of its own K copies itself and no ordering kernel runs,
+// which saves a launch and a dependency on the critical path.  A copy's row is its position in (instance,
+// token, k) order.  The block builds, in shared memory, the histogram of all
+// sent copies per instance and the histogram of the copies of earlier tokens
+// (plain atomic adds: counts do not depend on order), prefix-sums the first
+// into bucket offsets, and takes
+//   row = offset[e] + (copies of earlier tokens on e)
+//         + (this token's earlier copies on e),
+// the last from __match_any_sync over the token's K lanes.  Every block gets
+// the same counts, so the rows are the same on every run.  Block 0 also
+// writes counts and offsets.  Every block reads all the call's ids, so this
+// pays only for small calls: larger ones use route_kernel.
+
+constexpr int kMaxInstances = 1024;
+constexpr int kFusedRouteMax = 1024;  // copies up to which the token blocks route themselves
+
+template <int EMAX>
+struct RouteSmemT {
+    int cnt[EMAX];     // sent copies per instance
+    int before[EMAX];  // sent copies of earlier tokens per instance
+    int off[EMAX];     // exclusive prefix of cnt
+    int warp[32];
+    int key[32];       // this token's copy keys, by k
+    int row[32];       // this token's rows, by k (-1: not sent)
+};
+using RouteSmem = RouteSmemT<kMaxInstances>;
+
+template <int NT, class RS>
+__device__ __forceinline__ void block_route_clear(RS &rs, int E) {
+    for (int e = threadIdx.x; e < E; e += NT) {
+        rs.cnt[e] = 0;
+        rs.before[e] = 0;
+    }
+}
+
+// Call after pdl_wait, with block_route_clear done and a barrier between.
+// key0: for the threads of warp 0, copy_key of this token's copy k = lane
+// (-1 for lanes >= K).  Leaves rs.key and rs.row filled, after a barrier.
+template <int NT, class RS>
+__device__ void block_route(const DispatchArgs &a, int i, RS &rs, int key0) {
+    const int t = threadIdx.x, E = a.num_instances, K = a.top_k, N = a.bs * K, mine0 = i * K;
+    constexpr int U = 8;
+    for (int j0 = 0; j0 < N; j0 += NT * U) {  // loads unconditional (clamped), so all are in flight together
+        int id[U];
+        uint32_t ms[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) id[u] = __ldg(a.ids + min(j0 + u * NT + t, N - 1));
+        if (a.mask) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) ms[u] = __ldg(a.mask + min(j0 + u * NT + t, N - 1));
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; ++u) ms[u] = 1;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int j = j0 + u * NT + t;
+            if (j < N && ms[u] != 0 && id[u] >= 0 && id[u] < E) {
+                atomicAdd(&rs.cnt[id[u]], 1);
+                if (j < mine0) atomicAdd(&rs.before[id[u]], 1);
+            }
+        }
+    }
+    __syncthreads();
+    // exclusive scan of cnt: thread t owns P consecutive instances
+    const int P = (E + NT - 1) / NT;
+    int sum = 0;
+    for (int u = 0; u < P; ++u) {
+        const int e = t * P + u;
+        if (e < E) sum += rs.cnt[e];
+    }
+    const int incl = block_inclusive_scan(sum, rs.warp);
+    int run = incl - sum;
+    for (int u = 0; u < P; ++u) {
+        const int e = t * P + u;
+        if (e < E) {
+            rs.off[e] = run;
+            if (i == 0) {
+                a.counts[e] = rs.cnt[e];
+                a.offsets[e] = run;
+            }
+            run += rs.cnt[e];
+        }
+    }
+    if (i == 0 && t == NT - 1) a.offsets[E] = incl;  // the total
+    __syncthreads();
+    if (t < 32) {
+        const unsigned peers = __match_any_sync(kFull, key0);
+        int row = -1;
+        if (key0 >= 0) row = rs.off[key0] + rs.before[key0] + __popc(peers & ((1u << t) - 1u));
+        if (key0 == -2) raise_error(a.err, kDevBadId);
+        rs.key[t] = key0;
+        rs.row[t] = row;
+        if (t < K) {
+            a.expand_idx[mine0 + t] = row;
+            if (row >= 0) a.src_of_row[row] = mine0 + t;
+        }
+    }
+    __syncthreads();
+}
+
 // ---------------------------------------------------- route, many copies ---
 //
 // Past 8192 copies (several source ranks), rebuilding the whole histogram in
@@ -609,12 +713,16 @@ __device__ __forceinline__ void load_row(const uint16_t *row, int V, uint4 (&xv)
 
 // --------------------------------------------------------- token kernel ---
 
-template <int MODE, int NT>
+// FUSED: the block routes its own copies (block_route, small calls) instead
+// of reading the rows route_kernel wrote.
+template <int MODE, int NT, bool FUSED>
 __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
     __shared__ float s_red[NT / 32];
     __shared__ int s_row[16];
+    __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
     const int i = blockIdx.x, t = threadIdx.x;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
+    if constexpr (FUSED) block_route_clear<NT>(rs, a.num_instances);
 
     // inputs of the call only: safe before the route kernel is done
     uint4 xv[kDpVecs];
@@ -657,11 +765,18 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         }
     }
 
-    pdl_wait();  // the rows come from route_kernel
-    if (t < K) s_row[t] = a.expand_idx[i * K + t];
-    __syncthreads();
+    if constexpr (FUSED) {
+        __syncthreads();  // the counters are clear
+        pdl_wait();       // the instance ids may come from the previous kernel
+        block_route<NT>(a, i, rs, t < 32 && t < K ? copy_key(a, i * K + t) : -1);
+        pdl_launch_dependents();
+    } else {
+        pdl_wait();  // the rows come from route_kernel
+        if (t < K) s_row[t] = a.expand_idx[i * K + t];
+        __syncthreads();
+    }
     for (int k = 0; k < K; ++k) {
-        const int row = s_row[k];
+        const int row = FUSED ? rs.row[k] : s_row[k];
         if (row < 0) continue;
         if constexpr (MODE == 0) {
             uint16_t *dst = reinterpret_cast<uint16_t *>(a.expand_x) + (size_t)row * H;
@@ -699,13 +814,14 @@ __host__ __device__ inline int smooth_smem_floats(int hidden) {
     return hidden > NT * kDpVecs * 8 ? hidden : NT * kDpVecs * 8;
 }
 
-template <int MODE, int NT>
+template <int MODE, int NT, bool FUSED>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_kernel(DispatchArgs a) {
     constexpr int NW = NT / 32;
     extern __shared__ __align__(128) float s_smooth[];  // the current copy's smooth row, then zeros
     __shared__ float s_red[2][NW];
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_key[16], s_pos[16], s_row[16], s_ns;
+    __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
     const int i = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
     const uint32_t row_bytes = (uint32_t)H * sizeof(float);  // a multiple of 16 (H % 16 == 0)
@@ -724,17 +840,24 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         if (swap) xv[q] = make_uint4(xv[q].z, xv[q].w, xv[q].x, xv[q].y);
     const float *s_first = s_smooth + (swap ? 4 : 0), *s_second = s_smooth + (swap ? 0 : 4);
     for (int e = H + t; e < smooth_smem_floats<NT>(H); e += NT) s_smooth[e] = 0.0f;
+    if constexpr (FUSED) {
+        block_route_clear<NT>(rs, a.num_instances);
+        if (t == 0) mbar_init(&s_bar, 1);
+        __syncthreads();
+        pdl_wait();  // the instance ids may come from the previous kernel
+    }
+    int key0 = -1;
     if (w == 0) {  // the sent copies, in k order: instance and position k
-        const int key = lane < K ? copy_key(a, i * K + lane) : -1;
-        const unsigned sent = __ballot_sync(kFull, key >= 0);
-        if (key >= 0) {
+        key0 = lane < K ? copy_key(a, i * K + lane) : -1;
+        const unsigned sent = __ballot_sync(kFull, key0 >= 0);
+        if (key0 >= 0) {
             const int c = __popc(sent & ((1u << lane) - 1u));
-            s_key[c] = key;
+            s_key[c] = key0;
             s_pos[c] = lane;
         }
         if (lane == 0) {
             s_ns = __popc(sent);
-            mbar_init(&s_bar, 1);
+            if constexpr (!FUSED) mbar_init(&s_bar, 1);
         }
     }
     __syncthreads();
@@ -744,6 +867,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         bulk_copy_g2s(s_smooth, a.smooth + (size_t)s_key[c] * H, row_bytes, &s_bar);
     };
     if (t == 0 && ns > 0) fetch_smooth(0);
+    if constexpr (FUSED) block_route<NT>(a, i, rs, key0);  // while the first smooth row is in flight
 
     for (int c = 0; c < ns; ++c) {
         const bool landed = mbar_wait_bounded(&s_bar, c & 1);
@@ -790,7 +914,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         } else {
             quantize_local<MODE, NT>(xf, V, qv, seg);
         }
-        if (c == 0) {
+        if (!FUSED && c == 0) {
             pdl_wait();  // the rows come from the route kernel
             if (t < K) s_row[t] = a.expand_idx[i * K + t];
             __syncthreads();
@@ -798,7 +922,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
 #pragma unroll
         for (int q = 0; q < kDpVecs; ++q)
             if (swap) qv[q] = make_uint2(qv[q].y, qv[q].x);
-        write_row<MODE, NT>(a, s_row[s_pos[c]], V, qv, seg, row_scale);
+        write_row<MODE, NT>(a, FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], V, qv, seg, row_scale);
     }
 }
 

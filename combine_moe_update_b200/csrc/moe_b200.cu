@@ -148,22 +148,34 @@ cudaError_t launch_by_threads(const moe::DispatchArgs &a, cudaStream_t s) {
     }
 }
 
+// Small calls (at most kFusedRouteMax copies) use the instantiations whose
+// blocks route their own copies, and no route kernel runs.
+inline bool fused_route(const moe::DispatchArgs &a) { return a.bs * a.top_k <= moe::kFusedRouteMax; }
+
 template <int MODE, int NT>
 struct TokenLaunch {
-    static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
-        auto kernel = moe::dispatch_token_kernel<MODE, NT>;
+    template <bool FUSED>
+    static cudaError_t go_(const moe::DispatchArgs &a, cudaStream_t s) {
+        auto kernel = moe::dispatch_token_kernel<MODE, NT, FUSED>;
         if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
         return launch(kernel, a.bs, NT, 0, s, a);
+    }
+    static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
+        return fused_route(a) ? go_<true>(a, s) : go_<false>(a, s);
     }
 };
 
 template <int MODE, int NT>
 struct TokenSmoothLaunch {
-    static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
-        auto kernel = moe::dispatch_token_smooth_kernel<MODE, NT>;
+    template <bool FUSED>
+    static cudaError_t go_(const moe::DispatchArgs &a, cudaStream_t s) {
+        auto kernel = moe::dispatch_token_smooth_kernel<MODE, NT, FUSED>;
         const size_t smem = (size_t)moe::smooth_smem_floats<NT>(a.hidden) * sizeof(float);
         if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
         return launch(kernel, a.bs, NT, smem, s, a);
+    }
+    static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
+        return fused_route(a) ? go_<true>(a, s) : go_<false>(a, s);
     }
 };
 
@@ -342,7 +354,9 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     cudaStream_t s = as_stream(cuda_stream);
 
     const int copies = a.bs * p->top_k;
-    if (copies <= kRouteSinglePassMax) {
+    if (copies <= moe::kFusedRouteMax) {
+        // the scatter blocks route their own copies (no route kernel)
+    } else if (copies <= kRouteSinglePassMax) {
         const int slices = moe::route_slices(copies);
         const size_t rsmem = moe::route_smem_bytes(p->num_instances);
         if (!ensure_smem(moe::route_kernel, rsmem)) return MOE_ERR_CUDA;
