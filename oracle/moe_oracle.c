@@ -412,3 +412,46 @@ void orc_combine(int32_t bs, int32_t hidden, int32_t top_k,
         }
     }
 }
+
+/* ---------------------------------------------------------------------- */
+/* Between dispatch and combine: the instances' grouped matmul             */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * READING R24.  The pages name the expert step only by its place, between
+ * the dispatch and the combine ("AllToAllV" out and back), and do not define
+ * it.  Taken here as the one contraction that consumes the dispatch's output:
+ * deployed instance e applies its own weight to the rows it received,
+ * rows [expert_offsets[e], expert_offsets[e+1]) of expand_x.  The rows hold
+ * int8 codes q with one dequantization factor each (quantMode 2:
+ * x ~= q * dyn_scale); the weight is int8 w with one factor per output
+ * channel (W[e][n][h] ~= w[e][n][h] * w_scale[e][n]).  Then
+ *   acc[r][n] = Sum_h q[r][h] * w[e][n][h]            (an exact integer)
+ *   out[r][n] = acc[r][n] * dyn_scale[r] * w_scale[e][n],  rounded to bf16 once.
+ * Offsets must satisfy 0 <= off[0] <= ... <= off[E] <= rows; otherwise
+ * nothing is written and ORC_ERR_BAD_ID is returned.  Rows outside
+ * [off[0], off[E]) are not written.
+ */
+uint32_t orc_grouped_matmul(int32_t rows, int32_t hidden, int32_t out_dim, int32_t num_instances,
+                            const int8_t *expand_x, const float *dyn_scales,
+                            const int32_t *expert_offsets, const int8_t *weight,
+                            const float *weight_scales, uint16_t *out_bf16, double *out_f64) {
+    const int H = hidden, N = out_dim, E = num_instances;
+    if (expert_offsets[0] < 0 || expert_offsets[E] > rows) return ORC_ERR_BAD_ID;
+    for (int e = 0; e < E; ++e)
+        if (expert_offsets[e + 1] < expert_offsets[e]) return ORC_ERR_BAD_ID;
+    for (int e = 0; e < E; ++e) {
+        const int8_t *w = weight + (size_t)e * N * H;
+        for (int r = expert_offsets[e]; r < expert_offsets[e + 1]; ++r) {
+            const int8_t *q = expand_x + (size_t)r * H;
+            for (int n = 0; n < N; ++n) {
+                int64_t acc = 0;
+                for (int h = 0; h < H; ++h) acc += (int64_t)q[h] * (int64_t)w[(size_t)n * H + h];
+                double v = (double)acc * (double)dyn_scales[r] * (double)weight_scales[(size_t)e * N + n];
+                if (out_bf16) out_bf16[(size_t)r * N + n] = orc_bf16_from_double(v);
+                if (out_f64) out_f64[(size_t)r * N + n] = v;
+            }
+        }
+    }
+    return 0;
+}

@@ -81,6 +81,18 @@ void orc_combine(int32_t bs, int32_t hidden, int32_t top_k,
                  const float *expert_scales, const uint16_t *shared_x,
                  uint16_t *out_bf16, double *out_f64);
 
+/* The instances' grouped matmul between dispatch and combine (READING R24):
+ * out[r][n] = (Sum_h q[r][h] * w[e][n][h]) * dyn_scales[r] * weight_scales[e][n]
+ * for the rows r of instance e, [expert_offsets[e], expert_offsets[e+1]).
+ * expand_x [rows, hidden] int8, weight [E, out_dim, hidden] int8,
+ * weight_scales [E, out_dim] f32, out [rows, out_dim].  Returns
+ * ORC_ERR_BAD_ID (and writes nothing) for offsets that are not a
+ * non-decreasing sequence in [0, rows].  out_bf16 / out_f64 may be NULL. */
+uint32_t orc_grouped_matmul(int32_t rows, int32_t hidden, int32_t out_dim, int32_t num_instances,
+                            const int8_t *expand_x, const float *dyn_scales,
+                            const int32_t *expert_offsets, const int8_t *weight,
+                            const float *weight_scales, uint16_t *out_bf16, double *out_f64);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,8 @@ def lib():
             L.orc_combine.restype = None
             L.orc_combine.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
             L.orc_e4m3_encode.restype = ctypes.c_uint8
+            L.orc_grouped_matmul.restype = ctypes.c_uint32
+            L.orc_grouped_matmul.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
             L.orc_e4m3_encode.argtypes = [f32]
             L.orc_bf16_from_double.restype = ctypes.c_uint16
             L.orc_bf16_from_double.argtypes = [f64]
@@ -174,6 +176,27 @@ def combine(expand_x_bf16, expand_idx, expert_scales, shared_x=None):
     o64 = np.empty((bs, H), np.float64)
     lib().orc_combine(bs, H, k, _p(ex), _p(idx), _p(sc), _p(sh), _p(out), _p(o64))
     return dict(out=out, out_f64=o64)
+
+
+def grouped_matmul(expand_x, dyn_scales, expert_offsets, weight, weight_scales, out=None):
+    """The instances' grouped matmul between dispatch and combine: rows
+    [off[e], off[e+1]) of expand_x (int8) times instance e's int8 weight
+    [N, H], scaled by each row's dyn_scale and each output channel's weight
+    scale.  ``out`` (bf16 bits, [rows, N]) may be given pre-filled: rows the
+    call does not own keep their content.  Returns out, out_f64 (NaN where
+    not written) and the error word."""
+    ex = _c(expand_x, np.int8)
+    ds = _c(dyn_scales, np.float32)
+    off = _c(expert_offsets, np.int32)
+    w = _c(weight, np.int8)
+    ws = _c(weight_scales, np.float32)
+    rows, H = ex.shape
+    E, N = w.shape[0], w.shape[1]
+    assert w.shape == (E, N, H) and ws.shape == (E, N) and off.shape == (E + 1,) and ds.shape == (rows,)
+    out = np.zeros((rows, N), np.uint16) if out is None else _c(out, np.uint16).copy()
+    o64 = np.full((rows, N), np.nan, np.float64)
+    err = lib().orc_grouped_matmul(rows, H, N, E, _p(ex), _p(ds), _p(off), _p(w), _p(ws), _p(out), _p(o64))
+    return dict(out=out, out_f64=o64, err=int(err))
 
 
 def e4m3_encode(values):

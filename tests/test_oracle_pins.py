@@ -575,3 +575,103 @@ def test_combine_shared_expert_weighting(orc):
     sh = gen.bf16_to_f32(w.shared_x).astype(np.float64)
     np.testing.assert_array_equal(out["x_f64"][0], sh[0])            # 8 * 0.125 = 1
     np.testing.assert_array_equal(out["x_f64"][1], sh[1] * 0.625)    # 5 kept copies
+
+
+# --------------------------------------------------------------------------
+# grouped matmul between dispatch and combine (reading R24)
+# --------------------------------------------------------------------------
+
+def _gmm_inputs(rng, counts, H, N, lo, hi, spare=2):
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = int(off[-1]) + spare
+    q = rng.integers(lo, hi, (rows, H), dtype=np.int8, endpoint=True)
+    w = rng.integers(lo, hi, (len(counts), N, H), dtype=np.int8, endpoint=True)
+    return off, q, w
+
+
+def test_grouped_matmul_small_integers_equal_numpy_matmul(orc):
+    """Unit scales and |acc| <= 144: every output is an integer that bf16 holds
+    exactly, so each instance's block must equal numpy's integer matmul of its
+    rows with its own weight, bit for bit; empty instances are skipped and
+    rows past the last offset keep their content."""
+    rng = np.random.default_rng(11)
+    counts = [3, 0, 5, 1, 0, 4]
+    H, N = 16, 24
+    off, q, w = _gmm_inputs(rng, counts, H, N, -3, 3)
+    E, rows = len(counts), q.shape[0]
+    sentinel = np.full((rows, N), 0x7FC1, np.uint16)
+    r = orc.grouped_matmul(q, np.ones(rows, np.float32), off, w, np.ones((E, N), np.float32), out=sentinel)
+    assert r["err"] == 0
+    for e in range(E):
+        blk = q[off[e]:off[e + 1]].astype(np.int64) @ w[e].astype(np.int64).T
+        assert np.abs(blk).max(initial=0) <= 144
+        want = blk.astype(np.float32).astype(ml_dtypes.bfloat16).view(np.uint16)
+        np.testing.assert_array_equal(r["out"][off[e]:off[e + 1]], want)
+    np.testing.assert_array_equal(r["out"][off[-1]:], sentinel[off[-1]:])
+
+
+def test_grouped_matmul_scaled_against_numpy(orc):
+    """Full-range codes and weights with random row and channel scales: the
+    f64 result is numpy's int64 matmul times the two scales (exact integers
+    below 2^53, so only the two products round), and the bf16 output is that
+    value rounded by ml_dtypes."""
+    rng = np.random.default_rng(12)
+    counts = [7, 2, 0, 9]
+    H, N = 64, 32
+    off, q, w = _gmm_inputs(rng, counts, H, N, -128, 127)
+    E, rows = len(counts), q.shape[0]
+    ds = rng.uniform(1e-3, 2e-2, rows).astype(np.float32)
+    ws = rng.uniform(1e-3, 1e-2, (E, N)).astype(np.float32)
+    r = orc.grouped_matmul(q, ds, off, w, ws)
+    assert r["err"] == 0
+    for e in range(E):
+        s = slice(off[e], off[e + 1])
+        acc = q[s].astype(np.int64) @ w[e].astype(np.int64).T
+        want = acc.astype(np.float64) * ds[s].astype(np.float64)[:, None] * ws[e].astype(np.float64)[None, :]
+        np.testing.assert_allclose(r["out_f64"][s], want, rtol=1e-15, atol=0)
+        np.testing.assert_array_equal(r["out"][s], want.astype(ml_dtypes.bfloat16).view(np.uint16))
+
+
+def test_grouped_matmul_extreme_magnitude_closed_form(orc):
+    """H = 8192 with every code 127 and every weight -128 (instance 0) or 127
+    (instance 1): acc = -127*128*8192 = -133169152 and 127*127*8192 =
+    132128768.  With dyn = 2^-7 and weight scale 2^-10 the outputs are
+    -1016 exactly and 1008.0078125, which bf16 (spacing 4 in [512, 1024))
+    rounds to 1008."""
+    H, N = 8192, 2
+    q = np.full((3, H), 127, np.int8)
+    w = np.stack([np.full((N, H), -128, np.int8), np.full((N, H), 127, np.int8)])
+    off = np.array([0, 2, 3], np.int32)
+    r = orc.grouped_matmul(q, np.full(3, 2.0 ** -7, np.float32), off, w, np.full((2, N), 2.0 ** -10, np.float32))
+    assert r["err"] == 0
+    np.testing.assert_array_equal(r["out_f64"][:2], -1016.0)
+    np.testing.assert_array_equal(r["out_f64"][2], 132128768 * 2.0 ** -17)
+    np.testing.assert_array_equal(r["out"][:2], bits([-1016.0])[0])
+    np.testing.assert_array_equal(r["out"][2], bits([1008.0])[0])
+
+
+def test_grouped_matmul_identity_weight_dequantizes(orc):
+    """An identity weight (N = H, unit channel scales) turns the matmul into
+    the dispatch's dequantization: out[r][h] = q[r][h] * dyn[r]."""
+    rng = np.random.default_rng(13)
+    H = 48
+    q = rng.integers(-127, 127, (9, H), dtype=np.int8, endpoint=True)
+    ds = rng.uniform(1e-3, 1.0, 9).astype(np.float32)
+    eye = np.eye(H, dtype=np.int8)
+    r = orc.grouped_matmul(q, ds, np.array([0, 4, 9], np.int32), np.stack([eye, eye]), np.ones((2, H), np.float32))
+    assert r["err"] == 0
+    want = q.astype(np.float64) * ds.astype(np.float64)[:, None]
+    np.testing.assert_array_equal(r["out_f64"], want)
+    np.testing.assert_array_equal(r["out"], want.astype(ml_dtypes.bfloat16).view(np.uint16))
+
+
+@pytest.mark.parametrize("off", [[0, 3, 2, 4], [0, 1, 2, 6], [-1, 1, 2, 3]])
+def test_grouped_matmul_rejects_bad_offsets(orc, off):
+    """Offsets that decrease, overrun the rows (5 here) or start below 0 are an
+    error and nothing is written."""
+    q = np.ones((5, 16), np.int8)
+    pre = np.full((5, 16), 0x1234, np.uint16)
+    r = orc.grouped_matmul(q, np.ones(5, np.float32), np.array(off, np.int32), np.ones((3, 16, 16), np.int8),
+                           np.ones((3, 16), np.float32), out=pre)
+    assert r["err"] == orc.ERR_BAD_ID
+    np.testing.assert_array_equal(r["out"], pre)
