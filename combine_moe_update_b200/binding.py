@@ -44,12 +44,17 @@ class CombineParams(ctypes.Structure):
                 ("expand_rows", ctypes.c_int32), ("norm_eps", ctypes.c_float), ("sources", ctypes.c_int32)]
 
 
+class GmmParams(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int32), ("hidden", ctypes.c_int32), ("out_dim", ctypes.c_int32),
+                ("num_instances", ctypes.c_int32)]
+
+
 EXPORTS = (
     "moe_workspace_init", "moe_read_device_error", "moe_clear_device_error", "moe_status_string",
     "moe_update_expert_workspace_size", "moe_update_expert",
     "moe_dispatch_workspace_size", "moe_dispatch",
     "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm", "moe_combine",
-    "moe_dispatch_noalloc",
+    "moe_dispatch_noalloc", "moe_grouped_matmul_workspace_size", "moe_grouped_matmul",
 )
 
 
@@ -71,7 +76,10 @@ def _load():
     L.moe_dispatch.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_combine_add_rmsnorm_workspace_size.argtypes = [P(CombineParams), P(sz)]
     L.moe_combine_add_rmsnorm.argtypes = [P(CombineParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_combine.argtypes = [P(CombineParams), vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_dispatch_noalloc.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.moe_grouped_matmul_workspace_size.argtypes = [P(GmmParams), P(sz)]
+    L.moe_grouped_matmul.argtypes = [P(GmmParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for name in EXPORTS:
         if name != "moe_status_string":
             getattr(L, name).restype = ctypes.c_int
@@ -310,3 +318,36 @@ def dispatch_noalloc(x, instance_ids, num_instances, ep_world_size, quant_mode, 
         _ptr(out["offsets"]), _ptr(device_error), _stream(stream)))
     return out
 
+
+
+def grouped_matmul_workspace_bytes(rows, hidden, out_dim, num_instances) -> int:
+    p = GmmParams(int(rows), int(hidden), int(out_dim), int(num_instances))
+    n = ctypes.c_size_t(0)
+    _check("moe_grouped_matmul_workspace_size", lib.moe_grouped_matmul_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def grouped_matmul(expand_x, dyn_scales, expert_offsets, weight, weight_scales, out=None, workspace=None,
+                   stream=None):
+    """moe_grouped_matmul: out[r] = (expand_x[r] . weight[e]^T) * dyn_scales[r] * weight_scales[e] for the
+    rows r of each instance e, [expert_offsets[e], expert_offsets[e+1]).  expand_x [rows, H] int8,
+    weight [E, N, H] int8, weight_scales [E, N] f32; returns out [rows, N] bf16 (rows outside the
+    offsets keep whatever ``out`` held)."""
+    _req(expand_x, "expand_x", torch.int8)
+    rows, H = expand_x.shape
+    _req(weight, "weight", torch.int8)
+    E, N = weight.shape[0], weight.shape[1]
+    _req(weight, "weight", torch.int8, (E, N, H))
+    _req(weight_scales, "weight_scales", torch.float32, (E, N))
+    _req(dyn_scales, "dyn_scales", torch.float32, (rows,))
+    _req(expert_offsets, "expert_offsets", torch.int32, (E + 1,))
+    if out is None:
+        out = torch.empty((rows, N), dtype=torch.bfloat16, device=expand_x.device)
+    _req(out, "out", torch.bfloat16, (rows, N))
+    p = GmmParams(rows, H, N, E)
+    ws = workspace if workspace is not None else new_workspace(
+        expand_x.device, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
+    _check("moe_grouped_matmul", lib.moe_grouped_matmul(
+        ctypes.byref(p), _ptr(expand_x), _ptr(dyn_scales), _ptr(expert_offsets), _ptr(weight),
+        _ptr(weight_scales), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out

@@ -1,0 +1,306 @@
+// grouped_matmul.cuh -- the deployed instances' int8 matmul that sits between
+// the dispatch and the combine, on the fifth-generation tensor cores.
+//
+// The pages place an expert computation between "AllToAllV(quantOut)" (the
+// dispatch page's formula) and the gather of "ataOut" (the combine page's
+// formula) without defining it.  Built here as the one contraction that
+// consumes the dispatch output: instance e multiplies the rows it received,
+// [expert_offsets[e], expert_offsets[e+1]) of expand_x (int8 codes, one
+// dequantization factor per row), by its own int8 weight [N, H] (one factor
+// per output channel):
+//   out[r][n] = (sum_h q[r][h] * w[e][n][h]) * dyn_scale[r] * w_scale[e][n]
+// rounded to bf16.  The sum is exact: int8 x int8 products accumulate in
+// int32 (|sum| <= 8192 * 128 * 128 < 2^31).
+//
+// Design (sm_100a):
+//  * A planning kernel turns the per-instance offsets into work slots of at
+//    most 128 rows of one instance (one thread per instance, a block scan).
+//  * The matmul kernel computes one 128-channel x (<= 128 rows) tile per CTA
+//    with tcgen05.mma kind::i8, "swapped": the weight slab [128 channels, H]
+//    is the MMA's A operand (M = 128) and the slot's rows are B (N = rows
+//    rounded up to 16).  A decode batch gives an instance ~16 rows, so N
+//    follows the rows and no tensor work is spent on padding to 128 rows;
+//    every weight byte is read from HBM once per slot.
+//  * Operands are staged by TMA (cp.async.bulk.tensor, 128-byte swizzle, no
+//    multicast) through a ring of stages sized at run time from N, tracked by
+//    mbarriers; one elected thread issues both the copies and the MMAs, and
+//    tcgen05.commit frees each stage.  The int32 accumulator lives in TMEM
+//    (128 lanes = channels, N columns = rows).
+//  * The epilogue reads TMEM with tcgen05.ld (warp w owns lanes 32w..32w+31),
+//    applies the row and channel factors in fp32 and stores bf16.
+//  * Every wait is bounded; on a timeout the CTA records MOE_DEV_TIMEOUT,
+//    drains its copies in flight (again bounded), frees its TMEM and skips
+//    its stores.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kGmBM = 128;          // output channels per tile (the MMA's M)
+constexpr int kGmBN = 128;          // rows per slot at most (the MMA's N: 16..128)
+constexpr int kGmBK = 128;          // int8 contraction per stage: one 128-byte swizzled row
+constexpr int kGmBoxRows = 16;      // rows per TMA box of the row operand
+constexpr int kGmABytes = kGmBM * kGmBK;             // 16 KB of weight per stage
+constexpr int kGmPipeBytes = 96 * 1024;              // the stage ring
+constexpr int kGmMaxStages = 8;
+constexpr int kGmSmemBytes = kGmPipeBytes + 1024;    // + slack to align the ring to 1 KB
+constexpr int kGmThreads = 128;
+constexpr uint32_t kGmTmemCols = 128;                // int32 accumulator columns (>= N)
+
+struct GmmArgs {
+    int rows, hidden, out_dim, num_instances, max_slots;
+    const float *dyn;          // [rows] per-row factor
+    const int32_t *offsets;    // [E + 1]
+    const float *wscale;       // [E, N] per-channel factor
+    uint16_t *out;             // [rows, N] bf16
+    int4 *slots;               // [max_slots] {instance, first row, rows, 0}
+    int *nslots;
+    uint32_t *err;
+};
+
+__host__ __device__ inline int gmm_max_slots(int rows, int num_instances) {
+    // sum_e ceil(c_e / 128) <= sum_e (c_e + 127) / 128 < rows / 128 + E
+    return num_instances + (rows + kGmBN - 1) / kGmBN;
+}
+
+// --- planning: one block of 1024 threads, thread e = instance e ---
+__global__ void __launch_bounds__(1024) gmm_plan_kernel(GmmArgs a) {
+    __shared__ int s_warp[32];
+    __shared__ int s_bad;
+    const int e = threadIdx.x;
+    if (e == 0) s_bad = 0;
+    __syncthreads();
+    pdl_wait();  // the offsets come from the dispatch
+    int lo = 0, cnt = 0;
+    if (e < a.num_instances) {
+        lo = a.offsets[e];
+        const int hi = a.offsets[e + 1];
+        if (lo < 0 || hi < lo || hi > a.rows) s_bad = 1;
+        cnt = hi - lo;
+    }
+    __syncthreads();
+    const bool bad = s_bad != 0;
+    if (bad) cnt = 0;  // offsets that are not a non-decreasing run in [0, rows]: nothing is computed
+    const int ch = (cnt + kGmBN - 1) / kGmBN;
+    const int incl = block_inclusive_scan(ch, s_warp);
+    for (int c = 0, s = incl - ch; c < ch && s < a.max_slots; ++c, ++s)
+        a.slots[s] = make_int4(e, lo + c * kGmBN, min(kGmBN, cnt - c * kGmBN), 0);
+    if (e == (int)blockDim.x - 1) *a.nslots = min(incl, a.max_slots);
+    if (bad && e == 0) raise_error(a.err, kDevBadId);
+    pdl_launch_dependents();
+}
+
+// --- tcgen05 / TMA wrappers ---
+
+// Shared-memory matrix descriptor, K-major operand with the 128-byte swizzle:
+// rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset),
+// leading byte offset unused for this layout (encoded 1), descriptor
+// version 1, base offset 0 (every tile starts on a 1024-byte boundary).
+__device__ __forceinline__ uint64_t gm_smem_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor, kind::i8: int32 accumulator, signed A and B, both
+// K-major, M = 128, N = n (a multiple of 16, <= 256).
+__device__ __forceinline__ uint32_t gm_instr_desc(int n) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kGmBM >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 2-D tiled TMA load (no multicast); x is the innermost coordinate in
+// elements (here bytes), always a multiple of 128.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns: thread i of the warp gets lane
+// (base lane + i), columns col..col+15.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"  // in the same statement, so no use of v can precede it
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Bounded wait with a short sleep between polls, for threads that idle
+// through the main loop (about a second at most).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t phase) {
+    for (uint32_t it = 0; it < (1u << 24); ++it) {
+        if (mbar_try_wait(bar, phase)) return true;
+        __nanosleep(64);
+    }
+    return false;
+}
+
+// --- the matmul: grid (ceil(N / 128), max_slots), 128 threads ---
+__global__ void __launch_bounds__(kGmThreads, 1)
+    gmm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GmmArgs a) {
+    extern __shared__ uint8_t gm_smem_raw[];
+    __shared__ __align__(8) uint64_t s_full[kGmMaxStages];
+    __shared__ __align__(8) uint64_t s_empty[kGmMaxStages];
+    __shared__ __align__(8) uint64_t s_done;
+    __shared__ uint32_t s_tmem;
+    __shared__ int4 s_slot;
+    __shared__ int s_fail;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    // the ring starts on a 1 KB boundary (the 128-byte swizzle repeats every 1 KB)
+    uint8_t *ring = gm_smem_raw + ((1024u - (smem_u32(gm_smem_raw) & 1023u)) & 1023u);
+
+    if (t == 0) {
+        for (int s = 0; s < kGmMaxStages; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], 1);
+        }
+        mbar_init(&s_done, 1);
+        s_fail = 0;
+        tma_prefetch_map(&tm_w);
+        tma_prefetch_map(&tm_x);
+    }
+    pdl_wait();  // slots from the planning kernel; rows and factors from earlier kernels
+    if (t == 0) {
+        const int ns = *a.nslots;
+        s_slot = (int)blockIdx.y < ns ? a.slots[blockIdx.y] : make_int4(-1, 0, 0, 0);
+    }
+    __syncthreads();
+    const int4 slot = s_slot;
+    if (slot.x < 0) return;  // more slots were launched than the offsets need
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(kGmTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    const int n0 = blockIdx.x * kGmBM;
+    const int nr = slot.z;
+    const int mma_n = (nr + 15) & ~15;
+    const int nbox = mma_n / kGmBoxRows;
+    const int b_bytes = mma_n * kGmBK;
+    const int stage_bytes = kGmABytes + b_bytes;  // a multiple of 2 KB
+    const int nst = min(kGmMaxStages, kGmPipeBytes / stage_bytes);
+    const int nk = (a.hidden + kGmBK - 1) / kGmBK;
+
+    if (t == 0) {
+        const uint32_t tx = (uint32_t)stage_bytes;  // out-of-range box parts are zero-filled and still counted
+        const int wrow = slot.x * a.out_dim + n0;
+        const uint32_t idesc = gm_instr_desc(mma_n);
+        const uint32_t ring_s = smem_u32(ring);
+        int issued = 0;
+        auto issue = [&](int kb) {
+            const int s = kb % nst;
+            uint8_t *sa = ring + s * stage_bytes;
+            mbar_arrive_expect_tx(&s_full[s], tx);
+            tma_load_2d(sa, &tm_w, kb * kGmBK, wrow, &s_full[s]);
+            for (int b = 0; b < nbox; ++b)
+                tma_load_2d(sa + kGmABytes + b * kGmBoxRows * kGmBK, &tm_x, kb * kGmBK, slot.y + b * kGmBoxRows,
+                            &s_full[s]);
+        };
+        for (; issued < nst && issued < nk; ++issued) issue(issued);
+        bool ok = true;
+        int kb = 0;
+        for (; kb < nk; ++kb) {
+            const int s = kb % nst;
+            if (!mbar_wait_bounded(&s_full[s], (uint32_t)(kb / nst) & 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sa = ring_s + s * stage_bytes;
+            const uint64_t da = gm_smem_desc(sa), db = gm_smem_desc(sa + kGmABytes);
+#pragma unroll
+            for (int kk = 0; kk < kGmBK / 32; ++kk)  // K = 32 bytes per MMA: +2 in 16-byte units
+                umma_i8(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+            umma_commit(&s_empty[s]);
+            // refill the stage the previous step used, once its MMAs have read it
+            if (kb >= 1 && issued < nk) {
+                const int sp = (kb - 1) % nst;
+                if (!mbar_wait_bounded(&s_empty[sp], (uint32_t)((kb - 1) / nst) & 1u)) {
+                    ok = false;
+                    ++kb;  // step kb was consumed
+                    break;
+                }
+                issue(issued);
+                ++issued;
+            }
+        }
+        if (!ok) {
+            // drain the copies still in flight before the CTA can exit
+            for (int j = kb; j < issued; ++j) mbar_wait_bounded(&s_full[j % nst], (uint32_t)(j / nst) & 1u);
+            s_fail = 1;
+            raise_error(a.err, kDevTimeout);
+        }
+        umma_commit(&s_done);  // fires once every MMA above has completed
+    }
+    __syncwarp();
+    const bool done = mbar_wait_sleep(&s_done, 0);
+    if (!done && lane == 0) raise_error(a.err, kDevTimeout);
+    const bool all_done = __syncthreads_and(done);  // also publishes s_fail
+    tc_fence_after();
+    pdl_launch_dependents();
+    if (s_fail == 0 && all_done) {
+        const int ch = n0 + warp * 32 + lane;  // this thread's TMEM lane = output channel
+        const bool ch_ok = ch < a.out_dim;
+        const float wsc = ch_ok ? a.wscale[(size_t)slot.x * a.out_dim + ch] : 0.0f;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        for (int c0 = 0; c0 < mma_n; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(lane_base + (uint32_t)c0, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int r = c0 + j;
+                if (r < nr && ch_ok) {
+                    const int row = slot.y + r;
+                    const float val = __fmul_rn(__fmul_rn(__int2float_rn((int)v[j]), a.dyn[row]), wsc);
+                    a.out[(size_t)row * a.out_dim + ch] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGmTmemCols)
+                     : "memory");
+}
+
+}  // namespace moe

@@ -1,7 +1,10 @@
 // moe_b200.cu -- the C ABI of include/moe_b200.h: host-side validation,
 // workspace sizing and kernel launches.  All compute is in the kernels of
-// update_expert.cuh, dispatch.cuh and combine.cuh.
+// update_expert.cuh, dispatch.cuh, grouped_matmul.cuh and combine.cuh.
 #include "moe_b200.h"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <cstring>
@@ -10,6 +13,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "dispatch.cuh"
+#include "grouped_matmul.cuh"
 #include "update_expert.cuh"
 
 namespace {
@@ -113,6 +117,49 @@ bool valid_combine(const moe_combine_params &p) {
     return true;
 }
 
+bool valid_gmm(const moe_gmm_params &p) {
+    if (p.rows < 1 || p.num_instances < 1 || p.num_instances > MOE_MAX_EXPERTS) return false;
+    if (moe::gmm_max_slots(p.rows, p.num_instances) > 65535) return false;  // slots index grid.y
+    if (p.hidden < MOE_MIN_HIDDEN || p.hidden > MOE_MAX_HIDDEN || p.hidden % 16 != 0) return false;
+    if (p.out_dim < 16 || p.out_dim > MOE_GMM_MAX_OUT_DIM || p.out_dim % 16 != 0) return false;
+    return true;
+}
+
+// Grouped-matmul workspace: the error-word area, the slot count (padded to
+// 16 bytes), then the slots.
+size_t gmm_workspace_bytes(const moe_gmm_params &p) {
+    return kWorkspaceBytes + 16 + 16 * (size_t)moe::gmm_max_slots(p.rows, p.num_instances);
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A row-major int8 matrix [outer, inner] as a 2-D tensor map with boxes of
+// box_outer rows x 128 bytes, 128-byte swizzle, zero fill out of range.
+bool encode_i8_rows(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+    const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {(cuuint32_t)moe::kGmBK, box_outer};
+    const cuuint32_t elem[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Every kernel is launched as a programmatic dependent of whatever precedes it
 // on the stream: its blocks may be scheduled while the previous kernel drains,
 // and each kernel calls griddepcontrol.wait before it touches memory a
@@ -121,9 +168,9 @@ bool valid_combine(const moe_combine_params &p) {
 // call's own inputs; the route kernel only releases it after its own wait).
 // The attribute is harmless when the predecessor is not a kernel.
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, Args... args) {
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t s, Args... args) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
+    cfg.gridDim = grid;
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -457,6 +504,51 @@ moe_status moe_combine(const moe_combine_params *p, const void *expand_x, const 
     a.y = reinterpret_cast<uint16_t *>(out);
     a.err = reinterpret_cast<uint32_t *>(workspace);
     return launch_combine_k<false>(a, p->top_k, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ------------------------------------------------------- grouped matmul ---
+
+moe_status moe_grouped_matmul_workspace_size(const moe_gmm_params *p, size_t *bytes) {
+    if (p == nullptr || bytes == nullptr || !valid_gmm(*p)) return MOE_ERR_INVALID_ARG;
+    *bytes = gmm_workspace_bytes(*p);
+    return MOE_OK;
+}
+
+moe_status moe_grouped_matmul(const moe_gmm_params *p, const void *expand_x, const float *dyn_scales,
+                              const int32_t *expert_offsets, const void *weight, const float *weight_scales,
+                              void *out, void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr || !valid_gmm(*p)) return MOE_ERR_INVALID_ARG;
+    if (!expand_x || !dyn_scales || !expert_offsets || !weight || !weight_scales || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(expand_x, 16) || !aligned(weight, 16) || !aligned(out, 16) || !aligned(dyn_scales, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(weight_scales, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < gmm_workspace_bytes(*p))
+        return MOE_ERR_WORKSPACE;
+    CUtensorMap tm_w, tm_x;
+    if (!encode_i8_rows(&tm_w, weight, (uint64_t)p->hidden, (uint64_t)p->num_instances * p->out_dim, moe::kGmBM) ||
+        !encode_i8_rows(&tm_x, expand_x, (uint64_t)p->hidden, (uint64_t)p->rows, moe::kGmBoxRows))
+        return MOE_ERR_CUDA;
+    unsigned char *ws = reinterpret_cast<unsigned char *>(workspace);
+    moe::GmmArgs a = {};
+    a.rows = p->rows;
+    a.hidden = p->hidden;
+    a.out_dim = p->out_dim;
+    a.num_instances = p->num_instances;
+    a.max_slots = moe::gmm_max_slots(p->rows, p->num_instances);
+    a.dyn = dyn_scales;
+    a.offsets = expert_offsets;
+    a.wscale = weight_scales;
+    a.out = reinterpret_cast<uint16_t *>(out);
+    a.nslots = reinterpret_cast<int *>(ws + kWorkspaceBytes);
+    a.slots = reinterpret_cast<int4 *>(ws + kWorkspaceBytes + 16);
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    cudaStream_t s = as_stream(cuda_stream);
+    if (!ensure_smem(moe::gmm_kernel, moe::kGmSmemBytes)) return MOE_ERR_CUDA;
+    if (launch(moe::gmm_plan_kernel, dim3(1), 1024, 0, s, a) != cudaSuccess) return MOE_ERR_CUDA;
+    const dim3 grid((p->out_dim + moe::kGmBM - 1) / moe::kGmBM, a.max_slots);
+    return launch(moe::gmm_kernel, grid, moe::kGmThreads, moe::kGmSmemBytes, s, tm_w, tm_x, a) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 // ------------------------------------------------------- dispatch, no alloc ---

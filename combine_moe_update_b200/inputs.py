@@ -267,3 +267,61 @@ def make_layer_stack(seed=4, layers=32, bs=128, hidden=2048, num_experts=64, top
                       ep_world_size=ep_world_size, layers=layers, x0=x0, residual0=r0,
                       expert_ids=ids, expert_scales=scs, gammas=gs,
                       table=identity_table(num_experts, ep_world_size))
+
+
+# --------------------------------------------------------------------------
+# the instances' grouped matmul between dispatch and combine
+# --------------------------------------------------------------------------
+
+@dataclass
+class GmmInputs:
+    """One grouped-matmul call: int8 rows (the dispatch's expert-major receive
+    buffer) with one dequantization factor each, the per-instance offsets,
+    and every instance's int8 weight [N, H] with one factor per channel."""
+    expand_x: np.ndarray       # [rows, H] int8
+    dyn_scales: np.ndarray     # [rows] f32
+    offsets: np.ndarray        # [E + 1] int32
+    weight: np.ndarray         # [E, N, H] int8
+    weight_scales: np.ndarray  # [E, N] f32
+
+
+def gmm_inputs(seed, counts, hidden, out_dim, spare_rows=0, one_hot=False) -> GmmInputs:
+    """``counts[e]`` rows for instance e, ``spare_rows`` unused rows after
+    them.  Codes and weights are uniform over [-127, 127] (weights down to
+    -128); row factors ~U(0.005, 0.05) (a row max of 0.6..6 over 127), channel
+    factors ~U(1e-4, 1e-3).  ``one_hot``: each row holds a single non-zero
+    code in [-15, 15] at a random position and weights lie in [-15, 15], so
+    every output is one product, exact in bf16 with unit factors."""
+    rng = np.random.Generator(np.random.PCG64([seed, 77]))
+    counts = np.asarray(counts, np.int64)
+    E = len(counts)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = int(off[-1]) + int(spare_rows)
+    if one_hot:
+        x = np.zeros((rows, hidden), np.int8)
+        pos = rng.integers(0, hidden, rows)
+        x[np.arange(rows), pos] = rng.integers(-15, 15, rows, endpoint=True).astype(np.int8)
+        w = rng.integers(-15, 15, (E, out_dim, hidden), dtype=np.int8, endpoint=True)
+        ds = np.ones(rows, np.float32)
+        ws = np.ones((E, out_dim), np.float32)
+    else:
+        x = rng.integers(-127, 127, (rows, hidden), dtype=np.int8, endpoint=True)
+        w = rng.integers(-128, 127, (E, out_dim, hidden), dtype=np.int8, endpoint=True)
+        ds = rng.uniform(0.005, 0.05, rows).astype(np.float32)
+        ws = rng.uniform(1e-4, 1e-3, (E, out_dim)).astype(np.float32)
+    return GmmInputs(expand_x=x, dyn_scales=ds, offsets=off, weight=w, weight_scales=ws)
+
+
+def gmm_weights_device(seed, num_instances, out_dim, hidden, device):
+    """Instance weights too large to draw on the host (E x N x H int8, e.g.
+    256 x 7168 x 7168 = 13 GB), drawn on ``device`` by torch's seeded
+    generator: codes uniform over [-128, 127], channel factors ~U(1e-4, 1e-3).
+    Returns (weight [E, N, H] int8, weight_scales [E, N] f32)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    w = torch.empty((num_instances, out_dim, hidden), dtype=torch.int8, device=device)
+    for e in range(num_instances):  # one instance at a time bounds the int64 scratch
+        w[e] = torch.randint(-128, 128, (out_dim, hidden), generator=g, device=device, dtype=torch.int8)
+    ws = torch.rand((num_instances, out_dim), generator=g, device=device) * 9e-4 + 1e-4
+    return w, ws

@@ -271,6 +271,58 @@ MOE_API moe_status moe_combine(const moe_combine_params *p, const void *expand_x
                                size_t workspace_bytes, void *cuda_stream);
 
 /* ------------------------------------------------------------------------ */
+/* moe_grouped_matmul -- the instances' int8 matmul between dispatch and     */
+/* combine                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Output channels per instance at most. */
+#define MOE_GMM_MAX_OUT_DIM 65536
+
+typedef struct {
+    int32_t rows;           /* rows of expand_x and out, > 0 (the dispatch's receive rows) */
+    int32_t hidden;         /* H, the contraction length, [1024, 8192], H % 16 == 0 */
+    int32_t out_dim;        /* N, output channels per instance, [16, 65536], N % 16 == 0 */
+    int32_t num_instances;  /* deployed instances E, (0, 1024] */
+} moe_gmm_params;
+
+MOE_API moe_status moe_grouped_matmul_workspace_size(const moe_gmm_params *p, size_t *bytes);
+
+/*
+ * The expert step between the dispatch ("AllToAllV(quantOut)", dispatch page,
+ * "计算公式") and the gather the combine starts from ("ataOut", combine page,
+ * "计算公式").  The pages do not define it; this library takes it as the one
+ * contraction that consumes the dispatch output: instance e multiplies its
+ * rows, [expert_offsets[e], expert_offsets[e+1]) of expand_x, by its own
+ * weight:
+ *   out[r][n] = (sum_h expand_x[r][h] * weight[e][n][h]) * dyn_scales[r] * weight_scales[e][n]
+ * The sum is exact (int32); the two products are binary32; out is bf16
+ * (round to nearest even).  With N = H the result is the expand_x that
+ * moe_combine / moe_combine_add_rmsnorm gather.
+ *
+ *   expand_x       [rows, H] int8 device, 16-byte aligned (moe_dispatch, quant_mode 1 or 2)
+ *   dyn_scales     [rows] f32 device: each row's dequantization factor (the
+ *                  dispatch's mode-2 dyn_scales; a constant array for mode 1)
+ *   expert_offsets [E+1] int32 device (moe_dispatch's output): a non-decreasing
+ *                  run in [0, rows]
+ *   weight         [E, N, H] int8 device, 16-byte aligned: each output channel's
+ *                  H weights contiguous
+ *   weight_scales  [E, N] f32 device
+ *   out            [rows, N] bf16 device, 16-byte aligned; rows outside
+ *                  [expert_offsets[0], expert_offsets[E]) are left untouched
+ *   workspace      device, moe_grouped_matmul_workspace_size bytes, 16-byte aligned
+ *
+ * Host errors: MOE_ERR_INVALID_ARG for sizes outside the limits or NULL /
+ * misaligned pointers, MOE_ERR_WORKSPACE, MOE_ERR_CUDA if a tensor map cannot
+ * be encoded or a launch is refused.  Device errors: offsets that are not a
+ * non-decreasing run in [0, rows] set MOE_DEV_BAD_ID and nothing is written;
+ * a bounded wait that gives up sets MOE_DEV_TIMEOUT.
+ */
+MOE_API moe_status moe_grouped_matmul(const moe_gmm_params *p, const void *expand_x, const float *dyn_scales,
+                                      const int32_t *expert_offsets, const void *weight,
+                                      const float *weight_scales, void *out, void *workspace,
+                                      size_t workspace_bytes, void *cuda_stream);
+
+/* ------------------------------------------------------------------------ */
 /* moe_dispatch_noalloc -- moe_dispatch without a caller-provided workspace  */
 /* ------------------------------------------------------------------------ */
 

@@ -177,6 +177,41 @@ def test_combine_pointer_rules(L):
     assert call(ws=None) == L.MOE_ERR_WORKSPACE
 
 
+GMM_BAD = [dict(rows=0), dict(num_instances=0), dict(num_instances=1025), dict(hidden=1000), dict(hidden=9000),
+           dict(hidden=1032), dict(out_dim=0), dict(out_dim=8), dict(out_dim=200), dict(out_dim=65552),
+           dict(rows=(65535 - 1024) * 128 + 1, num_instances=1024)]
+
+
+def _gmm_params(L, **over):
+    base = dict(rows=4096, hidden=7168, out_dim=7168, num_instances=256)
+    base.update(over)
+    return L.GmmParams(base["rows"], base["hidden"], base["out_dim"], base["num_instances"])
+
+
+@pytest.mark.parametrize("bad", GMM_BAD)
+def test_grouped_matmul_rejects(L, bad):
+    p = _gmm_params(L, **bad)
+    assert ws_size(L, "moe_grouped_matmul_workspace_size", p)[0] == L.MOE_ERR_INVALID_ARG
+    f = ctypes.c_void_p(0x10000)
+    assert L.lib.moe_grouped_matmul(ctypes.byref(p), f, f, f, f, f, f, f, 1 << 20, None) == L.MOE_ERR_INVALID_ARG
+
+
+def test_grouped_matmul_workspace_and_pointer_rules(L):
+    p = _gmm_params(L)
+    st, n = ws_size(L, "moe_grouped_matmul_workspace_size", p)
+    assert st == L.MOE_OK and n == 256 + 16 + 16 * (256 + 4096 // 128)
+    edge = _gmm_params(L, rows=(65535 - 1024) * 128, num_instances=1024)  # the last row count grid.y allows
+    assert ws_size(L, "moe_grouped_matmul_workspace_size", edge)[0] == L.MOE_OK
+    f, f8, f2 = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10008), ctypes.c_void_p(0x10002)
+    call = lambda x=f, ds=f, off=f, w=f, wsc=f, out=f, ws=f, wsb=n: L.lib.moe_grouped_matmul(
+        ctypes.byref(p), x, ds, off, w, wsc, out, ws, wsb, None)
+    for kw in (dict(x=None), dict(ds=None), dict(off=None), dict(w=None), dict(wsc=None), dict(out=None),
+               dict(x=f8), dict(w=f8), dict(out=f8), dict(ds=f2), dict(off=f2), dict(wsc=f2)):
+        assert call(**kw) == L.MOE_ERR_INVALID_ARG, kw
+    assert call(ws=None) == L.MOE_ERR_WORKSPACE
+    assert call(wsb=n - 16) == L.MOE_ERR_WORKSPACE
+
+
 def test_no_cpu_fallback_in_product():
     """The product package never reaches the oracle."""
     pkg = os.path.join(ROOT, "combine_moe_update_b200")
