@@ -196,6 +196,8 @@ def run_b200(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     w = gen.make(args.workload, seed=None if rank == 0 else 1000 + rank)
+    if "expert_out_dim" in w.meta:
+        return run_b200_expert(args, rank, world, local_rank, w)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     bf = lambda a: dev(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16)
 
@@ -455,6 +457,211 @@ def run_b200(args, rank, world, local_rank):
     return out, w
 
 
+def gmm_bytes(offsets, hidden, out_dim):
+    """Algorithmic bytes of one grouped matmul: the weights of every instance
+    that received rows (read once), the rows (int8) and their factors, the
+    channel factors, the offsets, and the bf16 output rows."""
+    import numpy as np
+    off = np.asarray(offsets, np.int64)
+    used = int(np.count_nonzero(np.diff(off)))
+    n = int(off[-1] - off[0])
+    return used * out_dim * hidden + used * out_dim * 4 + n * hidden + n * 4 + n * out_dim * 2 + off.size * 4
+
+
+def run_b200_expert(args, rank, world, local_rank, w):
+    """The layer with the instances' grouped int8 matmul in the step:
+    moe_update_expert -> moe_dispatch (int8 rows) -> moe_grouped_matmul
+    (N = H, every instance's weight resident in HBM) -> moe_combine_add_rmsnorm
+    reading the matmul's output rows.  The weights (13 GB at 256 instances)
+    dwarf L2, and the activations are flushed out of L2 before every step."""
+    import numpy as np
+    import torch
+    from combine_moe_update_b200 import binding as B
+    from combine_moe_update_b200 import inputs as gen
+
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    bf = lambda a: dev(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16)
+    H, E, N = w.hidden, w.num_instances, int(w.meta["expert_out_dim"])
+    assert N == H, "the combine gathers rows of width H"
+    table = dev(w.table)
+    smooth = None if w.smooth is None else dev(w.smooth)
+    gamma = bf(w.gamma)
+    weight, wscale = gen.gmm_weights_device(w.meta["weight_seed"], E, N, H, "cuda")
+    ids, scales = dev(w.expert_ids), dev(w.expert_scales)
+    x, residual = bf(w.x), bf(w.residual)
+    shared = None if w.shared_x is None else bf(w.shared_x)
+    ws = B.new_workspace(nbytes=B.dispatch_workspace_bytes(
+        w.bs, H, w.top_k, w.ep_world_size, E, w.quant_mode, 0 if w.smooth is None else w.smooth.size))
+    rows = w.bs * w.top_k
+    gws = B.new_workspace(nbytes=B.grouped_matmul_workspace_bytes(rows, H, N, E))
+    bal = torch.empty_like(ids)
+    bm = torch.empty(ids.shape, dtype=torch.uint8, device="cuda")
+    d = B.alloc_dispatch_outputs(w.bs, H, w.top_k, E, w.quant_mode)
+    ex = torch.zeros((rows, N), dtype=torch.bfloat16, device="cuda")
+    c = dict(y=torch.empty_like(x), x_out=None, rstd=None)
+
+    def calls(xx=x, ii=ids, ss=scales, rr=residual, sh=shared, ev=None):
+        mark = (lambda j: ev[j].record()) if ev is not None else (lambda j: None)
+        B.update_expert(ii, table, w.ep_world_size, expert_scales=ss, prune_threshold=w.prune_threshold,
+                        workspace=ws, out=(bal, bm))
+        mark(1)
+        B.dispatch(xx, bal, E, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth, workspace=ws, out=d)
+        mark(2)
+        B.grouped_matmul(d["expand_x"], d["dyn_scales"], d["offsets"], weight, wscale, out=ex, workspace=gws)
+        mark(3)
+        B.combine_add_rmsnorm(ex, d["expand_idx"], ss, rr, gamma, w.norm_eps, shared_x=sh, workspace=ws, out=c)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clean = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.float32, device="cuda")
+
+    def flush_l2():
+        flush.zero_()
+        clean.sum()
+
+    for _ in range(args.warmup):
+        flush_l2()
+        calls()
+    torch.cuda.synchronize()
+    assert B.read_device_error(ws) == 0 and B.read_device_error(gws) == 0, "device error during warm-up"
+    off = d["offsets"].cpu().numpy()
+    n = int(off[-1])
+    alg = algorithmic_bytes(w, n)
+    alg["grouped_matmul"] = gmm_bytes(off, H, N)
+    # the combine reads the matmul's rows instead of the stand-in rows: same byte count
+
+    K = args.steps
+    G = max(g for g in range(1, 9) if K % g == 0)
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+
+    def capture(per_call):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(G)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for e in evs:
+                flush_l2()
+                e[0].record()
+                calls(ev=e if per_call else None)
+                e[4].record()
+        return g, evs
+
+    graph, ev_step = capture(False)
+    graph_ops, ev_ops = capture(True)
+    for g in (graph, graph_ops):
+        g.replay()
+    torch.cuda.synchronize()
+    sums = [0.0] * 5
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for _ in range(K // G):
+            graph.replay()
+            torch.cuda.synchronize()
+            for e in ev_step:
+                sums[0] += e[0].elapsed_time(e[4])
+        barrier()
+        torch.cuda.synchronize()
+        for _ in range(K // G):
+            graph_ops.replay()
+            torch.cuda.synchronize()
+            for e in ev_ops:
+                for j in range(4):
+                    sums[1 + j] += e[j].elapsed_time(e[j + 1])
+    barrier()
+    del graph, graph_ops
+    assert B.read_device_error(ws) == 0 and B.read_device_error(gws) == 0, "device error during the timed steps"
+
+    # The matmul on its own for the roofline: calls back to back (each kernel a
+    # programmatic dependent of the one before) in one graph; the weights are
+    # far larger than L2, so every call streams them from HBM.  Time per call =
+    # the span / count; a call is the planning kernel plus the matmul kernel.
+    M = 8
+    eb = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    graph_g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_g, stream=cap):
+        eb[0].record()
+        for _ in range(M):
+            B.grouped_matmul(d["expand_x"], d["dyn_scales"], d["offsets"], weight, wscale, out=ex, workspace=gws)
+        eb[1].record()
+    graph_g.replay()
+    torch.cuda.synchronize()
+    reps = max(3, min(20, K // 4))
+    t_gmm = 0.0
+    for _ in range(reps):
+        graph_g.replay()
+        torch.cuda.synchronize()
+        t_gmm += eb[0].elapsed_time(eb[1]) / M
+    t_gmm /= reps
+    del graph_g
+    assert B.read_device_error(gws) == 0, "device error during the matmul roofline calls"
+
+    t_step, t_upd, t_disp, t_gm, t_comb, t_gmm = reduce_over_ranks([v / K for v in sums] + [t_gmm], "max")
+    value = world * w.bs / (t_step * 1e-3)
+
+    # end to end through the public API with host buffers (weights and layer parameters resident)
+    pin = lambda t: t.cpu().pin_memory()
+    h_in = dict(x=pin(x), ids=pin(ids), scales=pin(scales), residual=pin(residual))
+    if shared is not None:
+        h_in["shared"] = pin(shared)
+    d_in = {k_: torch.empty_like(v) for k_, v in (("x", x), ("ids", ids), ("scales", scales), ("residual", residual))}
+    d_in["shared"] = None if shared is None else torch.empty_like(shared)
+    h_y = torch.empty(c["y"].shape, dtype=c["y"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = h_y.numel() * h_y.element_size()
+
+    def e2e_step():
+        for k_, t in h_in.items():
+            d_in[k_].copy_(t, non_blocking=True)
+        calls(d_in["x"], d_in["ids"], d_in["scales"], d_in["residual"], d_in["shared"])
+        h_y.copy_(c["y"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ke = max(5, min(K, 50))
+    e0.record()
+    for _ in range(ke):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    (t_e2e,) = reduce_over_ranks([e0.elapsed_time(e1) / ke], "max")
+
+    peak, peak_kind = measured_peak()
+    achieved = alg["grouped_matmul"] / (t_gmm * 1e-3) / 1e9
+    step_bytes = alg["update"] + alg["dispatch"] + alg["grouped_matmul"] + alg["combine"]
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8+int32 (matmul), fp32",
+        "data": "synthetic (seeded; pages' shapes; instance weights drawn on the device)",
+        "config": {"workload": args.workload, "bs": w.bs, "hidden": H, "top_k": w.top_k, "num_instances": E,
+                   "ep_world_size_simulated": w.ep_world_size, "quant_mode": w.quant_mode,
+                   "smooth_scales": w.smooth is not None, "shared_expert": w.shared_x is not None,
+                   "kept_copies": n, "expert_out_dim": N, "weight_bytes": E * N * H,
+                   "l2": "flushed before every timed step (512 MiB written, 256 MiB read); weights >> L2",
+                   "parallelism": f"replicas x{world}"},
+        "breakdown_us": {"update_expert": round(t_upd * 1e3, 2), "dispatch": round(t_disp * 1e3, 2),
+                         "grouped_matmul": round(t_gm * 1e3, 2), "combine": round(t_comb * 1e3, 2)},
+        "achieved_gbs": {"step": round(step_bytes / (t_step * 1e-3) / 1e9, 1), "grouped_matmul": round(achieved, 1)},
+        "roofline": {"bound": "hbm", "kernel": "gmm_kernel", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "launch_us": round(t_gmm * 1e3, 2),
+                     "timing": f"{M} back-to-back calls (planning + matmul kernel) in a graph, CUDA events around them",
+                     "traffic": stored_traffic("gmm_kernel", args.workload),
+                     "algorithmic_bytes": alg["grouped_matmul"],
+                     "tensor_tops": round(2.0 * n * N * H / (t_gmm * 1e-3) / 1e12, 1)},
+        "e2e": {"value": round(world * w.bs / (t_e2e * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "pinned host activations -> device, the four calls, y -> host; weights resident"},
+        "gpu_launches": 6 * K,  # update_expert, route, scatter, matmul planning, matmul, combine
+        "timing": f"CUDA graphs of {G} steps, L2 flushed before each step outside the events",
+        "clocks": clk.summary(),
+    }
+    return out, w
+
+
 # --------------------------------------------------------------------------
 # the CPU oracle, as a reported baseline and as the reference arm
 # --------------------------------------------------------------------------
@@ -463,8 +670,32 @@ def oracle_step(orc, w):
     bal, bm, _ = orc.update_expert(w.expert_ids, w.table, w.ep_world_size, expert_scales=w.expert_scales,
                                    prune_threshold=w.prune_threshold)
     d = orc.dispatch(w.x, bal, w.num_instances, w.quant_mode, mask=bm, smooth=w.smooth)
-    orc.combine_add_rmsnorm(w.expert_out, d["expand_idx"], w.expert_scales, w.residual, w.gamma, w.norm_eps,
+    rows = w.expert_out
+    if "expert_out_dim" in w.meta:
+        rows = _oracle_expert_rows(orc, w, d)
+    orc.combine_add_rmsnorm(rows, d["expand_idx"], w.expert_scales, w.residual, w.gamma, w.norm_eps,
                             shared_x=w.shared_x)
+
+
+def _oracle_expert_rows(orc, w, d):
+    """The oracle's grouped matmul over the instances this sample reaches (the
+    others have no rows, so dropping them from the offsets changes nothing);
+    their host weights are drawn once per sample and cached on it."""
+    import numpy as np
+    from combine_moe_update_b200 import inputs as gen
+    off = d["offsets"]
+    used = [e for e in range(w.num_instances) if off[e + 1] > off[e]]
+    cache = w.meta.setdefault("_host_weights", {})
+    key = tuple(used)
+    if key not in cache:
+        hw = gen.gmm_weights_host(w.meta["weight_seed"], used, w.meta["expert_out_dim"], w.hidden)
+        cache.clear()
+        cache[key] = (np.stack([hw[e][0] for e in used]), np.stack([hw[e][1] for e in used]))
+    wts, wss = cache[key]
+    off_c = np.array([off[e] for e in used] + [off[-1]], np.int32)
+    g = orc.grouped_matmul(d["expand_x"], d["dyn_scales"], off_c, wts, wss,
+                           out=np.zeros((d["expand_x"].shape[0], w.meta["expert_out_dim"]), np.uint16))
+    return g["out"]
 
 
 def subsample(w, tokens):
@@ -477,11 +708,30 @@ def subsample(w, tokens):
         if v is not None:
             setattr(s, k, v[:tokens].copy())
     s.expert_out = w.expert_out[: tokens * w.top_k].copy()
+    s.meta = {k: v for k, v in w.meta.items() if not k.startswith("_")}
     return s
 
 
 def cpu_baseline(w, budget_s=10.0):
     from oracle import oracle as orc
+    if "expert_out_dim" in w.meta:
+        # a full step of the matmul layer takes minutes on one core: time a
+        # sample of tokens sized from a one-token calibration run
+        one = subsample(w, 1)
+        t0 = time.perf_counter()
+        oracle_step(orc, one)
+        per_tok = time.perf_counter() - t0
+        # at most 4 tokens: each reaches up to K instances, whose weights (H * H
+        # bytes each) are drawn into host memory
+        tokens = int(max(1, min(4, budget_s / max(per_tok, 1e-9))))
+        sample = subsample(w, tokens)
+        oracle_step(orc, sample)  # draw and cache this sample's weights outside the timing
+        t0 = time.perf_counter()
+        oracle_step(orc, sample)
+        dt = time.perf_counter() - t0
+        return {"value": round(tokens / dt, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"one step of the first {tokens} of {w.bs} tokens ({dt:.1f} s, single-threaded C "
+                          "oracle; the weights of the instances they reach drawn on the host)"}
     oracle_step(orc, subsample(w, 8))  # build + warm
     t0 = time.perf_counter()
     steps = 0
@@ -504,11 +754,13 @@ def run_reference(args, rank):
     w = gen.make(args.workload)
     orc.build()
     # calibrate: seconds per token, then size each step so the run stays within ~2 minutes
+    cal = 1 if "expert_out_dim" in w.meta else 16
     t0 = time.perf_counter()
-    oracle_step(orc, subsample(w, 16))
-    per_tok = (time.perf_counter() - t0) / 16
+    oracle_step(orc, subsample(w, cal))
+    per_tok = (time.perf_counter() - t0) / cal
     budget = 120.0 / max(1, args.steps + args.warmup)
-    tokens = int(max(1, min(w.bs, budget / max(per_tok, 1e-9))))
+    # the matmul layer: at most 4 tokens, whose instances' weights are drawn on the host
+    tokens = int(max(1, min(4 if cal == 1 else w.bs, budget / max(per_tok, 1e-9))))
     sample = subsample(w, tokens)
     for _ in range(args.warmup):
         oracle_step(orc, sample)

@@ -197,6 +197,18 @@ def _static_layer(name, seed, **kw):
     return w
 
 
+def _expert_layer(name, seed, expert_out_dim, **kw):
+    """A uniform layer whose step includes the instances' grouped int8 matmul
+    between dispatch and combine: every instance owns an int8 weight
+    [expert_out_dim, H] with per-channel factors (drawn on the device by
+    gmm_weights_device from meta["weight_seed"]); expert_out_dim = H, so the
+    matmul's rows are what the combine gathers."""
+    w = uniform_layer(name, seed, **kw)
+    w.meta["expert_out_dim"] = expert_out_dim
+    w.meta["weight_seed"] = 500 + seed
+    return w
+
+
 WORKLOADS = {
     # Bs 8, H 1024, 8 experts, K 2, 4 simulated ranks, no quantization.
     "tiny": dict(builder=uniform_layer, seed=0, bs=8, hidden=1024, num_experts=8, top_k=2,
@@ -221,6 +233,15 @@ WORKLOADS = {
     "deepseek_ep8_all_ranks": dict(builder=_all_ranks_layer, seed=1, bs=512, sources=8, hidden=7168,
                                    num_experts=256, top_k=8, ep_world_size=8, quant_mode=2, smooth=True,
                                    shared=True),
+    # The Bs 512 decode layer with the instances' int8 matmul in the step:
+    # 256 instance weights of 7168 x 7168 int8 (13.2 GB, resident).
+    "deepseek_decode_bs512_expert": dict(builder=_expert_layer, seed=1, bs=512, hidden=7168, num_experts=256,
+                                         top_k=8, ep_world_size=32, quant_mode=2, smooth=True, shared=True,
+                                         expert_out_dim=7168),
+    # The same layer cut to 32 instances and Bs 128 (1.6 GB of weights), small
+    # enough for a profiler capture of the matmul kernel.
+    "expert_e32_bs128": dict(builder=_expert_layer, seed=1, bs=128, hidden=7168, num_experts=32, top_k=8,
+                             ep_world_size=8, quant_mode=2, smooth=True, shared=True, expert_out_dim=7168),
     # Zipf(1.2) routing over 128 experts, 160 instances on 16 ranks, mxfp8.
     "skewed_eplb": dict(builder=_skewed_eplb, seed=2, bs=512),
     # Largest shapes: H 8192, 1024 experts, K 16, 256 ranks, per-128-tile int8,
@@ -325,3 +346,17 @@ def gmm_weights_device(seed, num_instances, out_dim, hidden, device):
         w[e] = torch.randint(-128, 128, (out_dim, hidden), generator=g, device=device, dtype=torch.int8)
     ws = torch.rand((num_instances, out_dim), generator=g, device=device) * 9e-4 + 1e-4
     return w, ws
+
+
+def gmm_weights_host(seed, instances, out_dim, hidden):
+    """Host-side weights for the given instances, for CPU runs that touch only
+    a few of them: per instance an independent seeded stream, codes uniform
+    over [-128, 127], channel factors ~U(1e-4, 1e-3) (the distribution of
+    gmm_weights_device; the values differ).  Returns {e: (w [N, H] int8,
+    ws [N] f32)}."""
+    out = {}
+    for e in instances:
+        rng = np.random.Generator(np.random.PCG64([seed, 9000 + int(e)]))
+        out[int(e)] = (rng.integers(-128, 127, (out_dim, hidden), dtype=np.int8, endpoint=True),
+                       rng.uniform(1e-4, 1e-3, out_dim).astype(np.float32))
+    return out
