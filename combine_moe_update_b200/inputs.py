@@ -360,3 +360,45 @@ def gmm_weights_host(seed, instances, out_dim, hidden):
         out[int(e)] = (rng.integers(-128, 127, (out_dim, hidden), dtype=np.int8, endpoint=True),
                        rng.uniform(1e-4, 1e-3, out_dim).astype(np.float32))
     return out
+
+
+@dataclass
+class GmmMxInputs:
+    """One grouped-matmul call on mxfp8: E4M3 rows with one E8M0 factor per
+    32-element block (the dispatch's quantMode-4 output) and E4M3 instance
+    weights with their own E8M0 block factors."""
+    expand_x: np.ndarray   # [rows, H] uint8 E4M3 codes
+    x_sf: np.ndarray       # [rows, H/32] uint8 E8M0
+    offsets: np.ndarray    # [E + 1] int32
+    weight: np.ndarray     # [E, N, H] uint8 E4M3 codes
+    weight_sf: np.ndarray  # [E, N, H/32] uint8 E8M0
+
+
+def _e4m3_codes(rng, shape):
+    """Uniform over the 254 finite E4M3 codes (S.1111.111 is NaN)."""
+    c = rng.integers(0, 254, shape, dtype=np.uint16)  # 0..253 -> skip 0x7F and 0xFF
+    c = c + (c >= 0x7F) + (c >= 0xFE)
+    return c.astype(np.uint8)
+
+
+def gmm_inputs_mx(seed, counts, hidden, out_dim, spare_rows=0, one_hot=False) -> GmmMxInputs:
+    """Row codes and weights uniform over the finite E4M3 codes, block
+    factors 2^(b - 127) with b uniform in [117, 137].  ``one_hot``: one
+    non-zero row code per row (at a random position) and weights whose
+    codes are exact small values, so every output is a single scaled
+    product."""
+    rng = np.random.Generator(np.random.PCG64([seed, 78]))
+    counts = np.asarray(counts, np.int64)
+    E = len(counts)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = int(off[-1]) + int(spare_rows)
+    B = hidden // 32
+    xs = rng.integers(117, 137, (rows, B), dtype=np.uint8, endpoint=True)
+    wsf = rng.integers(117, 137, (E, out_dim, B), dtype=np.uint8, endpoint=True)
+    if one_hot:
+        x = np.zeros((rows, hidden), np.uint8)
+        x[np.arange(rows), rng.integers(0, hidden, rows)] = _e4m3_codes(rng, rows)
+    else:
+        x = _e4m3_codes(rng, (rows, hidden))
+    w = _e4m3_codes(rng, (E, out_dim, hidden))
+    return GmmMxInputs(expand_x=x, x_sf=xs, offsets=off, weight=w, weight_sf=wsf)

@@ -74,6 +74,15 @@ uint8_t orc_e4m3_encode(float v) {
     return s | (uint8_t)(((E + 7) << 3) | (int)m);
 }
 
+/* The value of an E4M3 ("fn") code: S.EEEE.MMM, exponent bias 7; E = 0 is
+ * subnormal (M * 2^-9); S.1111.111 is NaN; no infinities. */
+double orc_e4m3_decode(uint8_t c) {
+    const int s = c >> 7, E = (c >> 3) & 15, M = c & 7;
+    if (E == 15 && M == 7) return NAN;
+    double v = E == 0 ? ldexp((double)M, -9) : ldexp(1.0 + M / 8.0, E - 7);
+    return s ? -v : v;
+}
+
 /* ---------------------------------------------------------------------- */
 /* Step 1: aclnnMoeUpdateExpert                                            */
 /* ---------------------------------------------------------------------- */
@@ -450,6 +459,41 @@ uint32_t orc_grouped_matmul(int32_t rows, int32_t hidden, int32_t out_dim, int32
                 double v = (double)acc * (double)dyn_scales[r] * (double)weight_scales[(size_t)e * N + n];
                 if (out_bf16) out_bf16[(size_t)r * N + n] = orc_bf16_from_double(v);
                 if (out_f64) out_f64[(size_t)r * N + n] = v;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * The same step on mxfp8 rows (quantMode 4, READING R24): the rows are E4M3
+ * codes with one E8M0 factor 2^(b - 127) per 32-element block
+ * (x_sf [rows, H/32], the dispatch's dynamicScales bytes), and so is the
+ * weight (weight_sf [E, N, H/32]):
+ *   out[r][n] = Sum_h dec(q[r][h]) 2^(x_sf[r][h/32] - 127) dec(w[e][n][h]) 2^(weight_sf[e][n][h/32] - 127)
+ * summed in binary64 and rounded to bf16 once.  Offsets as above.
+ */
+uint32_t orc_grouped_matmul_mx(int32_t rows, int32_t hidden, int32_t out_dim, int32_t num_instances,
+                               const uint8_t *expand_x, const uint8_t *x_sf,
+                               const int32_t *expert_offsets, const uint8_t *weight,
+                               const uint8_t *weight_sf, uint16_t *out_bf16, double *out_f64) {
+    const int H = hidden, N = out_dim, E = num_instances, B = hidden / 32;
+    if (expert_offsets[0] < 0 || expert_offsets[E] > rows) return ORC_ERR_BAD_ID;
+    for (int e = 0; e < E; ++e)
+        if (expert_offsets[e + 1] < expert_offsets[e]) return ORC_ERR_BAD_ID;
+    for (int e = 0; e < E; ++e) {
+        for (int r = expert_offsets[e]; r < expert_offsets[e + 1]; ++r) {
+            for (int n = 0; n < N; ++n) {
+                const size_t wr = (size_t)e * N + n;
+                double acc = 0.0;
+                for (int h = 0; h < H; ++h) {
+                    const double xv = ldexp(orc_e4m3_decode(expand_x[(size_t)r * H + h]),
+                                            (int)x_sf[(size_t)r * B + h / 32] - 127);
+                    const double wv = ldexp(orc_e4m3_decode(weight[wr * H + h]), (int)weight_sf[wr * B + h / 32] - 127);
+                    acc += xv * wv;
+                }
+                if (out_bf16) out_bf16[(size_t)r * N + n] = orc_bf16_from_double(acc);
+                if (out_f64) out_f64[(size_t)r * N + n] = acc;
             }
         }
     }

@@ -93,6 +93,15 @@ uint32_t orc_grouped_matmul(int32_t rows, int32_t hidden, int32_t out_dim, int32
                             const int32_t *expert_offsets, const int8_t *weight,
                             const float *weight_scales, uint16_t *out_bf16, double *out_f64);
 
+/* The same on mxfp8 rows and weights: E4M3 codes with one E8M0 factor per
+ * 32-element block, x_sf [rows, hidden/32], weight_sf [E, out_dim, hidden/32];
+ * the sum in binary64, rounded to bf16 once. */
+uint32_t orc_grouped_matmul_mx(int32_t rows, int32_t hidden, int32_t out_dim, int32_t num_instances,
+                               const uint8_t *expand_x, const uint8_t *x_sf,
+                               const int32_t *expert_offsets, const uint8_t *weight,
+                               const uint8_t *weight_sf, uint16_t *out_bf16, double *out_f64);
+double orc_e4m3_decode(uint8_t c);  /* the value of an E4M3 code (NaN for S.1111.111) */
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,6 +65,10 @@ def lib():
             L.orc_e4m3_encode.restype = ctypes.c_uint8
             L.orc_grouped_matmul.restype = ctypes.c_uint32
             L.orc_grouped_matmul.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+            L.orc_grouped_matmul_mx.restype = ctypes.c_uint32
+            L.orc_grouped_matmul_mx.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+            L.orc_e4m3_decode.restype = f64
+            L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
             L.orc_e4m3_encode.argtypes = [f32]
             L.orc_bf16_from_double.restype = ctypes.c_uint16
             L.orc_bf16_from_double.argtypes = [f64]
@@ -197,6 +201,31 @@ def grouped_matmul(expand_x, dyn_scales, expert_offsets, weight, weight_scales, 
     o64 = np.full((rows, N), np.nan, np.float64)
     err = lib().orc_grouped_matmul(rows, H, N, E, _p(ex), _p(ds), _p(off), _p(w), _p(ws), _p(out), _p(o64))
     return dict(out=out, out_f64=o64, err=int(err))
+
+
+def grouped_matmul_mx(expand_x, x_sf, expert_offsets, weight, weight_sf, out=None):
+    """grouped_matmul on mxfp8: E4M3 rows [rows, H] with E8M0 block factors
+    x_sf [rows, H/32], E4M3 weights [E, N, H] with weight_sf [E, N, H/32].
+    Returns out (bf16 bits), out_f64 (NaN where not written) and err."""
+    ex = _c(expand_x, np.uint8)
+    xs = _c(x_sf, np.uint8)
+    off = _c(expert_offsets, np.int32)
+    w = _c(weight, np.uint8)
+    wsf = _c(weight_sf, np.uint8)
+    rows, H = ex.shape
+    E, N = w.shape[0], w.shape[1]
+    assert w.shape == (E, N, H) and wsf.shape == (E, N, H // 32) and xs.shape == (rows, H // 32)
+    assert off.shape == (E + 1,) and H % 32 == 0
+    out = np.zeros((rows, N), np.uint16) if out is None else _c(out, np.uint16).copy()
+    o64 = np.full((rows, N), np.nan, np.float64)
+    err = lib().orc_grouped_matmul_mx(rows, H, N, E, _p(ex), _p(xs), _p(off), _p(w), _p(wsf), _p(out), _p(o64))
+    return dict(out=out, out_f64=o64, err=int(err))
+
+
+def e4m3_decode(codes):
+    f = lib().orc_e4m3_decode
+    c = np.asarray(codes, np.uint8).ravel()
+    return np.array([f(int(t)) for t in c], np.float64).reshape(np.shape(codes))
 
 
 def e4m3_encode(values):

@@ -675,3 +675,54 @@ def test_grouped_matmul_rejects_bad_offsets(orc, off):
                            np.ones((3, 16), np.float32), out=pre)
     assert r["err"] == orc.ERR_BAD_ID
     np.testing.assert_array_equal(r["out"], pre)
+
+
+def test_e4m3_decode_against_library(orc):
+    """All 256 E4M3 codes against ml_dtypes' float8_e4m3fn."""
+    codes = np.arange(256, dtype=np.uint8)
+    want = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    got = orc.e4m3_decode(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    np.testing.assert_array_equal(got[ok], want[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(want[ok]))
+
+
+def _mx_dequant(codes, sf):
+    v = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    return np.ldexp(v, np.repeat(sf.astype(np.int64) - 127, 32, axis=-1))
+
+
+def test_grouped_matmul_mx_against_numpy(orc):
+    """mxfp8 rows and weights dequantized by ml_dtypes and np.ldexp, then
+    numpy's matmul per instance: the products are exact in binary64, so only
+    the summation order differs."""
+    counts = [5, 0, 9, 3]
+    H, N = 128, 48
+    gi = gen.gmm_inputs_mx(14, counts, H, N, spare_rows=1)
+    r = orc.grouped_matmul_mx(gi.expand_x, gi.x_sf, gi.offsets, gi.weight, gi.weight_sf)
+    assert r["err"] == 0
+    off = gi.offsets
+    for e in range(len(counts)):
+        s = slice(off[e], off[e + 1])
+        want = _mx_dequant(gi.expand_x[s], gi.x_sf[s]) @ _mx_dequant(gi.weight[e], gi.weight_sf[e]).T
+        np.testing.assert_allclose(r["out_f64"][s], want, rtol=1e-12, atol=1e-300)
+    assert np.isnan(r["out_f64"][off[-1]:]).all()
+    np.testing.assert_array_equal(r["out"][:off[-1]],
+                                  r["out_f64"][:off[-1]].astype(ml_dtypes.bfloat16).view(np.uint16))
+
+
+def test_grouped_matmul_mx_block_factors_closed_form(orc):
+    """Codes all 1.0 (0x38): block j contributes 32 * 2^(a_j + b_j) with
+    row factor 2^a_j and weight factor 2^b_j, so the output is
+    32 * Sum_j 2^(a_j + b_j); a single factor moved by one doubles only its
+    own block's share."""
+    H, N = 128, 2
+    x = np.full((1, H), 0x38, np.uint8)
+    w = np.full((1, N, H), 0x38, np.uint8)
+    xs = np.array([[127, 128, 126, 130]], np.uint8)   # a = 0, 1, -1, 3
+    ws = np.array([[[127, 127, 129, 120], [127, 127, 127, 127]]], np.uint8)  # b = (0, 0, 2, -7), 0
+    r = orc.grouped_matmul_mx(x, xs, np.array([0, 1], np.int32), w, ws)
+    assert r["err"] == 0
+    assert r["out_f64"][0, 0] == 32 * (1 + 2 + 2.0 ** 1 + 2.0 ** -4)
+    assert r["out_f64"][0, 1] == 32 * (1 + 2 + 0.5 + 8)
