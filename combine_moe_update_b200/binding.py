@@ -54,7 +54,7 @@ EXPORTS = (
     "moe_update_expert_workspace_size", "moe_update_expert",
     "moe_dispatch_workspace_size", "moe_dispatch",
     "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm", "moe_combine",
-    "moe_dispatch_noalloc", "moe_grouped_matmul_workspace_size", "moe_grouped_matmul",
+    "moe_dispatch_noalloc", "moe_grouped_matmul_workspace_size", "moe_grouped_matmul", "moe_grouped_matmul_mx",
 )
 
 
@@ -80,6 +80,7 @@ def _load():
     L.moe_dispatch_noalloc.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_grouped_matmul_workspace_size.argtypes = [P(GmmParams), P(sz)]
     L.moe_grouped_matmul.argtypes = [P(GmmParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_grouped_matmul_mx.argtypes = [P(GmmParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for name in EXPORTS:
         if name != "moe_status_string":
             getattr(L, name).restype = ctypes.c_int
@@ -350,4 +351,28 @@ def grouped_matmul(expand_x, dyn_scales, expert_offsets, weight, weight_scales, 
     _check("moe_grouped_matmul", lib.moe_grouped_matmul(
         ctypes.byref(p), _ptr(expand_x), _ptr(dyn_scales), _ptr(expert_offsets), _ptr(weight),
         _ptr(weight_scales), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def grouped_matmul_mx(expand_x, x_sf, expert_offsets, weight, weight_sf, out=None, workspace=None, stream=None):
+    """moe_grouped_matmul_mx: the instances' matmul on mxfp8 (E4M3 codes as uint8 with E8M0 block factors):
+    expand_x [rows, H], x_sf [rows, H/32], weight [E, N, H], weight_sf [E, N, H/32]; returns out [rows, N]
+    bf16."""
+    _req(expand_x, "expand_x", torch.uint8)
+    rows, H = expand_x.shape
+    _req(weight, "weight", torch.uint8)
+    E, N = weight.shape[0], weight.shape[1]
+    _req(weight, "weight", torch.uint8, (E, N, H))
+    _req(x_sf, "x_sf", torch.uint8, (rows, H // 32))
+    _req(weight_sf, "weight_sf", torch.uint8, (E, N, H // 32))
+    _req(expert_offsets, "expert_offsets", torch.int32, (E + 1,))
+    if out is None:
+        out = torch.empty((rows, N), dtype=torch.bfloat16, device=expand_x.device)
+    _req(out, "out", torch.bfloat16, (rows, N))
+    p = GmmParams(rows, H, N, E)
+    ws = workspace if workspace is not None else new_workspace(
+        expand_x.device, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
+    _check("moe_grouped_matmul_mx", lib.moe_grouped_matmul_mx(
+        ctypes.byref(p), _ptr(expand_x), _ptr(x_sf), _ptr(expert_offsets), _ptr(weight), _ptr(weight_sf),
+        _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out

@@ -48,12 +48,18 @@ constexpr int kGmMaxStages = 8;
 constexpr int kGmSmemBytes = kGmPipeBytes + 1024;    // + slack to align the ring to 1 KB
 constexpr int kGmThreads = 128;
 constexpr uint32_t kGmTmemCols = 128;                // int32 accumulator columns (>= N)
+// mxfp8: the fp32 accumulator (128 columns) then, per ring stage s, the
+// stage's block factors: 4 columns for the weight rows (A) at 128 + 8 s and
+// 4 for the token rows (B) at 128 + 8 s + 4.
+constexpr uint32_t kGmTmemColsMx = 256;
 
 struct GmmArgs {
     int rows, hidden, out_dim, num_instances, max_slots;
     const float *dyn;          // [rows] per-row factor
     const int32_t *offsets;    // [E + 1]
     const float *wscale;       // [E, N] per-channel factor
+    const uint8_t *xsf;        // mxfp8: [rows, H/32] E8M0 block factors of the rows
+    const uint8_t *wsf;        // mxfp8: [E, N, H/32] E8M0 block factors of the weights
     uint16_t *out;             // [rows, N] bf16
     int4 *slots;               // [max_slots] {instance, first row, rows, 0}
     int *nslots;
@@ -109,6 +115,15 @@ __device__ __forceinline__ uint32_t gm_instr_desc(int n) {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kGmBM >> 4) << 24);
 }
 
+// Block-scaled instruction descriptor, kind::mxf8f6f4: E4M3 A and B, both
+// K-major, E8M0 factors (bit 23), M = 128, N = n (a multiple of 8), and the
+// byte (0..3) of the factor columns this MMA reads, for A (bits 29-30) and B
+// (bits 4-5).  D is always fp32.
+__device__ __forceinline__ uint32_t gm_instr_desc_mx(int n, uint32_t sf_id) {
+    return (sf_id << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(kGmBM >> 4) << 24) | (sf_id << 29);
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -120,6 +135,27 @@ __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t da, uint64_t d
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(da), "l"(db), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// D[128 x N] (+)= A * diag-scaled B with per-32-block E8M0 factors read from
+// TMEM at tsfa / tsfb (the byte the descriptor names).
+__device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t tsfa,
+                                        uint32_t tsfb, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
+        : "memory");
+}
+
+// 32 lanes (this warp's quarter) x 4 consecutive 32-bit columns from v.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&v)[4]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
         : "memory");
 }
 
@@ -168,8 +204,19 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t phase) {
 }
 
 // --- the matmul: grid (ceil(N / 128), max_slots), 128 threads ---
+//
+// MX = false: int8 rows and weights (kind::i8, int32 accumulator), output
+// (acc * dyn[row]) * wscale[channel].  MX = true: E4M3 rows and weights with
+// E8M0 block factors (kind::mxf8f6f4.block_scale, fp32 accumulator), output
+// acc.  In MX mode every thread also places each stage's factors in TMEM:
+// weight rows n0 + 32c + lane and token rows 32c + lane go to column c of the
+// stage's factor slot, lane = row mod 32, one byte per 32-element block of
+// the stage (4 blocks = the 4 MMAs of a 128-element step), replicated into
+// all four lane quarters (warp w writes lanes 32w..32w+31).
+template <bool MX>
 __global__ void __launch_bounds__(kGmThreads, 1)
     gmm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GmmArgs a) {
+    constexpr uint32_t kCols = MX ? kGmTmemColsMx : kGmTmemCols;
     extern __shared__ uint8_t gm_smem_raw[];
     __shared__ __align__(8) uint64_t s_full[kGmMaxStages];
     __shared__ __align__(8) uint64_t s_empty[kGmMaxStages];
@@ -202,7 +249,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                     "r"(kGmTmemCols)
+                     "r"(kCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -213,59 +260,115 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
     const int n0 = blockIdx.x * kGmBM;
     const int nr = slot.z;
-    const int mma_n = (nr + 15) & ~15;
+    const int mma_n = MX ? (nr + 31) & ~31 : (nr + 15) & ~15;  // the factor layout wants whole 32-row groups
     const int nbox = mma_n / kGmBoxRows;
     const int b_bytes = mma_n * kGmBK;
     const int stage_bytes = kGmABytes + b_bytes;  // a multiple of 2 KB
     const int nst = min(kGmMaxStages, kGmPipeBytes / stage_bytes);
     const int nk = (a.hidden + kGmBK - 1) / kGmBK;
+    const uint32_t tx = (uint32_t)stage_bytes;  // out-of-range box parts are zero-filled and still counted
+    const int wrow = slot.x * a.out_dim + n0;
+    const uint32_t ring_s = smem_u32(ring);
 
-    if (t == 0) {
-        const uint32_t tx = (uint32_t)stage_bytes;  // out-of-range box parts are zero-filled and still counted
-        const int wrow = slot.x * a.out_dim + n0;
-        const uint32_t idesc = gm_instr_desc(mma_n);
-        const uint32_t ring_s = smem_u32(ring);
-        int issued = 0;
-        auto issue = [&](int kb) {
-            const int s = kb % nst;
-            uint8_t *sa = ring + s * stage_bytes;
-            mbar_arrive_expect_tx(&s_full[s], tx);
-            tma_load_2d(sa, &tm_w, kb * kGmBK, wrow, &s_full[s]);
-            for (int b = 0; b < nbox; ++b)
-                tma_load_2d(sa + kGmABytes + b * kGmBoxRows * kGmBK, &tm_x, kb * kGmBK, slot.y + b * kGmBoxRows,
-                            &s_full[s]);
-        };
-        for (; issued < nst && issued < nk; ++issued) issue(issued);
-        bool ok = true;
-        int kb = 0;
-        for (; kb < nk; ++kb) {
-            const int s = kb % nst;
-            if (!mbar_wait_bounded(&s_full[s], (uint32_t)(kb / nst) & 1u)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t sa = ring_s + s * stage_bytes;
-            const uint64_t da = gm_smem_desc(sa), db = gm_smem_desc(sa + kGmABytes);
+    auto issue = [&](int kb) {  // thread 0: the copies of k-step kb into its stage
+        const int s = kb % nst;
+        uint8_t *sa = ring + s * stage_bytes;
+        mbar_arrive_expect_tx(&s_full[s], tx);
+        tma_load_2d(sa, &tm_w, kb * kGmBK, wrow, &s_full[s]);
+        for (int b = 0; b < nbox; ++b)
+            tma_load_2d(sa + kGmABytes + b * kGmBoxRows * kGmBK, &tm_x, kb * kGmBK, slot.y + b * kGmBoxRows,
+                        &s_full[s]);
+    };
+    int issued = 0;
+    int pending = -1;  // thread 0, after a timeout: the first step whose copies were not consumed
+    // thread 0: wait for step kb's operands, issue its MMAs, refill the stage
+    // the previous step used.  Returns false on a timeout, with `pending` set.
+    auto mma_step = [&](int kb) -> bool {
+        const int s = kb % nst;
+        if (!mbar_wait_bounded(&s_full[s], (uint32_t)(kb / nst) & 1u)) {
+            pending = kb;
+            return false;
+        }
+        tc_fence_after();
+        const uint32_t sa = ring_s + s * stage_bytes;
+        const uint64_t da = gm_smem_desc(sa), db = gm_smem_desc(sa + kGmABytes);
 #pragma unroll
-            for (int kk = 0; kk < kGmBK / 32; ++kk)  // K = 32 bytes per MMA: +2 in 16-byte units
-                umma_i8(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
-            umma_commit(&s_empty[s]);
-            // refill the stage the previous step used, once its MMAs have read it
-            if (kb >= 1 && issued < nk) {
-                const int sp = (kb - 1) % nst;
-                if (!mbar_wait_bounded(&s_empty[sp], (uint32_t)((kb - 1) / nst) & 1u)) {
-                    ok = false;
-                    ++kb;  // step kb was consumed
-                    break;
-                }
-                issue(issued);
-                ++issued;
+        for (int kk = 0; kk < kGmBK / 32; ++kk) {  // K = 32 per MMA: +32 bytes = +2 in 16-byte units
+            if constexpr (MX) {
+                const uint32_t col = tmem + 128u + 8u * (uint32_t)s;
+                umma_mx(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc_mx(mma_n, (uint32_t)kk),
+                        col | ((uint32_t)kk << 30), (col + 4u) | ((uint32_t)kk << 30), (kb | kk) != 0);
+            } else {
+                umma_i8(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc(mma_n), (kb | kk) != 0);
             }
         }
-        if (!ok) {
+        umma_commit(&s_empty[s]);
+        if (kb >= 1 && issued < nk) {
+            const int sp = (kb - 1) % nst;
+            if (!mbar_wait_bounded(&s_empty[sp], (uint32_t)((kb - 1) / nst) & 1u)) {
+                pending = kb + 1;  // step kb was consumed
+                return false;
+            }
+            issue(issued);
+            ++issued;
+        }
+        return true;
+    };
+
+    if (t == 0)
+        for (; issued < nst && issued < nk; ++issued) issue(issued);
+    if constexpr (!MX) {
+        if (t == 0)
+            for (int kb = 0; kb < nk; ++kb)
+                if (!mma_step(kb)) break;
+        __syncwarp();
+    } else {
+        // every thread: this stage's factor words, two steps ahead in registers
+        const int B = a.hidden >> 5;  // factor bytes per row
+        auto load_sf = [&](int k, uint32_t(&fa)[4], uint32_t(&fb)[4]) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int ch = min(n0 + 32 * c + lane, a.out_dim - 1);
+                fa[c] = __ldg(reinterpret_cast<const uint32_t *>(a.wsf + ((size_t)slot.x * a.out_dim + ch) * B) + k);
+                const int r = min(32 * c + lane, nr - 1);
+                fb[c] = __ldg(reinterpret_cast<const uint32_t *>(a.xsf + (size_t)(slot.y + r) * B) + k);
+            }
+        };
+        const uint32_t quarter = (uint32_t)(warp * 32) << 16;
+        bool failed = false;  // thread 0: a wait of an earlier step gave up
+        // one step: this stage's factors into TMEM, then (thread 0) its MMAs;
+        // false once thread 0 has given up (the barrier hands every thread
+        // the same verdict)
+        auto sf_step = [&](int kb, const uint32_t(&fa)[4], const uint32_t(&fb)[4]) -> bool {
+            const int s = kb % nst;
+            // the slot's previous readers (the MMAs of step kb - nst) completed
+            // before thread 0 refilled that step's stage, two barriers ago
+            tc_fence_after();
+            const uint32_t col = tmem + quarter + 128u + 8u * (uint32_t)s;
+            tmem_st4(col, fa);
+            tmem_st4(col + 4u, fb);
+            tc_fence_before();
+            if (__syncthreads_or(failed)) return false;
+            if (t == 0 && !mma_step(kb)) failed = true;
+            return true;
+        };
+        // factor words two steps ahead, in two register sets used alternately
+        uint32_t fa0[4], fb0[4], fa1[4], fb1[4];
+        load_sf(0, fa0, fb0);
+        if (nk > 1) load_sf(1, fa1, fb1);
+        for (int kb = 0; kb < nk; kb += 2) {
+            if (!sf_step(kb, fa0, fb0)) break;
+            if (kb + 2 < nk) load_sf(kb + 2, fa0, fb0);
+            if (kb + 1 < nk) {
+                if (!sf_step(kb + 1, fa1, fb1)) break;
+                if (kb + 3 < nk) load_sf(kb + 3, fa1, fb1);
+            }
+        }
+    }
+    if (t == 0) {
+        if (pending >= 0) {
             // drain the copies still in flight before the CTA can exit
-            for (int j = kb; j < issued; ++j) mbar_wait_bounded(&s_full[j % nst], (uint32_t)(j / nst) & 1u);
+            for (int j = pending; j < issued; ++j) mbar_wait_bounded(&s_full[j % nst], (uint32_t)(j / nst) & 1u);
             s_fail = 1;
             raise_error(a.err, kDevTimeout);
         }
@@ -280,7 +383,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     if (s_fail == 0 && all_done) {
         const int ch = n0 + warp * 32 + lane;  // this thread's TMEM lane = output channel
         const bool ch_ok = ch < a.out_dim;
-        const float wsc = ch_ok ? a.wscale[(size_t)slot.x * a.out_dim + ch] : 0.0f;
+        float wsc = 0.0f;
+        if constexpr (!MX) wsc = ch_ok ? a.wscale[(size_t)slot.x * a.out_dim + ch] : 0.0f;
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         for (int c0 = 0; c0 < mma_n; c0 += 16) {
             uint32_t v[16];
@@ -290,7 +394,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 const int r = c0 + j;
                 if (r < nr && ch_ok) {
                     const int row = slot.y + r;
-                    const float val = __fmul_rn(__fmul_rn(__int2float_rn((int)v[j]), a.dyn[row]), wsc);
+                    float val;
+                    if constexpr (MX)
+                        val = __uint_as_float(v[j]);
+                    else
+                        val = __fmul_rn(__fmul_rn(__int2float_rn((int)v[j]), a.dyn[row]), wsc);
                     a.out[(size_t)row * a.out_dim + ch] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
                 }
             }
@@ -299,8 +407,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGmTmemCols)
-                     : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
 }
 
 }  // namespace moe

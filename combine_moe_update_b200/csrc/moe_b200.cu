@@ -514,6 +514,40 @@ moe_status moe_grouped_matmul_workspace_size(const moe_gmm_params *p, size_t *by
     return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The planning kernel, then the matmul kernel (int8 or mxfp8) over
+// ceil(N / 128) x max_slots CTAs.
+template <bool MX>
+moe_status launch_gmm(const moe_gmm_params *p, const void *expand_x, const void *weight, moe::GmmArgs a,
+                      void *workspace, cudaStream_t s) {
+    CUtensorMap tm_w, tm_x;
+    if (!encode_i8_rows(&tm_w, weight, (uint64_t)p->hidden, (uint64_t)p->num_instances * p->out_dim, moe::kGmBM) ||
+        !encode_i8_rows(&tm_x, expand_x, (uint64_t)p->hidden, (uint64_t)p->rows, moe::kGmBoxRows))
+        return MOE_ERR_CUDA;
+    unsigned char *ws = reinterpret_cast<unsigned char *>(workspace);
+    a.rows = p->rows;
+    a.hidden = p->hidden;
+    a.out_dim = p->out_dim;
+    a.num_instances = p->num_instances;
+    a.max_slots = moe::gmm_max_slots(p->rows, p->num_instances);
+    a.nslots = reinterpret_cast<int *>(ws + kWorkspaceBytes);
+    a.slots = reinterpret_cast<int4 *>(ws + kWorkspaceBytes + 16);
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    if (!ensure_smem(moe::gmm_kernel<MX>, moe::kGmSmemBytes)) return MOE_ERR_CUDA;
+    if (launch(moe::gmm_plan_kernel, dim3(1), 1024, 0, s, a) != cudaSuccess) return MOE_ERR_CUDA;
+    const dim3 grid((p->out_dim + moe::kGmBM - 1) / moe::kGmBM, a.max_slots);
+    return launch(moe::gmm_kernel<MX>, grid, moe::kGmThreads, moe::kGmSmemBytes, s, tm_w, tm_x, a) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
 moe_status moe_grouped_matmul(const moe_gmm_params *p, const void *expand_x, const float *dyn_scales,
                               const int32_t *expert_offsets, const void *weight, const float *weight_scales,
                               void *out, void *workspace, size_t workspace_bytes, void *cuda_stream) {
@@ -524,31 +558,30 @@ moe_status moe_grouped_matmul(const moe_gmm_params *p, const void *expand_x, con
         return MOE_ERR_INVALID_ARG;
     if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < gmm_workspace_bytes(*p))
         return MOE_ERR_WORKSPACE;
-    CUtensorMap tm_w, tm_x;
-    if (!encode_i8_rows(&tm_w, weight, (uint64_t)p->hidden, (uint64_t)p->num_instances * p->out_dim, moe::kGmBM) ||
-        !encode_i8_rows(&tm_x, expand_x, (uint64_t)p->hidden, (uint64_t)p->rows, moe::kGmBoxRows))
-        return MOE_ERR_CUDA;
-    unsigned char *ws = reinterpret_cast<unsigned char *>(workspace);
     moe::GmmArgs a = {};
-    a.rows = p->rows;
-    a.hidden = p->hidden;
-    a.out_dim = p->out_dim;
-    a.num_instances = p->num_instances;
-    a.max_slots = moe::gmm_max_slots(p->rows, p->num_instances);
     a.dyn = dyn_scales;
     a.offsets = expert_offsets;
     a.wscale = weight_scales;
     a.out = reinterpret_cast<uint16_t *>(out);
-    a.nslots = reinterpret_cast<int *>(ws + kWorkspaceBytes);
-    a.slots = reinterpret_cast<int4 *>(ws + kWorkspaceBytes + 16);
-    a.err = reinterpret_cast<uint32_t *>(workspace);
-    cudaStream_t s = as_stream(cuda_stream);
-    if (!ensure_smem(moe::gmm_kernel, moe::kGmSmemBytes)) return MOE_ERR_CUDA;
-    if (launch(moe::gmm_plan_kernel, dim3(1), 1024, 0, s, a) != cudaSuccess) return MOE_ERR_CUDA;
-    const dim3 grid((p->out_dim + moe::kGmBM - 1) / moe::kGmBM, a.max_slots);
-    return launch(moe::gmm_kernel, grid, moe::kGmThreads, moe::kGmSmemBytes, s, tm_w, tm_x, a) == cudaSuccess
-               ? MOE_OK
-               : MOE_ERR_CUDA;
+    return launch_gmm<false>(p, expand_x, weight, a, workspace, as_stream(cuda_stream));
+}
+
+moe_status moe_grouped_matmul_mx(const moe_gmm_params *p, const void *expand_x, const uint8_t *x_sf,
+                                 const int32_t *expert_offsets, const void *weight, const uint8_t *weight_sf,
+                                 void *out, void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr || !valid_gmm(*p) || p->hidden % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (!expand_x || !x_sf || !expert_offsets || !weight || !weight_sf || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(expand_x, 16) || !aligned(weight, 16) || !aligned(out, 16) || !aligned(x_sf, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(weight_sf, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < gmm_workspace_bytes(*p))
+        return MOE_ERR_WORKSPACE;
+    moe::GmmArgs a = {};
+    a.offsets = expert_offsets;
+    a.xsf = x_sf;
+    a.wsf = weight_sf;
+    a.out = reinterpret_cast<uint16_t *>(out);
+    return launch_gmm<true>(p, expand_x, weight, a, workspace, as_stream(cuda_stream));
 }
 
 // ------------------------------------------------------- dispatch, no alloc ---

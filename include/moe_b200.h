@@ -322,6 +322,26 @@ MOE_API moe_status moe_grouped_matmul(const moe_gmm_params *p, const void *expan
                                       const float *weight_scales, void *out, void *workspace,
                                       size_t workspace_bytes, void *cuda_stream);
 
+/*
+ * The same step on mxfp8 rows (moe_dispatch quant_mode 4) and mxfp8 weights,
+ * on the block-scaled tensor-core path:
+ *   out[r][n] = sum_h dec(expand_x[r][h]) * 2^(x_sf[r][h/32] - 127)
+ *                    * dec(weight[e][n][h]) * 2^(weight_sf[e][n][h/32] - 127)
+ * where dec is the E4M3 value of a code; the sum is formed by the tensor
+ * cores in fp32 and rounded to bf16 once.
+ *
+ *   expand_x   [rows, H] E4M3 codes (uint8) device, 16-byte aligned
+ *   x_sf       [rows, H/32] uint8 E8M0 device, 4-byte aligned (the dispatch's mode-4 dyn_scales)
+ *   weight     [E, N, H] E4M3 codes device, 16-byte aligned
+ *   weight_sf  [E, N, H/32] uint8 E8M0 device, 4-byte aligned
+ * Other arguments, limits and errors as moe_grouped_matmul, plus H % 128 == 0
+ * (each 128-element step reads one 4-byte word of factors per row).
+ */
+MOE_API moe_status moe_grouped_matmul_mx(const moe_gmm_params *p, const void *expand_x, const uint8_t *x_sf,
+                                         const int32_t *expert_offsets, const void *weight,
+                                         const uint8_t *weight_sf, void *out, void *workspace,
+                                         size_t workspace_bytes, void *cuda_stream);
+
 /* ------------------------------------------------------------------------ */
 /* moe_dispatch_noalloc -- moe_dispatch without a caller-provided workspace  */
 /* ------------------------------------------------------------------------ */

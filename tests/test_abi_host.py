@@ -220,3 +220,18 @@ def test_no_cpu_fallback_in_product():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b|moe_oracle|orc_", src, re.M), fn
+
+
+def test_grouped_matmul_mx_rules(L):
+    """mxfp8 adds H % 128 == 0 (one 4-byte factor word per row and step) and
+    4-byte aligned factor arrays."""
+    f, f2, f8 = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10002), ctypes.c_void_p(0x10008)
+    p = _gmm_params(L)
+    n = ws_size(L, "moe_grouped_matmul_workspace_size", p)[1]
+    call = lambda p=p, x=f, xs=f, off=f, w=f, wsf=f, out=f, ws=f, wsb=n: L.lib.moe_grouped_matmul_mx(
+        ctypes.byref(p), x, xs, off, w, wsf, out, ws, wsb, None)
+    assert call(p=_gmm_params(L, hidden=1056)) == L.MOE_ERR_INVALID_ARG  # % 32 but not % 128
+    for kw in (dict(x=None), dict(xs=None), dict(wsf=None), dict(x=f8), dict(w=f8), dict(xs=f2), dict(wsf=f2),
+               dict(off=f2)):
+        assert call(**kw) == L.MOE_ERR_INVALID_ARG, kw
+    assert call(wsb=n - 16) == L.MOE_ERR_WORKSPACE

@@ -185,3 +185,96 @@ def test_dispatch_gmm_combine_pipeline(B):
     _assert_gmm_parity(host(ex)[:n], dict(out=go["out"][:n], out_f64=go["out_f64"][:n]))
     assert_close_bf16(host(c["y"]), co["y_f64"], what="y")
     assert_close_bf16(host(c["x_out"]), co["x_f64"], what="x_out")
+
+
+# ------------------------------------------------------------------ mxfp8
+
+def _gpu_mx(B, gi):
+    rows, H = gi.expand_x.shape
+    E, N = gi.weight.shape[0], gi.weight.shape[1]
+    out = poison_(torch.empty((rows, N), dtype=torch.bfloat16, device="cuda"))
+    wsp = B.new_workspace(nbytes=B.grouped_matmul_workspace_bytes(rows, H, N, E))
+    B.grouped_matmul_mx(dev(gi.expand_x), dev(gi.x_sf), dev(gi.offsets), dev(gi.weight), dev(gi.weight_sf), out=out,
+                        workspace=wsp)
+    torch.cuda.synchronize()
+    return host(out), B.read_device_error(wsp)
+
+
+def _oracle_mx(gi):
+    rows, N = gi.expand_x.shape[0], gi.weight.shape[1]
+    return orc.grouped_matmul_mx(gi.expand_x, gi.x_sf, gi.offsets, gi.weight, gi.weight_sf,
+                                 out=np.full((rows, N), POISON16, np.uint16))
+
+
+@pytest.mark.parametrize("H,N,counts,spare", [
+    (1024, 256, [3, 0, 17, 130, 1, 128, 16], 5),
+    (1152, 208, [5, 33, 0, 260], 0),
+])
+def test_gmm_mx_single_products_bit_exact(B, H, N, counts, spare):
+    """One non-zero E4M3 code per row: every output is one product of two
+    E4M3 values (at most 8 significant bits) times two powers of two, exact
+    in bf16, so the operand layouts and the placement of every block factor
+    are checked bit for bit."""
+    gi = gen.gmm_inputs_mx(41, counts, H, N, spare_rows=spare, one_hot=True)
+    got, err = _gpu_mx(B, gi)
+    o = _oracle_mx(gi)
+    assert err == 0 and o["err"] == 0
+    np.testing.assert_array_equal(got, o["out"])
+
+
+@pytest.mark.parametrize("H,N,counts,spare", [
+    (1024, 128, [40, 0, 1, 129, 77], 3),
+    (2048, 256, [128, 256, 255, 16, 15], 0),
+    (7168, 384, [24, 9, 0, 140], 1),
+])
+def test_gmm_mx_parity_random(B, H, N, counts, spare):
+    """Full-range E4M3 rows and weights with random block factors: within the
+    1e-2 bar everywhere (the tensor cores sum in fp32, the oracle in
+    binary64), and nearly all outputs within one bf16 step."""
+    gi = gen.gmm_inputs_mx(42, counts, H, N, spare_rows=spare)
+    got, err = _gpu_mx(B, gi)
+    o = _oracle_mx(gi)
+    assert err == 0 and o["err"] == 0
+    written = ~np.isnan(o["out_f64"])
+    np.testing.assert_array_equal(got[~written], o["out"][~written])
+    rows = np.flatnonzero(written.any(axis=1))
+    assert_close_bf16(got[rows], o["out_f64"][rows], what="mx gmm out")
+    step = np.abs(got[written].astype(np.int32) - o["out"][written].astype(np.int32))
+    assert (step <= 1).mean() >= 0.99
+
+
+def test_dispatch_mx_gmm_combine_pipeline(B):
+    """update_expert -> dispatch (mxfp8) -> mxfp8 matmul (N = H) ->
+    combine+Add+RMSNorm on the GPU, against the same chain of oracle calls."""
+    w = gen.uniform_layer("pipe_mx", 33, bs=64, hidden=1024, num_experts=16, top_k=4, ep_world_size=4,
+                          quant_mode=4, shared=True)
+    wt = gen.gmm_inputs_mx(34, [0] * w.num_instances, w.hidden, w.hidden)
+    ids, table, sc = dev(w.expert_ids), dev(w.table), dev(w.expert_scales)
+    ws = B.new_workspace(nbytes=4096)
+    bal = torch.empty_like(ids)
+    bm = torch.empty(ids.shape, dtype=torch.uint8, device="cuda")
+    B.update_expert(ids, table, w.ep_world_size, expert_scales=sc, workspace=ws, out=(bal, bm))
+    d = B.alloc_dispatch_outputs(w.bs, w.hidden, w.top_k, w.num_instances, w.quant_mode)
+    B.dispatch(dev_bf16(w.x), bal, w.num_instances, w.ep_world_size, w.quant_mode, mask=bm, workspace=ws, out=d)
+    rows = d["expand_x"].shape[0]
+    ex = torch.zeros((rows, w.hidden), dtype=torch.bfloat16, device="cuda")
+    B.grouped_matmul_mx(d["expand_x"].view(torch.uint8), d["dyn_scales"].view(torch.uint8), d["offsets"],
+                        dev(wt.weight), dev(wt.weight_sf), out=ex,
+                        workspace=B.new_workspace(nbytes=B.grouped_matmul_workspace_bytes(rows, w.hidden, w.hidden,
+                                                                                          w.num_instances)))
+    c = B.combine_add_rmsnorm(ex, d["expand_idx"], sc, dev_bf16(w.residual), dev_bf16(w.gamma), w.norm_eps,
+                              shared_x=dev_bf16(w.shared_x), want_x_out=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert B.read_device_error(ws) == 0
+    bal_o, bm_o, e1 = orc.update_expert(w.expert_ids, w.table, w.ep_world_size, expert_scales=w.expert_scales)
+    do = orc.dispatch(w.x, bal_o, w.num_instances, w.quant_mode, mask=bm_o)
+    go = orc.grouped_matmul_mx(do["expand_x"], do["dyn_scales"], do["offsets"], wt.weight, wt.weight_sf,
+                               out=np.zeros((rows, w.hidden), np.uint16))
+    co = orc.combine_add_rmsnorm(go["out"], do["expand_idx"], w.expert_scales, w.residual, w.gamma, w.norm_eps,
+                                 shared_x=w.shared_x)
+    assert e1 == 0 and do["err"] == 0 and go["err"] == 0
+    n = do["n"]
+    np.testing.assert_array_equal(host(d["expand_x"].view(torch.uint8))[:n], do["expand_x"][:n])
+    np.testing.assert_array_equal(host(d["dyn_scales"].view(torch.uint8))[:n], do["dyn_scales"][:n])
+    assert_close_bf16(host(ex)[:n], go["out_f64"][:n], what="mx gmm out")
+    assert_close_bf16(host(c["y"]), co["y_f64"], what="y")
