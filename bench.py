@@ -457,15 +457,18 @@ def run_b200(args, rank, world, local_rank):
     return out, w
 
 
-def gmm_bytes(offsets, hidden, out_dim):
+def gmm_bytes(offsets, hidden, out_dim, mx=False):
     """Algorithmic bytes of one grouped matmul: the weights of every instance
-    that received rows (read once), the rows (int8) and their factors, the
-    channel factors, the offsets, and the bf16 output rows."""
+    that received rows (read once), the rows (one byte per element) and their
+    factors, the weights' factors, the offsets, and the bf16 output rows.
+    Factors: int8 one f32 per row and per channel; mxfp8 one byte per
+    32-element block of every row and weight row."""
     import numpy as np
     off = np.asarray(offsets, np.int64)
     used = int(np.count_nonzero(np.diff(off)))
     n = int(off[-1] - off[0])
-    return used * out_dim * hidden + used * out_dim * 4 + n * hidden + n * 4 + n * out_dim * 2 + off.size * 4
+    f_w, f_x = (out_dim * (hidden // 32), hidden // 32) if mx else (out_dim * 4, 4)
+    return used * out_dim * hidden + used * f_w + n * hidden + n * f_x + n * out_dim * 2 + off.size * 4
 
 
 def run_b200_expert(args, rank, world, local_rank, w):
@@ -486,7 +489,13 @@ def run_b200_expert(args, rank, world, local_rank, w):
     table = dev(w.table)
     smooth = None if w.smooth is None else dev(w.smooth)
     gamma = bf(w.gamma)
-    weight, wscale = gen.gmm_weights_device(w.meta["weight_seed"], E, N, H, "cuda")
+    mx = w.quant_mode == 4  # mxfp8 rows: mxfp8 weights on the block-scaled path
+    if mx:
+        weight, wscale = gen.gmm_weights_device_mx(w.meta["weight_seed"], E, N, H, "cuda")
+        gmm = functools.partial(B.grouped_matmul_mx, weight=weight, weight_sf=wscale)
+    else:
+        weight, wscale = gen.gmm_weights_device(w.meta["weight_seed"], E, N, H, "cuda")
+        gmm = functools.partial(B.grouped_matmul, weight=weight, weight_scales=wscale)
     ids, scales = dev(w.expert_ids), dev(w.expert_scales)
     x, residual = bf(w.x), bf(w.residual)
     shared = None if w.shared_x is None else bf(w.shared_x)
@@ -507,7 +516,7 @@ def run_b200_expert(args, rank, world, local_rank, w):
         mark(1)
         B.dispatch(xx, bal, E, w.ep_world_size, w.quant_mode, mask=bm, smooth=smooth, workspace=ws, out=d)
         mark(2)
-        B.grouped_matmul(d["expand_x"], d["dyn_scales"], d["offsets"], weight, wscale, out=ex, workspace=gws)
+        gmm(d["expand_x"], d["dyn_scales"], d["offsets"], out=ex, workspace=gws)
         mark(3)
         B.combine_add_rmsnorm(ex, d["expand_idx"], ss, rr, gamma, w.norm_eps, shared_x=sh, workspace=ws, out=c)
 
@@ -526,7 +535,7 @@ def run_b200_expert(args, rank, world, local_rank, w):
     off = d["offsets"].cpu().numpy()
     n = int(off[-1])
     alg = algorithmic_bytes(w, n)
-    alg["grouped_matmul"] = gmm_bytes(off, H, N)
+    alg["grouped_matmul"] = gmm_bytes(off, H, N, mx)
     # the combine reads the matmul's rows instead of the stand-in rows: same byte count
 
     K = args.steps
@@ -581,7 +590,7 @@ def run_b200_expert(args, rank, world, local_rank, w):
     with torch.cuda.graph(graph_g, stream=cap):
         eb[0].record()
         for _ in range(M):
-            B.grouped_matmul(d["expand_x"], d["dyn_scales"], d["offsets"], weight, wscale, out=ex, workspace=gws)
+            gmm(d["expand_x"], d["dyn_scales"], d["offsets"], out=ex, workspace=gws)
         eb[1].record()
     graph_g.replay()
     torch.cuda.synchronize()
@@ -634,7 +643,8 @@ def run_b200_expert(args, rank, world, local_rank, w):
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8+int32 (matmul), fp32",
+        "vs_baseline": None,
+        "dtype": "fp8e4m3 with E8M0 blocks (matmul fp32 accumulate)" if mx else "int8+int32 (matmul), fp32",
         "data": "synthetic (seeded; pages' shapes; instance weights drawn on the device)",
         "config": {"workload": args.workload, "bs": w.bs, "hidden": H, "top_k": w.top_k, "num_instances": E,
                    "ep_world_size_simulated": w.ep_world_size, "quant_mode": w.quant_mode,
@@ -645,11 +655,11 @@ def run_b200_expert(args, rank, world, local_rank, w):
         "breakdown_us": {"update_expert": round(t_upd * 1e3, 2), "dispatch": round(t_disp * 1e3, 2),
                          "grouped_matmul": round(t_gm * 1e3, 2), "combine": round(t_comb * 1e3, 2)},
         "achieved_gbs": {"step": round(step_bytes / (t_step * 1e-3) / 1e9, 1), "grouped_matmul": round(achieved, 1)},
-        "roofline": {"bound": "hbm", "kernel": "gmm_kernel", "achieved": round(achieved, 1), "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": "gmm_mx_kernel" if mx else "gmm_kernel", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "launch_us": round(t_gmm * 1e3, 2),
                      "timing": f"{M} back-to-back calls (planning + matmul kernel) in a graph, CUDA events around them",
-                     "traffic": stored_traffic("gmm_kernel", args.workload),
+                     "traffic": stored_traffic("gmm_mx_kernel" if mx else "gmm_kernel", args.workload),
                      "algorithmic_bytes": alg["grouped_matmul"],
                      "tensor_tops": round(2.0 * n * N * H / (t_gmm * 1e-3) / 1e12, 1)},
         "e2e": {"value": round(world * w.bs / (t_e2e * 1e-3), 1), "unit": "tokens/s",
@@ -687,14 +697,19 @@ def _oracle_expert_rows(orc, w, d):
     used = [e for e in range(w.num_instances) if off[e + 1] > off[e]]
     cache = w.meta.setdefault("_host_weights", {})
     key = tuple(used)
+    mx = w.quant_mode == 4
     if key not in cache:
-        hw = gen.gmm_weights_host(w.meta["weight_seed"], used, w.meta["expert_out_dim"], w.hidden)
+        draw = gen.gmm_weights_host_mx if mx else gen.gmm_weights_host
+        hw = draw(w.meta["weight_seed"], used, w.meta["expert_out_dim"], w.hidden)
         cache.clear()
         cache[key] = (np.stack([hw[e][0] for e in used]), np.stack([hw[e][1] for e in used]))
     wts, wss = cache[key]
     off_c = np.array([off[e] for e in used] + [off[-1]], np.int32)
-    g = orc.grouped_matmul(d["expand_x"], d["dyn_scales"], off_c, wts, wss,
-                           out=np.zeros((d["expand_x"].shape[0], w.meta["expert_out_dim"]), np.uint16))
+    out = np.zeros((d["expand_x"].shape[0], w.meta["expert_out_dim"]), np.uint16)
+    if mx:
+        g = orc.grouped_matmul_mx(d["expand_x"], d["dyn_scales"], off_c, wts, wss, out=out)
+    else:
+        g = orc.grouped_matmul(d["expand_x"], d["dyn_scales"], off_c, wts, wss, out=out)
     return g["out"]
 
 

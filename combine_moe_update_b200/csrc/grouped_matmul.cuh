@@ -150,12 +150,15 @@ __device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t da, uint64_t d
         : "memory");
 }
 
-// 32 lanes (this warp's quarter) x 4 consecutive 32-bit columns from v.
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&v)[4]) {
+// 32 lanes (this warp's quarter) x 8 consecutive 32-bit columns:
+// col..col+3 from va, col+4..col+7 from vb, with one wait for both.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&va)[4], const uint32_t (&vb)[4]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};\n\t"
+        "tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%2, %3, %4, %5};\n\t"
+        "tcgen05.st.sync.aligned.32x32b.x4.b32 [%1], {%6, %7, %8, %9};\n\t"
         "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+        "r"(taddr + 4u), "r"(va[0]), "r"(va[1]), "r"(va[2]), "r"(va[3]), "r"(vb[0]), "r"(vb[1]), "r"(vb[2]),
+        "r"(vb[3])
         : "memory");
 }
 
@@ -203,20 +206,14 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t phase) {
     return false;
 }
 
-// --- the matmul: grid (ceil(N / 128), max_slots), 128 threads ---
+// --- the int8 matmul: grid (ceil(N / 128), max_slots), 128 threads ---
 //
-// MX = false: int8 rows and weights (kind::i8, int32 accumulator), output
-// (acc * dyn[row]) * wscale[channel].  MX = true: E4M3 rows and weights with
-// E8M0 block factors (kind::mxf8f6f4.block_scale, fp32 accumulator), output
-// acc.  In MX mode every thread also places each stage's factors in TMEM:
-// weight rows n0 + 32c + lane and token rows 32c + lane go to column c of the
-// stage's factor slot, lane = row mod 32, one byte per 32-element block of
-// the stage (4 blocks = the 4 MMAs of a 128-element step), replicated into
-// all four lane quarters (warp w writes lanes 32w..32w+31).
-template <bool MX>
+// int8 rows and weights (kind::i8, int32 accumulator), output
+// (acc * dyn[row]) * wscale[channel].  One elected thread issues both the
+// copies and the MMAs; the other threads wait for the accumulator.
 __global__ void __launch_bounds__(kGmThreads, 1)
     gmm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GmmArgs a) {
-    constexpr uint32_t kCols = MX ? kGmTmemColsMx : kGmTmemCols;
+    constexpr uint32_t kCols = kGmTmemCols;
     extern __shared__ uint8_t gm_smem_raw[];
     __shared__ __align__(8) uint64_t s_full[kGmMaxStages];
     __shared__ __align__(8) uint64_t s_empty[kGmMaxStages];
@@ -260,7 +257,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
     const int n0 = blockIdx.x * kGmBM;
     const int nr = slot.z;
-    const int mma_n = MX ? (nr + 31) & ~31 : (nr + 15) & ~15;  // the factor layout wants whole 32-row groups
+    const int mma_n = (nr + 15) & ~15;
     const int nbox = mma_n / kGmBoxRows;
     const int b_bytes = mma_n * kGmBK;
     const int stage_bytes = kGmABytes + b_bytes;  // a multiple of 2 KB
@@ -293,15 +290,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         const uint32_t sa = ring_s + s * stage_bytes;
         const uint64_t da = gm_smem_desc(sa), db = gm_smem_desc(sa + kGmABytes);
 #pragma unroll
-        for (int kk = 0; kk < kGmBK / 32; ++kk) {  // K = 32 per MMA: +32 bytes = +2 in 16-byte units
-            if constexpr (MX) {
-                const uint32_t col = tmem + 128u + 8u * (uint32_t)s;
-                umma_mx(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc_mx(mma_n, (uint32_t)kk),
-                        col | ((uint32_t)kk << 30), (col + 4u) | ((uint32_t)kk << 30), (kb | kk) != 0);
-            } else {
-                umma_i8(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc(mma_n), (kb | kk) != 0);
-            }
-        }
+        for (int kk = 0; kk < kGmBK / 32; ++kk)  // K = 32 per MMA: +32 bytes = +2 in 16-byte units
+            umma_i8(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc(mma_n), (kb | kk) != 0);
         umma_commit(&s_empty[s]);
         if (kb >= 1 && issued < nk) {
             const int sp = (kb - 1) % nst;
@@ -317,54 +307,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
     if (t == 0)
         for (; issued < nst && issued < nk; ++issued) issue(issued);
-    if constexpr (!MX) {
-        if (t == 0)
-            for (int kb = 0; kb < nk; ++kb)
-                if (!mma_step(kb)) break;
-        __syncwarp();
-    } else {
-        // every thread: this stage's factor words, two steps ahead in registers
-        const int B = a.hidden >> 5;  // factor bytes per row
-        auto load_sf = [&](int k, uint32_t(&fa)[4], uint32_t(&fb)[4]) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int ch = min(n0 + 32 * c + lane, a.out_dim - 1);
-                fa[c] = __ldg(reinterpret_cast<const uint32_t *>(a.wsf + ((size_t)slot.x * a.out_dim + ch) * B) + k);
-                const int r = min(32 * c + lane, nr - 1);
-                fb[c] = __ldg(reinterpret_cast<const uint32_t *>(a.xsf + (size_t)(slot.y + r) * B) + k);
-            }
-        };
-        const uint32_t quarter = (uint32_t)(warp * 32) << 16;
-        bool failed = false;  // thread 0: a wait of an earlier step gave up
-        // one step: this stage's factors into TMEM, then (thread 0) its MMAs;
-        // false once thread 0 has given up (the barrier hands every thread
-        // the same verdict)
-        auto sf_step = [&](int kb, const uint32_t(&fa)[4], const uint32_t(&fb)[4]) -> bool {
-            const int s = kb % nst;
-            // the slot's previous readers (the MMAs of step kb - nst) completed
-            // before thread 0 refilled that step's stage, two barriers ago
-            tc_fence_after();
-            const uint32_t col = tmem + quarter + 128u + 8u * (uint32_t)s;
-            tmem_st4(col, fa);
-            tmem_st4(col + 4u, fb);
-            tc_fence_before();
-            if (__syncthreads_or(failed)) return false;
-            if (t == 0 && !mma_step(kb)) failed = true;
-            return true;
-        };
-        // factor words two steps ahead, in two register sets used alternately
-        uint32_t fa0[4], fb0[4], fa1[4], fb1[4];
-        load_sf(0, fa0, fb0);
-        if (nk > 1) load_sf(1, fa1, fb1);
-        for (int kb = 0; kb < nk; kb += 2) {
-            if (!sf_step(kb, fa0, fb0)) break;
-            if (kb + 2 < nk) load_sf(kb + 2, fa0, fb0);
-            if (kb + 1 < nk) {
-                if (!sf_step(kb + 1, fa1, fb1)) break;
-                if (kb + 3 < nk) load_sf(kb + 3, fa1, fb1);
-            }
-        }
-    }
+    if (t == 0)
+        for (int kb = 0; kb < nk; ++kb)
+            if (!mma_step(kb)) break;
+    __syncwarp();
     if (t == 0) {
         if (pending >= 0) {
             // drain the copies still in flight before the CTA can exit
@@ -383,8 +329,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     if (s_fail == 0 && all_done) {
         const int ch = n0 + warp * 32 + lane;  // this thread's TMEM lane = output channel
         const bool ch_ok = ch < a.out_dim;
-        float wsc = 0.0f;
-        if constexpr (!MX) wsc = ch_ok ? a.wscale[(size_t)slot.x * a.out_dim + ch] : 0.0f;
+        const float wsc = ch_ok ? a.wscale[(size_t)slot.x * a.out_dim + ch] : 0.0f;
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         for (int c0 = 0; c0 < mma_n; c0 += 16) {
             uint32_t v[16];
@@ -394,11 +339,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 const int r = c0 + j;
                 if (r < nr && ch_ok) {
                     const int row = slot.y + r;
-                    float val;
-                    if constexpr (MX)
-                        val = __uint_as_float(v[j]);
-                    else
-                        val = __fmul_rn(__fmul_rn(__int2float_rn((int)v[j]), a.dyn[row]), wsc);
+                    const float val = __fmul_rn(__fmul_rn(__int2float_rn((int)v[j]), a.dyn[row]), wsc);
                     a.out[(size_t)row * a.out_dim + ch] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
                 }
             }
@@ -408,6 +349,195 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     __syncthreads();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
+}
+
+// --- the mxfp8 matmul, warp-specialized: grid (ceil(N / 128), max_slots), 192 threads ---
+//
+// Warps 0-3 place each stage's block factors in TMEM (warp w writes lanes
+// 32w..32w+31, so the four copies the tensor cores read are all written) and
+// later run the epilogue; warp 4 (one lane) issues the TMA copies; warp 5
+// (one lane) issues the MMAs.  Per ring stage s three mbarriers hand the
+// stage around: full[s] (the copies landed), sf_full[s] (the four factor
+// warps wrote the stage's factors) and empty[s] (tcgen05.commit: the MMAs
+// that read the stage's operands and factors completed), so no role waits
+// for another except through the stage it needs.
+constexpr int kGmMxThreads = 192;
+
+__global__ void __launch_bounds__(kGmMxThreads, 1)
+    gmm_mx_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GmmArgs a) {
+    extern __shared__ uint8_t gm_smem_raw[];
+    __shared__ __align__(8) uint64_t s_full[kGmMaxStages];
+    __shared__ __align__(8) uint64_t s_sf[kGmMaxStages];
+    __shared__ __align__(8) uint64_t s_empty[kGmMaxStages];
+    __shared__ __align__(8) uint64_t s_done;
+    __shared__ uint32_t s_tmem;
+    __shared__ int4 s_slot;
+    __shared__ int s_fail;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    uint8_t *ring = gm_smem_raw + ((1024u - (smem_u32(gm_smem_raw) & 1023u)) & 1023u);
+
+    if (t == 0) {
+        for (int s = 0; s < kGmMaxStages; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_sf[s], 4);
+            mbar_init(&s_empty[s], 1);
+        }
+        mbar_init(&s_done, 1);
+        s_fail = 0;
+        tma_prefetch_map(&tm_w);
+        tma_prefetch_map(&tm_x);
+    }
+    pdl_wait();  // slots from the planning kernel; rows and factors from earlier kernels
+    if (t == 0) {
+        const int ns = *a.nslots;
+        s_slot = (int)blockIdx.y < ns ? a.slots[blockIdx.y] : make_int4(-1, 0, 0, 0);
+    }
+    __syncthreads();
+    const int4 slot = s_slot;
+    if (slot.x < 0) return;
+
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(kGmTmemColsMx)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    const int n0 = blockIdx.x * kGmBM;
+    const int nr = slot.z;
+    const int mma_n = (nr + 31) & ~31;  // the factor layout wants whole 32-row groups
+    const int nbox = mma_n / kGmBoxRows;
+    const int stage_bytes = kGmABytes + mma_n * kGmBK;  // a multiple of 2 KB
+    const int nst = min(kGmMaxStages, kGmPipeBytes / stage_bytes);
+    const int nk = (a.hidden + kGmBK - 1) / kGmBK;
+
+    if (warp == 4) {
+        if (lane == 0) {  // the TMA producer
+            const uint32_t tx = (uint32_t)stage_bytes;
+            const int wrow = slot.x * a.out_dim + n0;
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % nst;
+                if (kb >= nst && !mbar_wait_bounded(&s_empty[s], (uint32_t)(kb / nst - 1) & 1u)) {
+                    s_fail = 1;
+                    break;
+                }
+                uint8_t *sa = ring + s * stage_bytes;
+                mbar_arrive_expect_tx(&s_full[s], tx);
+                tma_load_2d(sa, &tm_w, kb * kGmBK, wrow, &s_full[s]);
+                for (int b = 0; b < nbox; ++b)
+                    tma_load_2d(sa + kGmABytes + b * kGmBoxRows * kGmBK, &tm_x, kb * kGmBK, slot.y + b * kGmBoxRows,
+                                &s_full[s]);
+                ++issued;
+            }
+            // every copy issued has landed before the CTA can end (at once, unless a wait gave up)
+            for (int j = max(0, issued - nst); j < issued; ++j)
+                if (!mbar_wait_bounded(&s_full[j % nst], (uint32_t)(j / nst) & 1u)) s_fail = 1;
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {  // the MMA issuer
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % nst;
+                const uint32_t ph = (uint32_t)(kb / nst) & 1u;
+                if (!mbar_wait_bounded(&s_full[s], ph) || !mbar_wait_bounded(&s_sf[s], ph)) {
+                    s_fail = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(ring + s * stage_bytes);
+                const uint64_t da = gm_smem_desc(sa), db = gm_smem_desc(sa + kGmABytes);
+                const uint32_t col = tmem + 128u + 8u * (uint32_t)s;
+#pragma unroll
+                for (int kk = 0; kk < kGmBK / 32; ++kk)
+                    umma_mx(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc_mx(mma_n, (uint32_t)kk),
+                            col | ((uint32_t)kk << 30), (col + 4u) | ((uint32_t)kk << 30), (kb | kk) != 0);
+                umma_commit(&s_empty[s]);
+            }
+            umma_commit(&s_done);  // fires once every MMA above has completed
+        }
+    } else {  // warps 0-3: the block factors of every stage
+        const int B = a.hidden >> 5;  // factor bytes per row
+        auto load_sf = [&](int k, uint32_t(&fa)[4], uint32_t(&fb)[4]) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int ch = min(n0 + 32 * c + lane, a.out_dim - 1);
+                fa[c] = __ldg(reinterpret_cast<const uint32_t *>(a.wsf + ((size_t)slot.x * a.out_dim + ch) * B) + k);
+                const int r = min(32 * c + lane, nr - 1);
+                fb[c] = __ldg(reinterpret_cast<const uint32_t *>(a.xsf + (size_t)(slot.y + r) * B) + k);
+            }
+        };
+        const uint32_t quarter = (uint32_t)(warp * 32) << 16;
+        auto sf_step = [&](int kb, const uint32_t(&fa)[4], const uint32_t(&fb)[4]) -> bool {
+            const int s = kb % nst;
+            // the slot is free once the MMAs of step kb - nst completed
+            bool ok = true;
+            if (kb >= nst) {
+                if (lane == 0) ok = mbar_wait_bounded(&s_empty[s], (uint32_t)(kb / nst - 1) & 1u);
+                ok = __shfl_sync(kFull, ok, 0);
+                if (!ok) return false;
+            }
+            tc_fence_after();
+            const uint32_t col = tmem + quarter + 128u + 8u * (uint32_t)s;
+            tmem_st8(col, fa, fb);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_sf[s]);
+            return true;
+        };
+        // factor words four steps ahead (a weight row's 32-byte sector holds
+        // eight steps, so one load in eight goes to DRAM), in four register
+        // sets used in turn
+        constexpr int kPre = 4;
+        uint32_t fa[kPre][4], fb[kPre][4];
+#pragma unroll
+        for (int q = 0; q < kPre; ++q)
+            if (q < nk) load_sf(q, fa[q], fb[q]);
+        bool stop = false;
+        for (int kb0 = 0; kb0 < nk && !stop; kb0 += kPre) {
+#pragma unroll
+            for (int q = 0; q < kPre; ++q) {  // constant register-set index after unrolling
+                const int kb = kb0 + q;
+                if (kb >= nk) break;
+                if (!sf_step(kb, fa[q], fb[q])) {
+                    if (lane == 0) s_fail = 1;
+                    stop = true;
+                    break;
+                }
+                if (kb + kPre < nk) load_sf(kb + kPre, fa[q], fb[q]);
+            }
+        }
+    }
+    __syncwarp();
+    const bool done = mbar_wait_sleep(&s_done, 0);
+    if (!done && lane == 0) raise_error(a.err, kDevTimeout);
+    const bool all_done = __syncthreads_and(done);  // also publishes s_fail
+    tc_fence_after();
+    pdl_launch_dependents();
+    if (s_fail != 0 && t == 0) raise_error(a.err, kDevTimeout);
+    if (s_fail == 0 && all_done && warp < 4) {
+        const int ch = n0 + warp * 32 + lane;  // this thread's TMEM lane = output channel
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        for (int c0 = 0; c0 < mma_n; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(lane_base + (uint32_t)c0, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int r = c0 + j;
+                if (r < nr && ch < a.out_dim)
+                    a.out[(size_t)(slot.y + r) * a.out_dim + ch] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGmTmemColsMx)
+                     : "memory");
 }
 
 }  // namespace moe

@@ -536,12 +536,12 @@ moe_status launch_gmm(const moe_gmm_params *p, const void *expand_x, const void 
     a.nslots = reinterpret_cast<int *>(ws + kWorkspaceBytes);
     a.slots = reinterpret_cast<int4 *>(ws + kWorkspaceBytes + 16);
     a.err = reinterpret_cast<uint32_t *>(workspace);
-    if (!ensure_smem(moe::gmm_kernel<MX>, moe::kGmSmemBytes)) return MOE_ERR_CUDA;
+    auto *kernel = MX ? moe::gmm_mx_kernel : moe::gmm_kernel;
+    if (!ensure_smem(kernel, moe::kGmSmemBytes)) return MOE_ERR_CUDA;
     if (launch(moe::gmm_plan_kernel, dim3(1), 1024, 0, s, a) != cudaSuccess) return MOE_ERR_CUDA;
     const dim3 grid((p->out_dim + moe::kGmBM - 1) / moe::kGmBM, a.max_slots);
-    return launch(moe::gmm_kernel<MX>, grid, moe::kGmThreads, moe::kGmSmemBytes, s, tm_w, tm_x, a) == cudaSuccess
-               ? MOE_OK
-               : MOE_ERR_CUDA;
+    const int threads = MX ? moe::kGmMxThreads : moe::kGmThreads;
+    return launch(kernel, grid, threads, moe::kGmSmemBytes, s, tm_w, tm_x, a) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace

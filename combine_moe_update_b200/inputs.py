@@ -238,6 +238,11 @@ WORKLOADS = {
     "deepseek_decode_bs512_expert": dict(builder=_expert_layer, seed=1, bs=512, hidden=7168, num_experts=256,
                                          top_k=8, ep_world_size=32, quant_mode=2, smooth=True, shared=True,
                                          expert_out_dim=7168),
+    # The Bs 512 layer dispatched as mxfp8 (quantMode 4, E8M0 block factors)
+    # with mxfp8 instance weights of 7168 x 7168 (13.2 GB + 0.4 GB of factors).
+    "deepseek_decode_bs512_expert_mx": dict(builder=_expert_layer, seed=1, bs=512, hidden=7168, num_experts=256,
+                                            top_k=8, ep_world_size=32, quant_mode=4, shared=True,
+                                            expert_out_dim=7168),
     # The same layer cut to 32 instances and Bs 128 (1.6 GB of weights), small
     # enough for a profiler capture of the matmul kernel.
     "expert_e32_bs128": dict(builder=_expert_layer, seed=1, bs=128, hidden=7168, num_experts=32, top_k=8,
@@ -402,3 +407,32 @@ def gmm_inputs_mx(seed, counts, hidden, out_dim, spare_rows=0, one_hot=False) ->
         x = _e4m3_codes(rng, (rows, hidden))
     w = _e4m3_codes(rng, (E, out_dim, hidden))
     return GmmMxInputs(expand_x=x, x_sf=xs, offsets=off, weight=w, weight_sf=wsf)
+
+
+def gmm_weights_device_mx(seed, num_instances, out_dim, hidden, device):
+    """mxfp8 instance weights drawn on ``device`` by torch's seeded generator:
+    codes uniform over the 254 finite E4M3 codes, block factors 2^(b - 127)
+    with b uniform in [117, 137].  Returns (weight [E, N, H] uint8,
+    weight_sf [E, N, H/32] uint8)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    w = torch.empty((num_instances, out_dim, hidden), dtype=torch.uint8, device=device)
+    for e in range(num_instances):
+        c = torch.randint(0, 254, (out_dim, hidden), generator=g, device=device, dtype=torch.int16)
+        w[e] = (c + (c >= 0x7F).to(torch.int16) + (c >= 0xFE).to(torch.int16)).to(torch.uint8)
+    sf = torch.randint(117, 138, (num_instances, out_dim, hidden // 32), generator=g, device=device,
+                       dtype=torch.int16).to(torch.uint8)
+    return w, sf
+
+
+def gmm_weights_host_mx(seed, instances, out_dim, hidden):
+    """Host-side mxfp8 weights for the given instances (the distribution of
+    gmm_weights_device_mx; the values differ): {e: (codes [N, H] uint8,
+    factors [N, H/32] uint8)}."""
+    out = {}
+    for e in instances:
+        rng = np.random.Generator(np.random.PCG64([seed, 9500 + int(e)]))
+        out[int(e)] = (_e4m3_codes(rng, (out_dim, hidden)),
+                       rng.integers(117, 137, (out_dim, hidden // 32), dtype=np.uint8, endpoint=True))
+    return out

@@ -470,8 +470,11 @@ uint32_t orc_grouped_matmul(int32_t rows, int32_t hidden, int32_t out_dim, int32
  * codes with one E8M0 factor 2^(b - 127) per 32-element block
  * (x_sf [rows, H/32], the dispatch's dynamicScales bytes), and so is the
  * weight (weight_sf [E, N, H/32]):
- *   out[r][n] = Sum_h dec(q[r][h]) 2^(x_sf[r][h/32] - 127) dec(w[e][n][h]) 2^(weight_sf[e][n][h/32] - 127)
- * summed in binary64 and rounded to bf16 once.  Offsets as above.
+ *   out[r][n] = Sum_j 2^(x_sf[r][j] - 127) 2^(weight_sf[e][n][j] - 127) Sum_{h in block j} dec(q[r][h]) dec(w[e][n][h])
+ * summed in binary64 and rounded to bf16 once.  Each block's sum is exact in
+ * binary64 (32 products of two E4M3 values: multiples of 2^-18 below 2^18)
+ * and the factors are powers of two, so only the sum over blocks rounds.
+ * Offsets as above.
  */
 uint32_t orc_grouped_matmul_mx(int32_t rows, int32_t hidden, int32_t out_dim, int32_t num_instances,
                                const uint8_t *expand_x, const uint8_t *x_sf,
@@ -481,16 +484,19 @@ uint32_t orc_grouped_matmul_mx(int32_t rows, int32_t hidden, int32_t out_dim, in
     if (expert_offsets[0] < 0 || expert_offsets[E] > rows) return ORC_ERR_BAD_ID;
     for (int e = 0; e < E; ++e)
         if (expert_offsets[e + 1] < expert_offsets[e]) return ORC_ERR_BAD_ID;
+    double dec[256];  /* the value of every code */
+    for (int c = 0; c < 256; ++c) dec[c] = orc_e4m3_decode((uint8_t)c);
     for (int e = 0; e < E; ++e) {
         for (int r = expert_offsets[e]; r < expert_offsets[e + 1]; ++r) {
+            const uint8_t *q = expand_x + (size_t)r * H;
             for (int n = 0; n < N; ++n) {
                 const size_t wr = (size_t)e * N + n;
+                const uint8_t *w = weight + wr * H;
                 double acc = 0.0;
-                for (int h = 0; h < H; ++h) {
-                    const double xv = ldexp(orc_e4m3_decode(expand_x[(size_t)r * H + h]),
-                                            (int)x_sf[(size_t)r * B + h / 32] - 127);
-                    const double wv = ldexp(orc_e4m3_decode(weight[wr * H + h]), (int)weight_sf[wr * B + h / 32] - 127);
-                    acc += xv * wv;
+                for (int j = 0; j < B; ++j) {
+                    double blk = 0.0;
+                    for (int h = 32 * j; h < 32 * j + 32; ++h) blk += dec[q[h]] * dec[w[h]];
+                    acc += ldexp(blk, (int)x_sf[(size_t)r * B + j] + (int)weight_sf[wr * B + j] - 254);
                 }
                 if (out_bf16) out_bf16[(size_t)r * N + n] = orc_bf16_from_double(acc);
                 if (out_f64) out_f64[(size_t)r * N + n] = acc;
