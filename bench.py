@@ -73,12 +73,21 @@ def algorithmic_bytes(w, n, x_out=False, rstd=False):
     return dict(update=upd, dispatch=disp, combine=comb)
 
 
-def source_hash():
-    """Hash of the CUDA sources, to tell whether stored ncu counters still
-    describe the kernels being timed."""
+# The sources a kernel is compiled from: stored ncu counters are kept while
+# these files are unchanged.
+KERNEL_SOURCES = {
+    "combine_token_kernel": ("combine.cuh", "common.cuh"),
+    "gmm_kernel": ("grouped_matmul.cuh", "common.cuh"),
+    "gmm_mx_kernel": ("grouped_matmul.cuh", "common.cuh"),
+}
+
+
+def source_hash(kernel):
+    """Hash of the CUDA sources of `kernel`, to tell whether stored ncu
+    counters still describe the kernel being timed."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_moe_update_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -86,13 +95,13 @@ def source_hash():
 
 def stored_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current sources; else None."""
+    the current sources of the kernel; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         rec = json.load(open(p))[f"{kernel}@{workload}"]
     except (OSError, KeyError, ValueError):
         return None
-    return rec.get("dram_bytes_per_launch") if rec.get("source_hash") == source_hash() else None
+    return rec.get("dram_bytes_per_launch") if rec.get("source_hash") == source_hash(kernel) else None
 
 
 def measured_peak():

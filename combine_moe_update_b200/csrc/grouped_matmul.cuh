@@ -43,7 +43,7 @@ constexpr int kGmBN = 128;          // rows per slot at most (the MMA's N: 16..1
 constexpr int kGmBK = 128;          // int8 contraction per stage: one 128-byte swizzled row
 constexpr int kGmBoxRows = 16;      // rows per TMA box of the row operand
 constexpr int kGmABytes = kGmBM * kGmBK;             // 16 KB of weight per stage
-constexpr int kGmPipeBytes = 96 * 1024;              // the stage ring
+constexpr int kGmPipeBytes = 110 * 1024;             // the stage ring (two CTAs per SM)
 constexpr int kGmMaxStages = 8;
 constexpr int kGmSmemBytes = kGmPipeBytes + 1024;    // + slack to align the ring to 1 KB
 constexpr int kGmThreads = 128;

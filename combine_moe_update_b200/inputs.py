@@ -247,6 +247,9 @@ WORKLOADS = {
     # enough for a profiler capture of the matmul kernel.
     "expert_e32_bs128": dict(builder=_expert_layer, seed=1, bs=128, hidden=7168, num_experts=32, top_k=8,
                              ep_world_size=8, quant_mode=2, smooth=True, shared=True, expert_out_dim=7168),
+    # ... and its mxfp8 form, for the profiler capture of the block-scaled kernel.
+    "expert_e32_bs128_mx": dict(builder=_expert_layer, seed=1, bs=128, hidden=7168, num_experts=32, top_k=8,
+                                ep_world_size=8, quant_mode=4, shared=True, expert_out_dim=7168),
     # Zipf(1.2) routing over 128 experts, 160 instances on 16 ranks, mxfp8.
     "skewed_eplb": dict(builder=_skewed_eplb, seed=2, bs=512),
     # Largest shapes: H 8192, 1024 experts, K 16, 256 ranks, per-128-tile int8,
