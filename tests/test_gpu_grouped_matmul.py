@@ -278,3 +278,25 @@ def test_dispatch_mx_gmm_combine_pipeline(B):
     np.testing.assert_array_equal(host(d["dyn_scales"].view(torch.uint8))[:n], do["dyn_scales"][:n])
     assert_close_bf16(host(ex)[:n], go["out_f64"][:n], what="mx gmm out")
     assert_close_bf16(host(c["y"]), co["y_f64"], what="y")
+
+
+def test_gmm_one_rank_region(B):
+    """One simulated rank runs its own L instances on its region of the
+    receive buffer: the offsets are that rank's slice of the dispatch's
+    offsets (the first one above 0), the weights its L instances'.  Rows of
+    the other ranks are left untouched."""
+    rng = np.random.default_rng(8)
+    counts = rng.poisson(20, 32)
+    gi = gen.gmm_inputs(26, counts, 1024, 256, spare_rows=3)
+    L, r = 8, 2  # 4 ranks of 8 instances; rank 2
+    sub = gen.GmmInputs(expand_x=gi.expand_x, dyn_scales=gi.dyn_scales,
+                        offsets=np.ascontiguousarray(gi.offsets[r * L:(r + 1) * L + 1]),
+                        weight=np.ascontiguousarray(gi.weight[r * L:(r + 1) * L]),
+                        weight_scales=np.ascontiguousarray(gi.weight_scales[r * L:(r + 1) * L]))
+    assert sub.offsets[0] > 0
+    got, err = _gpu(B, sub)
+    o = _oracle(sub)
+    assert err == 0 and o["err"] == 0
+    _assert_gmm_parity(got, o)
+    lo, hi = sub.offsets[0], sub.offsets[-1]
+    assert np.all(got[:lo] == POISON16) and np.all(got[hi:] == POISON16)
