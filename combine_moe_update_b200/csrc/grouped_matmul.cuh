@@ -14,8 +14,8 @@
 //
 // Design (sm_100a):
 //  * A planning kernel turns the per-instance offsets into work slots of at
-//    most 128 rows of one instance (one thread per instance, a block scan).
-//  * The matmul kernel computes one 128-channel x (<= 128 rows) tile per CTA
+//    most 256 rows of one instance (one thread per instance, a block scan).
+//  * The matmul kernel computes one 128-channel x (<= 256 rows) tile per CTA
 //    with tcgen05.mma kind::i8, "swapped": the weight slab [128 channels, H]
 //    is the MMA's A operand (M = 128) and the slot's rows are B (N = rows
 //    rounded up to 16).  A decode batch gives an instance ~16 rows, so N
@@ -25,7 +25,8 @@
 //    multicast) through a ring of stages sized at run time from N, tracked by
 //    mbarriers; one elected thread issues both the copies and the MMAs, and
 //    tcgen05.commit frees each stage.  The int32 accumulator lives in TMEM
-//    (128 lanes = channels, N columns = rows).
+//    (128 lanes = channels, N columns = rows; 256 columns allocated, two
+//    CTAs per SM).
 //  * The epilogue reads TMEM with tcgen05.ld (warp w owns lanes 32w..32w+31),
 //    applies the row and channel factors in fp32 and stores bf16.
 //  * Every wait is bounded; on a timeout the CTA records MOE_DEV_TIMEOUT,
@@ -39,7 +40,8 @@
 namespace moe {
 
 constexpr int kGmBM = 128;          // output channels per tile (the MMA's M)
-constexpr int kGmBN = 128;          // rows per slot at most (the MMA's N: 16..128)
+constexpr int kGmBN = 256;          // rows per slot at most, int8 (the MMA's N: 16..256)
+constexpr int kGmBNMx = 128;        // rows per slot at most, mxfp8 (TMEM also holds the factors)
 constexpr int kGmBK = 128;          // int8 contraction per stage: one 128-byte swizzled row
 constexpr int kGmBoxRows = 16;      // rows per TMA box of the row operand
 constexpr int kGmABytes = kGmBM * kGmBK;             // 16 KB of weight per stage
@@ -47,7 +49,7 @@ constexpr int kGmPipeBytes = 110 * 1024;             // the stage ring (two CTAs
 constexpr int kGmMaxStages = 8;
 constexpr int kGmSmemBytes = kGmPipeBytes + 1024;    // + slack to align the ring to 1 KB
 constexpr int kGmThreads = 128;
-constexpr uint32_t kGmTmemCols = 128;                // int32 accumulator columns (>= N)
+constexpr uint32_t kGmTmemCols = 256;                // int32 accumulator columns (>= N)
 // mxfp8: the fp32 accumulator (128 columns) then, per ring stage s, the
 // stage's block factors: 4 columns for the weight rows (A) at 128 + 8 s and
 // 4 for the token rows (B) at 128 + 8 s + 4.
@@ -55,6 +57,7 @@ constexpr uint32_t kGmTmemColsMx = 256;
 
 struct GmmArgs {
     int rows, hidden, out_dim, num_instances, max_slots;
+    int slot_rows;             // rows per slot at most: kGmBN (int8) or kGmBNMx (mxfp8)
     const float *dyn;          // [rows] per-row factor
     const int32_t *offsets;    // [E + 1]
     const float *wscale;       // [E, N] per-channel factor
@@ -66,9 +69,9 @@ struct GmmArgs {
     uint32_t *err;
 };
 
-__host__ __device__ inline int gmm_max_slots(int rows, int num_instances) {
-    // sum_e ceil(c_e / 128) <= sum_e (c_e + 127) / 128 < rows / 128 + E
-    return num_instances + (rows + kGmBN - 1) / kGmBN;
+__host__ __device__ inline int gmm_max_slots(int rows, int num_instances, int slot_rows) {
+    // sum_e ceil(c_e / R) <= sum_e (c_e + R - 1) / R < rows / R + E
+    return num_instances + (rows + slot_rows - 1) / slot_rows;
 }
 
 // --- planning: one block of 1024 threads, thread e = instance e ---
@@ -89,10 +92,11 @@ __global__ void __launch_bounds__(1024) gmm_plan_kernel(GmmArgs a) {
     __syncthreads();
     const bool bad = s_bad != 0;
     if (bad) cnt = 0;  // offsets that are not a non-decreasing run in [0, rows]: nothing is computed
-    const int ch = (cnt + kGmBN - 1) / kGmBN;
+    const int R = a.slot_rows;
+    const int ch = (cnt + R - 1) / R;
     const int incl = block_inclusive_scan(ch, s_warp);
     for (int c = 0, s = incl - ch; c < ch && s < a.max_slots; ++c, ++s)
-        a.slots[s] = make_int4(e, lo + c * kGmBN, min(kGmBN, cnt - c * kGmBN), 0);
+        a.slots[s] = make_int4(e, lo + c * R, min(R, cnt - c * R), 0);
     if (e == (int)blockDim.x - 1) *a.nslots = min(incl, a.max_slots);
     if (bad && e == 0) raise_error(a.err, kDevBadId);
     pdl_launch_dependents();

@@ -119,7 +119,7 @@ bool valid_combine(const moe_combine_params &p) {
 
 bool valid_gmm(const moe_gmm_params &p) {
     if (p.rows < 1 || p.num_instances < 1 || p.num_instances > MOE_MAX_EXPERTS) return false;
-    if (moe::gmm_max_slots(p.rows, p.num_instances) > 65535) return false;  // slots index grid.y
+    if (moe::gmm_max_slots(p.rows, p.num_instances, moe::kGmBNMx) > 65535) return false;  // slots index grid.y
     if (p.hidden < MOE_MIN_HIDDEN || p.hidden > MOE_MAX_HIDDEN || p.hidden % 16 != 0) return false;
     if (p.out_dim < 16 || p.out_dim > MOE_GMM_MAX_OUT_DIM || p.out_dim % 16 != 0) return false;
     return true;
@@ -128,7 +128,7 @@ bool valid_gmm(const moe_gmm_params &p) {
 // Grouped-matmul workspace: the error-word area, the slot count (padded to
 // 16 bytes), then the slots.
 size_t gmm_workspace_bytes(const moe_gmm_params &p) {
-    return kWorkspaceBytes + 16 + 16 * (size_t)moe::gmm_max_slots(p.rows, p.num_instances);
+    return kWorkspaceBytes + 16 + 16 * (size_t)moe::gmm_max_slots(p.rows, p.num_instances, moe::kGmBNMx);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
@@ -532,7 +532,8 @@ moe_status launch_gmm(const moe_gmm_params *p, const void *expand_x, const void 
     a.hidden = p->hidden;
     a.out_dim = p->out_dim;
     a.num_instances = p->num_instances;
-    a.max_slots = moe::gmm_max_slots(p->rows, p->num_instances);
+    a.slot_rows = MX ? moe::kGmBNMx : moe::kGmBN;
+    a.max_slots = moe::gmm_max_slots(p->rows, p->num_instances, a.slot_rows);
     a.nslots = reinterpret_cast<int *>(ws + kWorkspaceBytes);
     a.slots = reinterpret_cast<int4 *>(ws + kWorkspaceBytes + 16);
     a.err = reinterpret_cast<uint32_t *>(workspace);

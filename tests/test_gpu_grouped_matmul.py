@@ -64,7 +64,8 @@ def _assert_gmm_parity(got, o):
 
 
 @pytest.mark.parametrize("H,N,counts,spare", [
-    (1024, 256, [3, 0, 17, 130, 1, 128, 16], 5),  # padded N, two slots of one instance, empty instance
+    (1024, 256, [3, 0, 17, 130, 1, 128, 16], 5),  # padded N, empty instance
+    (1024, 128, [300, 256, 2, 513], 1),           # 256-row slots and remainders
     (1168, 208, [5, 33, 0, 260], 0),              # ragged K tail and a partial channel slab
 ])
 def test_gmm_single_products_bit_exact(B, H, N, counts, spare):
@@ -81,7 +82,8 @@ def test_gmm_single_products_bit_exact(B, H, N, counts, spare):
 @pytest.mark.parametrize("H,N,counts,spare", [
     (1024, 128, [40, 0, 1, 129, 77], 3),
     (1168, 208, [5, 33, 0, 260], 2),
-    (2048, 256, [128, 256, 255, 16, 15], 0),      # slot boundaries at 128 rows
+    (2048, 256, [128, 256, 255, 16, 15], 0),      # slot boundaries at 128 and 256 rows
+    (1024, 128, [511, 512, 513, 257, 1], 2),      # 256-row slots (N = 256) and their remainders
     (7168, 384, [24, 9, 0, 140], 1),              # the decode hidden size
 ])
 def test_gmm_parity_random(B, H, N, counts, spare):
