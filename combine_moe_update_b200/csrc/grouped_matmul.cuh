@@ -21,8 +21,8 @@
 //    rounded up to 16).  A decode batch gives an instance ~16 rows, so N
 //    follows the rows and no tensor work is spent on padding to 128 rows;
 //    every weight byte is read from HBM once per slot.
-//  * Operands are staged by TMA (cp.async.bulk.tensor, 128-byte swizzle, no
-//    multicast) through a ring of stages sized at run time from N, tracked by
+//  * Operands are staged by TMA (cp.async.bulk.tensor, 128-byte swizzle, each
+//    CTA loading its own tiles) through a ring of stages sized at run time from N, tracked by
 //    mbarriers; one elected thread issues both the copies and the MMAs, and
 //    tcgen05.commit frees each stage.  The int32 accumulator lives in TMEM
 //    (128 lanes = channels, N columns = rows; 256 columns allocated, two
@@ -173,7 +173,7 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                  : "memory");
 }
 
-// 2-D tiled TMA load (no multicast); x is the innermost coordinate in
+// 2-D tiled TMA load into this CTA's shared memory; x is the innermost coordinate in
 // elements (here bytes), always a multiple of 128.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
     asm volatile(
