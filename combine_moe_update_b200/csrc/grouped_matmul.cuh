@@ -22,8 +22,9 @@
 //    follows the rows and no tensor work is spent on padding to 128 rows;
 //    every weight byte is read from HBM once per slot.
 //  * Operands are staged by TMA (cp.async.bulk.tensor, 128-byte swizzle, each
-//    CTA loading its own tiles) through a ring of stages sized at run time from N, tracked by
-//    mbarriers; one elected thread issues both the copies and the MMAs, and
+//    CTA loading its own tiles) through a ring of stages sized at run time
+//    from N, tracked by mbarriers; one elected thread issues both the copies
+//    and the MMAs, and
 //    tcgen05.commit frees each stage.  The int32 accumulator lives in TMEM
 //    (128 lanes = channels, N columns = rows; 256 columns allocated, two
 //    CTAs per SM).
@@ -32,6 +33,13 @@
 //  * Every wait is bounded; on a timeout the CTA records MOE_DEV_TIMEOUT,
 //    drains its copies in flight (again bounded), frees its TMEM and skips
 //    its stores.
+//
+// On mxfp8 rows (the dispatch's quantMode 4: E4M3 codes with one E8M0 factor
+// per 32 elements) the weights are mxfp8 as well, and gmm_mx_kernel runs the
+// block-scaled MMA (kind::mxf8f6f4.block_scale, fp32 accumulator) with the
+// factors placed in TMEM stage by stage:
+//   out[r][n] = sum over 32-element blocks j of
+//               2^(sx[r][j] - 127) * 2^(sw[e][n][j] - 127) * sum_{h in j} dec(q[r][h]) * dec(w[e][n][h]).
 #pragma once
 #include <cuda.h>
 
