@@ -156,12 +156,14 @@ def dispatch_workspace_bytes(bs, hidden, top_k, ep_world_size, num_instances, qu
 
 
 def read_device_error(workspace: torch.Tensor, stream=None) -> int:
+    _req(workspace, "workspace", torch.uint8)
     bits = ctypes.c_uint32(0)
     _check("moe_read_device_error", lib.moe_read_device_error(_ptr(workspace), ctypes.byref(bits), _stream(stream)))
     return int(bits.value)
 
 
 def clear_device_error(workspace: torch.Tensor, stream=None) -> None:
+    _req(workspace, "workspace", torch.uint8)
     _check("moe_clear_device_error", lib.moe_clear_device_error(_ptr(workspace), _stream(stream)))
 
 
@@ -186,7 +188,7 @@ def update_expert(expert_ids, table, ep_world_size, expert_scales=None, active_m
     bal, bm = out
     _req(bal, "balanced_ids", torch.int32, (bs, k))
     _req(bm, "balanced_mask", torch.uint8, (bs, k))
-    ws = workspace if workspace is not None else new_workspace(expert_ids.device, stream)
+    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(expert_ids.device, stream)
     _check("moe_update_expert", lib.moe_update_expert(
         ctypes.byref(p), _ptr(expert_ids), _ptr(expert_scales), _ptr(active_mask), _ptr(table),
         _ptr(bal), _ptr(bm), _ptr(ws), ws.numel(), _stream(stream)))
@@ -242,7 +244,7 @@ def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=Non
     sl = 0 if smooth is None else smooth.numel()
     p = DispatchParams(_per_source(bs, sources, "dispatch"), H, k, int(ep_world_size), int(num_instances),
                        int(quant_mode), sl, int(sources))
-    ws = workspace if workspace is not None else new_workspace(
+    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
         x.device, stream, dispatch_workspace_bytes(p.bs, H, k, ep_world_size, num_instances, quant_mode, sl, sources))
     _check("moe_dispatch", lib.moe_dispatch(
         ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
@@ -269,7 +271,7 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
                    x_out=torch.empty((bs, H), dtype=torch.bfloat16, device=dev) if want_x_out else None,
                    rstd=torch.empty((bs,), dtype=torch.float32, device=dev) if want_rstd else None)
     p = CombineParams(_per_source(bs, sources, "combine_add_rmsnorm"), H, k, rows, float(norm_eps), int(sources))
-    ws = workspace if workspace is not None else new_workspace(expand_x.device, stream)
+    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(expand_x.device, stream)
     _check("moe_combine_add_rmsnorm", lib.moe_combine_add_rmsnorm(
         ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x),
         _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")), _ptr(out.get("rstd")),
@@ -289,7 +291,7 @@ def combine(expand_x, expand_idx, expert_scales, shared_x=None, workspace=None, 
         out = torch.empty((bs, H), dtype=torch.bfloat16, device=expand_x.device)
     _req(out, "out", torch.bfloat16, (bs, H))
     p = CombineParams(_per_source(bs, sources, "combine"), H, k, rows, 0.0, int(sources))
-    ws = workspace if workspace is not None else new_workspace(expand_x.device, stream)
+    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(expand_x.device, stream)
     _check("moe_combine", lib.moe_combine(
         ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x), _ptr(out),
         _ptr(ws), ws.numel(), _stream(stream)))
@@ -346,7 +348,7 @@ def grouped_matmul(expand_x, dyn_scales, expert_offsets, weight, weight_scales, 
         out = torch.empty((rows, N), dtype=torch.bfloat16, device=expand_x.device)
     _req(out, "out", torch.bfloat16, (rows, N))
     p = GmmParams(rows, H, N, E)
-    ws = workspace if workspace is not None else new_workspace(
+    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
         expand_x.device, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
     _check("moe_grouped_matmul", lib.moe_grouped_matmul(
         ctypes.byref(p), _ptr(expand_x), _ptr(dyn_scales), _ptr(expert_offsets), _ptr(weight),
@@ -370,7 +372,7 @@ def grouped_matmul_mx(expand_x, x_sf, expert_offsets, weight, weight_sf, out=Non
         out = torch.empty((rows, N), dtype=torch.bfloat16, device=expand_x.device)
     _req(out, "out", torch.bfloat16, (rows, N))
     p = GmmParams(rows, H, N, E)
-    ws = workspace if workspace is not None else new_workspace(
+    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
         expand_x.device, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
     _check("moe_grouped_matmul_mx", lib.moe_grouped_matmul_mx(
         ctypes.byref(p), _ptr(expand_x), _ptr(x_sf), _ptr(expert_offsets), _ptr(weight), _ptr(weight_sf),

@@ -235,3 +235,16 @@ def test_grouped_matmul_mx_rules(L):
                dict(off=f2)):
         assert call(**kw) == L.MOE_ERR_INVALID_ARG, kw
     assert call(wsb=n - 16) == L.MOE_ERR_WORKSPACE
+
+
+def test_binding_refuses_host_workspaces(L):
+    """A workspace is device memory the kernels write: the binding refuses a
+    host tensor (or one of another dtype) before any call is made."""
+    host_ws = torch.zeros(256, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.read_device_error(host_ws)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.clear_device_error(host_ws)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.grouped_matmul(torch.zeros((4, 1024), dtype=torch.int8), torch.ones(4), torch.zeros(2, dtype=torch.int32),
+                         torch.zeros((1, 16, 1024), dtype=torch.int8), torch.ones((1, 16)), workspace=host_ws)
