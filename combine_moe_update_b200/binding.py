@@ -126,6 +126,45 @@ def _opt(t, name, dtype, shape=None):
     return None if t is None else _req(t, name, dtype, shape)
 
 
+def _same_device(dev, *named):
+    """Every tensor of a call lives on the device of its first input: the
+    library launches on that device's current stream and looks per-device
+    state up with that device current."""
+    for name, t in named:
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the call's inputs on {dev}")
+
+
+def _check_dispatch_out(out, bs, hidden, top_k, num_instances, quant_mode):
+    """A caller-supplied output dict must hold exactly what
+    alloc_dispatch_outputs would allocate: the kernels write up to bs*K rows
+    of expand_x and every entry through raw device pointers."""
+    if not isinstance(out, dict):
+        raise TypeError("out must be a dict like alloc_dispatch_outputs returns")
+    rows = bs * top_k
+    _req(out.get("expand_x"), "out['expand_x']", expand_dtype(quant_mode), (rows, hidden))
+    ss = scales_shape(quant_mode, rows, hidden)
+    if ss is None:
+        if out.get("dyn_scales") is not None:
+            raise ValueError(f"quant_mode {quant_mode} sends no scales: out['dyn_scales'] must be None")
+    else:
+        _req(out.get("dyn_scales"), "out['dyn_scales']", ss[1], ss[0])
+    _req(out.get("expand_idx"), "out['expand_idx']", torch.int32, (bs, top_k))
+    _req(out.get("src_of_row"), "out['src_of_row']", torch.int32, (rows,))
+    _req(out.get("counts"), "out['counts']", torch.int32, (num_instances,))
+    _req(out.get("offsets"), "out['offsets']", torch.int32, (num_instances + 1,))
+    return out
+
+
+def _check_combine_out(out, bs, hidden):
+    if not isinstance(out, dict):
+        raise TypeError("out must be a dict with y (and optionally x_out, rstd)")
+    _req(out.get("y"), "out['y']", torch.bfloat16, (bs, hidden))
+    _opt(out.get("x_out"), "out['x_out']", torch.bfloat16, (bs, hidden))
+    _opt(out.get("rstd"), "out['rstd']", torch.float32, (bs,))
+    return out
+
+
 # --------------------------------------------------------------------------
 # workspace / device errors
 # --------------------------------------------------------------------------
@@ -135,7 +174,8 @@ def new_workspace(device=None, stream=None, nbytes=WORKSPACE_BYTES) -> torch.Ten
     several source ranks may need more than the default, see
     dispatch_workspace_bytes)."""
     ws = torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
-    _check("moe_workspace_init", lib.moe_workspace_init(_ptr(ws), nbytes, _stream(stream)))
+    with torch.cuda.device(ws.device):
+        _check("moe_workspace_init", lib.moe_workspace_init(_ptr(ws), nbytes, _stream(stream)))
     return ws
 
 
@@ -158,13 +198,16 @@ def dispatch_workspace_bytes(bs, hidden, top_k, ep_world_size, num_instances, qu
 def read_device_error(workspace: torch.Tensor, stream=None) -> int:
     _req(workspace, "workspace", torch.uint8)
     bits = ctypes.c_uint32(0)
-    _check("moe_read_device_error", lib.moe_read_device_error(_ptr(workspace), ctypes.byref(bits), _stream(stream)))
+    with torch.cuda.device(workspace.device):
+        _check("moe_read_device_error",
+               lib.moe_read_device_error(_ptr(workspace), ctypes.byref(bits), _stream(stream)))
     return int(bits.value)
 
 
 def clear_device_error(workspace: torch.Tensor, stream=None) -> None:
     _req(workspace, "workspace", torch.uint8)
-    _check("moe_clear_device_error", lib.moe_clear_device_error(_ptr(workspace), _stream(stream)))
+    with torch.cuda.device(workspace.device):
+        _check("moe_clear_device_error", lib.moe_clear_device_error(_ptr(workspace), _stream(stream)))
 
 
 # --------------------------------------------------------------------------
@@ -177,21 +220,25 @@ def update_expert(expert_ids, table, ep_world_size, expert_scales=None, active_m
     With sources = S the arrays hold S source ranks' tokens, rank-major."""
     _req(expert_ids, "expert_ids", torch.int32)
     bs, k = expert_ids.shape
+    dev = expert_ids.device
     _req(table, "table", torch.int32)
     _opt(expert_scales, "expert_scales", torch.float32, (bs, k))
     _opt(active_mask, "active_mask", torch.uint8, (bs,))
     p = UpdateParams(_per_source(bs, sources, "update_expert"), k, table.shape[0], table.shape[1],
                      int(ep_world_size), float(prune_threshold), int(sources))
     if out is None:
-        out = (torch.empty((bs, k), dtype=torch.int32, device=expert_ids.device),
-               torch.empty((bs, k), dtype=torch.uint8, device=expert_ids.device))
+        out = (torch.empty((bs, k), dtype=torch.int32, device=dev),
+               torch.empty((bs, k), dtype=torch.uint8, device=dev))
     bal, bm = out
     _req(bal, "balanced_ids", torch.int32, (bs, k))
     _req(bm, "balanced_mask", torch.uint8, (bs, k))
-    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(expert_ids.device, stream)
-    _check("moe_update_expert", lib.moe_update_expert(
-        ctypes.byref(p), _ptr(expert_ids), _ptr(expert_scales), _ptr(active_mask), _ptr(table),
-        _ptr(bal), _ptr(bm), _ptr(ws), ws.numel(), _stream(stream)))
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(dev, stream)
+        _same_device(dev, ("table", table), ("expert_scales", expert_scales), ("active_mask", active_mask),
+                     ("balanced_ids", bal), ("balanced_mask", bm), ("workspace", ws))
+        _check("moe_update_expert", lib.moe_update_expert(
+            ctypes.byref(p), _ptr(expert_ids), _ptr(expert_scales), _ptr(active_mask), _ptr(table),
+            _ptr(bal), _ptr(bm), _ptr(ws), ws.numel(), _stream(stream)))
     return bal, bm
 
 
@@ -234,22 +281,28 @@ def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=Non
     src_of_row, counts and offsets (see include/moe_b200.h for layouts)."""
     _req(x, "x", torch.bfloat16)
     bs, H = x.shape
+    dev = x.device
     _req(instance_ids, "instance_ids", torch.int32)
     k = instance_ids.shape[1]
     _req(instance_ids, "instance_ids", torch.int32, (bs, k))
     _opt(mask, "mask", torch.uint8, (bs, k))
     _check_scales(smooth, quant_mode, num_instances, H)
     if out is None:
-        out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
+        out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, dev)
+    _check_dispatch_out(out, bs, H, k, num_instances, quant_mode)
     sl = 0 if smooth is None else smooth.numel()
     p = DispatchParams(_per_source(bs, sources, "dispatch"), H, k, int(ep_world_size), int(num_instances),
                        int(quant_mode), sl, int(sources))
-    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
-        x.device, stream, dispatch_workspace_bytes(p.bs, H, k, ep_world_size, num_instances, quant_mode, sl, sources))
-    _check("moe_dispatch", lib.moe_dispatch(
-        ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
-        _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
-        _ptr(out["offsets"]), _ptr(ws), ws.numel(), _stream(stream)))
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
+            dev, stream, dispatch_workspace_bytes(p.bs, H, k, ep_world_size, num_instances, quant_mode, sl,
+                                                  sources))
+        _same_device(dev, ("instance_ids", instance_ids), ("mask", mask), ("smooth", smooth), ("workspace", ws),
+                     *((f"out['{n}']", t) for n, t in out.items()))
+        _check("moe_dispatch", lib.moe_dispatch(
+            ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
+            _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
+            _ptr(out["offsets"]), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
@@ -259,6 +312,7 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
     """moe_combine_add_rmsnorm.  Returns a dict with y (and x_out / rstd when asked)."""
     _req(expand_x, "expand_x", torch.bfloat16)
     rows, H = expand_x.shape
+    dev = expand_x.device
     _req(expand_idx, "expand_idx", torch.int32)
     bs, k = expand_idx.shape
     _req(expert_scales, "expert_scales", torch.float32, (bs, k))
@@ -266,16 +320,20 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
     _req(gamma, "gamma", torch.bfloat16, (H,))
     _opt(shared_x, "shared_x", torch.bfloat16, (bs, H))
     if out is None:
-        dev = expand_x.device
         out = dict(y=torch.empty((bs, H), dtype=torch.bfloat16, device=dev),
                    x_out=torch.empty((bs, H), dtype=torch.bfloat16, device=dev) if want_x_out else None,
                    rstd=torch.empty((bs,), dtype=torch.float32, device=dev) if want_rstd else None)
+    _check_combine_out(out, bs, H)
     p = CombineParams(_per_source(bs, sources, "combine_add_rmsnorm"), H, k, rows, float(norm_eps), int(sources))
-    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(expand_x.device, stream)
-    _check("moe_combine_add_rmsnorm", lib.moe_combine_add_rmsnorm(
-        ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x),
-        _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")), _ptr(out.get("rstd")),
-        _ptr(ws), ws.numel(), _stream(stream)))
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(dev, stream)
+        _same_device(dev, ("expand_idx", expand_idx), ("expert_scales", expert_scales), ("residual_x", residual_x),
+                     ("gamma", gamma), ("shared_x", shared_x), ("workspace", ws),
+                     *((f"out['{n}']", t) for n, t in out.items()))
+        _check("moe_combine_add_rmsnorm", lib.moe_combine_add_rmsnorm(
+            ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x),
+            _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")), _ptr(out.get("rstd")),
+            _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
@@ -283,18 +341,22 @@ def combine(expand_x, expand_idx, expert_scales, shared_x=None, workspace=None, 
     """moe_combine (the plain CombineV2-series combine): combineOut [bs, H] bf16."""
     _req(expand_x, "expand_x", torch.bfloat16)
     rows, H = expand_x.shape
+    dev = expand_x.device
     _req(expand_idx, "expand_idx", torch.int32)
     bs, k = expand_idx.shape
     _req(expert_scales, "expert_scales", torch.float32, (bs, k))
     _opt(shared_x, "shared_x", torch.bfloat16, (bs, H))
     if out is None:
-        out = torch.empty((bs, H), dtype=torch.bfloat16, device=expand_x.device)
+        out = torch.empty((bs, H), dtype=torch.bfloat16, device=dev)
     _req(out, "out", torch.bfloat16, (bs, H))
     p = CombineParams(_per_source(bs, sources, "combine"), H, k, rows, 0.0, int(sources))
-    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(expand_x.device, stream)
-    _check("moe_combine", lib.moe_combine(
-        ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x), _ptr(out),
-        _ptr(ws), ws.numel(), _stream(stream)))
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(dev, stream)
+        _same_device(dev, ("expand_idx", expand_idx), ("expert_scales", expert_scales), ("shared_x", shared_x),
+                     ("out", out), ("workspace", ws))
+        _check("moe_combine", lib.moe_combine(
+            ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x), _ptr(out),
+            _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
@@ -305,6 +367,7 @@ def dispatch_noalloc(x, instance_ids, num_instances, ep_world_size, quant_mode, 
     element that receives the call's device error word."""
     _req(x, "x", torch.bfloat16)
     bs, H = x.shape
+    dev = x.device
     _req(instance_ids, "instance_ids", torch.int32)
     k = instance_ids.shape[1]
     _req(instance_ids, "instance_ids", torch.int32, (bs, k))
@@ -312,15 +375,18 @@ def dispatch_noalloc(x, instance_ids, num_instances, ep_world_size, quant_mode, 
     _check_scales(smooth, quant_mode, num_instances, H)
     _opt(device_error, "device_error", torch.int32, (1,))
     if out is None:
-        out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, x.device)
+        out = alloc_dispatch_outputs(bs, H, k, num_instances, quant_mode, dev)
+    _check_dispatch_out(out, bs, H, k, num_instances, quant_mode)
+    _same_device(dev, ("instance_ids", instance_ids), ("mask", mask), ("smooth", smooth),
+                 ("device_error", device_error), *((f"out['{n}']", t) for n, t in out.items()))
     p = DispatchParams(_per_source(bs, sources, "dispatch_noalloc"), H, k, int(ep_world_size),
                        int(num_instances), int(quant_mode), 0 if smooth is None else smooth.numel(), int(sources))
-    _check("moe_dispatch_noalloc", lib.moe_dispatch_noalloc(
-        ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
-        _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
-        _ptr(out["offsets"]), _ptr(device_error), _stream(stream)))
+    with torch.cuda.device(dev):  # the library picks the scratch array of the current device
+        _check("moe_dispatch_noalloc", lib.moe_dispatch_noalloc(
+            ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
+            _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
+            _ptr(out["offsets"]), _ptr(device_error), _stream(stream)))
     return out
-
 
 
 def grouped_matmul_workspace_bytes(rows, hidden, out_dim, num_instances) -> int:
@@ -348,11 +414,15 @@ def grouped_matmul(expand_x, dyn_scales, expert_offsets, weight, weight_scales, 
         out = torch.empty((rows, N), dtype=torch.bfloat16, device=expand_x.device)
     _req(out, "out", torch.bfloat16, (rows, N))
     p = GmmParams(rows, H, N, E)
-    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
-        expand_x.device, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
-    _check("moe_grouped_matmul", lib.moe_grouped_matmul(
-        ctypes.byref(p), _ptr(expand_x), _ptr(dyn_scales), _ptr(expert_offsets), _ptr(weight),
-        _ptr(weight_scales), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    dev = expand_x.device
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
+            dev, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
+        _same_device(dev, ("dyn_scales", dyn_scales), ("expert_offsets", expert_offsets), ("weight", weight),
+                     ("weight_scales", weight_scales), ("out", out), ("workspace", ws))
+        _check("moe_grouped_matmul", lib.moe_grouped_matmul(
+            ctypes.byref(p), _ptr(expand_x), _ptr(dyn_scales), _ptr(expert_offsets), _ptr(weight),
+            _ptr(weight_scales), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
@@ -372,9 +442,13 @@ def grouped_matmul_mx(expand_x, x_sf, expert_offsets, weight, weight_sf, out=Non
         out = torch.empty((rows, N), dtype=torch.bfloat16, device=expand_x.device)
     _req(out, "out", torch.bfloat16, (rows, N))
     p = GmmParams(rows, H, N, E)
-    ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
-        expand_x.device, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
-    _check("moe_grouped_matmul_mx", lib.moe_grouped_matmul_mx(
-        ctypes.byref(p), _ptr(expand_x), _ptr(x_sf), _ptr(expert_offsets), _ptr(weight), _ptr(weight_sf),
-        _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    dev = expand_x.device
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
+            dev, stream, grouped_matmul_workspace_bytes(rows, H, N, E))
+        _same_device(dev, ("x_sf", x_sf), ("expert_offsets", expert_offsets), ("weight", weight),
+                     ("weight_sf", weight_sf), ("out", out), ("workspace", ws))
+        _check("moe_grouped_matmul_mx", lib.moe_grouped_matmul_mx(
+            ctypes.byref(p), _ptr(expand_x), _ptr(x_sf), _ptr(expert_offsets), _ptr(weight), _ptr(weight_sf),
+            _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out

@@ -12,7 +12,10 @@
 // kernel: everything that depends only on the call's inputs (loading the
 // token row and the smooth row, the absmax reduction, the quantization
 // itself) runs while the route kernel is still sorting, and only the final
-// row writes wait for it.
+// row writes wait for it.  That is safe because the route kernel releases
+// them only after its own wait, when everything before the call is complete.
+// A scatter kernel that routes its own copies (FUSED, small calls) is the
+// call's first kernel and reads nothing before its wait.
 //
 // dispatch_token_kernel<MODE>   no smooth scales: one block per token; the
 //   row is loaded, quantized once (all K copies are identical) and written K
@@ -722,55 +725,67 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
     __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
     const int i = blockIdx.x, t = threadIdx.x;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
-    if constexpr (FUSED) block_route_clear<NT>(rs, a.num_instances);
+    if constexpr (FUSED) {
+        // This kernel is the call's first: x itself may come from the kernel
+        // before it (a combine whose y feeds the next layer), so nothing is
+        // read before the wait.  The x loads issued right after it stay in
+        // flight while the block routes its copies.
+        block_route_clear<NT>(rs, a.num_instances);
+        pdl_wait();
+    }
 
-    // inputs of the call only: safe before the route kernel is done
+    // FUSED: after the wait.  Otherwise this kernel follows the call's route
+    // kernel, which releases it only after its own wait, so every input of
+    // the call is final and may be read before this kernel's wait.
     uint4 xv[kDpVecs];
     load_row<NT>(a.x + (size_t)i * H, V, xv);
     uint2 qv[kDpVecs];
     float seg[kDpVecs] = {0.0f, 0.0f, 0.0f, 0.0f};
     float row_scale = 0.0f;
-    if constexpr (MODE != 0) {
-        uint64_t xf[kDpVecs][4];
+    auto quantize = [&]() {
+        if constexpr (MODE != 0) {
+            uint64_t xf[kDpVecs][4];
 #pragma unroll
-        for (int q = 0; q < kDpVecs; ++q) vec_to_f2(xv[q], xf[q]);
-        if constexpr (MODE == 1) {  // xFp32 = x * scales: one coefficient, or one per column
-            if (a.scales_len == 1) {
-                const float c = __ldg(a.smooth);
-                const uint64_t c2 = f2_pack(c, c);
+            for (int q = 0; q < kDpVecs; ++q) vec_to_f2(xv[q], xf[q]);
+            if constexpr (MODE == 1) {  // xFp32 = x * scales: one coefficient, or one per column
+                if (a.scales_len == 1) {
+                    const float c = __ldg(a.smooth);
+                    const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
-                for (int q = 0; q < kDpVecs; ++q)
+                    for (int q = 0; q < kDpVecs; ++q)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) xf[q][j] = f2_mul(xf[q][j], c2);
-            } else {
+                        for (int j = 0; j < 4; ++j) xf[q][j] = f2_mul(xf[q][j], c2);
+                } else {
 #pragma unroll
-                for (int q = 0; q < kDpVecs; ++q) {
-                    const int p = t + q * NT;
-                    if (p >= V) continue;
-                    const float4 s0 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8));
-                    const float4 s1 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8) + 1);
-                    xf[q][0] = f2_mul(xf[q][0], f2_pack(s0.x, s0.y));
-                    xf[q][1] = f2_mul(xf[q][1], f2_pack(s0.z, s0.w));
-                    xf[q][2] = f2_mul(xf[q][2], f2_pack(s1.x, s1.y));
-                    xf[q][3] = f2_mul(xf[q][3], f2_pack(s1.z, s1.w));
+                    for (int q = 0; q < kDpVecs; ++q) {
+                        const int p = t + q * NT;
+                        if (p >= V) continue;
+                        const float4 s0 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8));
+                        const float4 s1 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8) + 1);
+                        xf[q][0] = f2_mul(xf[q][0], f2_pack(s0.x, s0.y));
+                        xf[q][1] = f2_mul(xf[q][1], f2_pack(s0.z, s0.w));
+                        xf[q][2] = f2_mul(xf[q][2], f2_pack(s1.x, s1.y));
+                        xf[q][3] = f2_mul(xf[q][3], f2_pack(s1.z, s1.w));
+                    }
                 }
             }
+            if constexpr (MODE == 2) {
+                const float dyn = block_dyn<NT>(abs_max_vecs(xf), s_red);
+                row_scale = __frcp_rn(dyn);  // 1 / dynamicScales
+                int8_vecs(xf, dyn, qv);
+            } else {
+                quantize_local<MODE, NT>(xf, V, qv, seg);
+            }
         }
-        if constexpr (MODE == 2) {
-            const float dyn = block_dyn<NT>(abs_max_vecs(xf), s_red);
-            row_scale = __frcp_rn(dyn);  // 1 / dynamicScales
-            int8_vecs(xf, dyn, qv);
-        } else {
-            quantize_local<MODE, NT>(xf, V, qv, seg);
-        }
-    }
+    };
 
     if constexpr (FUSED) {
         __syncthreads();  // the counters are clear
-        pdl_wait();       // the instance ids may come from the previous kernel
         block_route<NT>(a, i, rs, t < 32 && t < K ? copy_key(a, i * K + t) : -1);
         pdl_launch_dependents();
+        quantize();  // x arrived while the block routed
     } else {
+        quantize();  // while the route kernel is still sorting
         pdl_wait();  // the rows come from route_kernel
         if (t < K) s_row[t] = a.expand_idx[i * K + t];
         __syncthreads();
@@ -832,20 +847,24 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
     // swapped (x here, the smooth halves at the reads, the codes back at the
     // writes), so each quarter-warp's reads cover all 32 banks once.
     const bool swap = (lane >> 2) & 1;
-    // inputs of the call only: safe before the route kernel is done
+    for (int e = H + t; e < smooth_smem_floats<NT>(H); e += NT) s_smooth[e] = 0.0f;
+    if constexpr (FUSED) {
+        // The call's first kernel: x, the ids and the scales may all come
+        // from the kernel before it, so nothing is read before the wait.
+        block_route_clear<NT>(rs, a.num_instances);
+        if (t == 0) mbar_init(&s_bar, 1);
+        __syncthreads();
+        pdl_wait();
+    }
+    // FUSED: after the wait.  Otherwise the call's route kernel runs first
+    // and releases this kernel only after its own wait, so the call's inputs
+    // are final and may be read before this kernel's wait.
     uint4 xv[kDpVecs];
     load_row<NT>(a.x + (size_t)i * H, V, xv);
 #pragma unroll
     for (int q = 0; q < kDpVecs; ++q)
         if (swap) xv[q] = make_uint4(xv[q].z, xv[q].w, xv[q].x, xv[q].y);
     const float *s_first = s_smooth + (swap ? 4 : 0), *s_second = s_smooth + (swap ? 0 : 4);
-    for (int e = H + t; e < smooth_smem_floats<NT>(H); e += NT) s_smooth[e] = 0.0f;
-    if constexpr (FUSED) {
-        block_route_clear<NT>(rs, a.num_instances);
-        if (t == 0) mbar_init(&s_bar, 1);
-        __syncthreads();
-        pdl_wait();  // the instance ids may come from the previous kernel
-    }
     int key0 = -1;
     if (w == 0) {  // the sent copies, in k order: instance and position k
         key0 = lane < K ? copy_key(a, i * K + lane) : -1;

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -161,11 +162,15 @@ bool encode_i8_rows(CUtensorMap *m, const void *base, uint64_t inner, uint64_t o
 }
 
 // Every kernel is launched as a programmatic dependent of whatever precedes it
-// on the stream: its blocks may be scheduled while the previous kernel drains,
-// and each kernel calls griddepcontrol.wait before it touches memory a
-// predecessor could still be writing or reading (the route -> scatter pair
-// inside moe_dispatch is the one edge where the dependent first works on the
-// call's own inputs; the route kernel only releases it after its own wait).
+// on the stream: its blocks may be scheduled while the previous kernel drains.
+// The rule that keeps this safe: the FIRST kernel of every call reads no
+// global memory before griddepcontrol.wait, since any of the call's inputs
+// may be written by the kernel before it (a combine's y is the next layer's
+// x), and that kernel may release its dependents before its last store.  A
+// later kernel of the same call may read the call's inputs before its own
+// wait only when the call's first kernel releases dependents after its wait
+// (route -> scatter inside moe_dispatch): everything before the call has then
+// completed.  Outputs of earlier kernels of the call are read after the wait.
 // The attribute is harmless when the predecessor is not a kernel.
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t s, Args... args) {
@@ -596,15 +601,26 @@ namespace {
 // use this name as an address; the device address is looked up per device.
 __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
+// The array's device address on device `dev`, looked up by the first call
+// on that device (with `dev` current) and kept for the life of the process.
+// Host threads may make that first call at once: the lookup runs under a
+// lock and the address is published with release / acquire ordering.  A
+// failed lookup stores nothing, so a later call tries again.  The cache does
+// not survive cudaDeviceReset (which destroys the array with the context).
 void *noalloc_scratch_address(int dev) {
-    static void *addr[64];  // per device, filled on first use
-    if (dev < 0 || dev >= 64) return nullptr;
-    if (addr[dev] == nullptr) {
-        void *p = nullptr;
+    constexpr int kMaxDevices = 64;
+    static std::atomic<void *> addr[kMaxDevices];
+    static std::mutex mu;
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    void *p = addr[dev].load(std::memory_order_acquire);
+    if (p != nullptr) return p;
+    std::lock_guard<std::mutex> lock(mu);
+    p = addr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        addr[dev] = p;
+        addr[dev].store(p, std::memory_order_release);
     }
-    return addr[dev];
+    return p;
 }
 
 }  // namespace

@@ -346,8 +346,12 @@ MOE_API moe_status moe_grouped_matmul_mx(const moe_gmm_params *p, const void *ex
 /* moe_dispatch_noalloc -- moe_dispatch without a caller-provided workspace  */
 /* ------------------------------------------------------------------------ */
 
-/* Largest workspace moe_dispatch_noalloc can stand in for (bytes): enough for
- * every moe_dispatch the limits allow. */
+/* Size of the static scratch array behind moe_dispatch_noalloc (bytes), on
+ * every GPU that loads the library.  It covers every call with one source
+ * rank and any call of at most 8192 (token, k) copies; a call with several
+ * source ranks past 8192 copies needs a larger workspace (its route table)
+ * and moe_dispatch_noalloc refuses it with MOE_ERR_WORKSPACE, launching
+ * nothing. */
 #define MOE_NOALLOC_SCRATCH_BYTES MOE_MAX_WORKSPACE_BYTES
 
 /*
@@ -365,11 +369,14 @@ MOE_API moe_status moe_grouped_matmul_mx(const moe_gmm_params *p, const void *ex
  *                     this call's device error word (MOE_DEV_* bits) at its end.
  *
  * The first call on a device looks the array's device address up (with that
- * device current); make that first call before any stream capture.  Each call
- * zeroes the error word first, and every call on a device shares the one
- * array, so calls that overlap on the GPU (other streams, other threads) race
- * on it.  Returns MOE_ERR_WORKSPACE if the call would need more scratch than
- * the array holds; other errors as moe_dispatch.
+ * device current; several host threads may make it at once); make that first
+ * call before any stream capture.  The address is kept until the process
+ * exits and is not valid after cudaDeviceReset.  Each call zeroes the error
+ * word first, and every call on a device shares the one array, so calls that
+ * overlap on the GPU (other streams, other threads) race on it.  Returns
+ * MOE_ERR_WORKSPACE, enqueuing nothing, if the call would need more scratch
+ * than the array holds (see MOE_NOALLOC_SCRATCH_BYTES); other errors as
+ * moe_dispatch.
  */
 MOE_API moe_status moe_dispatch_noalloc(const moe_dispatch_params *p, const void *x, const int32_t *instance_ids,
                                         const uint8_t *mask, const float *smooth_scales, void *expand_x,

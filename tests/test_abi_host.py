@@ -248,3 +248,21 @@ def test_binding_refuses_host_workspaces(L):
     with pytest.raises(ValueError, match="CUDA"):
         L.grouped_matmul(torch.zeros((4, 1024), dtype=torch.int8), torch.ones(4), torch.zeros(2, dtype=torch.int32),
                          torch.zeros((1, 16, 1024), dtype=torch.int8), torch.ones((1, 16)), workspace=host_ws)
+
+
+def test_binding_refuses_host_outputs(L):
+    """Outputs a caller passes in are written through raw device pointers:
+    host tensors, wrong dtypes and missing entries are refused before any
+    call is made."""
+    rows, H, K, E = 16, 1024, 2, 8
+    host = dict(expand_x=torch.zeros((rows, H), dtype=torch.bfloat16), dyn_scales=None,
+                expand_idx=torch.zeros((8, K), dtype=torch.int32), src_of_row=torch.zeros(rows, dtype=torch.int32),
+                counts=torch.zeros(E, dtype=torch.int32), offsets=torch.zeros(E + 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA"):
+        L._check_dispatch_out(host, 8, H, K, E, 0)
+    with pytest.raises(TypeError, match="expand_x"):
+        L._check_dispatch_out(dict(host, expand_x=None), 8, H, K, E, 0)
+    with pytest.raises(TypeError):
+        L._check_dispatch_out([1, 2], 8, H, K, E, 0)
+    with pytest.raises(ValueError, match="CUDA"):
+        L._check_combine_out(dict(y=torch.zeros((8, H), dtype=torch.bfloat16)), 8, H)

@@ -16,7 +16,8 @@ import torch
 from combine_moe_update_b200 import inputs as gen
 from oracle import oracle as orc
 
-from gpu_harness import POISON, assert_close_bf16, dev, dev_bf16, host, poison_
+from gpu_harness import POISON, assert_close_bf16, assert_gmm_parity as _assert_gmm_parity, dev, dev_bf16, \
+    host, poison_
 
 pytestmark = pytest.mark.gpu
 
@@ -46,21 +47,6 @@ def _oracle(gi):
     rows, N = gi.expand_x.shape[0], gi.weight.shape[1]
     return orc.grouped_matmul(gi.expand_x, gi.dyn_scales, gi.offsets, gi.weight, gi.weight_scales,
                               out=np.full((rows, N), POISON16, np.uint16))
-
-
-def _assert_gmm_parity(got, o):
-    want = o["out"]
-    written = ~np.isnan(o["out_f64"])
-    # rows the call does not own keep the poison
-    np.testing.assert_array_equal(got[~written], want[~written])
-    g, w = got[written].astype(np.int32), want[written].astype(np.int32)
-    same = g == w
-    # where they differ: one bf16 step apart, same sign (adjacent bit patterns)
-    assert np.all(np.abs(g - w)[~same] == 1), "a bf16 output is more than one step from the oracle"
-    assert same.mean() >= 0.999, f"only {same.mean():.5f} of the outputs are bit-identical"
-    if written.any():
-        rows = np.flatnonzero(written.any(axis=1))
-        assert_close_bf16(got[rows], o["out_f64"][rows], what="gmm out")
 
 
 @pytest.mark.parametrize("H,N,counts,spare", [

@@ -454,6 +454,36 @@ def test_layer_stack_cuda_graph(B):
     torch.cuda.synchronize()
     assert B.read_device_error(wsp) == 0
 
+    # Every layer against the oracle run on the inputs the GPU actually had
+    # (its own y and x_out of the layer before): routing, rows and counts bit
+    # for bit, y and x_out element-wise within the 1e-2 bar.
+    x, r = st.x0, st.residual0
+    for l in range(L):
+        ob, om, e1 = orc.update_expert(st.expert_ids[l], st.table, st.ep_world_size,
+                                       expert_scales=st.expert_scales[l])
+        assert e1 == 0
+        np.testing.assert_array_equal(host(bal[l]), ob)
+        np.testing.assert_array_equal(host(bm[l]), om)
+        d = orc.dispatch(x, ob, E, 0, mask=om)
+        n = d["n"]
+        np.testing.assert_array_equal(host(dsp[l]["expand_idx"]), d["expand_idx"])
+        np.testing.assert_array_equal(host(dsp[l]["counts"]), d["counts"])
+        np.testing.assert_array_equal(host(dsp[l]["offsets"]), d["offsets"])
+        np.testing.assert_array_equal(host(dsp[l]["src_of_row"])[:n], d["src_of_row"])
+        np.testing.assert_array_equal(host(dsp[l]["expand_x"])[:n], d["expand_x"][:n])
+        c = orc.combine_add_rmsnorm(d["expand_x"], d["expand_idx"], st.expert_scales[l], r, st.gammas[l],
+                                    st.norm_eps)
+        y, xo = host(outs[l]["y"]), host(outs[l]["x_out"])
+        assert_close_bf16(y, c["y_f64"], what=f"y layer {l}")
+        assert_close_bf16(xo, c["x_f64"], what=f"x_out layer {l}")
+        x, r = y, xo
+
+    # Extra: the oracle chained on its own outputs drifts from the GPU chain
+    # only by rounding.  With identity experts x = S * y + x_out, where S is
+    # the sum of the fp32 weights (1 +- 1e-7): sums of two bf16 values sit on
+    # bf16 rounding ties that binary32 and binary64 break differently, and a
+    # flipped ulp rides along into later layers, so this chain is held to a
+    # per-row relative L2 bound.
     x, r = st.x0, st.residual0
     for l in range(L):
         ob, om, _ = orc.update_expert(st.expert_ids[l], st.table, st.ep_world_size,
@@ -461,19 +491,44 @@ def test_layer_stack_cuda_graph(B):
         d = orc.dispatch(x, ob, E, 0, mask=om)
         c = orc.combine_add_rmsnorm(d["expand_x"], d["expand_idx"], st.expert_scales[l], r, st.gammas[l],
                                     st.norm_eps)
-        np.testing.assert_array_equal(host(dsp[l]["expand_idx"]), d["expand_idx"])
-        if l == 0:
-            assert_close_bf16(host(outs[l]["y"]), c["y_f64"], what="y layer 0")
-            assert_close_bf16(host(outs[l]["x_out"]), c["x_f64"], what="x_out layer 0")
-        else:
-            # Later layers take each side's own bf16 outputs as inputs.  With
-            # identity experts x = S * y + x_out, S = sum of the fp32 weights
-            # = 1 +- 1e-7, so sums of two bf16 values sit on bf16 rounding
-            # ties that the fp32 (GPU) and f64 (oracle) weight sums break
-            # differently; a flipped ulp then rides along into later layers.
-            # The chain is therefore held to a per-row relative L2 bound.
-            for got, want in ((host(outs[l]["y"]), c["y_f64"]), (host(outs[l]["x_out"]), c["x_f64"])):
-                g = gen.bf16_to_f32(got).astype(np.float64)
-                rel = np.linalg.norm(g - want, axis=1) / np.linalg.norm(want, axis=1)
-                assert rel.max() < 1e-2, (l, float(rel.max()))
+        for got, want in ((host(outs[l]["y"]), c["y_f64"]), (host(outs[l]["x_out"]), c["x_f64"])):
+            g = gen.bf16_to_f32(got).astype(np.float64)
+            rel = np.linalg.norm(g - want, axis=1) / np.linalg.norm(want, axis=1)
+            assert rel.max() < 1e-2, (l, float(rel.max()))
         x, r = c["y"], c["x_out"]
+
+
+# ------------------------------------------------------------ binding checks
+
+def test_binding_checks_caller_outputs(B):
+    """Caller-supplied outputs reach the kernels as raw device pointers, so
+    the binding refuses any that is not exactly what the call writes (an
+    undersized buffer would be written past its end)."""
+    w = gen.make("tiny")
+    x, ids = dev_bf16(w.x), dev(w.expert_ids)
+    good = B.alloc_dispatch_outputs(w.bs, w.hidden, w.top_k, w.num_instances, 0)
+    B.dispatch(x, ids, w.num_instances, w.ep_world_size, 0, out=good)
+    torch.cuda.synchronize()
+    bad = dict(good, expand_x=good["expand_x"][: w.bs])  # too few rows
+    with pytest.raises(ValueError, match="expand_x"):
+        B.dispatch(x, ids, w.num_instances, w.ep_world_size, 0, out=bad)
+    with pytest.raises(ValueError, match="expand_x"):
+        B.dispatch_noalloc(x, ids, w.num_instances, w.ep_world_size, 0, out=bad)
+    bad = dict(good, counts=good["counts"].cpu())  # host memory
+    with pytest.raises(ValueError, match="CUDA"):
+        B.dispatch(x, ids, w.num_instances, w.ep_world_size, 0, out=bad)
+    bad = dict(good, expand_idx=good["expand_idx"].to(torch.int64))
+    with pytest.raises(TypeError, match="expand_idx"):
+        B.dispatch(x, ids, w.num_instances, w.ep_world_size, 0, out=bad)
+    with pytest.raises(TypeError, match="dyn_scales"):  # mode 2 sends scales: they must be given
+        B.dispatch(x, ids, w.num_instances, w.ep_world_size, 2,
+                   out=dict(B.alloc_dispatch_outputs(w.bs, w.hidden, w.top_k, w.num_instances, 2), dyn_scales=None))
+    idx = good["expand_idx"]
+    sc, res, gm = dev(w.expert_scales), dev_bf16(w.residual), dev_bf16(w.gamma)
+    ex = dev_bf16(w.expert_out)
+    y_small = torch.empty((w.bs - 1, w.hidden), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError, match="y"):
+        B.combine_add_rmsnorm(ex, idx, sc, res, gm, w.norm_eps, out=dict(y=y_small))
+    with pytest.raises(ValueError, match="rstd"):
+        B.combine_add_rmsnorm(ex, idx, sc, res, gm, w.norm_eps,
+                              out=dict(y=torch.empty_like(res), rstd=torch.empty(w.bs - 1, device="cuda")))

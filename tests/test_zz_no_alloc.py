@@ -91,3 +91,27 @@ def test_noalloc_rejects_bad_sizes_before_launch(B):
     with pytest.raises(B.MoeError) as e:
         B.dispatch_noalloc(x, ids, 8, 4, 0)
     assert e.value.status == B.MOE_ERR_INVALID_ARG
+
+
+def test_noalloc_refuses_calls_that_need_a_route_table(B):
+    """Several source ranks past 8192 copies need a workspace larger than the
+    static array (the route's slice table): the call is refused with
+    MOE_ERR_WORKSPACE and nothing is enqueued, so the outputs keep their
+    poison."""
+    S, bs, H, K, E, ws = 2, 512, 1024, 16, 64, 8
+    rng = np.random.Generator(np.random.PCG64(90))
+    x = dev_bf16(gen.bf16_bits(rng.standard_normal((S * bs, H), np.float32)))
+    ids = dev(gen.topk_uniform(rng, S * bs, E, K))
+    assert B.dispatch_workspace_bytes(bs, H, K, ws, E, 0, 0, S) > 256
+    out = B.alloc_dispatch_outputs(S * bs, H, K, E, 0)
+    for v in out.values():
+        if v is not None:
+            v.view(torch.uint8).fill_(0xA5)
+    torch.cuda.synchronize()
+    with pytest.raises(B.MoeError) as e:
+        B.dispatch_noalloc(x, ids, E, ws, 0, out=out, sources=S)
+    assert e.value.status == B.MOE_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    for k, v in out.items():
+        if v is not None:
+            assert bool((v.view(torch.uint8) == 0xA5).all()), k
