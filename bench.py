@@ -4,11 +4,17 @@
 One step = one MoE layer's hot path on one batch of seeded synthetic input:
 moe_update_expert -> moe_dispatch -> moe_combine_add_rmsnorm (the expert FFN
 between dispatch and combine is stood in for by a resident buffer of bf16
-expert-output rows).  Every timed step starts with a cold, clean L2 (a
-512 MiB buffer is overwritten and a 256 MiB one read before it, outside the
-timed events).
+expert-output rows).  The step's inputs are cold in L2 when it starts: where
+a few input sets (activations and the layer's parameters) together exceed
+twice L2, the timed steps cycle through them back to back with events only
+at the ends of each graph; smaller workloads flush L2 (512 MiB written, then
+256 MiB read) before every step, outside the timed events.  `config.l2` says
+which.  The line also carries the gate figure -- dispatch + combine alone,
+pairs back to back over the cold sets -- and each kernel's roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
+
+`--workload layer_stack` times 32 chained layers captured in one CUDA graph.
 
 With N > 1 it runs under torch.distributed.run, one process per GPU; the
 path has no exchange step on one GPU, so every rank runs an independent
@@ -73,10 +79,29 @@ def algorithmic_bytes(w, n, x_out=False, rstd=False):
     return dict(update=upd, dispatch=disp, combine=comb)
 
 
+def kernels_per_step(w):
+    """Kernels of this library one step launches: update_expert, the
+    dispatch's kernels, the combine.  Per-instance scales take the
+    instance-major kernel, which routes its own copies up to 8192 copies;
+    otherwise up to 1024 copies the scatter blocks route themselves, up to
+    8192 one route kernel runs first, and beyond that the three-pass route."""
+    copies = w.bs * w.top_k
+    per_instance = w.smooth is not None and w.smooth.size > w.hidden
+    if copies > 8192:
+        disp = 4
+    elif per_instance or copies <= 1024:
+        disp = 1
+    else:
+        disp = 2
+    return 1 + disp + 1
+
+
 # The sources a kernel is compiled from: stored ncu counters are kept while
 # these files are unchanged.
 KERNEL_SOURCES = {
     "combine_token_kernel": ("combine.cuh", "common.cuh"),
+    "dispatch_instance_kernel": ("dispatch.cuh", "common.cuh"),
+    "dispatch_token_kernel": ("dispatch.cuh", "common.cuh"),
     "gmm_kernel": ("grouped_matmul.cuh", "common.cuh"),
     "gmm_mx_kernel": ("grouped_matmul.cuh", "common.cuh"),
 }
@@ -348,52 +373,99 @@ def run_b200(args, rank, world, local_rank):
                 sums[3] += e[2].elapsed_time(e[3])
     barrier()
     del graph, graph_ops
+    assert B.read_device_error(ws) == 0, "device error during the timed steps"
+
+    def time_graph(body, count):
+        """Per-body time (ms): `body` captured `count` times in one graph with
+        events only at its ends, replayed a few times."""
+        eb = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            eb[0].record()
+            for n_ in range(count):
+                body(n_)
+            eb[1].record()
+        g.replay()
+        torch.cuda.synchronize()
+        reps = max(3, min(50, K // 4))
+        tot = 0.0
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            tot += eb[0].elapsed_time(eb[1]) / count
+        del g
+        return tot / reps
+
+    # The gate (dispatch + combine alone): pairs back to back over the cold
+    # input sets, each set's routing (update_expert's output) computed once
+    # beforehand, events only at the graph's ends, so each pair overlaps its
+    # predecessor's tail as consecutive layers would.
+    t_pair = None
+    if cold_sets:
+        routes = []
+        for xx, ii, ss, rr, ee, sh, tb, sm, gm in sets:
+            rb, rm = torch.empty_like(bal), torch.empty_like(bm)
+            upd(ii, tb, w.ep_world_size, expert_scales=ss, prune_threshold=w.prune_threshold, workspace=ws,
+                out=(rb, rm))
+            routes.append((rb, rm))
+
+        def pair(n_):
+            (xx, ii, ss, rr, ee, sh, tb, sm, gm), (rb, rm) = sets[n_ % R], routes[n_ % R]
+            disp(xx, rb, w.num_instances, w.ep_world_size, w.quant_mode, mask=rm, smooth=sm, workspace=ws, out=d)
+            comb(ee, d["expand_idx"], ss, rr, gm, w.norm_eps, shared_x=sh, workspace=ws, out=c)
+
+        t_pair = time_graph(pair, R * max(1, 16 // R))
+        del routes
+        assert B.read_device_error(ws) == 0, "device error during the gate pairs"
+        gate_timing = (f"{R * max(1, 16 // R)} dispatch+combine pairs back to back over {R} input sets "
+                       f"({R * per_set / 2**20:.0f} MiB > 2 x L2), routing computed beforehand, CUDA events around "
+                       "the whole run")
     if cold_sets:
         del sets
-    assert B.read_device_error(ws) == 0, "device error during the timed steps"
-    # Combine kernel on its own for the roofline: launches back to back (each a
-    # programmatic dependent of the one before, as in consecutive layers) over
-    # R input sets whose total exceeds L2, so every launch reads cold rows and
-    # no event sits between launches; the time per launch is the span / count.
-    # (Workloads too small for a few sets to exceed L2 use the event-bracketed
-    # call time of the breakdown graph instead, and say so.)
-    per_set = sum(t.numel() * t.element_size() for t in (expert_out, residual, shared) if t is not None)
-    R = -(-(2 * L2_BYTES) // per_set) + 1
-    if R <= 16:
-        sets = [dict(ee=torch.empty_like(expert_out).copy_(expert_out),
-                     rr=torch.empty_like(residual).copy_(residual),
-                     sh=None if shared is None else torch.empty_like(shared).copy_(shared)) for _ in range(R)]
-        M = max(1, 16 // R)  # passes over the sets per graph
-        eb = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-        graph_c = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_c, stream=cap):
-            eb[0].record()
-            for _ in range(M):
-                for st in sets:
-                    comb(st["ee"], d["expand_idx"], scales, st["rr"], gamma, w.norm_eps,
-                                          shared_x=st["sh"], workspace=ws, out=c)
-            eb[1].record()
-        graph_c.replay()
-        torch.cuda.synchronize()
-        reps_c = max(3, min(50, K // 16))
-        t_comb_kernel = 0.0
-        for _ in range(reps_c):
-            graph_c.replay()
-            torch.cuda.synchronize()
-            t_comb_kernel += eb[0].elapsed_time(eb[1]) / (M * R)
-        del graph_c, sets
-        t_comb_kernel /= reps_c
-        comb_timing = (f"{M * R} back-to-back launches over {R} input sets ({R * per_set / 2**20:.0f} MiB > L2), "
-                       "CUDA events around the whole run")
-        assert B.read_device_error(ws) == 0, "device error during the combine roofline launches"
+
+    # Each kernel on its own for the roofline: launches back to back (each a
+    # programmatic dependent of the one before, as in consecutive layers)
+    # over input sets whose total exceeds twice L2, so every launch reads
+    # cold inputs and no event sits between launches; time per launch = the
+    # span / count.  Workloads too small for that use the event-bracketed
+    # call of the breakdown graph instead, and say so.
+    def cold_copies(tensors):
+        per = sum(t.numel() * t.element_size() for t in tensors if t is not None)
+        n_ = -(-(2 * L2_BYTES) // per) + 1
+        return n_, per
+
+    R_c, per_c = cold_copies((expert_out, residual, shared))
+    if R_c <= 16:
+        csets = [[None if t is None else t.clone() for t in (expert_out, residual, shared)] for _ in range(R_c)]
+        t_comb_kernel = time_graph(
+            lambda n_: comb(csets[n_ % R_c][0], d["expand_idx"], scales, csets[n_ % R_c][1], gamma, w.norm_eps,
+                            shared_x=csets[n_ % R_c][2], workspace=ws, out=c), R_c * max(1, 16 // R_c))
+        del csets
+        comb_timing = (f"{R_c * max(1, 16 // R_c)} back-to-back launches over {R_c} input sets "
+                       f"({R_c * per_c / 2**20:.0f} MiB > 2 x L2), CUDA events around the whole run")
     else:
         t_comb_kernel = sums[3] / K
         comb_timing = "per-call CUDA events in the breakdown graph (inputs too small to exceed L2 in a few sets)"
 
-    t_step, t_upd, t_disp, t_comb, t_comb_kernel = reduce_over_ranks(
-        [v / K for v in sums] + [t_comb_kernel], "max")
+    R_d, per_d = cold_copies((x, smooth, bal, bm))
+    if R_d <= 32:
+        # copies of x, the scale rows and the routing (bal, bm hold this batch's)
+        dsets = [[None if t is None else t.clone() for t in (x, smooth, bal, bm)] for _ in range(R_d)]
+        t_disp_kernel = time_graph(
+            lambda n_: disp(dsets[n_ % R_d][0], dsets[n_ % R_d][2], w.num_instances, w.ep_world_size, w.quant_mode,
+                            mask=dsets[n_ % R_d][3], smooth=dsets[n_ % R_d][1], workspace=ws, out=d),
+            R_d * max(1, 32 // R_d))
+        del dsets
+        disp_timing = (f"{R_d * max(1, 32 // R_d)} back-to-back calls over {R_d} input sets "
+                       f"({R_d * per_d / 2**20:.0f} MiB > 2 x L2), CUDA events around the whole run")
+    else:
+        t_disp_kernel = sums[2] / K
+        disp_timing = "per-call CUDA events in the breakdown graph (inputs too small to exceed L2 in a few sets)"
+    assert B.read_device_error(ws) == 0, "device error during the roofline launches"
+
+    t_step, t_upd, t_disp, t_comb, t_comb_kernel, t_disp_kernel, t_pair = reduce_over_ranks(
+        [v / K for v in sums] + [t_comb_kernel, t_disp_kernel, t_pair if t_pair is not None else 0.0], "max")
     value = world * w.bs / (t_step * 1e-3)
-    dc_value = world * w.bs / ((t_disp + t_comb) * 1e-3)
 
     # ---- end to end through the public API with host buffers ----
     pin = lambda t: t.cpu().pin_memory()
@@ -427,16 +499,30 @@ def run_b200(args, rank, world, local_rank):
     (t_e2e,) = reduce_over_ranks([e0.elapsed_time(e1) / ke], "max")
 
     peak, peak_kind = measured_peak()
-    achieved = alg["combine"] / (t_comb_kernel * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "combine_token_kernel", "achieved": round(achieved, 1),
-                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "launch_us": round(t_comb_kernel * 1e3, 2),
-                "timing": comb_timing,
-                "traffic": stored_traffic("combine_token_kernel", args.workload),
-                "algorithmic_bytes": alg["combine"]}
-    disp_gbs = alg["dispatch"] / (t_disp * 1e-3) / 1e9
+    per_instance = w.smooth is not None and w.smooth.size > w.hidden
+    disp_name = "dispatch_instance_kernel" if per_instance else "dispatch_token_kernel"
+
+    def roof(kernel, nbytes, t_ms, timing, traffic_key):
+        a = nbytes / (t_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "kernel": kernel, "achieved": round(a, 1), "peak": peak, "peak_kind": peak_kind,
+                "unit": "GB/s", "frac": round(a / peak, 4), "launch_us": round(t_ms * 1e3, 2), "timing": timing,
+                "traffic": stored_traffic(traffic_key, args.workload) if traffic_key else None,
+                "algorithmic_bytes": nbytes}
+
+    r_comb = roof("combine_token_kernel", alg["combine"], t_comb_kernel, comb_timing, "combine_token_kernel")
+    r_disp = roof(disp_name, alg["dispatch"], t_disp_kernel, disp_timing,
+                  disp_name if disp_name in KERNEL_SOURCES else None)
+    r_disp["note"] = ("the whole moe_dispatch call: one kernel that routes its own copies"
+                      if kernels_per_step(w) == 3 else "the whole moe_dispatch call (route and scatter kernels)")
+    # the dominant kernel by time carries the line's roofline
+    roofline, other = (r_comb, r_disp) if t_comb_kernel >= t_disp_kernel else (r_disp, r_comb)
     step_gbs = (alg["update"] + alg["dispatch"] + alg["combine"]) / (t_step * 1e-3) / 1e9
-    dc_gbs = (alg["dispatch"] + alg["combine"]) / ((t_disp + t_comb) * 1e-3) / 1e9
+    gate = None
+    if t_pair:
+        gb = (alg["dispatch"] + alg["combine"]) / (t_pair * 1e-3) / 1e9
+        gate = {"us": round(t_pair * 1e3, 2), "tokens_per_s": round(world * w.bs / (t_pair * 1e-3), 1),
+                "hbm_gbs": round(gb, 1), "frac_of_peak": round(gb / peak, 4),
+                "algorithmic_bytes": alg["dispatch"] + alg["combine"], "timing": gate_timing}
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",
@@ -447,23 +533,226 @@ def run_b200(args, rank, world, local_rank):
                    "quant_mode": w.quant_mode, "smooth_scales": w.smooth is not None,
                    "shared_expert": w.shared_x is not None, "kept_copies": n,
                    "l2": l2_note, "parallelism": f"replicas x{world}"},
+        "gate": gate,
         "breakdown_us": {"update_expert": round(t_upd * 1e3, 2), "dispatch": round(t_disp * 1e3, 2),
-                         "combine": round(t_comb * 1e3, 2)},
-        "dispatch_plus_combine": {"tokens_per_s": round(dc_value, 1), "hbm_gbs": round(dc_gbs, 1),
-                                  "frac_of_peak": round(dc_gbs / peak, 4),
-                                  "algorithmic_bytes": alg["dispatch"] + alg["combine"]},
-        "achieved_gbs": {"step": round(step_gbs, 1), "dispatch_bracketed": round(disp_gbs, 1),
-                         "combine": round(achieved, 1)},
+                         "combine": round(t_comb * 1e3, 2),
+                         "note": "each call bracketed by its own events (about 4.5 us each, no launch overlap)"},
+        "achieved_gbs": {"step": round(step_gbs, 1), "dispatch": r_disp["achieved"], "combine": r_comb["achieved"]},
         "roofline": roofline,
+        "roofline_other": other,
         "e2e": {"value": round(world * w.bs / (t_e2e * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "pinned host activations -> device, the three calls, y -> host; layer parameters resident"},
-        "gpu_launches": 4 * K,  # update_expert, route, quantize-and-scatter, combine
+        "gpu_launches": kernels_per_step(w) * K,
         "timing": (f"CUDA graphs of {G} steps; breakdown_us from a second graph with the L2 flush before each step "
                    "and events between the calls (no launch overlap there, so its parts sum above a step)"),
         "clocks": clk.summary(),
     }
     return out, w
+
+
+def run_b200_layer_stack(args, rank, world, local_rank):
+    """32 chained MoE layers captured in one CUDA graph: each layer is
+    update_expert -> dispatch (bf16 rows) -> identity expert (the combine
+    reads the dispatch's rows) -> combine+Add+RMSNorm, with X_{l+1} = y_l and
+    residual_{l+1} = x_out_l.  A timed iteration is one replay of the whole
+    stack, with L2 flushed before it outside the events; per-layer time =
+    replay time / 32."""
+    import numpy as np
+    import torch
+    from combine_moe_update_b200 import binding as B
+    from combine_moe_update_b200 import inputs as gen
+
+    torch.cuda.set_device(local_rank)
+    st = gen.make_layer_stack(seed=4 if rank == 0 else 1000 + rank)
+    L, bs, H, K, E = st.layers, st.bs, st.hidden, st.top_k, st.num_experts
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    bf = lambda a: dev(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16)
+    ids = [dev(a) for a in st.expert_ids]
+    scs = [dev(a) for a in st.expert_scales]
+    gms = [bf(a) for a in st.gammas]
+    table = dev(st.table)
+    x0, r0 = bf(st.x0), bf(st.residual0)
+    wsp = B.new_workspace()
+    bal = [torch.empty((bs, K), dtype=torch.int32, device="cuda") for _ in range(L)]
+    bm = [torch.empty((bs, K), dtype=torch.uint8, device="cuda") for _ in range(L)]
+    dsp = [B.alloc_dispatch_outputs(bs, H, K, E, 0) for _ in range(L)]
+    outs = [dict(y=torch.empty((bs, H), dtype=torch.bfloat16, device="cuda"),
+                 x_out=torch.empty((bs, H), dtype=torch.bfloat16, device="cuda"), rstd=None) for _ in range(L)]
+
+    def stack():
+        x, r = x0, r0
+        for l in range(L):
+            B.update_expert(ids[l], table, st.ep_world_size, expert_scales=scs[l], workspace=wsp, out=(bal[l], bm[l]))
+            B.dispatch(x, bal[l], E, st.ep_world_size, 0, mask=bm[l], workspace=wsp, out=dsp[l])
+            B.combine_add_rmsnorm(dsp[l]["expand_x"], dsp[l]["expand_idx"], scs[l], r, gms[l], st.norm_eps,
+                                  workspace=wsp, out=outs[l])
+            x, r = outs[l]["y"], outs[l]["x_out"]
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clean = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.float32, device="cuda")
+
+    def flush_l2():
+        flush.zero_()
+        clean.sum()
+
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        for _ in range(args.warmup):
+            stack()
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+    assert B.read_device_error(wsp) == 0, "device error during warm-up"
+    n = int(dsp[0]["offsets"][-1].item())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        stack()
+    g.replay()
+    torch.cuda.synchronize()
+
+    K_ = args.steps
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K_)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K_)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for k_ in range(K_):
+            flush_l2()
+            e0[k_].record()
+            g.replay()
+            e1[k_].record()
+        torch.cuda.synchronize()
+    barrier()
+    t_stack = sum(a.elapsed_time(b) for a, b in zip(e0, e1)) / K_
+    assert B.read_device_error(wsp) == 0, "device error during the timed stacks"
+
+    # end to end: the stack's inputs (x0, residual0 and every layer's routing)
+    # from pinned host memory, the graph, the last y back to the host
+    pin = lambda t: t.cpu().pin_memory()
+    h_in = [(pin(x0), x0), (pin(r0), r0)] + [(pin(t), t) for t in ids + scs]
+    h_y = torch.empty((bs, H), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(h.numel() * h.element_size() for h, _ in h_in)
+    d2h = h_y.numel() * h_y.element_size()
+
+    def e2e_step():
+        for h, d_ in h_in:
+            d_.copy_(h, non_blocking=True)
+        g.replay()
+        h_y.copy_(outs[-1]["y"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ke = max(5, min(K_, 100))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(ke):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    t_stack, t_e2e = reduce_over_ranks([t_stack, a0.elapsed_time(a1) / ke], "max")
+    del g
+
+    class _W:  # the per-layer shape, for the byte count
+        pass
+    lw = _W()
+    lw.bs, lw.hidden, lw.top_k, lw.num_instances, lw.num_logical = bs, H, K, E, E
+    lw.quant_mode, lw.prune_threshold, lw.smooth, lw.shared_x, lw.meta = 0, 0.0, None, None, {}
+    alg = algorithmic_bytes(lw, n, x_out=True)
+    per_layer = t_stack / L
+    peak, peak_kind = measured_peak()
+    layer_bytes = alg["update"] + alg["dispatch"] + alg["combine"]
+    achieved = layer_bytes / (per_layer * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": round(world * bs / (per_layer * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K_, "warmup": args.warmup, "ms_per_step": round(t_stack, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16+fp32", "data": "synthetic (seeded; pages' shapes)",
+        "config": {"workload": "layer_stack", "layers": L, "bs": bs, "hidden": H, "top_k": K, "num_instances": E,
+                   "ep_world_size_simulated": st.ep_world_size, "quant_mode": 0, "kept_copies_per_layer": n,
+                   "l2": "flushed before every timed stack (512 MiB written, then 256 MiB read), outside the events",
+                   "parallelism": f"replicas x{world}"},
+        "per_layer_us": round(per_layer * 1e3, 3),
+        "step": "one replay of the 32-layer graph; value = tokens through one layer per second (Bs / per-layer time)",
+        "roofline": {"bound": "hbm", "kernel": "whole layer (update, dispatch, combine)", "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "algorithmic_bytes": layer_bytes,
+                     "note": "latency-bound: 7.9 MB per layer, three dependent launches"},
+        "e2e": {"value": round(world * bs * L / (t_e2e * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "per step: x0, residual0 and all 32 layers' routing host -> device, the graph, the last y "
+                        "device -> host; value = Bs / (step time / 32)"},
+        "gpu_launches": 3 * L * K_,
+        "timing": "CUDA events around each replay of the 32-layer graph, L2 flushed before each replay",
+        "clocks": clk.summary(),
+    }
+    return out, st
+
+
+def oracle_stack(orc, st, lo, hi):
+    """The oracle's 32 chained layers on tokens [lo, hi) of the stack."""
+    x, r = st.x0[lo:hi], st.residual0[lo:hi]
+    for l in range(st.layers):
+        bal, bm, _ = orc.update_expert(st.expert_ids[l][lo:hi], st.table, st.ep_world_size,
+                                       expert_scales=st.expert_scales[l][lo:hi])
+        d = orc.dispatch(x, bal, st.num_experts, 0, mask=bm)
+        c = orc.combine_add_rmsnorm(d["expand_x"], d["expand_idx"], st.expert_scales[l][lo:hi], r, st.gammas[l],
+                                    st.norm_eps)
+        x, r = c["y"], c["x_out"]
+
+
+def layer_stack_oracle_rate(st, workers, budget_s):
+    """Per-layer tokens/s of `workers` threads each running the oracle's
+    chained layers on its own slice of tokens.  Returns (tokens/s, slice)."""
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import oracle as orc
+    per = st.bs if workers == 1 else max(1, st.bs // workers)
+    span = max(1, st.bs - per + 1)
+    oracle_stack(orc, st, 0, 1)  # build and warm
+
+    def work(k):
+        lo = (k * per) % span
+        done, t0 = 0, time.perf_counter()
+        while True:
+            oracle_stack(orc, st, lo, lo + per)
+            done += per
+            if time.perf_counter() - t0 >= budget_s:
+                return done, time.perf_counter() - t0
+
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        res = list(ex.map(work, range(workers)))
+    # tokens through one layer per second: every pass moves `per` tokens through all the layers
+    return st.layers * sum(r[0] for r in res) / max(r[1] for r in res), per
+
+
+def layer_stack_cpu_baseline(st, budget_s):
+    cores, model = host_cpu()
+    one, _ = layer_stack_oracle_rate(st, 1, budget_s / 2)
+    many, per = layer_stack_oracle_rate(st, cores, budget_s / 2)
+    return {"value": round(many, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle", "cpu_model": model,
+            "single_thread": round(one, 2),
+            "sample": (f"{cores} threads, each repeating the 32 chained oracle layers on its own slice of {per} of the "
+                       f"{st.bs} tokens for {budget_s / 2:.0f} s; value = tokens through one layer per second")}
+
+
+def layer_stack_reference(args):
+    from combine_moe_update_b200 import inputs as gen
+    st = gen.make_layer_stack()
+    cores, model = host_cpu()
+    budget = max(2.0, 100.0 / max(1, args.steps + args.warmup))
+    value, per = layer_stack_oracle_rate(st, cores, budget)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 quant / f64 combine",
+        "data": "synthetic (seeded; pages' shapes)",
+        "config": {"workload": "layer_stack", "layers": st.layers, "bs": st.bs, "hidden": st.hidden,
+                   "top_k": st.top_k, "num_instances": st.num_experts, "quant_mode": 0},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "cpu_model": model,
+                         "sample": f"{cores} threads x {per} tokens through 32 chained layers, {budget:.0f} s"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
 
 
 def gmm_bytes(offsets, hidden, out_dim, mx=False):
@@ -722,22 +1011,64 @@ def _oracle_expert_rows(orc, w, d):
     return g["out"]
 
 
-def subsample(w, tokens):
-    """The first `tokens` tokens of the workload (same parameters)."""
+def subsample(w, tokens, start=0):
+    """Tokens [start, start + tokens) of the workload (same parameters)."""
     import copy
     s = copy.copy(w)
     s.bs = tokens
     for k in ("x", "expert_ids", "expert_scales", "residual", "shared_x", "active_mask"):
         v = getattr(w, k)
         if v is not None:
-            setattr(s, k, v[:tokens].copy())
-    s.expert_out = w.expert_out[: tokens * w.top_k].copy()
+            setattr(s, k, v[start:start + tokens].copy())
+    s.expert_out = w.expert_out[start * w.top_k:(start + tokens) * w.top_k].copy()
     s.meta = {k: v for k, v in w.meta.items() if not k.startswith("_")}
     return s
 
 
+def host_cpu():
+    """Cores this process may run on, and the CPU model."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return cores, model
+
+
+def oracle_rate(orc, w, workers, budget_s):
+    """Tokens per second of `workers` threads, each running the oracle step on
+    its own slice of the workload's tokens (data parallel over tokens) for
+    about `budget_s` seconds.  The oracle's C calls release the GIL, so the
+    threads run on separate cores.  Returns (tokens/s, tokens per slice)."""
+    from concurrent.futures import ThreadPoolExecutor
+    per = w.bs if workers == 1 else max(1, w.bs // workers)
+    span = max(1, w.bs - per + 1)
+    subs = [subsample(w, per, start=(k * per) % span) for k in range(workers)]
+    oracle_step(orc, subs[0])  # build and warm the oracle
+
+    def work(sub):
+        done, t0 = 0, time.perf_counter()
+        while True:
+            oracle_step(orc, sub)
+            done += sub.bs
+            if time.perf_counter() - t0 >= budget_s:
+                return done, time.perf_counter() - t0
+
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        res = list(ex.map(work, subs))
+    return sum(r[0] for r in res) / max(r[1] for r in res), per
+
+
 def cpu_baseline(w, budget_s=10.0):
+    """The oracle on this host: single-threaded, and on every core with one
+    token slice per core.  `value` is the all-cores figure."""
     from oracle import oracle as orc
+    cores, model = host_cpu()
     if "expert_out_dim" in w.meta:
         # a full step of the matmul layer takes minutes on one core: time a
         # sample of tokens sized from a one-token calibration run
@@ -754,19 +1085,17 @@ def cpu_baseline(w, budget_s=10.0):
         oracle_step(orc, sample)
         dt = time.perf_counter() - t0
         return {"value": round(tokens / dt, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "host_cores": cores, "cpu_model": model,
                 "sample": f"one step of the first {tokens} of {w.bs} tokens ({dt:.1f} s, single-threaded C "
                           "oracle; the weights of the instances they reach drawn on the host)"}
-    oracle_step(orc, subsample(w, 8))  # build + warm
-    t0 = time.perf_counter()
-    steps = 0
-    while True:
-        oracle_step(orc, w)
-        steps += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": round(steps * w.bs / dt, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{steps} full steps of {w.bs} tokens ({dt:.1f} s, single-threaded C oracle)"}
+    half = budget_s / 2
+    one, _ = oracle_rate(orc, w, 1, half)
+    many, per = oracle_rate(orc, w, cores, half)
+    return {"value": round(many, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "cpu_model": model, "single_thread": round(one, 2),
+            "sample": (f"{cores} threads, each repeating the oracle step on its own slice of {per} of the "
+                       f"{w.bs} tokens for {half:.0f} s (data parallel over tokens); single_thread: full "
+                       f"{w.bs}-token steps on one core for {half:.0f} s")}
 
 
 def run_reference(args, rank):
@@ -775,33 +1104,44 @@ def run_reference(args, rank):
         return None
     from combine_moe_update_b200 import inputs as gen
     from oracle import oracle as orc
-    w = gen.make(args.workload)
+    w = gen.make(args.workload) if args.workload != "layer_stack" else None
+    if w is None:
+        return layer_stack_reference(args)
     orc.build()
+    cores, model = host_cpu()
+    expert = "expert_out_dim" in w.meta
+    workers = 1 if expert else cores
     # calibrate: seconds per token, then size each step so the run stays within ~2 minutes
-    cal = 1 if "expert_out_dim" in w.meta else 16
+    cal = 1 if expert else 16
     t0 = time.perf_counter()
     oracle_step(orc, subsample(w, cal))
     per_tok = (time.perf_counter() - t0) / cal
     budget = 120.0 / max(1, args.steps + args.warmup)
-    # the matmul layer: at most 4 tokens, whose instances' weights are drawn on the host
-    tokens = int(max(1, min(4 if cal == 1 else w.bs, budget / max(per_tok, 1e-9))))
-    sample = subsample(w, tokens)
-    for _ in range(args.warmup):
-        oracle_step(orc, sample)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(orc, sample)
-    dt = time.perf_counter() - t0
-    value = args.steps * tokens / dt
+    # a step is one oracle step on a slice of the batch per thread; the matmul
+    # layer: at most 4 tokens, whose instances' weights are drawn on the host
+    tokens = int(max(1, min(4 if expert else max(1, w.bs // workers), budget / max(per_tok, 1e-9))))
+    span = max(1, w.bs - tokens + 1)
+    subs = [subsample(w, tokens, start=(k * tokens) % span) for k in range(workers)]
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        for _ in range(args.warmup):
+            list(ex.map(lambda sb: oracle_step(orc, sb), subs))
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            list(ex.map(lambda sb: oracle_step(orc, sb), subs))
+        dt = time.perf_counter() - t0
+    value = args.steps * tokens * workers / dt
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quant / f64 combine",
         "data": "synthetic (seeded; pages' shapes)",
         "config": {"workload": args.workload, "bs": w.bs, "hidden": w.hidden, "top_k": w.top_k,
-                   "num_instances": w.num_instances, "quant_mode": w.quant_mode, "tokens_per_step": tokens},
-        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{tokens} of {w.bs} tokens per step, {args.steps} steps"},
+                   "num_instances": w.num_instances, "quant_mode": w.quant_mode,
+                   "tokens_per_step": tokens * workers},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": workers, "kind": "oracle",
+                         "cpu_model": model,
+                         "sample": f"{workers} threads x {tokens} of the {w.bs} tokens per step, {args.steps} steps"},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -830,6 +1170,12 @@ def main(argv=None):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
+        if args.workload == "layer_stack":
+            out, st = run_b200_layer_stack(args, rank, world, local_rank)
+            if rank == 0:
+                out["cpu_baseline"] = layer_stack_cpu_baseline(st, args.cpu_baseline_seconds) if world == 1 else None
+                print(json.dumps(out), flush=True)
+            return 0
         out, w = run_b200(args, rank, world, local_rank)
         if rank == 0:
             out["cpu_baseline"] = cpu_baseline(w, args.cpu_baseline_seconds) if world == 1 else None

@@ -83,19 +83,32 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// 16-byte load through the non-coherent path without L1 allocation: for
-// rows that are read once per kernel.
+// Loads of kernel inputs.  Every kernel is launched as a programmatic
+// dependent of the one before it, so its lifetime overlaps its predecessor's
+// and any input may still be in flight from that kernel when this one
+// starts.  The non-coherent path (ld.global.nc, __ldg) promises data that
+// stays constant for the whole kernel and may be scheduled ahead of
+// griddepcontrol.wait, so it is never used here: these are ordinary coherent
+// loads, which the wait orders after the predecessor's stores.
+
+// 16 bytes, not allocated in L1: for rows that are read once per kernel.
 __device__ __forceinline__ uint4 ld_stream(const void *p) {
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
+                 : "l"(p)
+                 : "memory");
     return v;
 }
 
-// 16-byte read-only load that may be cached in L1 (rows reused by a block).
-__device__ __forceinline__ uint4 ld_cached(const void *p) {
-    return __ldg(reinterpret_cast<const uint4 *>(p));
+// 16 bytes that may stay in L1 (rows reused by a block).
+__device__ __forceinline__ uint4 ld_cached(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
+
+// One coherent element load (the plain C++ load, spelled out where a
+// read-only cache load would otherwise be the habit).
+template <typename T>
+__device__ __forceinline__ T ld_in(const T *p) {
+    return *p;
 }
 
 __device__ __forceinline__ void st_v4(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }

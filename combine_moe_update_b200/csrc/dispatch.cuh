@@ -63,8 +63,8 @@ struct DispatchArgs {
 // Key of copy j: its instance if it is sent, -1 if masked out, -2 if its id
 // is out of range (then it is dropped and reported).
 __device__ __forceinline__ int copy_key(const DispatchArgs &a, int j) {
-    const int id = __ldg(a.ids + j);  // both loads issue before either is used
-    const bool sent = a.mask ? __ldg(a.mask + j) != 0 : true;
+    const int id = ld_in(a.ids + j);  // both loads issue before either is used
+    const bool sent = a.mask ? ld_in(a.mask + j) != 0 : true;
     if (!sent) return -1;
     return (id >= 0 && id < a.num_instances) ? id : -2;
 }
@@ -120,14 +120,14 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
     int key[kRtKeys];
     uint8_t sent[kRtKeys];
     const int jm = mine0 + t;
-    int k = __ldg(a.ids + min(jm, N - 1));
+    int k = ld_in(a.ids + min(jm, N - 1));
     bool k_sent = jm < N;
 #pragma unroll
-    for (int u = 0; u < kRtKeys; ++u) key[u] = __ldg(a.ids + min(u * kRtThreads + t, N - 1));
+    for (int u = 0; u < kRtKeys; ++u) key[u] = ld_in(a.ids + min(u * kRtThreads + t, N - 1));
     if (a.mask) {
-        k_sent = k_sent && __ldg(a.mask + min(jm, N - 1)) != 0;
+        k_sent = k_sent && ld_in(a.mask + min(jm, N - 1)) != 0;
 #pragma unroll
-        for (int u = 0; u < kRtKeys; ++u) sent[u] = __ldg(a.mask + min(u * kRtThreads + t, N - 1));
+        for (int u = 0; u < kRtKeys; ++u) sent[u] = ld_in(a.mask + min(u * kRtThreads + t, N - 1));
     } else {
 #pragma unroll
         for (int u = 0; u < kRtKeys; ++u) sent[u] = 1;
@@ -252,10 +252,10 @@ __device__ void block_route(const DispatchArgs &a, int i, RS &rs, int key0) {
         int id[U];
         uint32_t ms[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) id[u] = __ldg(a.ids + min(j0 + u * NT + t, N - 1));
+        for (int u = 0; u < U; ++u) id[u] = ld_in(a.ids + min(j0 + u * NT + t, N - 1));
         if (a.mask) {
 #pragma unroll
-            for (int u = 0; u < U; ++u) ms[u] = __ldg(a.mask + min(j0 + u * NT + t, N - 1));
+            for (int u = 0; u < U; ++u) ms[u] = ld_in(a.mask + min(j0 + u * NT + t, N - 1));
         } else {
 #pragma unroll
             for (int u = 0; u < U; ++u) ms[u] = 1;
@@ -338,10 +338,10 @@ __device__ __forceinline__ void slice_keys(const DispatchArgs &a, int s, int (&k
     const int N = a.bs * a.top_k, E = a.num_instances, t = threadIdx.x;
     uint32_t sent[kRlRounds];
 #pragma unroll
-    for (int u = 0; u < kRlRounds; ++u) key[u] = __ldg(a.ids + min(s * kRlCopies + u * kRtThreads + t, N - 1));
+    for (int u = 0; u < kRlRounds; ++u) key[u] = ld_in(a.ids + min(s * kRlCopies + u * kRtThreads + t, N - 1));
     if (a.mask) {
 #pragma unroll
-        for (int u = 0; u < kRlRounds; ++u) sent[u] = __ldg(a.mask + min(s * kRlCopies + u * kRtThreads + t, N - 1));
+        for (int u = 0; u < kRlRounds; ++u) sent[u] = ld_in(a.mask + min(s * kRlCopies + u * kRtThreads + t, N - 1));
     } else {
 #pragma unroll
         for (int u = 0; u < kRlRounds; ++u) sent[u] = 1;
@@ -419,7 +419,7 @@ __global__ void __launch_bounds__(kRtThreads) route_place_kernel(DispatchArgs a,
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         const int b = t * 2 + u;
-        v2[u] = b < E ? __ldg(tot + b) : 0;
+        v2[u] = b < E ? ld_in(tot + b) : 0;
         sum += v2[u];
     }
     const int incl = block_inclusive_scan(sum, s_warp);
@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(kRtThreads) route_place_kernel(DispatchArgs a,
         run += v2[u];
     }
     if (s == 0 && t == 0) a.offsets[E] = total;
-    for (int e = t; e < E; e += kRtThreads) s_base[e] = __ldg(tab + (size_t)s * E + e);
+    for (int e = t; e < E; e += kRtThreads) s_base[e] = ld_in(tab + (size_t)s * E + e);
 
     uint32_t *cnt32 = reinterpret_cast<uint32_t *>(s_cnt);
     for (int u = 0; u < kRlRounds; ++u) {
@@ -714,6 +714,198 @@ __device__ __forceinline__ void load_row(const uint16_t *row, int V, uint4 (&xv)
     }
 }
 
+// ------------------------------------------------ instance-major scatter ---
+//
+// Per-instance scales (smooth rows in modes 2 and 3, static scales of shape
+// (E, H) in mode 1) make a copy's codes depend on its destination instance,
+// so every copy is quantized on its own.  Walking a token's K copies would
+// fetch a whole H-float scale row per copy (28 KB at H = 7168, twice the
+// token row it scales).  This kernel walks the instances instead: one block
+// per (instance e, split s) keeps e's scale row in registers for its whole
+// life and streams the token rows of its share of e's bucket through a ring
+// of shared-memory slots, each filled by one bulk asynchronous copy (the
+// block moves a 2H-byte token row per copy instead of a 4H-byte scale row).
+//
+// SELF_ROUTE (at most 8192 copies): the block also finds its bucket itself.
+// A copy's row is its position in (instance, token, k) order, so bucket e
+// starts at the number of sent copies with a smaller instance, and its
+// members are the copies with instance e in (token, k) order.  Each thread
+// counts both over a contiguous segment of the copies; one block scan of the
+// two counts (packed in one word) gives the bucket's offset, its size and
+// every thread's first position, with no histogram.  Otherwise the route
+// kernels have written counts, offsets and src_of_row, and the block reads
+// its bucket from them.
+//
+// Split s of a bucket of cnt copies owns positions [cnt*s/S, cnt*(s+1)/S).
+// A block lists up to kImListCap of its copies at a time (more take several
+// rounds).  Per copy: wait for the token row's slot, xFp32 = x * scale, the
+// row or tile maxima, one block barrier (which also frees the slot for the
+// copy D places ahead), then the codes and the row write.
+
+constexpr int kImListCap = 256;    // copies a block lists at once
+constexpr int kImMaxSlots = 8;     // token rows in flight per block, at most
+constexpr int kImRingBytes = 60 * 1024;  // shared memory for the ring, at most
+
+// Ring slots for rows of H bf16: as many as fit the ring's budget, 2 to 8.
+__host__ __device__ inline int im_slots(int hidden) {
+    const int n = kImRingBytes / (2 * hidden);
+    return n < 2 ? 2 : (n > kImMaxSlots ? kImMaxSlots : n);
+}
+
+template <int MODE, int NT, bool SELF_ROUTE>
+__global__ void __launch_bounds__(NT, 3) dispatch_instance_kernel(DispatchArgs a, int splits, int slots) {
+    constexpr int NW = NT / 32;
+    extern __shared__ __align__(128) uint8_t s_ring[];  // slots x 2H bytes
+    __shared__ __align__(8) uint64_t s_full[kImMaxSlots];
+    __shared__ int s_list[kImListCap];
+    __shared__ int s_warp[32];
+    __shared__ float s_red[2][NW];
+    __shared__ int s_bad;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int E = a.num_instances, e = blockIdx.x % E, s = blockIdx.x / E;
+    const int H = a.hidden, V = H >> 3, K = a.top_k, N = a.bs * K;
+    const uint32_t row_bytes = 2u * (uint32_t)H;  // a multiple of 32 (H % 16 == 0)
+
+    if (t == 0) {
+        for (int d = 0; d < slots; ++d) mbar_init(&s_full[d], 1);
+        s_bad = 0;
+    }
+    __syncthreads();
+    pdl_wait();  // the ids and x may come from the kernel before the call, the tables from the route kernels
+
+    // e's scale row, this thread's 4 vectors of 8 (zeros past the row's end)
+    uint64_t sc[kDpVecs][4];
+#pragma unroll
+    for (int q = 0; q < kDpVecs; ++q) {
+        const int p = t + q * NT;
+        float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+        if (p < V) {
+            const float4 *src = reinterpret_cast<const float4 *>(a.smooth + (size_t)e * H + p * 8);
+            s0 = ld_in(src);
+            s1 = ld_in(src + 1);
+        }
+        sc[q][0] = f2_pack(s0.x, s0.y);
+        sc[q][1] = f2_pack(s0.z, s0.w);
+        sc[q][2] = f2_pack(s1.x, s1.y);
+        sc[q][3] = f2_pack(s1.z, s1.w);
+    }
+
+    // the bucket: its offset off, its size cnt; this thread's copies [j0, j1)
+    // and the position of its first member pos0 (SELF_ROUTE)
+    int off, cnt, j0 = 0, j1 = 0, pos0 = 0;
+    if constexpr (SELF_ROUTE) {
+        const int seg = (N + NT - 1) / NT;
+        j0 = min(N, t * seg);
+        j1 = min(N, j0 + seg);
+        int eq = 0, lt = 0;
+        for (int j = j0; j < j1; ++j) {
+            const int key = copy_key(a, j);
+            eq += key == e;
+            lt += key >= 0 && key < e;
+            if (blockIdx.x == 0 && key < 0) {  // block 0 answers for the copies no bucket takes
+                a.expand_idx[j] = -1;
+                if (key == -2) s_bad = 1;
+            }
+        }
+        const int packed = (lt << 16) | eq;  // both counts <= 8192 < 2^16
+        const int incl = block_inclusive_scan(packed, s_warp);
+        const int total = s_warp[NW - 1];
+        off = total >> 16;
+        cnt = total & 0xffff;
+        pos0 = (incl - packed) & 0xffff;
+        if (t == 0 && s == 0) {
+            a.counts[e] = cnt;
+            a.offsets[e] = off;
+            if (e == E - 1) a.offsets[E] = off + cnt;
+        }
+        if (t == 0 && s_bad) raise_error(a.err, kDevBadId);
+    } else {
+        off = a.offsets[e];  // written by the route kernels
+        cnt = a.offsets[e + 1] - off;
+    }
+    const int lo = (int)((long long)cnt * s / splits), hi = (int)((long long)cnt * (s + 1) / splits);
+
+    auto issue = [&](int c, int cg) {  // thread 0: copy c of the round into slot cg % slots
+        const int tok = (int)div_by_magic((uint32_t)s_list[c], a.k_magic);
+        const int d = cg % slots;
+        mbar_arrive_expect_tx(&s_full[d], row_bytes);
+        bulk_copy_g2s(s_ring + (size_t)d * row_bytes, a.x + (size_t)tok * H, row_bytes, &s_full[d]);
+    };
+
+    int cg0 = 0;  // copies through the ring so far: slot = cg % slots, phase = (cg / slots) & 1
+    for (int w0 = lo; w0 < hi; w0 += kImListCap) {
+        const int m = min(hi - w0, kImListCap);
+        __syncthreads();  // the previous round's list is no longer read
+        if constexpr (SELF_ROUTE) {
+            int p = pos0;  // this thread's members of the bucket, in order
+            for (int j = j0; j < j1; ++j) {
+                if (copy_key(a, j) != e) continue;
+                if (p >= w0 && p < w0 + m) {
+                    s_list[p - w0] = j;
+                    a.expand_idx[j] = off + p;
+                    a.src_of_row[off + p] = j;
+                }
+                ++p;
+            }
+        } else {
+            for (int c = t; c < m; c += NT) s_list[c] = a.src_of_row[off + w0 + c];
+        }
+        __syncthreads();
+        if (t == 0) {
+            fence_proxy_async_smem();  // the slots were last read by the previous round
+            for (int c = 0; c < min(slots, m); ++c) issue(c, cg0 + c);
+        }
+
+        for (int c = 0; c < m; ++c) {
+            const int cg = cg0 + c, d = cg % slots;
+            const bool landed = mbar_wait_bounded(&s_full[d], (uint32_t)(cg / slots) & 1u);
+            const uint4 *xr = reinterpret_cast<const uint4 *>(s_ring + (size_t)d * row_bytes);
+            uint64_t xf[kDpVecs][4];
+#pragma unroll
+            for (int q = 0; q < kDpVecs; ++q) {  // xFp32 = x * scale (0 past the row's end)
+                const int p = t + q * NT;
+                uint64_t f[4];
+                vec_to_f2(p < V ? xr[p] : make_uint4(0, 0, 0, 0), f);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) xf[q][u] = f2_mul(f[u], sc[q][u]);
+            }
+            if constexpr (MODE == 2) {
+                const float mx = warp_max(abs_max_vecs(xf));
+                if (lane == 0) s_red[c & 1][w] = mx;
+            }
+            // every thread has read the slot (and published its partial max);
+            // a row that never landed stops the block, the same verdict in
+            // every thread, once a second bounded wait has given the copy in
+            // flight its chance to finish
+            if (__syncthreads_or(!landed)) {
+                if (t == 0) {  // copies c .. min(m, c + slots) - 1 were issued
+                    raise_error(a.err, kDevTimeout);
+                    for (int q = 0; q < slots && c + q < m; ++q)
+                        mbar_wait_bounded(&s_full[(cg + q) % slots], (uint32_t)((cg + q) / slots) & 1u);
+                }
+                return;
+            }
+            if (t == 0 && c + slots < m) {
+                fence_proxy_async_smem();
+                issue(c + slots, cg + slots);
+            }
+            if (w0 + c + 1 == hi) pdl_launch_dependents();  // this block's last copy
+            uint2 qv[kDpVecs];
+            float seg[kDpVecs] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float row_scale = 0.0f;
+            if constexpr (MODE == 2) {
+                const float dyn = __fdiv_rn(127.0f, max_partials<NW>(s_red[c & 1]));  // +inf when the max is 0
+                row_scale = __frcp_rn(dyn);                                          // or 127 / max overflows
+                int8_vecs(xf, dyn, qv);
+            } else {
+                quantize_local<MODE, NT>(xf, V, qv, seg);
+            }
+            write_row<MODE, NT>(a, off + w0 + c, V, qv, seg, row_scale);
+        }
+        cg0 += m;
+    }
+}
+
 // --------------------------------------------------------- token kernel ---
 
 // FUSED: the block routes its own copies (block_route, small calls) instead
@@ -749,7 +941,7 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
             for (int q = 0; q < kDpVecs; ++q) vec_to_f2(xv[q], xf[q]);
             if constexpr (MODE == 1) {  // xFp32 = x * scales: one coefficient, or one per column
                 if (a.scales_len == 1) {
-                    const float c = __ldg(a.smooth);
+                    const float c = ld_in(a.smooth);
                     const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
                     for (int q = 0; q < kDpVecs; ++q)
@@ -760,8 +952,8 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
                     for (int q = 0; q < kDpVecs; ++q) {
                         const int p = t + q * NT;
                         if (p >= V) continue;
-                        const float4 s0 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8));
-                        const float4 s1 = __ldg(reinterpret_cast<const float4 *>(a.smooth + p * 8) + 1);
+                        const float4 s0 = ld_in(reinterpret_cast<const float4 *>(a.smooth + p * 8));
+                        const float4 s1 = ld_in(reinterpret_cast<const float4 *>(a.smooth + p * 8) + 1);
                         xf[q][0] = f2_mul(xf[q][0], f2_pack(s0.x, s0.y));
                         xf[q][1] = f2_mul(xf[q][1], f2_pack(s0.z, s0.w));
                         xf[q][2] = f2_mul(xf[q][2], f2_pack(s1.x, s1.y));

@@ -477,9 +477,9 @@ __global__ void __launch_bounds__(kGmMxThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int ch = min(n0 + 32 * c + lane, a.out_dim - 1);
-                fa[c] = __ldg(reinterpret_cast<const uint32_t *>(a.wsf + ((size_t)slot.x * a.out_dim + ch) * B) + k);
+                fa[c] = ld_in(reinterpret_cast<const uint32_t *>(a.wsf + ((size_t)slot.x * a.out_dim + ch) * B) + k);
                 const int r = min(32 * c + lane, nr - 1);
-                fb[c] = __ldg(reinterpret_cast<const uint32_t *>(a.xsf + (size_t)(slot.y + r) * B) + k);
+                fb[c] = ld_in(reinterpret_cast<const uint32_t *>(a.xsf + (size_t)(slot.y + r) * B) + k);
             }
         };
         const uint32_t quarter = (uint32_t)(warp * 32) << 16;

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
         bulk_copy_g2s(const_cast<int32_t *>(s_tab), a.table, tab_bytes, &s_tab_bar);
     }
     if (a.table_mode == 1)
-        for (int q = t; q < E * F; q += kUeThreads) const_cast<int32_t *>(s_tab)[q] = __ldg(a.table + q);
+        for (int q = t; q < E * F; q += kUeThreads) const_cast<int32_t *>(s_tab)[q] = ld_in(a.table + q);
     const int items = a.bs * a.top_k;
     const int base = blockIdx.x * kUeThreads * kUeItems;  // this block's first copy
     // Every load is unconditional (indices clamped into range), so all of
@@ -106,20 +106,20 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     float ps[kUeItems];
     bool pa[kUeItems];
 #pragma unroll
-    for (int u = 0; u < kUeItems; ++u) pe[u] = __ldg(a.expert_ids + min(base + t + u * kUeThreads, items - 1));
+    for (int u = 0; u < kUeItems; ++u) pe[u] = ld_in(a.expert_ids + min(base + t + u * kUeThreads, items - 1));
 #pragma unroll
     for (int u = 0; u < kUeItems; ++u) ps[u] = 0.0f;
     if (a.expert_scales) {
 #pragma unroll
         for (int u = 0; u < kUeItems; ++u)
-            ps[u] = __ldg(a.expert_scales + min(base + t + u * kUeThreads, items - 1));
+            ps[u] = ld_in(a.expert_scales + min(base + t + u * kUeThreads, items - 1));
     }
 #pragma unroll
     for (int u = 0; u < kUeItems; ++u) pa[u] = true;
     if (a.active_mask) {
 #pragma unroll
         for (int u = 0; u < kUeItems; ++u)
-            pa[u] = __ldg(a.active_mask +
+            pa[u] = ld_in(a.active_mask +
                           div_by_magic((uint32_t)min(base + t + u * kUeThreads, items - 1), a.k_magic)) != 0;
     }
 #pragma unroll
