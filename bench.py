@@ -81,15 +81,13 @@ def algorithmic_bytes(w, n, x_out=False, rstd=False):
 
 def kernels_per_step(w):
     """Kernels of this library one step launches: update_expert, the
-    dispatch's kernels, the combine.  Per-instance scales take the
-    instance-major kernel, which routes its own copies up to 8192 copies;
-    otherwise up to 1024 copies the scatter blocks route themselves, up to
-    8192 one route kernel runs first, and beyond that the three-pass route."""
+    dispatch's kernels, the combine.  Up to 1024 copies the scatter blocks
+    route themselves, up to 8192 one route kernel runs first, and beyond that
+    the three-pass route."""
     copies = w.bs * w.top_k
-    per_instance = w.smooth is not None and w.smooth.size > w.hidden
     if copies > 8192:
         disp = 4
-    elif per_instance or copies <= 1024:
+    elif copies <= 1024:
         disp = 1
     else:
         disp = 2
@@ -100,7 +98,7 @@ def kernels_per_step(w):
 # these files are unchanged.
 KERNEL_SOURCES = {
     "combine_token_kernel": ("combine.cuh", "common.cuh"),
-    "dispatch_instance_kernel": ("dispatch.cuh", "common.cuh"),
+    "dispatch_token_smooth_kernel": ("dispatch.cuh", "common.cuh"),
     "dispatch_token_kernel": ("dispatch.cuh", "common.cuh"),
     "gmm_kernel": ("grouped_matmul.cuh", "common.cuh"),
     "gmm_mx_kernel": ("grouped_matmul.cuh", "common.cuh"),
@@ -500,7 +498,7 @@ def run_b200(args, rank, world, local_rank):
 
     peak, peak_kind = measured_peak()
     per_instance = w.smooth is not None and w.smooth.size > w.hidden
-    disp_name = "dispatch_instance_kernel" if per_instance else "dispatch_token_kernel"
+    disp_name = "dispatch_token_smooth_kernel" if per_instance else "dispatch_token_kernel"
 
     def roof(kernel, nbytes, t_ms, timing, traffic_key):
         a = nbytes / (t_ms * 1e-3) / 1e9

@@ -51,27 +51,43 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
         : "memory");
 }
 
+// A waiting thread asks to be suspended until the phase completes, for at
+// most this long per poll (ns), instead of spinning on the barrier and
+// taking issue slots from the warps that have work.
+constexpr uint32_t kWaitHintNs = 1u << 20;  // about a millisecond
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
+        : "r"(smem_u32(bar)), "r"(phase), "r"(kWaitHintNs)
         : "memory");
     return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
+// How long any bounded wait in this library waits before it gives up.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // one second
 
-// Wait for phase `phase` of an mbarrier, giving up after a bounded number of
-// polls (each poll may itself suspend for a while).  Returns false on
-// timeout, so a copy that never lands cannot hang the GPU.
+// Wait for phase `phase` of an mbarrier, giving up after kWaitLimitNs of
+// device time.  Each poll suspends the thread until the phase completes (or
+// the hint runs out), so a wait costs a poll or two, not a spin.  Returns
+// false on timeout, so a copy that never lands cannot hang the GPU.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase) {
-    for (uint32_t it = 0; it < (1u << 22); ++it)
+    if (mbar_try_wait(bar, phase)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
         if (mbar_try_wait(bar, phase)) return true;
-    return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
 }
 
 // Programmatic dependent launch (PTX griddepcontrol, sm_90 and later).  A
@@ -115,9 +131,11 @@ __device__ __forceinline__ void st_v4(void *p, uint4 v) { *reinterpret_cast<uint
 
 // --- packed fp32x2 arithmetic (sm_100): two independent IEEE binary32
 // operations, each rounded to nearest even, in one instruction.  A packed
-// multiply whose result feeds a packed add may be contracted into a fused
-// multiply-add; where the product's own rounding matters, multiply with the
-// scalar __fmul_rn instead. ---
+// multiply whose result feeds a packed add is contracted into a fused
+// multiply-add by ptxas, even with --fmad=false and explicit .rn rounding
+// (measured: codes off by one at rounding ties); where the product's own
+// rounding matters, multiply with the scalar __fmul_rn instead, which is
+// never contracted. ---
 
 // Pairs are built and split with register-pair moves, which cost no
 // instruction once registers are allocated.
@@ -141,6 +159,12 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
+}
+// max of three (sm_100a's three-input max; a NaN operand is ignored, as fmaxf ignores it).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 // A bf16 pair (one 32-bit word, element 0 in the low half) as an fp32 pair.

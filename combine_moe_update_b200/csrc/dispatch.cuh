@@ -498,17 +498,21 @@ __host__ __device__ inline int dp_threads(int V) {
 // in [-127, 127] and the clamp to that range is never active.
 //
 // The product must be rounded to fp32 on its own before the add (the page's
-// quantOut = CastToInt8(xFp32 * dynamicScales) rounds it).  Scalar
-// round-to-nearest intrinsics are never contracted into a fused multiply-add
-// (which would skip that rounding and break ties such as a product that
-// rounds to exactly 63.5), and unlike packed pairs they need no register
-// pairing moves.
+// quantOut = CastToInt8(xFp32 * dynamicScales) rounds it); a fused
+// multiply-add would skip that rounding and break ties such as a product
+// that rounds to exactly 63.5.  Scalar round-to-nearest intrinsics are never
+// contracted (packed fp32x2 pairs are, even with contraction switched off),
+// and unlike packed pairs they need no register pairing moves.
+constexpr float kRintMagic = 12582912.0f;  // 1.5 * 2^23
+
 __device__ __forceinline__ uint2 int8x8(const uint64_t (&v)[4], float dyn) {
+    const uint64_t d2 = f2_pack(dyn, dyn);
     uint32_t b[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        b[2 * q] = __float_as_uint(__fadd_rn(__fmul_rn(f2_lo(v[q]), dyn), 12582912.0f));
-        b[2 * q + 1] = __float_as_uint(__fadd_rn(__fmul_rn(f2_hi(v[q]), dyn), 12582912.0f));
+        const uint64_t p = f2_mul(v[q], d2);  // both products rounded (packed multiply)
+        b[2 * q] = __float_as_uint(__fadd_rn(f2_lo(p), kRintMagic));
+        b[2 * q + 1] = __float_as_uint(__fadd_rn(f2_hi(p), kRintMagic));
     }
     const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
@@ -526,8 +530,8 @@ __device__ __forceinline__ uint2 int8x8_static(const uint64_t (&v)[4]) {
         const float lo = f2_lo(v[q]), hi = f2_hi(v[q]);
         const float cl = lo != lo ? 0.0f : fminf(fmaxf(lo, -128.0f), 127.0f);
         const float ch = hi != hi ? 0.0f : fminf(fmaxf(hi, -128.0f), 127.0f);
-        b[2 * q] = __float_as_uint(__fadd_rn(cl, 12582912.0f));
-        b[2 * q + 1] = __float_as_uint(__fadd_rn(ch, 12582912.0f));
+        b[2 * q] = __float_as_uint(__fadd_rn(cl, kRintMagic));
+        b[2 * q + 1] = __float_as_uint(__fadd_rn(ch, kRintMagic));
     }
     const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
@@ -558,18 +562,17 @@ __device__ __forceinline__ void int8_vecs(const uint64_t (&v)[kDpVecs][4], float
     }
 }
 
-// max |v| of 8 values, as a balanced tree (3 dependent steps, not 8).
+// max |v| of 8 values with three-input maxima (4 steps, 2 dependent).
 __device__ __forceinline__ float abs_max8(const uint64_t (&v)[4]) {
-    float m[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) m[q] = fmaxf(fabsf(f2_lo(v[q])), fabsf(f2_hi(v[q])));
-    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+    const float m0 = fmax3(fabsf(f2_lo(v[0])), fabsf(f2_hi(v[0])), fabsf(f2_lo(v[1])));
+    const float m1 = fmax3(fabsf(f2_hi(v[1])), fabsf(f2_lo(v[2])), fabsf(f2_hi(v[2])));
+    return fmax3(m0, m1, fmaxf(fabsf(f2_lo(v[3])), fabsf(f2_hi(v[3]))));
 }
 
 // max |v| over this thread's vectors (vectors past the row's end hold 0).
 __device__ __forceinline__ float abs_max_vecs(const uint64_t (&v)[kDpVecs][4]) {
     static_assert(kDpVecs == 4, "the tree below covers four vectors");
-    return fmaxf(fmaxf(abs_max8(v[0]), abs_max8(v[1])), fmaxf(abs_max8(v[2]), abs_max8(v[3])));
+    return fmaxf(fmax3(abs_max8(v[0]), abs_max8(v[1]), abs_max8(v[2])), abs_max8(v[3]));
 }
 
 // 8 bf16 -> 4 fp32 pairs (exact).
@@ -711,198 +714,6 @@ __device__ __forceinline__ void load_row(const uint16_t *row, int V, uint4 (&xv)
     for (int q = 0; q < kDpVecs; ++q) {
         const int p = threadIdx.x + q * NT;
         xv[q] = p < V ? ld_stream(row + p * 8) : make_uint4(0, 0, 0, 0);
-    }
-}
-
-// ------------------------------------------------ instance-major scatter ---
-//
-// Per-instance scales (smooth rows in modes 2 and 3, static scales of shape
-// (E, H) in mode 1) make a copy's codes depend on its destination instance,
-// so every copy is quantized on its own.  Walking a token's K copies would
-// fetch a whole H-float scale row per copy (28 KB at H = 7168, twice the
-// token row it scales).  This kernel walks the instances instead: one block
-// per (instance e, split s) keeps e's scale row in registers for its whole
-// life and streams the token rows of its share of e's bucket through a ring
-// of shared-memory slots, each filled by one bulk asynchronous copy (the
-// block moves a 2H-byte token row per copy instead of a 4H-byte scale row).
-//
-// SELF_ROUTE (at most 8192 copies): the block also finds its bucket itself.
-// A copy's row is its position in (instance, token, k) order, so bucket e
-// starts at the number of sent copies with a smaller instance, and its
-// members are the copies with instance e in (token, k) order.  Each thread
-// counts both over a contiguous segment of the copies; one block scan of the
-// two counts (packed in one word) gives the bucket's offset, its size and
-// every thread's first position, with no histogram.  Otherwise the route
-// kernels have written counts, offsets and src_of_row, and the block reads
-// its bucket from them.
-//
-// Split s of a bucket of cnt copies owns positions [cnt*s/S, cnt*(s+1)/S).
-// A block lists up to kImListCap of its copies at a time (more take several
-// rounds).  Per copy: wait for the token row's slot, xFp32 = x * scale, the
-// row or tile maxima, one block barrier (which also frees the slot for the
-// copy D places ahead), then the codes and the row write.
-
-constexpr int kImListCap = 256;    // copies a block lists at once
-constexpr int kImMaxSlots = 8;     // token rows in flight per block, at most
-constexpr int kImRingBytes = 60 * 1024;  // shared memory for the ring, at most
-
-// Ring slots for rows of H bf16: as many as fit the ring's budget, 2 to 8.
-__host__ __device__ inline int im_slots(int hidden) {
-    const int n = kImRingBytes / (2 * hidden);
-    return n < 2 ? 2 : (n > kImMaxSlots ? kImMaxSlots : n);
-}
-
-template <int MODE, int NT, bool SELF_ROUTE>
-__global__ void __launch_bounds__(NT, 3) dispatch_instance_kernel(DispatchArgs a, int splits, int slots) {
-    constexpr int NW = NT / 32;
-    extern __shared__ __align__(128) uint8_t s_ring[];  // slots x 2H bytes
-    __shared__ __align__(8) uint64_t s_full[kImMaxSlots];
-    __shared__ int s_list[kImListCap];
-    __shared__ int s_warp[32];
-    __shared__ float s_red[2][NW];
-    __shared__ int s_bad;
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    const int E = a.num_instances, e = blockIdx.x % E, s = blockIdx.x / E;
-    const int H = a.hidden, V = H >> 3, K = a.top_k, N = a.bs * K;
-    const uint32_t row_bytes = 2u * (uint32_t)H;  // a multiple of 32 (H % 16 == 0)
-
-    if (t == 0) {
-        for (int d = 0; d < slots; ++d) mbar_init(&s_full[d], 1);
-        s_bad = 0;
-    }
-    __syncthreads();
-    pdl_wait();  // the ids and x may come from the kernel before the call, the tables from the route kernels
-
-    // e's scale row, this thread's 4 vectors of 8 (zeros past the row's end)
-    uint64_t sc[kDpVecs][4];
-#pragma unroll
-    for (int q = 0; q < kDpVecs; ++q) {
-        const int p = t + q * NT;
-        float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
-        if (p < V) {
-            const float4 *src = reinterpret_cast<const float4 *>(a.smooth + (size_t)e * H + p * 8);
-            s0 = ld_in(src);
-            s1 = ld_in(src + 1);
-        }
-        sc[q][0] = f2_pack(s0.x, s0.y);
-        sc[q][1] = f2_pack(s0.z, s0.w);
-        sc[q][2] = f2_pack(s1.x, s1.y);
-        sc[q][3] = f2_pack(s1.z, s1.w);
-    }
-
-    // the bucket: its offset off, its size cnt; this thread's copies [j0, j1)
-    // and the position of its first member pos0 (SELF_ROUTE)
-    int off, cnt, j0 = 0, j1 = 0, pos0 = 0;
-    if constexpr (SELF_ROUTE) {
-        const int seg = (N + NT - 1) / NT;
-        j0 = min(N, t * seg);
-        j1 = min(N, j0 + seg);
-        int eq = 0, lt = 0;
-        for (int j = j0; j < j1; ++j) {
-            const int key = copy_key(a, j);
-            eq += key == e;
-            lt += key >= 0 && key < e;
-            if (blockIdx.x == 0 && key < 0) {  // block 0 answers for the copies no bucket takes
-                a.expand_idx[j] = -1;
-                if (key == -2) s_bad = 1;
-            }
-        }
-        const int packed = (lt << 16) | eq;  // both counts <= 8192 < 2^16
-        const int incl = block_inclusive_scan(packed, s_warp);
-        const int total = s_warp[NW - 1];
-        off = total >> 16;
-        cnt = total & 0xffff;
-        pos0 = (incl - packed) & 0xffff;
-        if (t == 0 && s == 0) {
-            a.counts[e] = cnt;
-            a.offsets[e] = off;
-            if (e == E - 1) a.offsets[E] = off + cnt;
-        }
-        if (t == 0 && s_bad) raise_error(a.err, kDevBadId);
-    } else {
-        off = a.offsets[e];  // written by the route kernels
-        cnt = a.offsets[e + 1] - off;
-    }
-    const int lo = (int)((long long)cnt * s / splits), hi = (int)((long long)cnt * (s + 1) / splits);
-
-    auto issue = [&](int c, int cg) {  // thread 0: copy c of the round into slot cg % slots
-        const int tok = (int)div_by_magic((uint32_t)s_list[c], a.k_magic);
-        const int d = cg % slots;
-        mbar_arrive_expect_tx(&s_full[d], row_bytes);
-        bulk_copy_g2s(s_ring + (size_t)d * row_bytes, a.x + (size_t)tok * H, row_bytes, &s_full[d]);
-    };
-
-    int cg0 = 0;  // copies through the ring so far: slot = cg % slots, phase = (cg / slots) & 1
-    for (int w0 = lo; w0 < hi; w0 += kImListCap) {
-        const int m = min(hi - w0, kImListCap);
-        __syncthreads();  // the previous round's list is no longer read
-        if constexpr (SELF_ROUTE) {
-            int p = pos0;  // this thread's members of the bucket, in order
-            for (int j = j0; j < j1; ++j) {
-                if (copy_key(a, j) != e) continue;
-                if (p >= w0 && p < w0 + m) {
-                    s_list[p - w0] = j;
-                    a.expand_idx[j] = off + p;
-                    a.src_of_row[off + p] = j;
-                }
-                ++p;
-            }
-        } else {
-            for (int c = t; c < m; c += NT) s_list[c] = a.src_of_row[off + w0 + c];
-        }
-        __syncthreads();
-        if (t == 0) {
-            fence_proxy_async_smem();  // the slots were last read by the previous round
-            for (int c = 0; c < min(slots, m); ++c) issue(c, cg0 + c);
-        }
-
-        for (int c = 0; c < m; ++c) {
-            const int cg = cg0 + c, d = cg % slots;
-            const bool landed = mbar_wait_bounded(&s_full[d], (uint32_t)(cg / slots) & 1u);
-            const uint4 *xr = reinterpret_cast<const uint4 *>(s_ring + (size_t)d * row_bytes);
-            uint64_t xf[kDpVecs][4];
-#pragma unroll
-            for (int q = 0; q < kDpVecs; ++q) {  // xFp32 = x * scale (0 past the row's end)
-                const int p = t + q * NT;
-                uint64_t f[4];
-                vec_to_f2(p < V ? xr[p] : make_uint4(0, 0, 0, 0), f);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) xf[q][u] = f2_mul(f[u], sc[q][u]);
-            }
-            if constexpr (MODE == 2) {
-                const float mx = warp_max(abs_max_vecs(xf));
-                if (lane == 0) s_red[c & 1][w] = mx;
-            }
-            // every thread has read the slot (and published its partial max);
-            // a row that never landed stops the block, the same verdict in
-            // every thread, once a second bounded wait has given the copy in
-            // flight its chance to finish
-            if (__syncthreads_or(!landed)) {
-                if (t == 0) {  // copies c .. min(m, c + slots) - 1 were issued
-                    raise_error(a.err, kDevTimeout);
-                    for (int q = 0; q < slots && c + q < m; ++q)
-                        mbar_wait_bounded(&s_full[(cg + q) % slots], (uint32_t)((cg + q) / slots) & 1u);
-                }
-                return;
-            }
-            if (t == 0 && c + slots < m) {
-                fence_proxy_async_smem();
-                issue(c + slots, cg + slots);
-            }
-            if (w0 + c + 1 == hi) pdl_launch_dependents();  // this block's last copy
-            uint2 qv[kDpVecs];
-            float seg[kDpVecs] = {0.0f, 0.0f, 0.0f, 0.0f};
-            float row_scale = 0.0f;
-            if constexpr (MODE == 2) {
-                const float dyn = __fdiv_rn(127.0f, max_partials<NW>(s_red[c & 1]));  // +inf when the max is 0
-                row_scale = __frcp_rn(dyn);                                          // or 127 / max overflows
-                int8_vecs(xf, dyn, qv);
-            } else {
-                quantize_local<MODE, NT>(xf, V, qv, seg);
-            }
-            write_row<MODE, NT>(a, off + w0 + c, V, qv, seg, row_scale);
-        }
-        cg0 += m;
     }
 }
 

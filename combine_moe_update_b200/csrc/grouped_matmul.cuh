@@ -209,13 +209,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 
 // Bounded wait with a short sleep between polls, for threads that idle
-// through the main loop (about a second at most).
+// through the main loop (kWaitLimitNs of device time at most).
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t phase) {
-    for (uint32_t it = 0; it < (1u << 24); ++it) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
         if (mbar_try_wait(bar, phase)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
         __nanosleep(64);
     }
-    return false;
 }
 
 // --- the int8 matmul: grid (ceil(N / 128), max_slots), 128 threads ---

@@ -6,7 +6,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -232,49 +231,6 @@ struct TokenSmoothLaunch {
     }
 };
 
-// Streaming multiprocessors of the current device (cached per device).
-int device_sms() {
-    static std::mutex mu;
-    static int sms[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    std::lock_guard<std::mutex> lock(mu);
-    if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return 148;
-    return sms[dev];
-}
-
-// Splits per instance of the instance-major scatter: about one wave of
-// blocks (three per SM) over the E instances, with at least two copies per
-// split on average.
-int instance_splits(int copies, int num_instances) {
-    const int target = 3 * device_sms();
-    int sp = (target + num_instances / 2) / num_instances;
-    sp = std::min(sp, copies / (2 * num_instances));
-    return std::max(1, std::min(8, sp));
-}
-
-template <int MODE, int NT>
-struct InstanceLaunch {
-    template <bool SELF_ROUTE>
-    static cudaError_t go_(const moe::DispatchArgs &a, cudaStream_t s) {
-        auto kernel = moe::dispatch_instance_kernel<MODE, NT, SELF_ROUTE>;
-        const int slots = moe::im_slots(a.hidden);
-        const size_t smem = (size_t)slots * 2 * a.hidden;
-        if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
-        const int splits = instance_splits(a.bs * a.top_k, a.num_instances);
-        return launch(kernel, a.num_instances * splits, NT, smem, s, a, splits, slots);
-    }
-    static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
-        return a.bs * a.top_k <= kRouteSinglePassMax ? go_<true>(a, s) : go_<false>(a, s);
-    }
-};
-
-template <int MODE>
-cudaError_t launch_dispatch_instance(const moe::DispatchArgs &a, cudaStream_t s) {
-    return launch_by_threads<MODE, InstanceLaunch>(a, s);
-}
-
 template <int MODE>
 cudaError_t launch_dispatch_token(const moe::DispatchArgs &a, cudaStream_t s) {
     return launch_by_threads<MODE, TokenLaunch>(a, s);
@@ -450,14 +406,7 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     cudaStream_t s = as_stream(cuda_stream);
 
     const int copies = a.bs * p->top_k;
-    // scales that depend on the destination instance (a row per instance) need
-    // a quantization per copy: the instance-major kernel, which routes its
-    // own copies up to kRouteSinglePassMax copies; one coefficient or one per
-    // column is per token
-    const bool per_instance = smooth_scales && p->scales_len > p->hidden;
-    if (per_instance && copies <= kRouteSinglePassMax) {
-        // no route kernel
-    } else if (copies <= moe::kFusedRouteMax) {
+    if (copies <= moe::kFusedRouteMax) {
         // the scatter blocks route their own copies (no route kernel)
     } else if (copies <= kRouteSinglePassMax) {
         const int slices = moe::route_slices(copies);
@@ -478,11 +427,14 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
             return MOE_ERR_CUDA;
     }
     cudaError_t e = cudaSuccess;
+    // scales that depend on the destination instance (a row per instance) need
+    // the per-copy kernel; one coefficient or one per column is per token
+    const bool per_instance = smooth_scales && p->scales_len > p->hidden;
     if (per_instance) {
         switch (mode) {
-            case 1: e = launch_dispatch_instance<1>(a, s); break;
-            case 2: e = launch_dispatch_instance<2>(a, s); break;
-            case 3: e = launch_dispatch_instance<3>(a, s); break;
+            case 1: e = launch_dispatch_token_smooth<1>(a, s); break;
+            case 2: e = launch_dispatch_token_smooth<2>(a, s); break;
+            case 3: e = launch_dispatch_token_smooth<3>(a, s); break;
         }
     } else {
         switch (mode) {
