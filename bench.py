@@ -687,6 +687,76 @@ def run_b200_layer_stack(args, rank, world, local_rank):
     return out, st
 
 
+def run_b200_ep(args, rank, world, local_rank):
+    """Expert parallelism across the GPUs of the job: GPU g owns instances
+    [g E / N, (g + 1) E / N) and dispatches its own batch; every step is
+    update + dispatch of its tokens, the gather of every GPU's counts, the
+    plan and push of its rows into their owners' receive buffers (peer
+    memory), a barrier, the expert step (the owner's output buffer, resident),
+    a barrier, the pull of its rows' outputs and combine+Add+RMSNorm.  Timed
+    with events on each rank, max over ranks."""
+    import numpy as np
+    import torch
+    from combine_moe_update_b200 import binding as B
+    from combine_moe_update_b200 import ep as EP
+    from combine_moe_update_b200 import inputs as gen
+
+    torch.cuda.set_device(local_rank)
+    w = gen.make(args.workload, seed=None if rank == 0 else 1000 + rank)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    bf = lambda a: dev(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16)
+    grp = EP.ProcessGroupEP(bs=w.bs, hidden=w.hidden, top_k=w.top_k, num_instances=w.num_instances,
+                            ep_world_size=w.ep_world_size, quant_mode=w.quant_mode)
+    r = grp.r
+    table, smooth, gamma = dev(w.table), None if w.smooth is None else dev(w.smooth), bf(w.gamma)
+    ids, scales, x, residual = dev(w.expert_ids), dev(w.expert_scales), bf(w.x), bf(w.residual)
+    shared = None if w.shared_x is None else bf(w.shared_x)
+    r.expert_out.copy_(bf(np.resize(w.expert_out, (r.cap, w.hidden))))  # the expert step's output, resident
+    out = dict(y=torch.empty_like(x), x_out=None, rstd=None)
+
+    def step():
+        grp.dispatch(expert_ids=ids, table=table, x=x, expert_scales=scales, smooth=smooth,
+                     prune_threshold=w.prune_threshold)
+        grp.combine(expert_scales=scales, residual=residual, gamma=gamma, norm_eps=w.norm_eps, shared_x=shared,
+                    out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert r.device_errors() == 0, "device error during warm-up"
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record()
+        for _ in range(K):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    (t_step,) = reduce_over_ranks([e0.elapsed_time(e1) / K], "max")
+    recv = r.received()
+    assert r.device_errors() == 0, "device error during the timed steps"
+    grp.close()
+    n_kernels = kernels_per_step(w) + 3  # + plan, push, pull
+    return {
+        "metric": METRIC, "value": round(world * w.bs / (t_step * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": {0: "bf16", 1: "int8", 2: "int8", 3: "int8", 4: "fp8e4m3"}[w.quant_mode] + "+fp32",
+        "data": "synthetic (seeded; pages' shapes; every GPU its own batch)",
+        "config": {"workload": args.workload, "bs_per_gpu": w.bs, "hidden": w.hidden, "top_k": w.top_k,
+                   "num_instances": w.num_instances, "ep_world_size_simulated": w.ep_world_size,
+                   "quant_mode": w.quant_mode, "parallelism": f"ep{world}: instances split over the GPUs",
+                   "rows_received_rank0": recv,
+                   "l2": "not flushed: each step's exchange and gathers touch more than L2 across the group"},
+        "e2e": None,
+        "gpu_launches": n_kernels * K,
+        "timing": "CUDA events around K eager steps (each with two barriers), max over ranks",
+        "clocks": clk.summary(),
+    }, w
+
+
 def oracle_stack(orc, st, lo, hi):
     """The oracle's 32 chained layers on tokens [lo, hi) of the stack."""
     x, r = st.x0[lo:hi], st.residual0[lo:hi]
@@ -1152,6 +1222,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism across the job's GPUs (real exchange through peer memory) "
+                         "instead of independent replicas")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1165,9 +1238,23 @@ def main(argv=None):
 
     import datetime
     import torch.distributed as dist
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if world > 1 or args.ep:
+        if world == 1:  # a one-GPU group, so --ep runs the same code path alone
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29511")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
+        import torch
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
     try:
+        if args.ep:
+            out, w = run_b200_ep(args, rank, world, local_rank)
+            if rank == 0:
+                out["cpu_baseline"] = None
+                print(json.dumps(out), flush=True)
+            return 0
         if args.workload == "layer_stack":
             out, st = run_b200_layer_stack(args, rank, world, local_rank)
             if rank == 0:
@@ -1179,7 +1266,7 @@ def main(argv=None):
             out["cpu_baseline"] = cpu_baseline(w, args.cpu_baseline_seconds) if world == 1 else None
             print(json.dumps(out), flush=True)
     finally:
-        if world > 1:
+        if dist.is_initialized():
             dist.destroy_process_group()
     return 0
 

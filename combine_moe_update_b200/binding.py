@@ -44,6 +44,12 @@ class CombineParams(ctypes.Structure):
                 ("expand_rows", ctypes.c_int32), ("norm_eps", ctypes.c_float), ("sources", ctypes.c_int32)]
 
 
+class EpParams(ctypes.Structure):
+    _fields_ = [("bs", ctypes.c_int32), ("top_k", ctypes.c_int32), ("num_instances", ctypes.c_int32),
+                ("gpus", ctypes.c_int32), ("rank", ctypes.c_int32), ("row_bytes", ctypes.c_int32),
+                ("scale_bytes", ctypes.c_int32), ("recv_rows", ctypes.c_int32)]
+
+
 class GmmParams(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int32), ("hidden", ctypes.c_int32), ("out_dim", ctypes.c_int32),
                 ("num_instances", ctypes.c_int32)]
@@ -55,6 +61,8 @@ EXPORTS = (
     "moe_dispatch_workspace_size", "moe_dispatch",
     "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm", "moe_combine",
     "moe_dispatch_noalloc", "moe_grouped_matmul_workspace_size", "moe_grouped_matmul", "moe_grouped_matmul_mx",
+    "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_push", "moe_ep_pull",
+    "moe_ipc_export", "moe_ipc_import", "moe_ipc_close",
 )
 
 
@@ -81,6 +89,13 @@ def _load():
     L.moe_grouped_matmul_workspace_size.argtypes = [P(GmmParams), P(sz)]
     L.moe_grouped_matmul.argtypes = [P(GmmParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_grouped_matmul_mx.argtypes = [P(GmmParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_ep_workspace_size.argtypes = [P(EpParams), P(sz)]
+    L.moe_ep_plan.argtypes = [P(EpParams), vp, vp, vp, vp, sz, vp]
+    L.moe_ep_push.argtypes = [P(EpParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_ep_pull.argtypes = [P(EpParams), vp, vp, vp, vp, sz, vp]
+    L.moe_ipc_export.argtypes = [vp, vp, P(ctypes.c_uint64)]
+    L.moe_ipc_import.argtypes = [vp, ctypes.c_uint64, P(vp), P(vp)]
+    L.moe_ipc_close.argtypes = [vp]
     for name in EXPORTS:
         if name != "moe_status_string":
             getattr(L, name).restype = ctypes.c_int
@@ -452,3 +467,110 @@ def grouped_matmul_mx(expand_x, x_sf, expert_offsets, weight, weight_sf, out=Non
             ctypes.byref(p), _ptr(expand_x), _ptr(x_sf), _ptr(expert_offsets), _ptr(weight), _ptr(weight_sf),
             _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+# --------------------------------------------------------------------------
+# expert parallelism across GPUs (see combine_moe_update_b200/ep.py)
+# --------------------------------------------------------------------------
+
+IPC_HANDLE_BYTES = 64
+DEV_CAPACITY = 8
+
+
+def ep_row_bytes(quant_mode, hidden):
+    """(row_bytes, scale_bytes) of a dispatched row in quant_mode."""
+    return ((2 * hidden if quant_mode == 0 else hidden),
+            {0: 0, 1: 0, 2: 4, 3: 4 * ((hidden + 127) // 128), 4: hidden // 32}[quant_mode])
+
+
+def ep_params(bs, top_k, num_instances, gpus, rank, row_bytes, scale_bytes, recv_rows):
+    return EpParams(int(bs), int(top_k), int(num_instances), int(gpus), int(rank), int(row_bytes),
+                    int(scale_bytes), int(recv_rows))
+
+
+def ep_workspace_bytes(p: EpParams) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_ep_workspace_size", lib.moe_ep_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return int(n.value)
+
+
+def _ptr_table(t, name):
+    """A [G] int64 CUDA tensor of device addresses (the pointer tables)."""
+    return _req(t, name, torch.int64)
+
+
+def ep_plan(p: EpParams, counts_all, recv_counts, recv_offsets, workspace, stream=None):
+    G, E = p.gpus, p.num_instances
+    _req(counts_all, "counts_all", torch.int32, (G, E))
+    _req(recv_counts, "recv_counts", torch.int32, (E // G,))
+    _req(recv_offsets, "recv_offsets", torch.int32, (E // G + 1,))
+    _req(workspace, "workspace", torch.uint8)
+    dev = counts_all.device
+    _same_device(dev, ("recv_counts", recv_counts), ("recv_offsets", recv_offsets), ("workspace", workspace))
+    with torch.cuda.device(dev):
+        _check("moe_ep_plan", lib.moe_ep_plan(ctypes.byref(p), _ptr(counts_all), _ptr(recv_counts),
+                                              _ptr(recv_offsets), _ptr(workspace), workspace.numel(),
+                                              _stream(stream)))
+
+
+def ep_push(p: EpParams, local: dict, instance_ids, peer_rows, peer_scales, peer_src, global_idx, workspace,
+            stream=None):
+    """local: moe_dispatch's outputs on this GPU (alloc_dispatch_outputs layout)."""
+    rows = p.bs * p.top_k
+    _req(local["expand_x"], "expand_x", local["expand_x"].dtype)
+    if local["expand_x"].numel() * local["expand_x"].element_size() != rows * p.row_bytes:
+        raise ValueError("expand_x does not hold bs * K rows of row_bytes")
+    sc = local.get("dyn_scales")
+    if p.scale_bytes:
+        _req(sc, "dyn_scales", sc.dtype if sc is not None else torch.float32)
+        if sc.numel() * sc.element_size() != rows * p.scale_bytes:
+            raise ValueError("dyn_scales does not hold bs * K rows of scale_bytes")
+        _ptr_table(peer_scales, "peer_scales")
+    _req(local["offsets"], "offsets", torch.int32, (p.num_instances + 1,))
+    _req(local["src_of_row"], "src_of_row", torch.int32, (rows,))
+    _req(local["expand_idx"], "expand_idx", torch.int32, (p.bs, p.top_k))
+    _req(instance_ids, "instance_ids", torch.int32, (p.bs, p.top_k))
+    _req(global_idx, "global_idx", torch.int32, (p.bs, p.top_k))
+    _ptr_table(peer_rows, "peer_rows")
+    if peer_src is not None:
+        _ptr_table(peer_src, "peer_src")
+    dev = instance_ids.device
+    with torch.cuda.device(dev):
+        _check("moe_ep_push", lib.moe_ep_push(
+            ctypes.byref(p), _ptr(local["expand_x"]), _ptr(sc if p.scale_bytes else None), _ptr(local["offsets"]),
+            _ptr(local["src_of_row"]), _ptr(local["expand_idx"]), _ptr(instance_ids), _ptr(peer_rows),
+            _ptr(peer_scales if p.scale_bytes else None), _ptr(peer_src), _ptr(global_idx), _ptr(workspace),
+            workspace.numel(), _stream(stream)))
+
+
+def ep_pull(p: EpParams, peer_rows, local_offsets, local_rows, workspace, stream=None):
+    _ptr_table(peer_rows, "peer_rows")
+    _req(local_offsets, "local_offsets", torch.int32, (p.num_instances + 1,))
+    _req(local_rows, "local_rows", local_rows.dtype)
+    if local_rows.numel() * local_rows.element_size() != p.bs * p.top_k * p.row_bytes:
+        raise ValueError("local_rows does not hold bs * K rows of row_bytes")
+    with torch.cuda.device(local_rows.device):
+        _check("moe_ep_pull", lib.moe_ep_pull(ctypes.byref(p), _ptr(peer_rows), _ptr(local_offsets),
+                                              _ptr(local_rows), _ptr(workspace), workspace.numel(),
+                                              _stream(stream)))
+
+
+def ipc_export(t: torch.Tensor):
+    """(handle bytes, offset) for a CUDA tensor's memory, for moe_ipc_import in another process."""
+    h = (ctypes.c_uint8 * IPC_HANDLE_BYTES)()
+    off = ctypes.c_uint64(0)
+    with torch.cuda.device(t.device):
+        _check("moe_ipc_export", lib.moe_ipc_export(_ptr(t), h, ctypes.byref(off)))
+    return bytes(h), int(off.value)
+
+
+def ipc_import(handle: bytes, offset: int):
+    """(base, device address) of a peer's exported memory, mapped on the current device."""
+    h = (ctypes.c_uint8 * IPC_HANDLE_BYTES).from_buffer_copy(handle)
+    base, ptr = ctypes.c_void_p(), ctypes.c_void_p()
+    _check("moe_ipc_import", lib.moe_ipc_import(h, ctypes.c_uint64(offset), ctypes.byref(base), ctypes.byref(ptr)))
+    return base.value, ptr.value
+
+
+def ipc_close(base: int):
+    _check("moe_ipc_close", lib.moe_ipc_close(ctypes.c_void_p(base)))

@@ -14,6 +14,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "dispatch.cuh"
+#include "ep.cuh"
 #include "grouped_matmul.cuh"
 #include "update_expert.cuh"
 
@@ -652,3 +653,168 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_dispatch_params *p, const v
         return MOE_ERR_CUDA;
     return MOE_OK;
 }
+
+// -------------------------------------------- expert parallelism across GPUs ---
+
+namespace {
+
+bool valid_ep(const moe_ep_params &p) {
+    if (p.bs < 1 || p.bs > MOE_MAX_BS || p.top_k < 1 || p.top_k > MOE_MAX_TOP_K) return false;
+    if (p.gpus < 1 || p.gpus > MOE_EP_MAX_GPUS || p.rank < 0 || p.rank >= p.gpus) return false;
+    if (p.num_instances < 1 || p.num_instances > MOE_MAX_EXPERTS || p.num_instances % p.gpus != 0) return false;
+    if (p.row_bytes < 16 || p.row_bytes % 16 != 0 || p.row_bytes > 2 * MOE_MAX_HIDDEN) return false;
+    if (p.scale_bytes < 0 || p.scale_bytes > 4 * MOE_MAX_HIDDEN / 32) return false;
+    if (p.recv_rows < 0) return false;
+    return true;
+}
+
+// The EP workspace: the error-word area, then gstart [E] and base [G + 1].
+size_t ep_workspace_bytes(const moe_ep_params &p) {
+    return kWorkspaceBytes + (((size_t)p.num_instances + p.gpus + 1) * sizeof(int32_t) + 15) / 16 * 16;
+}
+
+moe::EpArgs ep_args(const moe_ep_params &p, void *workspace) {
+    moe::EpArgs a = {};
+    a.bs = p.bs;
+    a.top_k = p.top_k;
+    a.num_instances = p.num_instances;
+    a.gpus = p.gpus;
+    a.rank = p.rank;
+    a.row_bytes = p.row_bytes;
+    a.scale_bytes = p.scale_bytes;
+    a.recv_rows = p.recv_rows;
+    unsigned char *ws = reinterpret_cast<unsigned char *>(workspace);
+    a.err = reinterpret_cast<uint32_t *>(ws);
+    a.gstart = reinterpret_cast<int32_t *>(ws + kWorkspaceBytes);
+    a.base = a.gstart + p.num_instances;
+    return a;
+}
+
+size_t ep_copy_smem(const moe_ep_params &p) { return ((size_t)2 * p.num_instances + p.gpus + 2) * sizeof(int); }
+
+int ep_copy_blocks(const moe_ep_params &p) {
+    return (p.bs * p.top_k + moe::kEpRowsPerBlock - 1) / moe::kEpRowsPerBlock;
+}
+
+PFN_cuMemGetAddressRange_v3020 address_range_fn() {
+    static PFN_cuMemGetAddressRange_v3020 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *q = nullptr;
+        cudaDriverEntryPointQueryResult r;
+        if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &q, 12000, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(q);
+    });
+    return fn;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_ep_workspace_size(const moe_ep_params *p, size_t *bytes) {
+    if (p == nullptr || bytes == nullptr || !valid_ep(*p)) return MOE_ERR_INVALID_ARG;
+    *bytes = ep_workspace_bytes(*p);
+    return MOE_OK;
+}
+
+moe_status moe_ep_plan(const moe_ep_params *p, const int32_t *counts_all, int32_t *recv_counts,
+                       int32_t *recv_offsets, void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr || !valid_ep(*p)) return MOE_ERR_INVALID_ARG;
+    if (!counts_all || !recv_counts || !recv_offsets || !aligned(counts_all, 4) || !aligned(recv_counts, 4) ||
+        !aligned(recv_offsets, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < ep_workspace_bytes(*p))
+        return MOE_ERR_WORKSPACE;
+    moe::EpArgs a = ep_args(*p, workspace);
+    a.counts_all = counts_all;
+    return launch(moe::ep_plan_kernel, 1, 1024, 0, as_stream(cuda_stream), a, recv_counts, recv_offsets) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_push(const moe_ep_params *p, const void *local_rows, const void *local_scales,
+                       const int32_t *local_offsets, const int32_t *src_of_row, const int32_t *expand_idx,
+                       const int32_t *instance_ids, void *const *peer_rows, void *const *peer_scales,
+                       int32_t *const *peer_src, int32_t *global_idx, void *workspace, size_t workspace_bytes,
+                       void *cuda_stream) {
+    if (p == nullptr || !valid_ep(*p)) return MOE_ERR_INVALID_ARG;
+    if (!local_rows || !local_offsets || !src_of_row || !expand_idx || !instance_ids || !peer_rows || !global_idx)
+        return MOE_ERR_INVALID_ARG;
+    if ((p->scale_bytes > 0) != (local_scales != nullptr && peer_scales != nullptr)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(local_rows, 16) || !aligned(peer_rows, 8) || (peer_scales && !aligned(peer_scales, 8)) ||
+        (peer_src && !aligned(peer_src, 8)) || !aligned(local_offsets, 4) || !aligned(src_of_row, 4) ||
+        !aligned(expand_idx, 4) || !aligned(instance_ids, 4) || !aligned(global_idx, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < ep_workspace_bytes(*p))
+        return MOE_ERR_WORKSPACE;
+    moe::EpArgs a = ep_args(*p, workspace);
+    a.local_offsets = local_offsets;
+    const size_t smem = ep_copy_smem(*p);
+    auto kernel = moe::ep_copy_kernel<true>;
+    if (!ensure_smem(kernel, smem)) return MOE_ERR_CUDA;
+    return launch(kernel, ep_copy_blocks(*p), moe::kEpThreads, smem, as_stream(cuda_stream), a,
+                  reinterpret_cast<const uint8_t *>(local_rows), (uint8_t *)nullptr,
+                  reinterpret_cast<const uint8_t *>(local_scales), reinterpret_cast<uint8_t *const *>(peer_rows),
+                  reinterpret_cast<uint8_t *const *>(peer_scales), peer_src, src_of_row, expand_idx, global_idx,
+                  instance_ids) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_pull(const moe_ep_params *p, void *const *peer_rows, const int32_t *local_offsets, void *local_rows,
+                       void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr || !valid_ep(*p)) return MOE_ERR_INVALID_ARG;
+    if (!peer_rows || !local_offsets || !local_rows) return MOE_ERR_INVALID_ARG;
+    if (!aligned(local_rows, 16) || !aligned(peer_rows, 8) || !aligned(local_offsets, 4)) return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < ep_workspace_bytes(*p))
+        return MOE_ERR_WORKSPACE;
+    moe::EpArgs a = ep_args(*p, workspace);
+    a.local_offsets = local_offsets;
+    const size_t smem = ep_copy_smem(*p);
+    auto kernel = moe::ep_copy_kernel<false>;
+    if (!ensure_smem(kernel, smem)) return MOE_ERR_CUDA;
+    return launch(kernel, ep_copy_blocks(*p), moe::kEpThreads, smem, as_stream(cuda_stream), a,
+                  (const uint8_t *)nullptr, reinterpret_cast<uint8_t *>(local_rows), (const uint8_t *)nullptr,
+                  reinterpret_cast<uint8_t *const *>(peer_rows), (uint8_t *const *)nullptr, (int32_t *const *)nullptr,
+                  (const int32_t *)nullptr, (const int32_t *)nullptr, (int32_t *)nullptr,
+                  (const int32_t *)nullptr) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_ipc_export(const void *dev_ptr, void *handle, uint64_t *offset) {
+    if (dev_ptr == nullptr || handle == nullptr || offset == nullptr) return MOE_ERR_INVALID_ARG;
+    const PFN_cuMemGetAddressRange_v3020 range = address_range_fn();
+    if (range == nullptr) return MOE_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) return MOE_ERR_CUDA;
+    static_assert(sizeof(h) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+    std::memcpy(handle, &h, sizeof h);
+    *offset = reinterpret_cast<uint64_t>(dev_ptr) - static_cast<uint64_t>(base);
+    return MOE_OK;
+}
+
+moe_status moe_ipc_import(const void *handle, uint64_t offset, void **base, void **dev_ptr) {
+    if (handle == nullptr || base == nullptr || dev_ptr == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof h);
+    void *b = nullptr;
+    if (cudaIpcOpenMemHandle(&b, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return MOE_ERR_CUDA;
+    *base = b;
+    *dev_ptr = static_cast<unsigned char *>(b) + offset;
+    return MOE_OK;
+}
+
+moe_status moe_ipc_close(void *base) {
+    if (base == nullptr) return MOE_ERR_INVALID_ARG;
+    return cudaIpcCloseMemHandle(base) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

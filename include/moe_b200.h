@@ -75,6 +75,7 @@ typedef enum {
 #define MOE_DEV_BAD_ID    1u  /* an expert / instance id or an expand_idx row out of range */
 #define MOE_DEV_BAD_TABLE 2u  /* mapping table broke its restrictions; every copy was dropped */
 #define MOE_DEV_TIMEOUT   4u  /* a bounded wait for an asynchronous copy gave up; outputs incomplete */
+#define MOE_DEV_CAPACITY  8u  /* expert parallelism: a receive buffer too small; rows beyond it dropped */
 
 /* The largest workspace any *_workspace_size call reports for one source
  * rank (bytes): the 256-byte area that holds the error word. */
@@ -383,6 +384,117 @@ MOE_API moe_status moe_dispatch_noalloc(const moe_dispatch_params *p, const void
                                         void *dyn_scales, int32_t *expand_idx, int32_t *src_of_row,
                                         int32_t *expert_counts, int32_t *expert_offsets, uint32_t *device_error_out,
                                         void *cuda_stream);
+
+/* ------------------------------------------------------------------------ */
+/* Expert parallelism across GPUs: the AllToAllV of dispatch and of combine  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The pages' EP AllToAllV moves every quantized copy to the rank hosting its
+ * instance (aclnnMoeDistributeDispatchV2, "功能说明", "计算公式": quantOut
+ * then AllToAllV) and the expert outputs back (aclnnMoeDistributeCombineAddRmsNorm,
+ * "计算公式": ataOut = AllToAllV).  Across G GPUs, GPU q owns the instances
+ * [q * E / G, (q + 1) * E / G) (and so the simulated ranks that host them)
+ * and every GPU is one source of its own bs tokens.  The rows of the group
+ * are then exactly those of moe_dispatch with sources = G on one GPU,
+ * ordered by (instance, source GPU, token, k); GPU q's receive buffer holds
+ * the stretch of that order its instances own, so its row r is global row
+ * base[q] + r.
+ *
+ * A layer on GPU g:
+ *   1. moe_update_expert and moe_dispatch on its own tokens over all E
+ *      instances (local rows, counts [E], offsets [E+1]);
+ *   2. the counts of every GPU gathered into counts_all [G][E] on every GPU
+ *      (a collective of E ints per GPU, by the caller);
+ *   3. moe_ep_plan, then moe_ep_push: every local row (and its scales) is
+ *      stored into its owner's receive buffer through the owner's pointer;
+ *   4. a group barrier (every push done), then the expert step on the
+ *      receive buffer (moe_ep_plan's recv_counts / recv_offsets describe it);
+ *   5. a group barrier (every expert output written), then moe_ep_pull: each
+ *      local row reads its output back from the owner, in the local row order
+ *      moe_dispatch made, so moe_combine_add_rmsnorm runs with the local
+ *      expand_idx unchanged;
+ *   6. a group barrier before the buffers are reused.
+ * The pointer tables hold, per GPU q, a pointer this GPU can dereference:
+ * its own buffer for q = g, a peer mapping (moe_ipc_import, or any mapping
+ * the caller set up) otherwise.  The copies are plain 16-byte loads and
+ * stores by the SMs over NVLink; no TMA load reads peer memory.  With every
+ * pointer in one GPU's memory (G buffers of one device), the calls emulate a
+ * group of G on one GPU.
+ */
+
+#define MOE_EP_MAX_GPUS       64
+#define MOE_IPC_HANDLE_BYTES  64
+
+typedef struct {
+    int32_t bs;             /* tokens of this GPU (one source), (0, 512] */
+    int32_t top_k;          /* K, (0, 16] */
+    int32_t num_instances;  /* E over the whole group, (0, 1024], a multiple of gpus */
+    int32_t gpus;           /* G, [1, MOE_EP_MAX_GPUS] */
+    int32_t rank;           /* this GPU, [0, G) */
+    int32_t row_bytes;      /* bytes of one row moved: H for int8 / e4m3 rows, 2H for bf16 rows;
+                               a multiple of 16 */
+    int32_t scale_bytes;    /* bytes of one row's scales: 0 (quant modes 0, 1), 4 (2),
+                               4 * ceil(H / 128) (3), H / 32 (4); push only */
+    int32_t recv_rows;      /* rows of every GPU's receive (and expert output) buffer, >= 0 */
+} moe_ep_params;
+
+/* Workspace of the plan / push / pull calls of one layer (they share it:
+ * the plan is stored there), 16-byte aligned, zeroed once. */
+MOE_API moe_status moe_ep_workspace_size(const moe_ep_params *p, size_t *bytes);
+
+/*
+ * From the gathered counts, the global row of this GPU's first copy of
+ * every instance (kept in the workspace for push and pull), and this GPU's
+ * receive layout:
+ *   counts_all    [G][E] int32 device: row g' = moe_dispatch's expert_counts on GPU g'
+ *   recv_counts   [E/G]   int32 device, out: rows this GPU receives per own instance
+ *   recv_offsets  [E/G+1] int32 device, out: their exclusive prefix; [E/G] = rows received
+ * Device errors: more rows than recv_rows sets MOE_DEV_CAPACITY (push and
+ * pull then drop the rows beyond it).
+ */
+MOE_API moe_status moe_ep_plan(const moe_ep_params *p, const int32_t *counts_all, int32_t *recv_counts,
+                               int32_t *recv_offsets, void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * Stores this GPU's dispatched rows into their owners' receive buffers:
+ *   local_rows     [bs*K, row_bytes] device: moe_dispatch's expand_x
+ *   local_scales   [bs*K, scale_bytes] device: its dyn_scales (NULL when scale_bytes = 0)
+ *   local_offsets  [E+1], src_of_row [bs*K], expand_idx [bs, K], instance_ids [bs, K]:
+ *                  moe_dispatch's outputs and its instance ids
+ *   peer_rows      [G] device array of pointers: receive buffers, [recv_rows, row_bytes] each
+ *   peer_scales    [G] device array of pointers, [recv_rows, scale_bytes] each (NULL when scale_bytes = 0)
+ *   peer_src       [G] device array of pointers, optional: [recv_rows] int32 each,
+ *                  receives every row's copy id in the group, (g * bs + i) * K + k
+ *   global_idx     [bs, K] int32 device, out: every copy's global row (-1 if not sent)
+ */
+MOE_API moe_status moe_ep_push(const moe_ep_params *p, const void *local_rows, const void *local_scales,
+                               const int32_t *local_offsets, const int32_t *src_of_row, const int32_t *expand_idx,
+                               const int32_t *instance_ids, void *const *peer_rows, void *const *peer_scales,
+                               int32_t *const *peer_src, int32_t *global_idx, void *workspace,
+                               size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * Brings every local row's expert output back from its owner:
+ *   peer_rows   [G] device array of pointers: expert output buffers, [recv_rows, row_bytes] each
+ *   local_offsets [E+1] int32 device: moe_dispatch's offsets on this GPU
+ *   local_rows  [bs*K, row_bytes] device, out: the outputs in local row order
+ *               (rows >= local_offsets[E] untouched)
+ */
+MOE_API moe_status moe_ep_pull(const moe_ep_params *p, void *const *peer_rows, const int32_t *local_offsets,
+                               void *local_rows, void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * Peer mappings for the pointer tables (CUDA IPC, no multicast object):
+ * moe_ipc_export writes a MOE_IPC_HANDLE_BYTES handle (host memory) for the
+ * device allocation that holds dev_ptr and dev_ptr's offset in it; another
+ * process on the same node maps it with moe_ipc_import (base = the mapping to
+ * give moe_ipc_close later, dev_ptr = base + offset).  The exporter keeps the
+ * allocation alive until every importer has closed it.
+ */
+MOE_API moe_status moe_ipc_export(const void *dev_ptr, void *handle, uint64_t *offset);
+MOE_API moe_status moe_ipc_import(const void *handle, uint64_t offset, void **base, void **dev_ptr);
+MOE_API moe_status moe_ipc_close(void *base);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,130 @@
+"""Expert parallelism across GPUs, emulated on one GPU: G ranks' buffers in
+this GPU's memory, the library's plan / push / pull kernels moving rows
+between them through the same pointer tables a real group uses.
+
+Across G GPUs every GPU is one source of its own tokens, so the group's rows
+must be exactly the single-GPU dispatch of all G * bs tokens (ordered by
+instance, source, token, k; aclnnMoeDistributeDispatchV2, 计算公式), with GPU
+q's receive buffer holding the stretch its instances own.  The tests compare
+every receive buffer, its scales and copy ids, the receive counts and
+offsets, every rank's global row of each copy, and the combine+Add+RMSNorm
+output (aclnnMoeDistributeCombineAddRmsNorm, 计算公式) with the oracle run on
+all G * bs tokens on one device.  Identity mapping tables keep the replica
+choice out of the comparison (a GPU's update_expert numbers its own tokens)."""
+import numpy as np
+import pytest
+import torch
+
+from combine_moe_update_b200 import inputs as gen
+from oracle import oracle as orc
+
+from gpu_harness import assert_close_bf16, dev, dev_bf16, host, poison_
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from combine_moe_update_b200 import binding
+    return binding
+
+
+@pytest.fixture(scope="module")
+def EP():
+    from combine_moe_update_b200 import ep
+    return ep
+
+
+def _bytes(a, lo, hi):
+    a = np.ascontiguousarray(a)
+    return a.view(np.uint8).reshape(a.shape[0], -1)[lo:hi]
+
+
+def _inputs(seed, G, bs, H, E, K, ws, smooth):
+    rng = np.random.Generator(np.random.PCG64([81, seed]))
+    T = G * bs
+    return dict(
+        x=gen.bf16_bits(rng.standard_normal((T, H), np.float32)),
+        ids=gen.topk_uniform(rng, T, E, K),
+        scales=gen.softmax_scales(rng, T, K),
+        residual=gen.bf16_bits(rng.standard_normal((T, H), np.float32)),
+        shared=gen.bf16_bits(rng.standard_normal((T, H), np.float32)),
+        gamma=gen.bf16_bits(rng.uniform(0.5, 1.5, size=H).astype(np.float32)),
+        expert_rows=gen.bf16_bits(rng.standard_normal((T * K, H), np.float32)),  # by global row
+        smooth=rng.uniform(0.5, 2.0, size=(E, H)).astype(np.float32) if smooth else None,
+        table=gen.identity_table(E, ws))
+
+
+@pytest.mark.parametrize("G,bs,H,E,K,ws,mode,smooth", [
+    (2, 64, 1024, 16, 4, 4, 0, False),
+    (4, 48, 2048, 32, 6, 8, 2, True),
+    (2, 40, 1040, 32, 8, 8, 3, False),    # ragged last tile
+    (4, 32, 1024, 64, 8, 16, 4, False),   # mxfp8
+    (8, 24, 7168, 256, 8, 32, 2, True),   # the decode row length, eight GPUs
+    (2, 512, 1024, 16, 8, 2, 1, True),    # static per-instance scales, 4096 copies per GPU
+])
+def test_emulated_group_equals_one_gpu_dispatch(B, EP, G, bs, H, E, K, ws, mode, smooth):
+    inp = _inputs(G * 1000 + mode, G, bs, H, E, K, ws, smooth or mode == 1)
+    grp = EP.EmulatedGroup(G, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws, quant_mode=mode)
+    for r in grp.ranks:
+        for t in r.buffers() + [r.global_idx, r.recv_counts, r.recv_offsets]:
+            if t is not None:
+                poison_(t)
+    sm = None if inp["smooth"] is None else dev(inp["smooth"])
+    table = dev(inp["table"])
+    sl = lambda a, g: np.ascontiguousarray(a[g * bs:(g + 1) * bs])
+    grp.dispatch([dict(expert_ids=dev(sl(inp["ids"], g)), table=table, x=dev_bf16(sl(inp["x"], g)),
+                       expert_scales=dev(sl(inp["scales"], g)), smooth=sm) for g in range(G)])
+    torch.cuda.synchronize()
+    for r in grp.ranks:
+        assert r.device_errors() == 0
+
+    # the oracle: all G * bs tokens on one device
+    bal, bm, _ = orc.update_expert(inp["ids"], inp["table"], ws, expert_scales=inp["scales"])
+    od = orc.dispatch(inp["x"], bal, E, mode, mask=bm, smooth=inp["smooth"])
+    off, El = od["offsets"], E // G
+    for q, r in enumerate(grp.ranks):
+        b, e_ = int(off[q * El]), int(off[(q + 1) * El])
+        np.testing.assert_array_equal(host(r.recv_counts), od["counts"][q * El:(q + 1) * El])
+        np.testing.assert_array_equal(host(r.recv_offsets), off[q * El:(q + 1) * El + 1] - b)
+        np.testing.assert_array_equal(_bytes(host(r.recv_x), 0, e_ - b), _bytes(od["expand_x"], b, e_))
+        np.testing.assert_array_equal(host(r.recv_src)[:e_ - b], od["src_of_row"][b:e_])
+        if od["dyn_scales"] is not None:
+            np.testing.assert_array_equal(_bytes(host(r.recv_scales), 0, e_ - b), _bytes(od["dyn_scales"], b, e_))
+        np.testing.assert_array_equal(host(r.global_idx), od["expand_idx"][q * bs:(q + 1) * bs])
+
+    # the expert step: each GPU's output rows are the synthetic rows of its global rows
+    for q, r in enumerate(grp.ranks):
+        b, e_ = int(off[q * El]), int(off[(q + 1) * El])
+        poison_(r.expert_out)
+        r.expert_out[:e_ - b].copy_(dev_bf16(inp["expert_rows"][b:e_]))
+    outs = grp.combine([dict(expert_scales=dev(sl(inp["scales"], g)), residual=dev_bf16(sl(inp["residual"], g)),
+                             gamma=dev_bf16(inp["gamma"]), norm_eps=1e-6, shared_x=dev_bf16(sl(inp["shared"], g)))
+                        for g in range(G)])
+    torch.cuda.synchronize()
+    oc = orc.combine_add_rmsnorm(inp["expert_rows"], od["expand_idx"], inp["scales"], inp["residual"],
+                                 inp["gamma"], 1e-6, shared_x=inp["shared"])
+    for g, (r, o) in enumerate(zip(grp.ranks, outs)):
+        assert r.device_errors() == 0
+        assert_close_bf16(host(o["y"]), oc["y_f64"][g * bs:(g + 1) * bs], what=f"y of GPU {g}")
+
+
+def test_receive_buffer_too_small_is_flagged(B, EP):
+    G, bs, H, E, K, ws = 2, 64, 1024, 16, 4, 4
+    inp = _inputs(7, G, bs, H, E, K, ws, False)
+    grp = EP.EmulatedGroup(G, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws, quant_mode=0,
+                           recv_rows=16)
+    for r in grp.ranks:
+        poison_(r.recv_x)
+    sl = lambda a, g: np.ascontiguousarray(a[g * bs:(g + 1) * bs])
+    grp.dispatch([dict(expert_ids=dev(sl(inp["ids"], g)), table=dev(inp["table"]), x=dev_bf16(sl(inp["x"], g)))
+                  for g in range(G)])
+    torch.cuda.synchronize()
+    bal, bm, _ = orc.update_expert(inp["ids"], inp["table"], ws)
+    od = orc.dispatch(inp["x"], bal, E, 0, mask=bm)
+    for q, r in enumerate(grp.ranks):
+        assert r.device_errors() & B.DEV_CAPACITY
+        b = int(od["offsets"][q * (E // G)])
+        # the rows that fit are right; nothing past the buffer was written (it has 16 rows)
+        np.testing.assert_array_equal(_bytes(host(r.recv_x), 0, 16), _bytes(od["expand_x"], b, b + 16))
