@@ -34,18 +34,33 @@ struct CombineArgs {
     uint32_t *err;
 };
 
-// NT is the dispatch token block size for the row (dp_threads), so every
-// thread owns exactly kCbVecs = 4 vectors when 32 * 4 divides H / 8.
-constexpr int kCbVecs = 4;
+// Threads of a block for NV vectors of 8 elements per block and VECS vectors
+// per thread, from the same fixed set of block sizes as the dispatch.
+__host__ __device__ inline int cb_threads(int NV, int vecs) {
+    const int need = ((NV + vecs - 1) / vecs + 31) / 32 * 32;
+    return need <= 64 ? 64 : need <= 128 ? 128 : need <= 192 ? 192 : need <= 224 ? 224 : 256;
+}
 
-// NORM false: the plain combine (combineOut to y; no residual, no norm).
-template <int KMAX, bool SHARED, int NT, bool NORM>
+// One token per block (SPLIT = 1, VECS = 4: 224 threads at H = 7168, four
+// blocks per SM, a 512-token batch in one wave), or per cluster of two
+// blocks (SPLIT = 2, VECS = 2) when that takes fewer waves: block h of the
+// cluster holds vectors [h * V / 2, (h + 1) * V / 2) of the row and the two
+// sums of x^2 meet through distributed shared memory.  Every thread issues
+// the loads of one vector together -- all K rows (a pruned copy issues
+// none), the shared row and the residual row -- so a vector costs one round
+// trip to memory.  NORM false: the plain combine (combineOut to y; no
+// residual, no norm).
+template <int KMAX, bool SHARED, int NT, bool NORM, int SPLIT>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(CombineArgs a) {
+    constexpr int VECS = SPLIT == 1 ? 4 : 2;
+    constexpr int NW = NT / 32;
     __shared__ int s_row[16];
     __shared__ float s_w[16];
-    __shared__ float s_red[NT / 32];
-    const int i = blockIdx.x, t = threadIdx.x;
-    const int H = a.hidden, V = H >> 3, K = a.top_k;
+    __shared__ float s_red[NW];
+    __shared__ float s_part;
+    const int t = threadIdx.x;
+    const int i = blockIdx.x / SPLIT, h = SPLIT == 1 ? 0 : (int)cluster_ctarank();
+    const int H = a.hidden, V = H >> 3, K = a.top_k, Vh = V / SPLIT, p0 = h * Vh;  // V is even (H % 16 == 0)
 
     pdl_wait();  // expand_idx and the expert rows come from earlier kernels
     if (t < K) {
@@ -70,14 +85,14 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
     }
 
     const size_t tok = (size_t)i * H;
-    float xs[kCbVecs][8];
+    float xs[VECS][8];
     float ss = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kCbVecs; ++j) {
-        const int p = t + j * NT;
+    for (int j = 0; j < VECS; ++j) {
+        const int pl = t + j * NT, p = p0 + pl;
 #pragma unroll
         for (int e = 0; e < 8; ++e) xs[j][e] = 0.0f;
-        if (p >= V) continue;
+        if (pl >= Vh) continue;
         uint4 rv[KMAX];
 #pragma unroll
         for (int k = 0; k < KMAX; ++k)
@@ -115,9 +130,9 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
     if constexpr (!NORM) {  // the plain combine: combineOut, rounded to bf16 once
         pdl_launch_dependents();
 #pragma unroll
-        for (int j = 0; j < kCbVecs; ++j) {
-            const int p = t + j * NT;
-            if (p >= V) continue;
+        for (int j = 0; j < VECS; ++j) {
+            const int pl = t + j * NT, p = p0 + pl;
+            if (pl >= Vh) continue;
             uint4 o;
             o.x = pack_bf16x2(xs[j][0], xs[j][1]);
             o.y = pack_bf16x2(xs[j][2], xs[j][3]);
@@ -127,14 +142,21 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
         }
         return;
     }
-    const float tot = block_sum<NT / 32>(ss, s_red);
+    float tot = block_sum<NW>(ss, s_red);
+    if constexpr (SPLIT == 2) {  // the row's two halves: the same sum, in the same order, in both blocks
+        if (t == 0) s_part = tot;
+        cluster_sync();
+        const float p_0 = ld_cluster_f32(&s_part, 0), p_1 = ld_cluster_f32(&s_part, 1);
+        tot = p_0 + p_1;
+        cluster_sync();  // the peer has read this block's partial before either block leaves
+    }
     pdl_launch_dependents();
     const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));
-    if (t == 0 && a.rstd_out) a.rstd_out[i] = rstd;
+    if (t == 0 && h == 0 && a.rstd_out) a.rstd_out[i] = rstd;
 #pragma unroll
-    for (int j = 0; j < kCbVecs; ++j) {
-        const int p = t + j * NT;
-        if (p >= V) continue;
+    for (int j = 0; j < VECS; ++j) {
+        const int pl = t + j * NT, p = p0 + pl;
+        if (pl >= Vh) continue;
         float g[8];
         unpack8(ld_cached(a.gamma + p * 8), g);
         uint4 yo;

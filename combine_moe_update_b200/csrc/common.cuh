@@ -90,6 +90,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase)
     }
 }
 
+// --- thread-block clusters: rank, barrier, and a float from a peer block's
+// shared memory (distributed shared memory; plain loads, no multicast) ---
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of every block of the cluster; orders shared-memory writes
+// before it with reads after it, across the cluster.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(const float *local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
 // Programmatic dependent launch (PTX griddepcontrol, sm_90 and later).  A
 // kernel launched with the programmatic-serialization attribute may start
 // while its predecessor runs; it must call pdl_wait() before it touches
