@@ -62,6 +62,12 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
     const int i = blockIdx.x / SPLIT, h = SPLIT == 1 ? 0 : (int)cluster_ctarank();
     const int H = a.hidden, V = H >> 3, K = a.top_k, Vh = V / SPLIT, p0 = h * Vh;  // V is even (H % 16 == 0)
 
+    if (t == 0) {  // this block's part of the residual and shared rows, into L2 while the predecessor drains
+        const size_t off = (size_t)i * H + (size_t)p0 * 8;
+        const uint32_t bytes = (uint32_t)Vh * 16;
+        if constexpr (NORM) prefetch_l2(a.residual + off, bytes);
+        if constexpr (SHARED) prefetch_l2(a.shared_x + off, bytes);
+    }
     pdl_wait();  // expand_idx and the expert rows come from earlier kernels
     if (t < K) {
         int row = a.expand_idx[i * K + t];

@@ -56,6 +56,14 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
 // taking issue slots from the warps that have work.
 constexpr uint32_t kWaitHintNs = 1u << 20;  // about a millisecond
 
+// Ask L2 to fetch `bytes` (a multiple of 16, 16-byte aligned) from global
+// memory.  Nothing comes back to the program and L2 is the point of
+// coherence, so this is safe on data a predecessor kernel may still write:
+// its later stores update the lines in L2.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     uint32_t ok;
     asm volatile(
