@@ -20,6 +20,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libmoe_b200.so")
+# Test-only build: every kernel with a bulk copy can leave one out, so that
+# the tests can run the bounded waits' timeout path (never shipped, never
+# loaded by the package).
+FAULT_LIB_PATH = os.path.join(LIB_DIR, "libmoe_b200_faultinj.so")
 PTXAS_LOG = os.path.join(LIB_DIR, "ptxas.log")
 
 NVCC_FLAGS = [
@@ -44,30 +48,33 @@ def sources():
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB_PATH):
+def stale(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB_PATH
+def build(force: bool = False, verbose: bool = False, fault_injection: bool = False) -> str:
+    path = FAULT_LIB_PATH if fault_injection else LIB_PATH
+    if not force and not stale(path):
+        return path
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, os.path.join(CSRC, "moe_b200.cu")]
+    tmp = path + f".tmp{os.getpid()}"
+    extra = ["-DMOE_FAULT_INJECTION"] if fault_injection else []
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-o", tmp, os.path.join(CSRC, "moe_b200.cu")]
     proc = subprocess.run(cmd, capture_output=True, text=True)
-    with open(PTXAS_LOG, "w") as f:
+    log = PTXAS_LOG if not fault_injection else PTXAS_LOG + ".faultinj"
+    with open(log, "w") as f:
         f.write(" ".join(cmd) + "\n" + proc.stdout + proc.stderr)
     if proc.returncode != 0:
         sys.stderr.write(proc.stdout + proc.stderr)
-        raise RuntimeError(f"nvcc failed ({proc.returncode}); see {PTXAS_LOG}")
+        raise RuntimeError(f"nvcc failed ({proc.returncode}); see {log}")
     if verbose:
         sys.stdout.write(proc.stdout + proc.stderr)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, fault_injection="--fault-injection" in sys.argv))

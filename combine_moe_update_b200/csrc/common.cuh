@@ -8,6 +8,16 @@
 
 namespace moe {
 
+// Test builds only (-DMOE_FAULT_INJECTION, a separate library the tests load):
+// a kernel leaves out one of its bulk copies, so that the bounded wait for it
+// runs out with nothing in flight and the timeout path runs.  The shipped
+// library never defines it.
+#ifdef MOE_FAULT_INJECTION
+constexpr bool kSkipOneCopy = true;
+#else
+constexpr bool kSkipOneCopy = false;
+#endif
+
 constexpr uint32_t kDevBadId = 1u;     // id or row index out of range: item dropped
 constexpr uint32_t kDevBadTable = 2u;  // mapping table broke its restrictions
 constexpr uint32_t kDevTimeout = 4u;   // a bounded wait gave up

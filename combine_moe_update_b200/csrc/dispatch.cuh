@@ -924,7 +924,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
             }
             return;
         }
-        if (t == 0 && c + 1 < ns) {
+        if (t == 0 && c + 1 < ns && !(kSkipOneCopy && blockIdx.x == 0 && c == 0)) {
             fence_proxy_async_smem();
             fetch_smooth(c + 1);
         }

@@ -93,8 +93,10 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     // which do not depend on it, so that all the loads are in flight together.
     if (a.table_mode == 2 && t == 0) {
         mbar_init(&s_tab_bar, 1);
-        mbar_arrive_expect_tx(&s_tab_bar, tab_bytes);
-        bulk_copy_g2s(const_cast<int32_t *>(s_tab), a.table, tab_bytes, &s_tab_bar);
+        if (!kSkipOneCopy) {
+            mbar_arrive_expect_tx(&s_tab_bar, tab_bytes);
+            bulk_copy_g2s(const_cast<int32_t *>(s_tab), a.table, tab_bytes, &s_tab_bar);
+        }
     }
     if (a.table_mode == 1)
         for (int q = t; q < E * F; q += kUeThreads) const_cast<int32_t *>(s_tab)[q] = ld_in(a.table + q);
