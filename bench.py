@@ -737,8 +737,18 @@ def run_b200_ep(args, rank, world, local_rank):
     (t_step,) = reduce_over_ranks([e0.elapsed_time(e1) / K], "max")
     recv = r.received()
     assert r.device_errors() == 0, "device error during the timed steps"
+    n = int(r.d["offsets"][-1].item())
     grp.close()
     n_kernels = kernels_per_step(w) + 3  # + plan, push, pull
+    # the whole step against HBM: the single-GPU path's bytes plus the exchange (each row read locally and
+    # written to its owner; each output read from its owner and written locally)
+    w.meta["distinct_instances"] = list(range(w.num_instances)) if w.smooth is not None else []
+    alg = algorithmic_bytes(w, n)
+    rb, sb = B.ep_row_bytes(w.quant_mode, w.hidden)
+    exch = 2 * n * (rb + sb) + 2 * n * 2 * w.hidden
+    peak, peak_kind = measured_peak()
+    step_bytes = alg["update"] + alg["dispatch"] + alg["combine"] + exch
+    ach = step_bytes / (t_step * 1e-3) / 1e9
     return {
         "metric": METRIC, "value": round(world * w.bs / (t_step * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True,
@@ -750,6 +760,10 @@ def run_b200_ep(args, rank, world, local_rank):
                    "quant_mode": w.quant_mode, "parallelism": f"ep{world}: instances split over the GPUs",
                    "rows_received_rank0": recv,
                    "l2": "not flushed: each step's exchange and gathers touch more than L2 across the group"},
+        "roofline": {"bound": "hbm", "kernel": "whole step (update, dispatch, plan, push, pull, combine)",
+                     "achieved": round(ach, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(ach / peak, 4), "traffic": None, "algorithmic_bytes": step_bytes,
+                     "note": "eager launches with two NCCL barriers and a count gather per step"},
         "e2e": None,
         "gpu_launches": n_kernels * K,
         "timing": "CUDA events around K eager steps (each with two barriers), max over ranks",
