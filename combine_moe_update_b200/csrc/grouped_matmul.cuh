@@ -474,13 +474,20 @@ __global__ void __launch_bounds__(kGmMxThreads, 1)
         }
     } else {  // warps 0-3: the block factors of every stage
         const int B = a.hidden >> 5;  // factor bytes per row
+        // this thread's factor rows: channel n0 + 32c + lane of the weight, row 32c + lane of the slot
+        const uint32_t *pa[4], *pb[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int ch = min(n0 + 32 * c + lane, a.out_dim - 1);
+            pa[c] = reinterpret_cast<const uint32_t *>(a.wsf + ((size_t)slot.x * a.out_dim + ch) * B);
+            const int r = min(32 * c + lane, nr - 1);
+            pb[c] = reinterpret_cast<const uint32_t *>(a.xsf + (size_t)(slot.y + r) * B);
+        }
         auto load_sf = [&](int k, uint32_t(&fa)[4], uint32_t(&fb)[4]) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const int ch = min(n0 + 32 * c + lane, a.out_dim - 1);
-                fa[c] = ld_in(reinterpret_cast<const uint32_t *>(a.wsf + ((size_t)slot.x * a.out_dim + ch) * B) + k);
-                const int r = min(32 * c + lane, nr - 1);
-                fb[c] = ld_in(reinterpret_cast<const uint32_t *>(a.xsf + (size_t)(slot.y + r) * B) + k);
+                fa[c] = ld_in(pa[c] + k);
+                fb[c] = ld_in(pb[c] + k);
             }
         };
         const uint32_t quarter = (uint32_t)(warp * 32) << 16;
@@ -501,10 +508,11 @@ __global__ void __launch_bounds__(kGmMxThreads, 1)
             if (lane == 0) mbar_arrive(&s_sf[s]);
             return true;
         };
-        // factor words four steps ahead (a weight row's 32-byte sector holds
-        // eight steps, so one load in eight goes to DRAM), in four register
-        // sets used in turn
-        constexpr int kPre = 4;
+        // factor words eight steps ahead (a weight row's 32-byte sector holds
+        // eight steps, so one load in eight goes to DRAM), in eight register
+        // sets used in turn: four steps ahead left the MMA issuer waiting for
+        // the factors (measured: 409 -> 376 us at 32 instances of 7168 x 7168)
+        constexpr int kPre = 8;
         uint32_t fa[kPre][4], fb[kPre][4];
 #pragma unroll
         for (int q = 0; q < kPre; ++q)
