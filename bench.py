@@ -690,11 +690,13 @@ def run_b200_layer_stack(args, rank, world, local_rank):
 def run_b200_ep(args, rank, world, local_rank):
     """Expert parallelism across the GPUs of the job: GPU g owns instances
     [g E / N, (g + 1) E / N) and dispatches its own batch; every step is
-    update + dispatch of its tokens, the gather of every GPU's counts, the
-    plan and push of its rows into their owners' receive buffers (peer
-    memory), a barrier, the expert step (the owner's output buffer, resident),
-    a barrier, the pull of its rows' outputs and combine+Add+RMSNorm.  Timed
-    with events on each rank, max over ranks."""
+    update + routing of its tokens, the gather of every GPU's counts, the
+    plan, the EP dispatch storing each quantized copy into its owner's
+    receive buffer (peer memory), a barrier, the expert step (the owner's
+    output buffer, resident), a barrier, and the EP combine+Add+RMSNorm
+    reading every copy's output from its owner.  The two-step form
+    dispatches locally, pushes the rows, and pulls the outputs back before a
+    local combine.  Timed with events on each rank, max over ranks."""
     import numpy as np
     import torch
     from combine_moe_update_b200 import binding as B
@@ -705,7 +707,8 @@ def run_b200_ep(args, rank, world, local_rank):
     w = gen.make(args.workload, seed=None if rank == 0 else 1000 + rank)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     bf = lambda a: dev(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16)
-    grp = EP.ProcessGroupEP(bs=w.bs, hidden=w.hidden, top_k=w.top_k, num_instances=w.num_instances,
+    fused = not args.ep_two_step
+    grp = EP.ProcessGroupEP(fused=fused, bs=w.bs, hidden=w.hidden, top_k=w.top_k, num_instances=w.num_instances,
                             ep_world_size=w.ep_world_size, quant_mode=w.quant_mode)
     r = grp.r
     table, smooth, gamma = dev(w.table), None if w.smooth is None else dev(w.smooth), bf(w.gamma)
@@ -739,13 +742,17 @@ def run_b200_ep(args, rank, world, local_rank):
     assert r.device_errors() == 0, "device error during the timed steps"
     n = int(r.d["offsets"][-1].item())
     grp.close()
-    n_kernels = kernels_per_step(w) + 3  # + plan, push, pull
-    # the whole step against HBM: the single-GPU path's bytes plus the exchange (each row read locally and
-    # written to its owner; each output read from its owner and written locally)
+    copies = w.bs * w.top_k
+    route = 3 if copies > 8192 else 1
+    # fused: update, route, plan, EP dispatch, EP combine; two-step: the one-GPU step + plan, push, pull
+    n_kernels = 1 + route + 3 if fused else kernels_per_step(w) + 3
+    # the whole step against HBM: the single-GPU path's bytes, plus for the two-step form the exchange (each
+    # row read locally and written to its owner; each output read from its owner and written locally).  The
+    # fused form writes each row once, at its owner, and reads each output once, from its owner.
     w.meta["distinct_instances"] = list(range(w.num_instances)) if w.smooth is not None else []
     alg = algorithmic_bytes(w, n)
     rb, sb = B.ep_row_bytes(w.quant_mode, w.hidden)
-    exch = 2 * n * (rb + sb) + 2 * n * 2 * w.hidden
+    exch = 0 if fused else 2 * n * (rb + sb) + 2 * n * 2 * w.hidden
     peak, peak_kind = measured_peak()
     step_bytes = alg["update"] + alg["dispatch"] + alg["combine"] + exch
     ach = step_bytes / (t_step * 1e-3) / 1e9
@@ -758,9 +765,11 @@ def run_b200_ep(args, rank, world, local_rank):
         "config": {"workload": args.workload, "bs_per_gpu": w.bs, "hidden": w.hidden, "top_k": w.top_k,
                    "num_instances": w.num_instances, "ep_world_size_simulated": w.ep_world_size,
                    "quant_mode": w.quant_mode, "parallelism": f"ep{world}: instances split over the GPUs",
+                   "exchange": "fused into dispatch and combine" if fused else "push and pull",
                    "rows_received_rank0": recv,
                    "l2": "not flushed: each step's exchange and gathers touch more than L2 across the group"},
-        "roofline": {"bound": "hbm", "kernel": "whole step (update, dispatch, plan, push, pull, combine)",
+        "roofline": {"bound": "hbm", "kernel": ("whole step (update, route, plan, EP dispatch, EP combine)" if fused
+                                                else "whole step (update, dispatch, plan, push, pull, combine)"),
                      "achieved": round(ach, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(ach / peak, 4), "traffic": None, "algorithmic_bytes": step_bytes,
                      "note": "eager launches with two NCCL barriers and a count gather per step"},
@@ -1239,6 +1248,9 @@ def main(argv=None):
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism across the job's GPUs (real exchange through peer memory) "
                          "instead of independent replicas")
+    ap.add_argument("--ep-two-step", action="store_true",
+                    help="with --ep: dispatch locally, then push / pull the rows (instead of the fused "
+                         "EP dispatch and combine that read and write the owners' buffers directly)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

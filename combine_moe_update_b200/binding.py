@@ -58,10 +58,11 @@ class GmmParams(ctypes.Structure):
 EXPORTS = (
     "moe_workspace_init", "moe_read_device_error", "moe_clear_device_error", "moe_status_string",
     "moe_update_expert_workspace_size", "moe_update_expert",
-    "moe_dispatch_workspace_size", "moe_dispatch",
+    "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_route",
     "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm", "moe_combine",
     "moe_dispatch_noalloc", "moe_grouped_matmul_workspace_size", "moe_grouped_matmul", "moe_grouped_matmul_mx",
-    "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_push", "moe_ep_pull",
+    "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_push", "moe_ep_pull", "moe_ep_dispatch",
+    "moe_ep_combine_add_rmsnorm",
     "moe_ipc_export", "moe_ipc_import", "moe_ipc_close",
 )
 
@@ -93,6 +94,11 @@ def _load():
     L.moe_ep_plan.argtypes = [P(EpParams), vp, vp, vp, vp, sz, vp]
     L.moe_ep_push.argtypes = [P(EpParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_ep_pull.argtypes = [P(EpParams), vp, vp, vp, vp, sz, vp]
+    L.moe_dispatch_route.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_ep_dispatch.argtypes = [P(DispatchParams), P(EpParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                  vp]
+    L.moe_ep_combine_add_rmsnorm.argtypes = [P(CombineParams), P(EpParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                             sz, vp]
     L.moe_ipc_export.argtypes = [vp, vp, P(ctypes.c_uint64)]
     L.moe_ipc_import.argtypes = [vp, ctypes.c_uint64, P(vp), P(vp)]
     L.moe_ipc_close.argtypes = [vp]
@@ -318,6 +324,40 @@ def dispatch(x, instance_ids, num_instances, ep_world_size, quant_mode, mask=Non
             ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth), _ptr(out["expand_x"]),
             _ptr(out["dyn_scales"]), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]), _ptr(out["counts"]),
             _ptr(out["offsets"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def dispatch_route(instance_ids, num_instances, ep_world_size, hidden, quant_mode, mask=None, scales_len=0,
+                   workspace=None, out=None, stream=None):
+    """moe_dispatch_route: the routing outputs of moe_dispatch (expand_idx,
+    src_of_row, counts, offsets), no rows moved.  hidden, quant_mode and
+    scales_len are the later moe_ep_dispatch's (they size the workspace)."""
+    _req(instance_ids, "instance_ids", torch.int32)
+    bs, k = instance_ids.shape
+    dev = instance_ids.device
+    _opt(mask, "mask", torch.uint8, (bs, k))
+    rows = bs * k
+    if out is None:
+        out = dict(expand_idx=torch.empty((bs, k), dtype=torch.int32, device=dev),
+                   src_of_row=torch.empty((rows,), dtype=torch.int32, device=dev),
+                   counts=torch.empty((num_instances,), dtype=torch.int32, device=dev),
+                   offsets=torch.empty((num_instances + 1,), dtype=torch.int32, device=dev))
+    if not isinstance(out, dict):
+        raise TypeError("out must be a dict with expand_idx, src_of_row, counts and offsets")
+    _req(out.get("expand_idx"), "out['expand_idx']", torch.int32, (bs, k))
+    _req(out.get("src_of_row"), "out['src_of_row']", torch.int32, (rows,))
+    _req(out.get("counts"), "out['counts']", torch.int32, (num_instances,))
+    _req(out.get("offsets"), "out['offsets']", torch.int32, (num_instances + 1,))
+    p = DispatchParams(bs, int(hidden), k, int(ep_world_size), int(num_instances), int(quant_mode),
+                       int(scales_len), 1)
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(
+            dev, stream, dispatch_workspace_bytes(bs, hidden, k, ep_world_size, num_instances, quant_mode,
+                                                  scales_len))
+        _same_device(dev, ("mask", mask), ("workspace", ws), *((f"out['{n}']", t) for n, t in out.items()))
+        _check("moe_dispatch_route", lib.moe_dispatch_route(
+            ctypes.byref(p), _ptr(instance_ids), _ptr(mask), _ptr(out["expand_idx"]), _ptr(out["src_of_row"]),
+            _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
@@ -553,6 +593,75 @@ def ep_pull(p: EpParams, peer_rows, local_offsets, local_rows, workspace, stream
         _check("moe_ep_pull", lib.moe_ep_pull(ctypes.byref(p), _ptr(peer_rows), _ptr(local_offsets),
                                               _ptr(local_rows), _ptr(workspace), workspace.numel(),
                                               _stream(stream)))
+
+
+def ep_dispatch(p: EpParams, x, instance_ids, ep_world_size, quant_mode, route: dict, peer_rows, peer_scales,
+                peer_src, global_idx, workspace, mask=None, smooth=None, stream=None):
+    """moe_ep_dispatch: quantize this GPU's tokens and store every sent copy
+    into its owner's receive buffer.  route: dispatch_route's outputs."""
+    _req(x, "x", torch.bfloat16)
+    if x.dim() != 2 or x.shape[0] != p.bs:
+        raise ValueError(f"x must have shape ({p.bs}, H), got {tuple(x.shape)}")
+    H = x.shape[1]
+    dev = x.device
+    _req(instance_ids, "instance_ids", torch.int32, (p.bs, p.top_k))
+    _opt(mask, "mask", torch.uint8, (p.bs, p.top_k))
+    _check_scales(smooth, quant_mode, p.num_instances, H)
+    if not isinstance(route, dict):
+        raise TypeError("route must be dispatch_route's output dict")
+    _req(route.get("expand_idx"), "route['expand_idx']", torch.int32, (p.bs, p.top_k))
+    _req(route.get("offsets"), "route['offsets']", torch.int32, (p.num_instances + 1,))
+    _req(global_idx, "global_idx", torch.int32, (p.bs, p.top_k))
+    _ptr_table(peer_rows, "peer_rows")
+    if p.scale_bytes:
+        _ptr_table(peer_scales, "peer_scales")
+    if peer_src is not None:
+        _ptr_table(peer_src, "peer_src")
+    _req(workspace, "workspace", torch.uint8)
+    sl = 0 if smooth is None else smooth.numel()
+    dp = DispatchParams(p.bs, H, p.top_k, int(ep_world_size), p.num_instances, int(quant_mode), sl, 1)
+    _same_device(dev, ("instance_ids", instance_ids), ("mask", mask), ("smooth", smooth),
+                 ("route['expand_idx']", route["expand_idx"]), ("route['offsets']", route["offsets"]),
+                 ("global_idx", global_idx), ("peer_rows", peer_rows), ("peer_scales", peer_scales),
+                 ("peer_src", peer_src), ("workspace", workspace))
+    with torch.cuda.device(dev):
+        _check("moe_ep_dispatch", lib.moe_ep_dispatch(
+            ctypes.byref(dp), ctypes.byref(p), _ptr(x), _ptr(instance_ids), _ptr(mask), _ptr(smooth),
+            _ptr(route["expand_idx"]), _ptr(route["offsets"]), _ptr(peer_rows),
+            _ptr(peer_scales if p.scale_bytes else None), _ptr(peer_src), _ptr(global_idx), _ptr(workspace),
+            workspace.numel(), _stream(stream)))
+
+
+def ep_combine_add_rmsnorm(p: EpParams, peer_rows, global_idx, expert_scales, residual_x, gamma, norm_eps,
+                           workspace, shared_x=None, want_x_out=False, want_rstd=False, out=None, stream=None):
+    """moe_ep_combine_add_rmsnorm: the combine reading each copy's expert
+    output from the GPU that owns its row.  Returns a dict like
+    combine_add_rmsnorm."""
+    _ptr_table(peer_rows, "peer_rows")
+    _req(global_idx, "global_idx", torch.int32, (p.bs, p.top_k))
+    _req(residual_x, "residual_x", torch.bfloat16)
+    H = residual_x.shape[1]
+    _req(residual_x, "residual_x", torch.bfloat16, (p.bs, H))
+    dev = residual_x.device
+    _req(expert_scales, "expert_scales", torch.float32, (p.bs, p.top_k))
+    _req(gamma, "gamma", torch.bfloat16, (H,))
+    _opt(shared_x, "shared_x", torch.bfloat16, (p.bs, H))
+    _req(workspace, "workspace", torch.uint8)
+    if out is None:
+        out = dict(y=torch.empty((p.bs, H), dtype=torch.bfloat16, device=dev),
+                   x_out=torch.empty((p.bs, H), dtype=torch.bfloat16, device=dev) if want_x_out else None,
+                   rstd=torch.empty((p.bs,), dtype=torch.float32, device=dev) if want_rstd else None)
+    _check_combine_out(out, p.bs, H)
+    cp = CombineParams(p.bs, H, p.top_k, max(p.recv_rows, 1), float(norm_eps), 1)
+    _same_device(dev, ("peer_rows", peer_rows), ("global_idx", global_idx), ("expert_scales", expert_scales),
+                 ("gamma", gamma), ("shared_x", shared_x), ("workspace", workspace),
+                 *((f"out['{n}']", t) for n, t in out.items()))
+    with torch.cuda.device(dev):
+        _check("moe_ep_combine_add_rmsnorm", lib.moe_ep_combine_add_rmsnorm(
+            ctypes.byref(cp), ctypes.byref(p), _ptr(peer_rows), _ptr(global_idx), _ptr(expert_scales),
+            _ptr(shared_x), _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")),
+            _ptr(out.get("rstd")), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
 
 
 def ipc_export(t: torch.Tensor):

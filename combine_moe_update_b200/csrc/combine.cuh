@@ -32,6 +32,12 @@ struct CombineArgs {
     uint16_t *x_out;  // may be null
     float *rstd_out;  // may be null
     uint32_t *err;
+    // Expert parallelism across GPUs (EP kernels): expand_idx holds global
+    // rows; row g lives on GPU q with gbase[q] <= g < gbase[q + 1], at row
+    // g - gbase[q] of peer_rows[q] (peer memory, plain loads).
+    const uint16_t *const *peer_rows;
+    const int32_t *gbase;  // [G + 1]
+    int gpus, recv_rows;
 };
 
 // Threads of a block for NV vectors of 8 elements per block and VECS vectors
@@ -50,12 +56,15 @@ __host__ __device__ inline int cb_threads(int NV, int vecs) {
 // none), the shared row and the residual row -- so a vector costs one round
 // trip to memory.  NORM false: the plain combine (combineOut to y; no
 // residual, no norm).
-template <int KMAX, bool SHARED, int NT, bool NORM, int SPLIT>
+// EP: the rows come from the GPUs that own them (expert parallelism across
+// GPUs, the AllToAllV back fused into the gather).
+template <int KMAX, bool SHARED, int NT, bool NORM, int SPLIT, bool EP = false>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(CombineArgs a) {
     constexpr int VECS = SPLIT == 1 ? 4 : 2;
     constexpr int NW = NT / 32;
     __shared__ int s_row[16];
     __shared__ float s_w[16];
+    __shared__ const uint16_t *s_src[EP ? 16 : 1];
     __shared__ float s_red[NW];
     __shared__ float s_part;
     const int t = threadIdx.x;
@@ -75,6 +84,22 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
         if (row < -1 || row >= a.expand_rows) {
             raise_error(a.err, kDevBadId);
             row = -1;
+        }
+        if constexpr (EP) {  // the owner of global row `row` (the last GPU whose first row is <= row)
+            if (row >= 0) {
+                int lo = 0, hi = a.gpus - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (a.gbase[mid] <= row) lo = mid; else hi = mid - 1;
+                }
+                const int prow = row - a.gbase[lo];
+                if (prow >= a.recv_rows || row >= a.gbase[a.gpus]) {
+                    raise_error(a.err, kDevBadId);
+                    row = -1;
+                } else {
+                    s_src[t] = a.peer_rows[lo] + (size_t)prow * H;
+                }
+            }
         }
         s_row[t] = row;
         s_w[t] = row >= 0 ? w : 0.0f;  // a pruned copy weighs nothing
@@ -99,24 +124,31 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
 #pragma unroll
         for (int e = 0; e < 8; ++e) xs[j][e] = 0.0f;
         if (pl >= Vh) continue;
-        uint4 rv[KMAX];
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            if (row[k] >= 0) rv[k] = ld_stream(a.expand_x + (size_t)row[k] * H + p * 8);
-        uint4 res = make_uint4(0, 0, 0, 0);
-        if constexpr (NORM) res = ld_stream(a.residual + tok + p * 8);
-        uint4 sh = make_uint4(0, 0, 0, 0);
-        if constexpr (SHARED) sh = ld_stream(a.shared_x + tok + p * 8);
+        uint4 res = make_uint4(0, 0, 0, 0), sh = make_uint4(0, 0, 0, 0);
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        // at most eight rows in flight per thread (sixteen spill the registers); the sum stays in k order
+        constexpr int CH = KMAX < 8 ? KMAX : 8;
 #pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            if (row[k] < 0) continue;
-            float f[8];
-            unpack8(rv[k], f);
+        for (int k0 = 0; k0 < KMAX; k0 += CH) {
+            uint4 rv[CH];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(wk[k], f[e], acc[e]);
+            for (int k = 0; k < CH; ++k)
+                if (row[k0 + k] >= 0)
+                    rv[k] = ld_stream((EP ? s_src[k0 + k] : a.expand_x + (size_t)row[k0 + k] * H) + p * 8);
+            if (k0 == 0) {
+                if constexpr (NORM) res = ld_stream(a.residual + tok + p * 8);
+                if constexpr (SHARED) sh = ld_stream(a.shared_x + tok + p * 8);
+            }
+#pragma unroll
+            for (int k = 0; k < CH; ++k) {
+                if (row[k0 + k] < 0) continue;
+                float f[8];
+                unpack8(rv[k], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wk[k0 + k], f[e], acc[e]);
+            }
         }
         if constexpr (SHARED) {
             float f[8];

@@ -21,6 +21,7 @@ constexpr bool kSkipOneCopy = false;
 constexpr uint32_t kDevBadId = 1u;     // id or row index out of range: item dropped
 constexpr uint32_t kDevBadTable = 2u;  // mapping table broke its restrictions
 constexpr uint32_t kDevTimeout = 4u;   // a bounded wait gave up
+constexpr uint32_t kDevCapacity = 8u;  // expert parallelism: a receive buffer too small, rows beyond it dropped
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ void raise_error(uint32_t *err, uint32_t bits) { atomicOr(err, bits); }

@@ -58,7 +58,48 @@ struct DispatchArgs {
     int32_t *counts;
     int32_t *offsets;
     uint32_t *err;
+    // The call's first kernel reads nothing before griddepcontrol.wait (set
+    // when a scatter kernel runs without a route kernel of its own call).
+    int wait_first;
+    // Expert parallelism across GPUs (peer_x null: rows go to expand_x on
+    // this GPU).  Copy (instance e, local row r) goes to GPU q = e / ep_el,
+    // row gstart[e] + (r - offsets[e]) - gbase[q] of q's receive buffer.
+    uint8_t *const *peer_x;      // [G] receive buffers
+    uint8_t *const *peer_sc;     // [G] their scales (modes 2 to 4)
+    int32_t *const *peer_src;    // [G] copy ids, optional
+    const int32_t *gstart;       // [E] global row of this GPU's first copy of each instance
+    const int32_t *gbase;        // [G + 1] first global row of every GPU
+    int32_t *global_idx;         // [bs, K] out: every copy's global row (-1 if not sent)
+    int ep_el, ep_recv_rows, ep_src_base;
+    int scale_bytes;             // bytes of one row's scales in the receive buffers
 };
+
+// Where a copy's row goes: the row buffer, its scales and the row in them.
+struct RowDst {
+    uint8_t *x;
+    uint8_t *sc;
+    int row;
+};
+
+// Copy j of instance e at local row r.  On one GPU, row r of expand_x; with
+// expert parallelism, the owner's receive buffer (also records the copy's
+// global row and id there).  False if the row falls past the receive buffer
+// (reported; the copy is dropped).
+__device__ __forceinline__ bool copy_dst(const DispatchArgs &a, int e, int r, int j, RowDst &d) {
+    if (a.peer_x == nullptr) {
+        d.x = reinterpret_cast<uint8_t *>(a.expand_x);
+        d.sc = reinterpret_cast<uint8_t *>(a.dyn_scales);
+        d.row = r;
+        return true;
+    }
+    const int q = e / a.ep_el;
+    const int grow = a.gstart[e] + (r - a.offsets[e]);
+    d.row = grow - a.gbase[q];
+    if (d.row < 0 || d.row >= a.ep_recv_rows) return false;
+    d.x = a.peer_x[q];
+    d.sc = a.peer_sc != nullptr ? a.peer_sc[q] : nullptr;
+    return true;
+}
 
 // Key of copy j: its instance if it is sent, -1 if masked out, -2 if its id
 // is out of range (then it is dropped and reported).
@@ -684,27 +725,41 @@ __device__ __forceinline__ void quantize_local(const uint64_t (&xf)[kDpVecs][4],
 
 // Write this thread's codes (and scales) of one row.
 template <int MODE, int NT>
-__device__ __forceinline__ void write_row(const DispatchArgs &a, int row, int V, const uint2 (&qv)[kDpVecs],
+__device__ __forceinline__ void write_row(const DispatchArgs &a, const RowDst &d, int V, const uint2 (&qv)[kDpVecs],
                                           const float (&seg)[kDpVecs], float row_scale) {
-    const int t = threadIdx.x, H = a.hidden;
-    uint8_t *dst = reinterpret_cast<uint8_t *>(a.expand_x) + (size_t)row * H;
+    const int t = threadIdx.x, H = a.hidden, row = d.row;
+    uint8_t *dst = d.x + (size_t)row * H;
 #pragma unroll
     for (int q = 0; q < kDpVecs; ++q) {
         const int p = t + q * NT;
         if (p >= V) continue;
         *reinterpret_cast<uint2 *>(dst + p * 8) = qv[q];
         if constexpr (MODE == 3) {
-            if ((t & 15) == 0) reinterpret_cast<float *>(a.dyn_scales)[(size_t)row * a.tiles + (p >> 4)] = seg[q];
+            if ((t & 15) == 0) reinterpret_cast<float *>(d.sc)[(size_t)row * a.tiles + (p >> 4)] = seg[q];
         }
         if constexpr (MODE == 4) {
-            if ((t & 3) == 0)
-                reinterpret_cast<uint8_t *>(a.dyn_scales)[(size_t)row * (H >> 5) + (p >> 2)] =
-                    (uint8_t)__float_as_int(seg[q]);
+            if ((t & 3) == 0) d.sc[(size_t)row * (H >> 5) + (p >> 2)] = (uint8_t)__float_as_int(seg[q]);
         }
     }
     if constexpr (MODE == 2) {
-        if (t == 0) reinterpret_cast<float *>(a.dyn_scales)[row] = row_scale;
+        if (t == 0) reinterpret_cast<float *>(d.sc)[row] = row_scale;
     }
+}
+
+// With expert parallelism, thread t < K of a token block records copy t's
+// global row and, at its owner, the copy's id in the group.
+__device__ __forceinline__ void ep_record(const DispatchArgs &a, int j, int e, int r) {
+    if (a.peer_x == nullptr) return;
+    int g = -1;
+    if (r >= 0) {
+        const int q = e / a.ep_el;
+        g = a.gstart[e] + (r - a.offsets[e]);
+        const int prow = g - a.gbase[q];
+        if (prow < 0) raise_error(a.err, kDevBadId);  // the plan does not match this GPU's routing
+        else if (prow >= a.ep_recv_rows) raise_error(a.err, kDevCapacity);
+        else if (a.peer_src != nullptr) a.peer_src[q][prow] = a.ep_src_base + j;
+    }
+    a.global_idx[j] = g;
 }
 
 // This thread's vectors of a bf16 row (zeros past the row's end).
@@ -724,7 +779,7 @@ __device__ __forceinline__ void load_row(const uint16_t *row, int V, uint4 (&xv)
 template <int MODE, int NT, bool FUSED>
 __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
     __shared__ float s_red[NT / 32];
-    __shared__ int s_row[16];
+    __shared__ int s_row[16], s_inst[16];
     __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
     const int i = blockIdx.x, t = threadIdx.x;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
@@ -735,6 +790,8 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         // flight while the block routes its copies.
         block_route_clear<NT>(rs, a.num_instances);
         pdl_wait();
+    } else if (a.wait_first) {
+        pdl_wait();  // no route kernel of this call ran first (the rows were routed by an earlier call)
     }
 
     // FUSED: after the wait.  Otherwise this kernel follows the call's route
@@ -790,21 +847,28 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
     } else {
         quantize();  // while the route kernel is still sorting
         pdl_wait();  // the rows come from route_kernel
-        if (t < K) s_row[t] = a.expand_idx[i * K + t];
+        if (t < K) {
+            const int r = a.expand_idx[i * K + t];
+            s_row[t] = r;
+            s_inst[t] = a.peer_x != nullptr ? a.ids[i * K + t] : 0;
+            ep_record(a, i * K + t, s_inst[t], r);
+        }
         __syncthreads();
     }
     for (int k = 0; k < K; ++k) {
         const int row = FUSED ? rs.row[k] : s_row[k];
         if (row < 0) continue;
+        RowDst d;
+        if (!copy_dst(a, FUSED ? 0 : s_inst[k], row, i * K + k, d)) continue;
         if constexpr (MODE == 0) {
-            uint16_t *dst = reinterpret_cast<uint16_t *>(a.expand_x) + (size_t)row * H;
+            uint16_t *dst = reinterpret_cast<uint16_t *>(d.x) + (size_t)d.row * H;
 #pragma unroll
             for (int q = 0; q < kDpVecs; ++q) {
                 const int p = t + q * NT;
                 if (p < V) st_v4(dst + p * 8, xv[q]);
             }
         } else {
-            write_row<MODE, NT>(a, row, V, qv, seg, row_scale);
+            write_row<MODE, NT>(a, d, V, qv, seg, row_scale);
         }
     }
 }
@@ -858,6 +922,8 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         if (t == 0) mbar_init(&s_bar, 1);
         __syncthreads();
         pdl_wait();
+    } else if (a.wait_first) {
+        pdl_wait();  // no route kernel of this call ran first (the rows were routed by an earlier call)
     }
     // FUSED: after the wait.  Otherwise the call's route kernel runs first
     // and releases this kernel only after its own wait, so the call's inputs
@@ -938,13 +1004,19 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         }
         if (!FUSED && c == 0) {
             pdl_wait();  // the rows come from the route kernel
-            if (t < K) s_row[t] = a.expand_idx[i * K + t];
+            if (t < K) {
+                const int r = a.expand_idx[i * K + t];
+                s_row[t] = r;
+                if (a.peer_x != nullptr) ep_record(a, i * K + t, a.ids[i * K + t], r);
+            }
             __syncthreads();
         }
 #pragma unroll
         for (int q = 0; q < kDpVecs; ++q)
             if (swap) qv[q] = make_uint2(qv[q].y, qv[q].x);
-        write_row<MODE, NT>(a, FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], V, qv, seg, row_scale);
+        RowDst d;
+        if (copy_dst(a, s_key[c], FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], i * K + s_pos[c], d))
+            write_row<MODE, NT>(a, d, V, qv, seg, row_scale);
     }
 }
 

@@ -38,8 +38,6 @@
 
 namespace moe {
 
-constexpr uint32_t kDevCapacity = 8u;  // a receive buffer too small: rows beyond it dropped
-
 struct EpArgs {
     int bs, top_k, num_instances, gpus, rank;
     int row_bytes;    // bytes of one row (a multiple of 16)

@@ -228,7 +228,9 @@ cudaError_t launch_by_threads(const moe::DispatchArgs &a, cudaStream_t s) {
 
 // Small calls (at most kFusedRouteMax copies) use the instantiations whose
 // blocks route their own copies, and no route kernel runs.
-inline bool fused_route(const moe::DispatchArgs &a) { return a.bs * a.top_k <= moe::kFusedRouteMax; }
+inline bool fused_route(const moe::DispatchArgs &a) {
+    return a.bs * a.top_k <= moe::kFusedRouteMax && !a.wait_first;  // wait_first: routed by an earlier call
+}
 
 template <int MODE, int NT>
 struct TokenLaunch {
@@ -298,6 +300,32 @@ cudaError_t launch_combine_split(const moe::CombineArgs &a, cudaStream_t s) {
     if (a.shared_x)
         return split ? launch_combine_tok<KMAX, true, NORM, 2>(a, s) : launch_combine_tok<KMAX, true, NORM, 1>(a, s);
     return split ? launch_combine_tok<KMAX, false, NORM, 2>(a, s) : launch_combine_tok<KMAX, false, NORM, 1>(a, s);
+}
+
+// The combine that gathers its rows from the GPUs that own them (one block per token).
+template <int KMAX, bool SHARED, int NT>
+cudaError_t launch_combine_ep_nt(const moe::CombineArgs &a, cudaStream_t s) {
+    auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, true, 1, true>;
+    if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
+    return launch(kernel, a.bs, NT, 0, s, a);
+}
+
+template <int KMAX, bool SHARED>
+cudaError_t launch_combine_ep_tok(const moe::CombineArgs &a, cudaStream_t s) {
+    switch (moe::cb_threads(a.hidden >> 3, 4)) {
+        case 64: return launch_combine_ep_nt<KMAX, SHARED, 64>(a, s);
+        case 128: return launch_combine_ep_nt<KMAX, SHARED, 128>(a, s);
+        case 192: return launch_combine_ep_nt<KMAX, SHARED, 192>(a, s);
+        case 224: return launch_combine_ep_nt<KMAX, SHARED, 224>(a, s);
+        default: return launch_combine_ep_nt<KMAX, SHARED, 256>(a, s);
+    }
+}
+
+cudaError_t launch_combine_ep(const moe::CombineArgs &a, int top_k, cudaStream_t s) {
+    const bool sh = a.shared_x != nullptr;
+    if (top_k <= 4) return sh ? launch_combine_ep_tok<4, true>(a, s) : launch_combine_ep_tok<4, false>(a, s);
+    if (top_k <= 8) return sh ? launch_combine_ep_tok<8, true>(a, s) : launch_combine_ep_tok<8, false>(a, s);
+    return sh ? launch_combine_ep_tok<16, true>(a, s) : launch_combine_ep_tok<16, false>(a, s);
 }
 
 template <bool NORM>
@@ -400,6 +428,96 @@ moe_status moe_dispatch_workspace_size(const moe_dispatch_params *p, size_t *byt
     return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The arguments every dispatch kernel shares (pointer checks done by the caller).
+moe::DispatchArgs dispatch_args(const moe_dispatch_params &p, const void *x, const int32_t *instance_ids,
+                                const uint8_t *mask, const float *smooth_scales, void *expand_x, void *dyn_scales,
+                                int32_t *expand_idx, int32_t *src_of_row, int32_t *expert_counts,
+                                int32_t *expert_offsets, void *workspace) {
+    moe::DispatchArgs a = {};
+    a.bs = total_tokens(p.bs, p.sources);  // the kernels see every source rank's tokens
+    a.hidden = p.hidden;
+    a.top_k = p.top_k;
+    a.num_instances = p.num_instances;
+    a.tiles = (p.hidden + 127) / 128;
+    a.k_magic = moe::div_magic((uint32_t)p.top_k);
+    a.x = reinterpret_cast<const uint16_t *>(x);
+    a.ids = instance_ids;
+    a.mask = mask;
+    a.smooth = smooth_scales;
+    a.scales_len = p.scales_len;
+    a.expand_x = expand_x;
+    a.dyn_scales = dyn_scales;
+    a.expand_idx = expand_idx;
+    a.src_of_row = src_of_row;
+    a.counts = expert_counts;
+    a.offsets = expert_offsets;
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    return a;
+}
+
+// The route kernels: one pass up to kRouteSinglePassMax copies, three passes
+// (with the slice table in the workspace) beyond.
+cudaError_t launch_route(const moe::DispatchArgs &a, int num_instances, void *workspace, cudaStream_t s) {
+    const int copies = a.bs * a.top_k;
+    if (copies <= kRouteSinglePassMax) {
+        const int slices = moe::route_slices(copies);
+        const size_t rsmem = moe::route_smem_bytes(num_instances);
+        if (!ensure_smem(moe::route_kernel, rsmem)) return cudaErrorInvalidValue;
+        return launch(moe::route_kernel, slices, moe::kRtThreads, rsmem, s, a);
+    }
+    const int S = moe::route_large_slices(copies), E = num_instances;
+    int *tab = reinterpret_cast<int *>(reinterpret_cast<unsigned char *>(workspace) + kWorkspaceBytes);
+    int *tot = tab + (size_t)S * E;
+    const size_t hsmem = (size_t)E * sizeof(int), psmem = moe::route_place_smem_bytes(E);
+    if (!ensure_smem(moe::route_hist_kernel, hsmem) || !ensure_smem(moe::route_place_kernel, psmem))
+        return cudaErrorInvalidValue;
+    cudaError_t e = launch(moe::route_hist_kernel, S, moe::kRtThreads, hsmem, s, a, tab);
+    if (e == cudaSuccess) e = launch(moe::route_scan_kernel, (E + 1023) / 1024, 1024, 0, s, a, tab, tot, S);
+    if (e == cudaSuccess)
+        e = launch(moe::route_place_kernel, S, moe::kRtThreads, psmem, s, a, (const int *)tab, (const int *)tot);
+    return e;
+}
+
+// The quantize-and-scatter kernel for the mode and the scales' shape.
+cudaError_t launch_scatter(const moe::DispatchArgs &a, const moe_dispatch_params &p, cudaStream_t s) {
+    // scales that depend on the destination instance (a row per instance) need
+    // the per-copy kernel; one coefficient or one per column is per token
+    const bool per_instance = a.smooth != nullptr && p.scales_len > p.hidden;
+    if (per_instance) {
+        switch (p.quant_mode) {
+            case 1: return launch_dispatch_token_smooth<1>(a, s);
+            case 2: return launch_dispatch_token_smooth<2>(a, s);
+            case 3: return launch_dispatch_token_smooth<3>(a, s);
+        }
+        return cudaErrorInvalidValue;
+    }
+    switch (p.quant_mode) {
+        case 0: return launch_dispatch_token<0>(a, s);
+        case 1: return launch_dispatch_token<1>(a, s);
+        case 2: return launch_dispatch_token<2>(a, s);
+        case 3: return launch_dispatch_token<3>(a, s);
+        case 4: return launch_dispatch_token<4>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// Pointer rules shared by moe_dispatch and moe_ep_dispatch (the outputs they write differ).
+bool dispatch_inputs_ok(const moe_dispatch_params &p, const void *x, const int32_t *instance_ids,
+                        const float *smooth_scales) {
+    if (!x || !instance_ids) return false;
+    if ((smooth_scales != nullptr) != (p.scales_len > 0)) return false;
+    return aligned(x, 16) && aligned(instance_ids, 4) &&
+           (!smooth_scales || aligned(smooth_scales, p.scales_len == 1 ? 4 : 16));
+}
+
+}  // namespace
+
+extern "C" {
+
 moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32_t *instance_ids,
                         const uint8_t *mask, const float *smooth_scales, void *expand_x, void *dyn_scales,
                         int32_t *expand_idx, int32_t *src_of_row, int32_t *expert_counts, int32_t *expert_offsets,
@@ -408,79 +526,40 @@ moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, const int32
     moe_status st = valid_dispatch(*p);
     if (st != MOE_OK) return st;
     const int mode = p->quant_mode;
-    if (!x || !instance_ids || !expand_x || !expand_idx || !src_of_row || !expert_counts || !expert_offsets)
-        return MOE_ERR_INVALID_ARG;
+    if (!dispatch_inputs_ok(*p, x, instance_ids, smooth_scales)) return MOE_ERR_INVALID_ARG;
+    if (!expand_x || !expand_idx || !src_of_row || !expert_counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
     if ((mode == 0 || mode == 1) != (dyn_scales == nullptr)) return MOE_ERR_INVALID_ARG;  // no scales sent
-    if ((smooth_scales != nullptr) != (p->scales_len > 0)) return MOE_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(instance_ids, 4) || !aligned(expand_idx, 4) ||
-        !aligned(src_of_row, 4) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
-        (smooth_scales && !aligned(smooth_scales, p->scales_len == 1 ? 4 : 16)) ||
+    if (!aligned(expand_x, 16) || !aligned(expand_idx, 4) || !aligned(src_of_row, 4) ||
+        !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
         ((mode == 2 || mode == 3) && !aligned(dyn_scales, 4)))
         return MOE_ERR_INVALID_ARG;
     if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < dispatch_workspace_bytes(*p))
         return MOE_ERR_WORKSPACE;
-    moe::DispatchArgs a;
-    a.bs = total_tokens(p->bs, p->sources);  // the kernels see every source rank's tokens
-    a.hidden = p->hidden;
-    a.top_k = p->top_k;
-    a.num_instances = p->num_instances;
-    a.tiles = (p->hidden + 127) / 128;
-    a.k_magic = moe::div_magic((uint32_t)p->top_k);
-    a.x = reinterpret_cast<const uint16_t *>(x);
-    a.ids = instance_ids;
-    a.mask = mask;
-    a.smooth = smooth_scales;
-    a.scales_len = p->scales_len;
-    a.expand_x = expand_x;
-    a.dyn_scales = dyn_scales;
-    a.expand_idx = expand_idx;
-    a.src_of_row = src_of_row;
-    a.counts = expert_counts;
-    a.offsets = expert_offsets;
-    a.err = reinterpret_cast<uint32_t *>(workspace);
+    const moe::DispatchArgs a = dispatch_args(*p, x, instance_ids, mask, smooth_scales, expand_x, dyn_scales,
+                                              expand_idx, src_of_row, expert_counts, expert_offsets, workspace);
     cudaStream_t s = as_stream(cuda_stream);
+    // up to kFusedRouteMax copies the scatter blocks route their own copies (no route kernel)
+    if (a.bs * a.top_k > moe::kFusedRouteMax && launch_route(a, p->num_instances, workspace, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_scatter(a, *p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
-    const int copies = a.bs * p->top_k;
-    if (copies <= moe::kFusedRouteMax) {
-        // the scatter blocks route their own copies (no route kernel)
-    } else if (copies <= kRouteSinglePassMax) {
-        const int slices = moe::route_slices(copies);
-        const size_t rsmem = moe::route_smem_bytes(p->num_instances);
-        if (!ensure_smem(moe::route_kernel, rsmem)) return MOE_ERR_CUDA;
-        if (launch(moe::route_kernel, slices, moe::kRtThreads, rsmem, s, a) != cudaSuccess) return MOE_ERR_CUDA;
-    } else {
-        const int S = moe::route_large_slices(copies), E = p->num_instances;
-        int *tab = reinterpret_cast<int *>(reinterpret_cast<unsigned char *>(workspace) + kWorkspaceBytes);
-        int *tot = tab + (size_t)S * E;
-        const size_t hsmem = (size_t)E * sizeof(int), psmem = moe::route_place_smem_bytes(E);
-        if (!ensure_smem(moe::route_hist_kernel, hsmem) || !ensure_smem(moe::route_place_kernel, psmem))
-            return MOE_ERR_CUDA;
-        if (launch(moe::route_hist_kernel, S, moe::kRtThreads, hsmem, s, a, tab) != cudaSuccess ||
-            launch(moe::route_scan_kernel, (E + 1023) / 1024, 1024, 0, s, a, tab, tot, S) != cudaSuccess ||
-            launch(moe::route_place_kernel, S, moe::kRtThreads, psmem, s, a, (const int *)tab, (const int *)tot) !=
-                cudaSuccess)
-            return MOE_ERR_CUDA;
-    }
-    cudaError_t e = cudaSuccess;
-    // scales that depend on the destination instance (a row per instance) need
-    // the per-copy kernel; one coefficient or one per column is per token
-    const bool per_instance = smooth_scales && p->scales_len > p->hidden;
-    if (per_instance) {
-        switch (mode) {
-            case 1: e = launch_dispatch_token_smooth<1>(a, s); break;
-            case 2: e = launch_dispatch_token_smooth<2>(a, s); break;
-            case 3: e = launch_dispatch_token_smooth<3>(a, s); break;
-        }
-    } else {
-        switch (mode) {
-            case 0: e = launch_dispatch_token<0>(a, s); break;
-            case 1: e = launch_dispatch_token<1>(a, s); break;
-            case 2: e = launch_dispatch_token<2>(a, s); break;
-            case 3: e = launch_dispatch_token<3>(a, s); break;
-            case 4: e = launch_dispatch_token<4>(a, s); break;
-        }
-    }
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+moe_status moe_dispatch_route(const moe_dispatch_params *p, const int32_t *instance_ids, const uint8_t *mask,
+                              int32_t *expand_idx, int32_t *src_of_row, int32_t *expert_counts,
+                              int32_t *expert_offsets, void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr) return MOE_ERR_INVALID_ARG;
+    moe_status st = valid_dispatch(*p);
+    if (st != MOE_OK) return st;
+    if (!instance_ids || !expand_idx || !src_of_row || !expert_counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (!aligned(instance_ids, 4) || !aligned(expand_idx, 4) || !aligned(src_of_row, 4) ||
+        !aligned(expert_counts, 4) || !aligned(expert_offsets, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes) || workspace_bytes < dispatch_workspace_bytes(*p))
+        return MOE_ERR_WORKSPACE;
+    const moe::DispatchArgs a = dispatch_args(*p, nullptr, instance_ids, mask, nullptr, nullptr, nullptr, expand_idx,
+                                              src_of_row, expert_counts, expert_offsets, workspace);
+    return launch_route(a, p->num_instances, workspace, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK
+                                                                                                : MOE_ERR_CUDA;
 }
 
 // --------------------------------------------------------------- combine ---
@@ -503,7 +582,7 @@ moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expa
         return MOE_ERR_INVALID_ARG;
     if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
 
-    moe::CombineArgs a;
+    moe::CombineArgs a = {};
     a.bs = total_tokens(p->bs, p->sources);
     a.hidden = p->hidden;
     a.top_k = p->top_k;
@@ -818,6 +897,85 @@ moe_status moe_ep_pull(const moe_ep_params *p, void *const *peer_rows, const int
                   (const int32_t *)nullptr) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_dispatch(const moe_dispatch_params *p, const moe_ep_params *ep, const void *x,
+                           const int32_t *instance_ids, const uint8_t *mask, const float *smooth_scales,
+                           const int32_t *expand_idx, const int32_t *expert_offsets, void *const *peer_rows,
+                           void *const *peer_scales, int32_t *const *peer_src, int32_t *global_idx,
+                           void *ep_workspace, size_t ep_ws_bytes, void *cuda_stream) {
+    if (p == nullptr || ep == nullptr || !valid_ep(*ep)) return MOE_ERR_INVALID_ARG;
+    moe_status st = valid_dispatch(*p);
+    if (st != MOE_OK) return st;
+    const int mode = p->quant_mode;
+    // one source per GPU; the EP parameters describe the same call
+    if (p->sources > 1 || ep->bs != p->bs || ep->top_k != p->top_k || ep->num_instances != p->num_instances)
+        return MOE_ERR_INVALID_ARG;
+    if (ep->row_bytes != (mode == 0 ? 2 : 1) * p->hidden) return MOE_ERR_INVALID_ARG;
+    const int sb = mode == 2 ? 4 : mode == 3 ? 4 * ((p->hidden + 127) / 128) : mode == 4 ? p->hidden / 32 : 0;
+    if (ep->scale_bytes != sb) return MOE_ERR_INVALID_ARG;
+    if (!dispatch_inputs_ok(*p, x, instance_ids, smooth_scales)) return MOE_ERR_INVALID_ARG;
+    if (!expand_idx || !expert_offsets || !peer_rows || !global_idx || ((sb > 0) != (peer_scales != nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(expand_idx, 4) || !aligned(expert_offsets, 4) || !aligned(global_idx, 4) || !aligned(peer_rows, 8) ||
+        (peer_scales && !aligned(peer_scales, 8)) || (peer_src && !aligned(peer_src, 8)))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(ep_workspace, ep_ws_bytes) || ep_ws_bytes < ep_workspace_bytes(*ep))
+        return MOE_ERR_WORKSPACE;
+    moe::DispatchArgs a = dispatch_args(*p, x, instance_ids, mask, smooth_scales, nullptr, nullptr,
+                                        const_cast<int32_t *>(expand_idx), nullptr, nullptr,
+                                        const_cast<int32_t *>(expert_offsets), ep_workspace);
+    const moe::EpArgs plan = ep_args(*ep, ep_workspace);
+    a.wait_first = 1;  // this call's scatter is its first kernel
+    a.peer_x = reinterpret_cast<uint8_t *const *>(peer_rows);
+    a.peer_sc = reinterpret_cast<uint8_t *const *>(peer_scales);
+    a.peer_src = peer_src;
+    a.gstart = plan.gstart;
+    a.gbase = plan.base;
+    a.global_idx = global_idx;
+    a.ep_el = ep->num_instances / ep->gpus;
+    a.ep_recv_rows = ep->recv_rows;
+    a.ep_src_base = ep->rank * ep->bs * ep->top_k;
+    a.scale_bytes = sb;
+    return launch_scatter(a, *p, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_combine_add_rmsnorm(const moe_combine_params *p, const moe_ep_params *ep, void *const *peer_rows,
+                                      const int32_t *global_idx, const float *expert_scales, const void *shared_x,
+                                      const void *residual_x, const void *gamma, void *y, void *x_out,
+                                      float *rstd_out, void *ep_workspace, size_t ep_ws_bytes,
+                                      void *cuda_stream) {
+    if (p == nullptr || ep == nullptr || !valid_combine(*p) || !valid_ep(*ep)) return MOE_ERR_INVALID_ARG;
+    if (p->sources > 1 || ep->bs != p->bs || ep->top_k != p->top_k || ep->row_bytes != 2 * p->hidden)
+        return MOE_ERR_INVALID_ARG;
+    if (!peer_rows || !global_idx || !expert_scales || !residual_x || !gamma || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned(peer_rows, 8) || !aligned(residual_x, 16) || !aligned(gamma, 16) || !aligned(y, 16) ||
+        (shared_x && !aligned(shared_x, 16)) || (x_out && !aligned(x_out, 16)) || !aligned(global_idx, 4) ||
+        !aligned(expert_scales, 4) || (rstd_out && !aligned(rstd_out, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(ep_workspace, ep_ws_bytes) || ep_ws_bytes < ep_workspace_bytes(*ep))
+        return MOE_ERR_WORKSPACE;
+    const moe::EpArgs plan = ep_args(*ep, ep_workspace);
+    moe::CombineArgs a = {};
+    a.bs = p->bs;
+    a.hidden = p->hidden;
+    a.top_k = p->top_k;
+    a.expand_rows = 0x7fffffff;  // global rows: bounded by the plan's last base instead
+    a.norm_eps = p->norm_eps;
+    a.expand_idx = global_idx;
+    a.scales = expert_scales;
+    a.shared_x = reinterpret_cast<const uint16_t *>(shared_x);
+    a.residual = reinterpret_cast<const uint16_t *>(residual_x);
+    a.gamma = reinterpret_cast<const uint16_t *>(gamma);
+    a.y = reinterpret_cast<uint16_t *>(y);
+    a.x_out = reinterpret_cast<uint16_t *>(x_out);
+    a.rstd_out = rstd_out;
+    a.err = plan.err;
+    a.peer_rows = reinterpret_cast<const uint16_t *const *>(peer_rows);
+    a.gbase = plan.base;
+    a.gpus = ep->gpus;
+    a.recv_rows = ep->recv_rows;
+    return launch_combine_ep(a, p->top_k, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_ipc_export(const void *dev_ptr, void *handle, uint64_t *offset) {

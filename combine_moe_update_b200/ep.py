@@ -10,16 +10,20 @@ the group's rows are those of the multi-source dispatch on one GPU (ordered
 by instance, source GPU, token, k) and GPU q's receive buffer is the stretch
 of that order its instances own.
 
-A layer on every GPU g:
-  local_dispatch   update_expert + dispatch of its own tokens over all E
-                   instances (the library's kernels);
+A layer on every GPU g (fused, the default):
+  route            update_expert + the routing half of the dispatch
+                   (moe_dispatch_route) of its own tokens over all E
+                   instances;
   gather counts    every GPU's per-instance counts into counts_all [G, E];
-  plan, push       each local row into its owner's receive buffer through
-                   peer memory (moe_ep_plan, moe_ep_push), then a barrier;
+  plan, dispatch   moe_ep_plan, then moe_ep_dispatch: each token is
+                   quantized once and its copies stored straight into their
+                   owners' receive buffers through peer memory; a barrier;
   expert step      on the receive buffer (the caller's), then a barrier;
-  pull, combine    each local row's output back from its owner
-                   (moe_ep_pull), then combine+Add+RMSNorm with the local
-                   expand_idx.
+  combine          moe_ep_combine_add_rmsnorm: the weighted sum reads each
+                   copy's expert output from its owner's buffer.
+The two-step form (fused=False) dispatches into a local buffer first and
+moves the rows with moe_ep_push, and brings the outputs back with
+moe_ep_pull before the one-GPU combine; it computes the same rows.
 The barriers are one-element all-reduces on the stream, so every kernel
 before them has finished on every GPU when the next step starts.
 
@@ -58,6 +62,7 @@ class EPRank:
         self.bal = torch.empty((bs, top_k), dtype=torch.int32, device=dev)
         self.bm = torch.empty((bs, top_k), dtype=torch.uint8, device=dev)
         self.d = B.alloc_dispatch_outputs(bs, hidden, top_k, num_instances, quant_mode, dev)
+        self.route_out = {n: self.d[n] for n in ("expand_idx", "src_of_row", "counts", "offsets")}
         self.recv_x = torch.empty((self.cap, hidden), dtype=B.expand_dtype(quant_mode), device=dev)
         self.recv_scales = (torch.empty((self.cap, scale_bytes), dtype=torch.uint8, device=dev)
                             if scale_bytes else None)
@@ -78,6 +83,26 @@ class EPRank:
                         prune_threshold=prune_threshold, workspace=self.ws, out=(self.bal, self.bm), stream=stream)
         B.dispatch(x, self.bal, self.E, self.ep_world_size, self.quant_mode, mask=self.bm, smooth=smooth,
                    workspace=self.ws, out=self.d, stream=stream)
+
+    def route(self, expert_ids, table, expert_scales=None, prune_threshold=0.0, active_mask=None, scales_len=0,
+              stream=None):
+        """update_expert + moe_dispatch_route of this GPU's own tokens (fused form)."""
+        B.update_expert(expert_ids, table, self.ep_world_size, expert_scales=expert_scales, active_mask=active_mask,
+                        prune_threshold=prune_threshold, workspace=self.ws, out=(self.bal, self.bm), stream=stream)
+        B.dispatch_route(self.bal, self.E, self.ep_world_size, self.hidden, self.quant_mode, mask=self.bm,
+                         scales_len=scales_len, workspace=self.ws, out=self.route_out, stream=stream)
+
+    def ep_dispatch(self, x, tables: "PeerTables", smooth=None, stream=None):
+        """moe_ep_dispatch: this GPU's copies into their owners' receive buffers."""
+        B.ep_dispatch(self.p_push, x, self.bal, self.ep_world_size, self.quant_mode, self.route_out, tables.recv_x,
+                      tables.recv_scales, tables.recv_src, self.global_idx, self.ep_ws, mask=self.bm, smooth=smooth,
+                      stream=stream)
+
+    def ep_combine(self, tables: "PeerTables", expert_scales, residual, gamma, norm_eps, shared_x=None, out=None,
+                   stream=None):
+        """moe_ep_combine_add_rmsnorm: combine+Add+RMSNorm reading the owners' expert outputs."""
+        return B.ep_combine_add_rmsnorm(self.p_pull, tables.expert_out, self.global_idx, expert_scales, residual,
+                                        gamma, norm_eps, self.ep_ws, shared_x=shared_x, out=out, stream=stream)
 
     def plan(self, stream=None):
         B.ep_plan(self.p_push, self.counts_all, self.recv_counts, self.recv_offsets, self.ep_ws, stream=stream)
@@ -121,7 +146,8 @@ class EmulatedGroup:
     GPU's memory, each step run for every GPU in turn.  No kernel waits on
     another, so the order on one stream is enough."""
 
-    def __init__(self, gpus, **kw):
+    def __init__(self, gpus, fused=True, **kw):
+        self.fused = fused
         self.ranks = [EPRank(gpus=gpus, rank=g, **kw) for g in range(gpus)]
         addr = lambda ts: None if ts[0] is None else [t.data_ptr() for t in ts]
         rs = self.ranks
@@ -131,16 +157,26 @@ class EmulatedGroup:
     def dispatch(self, inputs):
         """inputs[g]: the keyword arguments of EPRank.local_dispatch for GPU g."""
         for r, kw in zip(self.ranks, inputs):
-            r.local_dispatch(**kw)
+            if self.fused:
+                kw = dict(kw)
+                x, smooth = kw.pop("x"), kw.pop("smooth", None)
+                r.route(scales_len=0 if smooth is None else smooth.numel(), **kw)
+            else:
+                r.local_dispatch(**kw)
         counts_all = torch.stack([r.d["counts"] for r in self.ranks])  # the gather
         for r in self.ranks:
             r.counts_all.copy_(counts_all)
             r.plan()
-        for r in self.ranks:
-            r.push(self.tables)
+        for r, kw in zip(self.ranks, inputs):
+            if self.fused:
+                r.ep_dispatch(kw["x"], self.tables, smooth=kw.get("smooth"))
+            else:
+                r.push(self.tables)
 
     def combine(self, inputs):
         """inputs[g]: the keyword arguments of EPRank.combine for GPU g."""
+        if self.fused:
+            return [r.ep_combine(self.tables, **kw) for r, kw in zip(self.ranks, inputs)]
         for r in self.ranks:
             r.pull(self.tables)
         return [r.combine(**kw) for r, kw in zip(self.ranks, inputs)]
@@ -165,9 +201,9 @@ class ProcessGroupEP:
     peer mappings, no multicast object); call close() before the process
     group is destroyed."""
 
-    def __init__(self, group=None, **kw):
+    def __init__(self, group=None, fused=True, **kw):
         import torch.distributed as dist
-        self.group = group
+        self.group, self.fused = group, fused
         G, g = dist.get_world_size(group), dist.get_rank(group)
         self.r = EPRank(gpus=G, rank=g, **kw)
         self.flag = torch.zeros(1, dtype=torch.float32, device=self.r.device)
@@ -189,17 +225,28 @@ class ProcessGroupEP:
         self.tables = PeerTables(*(None if c[0] is None else c for c in cols), self.r.device)
 
     def dispatch(self, **kw):
-        """local dispatch, gather counts, plan, push, barrier: afterwards
-        self.r.recv_x[:received] holds this GPU's rows."""
-        self.r.local_dispatch(**kw)
+        """route (or local dispatch), gather counts, plan, EP dispatch (or
+        push), barrier: afterwards self.r.recv_x[:received] holds this GPU's
+        rows."""
+        if self.fused:
+            x, smooth = kw.pop("x"), kw.pop("smooth", None)
+            self.r.route(scales_len=0 if smooth is None else smooth.numel(), **kw)
+        else:
+            self.r.local_dispatch(**kw)
         gather_counts(self.r.d["counts"], self.r.counts_all, self.group)
         self.r.plan()
-        self.r.push(self.tables)
+        if self.fused:
+            self.r.ep_dispatch(x, self.tables, smooth=smooth)
+        else:
+            self.r.push(self.tables)
         group_barrier(self.flag, self.group)
 
     def combine(self, **kw):
-        """barrier (every expert output written), pull, combine."""
+        """barrier (every expert output written), then the EP combine (or
+        pull and the one-GPU combine)."""
         group_barrier(self.flag, self.group)
+        if self.fused:
+            return self.r.ep_combine(self.tables, **kw)
         self.r.pull(self.tables)
         return self.r.combine(**kw)
 

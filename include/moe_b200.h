@@ -217,6 +217,17 @@ MOE_API moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, con
                         int32_t *expert_counts, int32_t *expert_offsets, void *workspace,
                         size_t workspace_bytes, void *cuda_stream);
 
+/*
+ * The routing half of moe_dispatch alone: expand_idx, src_of_row,
+ * expert_counts and expert_offsets exactly as moe_dispatch writes them, with
+ * no row moved (the rows follow from moe_ep_dispatch once the group's counts
+ * are known).  Arguments, limits and errors as moe_dispatch.
+ */
+MOE_API moe_status moe_dispatch_route(const moe_dispatch_params *p, const int32_t *instance_ids,
+                                      const uint8_t *mask, int32_t *expand_idx, int32_t *src_of_row,
+                                      int32_t *expert_counts, int32_t *expert_offsets, void *workspace,
+                                      size_t workspace_bytes, void *cuda_stream);
+
 /* ------------------------------------------------------------------------ */
 /* moe_combine_add_rmsnorm -- aclnnMoeDistributeCombineAddRmsNorm            */
 /* ------------------------------------------------------------------------ */
@@ -483,6 +494,51 @@ MOE_API moe_status moe_ep_push(const moe_ep_params *p, const void *local_rows, c
  */
 MOE_API moe_status moe_ep_pull(const moe_ep_params *p, void *const *peer_rows, const int32_t *local_offsets,
                                void *local_rows, void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * Steps 1 and 3 fused: the rows are quantized once and stored straight into
+ * their owners' receive buffers (no local expand_x), after moe_dispatch_route
+ * and moe_ep_plan of the same layer on this GPU:
+ *   p              the moe_dispatch parameters of the route call (sources = 1;
+ *                  bs, top_k and num_instances equal to the EP parameters')
+ *   x, instance_ids, mask, smooth_scales: as moe_dispatch
+ *   expand_idx, expert_offsets: moe_dispatch_route's outputs
+ *   peer_rows, peer_scales, peer_src, global_idx: as moe_ep_push (row_bytes
+ *                  must be the mode's row size, scale_bytes its scale size)
+ *   ep_workspace   the EP workspace the plan wrote
+ * The receive buffers hold, row for row, what moe_dispatch with sources = G
+ * writes on one GPU.  Host errors: MOE_ERR_INVALID_ARG for parameters that do
+ * not agree or NULL / misaligned pointers, MOE_ERR_WORKSPACE.  Device errors
+ * (in the EP workspace): MOE_DEV_BAD_ID for out-of-range ids or a plan that
+ * does not match the routing, MOE_DEV_CAPACITY for rows past recv_rows
+ * (dropped).
+ */
+MOE_API moe_status moe_ep_dispatch(const moe_dispatch_params *p, const moe_ep_params *ep, const void *x,
+                                   const int32_t *instance_ids, const uint8_t *mask, const float *smooth_scales,
+                                   const int32_t *expand_idx, const int32_t *expert_offsets,
+                                   void *const *peer_rows, void *const *peer_scales, int32_t *const *peer_src,
+                                   int32_t *global_idx, void *ep_workspace, size_t ep_workspace_bytes,
+                                   void *cuda_stream);
+
+/*
+ * Steps 5 and the combine fused: moe_combine_add_rmsnorm whose top-K rows are
+ * read from the GPUs that own them: copy (i, k) with global row
+ * g = global_idx[i*K + k] reads row g - base[q] of peer_rows[q], q the owner
+ * of g (the plan's base), through a plain load over NVLink.
+ *   p           the combine parameters (sources = 1; bs and top_k equal to the EP parameters')
+ *   ep          row_bytes = 2H (bf16 expert outputs)
+ *   peer_rows   [G] device array of pointers: expert output buffers, [recv_rows, H] bf16 each
+ *   global_idx  [bs, K] int32 device: moe_ep_dispatch's (or moe_ep_push's) output
+ *   expert_scales, shared_x, residual_x, gamma, y, x_out, rstd_out: as moe_combine_add_rmsnorm
+ * Errors as moe_combine_add_rmsnorm; device errors go to the EP workspace
+ * (MOE_DEV_BAD_ID for a global row outside the group's rows).
+ */
+MOE_API moe_status moe_ep_combine_add_rmsnorm(const moe_combine_params *p, const moe_ep_params *ep,
+                                              void *const *peer_rows, const int32_t *global_idx,
+                                              const float *expert_scales, const void *shared_x,
+                                              const void *residual_x, const void *gamma, void *y, void *x_out,
+                                              float *rstd_out, void *ep_workspace, size_t ep_workspace_bytes,
+                                              void *cuda_stream);
 
 /*
  * Peer mappings for the pointer tables (CUDA IPC, no multicast object):

@@ -1,6 +1,9 @@
 """Expert parallelism across GPUs, emulated on one GPU: G ranks' buffers in
-this GPU's memory, the library's plan / push / pull kernels moving rows
-between them through the same pointer tables a real group uses.
+this GPU's memory, the library's EP kernels moving rows between them through
+the same pointer tables a real group uses -- fused (moe_dispatch_route,
+moe_ep_plan, moe_ep_dispatch storing each quantized copy at its owner,
+moe_ep_combine_add_rmsnorm reading the owners' outputs) and two-step
+(moe_dispatch, moe_ep_push, moe_ep_pull, moe_combine_add_rmsnorm).
 
 Across G GPUs every GPU is one source of its own tokens, so the group's rows
 must be exactly the single-GPU dispatch of all G * bs tokens (ordered by
@@ -63,10 +66,13 @@ def _inputs(seed, G, bs, H, E, K, ws, smooth):
     (4, 32, 1024, 64, 8, 16, 4, False),   # mxfp8
     (8, 24, 7168, 256, 8, 32, 2, True),   # the decode row length, eight GPUs
     (2, 512, 1024, 16, 8, 2, 1, True),    # static per-instance scales, 4096 copies per GPU
+    (2, 512, 2048, 64, 16, 8, 3, False),  # 8192 copies per GPU, per-tile int8
 ])
-def test_emulated_group_equals_one_gpu_dispatch(B, EP, G, bs, H, E, K, ws, mode, smooth):
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "two_step"])
+def test_emulated_group_equals_one_gpu_dispatch(B, EP, G, bs, H, E, K, ws, mode, smooth, fused):
     inp = _inputs(G * 1000 + mode, G, bs, H, E, K, ws, smooth or mode == 1)
-    grp = EP.EmulatedGroup(G, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws, quant_mode=mode)
+    grp = EP.EmulatedGroup(G, fused=fused, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws,
+                           quant_mode=mode)
     for r in grp.ranks:
         for t in r.buffers() + [r.global_idx, r.recv_counts, r.recv_offsets]:
             if t is not None:
@@ -110,11 +116,12 @@ def test_emulated_group_equals_one_gpu_dispatch(B, EP, G, bs, H, E, K, ws, mode,
         assert_close_bf16(host(o["y"]), oc["y_f64"][g * bs:(g + 1) * bs], what=f"y of GPU {g}")
 
 
-def test_receive_buffer_too_small_is_flagged(B, EP):
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "two_step"])
+def test_receive_buffer_too_small_is_flagged(B, EP, fused):
     G, bs, H, E, K, ws = 2, 64, 1024, 16, 4, 4
     inp = _inputs(7, G, bs, H, E, K, ws, False)
-    grp = EP.EmulatedGroup(G, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws, quant_mode=0,
-                           recv_rows=16)
+    grp = EP.EmulatedGroup(G, fused=fused, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws,
+                           quant_mode=0, recv_rows=16)
     for r in grp.ranks:
         poison_(r.recv_x)
     sl = lambda a, g: np.ascontiguousarray(a[g * bs:(g + 1) * bs])
@@ -128,3 +135,47 @@ def test_receive_buffer_too_small_is_flagged(B, EP):
         b = int(od["offsets"][q * (E // G)])
         # the rows that fit are right; nothing past the buffer was written (it has 16 rows)
         np.testing.assert_array_equal(_bytes(host(r.recv_x), 0, 16), _bytes(od["expand_x"], b, b + 16))
+
+
+def test_ep_combine_flags_a_row_outside_the_group(B, EP):
+    """A global row past the group's last row is reported (MOE_DEV_BAD_ID)
+    and that copy is dropped from the sum, as a pruned copy."""
+    G, bs, H, E, K, ws = 2, 32, 1024, 16, 4, 4
+    inp = _inputs(11, G, bs, H, E, K, ws, False)
+    grp = EP.EmulatedGroup(G, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws, quant_mode=0)
+    sl = lambda a, g: np.ascontiguousarray(a[g * bs:(g + 1) * bs])
+    grp.dispatch([dict(expert_ids=dev(sl(inp["ids"], g)), table=dev(inp["table"]), x=dev_bf16(sl(inp["x"], g)))
+                  for g in range(G)])
+    bal, bm, _ = orc.update_expert(inp["ids"], inp["table"], ws)
+    od = orc.dispatch(inp["x"], bal, E, 0, mask=bm)
+    total = int(od["offsets"][-1])
+    off, El = od["offsets"], E // G
+    for q, r in enumerate(grp.ranks):
+        b, e_ = int(off[q * El]), int(off[(q + 1) * El])
+        r.expert_out[:e_ - b].copy_(dev_bf16(inp["expert_rows"][b:e_]))
+    idx = od["expand_idx"].copy()
+    grp.ranks[0].global_idx[0, 0] = total  # one past the group's rows
+    idx[0, 0] = -1
+    outs = grp.combine([dict(expert_scales=dev(sl(inp["scales"], g)), residual=dev_bf16(sl(inp["residual"], g)),
+                             gamma=dev_bf16(inp["gamma"]), norm_eps=1e-6) for g in range(G)])
+    torch.cuda.synchronize()
+    assert grp.ranks[0].device_errors() & B.DEV_BAD_ID
+    assert grp.ranks[1].device_errors() == 0
+    oc = orc.combine_add_rmsnorm(inp["expert_rows"], idx, inp["scales"], inp["residual"], inp["gamma"], 1e-6)
+    for g, o in enumerate(outs):
+        assert_close_bf16(host(o["y"]), oc["y_f64"][g * bs:(g + 1) * bs], what=f"y of GPU {g}")
+
+
+def test_ep_dispatch_refuses_parameters_that_disagree(B, EP):
+    """moe_ep_dispatch checks the dispatch parameters against the EP ones."""
+    G, bs, H, E, K, ws = 2, 16, 1024, 16, 4, 4
+    grp = EP.EmulatedGroup(G, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws, quant_mode=0)
+    r = grp.ranks[0]
+    x = torch.zeros((bs, H), dtype=torch.bfloat16, device="cuda")
+    bad = B.ep_params(bs, K, E, G, 0, H, 0, r.cap)  # mode 0 rows are 2H bytes
+    with pytest.raises(B.MoeError):
+        B.ep_dispatch(bad, x, r.bal, ws, 0, r.route_out, grp.tables.recv_x, None, None, r.global_idx, r.ep_ws)
+    bad = B.ep_params(bs, K, E, G, 0, 2 * H, 4, r.cap)  # mode 0 sends no scales
+    with pytest.raises(B.MoeError):
+        B.ep_dispatch(bad, x, r.bal, ws, 0, r.route_out, grp.tables.recv_x, grp.tables.recv_x, None,
+                      r.global_idx, r.ep_ws)
