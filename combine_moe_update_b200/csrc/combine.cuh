@@ -40,6 +40,17 @@ struct CombineArgs {
     int gpus, recv_rows;
 };
 
+// K 16 with the norm keeps the pre-norm row in shared memory (XS) and runs
+// four blocks per SM; otherwise four blocks up to 224 threads, three beyond.
+__host__ __device__ constexpr bool cb_xs(int kmax, bool norm) { return norm && kmax == 16; }
+__host__ __device__ constexpr int cb_min_blocks(int kmax, int nt, bool norm) {
+    return cb_xs(kmax, norm) || nt <= 224 ? 4 : 3;
+}
+// Dynamic shared memory of a combine block (the XS row).
+__host__ __device__ constexpr int cb_smem_bytes(int kmax, int nt, bool norm, int split) {
+    return cb_xs(kmax, norm) ? (split == 1 ? 4 : 2) * nt * 32 : 0;
+}
+
 // Threads of a block for NV vectors of 8 elements per block and VECS vectors
 // per thread, from the same fixed set of block sizes as the dispatch.
 __host__ __device__ inline int cb_threads(int NV, int vecs) {
@@ -59,8 +70,13 @@ __host__ __device__ inline int cb_threads(int NV, int vecs) {
 // EP: the rows come from the GPUs that own them (expert parallelism across
 // GPUs, the AllToAllV back fused into the gather).
 template <int KMAX, bool SHARED, int NT, bool NORM, int SPLIT, bool EP = false>
-__global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_token_kernel(CombineArgs a) {
     constexpr int VECS = SPLIT == 1 ? 4 : 2;
+    // XS: the pre-norm row waits for the sum of squares in shared memory
+    // rather than in registers, which (with the top-K rows loaded eight at a
+    // time) lets four blocks of 256 threads share an SM at K 16
+    constexpr bool XS = cb_xs(KMAX, NORM);
+    extern __shared__ float4 s_x[];  // XS: [VECS][NT][2]
     constexpr int NW = NT / 32;
     __shared__ int s_row[16];
     __shared__ float s_w[16];
@@ -128,8 +144,9 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-        // at most eight rows in flight per thread (sixteen spill the registers); the sum stays in k order
-        constexpr int CH = KMAX < 8 ? KMAX : 8;
+        // all top-K rows in flight at once, except with XS (registers for
+        // four blocks per SM)
+        constexpr int CH = XS ? 8 : KMAX;
 #pragma unroll
         for (int k0 = 0; k0 < KMAX; k0 += CH) {
             uint4 rv[CH];
@@ -163,6 +180,10 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
             xs[j][e] = acc[e] + r[e];
             ss = fmaf(xs[j][e], xs[j][e], ss);
         }
+        if constexpr (XS) {
+            s_x[(j * NT + t) * 2] = make_float4(xs[j][0], xs[j][1], xs[j][2], xs[j][3]);
+            s_x[(j * NT + t) * 2 + 1] = make_float4(xs[j][4], xs[j][5], xs[j][6], xs[j][7]);
+        }
     }
 
     if constexpr (!NORM) {  // the plain combine: combineOut, rounded to bf16 once
@@ -195,6 +216,11 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) combine_token_kernel(Co
     for (int j = 0; j < VECS; ++j) {
         const int pl = t + j * NT, p = p0 + pl;
         if (pl >= Vh) continue;
+        if constexpr (XS) {  // written by this thread
+            const float4 u = s_x[(j * NT + t) * 2], v = s_x[(j * NT + t) * 2 + 1];
+            xs[j][0] = u.x, xs[j][1] = u.y, xs[j][2] = u.z, xs[j][3] = u.w;
+            xs[j][4] = v.x, xs[j][5] = v.y, xs[j][6] = v.z, xs[j][7] = v.w;
+        }
         float g[8];
         unpack8(ld_cached(a.gamma + p * 8), g);
         uint4 yo;

@@ -58,12 +58,10 @@ struct DispatchArgs {
     int32_t *counts;
     int32_t *offsets;
     uint32_t *err;
-    // The call's first kernel reads nothing before griddepcontrol.wait (set
-    // when a scatter kernel runs without a route kernel of its own call).
-    int wait_first;
-    // Expert parallelism across GPUs (peer_x null: rows go to expand_x on
-    // this GPU).  Copy (instance e, local row r) goes to GPU q = e / ep_el,
-    // row gstart[e] + (r - offsets[e]) - gbase[q] of q's receive buffer.
+    // Expert parallelism across GPUs (the EP kernels; the others write
+    // expand_x on this GPU).  Copy (instance e, local row r) goes to GPU
+    // q = e / ep_el, row gstart[e] + (r - offsets[e]) - gbase[q] of q's
+    // receive buffer.
     uint8_t *const *peer_x;      // [G] receive buffers
     uint8_t *const *peer_sc;     // [G] their scales (modes 2 to 4)
     int32_t *const *peer_src;    // [G] copy ids, optional
@@ -82,11 +80,12 @@ struct RowDst {
 };
 
 // Copy j of instance e at local row r.  On one GPU, row r of expand_x; with
-// expert parallelism, the owner's receive buffer (also records the copy's
-// global row and id there).  False if the row falls past the receive buffer
-// (reported; the copy is dropped).
-__device__ __forceinline__ bool copy_dst(const DispatchArgs &a, int e, int r, int j, RowDst &d) {
-    if (a.peer_x == nullptr) {
+// expert parallelism (EP), the owner's receive buffer.  False if the row
+// falls outside the receive buffer (reported by ep_record; the copy is
+// dropped).
+template <bool EP>
+__device__ __forceinline__ bool copy_dst(const DispatchArgs &a, int e, int r, RowDst &d) {
+    if constexpr (!EP) {
         d.x = reinterpret_cast<uint8_t *>(a.expand_x);
         d.sc = reinterpret_cast<uint8_t *>(a.dyn_scales);
         d.row = r;
@@ -749,7 +748,6 @@ __device__ __forceinline__ void write_row(const DispatchArgs &a, const RowDst &d
 // With expert parallelism, thread t < K of a token block records copy t's
 // global row and, at its owner, the copy's id in the group.
 __device__ __forceinline__ void ep_record(const DispatchArgs &a, int j, int e, int r) {
-    if (a.peer_x == nullptr) return;
     int g = -1;
     if (r >= 0) {
         const int q = e / a.ep_el;
@@ -776,10 +774,14 @@ __device__ __forceinline__ void load_row(const uint16_t *row, int V, uint4 (&xv)
 
 // FUSED: the block routes its own copies (block_route, small calls) instead
 // of reading the rows route_kernel wrote.
-template <int MODE, int NT, bool FUSED>
+// EP: rows go to their owners' receive buffers (expert parallelism across
+// GPUs); the rows were routed by an earlier call, so this kernel is its
+// call's first and waits before it reads anything.
+template <int MODE, int NT, bool FUSED, bool EP = false>
 __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
+    static_assert(!(FUSED && EP), "an EP scatter follows an earlier route call");
     __shared__ float s_red[NT / 32];
-    __shared__ int s_row[16], s_inst[16];
+    __shared__ int s_row[16], s_inst[EP ? 16 : 1];
     __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
     const int i = blockIdx.x, t = threadIdx.x;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
@@ -790,8 +792,8 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         // flight while the block routes its copies.
         block_route_clear<NT>(rs, a.num_instances);
         pdl_wait();
-    } else if (a.wait_first) {
-        pdl_wait();  // no route kernel of this call ran first (the rows were routed by an earlier call)
+    } else if constexpr (EP) {
+        pdl_wait();
     }
 
     // FUSED: after the wait.  Otherwise this kernel follows the call's route
@@ -850,8 +852,10 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         if (t < K) {
             const int r = a.expand_idx[i * K + t];
             s_row[t] = r;
-            s_inst[t] = a.peer_x != nullptr ? a.ids[i * K + t] : 0;
-            ep_record(a, i * K + t, s_inst[t], r);
+            if constexpr (EP) {
+                s_inst[t] = a.ids[i * K + t];
+                ep_record(a, i * K + t, s_inst[t], r);
+            }
         }
         __syncthreads();
     }
@@ -859,7 +863,7 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         const int row = FUSED ? rs.row[k] : s_row[k];
         if (row < 0) continue;
         RowDst d;
-        if (!copy_dst(a, FUSED ? 0 : s_inst[k], row, i * K + k, d)) continue;
+        if (!copy_dst<EP>(a, EP ? s_inst[k] : 0, row, d)) continue;
         if constexpr (MODE == 0) {
             uint16_t *dst = reinterpret_cast<uint16_t *>(d.x) + (size_t)d.row * H;
 #pragma unroll
@@ -896,8 +900,9 @@ __host__ __device__ inline int smooth_smem_floats(int hidden) {
     return hidden > NT * kDpVecs * 8 ? hidden : NT * kDpVecs * 8;
 }
 
-template <int MODE, int NT, bool FUSED>
+template <int MODE, int NT, bool FUSED, bool EP = false>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_kernel(DispatchArgs a) {
+    static_assert(!(FUSED && EP), "an EP scatter follows an earlier route call");
     constexpr int NW = NT / 32;
     extern __shared__ __align__(128) float s_smooth[];  // the current copy's smooth row, then zeros
     __shared__ float s_red[2][NW];
@@ -922,8 +927,8 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         if (t == 0) mbar_init(&s_bar, 1);
         __syncthreads();
         pdl_wait();
-    } else if (a.wait_first) {
-        pdl_wait();  // no route kernel of this call ran first (the rows were routed by an earlier call)
+    } else if constexpr (EP) {
+        pdl_wait();  // the call's first kernel (routed by an earlier call)
     }
     // FUSED: after the wait.  Otherwise the call's route kernel runs first
     // and releases this kernel only after its own wait, so the call's inputs
@@ -1007,7 +1012,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
             if (t < K) {
                 const int r = a.expand_idx[i * K + t];
                 s_row[t] = r;
-                if (a.peer_x != nullptr) ep_record(a, i * K + t, a.ids[i * K + t], r);
+                if constexpr (EP) ep_record(a, i * K + t, a.ids[i * K + t], r);
             }
             __syncthreads();
         }
@@ -1015,7 +1020,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         for (int q = 0; q < kDpVecs; ++q)
             if (swap) qv[q] = make_uint2(qv[q].y, qv[q].x);
         RowDst d;
-        if (copy_dst(a, s_key[c], FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], i * K + s_pos[c], d))
+        if (copy_dst<EP>(a, s_key[c], FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], d))
             write_row<MODE, NT>(a, d, V, qv, seg, row_scale);
     }
 }

@@ -229,33 +229,35 @@ cudaError_t launch_by_threads(const moe::DispatchArgs &a, cudaStream_t s) {
 // Small calls (at most kFusedRouteMax copies) use the instantiations whose
 // blocks route their own copies, and no route kernel runs.
 inline bool fused_route(const moe::DispatchArgs &a) {
-    return a.bs * a.top_k <= moe::kFusedRouteMax && !a.wait_first;  // wait_first: routed by an earlier call
+    return a.bs * a.top_k <= moe::kFusedRouteMax && a.peer_x == nullptr;  // EP: routed by an earlier call
 }
 
 template <int MODE, int NT>
 struct TokenLaunch {
-    template <bool FUSED>
+    template <bool FUSED, bool EP>
     static cudaError_t go_(const moe::DispatchArgs &a, cudaStream_t s) {
-        auto kernel = moe::dispatch_token_kernel<MODE, NT, FUSED>;
+        auto kernel = moe::dispatch_token_kernel<MODE, NT, FUSED, EP>;
         if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
         return launch(kernel, a.bs, NT, 0, s, a);
     }
     static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
-        return fused_route(a) ? go_<true>(a, s) : go_<false>(a, s);
+        if (a.peer_x != nullptr) return go_<false, true>(a, s);
+        return fused_route(a) ? go_<true, false>(a, s) : go_<false, false>(a, s);
     }
 };
 
 template <int MODE, int NT>
 struct TokenSmoothLaunch {
-    template <bool FUSED>
+    template <bool FUSED, bool EP>
     static cudaError_t go_(const moe::DispatchArgs &a, cudaStream_t s) {
-        auto kernel = moe::dispatch_token_smooth_kernel<MODE, NT, FUSED>;
+        auto kernel = moe::dispatch_token_smooth_kernel<MODE, NT, FUSED, EP>;
         const size_t smem = (size_t)moe::smooth_smem_floats<NT>(a.hidden) * sizeof(float);
         if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
         return launch(kernel, a.bs, NT, smem, s, a);
     }
     static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
-        return fused_route(a) ? go_<true>(a, s) : go_<false>(a, s);
+        if (a.peer_x != nullptr) return go_<false, true>(a, s);
+        return fused_route(a) ? go_<true, false>(a, s) : go_<false, false>(a, s);
     }
 };
 
@@ -274,8 +276,9 @@ cudaError_t launch_dispatch_token_smooth(const moe::DispatchArgs &a, cudaStream_
 template <int KMAX, bool SHARED, int NT, bool NORM, int SPLIT>
 cudaError_t launch_combine_nt(const moe::CombineArgs &a, cudaStream_t s) {
     auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, NORM, SPLIT>;
-    if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
-    return launch_in_clusters(kernel, a.bs * SPLIT, NT, 0, s, SPLIT, a);
+    constexpr int smem = moe::cb_smem_bytes(KMAX, NT, NORM, SPLIT);
+    if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
+    return launch_in_clusters(kernel, a.bs * SPLIT, NT, smem, s, SPLIT, a);
 }
 
 template <int KMAX, bool SHARED, bool NORM, int SPLIT>
@@ -306,8 +309,9 @@ cudaError_t launch_combine_split(const moe::CombineArgs &a, cudaStream_t s) {
 template <int KMAX, bool SHARED, int NT>
 cudaError_t launch_combine_ep_nt(const moe::CombineArgs &a, cudaStream_t s) {
     auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, true, 1, true>;
-    if (!ensure_smem(kernel, 0)) return cudaErrorInvalidValue;
-    return launch(kernel, a.bs, NT, 0, s, a);
+    constexpr int smem = moe::cb_smem_bytes(KMAX, NT, true, 1);
+    if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
+    return launch(kernel, a.bs, NT, smem, s, a);
 }
 
 template <int KMAX, bool SHARED>
@@ -926,7 +930,6 @@ moe_status moe_ep_dispatch(const moe_dispatch_params *p, const moe_ep_params *ep
                                         const_cast<int32_t *>(expand_idx), nullptr, nullptr,
                                         const_cast<int32_t *>(expert_offsets), ep_workspace);
     const moe::EpArgs plan = ep_args(*ep, ep_workspace);
-    a.wait_first = 1;  // this call's scatter is its first kernel
     a.peer_x = reinterpret_cast<uint8_t *const *>(peer_rows);
     a.peer_sc = reinterpret_cast<uint8_t *const *>(peer_scales);
     a.peer_src = peer_src;
