@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
     __shared__ int s_row[16];
     __shared__ float s_w[16];
     __shared__ const uint16_t *s_src[EP ? 16 : 1];
+    __shared__ int s_nk;
     __shared__ float s_red[NW];
     __shared__ float s_part;
     const int t = threadIdx.x;
@@ -94,40 +95,52 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
         if constexpr (SHARED) prefetch_l2(a.shared_x + off, bytes);
     }
     pdl_wait();  // expand_idx and the expert rows come from earlier kernels
-    if (t < K) {
-        int row = a.expand_idx[i * K + t];
-        const float w = a.scales[i * K + t];
-        if (row < -1 || row >= a.expand_rows) {
-            raise_error(a.err, kDevBadId);
-            row = -1;
-        }
-        if constexpr (EP) {  // the owner of global row `row` (the last GPU whose first row is <= row)
-            if (row >= 0) {
-                int lo = 0, hi = a.gpus - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (a.gbase[mid] <= row) lo = mid; else hi = mid - 1;
-                }
-                const int prow = row - a.gbase[lo];
-                if (prow >= a.recv_rows || row >= a.gbase[a.gpus]) {
-                    raise_error(a.err, kDevBadId);
-                    row = -1;
-                } else {
-                    s_src[t] = a.peer_rows[lo] + (size_t)prow * H;
+    if (t < 32) {  // warp 0: the kept copies, compacted in k order (a pruned copy adds nothing)
+        int row = -1;
+        float w = 0.0f;
+        const uint16_t *src = nullptr;
+        if (t < K) {
+            row = a.expand_idx[i * K + t];
+            w = a.scales[i * K + t];
+            if (row < -1 || row >= a.expand_rows) {
+                raise_error(a.err, kDevBadId);
+                row = -1;
+            }
+            if constexpr (EP) {  // the owner of global row `row` (the last GPU whose first row is <= row)
+                if (row >= 0) {
+                    int lo = 0, hi = a.gpus - 1;
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (a.gbase[mid] <= row) lo = mid; else hi = mid - 1;
+                    }
+                    const int prow = row - a.gbase[lo];
+                    if (prow >= a.recv_rows || row >= a.gbase[a.gpus]) {
+                        raise_error(a.err, kDevBadId);
+                        row = -1;
+                    } else {
+                        src = a.peer_rows[lo] + (size_t)prow * H;
+                    }
                 }
             }
         }
-        s_row[t] = row;
-        s_w[t] = row >= 0 ? w : 0.0f;  // a pruned copy weighs nothing
+        const unsigned kept = __ballot_sync(kFull, row >= 0);
+        if (row >= 0) {
+            const int c = __popc(kept & ((1u << t) - 1u));
+            s_row[c] = row;
+            s_w[c] = w;
+            if constexpr (EP) s_src[c] = src;
+        }
+        if (t == 0) s_nk = __popc(kept);
     }
     __syncthreads();
+    const int nk = s_nk;  // kept copies: rows [0, nk) of s_row
     int row[KMAX];
     float wk[KMAX];
     float wsum = 0.0f;  // sum of the kept weights, in k order
 #pragma unroll
     for (int k = 0; k < KMAX; ++k) {
-        row[k] = k < K ? s_row[k] : -1;
-        wk[k] = k < K ? s_w[k] : 0.0f;
+        row[k] = k < nk ? s_row[k] : -1;
+        wk[k] = k < nk ? s_w[k] : 0.0f;
         wsum += wk[k];
     }
 
@@ -144,23 +157,24 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-        // all top-K rows in flight at once, except with XS (registers for
-        // four blocks per SM)
-        constexpr int CH = XS ? 8 : KMAX;
+        // all top-K rows in flight at once up to K 8; at K 16 eight at a
+        // time (registers: four blocks per SM with XS, no spills without)
+        constexpr int CH = KMAX == 16 ? 8 : KMAX;
 #pragma unroll
         for (int k0 = 0; k0 < KMAX; k0 += CH) {
             uint4 rv[CH];
 #pragma unroll
-            for (int k = 0; k < CH; ++k)
-                if (row[k0 + k] >= 0)
-                    rv[k] = ld_stream((EP ? s_src[k0 + k] : a.expand_x + (size_t)row[k0 + k] * H) + p * 8);
+            for (int k = 0; k < CH; ++k) {  // nk is the same in every thread: a uniform branch
+                if (k0 + k >= nk) break;
+                rv[k] = ld_stream((EP ? s_src[k0 + k] : a.expand_x + (size_t)row[k0 + k] * H) + p * 8);
+            }
             if (k0 == 0) {
                 if constexpr (NORM) res = ld_stream(a.residual + tok + p * 8);
                 if constexpr (SHARED) sh = ld_stream(a.shared_x + tok + p * 8);
             }
 #pragma unroll
             for (int k = 0; k < CH; ++k) {
-                if (row[k0 + k] < 0) continue;
+                if (k0 + k >= nk) break;
                 float f[8];
                 unpack8(rv[k], f);
 #pragma unroll
@@ -180,18 +194,7 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
             xs[j][e] = acc[e] + r[e];
             ss = fmaf(xs[j][e], xs[j][e], ss);
         }
-        if constexpr (XS) {
-            s_x[(j * NT + t) * 2] = make_float4(xs[j][0], xs[j][1], xs[j][2], xs[j][3]);
-            s_x[(j * NT + t) * 2 + 1] = make_float4(xs[j][4], xs[j][5], xs[j][6], xs[j][7]);
-        }
-    }
-
-    if constexpr (!NORM) {  // the plain combine: combineOut, rounded to bf16 once
-        pdl_launch_dependents();
-#pragma unroll
-        for (int j = 0; j < VECS; ++j) {
-            const int pl = t + j * NT, p = p0 + pl;
-            if (pl >= Vh) continue;
+        if constexpr (!NORM) {  // the plain combine: combineOut, rounded to bf16 once
             uint4 o;
             o.x = pack_bf16x2(xs[j][0], xs[j][1]);
             o.y = pack_bf16x2(xs[j][2], xs[j][3]);
@@ -199,6 +202,14 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
             o.w = pack_bf16x2(xs[j][6], xs[j][7]);
             st_v4(a.y + tok + p * 8, o);
         }
+        if constexpr (XS) {
+            s_x[(j * NT + t) * 2] = make_float4(xs[j][0], xs[j][1], xs[j][2], xs[j][3]);
+            s_x[(j * NT + t) * 2 + 1] = make_float4(xs[j][4], xs[j][5], xs[j][6], xs[j][7]);
+        }
+    }
+
+    if constexpr (!NORM) {  // the rows are written (no residual, no norm)
+        pdl_launch_dependents();
         return;
     }
     float tot = block_sum<NW>(ss, s_red);
