@@ -374,8 +374,14 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 // warps wrote the stage's factors) and empty[s] (tcgen05.commit: the MMAs
 // that read the stage's operands and factors completed), so no role waits
 // for another except through the stage it needs.
+//
+// VEC: the factor rows are 16-byte aligned (H % 512 == 0 and aligned bases),
+// so each thread loads four steps of a row in one 16-byte load.  A warp's
+// factor load touches 32 rows, i.e. 32 cache lines; four-byte loads (one
+// step each) made the factor warps L1-bound and left the MMA issuer waiting.
 constexpr int kGmMxThreads = 192;
 
+template <bool VEC>
 __global__ void __launch_bounds__(kGmMxThreads, 1)
     gmm_mx_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GmmArgs a) {
     extern __shared__ uint8_t gm_smem_raw[];
@@ -508,27 +514,74 @@ __global__ void __launch_bounds__(kGmMxThreads, 1)
             if (lane == 0) mbar_arrive(&s_sf[s]);
             return true;
         };
-        // factor words eight steps ahead (a weight row's 32-byte sector holds
-        // eight steps, so one load in eight goes to DRAM), in eight register
-        // sets used in turn: four steps ahead left the MMA issuer waiting for
-        // the factors (measured: 409 -> 376 us at 32 instances of 7168 x 7168)
-        constexpr int kPre = 8;
-        uint32_t fa[kPre][4], fb[kPre][4];
+        if constexpr (VEC) {
+            // four steps per 16-byte load, two groups (eight steps) ahead, in
+            // two register sets used in turn
+            const uint4 *qa[4], *qb[4];
 #pragma unroll
-        for (int q = 0; q < kPre; ++q)
-            if (q < nk) load_sf(q, fa[q], fb[q]);
-        bool stop = false;
-        for (int kb0 = 0; kb0 < nk && !stop; kb0 += kPre) {
+            for (int c = 0; c < 4; ++c) {
+                qa[c] = reinterpret_cast<const uint4 *>(pa[c]);
+                qb[c] = reinterpret_cast<const uint4 *>(pb[c]);
+            }
+            const int ng = nk >> 2;  // nk % 4 == 0 here
+            uint4 ga[2][4], gb[2][4];
+            auto load_group = [&](int g, uint4(&va)[4], uint4(&vb)[4]) {
 #pragma unroll
-            for (int q = 0; q < kPre; ++q) {  // constant register-set index after unrolling
-                const int kb = kb0 + q;
-                if (kb >= nk) break;
-                if (!sf_step(kb, fa[q], fb[q])) {
-                    if (lane == 0) s_fail = 1;
-                    stop = true;
-                    break;
+                for (int c = 0; c < 4; ++c) {
+                    va[c] = ld_in(qa[c] + g);
+                    vb[c] = ld_in(qb[c] + g);
                 }
-                if (kb + kPre < nk) load_sf(kb + kPre, fa[q], fb[q]);
+            };
+            auto word = [](const uint4 &v, int q) { return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w; };
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+                if (b < ng) load_group(b, ga[b], gb[b]);
+            bool stop = false;
+            for (int g0 = 0; g0 < ng && !stop; g0 += 2) {
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {  // constant register-set index after unrolling
+                    const int g = g0 + b;
+                    if (g >= ng) break;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t fa[4], fb[4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            fa[c] = word(ga[b][c], q);
+                            fb[c] = word(gb[b][c], q);
+                        }
+                        if (!sf_step(4 * g + q, fa, fb)) {
+                            if (lane == 0) s_fail = 1;
+                            stop = true;
+                            break;
+                        }
+                    }
+                    if (stop) break;
+                    if (g + 2 < ng) load_group(g + 2, ga[b], gb[b]);
+                }
+            }
+        } else {
+            // factor words eight steps ahead (a weight row's 32-byte sector
+            // holds eight steps, so one load in eight goes to DRAM), in eight
+            // register sets used in turn
+            constexpr int kPre = 8;
+            uint32_t fa[kPre][4], fb[kPre][4];
+#pragma unroll
+            for (int q = 0; q < kPre; ++q)
+                if (q < nk) load_sf(q, fa[q], fb[q]);
+            bool stop = false;
+            for (int kb0 = 0; kb0 < nk && !stop; kb0 += kPre) {
+#pragma unroll
+                for (int q = 0; q < kPre; ++q) {  // constant register-set index after unrolling
+                    const int kb = kb0 + q;
+                    if (kb >= nk) break;
+                    if (!sf_step(kb, fa[q], fb[q])) {
+                        if (lane == 0) s_fail = 1;
+                        stop = true;
+                        break;
+                    }
+                    if (kb + kPre < nk) load_sf(kb + kPre, fa[q], fb[q]);
+                }
             }
         }
     }

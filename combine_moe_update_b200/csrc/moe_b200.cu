@@ -660,7 +660,9 @@ moe_status launch_gmm(const moe_gmm_params *p, const void *expand_x, const void 
     a.nslots = reinterpret_cast<int *>(ws + kWorkspaceBytes);
     a.slots = reinterpret_cast<int4 *>(ws + kWorkspaceBytes + 16);
     a.err = reinterpret_cast<uint32_t *>(workspace);
-    auto *kernel = MX ? moe::gmm_mx_kernel : moe::gmm_kernel;
+    // mxfp8: 16-byte factor loads when every factor row starts on a 16-byte boundary
+    const bool vec = MX && p->hidden % 512 == 0 && aligned(a.xsf, 16) && aligned(a.wsf, 16);
+    auto *kernel = !MX ? moe::gmm_kernel : vec ? moe::gmm_mx_kernel<true> : moe::gmm_mx_kernel<false>;
     if (!ensure_smem(kernel, moe::kGmSmemBytes)) return MOE_ERR_CUDA;
     if (launch(moe::gmm_plan_kernel, dim3(1), 1024, 0, s, a) != cudaSuccess) return MOE_ERR_CUDA;
     const dim3 grid((p->out_dim + moe::kGmBM - 1) / moe::kGmBM, a.max_slots);

@@ -177,13 +177,23 @@ def test_dispatch_gmm_combine_pipeline(B):
 
 # ------------------------------------------------------------------ mxfp8
 
-def _gpu_mx(B, gi):
+def _at_offset(a, off):
+    """a's bytes on the device starting `off` bytes into a larger buffer (a
+    base that is 4-byte but not 16-byte aligned when off = 4)."""
+    buf = torch.zeros(a.nbytes + 16, dtype=torch.uint8, device="cuda")
+    t = buf[off:off + a.nbytes]
+    t.copy_(torch.from_numpy(np.ascontiguousarray(a).reshape(-1).view(np.uint8)).cuda())
+    return t.view(a.shape)
+
+
+def _gpu_mx(B, gi, sf_offset=0):
     rows, H = gi.expand_x.shape
     E, N = gi.weight.shape[0], gi.weight.shape[1]
     out = poison_(torch.empty((rows, N), dtype=torch.bfloat16, device="cuda"))
     wsp = B.new_workspace(nbytes=B.grouped_matmul_workspace_bytes(rows, H, N, E))
-    B.grouped_matmul_mx(dev(gi.expand_x), dev(gi.x_sf), dev(gi.offsets), dev(gi.weight), dev(gi.weight_sf), out=out,
-                        workspace=wsp)
+    x_sf = dev(gi.x_sf) if sf_offset == 0 else _at_offset(gi.x_sf, sf_offset)
+    w_sf = dev(gi.weight_sf) if sf_offset == 0 else _at_offset(gi.weight_sf, sf_offset)
+    B.grouped_matmul_mx(dev(gi.expand_x), x_sf, dev(gi.offsets), dev(gi.weight), w_sf, out=out, workspace=wsp)
     torch.cuda.synchronize()
     return host(out), B.read_device_error(wsp)
 
@@ -195,8 +205,9 @@ def _oracle_mx(gi):
 
 
 @pytest.mark.parametrize("H,N,counts,spare", [
-    (1024, 256, [3, 0, 17, 130, 1, 128, 16], 5),
-    (1152, 208, [5, 33, 0, 260], 0),
+    (1024, 256, [3, 0, 17, 130, 1, 128, 16], 5),   # factor rows of 32 B: 16-byte factor loads
+    (1152, 208, [5, 33, 0, 260], 0),               # 36 B: four-byte factor loads
+    (3072, 128, [64, 1, 31], 2),                   # 96 B: 16-byte loads, six groups of four steps
 ])
 def test_gmm_mx_single_products_bit_exact(B, H, N, counts, spare):
     """One non-zero E4M3 code per row: every output is one product of two
@@ -229,6 +240,20 @@ def test_gmm_mx_parity_random(B, H, N, counts, spare):
     assert_close_bf16(got[rows], o["out_f64"][rows], what="mx gmm out")
     step = np.abs(got[written].astype(np.int32) - o["out"][written].astype(np.int32))
     assert (step <= 1).mean() >= 0.99
+
+
+@pytest.mark.parametrize("H", [1024, 2048])
+def test_gmm_mx_factor_alignment_paths_agree(B, H):
+    """Factor arrays whose bases are 4- but not 16-byte aligned take the
+    four-byte factor loads; the result is the same, bit for bit, as with
+    16-byte aligned bases (the 16-byte loads), and both equal the oracle on
+    single products."""
+    gi = gen.gmm_inputs_mx(43, [7, 40, 0, 129], H, 128, spare_rows=2, one_hot=True)
+    got16, err16 = _gpu_mx(B, gi)
+    got4, err4 = _gpu_mx(B, gi, sf_offset=4)
+    assert err16 == 0 and err4 == 0
+    np.testing.assert_array_equal(got4, got16)
+    np.testing.assert_array_equal(got16, _oracle_mx(gi)["out"])
 
 
 def test_dispatch_mx_gmm_combine_pipeline(B):
