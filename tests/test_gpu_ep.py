@@ -179,3 +179,43 @@ def test_ep_dispatch_refuses_parameters_that_disagree(B, EP):
     with pytest.raises(B.MoeError):
         B.ep_dispatch(bad, x, r.bal, ws, 0, r.route_out, grp.tables.recv_x, grp.tables.recv_x, None,
                       r.global_idx, r.ep_ws)
+
+
+def test_process_group_ep_one_rank(B, EP):
+    """ProcessGroupEP on a one-GPU NCCL group (the counts gathered by
+    all_gather_into_tensor, the barriers as all-reduces, fused dispatch and
+    combine through the group's pointer tables) equals the oracle."""
+    import datetime
+    import socket
+    import torch.distributed as dist
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    bs, H, E, K, ws = 96, 2048, 32, 6, 8
+    inp = _inputs(5, 1, bs, H, E, K, ws, True)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        grp = EP.ProcessGroupEP(bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws, quant_mode=2)
+        r = grp.r
+        grp.dispatch(expert_ids=dev(inp["ids"]), table=dev(inp["table"]), x=dev_bf16(inp["x"]),
+                     expert_scales=dev(inp["scales"]), smooth=dev(inp["smooth"]))
+        bal, bm, _ = orc.update_expert(inp["ids"], inp["table"], ws, expert_scales=inp["scales"])
+        od = orc.dispatch(inp["x"], bal, E, 2, mask=bm, smooth=inp["smooth"])
+        n = int(od["offsets"][-1])
+        torch.cuda.synchronize()
+        assert r.received() == n
+        np.testing.assert_array_equal(_bytes(host(r.recv_x), 0, n), _bytes(od["expand_x"], 0, n))
+        np.testing.assert_array_equal(_bytes(host(r.recv_scales), 0, n), _bytes(od["dyn_scales"], 0, n))
+        np.testing.assert_array_equal(host(r.global_idx), od["expand_idx"])
+        r.expert_out[:n].copy_(dev_bf16(inp["expert_rows"][:n]))
+        out = grp.combine(expert_scales=dev(inp["scales"]), residual=dev_bf16(inp["residual"]),
+                          gamma=dev_bf16(inp["gamma"]), norm_eps=1e-6, shared_x=dev_bf16(inp["shared"]))
+        torch.cuda.synchronize()
+        assert r.device_errors() == 0
+        oc = orc.combine_add_rmsnorm(inp["expert_rows"], od["expand_idx"], inp["scales"], inp["residual"],
+                                     inp["gamma"], 1e-6, shared_x=inp["shared"])
+        assert_close_bf16(host(out["y"]), oc["y_f64"], what="y")
+        grp.close()
+    finally:
+        dist.destroy_process_group()
