@@ -505,3 +505,36 @@ uint32_t orc_grouped_matmul_mx(int32_t rows, int32_t hidden, int32_t out_dim, in
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------- */
+/* TP domain of two ranks (READING R26)                                    */
+/* ---------------------------------------------------------------------- */
+
+/* AllGatherV over the TP pair (dispatch page, 计算公式): both TP ranks of EP
+ * rank e end with the rows each of them received from its own EP domain,
+ * domain 0's first.  With one instance per rank the ranks are the
+ * instances, taken in order. */
+void orc_tp_allgather(int32_t num_instances, int64_t row_bytes, const uint8_t *d0, const int32_t *off0,
+                      const uint8_t *d1, const int32_t *off1, uint8_t *out, int32_t *map0, int32_t *map1,
+                      int32_t *tp_counts) {
+    int64_t o = 0;
+    for (int32_t e = 0; e < num_instances; ++e) {
+        for (int t = 0; t < 2; ++t) {
+            const uint8_t *d = t ? d1 : d0;
+            const int32_t *off = t ? off1 : off0;
+            int32_t *map = t ? map1 : map0;
+            for (int32_t r = off[e]; r < off[e + 1]; ++r, ++o) {
+                if (row_bytes > 0) memcpy(out + o * row_bytes, d + (int64_t)r * row_bytes, (size_t)row_bytes);
+                if (map) map[r] = (int32_t)o;
+            }
+            if (tp_counts) tp_counts[2 * e + t] = off[e + 1] - off[e];
+        }
+    }
+}
+
+/* ReduceScatterV over the TP pair (combine page, 计算公式): the sum of the two
+ * partial bf16 outputs of a row, exact in binary64, rounded once to bf16. */
+void orc_tp_reduce(int64_t n, const uint16_t *p0, const uint16_t *p1, uint16_t *out) {
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = orc_bf16_from_double((double)bf16_to_float(p0[i]) + (double)bf16_to_float(p1[i]));
+}

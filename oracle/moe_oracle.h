@@ -102,6 +102,23 @@ uint32_t orc_grouped_matmul_mx(int32_t rows, int32_t hidden, int32_t out_dim, in
                                const uint8_t *weight_sf, uint16_t *out_bf16, double *out_f64);
 double orc_e4m3_decode(uint8_t c);  /* the value of an E4M3 code (NaN for S.1111.111) */
 
+/* The TP domain of two ranks (READING R26; dispatch page 计算公式
+ * expandXOut = AllGatherV(allToAllXOut), combine page 计算公式
+ * rsOut = ReduceScatterV(expandX)), for localExpertNum = 1 (instance e is
+ * EP rank e):
+ * orc_tp_allgather: rank e's gathered rows are [TP domain 0's rows of e ;
+ * TP domain 1's rows of e], in rank order.  d0 / d1 are the two domains'
+ * AllToAllV outputs (rows of row_bytes, offsets off0 / off1 [E+1]); map0 /
+ * map1 receive each domain row's row in out; tp_counts [E][2] the rows of
+ * each (rank, domain).
+ * orc_tp_reduce: the two TP ranks' partial expert outputs of the same rows,
+ * summed exactly and rounded to bf16 (ties to even); the scatter half is
+ * each domain reading its own rows. */
+void orc_tp_allgather(int32_t num_instances, int64_t row_bytes, const uint8_t *d0, const int32_t *off0,
+                      const uint8_t *d1, const int32_t *off1, uint8_t *out, int32_t *map0, int32_t *map1,
+                      int32_t *tp_counts);
+void orc_tp_reduce(int64_t n, const uint16_t *p0, const uint16_t *p1, uint16_t *out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -72,6 +72,10 @@ def lib():
             L.orc_e4m3_encode.argtypes = [f32]
             L.orc_bf16_from_double.restype = ctypes.c_uint16
             L.orc_bf16_from_double.argtypes = [f64]
+            L.orc_tp_allgather.restype = None
+            L.orc_tp_allgather.argtypes = [i32, ctypes.c_int64, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.orc_tp_reduce.restype = None
+            L.orc_tp_reduce.argtypes = [ctypes.c_int64, vp, vp, vp]
             _lib = L
     return _lib
 
@@ -239,3 +243,74 @@ def bf16_from_double(values):
     f = lib().orc_bf16_from_double
     v = np.asarray(values, np.float64).ravel()
     return np.array([f(float(t)) for t in v], np.uint16).reshape(np.shape(values))
+
+
+def dispatch_tp(x_bf16, instance_ids, num_instances, quant_mode, ep_world_size, bs, mask=None, smooth=None):
+    """aclnnMoeDistributeDispatchV2 with a TP domain of two ranks (READING
+    R26): 2 * ep_world_size devices of bs tokens each, TP-major (device
+    t * ep_world_size + g is EP rank g of TP domain t).  Each TP domain runs
+    its own EP AllToAllV (the one-rank-per-source dispatch of its tokens),
+    then every EP rank's pair gathers both domains' rows (AllGatherV).
+    Needs one instance per rank.  Returns the dispatch dict over all
+    2 * ep_world_size * bs tokens (expand_idx and src_of_row in global
+    numbering) plus tp_counts [E, 2]."""
+    if num_instances != ep_world_size:
+        raise ValueError("the TP domain needs one instance per EP rank")
+    x = _c(x_bf16, np.uint16)
+    ids = _c(instance_ids, np.int32)
+    m = _c(mask, np.uint8)
+    K = ids.shape[1]
+    T = 2 * ep_world_size * bs
+    if x.shape[0] != T or ids.shape[0] != T:
+        raise ValueError("x and the ids hold 2 * ep_world_size * bs tokens")
+    dom = [slice(t * ep_world_size * bs, (t + 1) * ep_world_size * bs) for t in range(2)]
+    d = [dispatch(x[s], ids[s], num_instances, quant_mode, mask=None if m is None else m[s], smooth=smooth)
+         for s in dom]
+    n = d[0]["n"] + d[1]["n"]
+    E = num_instances
+
+    def gather(a0, a1):
+        rb = int(a0[0].nbytes) if a0.ndim > 1 else a0.dtype.itemsize
+        out = np.zeros((T * K,) + a0.shape[1:], a0.dtype)
+        m0 = np.full((a0.shape[0],), -1, np.int32)
+        m1 = np.full((a1.shape[0],), -1, np.int32)
+        tc = np.zeros((E, 2), np.int32)
+        lib().orc_tp_allgather(E, rb, _p(np.ascontiguousarray(a0)), _p(d[0]["offsets"]),
+                               _p(np.ascontiguousarray(a1)), _p(d[1]["offsets"]), _p(out), _p(m0), _p(m1), _p(tc))
+        return out, m0, m1, tc
+
+    ex, m0, m1, tc = gather(d[0]["expand_x"], d[1]["expand_x"])
+    ds = None if d[0]["dyn_scales"] is None else gather(d[0]["dyn_scales"], d[1]["dyn_scales"])[0]
+    idx = np.empty((T, K), np.int32)
+    for t, mp in enumerate((m0, m1)):
+        di = d[t]["expand_idx"]
+        idx[dom[t]] = np.where(di >= 0, mp[np.maximum(di, 0)], -1)
+    src = np.empty((n,), np.int32)
+    for t, mp in enumerate((m0, m1)):
+        nt = d[t]["n"]
+        src[mp[:nt]] = d[t]["src_of_row"] + t * ep_world_size * bs * K
+    cnt = tc.sum(axis=1).astype(np.int32)
+    off = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32)
+    return dict(expand_x=ex, dyn_scales=ds, expand_idx=idx, src_of_row=src, counts=cnt, offsets=off, n=n,
+                tp_counts=tc, err=d[0]["err"] | d[1]["err"])
+
+
+def tp_reduce(p0_bf16, p1_bf16):
+    """ReduceScatterV of the TP pair (READING R26): bf16 of the exact sum of
+    the two partial outputs of each row."""
+    a = _c(p0_bf16, np.uint16)
+    b = _c(p1_bf16, np.uint16)
+    if a.shape != b.shape:
+        raise ValueError("the two partial outputs must have the same shape")
+    out = np.empty_like(a)
+    lib().orc_tp_reduce(a.size, _p(a), _p(b), _p(out))
+    return out
+
+
+def combine_add_rmsnorm_tp(p0_bf16, p1_bf16, expand_idx, expert_scales, residual_x, gamma, norm_eps,
+                           shared_x=None):
+    """aclnnMoeDistributeCombineAddRmsNorm with a TP domain of two ranks:
+    rsOut = ReduceScatterV(expandX), then the AllToAllV back, the weighted
+    sum, the residual and RMSNorm as without TP."""
+    return combine_add_rmsnorm(tp_reduce(p0_bf16, p1_bf16), expand_idx, expert_scales, residual_x, gamma,
+                               norm_eps, shared_x=shared_x)

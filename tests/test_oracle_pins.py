@@ -726,3 +726,79 @@ def test_grouped_matmul_mx_block_factors_closed_form(orc):
     assert r["err"] == 0
     assert r["out_f64"][0, 0] == 32 * (1 + 2 + 2.0 ** 1 + 2.0 ** -4)
     assert r["out_f64"][0, 1] == 32 * (1 + 2 + 0.5 + 8)
+
+
+# --------------------------------------------------------------------------
+# TP domain of two ranks (READING R26)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode,smooth", [(0, False), (2, True), (3, False), (4, False)])
+def test_tp_dispatch_is_the_tp_major_multi_source_order(orc, mode, smooth):
+    """Each TP domain's AllToAllV followed by the pair's AllGatherV (the
+    pages' two steps, done separately) gives, with one instance per rank,
+    the same rows as one dispatch of all 2 * ws * Bs tokens numbered
+    TP-major; tp_counts are the per-domain counts by brute force."""
+    rng = np.random.default_rng(26)
+    ws, bs, K, H = 8, 5, 3, 1024
+    E, T = ws, 2 * ws * bs
+    x = gen.bf16_bits(rng.standard_normal((T, H), np.float32))
+    ids = gen.topk_uniform(rng, T, E, K)
+    mask = (rng.random((T, K)) > 0.2).astype(np.uint8)
+    sm = rng.uniform(0.5, 2.0, size=(E, H)).astype(np.float32) if smooth else None
+    tp = orc.dispatch_tp(x, ids, E, mode, ws, bs, mask=mask, smooth=sm)
+    one = orc.dispatch(x, ids, E, mode, mask=mask, smooth=sm)
+    assert tp["err"] == 0 and one["err"] == 0
+    n = one["n"]
+    assert tp["n"] == n
+    for key in ("expand_idx", "counts", "offsets", "src_of_row"):
+        np.testing.assert_array_equal(tp[key], one[key])
+    np.testing.assert_array_equal(tp["expand_x"][:n], one["expand_x"][:n])
+    if one["dyn_scales"] is not None:
+        np.testing.assert_array_equal(tp["dyn_scales"][:n], one["dyn_scales"][:n])
+    for t in range(2):
+        dom = slice(t * ws * bs, (t + 1) * ws * bs)
+        for e in range(E):
+            assert tp["tp_counts"][e, t] == int(((ids[dom] == e) & (mask[dom] != 0)).sum())
+
+
+def test_tp_reduce_against_ml_dtypes(orc):
+    """ReduceScatterV's bf16 result: the exact sum of two bf16 values
+    (exact in binary64) rounded by ml_dtypes' bfloat16 cast; includes exact
+    ties (1 + 2^-8 -> 1, (1 + 2^-7) + 2^-8 -> 1 + 2^-6), a partial of zero,
+    and swapped operands."""
+    rng = np.random.default_rng(126)
+    a = gen.bf16_bits(rng.standard_normal(4096, np.float32) * np.exp2(rng.integers(-20, 20, 4096)))
+    b = gen.bf16_bits(rng.standard_normal(4096, np.float32) * np.exp2(rng.integers(-20, 20, 4096)))
+    ties = bits([1.0, 1.0 + 2.0 ** -7, -1.0])
+    tie_b = bits([2.0 ** -8, 2.0 ** -8, -(2.0 ** -8)])
+    a, b = np.concatenate([a, ties]), np.concatenate([b, tie_b])
+    got = orc.tp_reduce(a, b)
+    f = lambda u: (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    want = (f(a) + f(b)).astype(ml_dtypes.bfloat16).view(np.uint16)
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(got[-3:], bits([1.0, 1.0 + 2.0 ** -6, -1.0]))
+    np.testing.assert_array_equal(orc.tp_reduce(b, a), got)
+    nz = f(a) != 0
+    np.testing.assert_array_equal(orc.tp_reduce(a, np.zeros_like(a))[nz], a[nz])
+
+
+def test_tp_combine_closed_forms(orc):
+    """With one partial zero the TP combine is the combine of the other;
+    with two equal partials of exactly representable doubles it is the
+    combine of the doubled rows."""
+    rng = np.random.default_rng(226)
+    bs, K, H, rows = 6, 3, 1024, 18
+    p0 = gen.bf16_bits(rng.standard_normal((rows, H), np.float32))
+    idx = rng.permutation(rows).reshape(bs, K).astype(np.int32)
+    idx[0, 1] = -1
+    w = rng.random((bs, K)).astype(np.float32)
+    res = gen.bf16_bits(rng.standard_normal((bs, H), np.float32))
+    g = gen.bf16_bits(rng.uniform(0.5, 1.5, H).astype(np.float32))
+    a = orc.combine_add_rmsnorm_tp(p0, np.zeros_like(p0), idx, w, res, g, 1e-6)
+    b = orc.combine_add_rmsnorm(p0, idx, w, res, g, 1e-6)
+    np.testing.assert_array_equal(a["y"], b["y"])
+    f = (p0.astype(np.uint32) << 16).view(np.float32)
+    doubled = gen.bf16_bits(f * 2.0)  # exact: a power-of-two scale
+    c = orc.combine_add_rmsnorm_tp(p0, p0, idx, w, res, g, 1e-6)
+    d = orc.combine_add_rmsnorm(doubled, idx, w, res, g, 1e-6)
+    np.testing.assert_array_equal(c["y"], d["y"])
