@@ -58,8 +58,9 @@ class GmmParams(ctypes.Structure):
 EXPORTS = (
     "moe_workspace_init", "moe_read_device_error", "moe_clear_device_error", "moe_status_string",
     "moe_update_expert_workspace_size", "moe_update_expert",
-    "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_route",
-    "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm", "moe_combine",
+    "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_route", "moe_dispatch_tp_counts",
+    "moe_combine_add_rmsnorm_workspace_size", "moe_combine_add_rmsnorm", "moe_combine_add_rmsnorm_tp2",
+    "moe_combine",
     "moe_dispatch_noalloc", "moe_grouped_matmul_workspace_size", "moe_grouped_matmul", "moe_grouped_matmul_mx",
     "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_push", "moe_ep_pull", "moe_ep_dispatch",
     "moe_ep_combine_add_rmsnorm",
@@ -95,6 +96,8 @@ def _load():
     L.moe_ep_push.argtypes = [P(EpParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_ep_pull.argtypes = [P(EpParams), vp, vp, vp, vp, sz, vp]
     L.moe_dispatch_route.argtypes = [P(DispatchParams), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_dispatch_tp_counts.argtypes = [P(DispatchParams), vp, vp, vp, vp, sz, vp]
+    L.moe_combine_add_rmsnorm_tp2.argtypes = [P(CombineParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_ep_dispatch.argtypes = [P(DispatchParams), P(EpParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                   vp]
     L.moe_ep_combine_add_rmsnorm.argtypes = [P(CombineParams), P(EpParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
@@ -389,6 +392,65 @@ def combine_add_rmsnorm(expand_x, expand_idx, expert_scales, residual_x, gamma, 
             ctypes.byref(p), _ptr(expand_x), _ptr(expand_idx), _ptr(expert_scales), _ptr(shared_x),
             _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")), _ptr(out.get("rstd")),
             _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def dispatch_tp_counts(route: dict, bs, hidden, top_k, ep_world_size, quant_mode, scales_len=0, workspace=None,
+                       out=None, stream=None):
+    """moe_dispatch_tp_counts: [E, 2] rows per (instance, TP domain) of a
+    dispatch over 2 * ep_world_size TP-major sources with one instance per
+    rank.  route: the dispatch's output dict (src_of_row, offsets)."""
+    E = ep_world_size
+    S = 2 * ep_world_size
+    if not isinstance(route, dict):
+        raise TypeError("route must be the dispatch's output dict")
+    src, off = route.get("src_of_row"), route.get("offsets")
+    _req(src, "route['src_of_row']", torch.int32, (S * bs * top_k,))
+    _req(off, "route['offsets']", torch.int32, (E + 1,))
+    dev = src.device
+    if out is None:
+        out = torch.empty((E, 2), dtype=torch.int32, device=dev)
+    _req(out, "out", torch.int32, (E, 2))
+    p = DispatchParams(int(bs), int(hidden), int(top_k), int(ep_world_size), E, int(quant_mode), int(scales_len), S)
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(dev, stream)
+        _same_device(dev, ("route['offsets']", off), ("out", out), ("workspace", ws))
+        _check("moe_dispatch_tp_counts", lib.moe_dispatch_tp_counts(
+            ctypes.byref(p), _ptr(src), _ptr(off), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def combine_add_rmsnorm_tp2(expand_x0, expand_x1, expand_idx, expert_scales, residual_x, gamma, norm_eps,
+                            shared_x=None, want_x_out=False, want_rstd=False, workspace=None, out=None,
+                            stream=None, sources=1):
+    """moe_combine_add_rmsnorm_tp2: the combine whose rows are the bf16 sums
+    of the TP pair's two partial outputs.  Returns a dict like
+    combine_add_rmsnorm."""
+    _req(expand_x0, "expand_x0", torch.bfloat16)
+    _req(expand_x1, "expand_x1", torch.bfloat16, tuple(expand_x0.shape))
+    rows, H = expand_x0.shape
+    dev = expand_x0.device
+    _req(expand_idx, "expand_idx", torch.int32)
+    bs, k = expand_idx.shape
+    _req(expert_scales, "expert_scales", torch.float32, (bs, k))
+    _req(residual_x, "residual_x", torch.bfloat16, (bs, H))
+    _req(gamma, "gamma", torch.bfloat16, (H,))
+    _opt(shared_x, "shared_x", torch.bfloat16, (bs, H))
+    if out is None:
+        out = dict(y=torch.empty((bs, H), dtype=torch.bfloat16, device=dev),
+                   x_out=torch.empty((bs, H), dtype=torch.bfloat16, device=dev) if want_x_out else None,
+                   rstd=torch.empty((bs,), dtype=torch.float32, device=dev) if want_rstd else None)
+    _check_combine_out(out, bs, H)
+    p = CombineParams(_per_source(bs, sources, "combine_add_rmsnorm_tp2"), H, k, rows, float(norm_eps), int(sources))
+    with torch.cuda.device(dev):
+        ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(dev, stream)
+        _same_device(dev, ("expand_x1", expand_x1), ("expand_idx", expand_idx), ("expert_scales", expert_scales),
+                     ("residual_x", residual_x), ("gamma", gamma), ("shared_x", shared_x), ("workspace", ws),
+                     *((f"out['{n}']", t) for n, t in out.items()))
+        _check("moe_combine_add_rmsnorm_tp2", lib.moe_combine_add_rmsnorm_tp2(
+            ctypes.byref(p), _ptr(expand_x0), _ptr(expand_x1), _ptr(expand_idx), _ptr(expert_scales),
+            _ptr(shared_x), _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")),
+            _ptr(out.get("rstd")), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 

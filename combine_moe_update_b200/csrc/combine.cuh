@@ -38,6 +38,10 @@ struct CombineArgs {
     const uint16_t *const *peer_rows;
     const int32_t *gbase;  // [G + 1]
     int gpus, recv_rows;
+    // TP domain of two ranks (TP2 kernels): the second TP rank's partial
+    // expert outputs of the same rows; each gathered row is the bf16 of the
+    // sum of the two (the ReduceScatterV).
+    const uint16_t *expand_x1;
 };
 
 // K 16 with the norm keeps the pre-norm row in shared memory (XS) and runs
@@ -69,7 +73,10 @@ __host__ __device__ inline int cb_threads(int NV, int vecs) {
 // residual, no norm).
 // EP: the rows come from the GPUs that own them (expert parallelism across
 // GPUs, the AllToAllV back fused into the gather).
-template <int KMAX, bool SHARED, int NT, bool NORM, int SPLIT, bool EP = false>
+// TP2: each gathered row is bf16(expand_x[row] + expand_x1[row]) (the TP
+// pair's ReduceScatterV fused into the gather; the fp32 sum of two bf16
+// values rounds to the same bf16 as their exact sum).
+template <int KMAX, bool SHARED, int NT, bool NORM, int SPLIT, bool EP = false, bool TP2 = false>
 __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_token_kernel(CombineArgs a) {
     constexpr int VECS = SPLIT == 1 ? 4 : 2;
     // XS: the pre-norm row waits for the sum of squares in shared memory
@@ -158,15 +165,17 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
         // all top-K rows in flight at once up to K 8; at K 16 eight at a
-        // time (registers: four blocks per SM with XS, no spills without)
-        constexpr int CH = KMAX == 16 ? 8 : KMAX;
+        // time (registers: four blocks per SM with XS, no spills without);
+        // TP2 loads two rows per copy, four copies at a time
+        constexpr int CH = TP2 ? (KMAX < 4 ? KMAX : 4) : (KMAX == 16 ? 8 : KMAX);
 #pragma unroll
         for (int k0 = 0; k0 < KMAX; k0 += CH) {
-            uint4 rv[CH];
+            uint4 rv[CH], rw[TP2 ? CH : 1];
 #pragma unroll
             for (int k = 0; k < CH; ++k) {  // nk is the same in every thread: a uniform branch
                 if (k0 + k >= nk) break;
                 rv[k] = ld_stream((EP ? s_src[k0 + k] : a.expand_x + (size_t)row[k0 + k] * H) + p * 8);
+                if constexpr (TP2) rw[k] = ld_stream(a.expand_x1 + (size_t)row[k0 + k] * H + p * 8);
             }
             if (k0 == 0) {
                 if constexpr (NORM) res = ld_stream(a.residual + tok + p * 8);
@@ -177,6 +186,12 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
                 if (k0 + k >= nk) break;
                 float f[8];
                 unpack8(rv[k], f);
+                if constexpr (TP2) {
+                    float g2[8];
+                    unpack8(rw[k], g2);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = __bfloat162float(__float2bfloat16_rn(f[e] + g2[e]));
+                }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) acc[e] = fmaf(wk[k0 + k], f[e], acc[e]);
             }

@@ -243,6 +243,36 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(DispatchArgs a) {
     }
 }
 
+// --------------------------------------------------- TP domain counts ---
+//
+// With a TP domain of two ranks and one instance per EP rank, the rows of
+// instance e come from the 2 * ws source devices in TP-major order, so
+// TP domain 0's rows of e (sources < ws) come first.  One thread per
+// instance finds the first row of domain 1 by a binary search over the
+// rows' copy ids (source = id / (bs * K)).
+__global__ void __launch_bounds__(1024) tp_counts_kernel(const int32_t *src_of_row, const int32_t *offsets,
+                                                         int32_t *tp_counts, int num_instances, int copies,
+                                                         int copies_per_source, int ws, uint32_t *err) {
+    pdl_wait();  // the routing comes from earlier kernels
+    for (int e = threadIdx.x; e < num_instances; e += blockDim.x) {
+        const int lo0 = ld_in(offsets + e), hi0 = ld_in(offsets + e + 1);
+        if (lo0 < 0 || hi0 < lo0 || hi0 > copies) {
+            raise_error(err, kDevBadId);
+            tp_counts[2 * e] = 0;
+            tp_counts[2 * e + 1] = 0;
+            continue;
+        }
+        int lo = lo0, hi = hi0;  // first row in [lo0, hi0) whose source is >= ws
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (ld_in(src_of_row + mid) / copies_per_source < ws) lo = mid + 1; else hi = mid;
+        }
+        tp_counts[2 * e] = lo - lo0;
+        tp_counts[2 * e + 1] = hi0 - lo;
+    }
+    pdl_launch_dependents();
+}
+
 // ----------------------------------------------------------- block route ---
 //
 // For a small call (at most kFusedRouteMax copies) every token block

@@ -85,7 +85,7 @@ bool valid_update(const moe_update_params &p) {
     if (p.ep_world_size < MOE_MIN_EP_WORLD || p.ep_world_size > MOE_MAX_EP_WORLD) return false;
     if (p.table_cols < 2 || p.table_cols > p.ep_world_size + 1) return false;
     if (!(p.prune_threshold == p.prune_threshold)) return false;  // NaN
-    if (p.sources < 0 || p.sources > p.ep_world_size) return false;
+    if (p.sources < 0 || p.sources > 2 * p.ep_world_size) return false;  // 2 * ws with a TP domain of two
     return true;
 }
 
@@ -97,7 +97,7 @@ moe_status valid_dispatch(const moe_dispatch_params &p) {
     if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K || p.top_k > p.num_instances) return MOE_ERR_INVALID_ARG;
     if (p.ep_world_size < MOE_MIN_EP_WORLD || p.ep_world_size > MOE_MAX_EP_WORLD) return MOE_ERR_INVALID_ARG;
     if (p.num_instances % p.ep_world_size != 0) return MOE_ERR_INVALID_ARG;  // equal instances per rank
-    if (p.sources < 0 || p.sources > p.ep_world_size) return MOE_ERR_INVALID_ARG;
+    if (p.sources < 0 || p.sources > 2 * p.ep_world_size) return MOE_ERR_INVALID_ARG;  // 2 * ws with TP
     if (p.quant_mode < 0 || p.quant_mode > 4) return MOE_ERR_INVALID_ARG;
     const long long eh = (long long)p.num_instances * p.hidden;
     if (p.quant_mode == 1 && p.scales_len != 1 && p.scales_len != p.hidden && p.scales_len != eh)
@@ -115,7 +115,7 @@ bool valid_combine(const moe_combine_params &p) {
     if (p.top_k < 1 || p.top_k > MOE_MAX_TOP_K) return false;
     if (p.expand_rows < 1) return false;
     if (!(p.norm_eps >= 0.0f) || p.norm_eps > 3.0e38f) return false;  // rejects NaN and inf
-    if (p.sources < 0 || p.sources > MOE_MAX_EP_WORLD) return false;
+    if (p.sources < 0 || p.sources > 2 * MOE_MAX_EP_WORLD) return false;
     return true;
 }
 
@@ -305,6 +305,33 @@ cudaError_t launch_combine_split(const moe::CombineArgs &a, cudaStream_t s) {
     return split ? launch_combine_tok<KMAX, false, NORM, 2>(a, s) : launch_combine_tok<KMAX, false, NORM, 1>(a, s);
 }
 
+// The combine of a TP pair: each row is the bf16 sum of the two partial outputs (one block per token).
+template <int KMAX, bool SHARED, int NT>
+cudaError_t launch_combine_tp2_nt(const moe::CombineArgs &a, cudaStream_t s) {
+    auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, true, 1, false, true>;
+    constexpr int smem = moe::cb_smem_bytes(KMAX, NT, true, 1);
+    if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
+    return launch(kernel, a.bs, NT, smem, s, a);
+}
+
+template <int KMAX, bool SHARED>
+cudaError_t launch_combine_tp2_tok(const moe::CombineArgs &a, cudaStream_t s) {
+    switch (moe::cb_threads(a.hidden >> 3, 4)) {
+        case 64: return launch_combine_tp2_nt<KMAX, SHARED, 64>(a, s);
+        case 128: return launch_combine_tp2_nt<KMAX, SHARED, 128>(a, s);
+        case 192: return launch_combine_tp2_nt<KMAX, SHARED, 192>(a, s);
+        case 224: return launch_combine_tp2_nt<KMAX, SHARED, 224>(a, s);
+        default: return launch_combine_tp2_nt<KMAX, SHARED, 256>(a, s);
+    }
+}
+
+cudaError_t launch_combine_tp2(const moe::CombineArgs &a, int top_k, cudaStream_t s) {
+    const bool sh = a.shared_x != nullptr;
+    if (top_k <= 4) return sh ? launch_combine_tp2_tok<4, true>(a, s) : launch_combine_tp2_tok<4, false>(a, s);
+    if (top_k <= 8) return sh ? launch_combine_tp2_tok<8, true>(a, s) : launch_combine_tp2_tok<8, false>(a, s);
+    return sh ? launch_combine_tp2_tok<16, true>(a, s) : launch_combine_tp2_tok<16, false>(a, s);
+}
+
 // The combine that gathers its rows from the GPUs that own them (one block per token).
 template <int KMAX, bool SHARED, int NT>
 cudaError_t launch_combine_ep_nt(const moe::CombineArgs &a, cudaStream_t s) {
@@ -337,6 +364,36 @@ cudaError_t launch_combine_k(const moe::CombineArgs &a, int top_k, cudaStream_t 
     if (top_k <= 4) return launch_combine_split<4, NORM>(a, s);
     if (top_k <= 8) return launch_combine_split<8, NORM>(a, s);
     return launch_combine_split<16, NORM>(a, s);
+}
+
+// Checks and arguments shared by the normed combine calls.
+moe_status combine_norm_args(const moe_combine_params *p, const void *expand_x, const int32_t *expand_idx,
+                             const float *expert_scales, const void *shared_x, const void *residual_x,
+                             const void *gamma, void *y, void *x_out, float *rstd_out, void *workspace,
+                             size_t workspace_bytes, moe::CombineArgs &a) {
+    if (p == nullptr || !valid_combine(*p)) return MOE_ERR_INVALID_ARG;
+    if (!expand_x || !expand_idx || !expert_scales || !residual_x || !gamma || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned(expand_x, 16) || !aligned(residual_x, 16) || !aligned(gamma, 16) || !aligned(y, 16) ||
+        (shared_x && !aligned(shared_x, 16)) || (x_out && !aligned(x_out, 16)) || !aligned(expand_idx, 4) ||
+        !aligned(expert_scales, 4) || (rstd_out && !aligned(rstd_out, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
+    a.bs = total_tokens(p->bs, p->sources);
+    a.hidden = p->hidden;
+    a.top_k = p->top_k;
+    a.expand_rows = p->expand_rows;
+    a.norm_eps = p->norm_eps;
+    a.expand_x = reinterpret_cast<const uint16_t *>(expand_x);
+    a.expand_idx = expand_idx;
+    a.scales = expert_scales;
+    a.shared_x = reinterpret_cast<const uint16_t *>(shared_x);
+    a.residual = reinterpret_cast<const uint16_t *>(residual_x);
+    a.gamma = reinterpret_cast<const uint16_t *>(gamma);
+    a.y = reinterpret_cast<uint16_t *>(y);
+    a.x_out = reinterpret_cast<uint16_t *>(x_out);
+    a.rstd_out = rstd_out;
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    return MOE_OK;
 }
 
 }  // namespace
@@ -578,31 +635,46 @@ moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const void *expa
                                    const float *expert_scales, const void *shared_x, const void *residual_x,
                                    const void *gamma, void *y, void *x_out, float *rstd_out, void *workspace,
                                    size_t workspace_bytes, void *cuda_stream) {
-    if (p == nullptr || !valid_combine(*p)) return MOE_ERR_INVALID_ARG;
-    if (!expand_x || !expand_idx || !expert_scales || !residual_x || !gamma || !y) return MOE_ERR_INVALID_ARG;
-    if (!aligned(expand_x, 16) || !aligned(residual_x, 16) || !aligned(gamma, 16) || !aligned(y, 16) ||
-        (shared_x && !aligned(shared_x, 16)) || (x_out && !aligned(x_out, 16)) || !aligned(expand_idx, 4) ||
-        !aligned(expert_scales, 4) || (rstd_out && !aligned(rstd_out, 4)))
+    moe::CombineArgs a = {};
+    const moe_status st = combine_norm_args(p, expand_x, expand_idx, expert_scales, shared_x, residual_x, gamma, y,
+                                            x_out, rstd_out, workspace, workspace_bytes, a);
+    if (st != MOE_OK) return st;
+    return launch_combine_k<true>(a, p->top_k, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_combine_add_rmsnorm_tp2(const moe_combine_params *p, const void *expand_x0, const void *expand_x1,
+                                       const int32_t *expand_idx, const float *expert_scales, const void *shared_x,
+                                       const void *residual_x, const void *gamma, void *y, void *x_out,
+                                       float *rstd_out, void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    moe::CombineArgs a = {};
+    const moe_status st = combine_norm_args(p, expand_x0, expand_idx, expert_scales, shared_x, residual_x, gamma, y,
+                                            x_out, rstd_out, workspace, workspace_bytes, a);
+    if (st != MOE_OK) return st;
+    if (!expand_x1 || !aligned(expand_x1, 16)) return MOE_ERR_INVALID_ARG;
+    a.expand_x1 = reinterpret_cast<const uint16_t *>(expand_x1);
+    return launch_combine_tp2(a, p->top_k, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_dispatch_tp_counts(const moe_dispatch_params *p, const int32_t *src_of_row,
+                                  const int32_t *expert_offsets, int32_t *tp_counts, void *workspace,
+                                  size_t workspace_bytes, void *cuda_stream) {
+    if (p == nullptr) return MOE_ERR_INVALID_ARG;
+    moe_status st = valid_dispatch(*p);
+    if (st != MOE_OK) return st;
+    // a TP domain of two ranks: one instance per EP rank, every one of the 2 * ws devices a source
+    if (p->num_instances != p->ep_world_size || p->sources != 2 * p->ep_world_size) return MOE_ERR_INVALID_ARG;
+    if (!src_of_row || !expert_offsets || !tp_counts || !aligned(src_of_row, 4) || !aligned(expert_offsets, 4) ||
+        !aligned(tp_counts, 4))
         return MOE_ERR_INVALID_ARG;
     if (!check_workspace(workspace, workspace_bytes)) return MOE_ERR_WORKSPACE;
-
-    moe::CombineArgs a = {};
-    a.bs = total_tokens(p->bs, p->sources);
-    a.hidden = p->hidden;
-    a.top_k = p->top_k;
-    a.expand_rows = p->expand_rows;
-    a.norm_eps = p->norm_eps;
-    a.expand_x = reinterpret_cast<const uint16_t *>(expand_x);
-    a.expand_idx = expand_idx;
-    a.scales = expert_scales;
-    a.shared_x = reinterpret_cast<const uint16_t *>(shared_x);
-    a.residual = reinterpret_cast<const uint16_t *>(residual_x);
-    a.gamma = reinterpret_cast<const uint16_t *>(gamma);
-    a.y = reinterpret_cast<uint16_t *>(y);
-    a.x_out = reinterpret_cast<uint16_t *>(x_out);
-    a.rstd_out = rstd_out;
-    a.err = reinterpret_cast<uint32_t *>(workspace);
-    return launch_combine_k<true>(a, p->top_k, as_stream(cuda_stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    const int per_source = p->bs * p->top_k;
+    const int copies = per_source * p->sources;
+    const int threads = p->num_instances < 1024 ? ((p->num_instances + 31) / 32) * 32 : 1024;
+    return launch(moe::tp_counts_kernel, 1, threads, 0, as_stream(cuda_stream), src_of_row, expert_offsets,
+                  tp_counts, p->num_instances, copies, per_source, p->ep_world_size,
+                  reinterpret_cast<uint32_t *>(workspace)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 // The plain combine (CombineV2 series): combineOut only.

@@ -44,7 +44,11 @@
  *     every EP rank send Bs tokens.  With sources = S, the calls take
  *     T = S * bs tokens, rank-major (token t = r * bs + i of source rank r);
  *     rows are ordered by (instance, r, i, k), the same as (instance, t, k).
- *     0 means 1.
+ *     0 means 1.  S goes up to 2 * ep_world_size: with a TP domain of two
+ *     ranks (tpWorldSize 2 on the pages) every one of the 2 * ep_world_size
+ *     devices is a source, numbered TP-major (device t * ep_world_size + g
+ *     is EP rank g of TP domain t); see moe_dispatch_tp_counts and
+ *     moe_combine_add_rmsnorm_tp2.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -119,7 +123,7 @@ typedef struct {
     int32_t ep_world_size;  /* simulated ranks, [2, 768] */
     float prune_threshold;  /* copies whose expert_scales entry is strictly below this are
                                pruned; <= 0 (or expert_scales == NULL) disables */
-    int32_t sources;        /* source ranks S, [0, ep_world_size] (0 = 1): arrays hold S * bs tokens */
+    int32_t sources;        /* source ranks S, [0, 2 * ep_world_size] (0 = 1): arrays hold S * bs tokens */
 } moe_update_params;
 
 MOE_API moe_status moe_update_expert_workspace_size(const moe_update_params *p, size_t *bytes);
@@ -168,7 +172,7 @@ typedef struct {
     int32_t quant_mode;     /* 0 none, 1 static int8, 2 per-token int8, 3 per-128-tile int8, 4 mxfp8 */
     int32_t scales_len;     /* floats in smooth_scales: 0 when it is NULL; modes 2/3 num_instances * H;
                                mode 1: 1, H or num_instances * H (the static scales' shape) */
-    int32_t sources;        /* source ranks S, [0, ep_world_size] (0 = 1): x and the routing hold
+    int32_t sources;        /* source ranks S, [0, 2 * ep_world_size] (0 = 1): x and the routing hold
                                S * bs tokens, expand_x S * bs * K rows */
 } moe_dispatch_params;
 
@@ -223,6 +227,26 @@ MOE_API moe_status moe_dispatch(const moe_dispatch_params *p, const void *x, con
  * no row moved (the rows follow from moe_ep_dispatch once the group's counts
  * are known).  Arguments, limits and errors as moe_dispatch.
  */
+/*
+ * The per-(rank, TP domain) row counts of a dispatch with a TP domain of two
+ * ranks (aclnnMoeDistributeDispatchV2, "计算公式": expandXOut =
+ * AllGatherV(allToAllXOut); its expertTokenNums has epWorldSize * tpWorldSize
+ * * localExpertNum entries).  With one instance per EP rank
+ * (num_instances == ep_world_size, the pages allow TP only then) and
+ * sources = 2 * ep_world_size numbered TP-major, moe_dispatch's rows of
+ * instance e are rank e's gathered buffer: TP domain 0's rows first, then
+ * domain 1's.  This call splits each instance's rows at that boundary.
+ *   p              the moe_dispatch parameters of the call (sources = 2 * ws,
+ *                  num_instances = ws, else MOE_ERR_INVALID_ARG)
+ *   src_of_row, expert_offsets: moe_dispatch's outputs
+ *   tp_counts      [E, 2] int32 device, out: rows of (instance e, TP domain t)
+ * Device errors: offsets outside [0, rows] set MOE_DEV_BAD_ID (that
+ * instance's counts are 0).
+ */
+MOE_API moe_status moe_dispatch_tp_counts(const moe_dispatch_params *p, const int32_t *src_of_row,
+                                          const int32_t *expert_offsets, int32_t *tp_counts, void *workspace,
+                                          size_t workspace_bytes, void *cuda_stream);
+
 MOE_API moe_status moe_dispatch_route(const moe_dispatch_params *p, const int32_t *instance_ids,
                                       const uint8_t *mask, int32_t *expand_idx, int32_t *src_of_row,
                                       int32_t *expert_counts, int32_t *expert_offsets, void *workspace,
@@ -238,7 +262,7 @@ typedef struct {
     int32_t top_k;        /* K, (0, 16] */
     int32_t expand_rows;  /* rows of expand_x (>= every non-negative expand_idx + 1), > 0 */
     float norm_eps;       /* normEps, finite and >= 0 */
-    int32_t sources;      /* source ranks S, [0, 768] (0 = 1): the token arrays hold S * bs tokens */
+    int32_t sources;      /* source ranks S, [0, 1536] (0 = 1): the token arrays hold S * bs tokens */
 } moe_combine_params;
 
 MOE_API moe_status moe_combine_add_rmsnorm_workspace_size(const moe_combine_params *p, size_t *bytes);
@@ -269,6 +293,27 @@ MOE_API moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const vo
                                    const void *shared_x, const void *residual_x, const void *gamma,
                                    void *y, void *x_out, float *rstd_out, void *workspace,
                                    size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * The same with a TP domain of two ranks (aclnnMoeDistributeCombineAddRmsNorm,
+ * "计算公式": rsOut = ReduceScatterV(expandX), then ataOut = AllToAllV(rsOut)):
+ * each TP rank holds a partial expert output of all its pair's rows; row r
+ * of rsOut is the bf16 (round to nearest even) of expand_x0[r] + expand_x1[r]
+ * (the sum of two bf16 values in fp32 rounds to the same bf16 as their
+ * exact sum), and each token reads its own rows of it.  On one device the
+ * token arrays hold every source device's tokens (sources = 2 * ws,
+ * TP-major), so the scatter half and the AllToAllV back are the gather
+ * through expand_idx.
+ *   expand_x0, expand_x1 [expand_rows, H] bf16 device, 16-byte aligned: the
+ *                        two TP ranks' partial outputs
+ * Other arguments and errors as moe_combine_add_rmsnorm.
+ */
+MOE_API moe_status moe_combine_add_rmsnorm_tp2(const moe_combine_params *p, const void *expand_x0,
+                                               const void *expand_x1, const int32_t *expand_idx,
+                                               const float *expert_scales, const void *shared_x,
+                                               const void *residual_x, const void *gamma, void *y, void *x_out,
+                                               float *rstd_out, void *workspace, size_t workspace_bytes,
+                                               void *cuda_stream);
 
 /*
  * The plain combine of the CombineV2 series, which the dispatch page names as
