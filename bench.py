@@ -69,7 +69,9 @@ def algorithmic_bytes(w, n, x_out=False, rstd=False):
             + items * (4 + 1)               # instance ids + mask
             + items * 4 + n * 4             # expand_idx + src_of_row
             + 4 * E + 4 * (E + 1))          # counts + offsets
-    comb = (n * 2 * H                       # expert rows gathered back
+    if int(w.meta.get("tp", 1)) == 2:       # the per-(rank, domain) counts
+        disp += 4 * (E + 1) + 8 * E
+    comb = (n * 2 * H * int(w.meta.get("tp", 1))  # expert rows gathered back (both TP partials)
             + 2 * bs * H                    # residual
             + (2 * bs * H if w.shared_x is not None else 0)
             + 2 * H                         # gamma
@@ -91,6 +93,8 @@ def kernels_per_step(w):
         disp = 1
     else:
         disp = 2
+    if int(w.meta.get("tp", 1)) == 2:
+        disp += 1  # the per-(rank, domain) counts
     return 1 + disp + 1
 
 
@@ -239,13 +243,29 @@ def run_b200(args, rank, world, local_rank):
     gamma = bf(w.gamma)
     # this batch's activations
     ids, scales = dev(w.expert_ids), dev(w.expert_scales)
-    x, residual, expert_out = bf(w.x), bf(w.residual), bf(w.expert_out)
-    shared = None if w.shared_x is None else bf(w.shared_x)
-    # several source ranks (every simulated rank sends its own tokens)
+    # several source ranks (every simulated rank sends its own tokens); a TP
+    # pair's two partial expert outputs of every row as one [2, rows, H] tensor
     S = int(w.meta.get("sources", 1))
+    TP = int(w.meta.get("tp", 1))
+    x, residual = bf(w.x), bf(w.residual)
+    expert_out = bf(w.expert_out) if TP == 1 else bf(np.stack([w.expert_out, w.meta["expert_out_tp1"]]))
+    shared = None if w.shared_x is None else bf(w.shared_x)
     upd = functools.partial(B.update_expert, sources=S)
-    disp = functools.partial(B.dispatch, sources=S)
-    comb = functools.partial(B.combine_add_rmsnorm, sources=S)
+    if TP == 1:
+        disp = functools.partial(B.dispatch, sources=S)
+        comb = functools.partial(B.combine_add_rmsnorm, sources=S)
+    else:
+        tpc = torch.empty((w.num_instances, 2), dtype=torch.int32, device="cuda")
+        tp_sl = 0 if w.smooth is None else w.smooth.size
+
+        def disp(xx, *a, **k):  # the dispatch over the TP-major sources, then the per-(rank, domain) counts
+            o = B.dispatch(xx, *a, sources=S, **k)
+            B.dispatch_tp_counts(o, w.bs // S, w.hidden, w.top_k, w.ep_world_size, w.quant_mode, scales_len=tp_sl,
+                                 workspace=k.get("workspace"), out=tpc)
+            return o
+
+        def comb(ee, *a, **k):  # the ReduceScatterV of the two partials fused into the gather
+            return B.combine_add_rmsnorm_tp2(ee[0], ee[1], *a, sources=S, **k)
     ws = B.new_workspace(nbytes=B.dispatch_workspace_bytes(
         w.bs // S, w.hidden, w.top_k, w.ep_world_size, w.num_instances, w.quant_mode,
         0 if w.smooth is None else w.smooth.size, S))
@@ -529,8 +549,8 @@ def run_b200(args, rank, world, local_rank):
         "config": {"workload": args.workload, "bs": w.bs, "hidden": w.hidden, "top_k": w.top_k,
                    "num_instances": w.num_instances, "ep_world_size_simulated": w.ep_world_size,
                    "quant_mode": w.quant_mode, "smooth_scales": w.smooth is not None,
-                   "shared_expert": w.shared_x is not None, "kept_copies": n,
-                   "l2": l2_note, "parallelism": f"replicas x{world}"},
+                   "shared_expert": w.shared_x is not None, "kept_copies": n, "source_ranks": S,
+                   "tp_world_size": TP, "l2": l2_note, "parallelism": f"replicas x{world}"},
         "gate": gate,
         "breakdown_us": {"update_expert": round(t_upd * 1e3, 2), "dispatch": round(t_disp * 1e3, 2),
                          "combine": round(t_comb * 1e3, 2),
@@ -1072,6 +1092,10 @@ def oracle_step(orc, w):
     rows = w.expert_out
     if "expert_out_dim" in w.meta:
         rows = _oracle_expert_rows(orc, w, d)
+    if int(w.meta.get("tp", 1)) == 2:  # a slice of the TP-major tokens: its rows are the pair's gathered order
+        orc.combine_add_rmsnorm_tp(rows, w.meta["expert_out_tp1"], d["expand_idx"], w.expert_scales, w.residual,
+                                   w.gamma, w.norm_eps, shared_x=w.shared_x)
+        return
     orc.combine_add_rmsnorm(rows, d["expand_idx"], w.expert_scales, w.residual, w.gamma, w.norm_eps,
                             shared_x=w.shared_x)
 
@@ -1113,6 +1137,8 @@ def subsample(w, tokens, start=0):
             setattr(s, k, v[start:start + tokens].copy())
     s.expert_out = w.expert_out[start * w.top_k:(start + tokens) * w.top_k].copy()
     s.meta = {k: v for k, v in w.meta.items() if not k.startswith("_")}
+    if "expert_out_tp1" in w.meta:
+        s.meta["expert_out_tp1"] = w.meta["expert_out_tp1"][start * w.top_k:(start + tokens) * w.top_k].copy()
     return s
 
 

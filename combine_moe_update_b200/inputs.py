@@ -187,6 +187,17 @@ def _all_ranks_layer(name, seed, bs, sources, **kw):
     return w
 
 
+def _tp_layer(name, seed, bs, ep_world_size, **kw):
+    """A TP domain of two ranks: 2 * ep_world_size devices of Bs tokens each
+    (TP-major), one instance per EP rank, and the TP pair's second partial
+    expert output of every row (the first is the workload's expert_out)."""
+    S = 2 * ep_world_size
+    w = uniform_layer(name, seed, bs=bs * S, num_experts=ep_world_size, ep_world_size=ep_world_size, **kw)
+    rng = np.random.Generator(np.random.PCG64([seed, 26]))
+    w.meta.update(sources=S, tp=2, expert_out_tp1=bf16_bits(rng.standard_normal(w.expert_out.shape, np.float32)))
+    return w
+
+
 def _static_layer(name, seed, **kw):
     """A uniform layer with static int8 quantization (quantMode 1): per-instance
     static scales U(10, 40), so x ~ N(0, 1) fills much of the int8 range and
@@ -252,6 +263,12 @@ WORKLOADS = {
                                 ep_world_size=8, quant_mode=4, shared=True, expert_out_dim=7168),
     # Zipf(1.2) routing over 128 experts, 160 instances on 16 ranks, mxfp8.
     "skewed_eplb": dict(builder=_skewed_eplb, seed=2, bs=512),
+    # A TP domain of two ranks: 32 EP ranks with one expert each, every EP rank
+    # a TP pair (64 devices of Bs 64 tokens, 4096 tokens, 32768 copies), H
+    # 7168, K 8, per-token int8 with smooth scales, shared expert; the combine
+    # reads both TP ranks' partial outputs of every row.
+    "tp2_decode": dict(builder=_tp_layer, seed=5, bs=64, ep_world_size=32, hidden=7168, top_k=8, quant_mode=2,
+                       smooth=True, shared=True),
     # Largest shapes: H 8192, 1024 experts, K 16, 256 ranks, per-128-tile int8,
     # threshold pruning at 0.05 on softmax weights of N(0, 2) logits.
     "max_shape": dict(builder=uniform_layer, seed=3, bs=512, hidden=8192, num_experts=1024,
