@@ -707,6 +707,42 @@ def run_b200_layer_stack(args, rank, world, local_rank):
     return out, st
 
 
+def graph_time(body, sets, steps):
+    """Per-call time (ms) of `body(n)` captured for n < count (count = sets
+    rounded up to at least 16 calls) in one CUDA graph with events only at
+    its ends, averaged over a few replays."""
+    import torch
+    count = sets * max(1, -(-16 // sets))
+    eb = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        eb[0].record()
+        for n_ in range(count):
+            body(n_)
+        eb[1].record()
+    g.replay()
+    torch.cuda.synchronize()
+    reps = max(3, min(50, steps // 4))
+    tot = 0.0
+    for _ in range(reps):
+        g.replay()
+        torch.cuda.synchronize()
+        tot += eb[0].elapsed_time(eb[1]) / count
+    del g
+    return tot / reps
+
+
+def ep_kernel_roofline(kernel, alg_bytes, t_ms, peak, peak_kind):
+    ach = alg_bytes / (t_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(ach, 1), "peak": peak, "peak_kind": peak_kind,
+            "unit": "GB/s", "frac": round(ach / peak, 4), "launch_us": round(t_ms * 1e3, 2), "traffic": None,
+            "algorithmic_bytes": alg_bytes,
+            "timing": "launches back to back over input sets larger than twice L2, CUDA events at the graph's ends; "
+                      "the dispatch's bytes include the route's outputs (about 0.1 %)"}
+
+
 def run_b200_ep(args, rank, world, local_rank):
     """Expert parallelism across the GPUs of the job: GPU g owns instances
     [g E / N, (g + 1) E / N) and dispatches its own batch; every step is
@@ -761,6 +797,27 @@ def run_b200_ep(args, rank, world, local_rank):
     recv = r.received()
     assert r.device_errors() == 0, "device error during the timed steps"
     n = int(r.d["offsets"][-1].item())
+    # The two EP kernels on their own (one GPU: every owner is this GPU): launches back to back over input sets
+    # larger than twice L2 (x for the dispatch; expert outputs, residual and shared rows for the combine, each
+    # set behind its own pointer table), events only at the graph's ends.
+    t_epd = t_epc = None
+    if fused and world == 1:
+        per_x = x.numel() * x.element_size()
+        Rd = -(-(2 * L2_BYTES) // per_x) + 1
+        xs = [x.clone() for _ in range(Rd)]
+        t_epd = graph_time(lambda n_: r.ep_dispatch(xs[n_ % Rd], grp.tables, smooth=smooth), Rd, K)
+        del xs
+        cset = (r.expert_out, residual, shared)
+        per_c = sum(t.numel() * t.element_size() for t in cset if t is not None)
+        Rc = -(-(2 * L2_BYTES) // per_c) + 1
+        cl = [[None if t is None else t.clone() for t in cset] for _ in range(Rc)]
+        tabs = [EP.PeerTables(None, None, None, [c[0].data_ptr()], r.device) for c in cl]
+        t_epc = graph_time(lambda n_: B.ep_combine_add_rmsnorm(r.p_pull, tabs[n_ % Rc].expert_out, r.global_idx,
+                                                               scales, cl[n_ % Rc][1], gamma, w.norm_eps, r.ep_ws,
+                                                               shared_x=cl[n_ % Rc][2], out=out),
+                           Rc * max(1, 16 // Rc), K)
+        del cl, tabs
+        assert r.device_errors() == 0, "device error in the EP kernel timing"
     grp.close()
     copies = w.bs * w.top_k
     route = 3 if copies > 8192 else 1
@@ -788,11 +845,17 @@ def run_b200_ep(args, rank, world, local_rank):
                    "exchange": "fused into dispatch and combine" if fused else "push and pull",
                    "rows_received_rank0": recv,
                    "l2": "not flushed: each step's exchange and gathers touch more than L2 across the group"},
-        "roofline": {"bound": "hbm", "kernel": ("whole step (update, route, plan, EP dispatch, EP combine)" if fused
-                                                else "whole step (update, dispatch, plan, push, pull, combine)"),
-                     "achieved": round(ach, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(ach / peak, 4), "traffic": None, "algorithmic_bytes": step_bytes,
-                     "note": "eager launches with two NCCL barriers and a count gather per step"},
+        "roofline": ep_kernel_roofline("combine_token_kernel (EP)", alg["combine"], t_epc, peak, peak_kind)
+        if t_epc else None,
+        "roofline_other": ep_kernel_roofline("dispatch_token_smooth_kernel (EP)" if w.smooth is not None
+                                             else "dispatch_token_kernel (EP)", alg["dispatch"], t_epd, peak,
+                                             peak_kind) if t_epd else None,
+        "step_roofline": {"bound": "hbm", "kernel": ("whole step (update, route, plan, EP dispatch, EP combine)"
+                                                     if fused else
+                                                     "whole step (update, dispatch, plan, push, pull, combine)"),
+                          "achieved": round(ach, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                          "frac": round(ach / peak, 4), "traffic": None, "algorithmic_bytes": step_bytes,
+                          "note": "eager launches with two NCCL barriers and a count gather per step"},
         "e2e": None,
         "gpu_launches": n_kernels * K,
         "timing": "CUDA events around K eager steps (each with two barriers), max over ranks",
