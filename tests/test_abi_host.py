@@ -266,3 +266,90 @@ def test_binding_refuses_host_outputs(L):
         L._check_dispatch_out([1, 2], 8, H, K, E, 0)
     with pytest.raises(ValueError, match="CUDA"):
         L._check_combine_out(dict(y=torch.zeros((8, H), dtype=torch.bfloat16)), 8, H)
+
+
+# --------------------------------------------------------------------------
+# expert parallelism (fused), the routing-only dispatch, the TP domain
+# --------------------------------------------------------------------------
+
+def test_dispatch_route_rules(L):
+    f = ctypes.c_void_p(0x10000)
+    p = L.DispatchParams(64, 1024, 4, 8, 32, 0, 0, 1)
+    call = lambda p_=p, idx=f, ws=f, wsb=256: L.lib.moe_dispatch_route(ctypes.byref(p_), f, None, idx, f, f, f, ws,
+                                                                        wsb, None)
+    assert call(idx=None) == L.MOE_ERR_INVALID_ARG
+    assert call(p_=L.DispatchParams(0, 1024, 4, 8, 32, 0, 0, 1)) == L.MOE_ERR_INVALID_ARG
+    assert call(ws=None) == L.MOE_ERR_WORKSPACE
+
+
+def test_ep_dispatch_rules(L):
+    """The EP dispatch checks its parameters against the EP ones (same bs, K,
+    E; one source; row and scale bytes of the mode) before anything runs."""
+    f = ctypes.c_void_p(0x10000)
+    dp = lambda mode=2, bs=64, sources=1: L.DispatchParams(bs, 1024, 4, 8, 32, mode, 32 * 1024 if mode == 2 else 0,
+                                                           sources)
+    ep = lambda bs=64, row=1024, sc=4: L.EpParams(bs, 4, 32, 2, 0, row, sc, 512)
+    n = ctypes.c_size_t(0)
+    assert L.lib.moe_ep_workspace_size(ctypes.byref(ep()), ctypes.byref(n)) == L.MOE_OK
+    big = n.value
+
+    def call(d=None, e=None, peer=f, scales=f, gidx=f, wsb=None):
+        d = d or dp()
+        e = e or ep()
+        return L.lib.moe_ep_dispatch(ctypes.byref(d), ctypes.byref(e), f, f, None, f, f, f, peer, scales, None,
+                                     gidx, f, big if wsb is None else wsb, None)
+    assert call(d=dp(bs=32)) == L.MOE_ERR_INVALID_ARG          # bs differs from the EP parameters'
+    assert call(d=dp(sources=2)) == L.MOE_ERR_INVALID_ARG      # one source per GPU
+    assert call(e=ep(row=2048)) == L.MOE_ERR_INVALID_ARG       # int8 rows are H bytes
+    assert call(e=ep(sc=0)) == L.MOE_ERR_INVALID_ARG           # mode 2 sends a 4-byte scale
+    assert call(d=dp(mode=0), e=ep(row=2048, sc=0), scales=f) == L.MOE_ERR_INVALID_ARG  # no scale table in mode 0
+    assert call(peer=None) == L.MOE_ERR_INVALID_ARG
+    assert call(gidx=None) == L.MOE_ERR_INVALID_ARG
+    assert call(wsb=16) == L.MOE_ERR_WORKSPACE
+
+
+def test_ep_combine_rules(L):
+    f = ctypes.c_void_p(0x10000)
+    cp = lambda bs=64, sources=1: L.CombineParams(bs, 1024, 4, 512, 1e-6, sources)
+    ep = lambda row=2048: L.EpParams(64, 4, 32, 2, 0, row, 0, 512)
+    n = ctypes.c_size_t(0)
+    assert L.lib.moe_ep_workspace_size(ctypes.byref(ep()), ctypes.byref(n)) == L.MOE_OK
+
+    def call(c=None, e=None, peer=f, gidx=f, wsb=None):
+        c = c or cp()
+        e = e or ep()
+        return L.lib.moe_ep_combine_add_rmsnorm(ctypes.byref(c), ctypes.byref(e), peer, gidx, f, None, f, f, f,
+                                                None, None, f, n.value if wsb is None else wsb, None)
+    assert call(c=cp(bs=32)) == L.MOE_ERR_INVALID_ARG
+    assert call(c=cp(sources=2)) == L.MOE_ERR_INVALID_ARG
+    assert call(e=ep(row=1024)) == L.MOE_ERR_INVALID_ARG       # bf16 outputs are 2H bytes
+    assert call(peer=None) == L.MOE_ERR_INVALID_ARG
+    assert call(gidx=None) == L.MOE_ERR_INVALID_ARG
+    assert call(wsb=16) == L.MOE_ERR_WORKSPACE
+
+
+def test_tp_rules(L):
+    """The TP counts need one instance per EP rank and 2 * ws TP-major
+    sources; the TP combine needs both partial buffers, 16-byte aligned."""
+    f, f8 = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10008)
+    tp = lambda E=8, S=16: L.DispatchParams(16, 1024, 2, 8, E, 0, 0, S)
+    call = lambda p, out=f: L.lib.moe_dispatch_tp_counts(ctypes.byref(p), f, f, out, f, 256, None)
+    assert call(tp(S=8)) == L.MOE_ERR_INVALID_ARG        # sources != 2 * ws
+    assert call(tp(E=16)) == L.MOE_ERR_INVALID_ARG       # two instances per rank
+    assert call(tp(S=17)) == L.MOE_ERR_INVALID_ARG       # past 2 * ws
+    assert call(tp(), out=None) == L.MOE_ERR_INVALID_ARG
+    cp = L.CombineParams(8, 1024, 2, 16, 1e-6, 1)
+    comb = lambda x1: L.lib.moe_combine_add_rmsnorm_tp2(ctypes.byref(cp), f, x1, f, f, None, f, f, f, None, None,
+                                                        f, 256, None)
+    assert comb(None) == L.MOE_ERR_INVALID_ARG
+    assert comb(f8) == L.MOE_ERR_INVALID_ARG
+
+
+def test_sources_up_to_twice_the_ranks(L):
+    """With a TP domain of two ranks all 2 * ws devices are sources; more
+    are refused."""
+    n = ctypes.c_size_t(0)
+    ok = L.DispatchParams(64, 1024, 4, 8, 32, 0, 0, 16)
+    bad = L.DispatchParams(64, 1024, 4, 8, 32, 0, 0, 17)
+    assert L.lib.moe_dispatch_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == L.MOE_OK
+    assert L.lib.moe_dispatch_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == L.MOE_ERR_INVALID_ARG
