@@ -82,6 +82,20 @@ __global__ void __launch_bounds__(kUeThreads) update_expert_kernel(UpdateArgs a)
     __shared__ int s_warp[32];
     __shared__ int s_bad, s_total;
 
+    // Ask L2 for the table and this block's slice of ids and scales while
+    // the previous kernel drains: a prefetch returns nothing to the program
+    // and L2 is the point of coherence, so it is safe on data a predecessor
+    // may still write.  Only whole 16-byte words inside each array.
+    if (threadIdx.x < 3) {
+        const int items = a.bs * a.top_k, base = blockIdx.x * kUeThreads * kUeItems;
+        const int mine = min(kUeThreads * kUeItems, items - base);
+        const void *ptr = threadIdx.x == 0 ? (const void *)a.table
+                        : threadIdx.x == 1 ? (const void *)(a.expert_ids + base)
+                                           : (const void *)(a.expert_scales ? a.expert_scales + base : nullptr);
+        const uint32_t bytes = threadIdx.x == 0 ? (uint32_t)(a.num_logical * a.table_cols) * 4u : (uint32_t)mine * 4u;
+        if (ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15) == 0 && (bytes & ~15u) != 0)
+            prefetch_l2(ptr, bytes & ~15u);
+    }
     pdl_wait();               // the ids may come from the previous kernel
     pdl_launch_dependents();  // the next kernel waits for this one before it reads anything
 
