@@ -541,7 +541,7 @@ __global__ void __launch_bounds__(kRtThreads) route_place_kernel(DispatchArgs a,
                 a.src_of_row[row] = j;
             }
         }
-        __syncthreads();  // every thread has read this round's counters
+        __syncthreads();  // every thread has read this pass's counters
     }
 }
 
