@@ -23,9 +23,9 @@
 //    every weight byte is read from HBM once per slot.
 //  * Operands are staged by TMA (cp.async.bulk.tensor, 128-byte swizzle, each
 //    CTA loading its own tiles) through a ring of stages sized at run time
-//    from N, tracked by mbarriers; one elected thread issues both the copies
-//    and the MMAs, and
-//    tcgen05.commit frees each stage.  The int32 accumulator lives in TMEM
+//    from N, tracked by mbarriers; one lane of one warp issues the copies,
+//    one lane of another the MMAs, and tcgen05.commit frees each stage for
+//    the next copy.  The int32 accumulator lives in TMEM
 //    (128 lanes = channels, N columns = rows; 256 columns allocated, two
 //    CTAs per SM).
 //  * The epilogue reads TMEM with tcgen05.ld (warp w owns lanes 32w..32w+31),
@@ -56,7 +56,7 @@ constexpr int kGmABytes = kGmBM * kGmBK;             // 16 KB of weight per stag
 constexpr int kGmPipeBytes = 110 * 1024;             // the stage ring (two CTAs per SM)
 constexpr int kGmMaxStages = 8;
 constexpr int kGmSmemBytes = kGmPipeBytes + 1024;    // + slack to align the ring to 1 KB
-constexpr int kGmThreads = 128;
+constexpr int kGmThreads = 192;  // warps 0-3 epilogue, warp 4 copies, warp 5 MMAs
 constexpr uint32_t kGmTmemCols = 256;                // int32 accumulator columns (>= N)
 // mxfp8: the fp32 accumulator (128 columns) then, per ring stage s, the
 // stage's block factors: 4 columns for the weight rows (A) at 128 + 8 s and
@@ -219,11 +219,16 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t phase) {
     }
 }
 
-// --- the int8 matmul: grid (ceil(N / 128), max_slots), 128 threads ---
+// --- the int8 matmul, warp-specialized: grid (ceil(N / 128), max_slots), 192 threads ---
 //
 // int8 rows and weights (kind::i8, int32 accumulator), output
-// (acc * dyn[row]) * wscale[channel].  One elected thread issues both the
-// copies and the MMAs; the other threads wait for the accumulator.
+// (acc * dyn[row]) * wscale[channel].  Warp 4 (one lane) issues the TMA
+// copies, refilling each stage as soon as the MMAs that read it completed;
+// warp 5 (one lane) issues the MMAs and owns the TMEM allocation; warps 0-3
+// wait for the accumulator and run the epilogue.  Per ring stage s, full[s]
+// (the copies landed) and empty[s] (tcgen05.commit: its MMAs completed) hand
+// the stage between the two roles, so neither waits for the other except
+// through the stage it needs.
 __global__ void __launch_bounds__(kGmThreads, 1)
     gmm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GmmArgs a) {
     constexpr uint32_t kCols = kGmTmemCols;
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const int4 slot = s_slot;
     if (slot.x < 0) return;  // more slots were launched than the offsets need
 
-    if (warp == 0) {
+    if (warp == 5) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
                      "r"(kCols)
                      : "memory");
@@ -272,66 +277,51 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const int nr = slot.z;
     const int mma_n = (nr + 15) & ~15;
     const int nbox = mma_n / kGmBoxRows;
-    const int b_bytes = mma_n * kGmBK;
-    const int stage_bytes = kGmABytes + b_bytes;  // a multiple of 2 KB
+    const int stage_bytes = kGmABytes + mma_n * kGmBK;  // a multiple of 2 KB
     const int nst = min(kGmMaxStages, kGmPipeBytes / stage_bytes);
     const int nk = (a.hidden + kGmBK - 1) / kGmBK;
-    const uint32_t tx = (uint32_t)stage_bytes;  // out-of-range box parts are zero-filled and still counted
-    const int wrow = slot.x * a.out_dim + n0;
-    const uint32_t ring_s = smem_u32(ring);
 
-    auto issue = [&](int kb) {  // thread 0: the copies of k-step kb into its stage
-        const int s = kb % nst;
-        uint8_t *sa = ring + s * stage_bytes;
-        mbar_arrive_expect_tx(&s_full[s], tx);
-        tma_load_2d(sa, &tm_w, kb * kGmBK, wrow, &s_full[s]);
-        for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sa + kGmABytes + b * kGmBoxRows * kGmBK, &tm_x, kb * kGmBK, slot.y + b * kGmBoxRows,
-                        &s_full[s]);
-    };
-    int issued = 0;
-    int pending = -1;  // thread 0, after a timeout: the first step whose copies were not consumed
-    // thread 0: wait for step kb's operands, issue its MMAs, refill the stage
-    // the previous step used.  Returns false on a timeout, with `pending` set.
-    auto mma_step = [&](int kb) -> bool {
-        const int s = kb % nst;
-        if (!mbar_wait_bounded(&s_full[s], (uint32_t)(kb / nst) & 1u)) {
-            pending = kb;
-            return false;
-        }
-        tc_fence_after();
-        const uint32_t sa = ring_s + s * stage_bytes;
-        const uint64_t da = gm_smem_desc(sa), db = gm_smem_desc(sa + kGmABytes);
-#pragma unroll
-        for (int kk = 0; kk < kGmBK / 32; ++kk)  // K = 32 per MMA: +32 bytes = +2 in 16-byte units
-            umma_i8(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc(mma_n), (kb | kk) != 0);
-        umma_commit(&s_empty[s]);
-        if (kb >= 1 && issued < nk) {
-            const int sp = (kb - 1) % nst;
-            if (!mbar_wait_bounded(&s_empty[sp], (uint32_t)((kb - 1) / nst) & 1u)) {
-                pending = kb + 1;  // step kb was consumed
-                return false;
+    if (warp == 4) {
+        if (lane == 0) {  // the TMA producer
+            const uint32_t tx = (uint32_t)stage_bytes;  // out-of-range box parts are zero-filled and still counted
+            const int wrow = slot.x * a.out_dim + n0;
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % nst;
+                if (kb >= nst && !mbar_wait_bounded(&s_empty[s], (uint32_t)(kb / nst - 1) & 1u)) {
+                    s_fail = 1;
+                    break;
+                }
+                uint8_t *sa = ring + s * stage_bytes;
+                mbar_arrive_expect_tx(&s_full[s], tx);
+                tma_load_2d(sa, &tm_w, kb * kGmBK, wrow, &s_full[s]);
+                for (int b = 0; b < nbox; ++b)
+                    tma_load_2d(sa + kGmABytes + b * kGmBoxRows * kGmBK, &tm_x, kb * kGmBK, slot.y + b * kGmBoxRows,
+                                &s_full[s]);
+                ++issued;
             }
-            issue(issued);
-            ++issued;
+            // every copy issued has landed before the CTA can end (at once, unless a wait gave up)
+            for (int j = max(0, issued - nst); j < issued; ++j)
+                if (!mbar_wait_bounded(&s_full[j % nst], (uint32_t)(j / nst) & 1u)) s_fail = 1;
         }
-        return true;
-    };
-
-    if (t == 0)
-        for (; issued < nst && issued < nk; ++issued) issue(issued);
-    if (t == 0)
-        for (int kb = 0; kb < nk; ++kb)
-            if (!mma_step(kb)) break;
-    __syncwarp();
-    if (t == 0) {
-        if (pending >= 0) {
-            // drain the copies still in flight before the CTA can exit
-            for (int j = pending; j < issued; ++j) mbar_wait_bounded(&s_full[j % nst], (uint32_t)(j / nst) & 1u);
-            s_fail = 1;
-            raise_error(a.err, kDevTimeout);
+    } else if (warp == 5) {
+        if (lane == 0) {  // the MMA issuer
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % nst;
+                if (!mbar_wait_bounded(&s_full[s], (uint32_t)(kb / nst) & 1u)) {
+                    s_fail = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(ring + s * stage_bytes);
+                const uint64_t da = gm_smem_desc(sa), db = gm_smem_desc(sa + kGmABytes);
+#pragma unroll
+                for (int kk = 0; kk < kGmBK / 32; ++kk)  // K = 32 per MMA: +32 bytes = +2 in 16-byte units
+                    umma_i8(tmem, da + 2 * kk, db + 2 * kk, gm_instr_desc(mma_n), (kb | kk) != 0);
+                umma_commit(&s_empty[s]);
+            }
+            umma_commit(&s_done);  // fires once every MMA above has completed
         }
-        umma_commit(&s_done);  // fires once every MMA above has completed
     }
     __syncwarp();
     const bool done = mbar_wait_sleep(&s_done, 0);
@@ -339,7 +329,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const bool all_done = __syncthreads_and(done);  // also publishes s_fail
     tc_fence_after();
     pdl_launch_dependents();
-    if (s_fail == 0 && all_done) {
+    if (s_fail != 0 && t == 0) raise_error(a.err, kDevTimeout);
+    if (s_fail == 0 && all_done && warp < 4) {
         const int ch = n0 + warp * 32 + lane;  // this thread's TMEM lane = output channel
         const bool ch_ok = ch < a.out_dim;
         const float wsc = ch_ok ? a.wscale[(size_t)slot.x * a.out_dim + ch] : 0.0f;
@@ -360,7 +351,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0)
+    if (warp == 5)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
 }
 
