@@ -457,20 +457,23 @@ MOE_API moe_status moe_dispatch_noalloc(const moe_dispatch_params *p, const void
  * the stretch of that order its instances own, so its row r is global row
  * base[q] + r.
  *
- * A layer on GPU g:
- *   1. moe_update_expert and moe_dispatch on its own tokens over all E
- *      instances (local rows, counts [E], offsets [E+1]);
+ * A layer on GPU g, fused form:
+ *   1. moe_update_expert and moe_dispatch_route on its own tokens over all E
+ *      instances (local rows, counts [E], offsets [E+1]; no row moved);
  *   2. the counts of every GPU gathered into counts_all [G][E] on every GPU
  *      (a collective of E ints per GPU, by the caller);
- *   3. moe_ep_plan, then moe_ep_push: every local row (and its scales) is
- *      stored into its owner's receive buffer through the owner's pointer;
- *   4. a group barrier (every push done), then the expert step on the
+ *   3. moe_ep_plan, then moe_ep_dispatch: each token is quantized once and
+ *      each copy (and its scales) stored straight into its owner's receive
+ *      buffer through the owner's pointer;
+ *   4. a group barrier (every row stored), then the expert step on the
  *      receive buffer (moe_ep_plan's recv_counts / recv_offsets describe it);
- *   5. a group barrier (every expert output written), then moe_ep_pull: each
- *      local row reads its output back from the owner, in the local row order
- *      moe_dispatch made, so moe_combine_add_rmsnorm runs with the local
- *      expand_idx unchanged;
+ *   5. a group barrier (every expert output written), then
+ *      moe_ep_combine_add_rmsnorm: each copy's output read from its owner;
  *   6. a group barrier before the buffers are reused.
+ * Two-step form: moe_dispatch into a local buffer in step 1, moe_ep_push in
+ * step 3 (every local row stored into its owner's buffer), and in step 5
+ * moe_ep_pull (each local row's output brought back in the local row order)
+ * followed by moe_combine_add_rmsnorm with the local expand_idx.
  * The pointer tables hold, per GPU q, a pointer this GPU can dereference:
  * its own buffer for q = g, a peer mapping (moe_ipc_import, or any mapping
  * the caller set up) otherwise.  The copies are plain 16-byte loads and
