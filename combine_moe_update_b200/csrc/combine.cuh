@@ -63,9 +63,9 @@ __host__ __device__ inline int cb_threads(int NV, int vecs) {
 }
 
 // One token per block (SPLIT = 1, VECS = 4: 224 threads at H = 7168, four
-// blocks per SM, a 512-token batch in one wave), or per cluster of two
-// blocks (SPLIT = 2, VECS = 2) when that takes fewer waves: block h of the
-// cluster holds vectors [h * V / 2, (h + 1) * V / 2) of the row and the two
+// blocks per SM, a 512-token batch in one wave), or per cluster of SPLIT = 2
+// or 4 blocks (VECS = 2) for smaller batches: block h of the cluster holds
+// vectors [h * V / SPLIT, (h + 1) * V / SPLIT) of the row and the blocks'
 // sums of x^2 meet through distributed shared memory.  Every thread issues
 // the loads of one vector together -- all K rows (a pruned copy issues
 // none), the shared row and the residual row -- so a vector costs one round
@@ -228,12 +228,13 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
         return;
     }
     float tot = block_sum<NW>(ss, s_red);
-    if constexpr (SPLIT == 2) {  // the row's two halves: the same sum, in the same order, in both blocks
+    if constexpr (SPLIT > 1) {  // the row's parts: the same sum, in the same order, in every block
         if (t == 0) s_part = tot;
         cluster_sync();
-        const float p_0 = ld_cluster_f32(&s_part, 0), p_1 = ld_cluster_f32(&s_part, 1);
-        tot = p_0 + p_1;
-        cluster_sync();  // the peer has read this block's partial before either block leaves
+        tot = ld_cluster_f32(&s_part, 0);
+#pragma unroll
+        for (int q = 1; q < SPLIT; ++q) tot += ld_cluster_f32(&s_part, (uint32_t)q);
+        cluster_sync();  // the peers have read this block's partial before any block leaves
     }
     pdl_launch_dependents();
     const float rstd = __frcp_rn(__fsqrt_rn(__fdiv_rn(tot, (float)H) + a.norm_eps));

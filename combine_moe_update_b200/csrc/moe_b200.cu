@@ -293,16 +293,21 @@ cudaError_t launch_combine_tok(const moe::CombineArgs &a, cudaStream_t s) {
     }
 }
 
-// Two half-row blocks per token when the batch has fewer than two tokens per
-// SM: measured at Bs 256, H 7168 (10.9 against 11.6 us), while every batch of
-// 512 tokens ran fastest with one block per token (the gate shape 16.6
-// against 18.8 us, H 4096 10.2 against 12.9 us, H 8192 23.5 against 24.1 us).
+// Quarter-row blocks per token when the batch has fewer tokens than SMs,
+// half-row blocks when it has fewer than two per SM: measured at Bs 128,
+// H 2048 (the 32-layer stack: 10.97 against 10.24 us per layer with
+// quarters) and at Bs 256, H 7168 (halves 10.9 against 11.6 us unsplit and
+// 13.3 us in quarters), while every batch of 512 tokens ran fastest with
+// one block per token (the gate shape 16.6 against 18.8 us, H 4096 10.2
+// against 12.9 us, H 8192 23.5 against 24.1 us).
 template <int KMAX, bool NORM>
 cudaError_t launch_combine_split(const moe::CombineArgs &a, cudaStream_t s) {
-    const bool split = a.bs < 2 * device_sms();
-    if (a.shared_x)
-        return split ? launch_combine_tok<KMAX, true, NORM, 2>(a, s) : launch_combine_tok<KMAX, true, NORM, 1>(a, s);
-    return split ? launch_combine_tok<KMAX, false, NORM, 2>(a, s) : launch_combine_tok<KMAX, false, NORM, 1>(a, s);
+    const int sms = device_sms();
+    const int split = a.bs < sms && (a.hidden >> 3) % 4 == 0 ? 4 : a.bs < 2 * sms ? 2 : 1;
+    const bool sh = a.shared_x != nullptr;
+    if (split == 4) return sh ? launch_combine_tok<KMAX, true, NORM, 4>(a, s) : launch_combine_tok<KMAX, false, NORM, 4>(a, s);
+    if (split == 2) return sh ? launch_combine_tok<KMAX, true, NORM, 2>(a, s) : launch_combine_tok<KMAX, false, NORM, 2>(a, s);
+    return sh ? launch_combine_tok<KMAX, true, NORM, 1>(a, s) : launch_combine_tok<KMAX, false, NORM, 1>(a, s);
 }
 
 // The combine of a TP pair: each row is the bf16 sum of the two partial outputs (one block per token).
