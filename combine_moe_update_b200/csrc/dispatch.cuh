@@ -315,7 +315,7 @@ __device__ __forceinline__ void block_route_clear(RS &rs, int E) {
 // key0: for the threads of warp 0, copy_key of this token's copy k = lane
 // (-1 for lanes >= K).  Leaves rs.key and rs.row filled, after a barrier.
 template <int NT, class RS>
-__device__ void block_route(const DispatchArgs &a, int i, RS &rs, int key0) {
+__device__ void block_route(const DispatchArgs &a, int i, RS &rs, int key0, bool writer = true) {
     const int t = threadIdx.x, E = a.num_instances, K = a.top_k, N = a.bs * K, mine0 = i * K;
     constexpr int U = 8;
     for (int j0 = 0; j0 < N; j0 += NT * U) {  // loads unconditional (clamped), so all are in flight together
@@ -353,14 +353,14 @@ __device__ void block_route(const DispatchArgs &a, int i, RS &rs, int key0) {
         const int e = t * P + u;
         if (e < E) {
             rs.off[e] = run;
-            if (i == 0) {
+            if (i == 0 && writer) {
                 a.counts[e] = rs.cnt[e];
                 a.offsets[e] = run;
             }
             run += rs.cnt[e];
         }
     }
-    if (i == 0 && t == NT - 1) a.offsets[E] = incl;  // the total
+    if (i == 0 && writer && t == NT - 1) a.offsets[E] = incl;  // the total
     __syncthreads();
     if (t < 32) {
         const unsigned peers = __match_any_sync(kFull, key0);
@@ -369,7 +369,7 @@ __device__ void block_route(const DispatchArgs &a, int i, RS &rs, int key0) {
         if (key0 == -2) raise_error(a.err, kDevBadId);
         rs.key[t] = key0;
         rs.row[t] = row;
-        if (t < K) {
+        if (t < K && writer) {
             a.expand_idx[mine0 + t] = row;
             if (row >= 0) a.src_of_row[row] = mine0 + t;
         }
@@ -917,6 +917,11 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
 // thread at 224 threads) for four blocks per SM, so a 512-token batch runs
 // in a single wave with the other blocks covering each one's waits.
 //
+// Small batches (too few tokens to fill the SMs) split each token's sent
+// copies over P = gridDim.y blocks: block (i, p) quantizes copies p, p + P,
+// ... of token i, so more copies run at once; every such block loads the
+// token's row itself.
+//
 // Per copy: wait for the smooth row; xFp32 = x * smooth; mode 2 publishes
 // each warp's partial max and takes one barrier (which also frees the
 // shared row for the next copy's load), then every thread finishes the max,
@@ -930,9 +935,10 @@ __host__ __device__ inline int smooth_smem_floats(int hidden) {
     return hidden > NT * kDpVecs * 8 ? hidden : NT * kDpVecs * 8;
 }
 
-template <int MODE, int NT, bool FUSED, bool EP = false>
+template <int MODE, int NT, bool FUSED, bool EP = false, bool GROUPS = false>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_kernel(DispatchArgs a) {
     static_assert(!(FUSED && EP), "an EP scatter follows an earlier route call");
+    static_assert(!(GROUPS && EP), "an EP scatter takes one block per token");
     constexpr int NW = NT / 32;
     extern __shared__ __align__(128) float s_smooth[];  // the current copy's smooth row, then zeros
     __shared__ float s_red[2][NW];
@@ -940,6 +946,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
     __shared__ int s_key[16], s_pos[16], s_row[16], s_ns;
     __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
     const int i = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int P = GROUPS ? (int)gridDim.y : 1, p = GROUPS ? (int)blockIdx.y : 0;  // copy group p of the token's P
     const int H = a.hidden, V = H >> 3, K = a.top_k;
     const uint32_t row_bytes = (uint32_t)H * sizeof(float);  // a multiple of 16 (H % 16 == 0)
 
@@ -989,11 +996,13 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         mbar_arrive_expect_tx(&s_bar, row_bytes);
         bulk_copy_g2s(s_smooth, a.smooth + (size_t)s_key[c] * H, row_bytes, &s_bar);
     };
-    if (t == 0 && ns > 0) fetch_smooth(0);
-    if constexpr (FUSED) block_route<NT>(a, i, rs, key0);  // while the first smooth row is in flight
+    if (t == 0 && p < ns) fetch_smooth(p);
+    if constexpr (FUSED) block_route<NT>(a, i, rs, key0, p == 0);  // while the first smooth row is in flight
 
-    for (int c = 0; c < ns; ++c) {
-        const bool landed = mbar_wait_bounded(&s_bar, c & 1);
+    int jj = 0;  // copies this block has taken (the mbarrier's phase and the partials' buffer)
+    for (int c = p; c < ns; c += P, ++jj) {
+        const int j = GROUPS ? jj : c;
+        const bool landed = mbar_wait_bounded(&s_bar, j & 1);
         uint64_t xf[kDpVecs][4];
 #pragma unroll
         for (int q = 0; q < kDpVecs; ++q) {  // xFp32 = x * smooth (0 past the row's end)
@@ -1012,7 +1021,7 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         float row_scale = 0.0f;
         if constexpr (MODE == 2) {
             const float m = warp_max(abs_max_vecs(xf));
-            if (lane == 0) s_red[c & 1][w] = m;
+            if (lane == 0) s_red[j & 1][w] = m;
         }
         // every thread has read the smooth row (and published its partial):
         // the buffer may be refilled.  A row that never landed stops the
@@ -1021,23 +1030,23 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         if (__syncthreads_or(!landed)) {
             if (t == 0) {
                 raise_error(a.err, kDevTimeout);
-                mbar_wait_bounded(&s_bar, c & 1);
+                mbar_wait_bounded(&s_bar, j & 1);
             }
             return;
         }
-        if (t == 0 && c + 1 < ns && !(kSkipOneCopy && blockIdx.x == 0 && c == 0)) {
+        if (t == 0 && c + P < ns && !(kSkipOneCopy && blockIdx.x == 0 && c == 0)) {
             fence_proxy_async_smem();
-            fetch_smooth(c + 1);
+            fetch_smooth(c + P);
         }
-        if (c + 1 == ns) pdl_launch_dependents();  // the next kernel may be scheduled as blocks finish
+        if (c + P >= ns) pdl_launch_dependents();  // the next kernel may be scheduled as blocks finish
         if constexpr (MODE == 2) {
-            const float dyn = __fdiv_rn(127.0f, max_partials<NW>(s_red[c & 1]));  // +inf when the max is 0
+            const float dyn = __fdiv_rn(127.0f, max_partials<NW>(s_red[j & 1]));  // +inf when the max is 0
             row_scale = __frcp_rn(dyn);                                           // or 127 / max overflows
             int8_vecs(xf, dyn, qv);
         } else {
             quantize_local<MODE, NT>(xf, V, qv, seg);
         }
-        if (!FUSED && c == 0) {
+        if (!FUSED && j == 0) {
             pdl_wait();  // the rows come from the route kernel
             if (t < K) {
                 const int r = a.expand_idx[i * K + t];
@@ -1053,6 +1062,10 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         if (copy_dst<EP>(a, s_key[c], FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], d))
             write_row<MODE, NT>(a, d, V, qv, seg, row_scale);
     }
+    // A block with no copy still waits for the route kernel, so that this
+    // grid ends after it: the next call reads the rows and counts it wrote.
+    if constexpr (!FUSED && !EP)
+        if (ns <= p) pdl_wait();
 }
 
 }  // namespace moe
