@@ -289,13 +289,16 @@ struct TokenSmoothLaunch {
     }
     // Copy groups per token: double them (up to 4, and while a group keeps
     // one copy or more) as long as the batch's blocks still fit on the SMs
-    // at once.  Measured at Bs 256, H 7168, K 8 (two groups): the dispatch
-    // call 13.2 -> 12.0 us.
+    // at once; with static scales (mode 1: no per-copy maximum) up to a
+    // second wave.  Measured at H 7168, K 8: mode 2 at Bs 256 two groups
+    // 13.2 -> 12.0 us per dispatch call, four 13.4 us; mode 2 at Bs 512 two
+    // groups 18.1 -> 19.8 us; mode 1 at Bs 512 two groups 20.4 -> 19.4 us.
     template <typename Kernel>
     static int copy_groups(const moe::DispatchArgs &a, Kernel kernel, size_t smem) {
         const long slots = (long)device_sms() * resident_blocks_fn(reinterpret_cast<const void *>(kernel), NT, smem);
+        const long fill = MODE == 1 ? 1 : 2;
         int P = 1;
-        while (P < 4 && 2 * P <= a.top_k && (long)a.bs * 2 * P <= slots) P *= 2;
+        while (P < 4 && 2 * P <= a.top_k && (long)a.bs * fill * P <= slots) P *= 2;
         return P;
     }
     static cudaError_t go(const moe::DispatchArgs &a, cudaStream_t s) {
