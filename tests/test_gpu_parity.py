@@ -72,6 +72,24 @@ def test_parity_active_mask(B):
     assert_parity(w, run_gpu(w, B), run_oracle(w))
 
 
+@pytest.mark.parametrize("bs,K,H,mode,E", [(160, 8, 7168, 2, 256), (72, 16, 2048, 3, 64), (40, 8, 4096, 2, 32),
+                                           (300, 4, 7168, 2, 64)])
+def test_parity_copy_groups(B, bs, K, H, mode, E):
+    """Batches small enough that the smooth-scale scatter splits each token's
+    sent copies over two or four blocks (copy groups), past the self-routing
+    limit (routed by the route kernel: 1280 and 1152 copies) and below it;
+    inactive tokens and a pruning threshold leave tokens with fewer sent
+    copies than groups, or none, so some blocks have nothing to write.  The
+    last case (Bs 300) is one group per token."""
+    w = gen.uniform_layer(f"groups_{bs}_{K}", seed=bs * 100 + K, bs=bs, hidden=H, num_experts=E, top_k=K,
+                          ep_world_size=8, quant_mode=mode, smooth=True, shared=True, prune_threshold=0.1)
+    w.active_mask = (np.random.default_rng(bs).random(bs) < 0.7).astype(np.uint8)
+    g, o = run_gpu(w, B), run_oracle(w)
+    sent = (o["dispatch"]["expand_idx"] >= 0).sum(axis=1)
+    assert (sent == 0).any() and (sent == 1).any() and (sent >= 3).any()
+    assert_parity(w, g, o)
+
+
 @pytest.mark.parametrize("seed", range(4))
 def test_parity_random_replicated_tables(B, seed):
     rng = np.random.default_rng(seed)
