@@ -425,9 +425,21 @@ def combine_add_rmsnorm_tp2(expand_x0, expand_x1, expand_idx, expert_scales, res
                             stream=None, sources=1):
     """moe_combine_add_rmsnorm_tp2: the combine whose rows are the bf16 sums
     of the TP pair's two partial outputs.  Returns a dict like
-    combine_add_rmsnorm."""
+    combine_add_rmsnorm.  Either partial may be given as an int: the device
+    address, as this device dereferences it, of a [rows, H] bf16 buffer with
+    the other's shape (another GPU's buffer mapped by ipc_import); a tensor
+    partial sets the shape and the device."""
+    peer0, peer1 = isinstance(expand_x0, int), isinstance(expand_x1, int)
+    if peer0 and peer1:
+        raise TypeError("at least one partial must be a tensor (it gives the shape and the device)")
+    if peer0:  # the same call with the partials' roles swapped: the sum is symmetric
+        expand_x0, expand_x1, peer1 = expand_x1, expand_x0, True
     _req(expand_x0, "expand_x0", torch.bfloat16)
-    _req(expand_x1, "expand_x1", torch.bfloat16, tuple(expand_x0.shape))
+    if peer1:
+        if expand_x1 <= 0 or expand_x1 % 16:
+            raise ValueError("a peer partial's address must be non-null and 16-byte aligned")
+    else:
+        _req(expand_x1, "expand_x1", torch.bfloat16, tuple(expand_x0.shape))
     rows, H = expand_x0.shape
     dev = expand_x0.device
     _req(expand_idx, "expand_idx", torch.int32)
@@ -444,11 +456,12 @@ def combine_add_rmsnorm_tp2(expand_x0, expand_x1, expand_idx, expert_scales, res
     p = CombineParams(_per_source(bs, sources, "combine_add_rmsnorm_tp2"), H, k, rows, float(norm_eps), int(sources))
     with torch.cuda.device(dev):
         ws = _req(workspace, "workspace", torch.uint8) if workspace is not None else new_workspace(dev, stream)
-        _same_device(dev, ("expand_x1", expand_x1), ("expand_idx", expand_idx), ("expert_scales", expert_scales),
-                     ("residual_x", residual_x), ("gamma", gamma), ("shared_x", shared_x), ("workspace", ws),
-                     *((f"out['{n}']", t) for n, t in out.items()))
+        _same_device(dev, ("expand_x1", None if peer1 else expand_x1), ("expand_idx", expand_idx),
+                     ("expert_scales", expert_scales), ("residual_x", residual_x), ("gamma", gamma),
+                     ("shared_x", shared_x), ("workspace", ws), *((f"out['{n}']", t) for n, t in out.items()))
+        x1 = ctypes.c_void_p(expand_x1) if peer1 else _ptr(expand_x1)
         _check("moe_combine_add_rmsnorm_tp2", lib.moe_combine_add_rmsnorm_tp2(
-            ctypes.byref(p), _ptr(expand_x0), _ptr(expand_x1), _ptr(expand_idx), _ptr(expert_scales),
+            ctypes.byref(p), _ptr(expand_x0), x1, _ptr(expand_idx), _ptr(expert_scales),
             _ptr(shared_x), _ptr(residual_x), _ptr(gamma), _ptr(out["y"]), _ptr(out.get("x_out")),
             _ptr(out.get("rstd")), _ptr(ws), ws.numel(), _stream(stream)))
     return out

@@ -141,3 +141,69 @@ def test_tp_counts_refuses_other_layouts(B):
             torch.empty((ws, 2), dtype=torch.int32, device="cuda").data_ptr(),
             B.new_workspace().data_ptr(), B.WORKSPACE_BYTES, None)
         B._check("moe_dispatch_tp_counts", rc)
+
+
+@pytest.mark.parametrize("ws,bs,K,H,mode,smooth,prune,by_address", [
+    (4, 8, 4, 1024, 0, False, 0.0, False),   # 256 copies: the self-routing scatter
+    (8, 32, 6, 2048, 2, True, 0.05, True),   # 3072 copies: the route kernel; the peer's partial by address
+    (8, 24, 8, 1040, 3, False, 0.1, True),   # ragged tile, pruning
+])
+def test_tp_pair_across_two_gpus_emulated(B, ws, bs, K, H, mode, smooth, prune, by_address):
+    """The TP pair split over two GPUs (combine_moe_update_b200.tp), both
+    emulated on this device: GPU t holds TP domain t's tokens; after the
+    gather each GPU's dispatch of the pair's tokens must equal the oracle's
+    AllToAllV per domain + AllGatherV bit for bit (so both GPUs hold the same
+    rows), and each GPU's combine of its own tokens, reading the peer's
+    partial outputs, must equal the one-GPU TP combine of those tokens bit
+    for bit and the oracle's ReduceScatterV + combine element-wise."""
+    from combine_moe_update_b200 import tp as TP
+    S, E = 2 * ws, ws
+    T, Th = S * bs, ws * bs
+    rng = np.random.Generator(np.random.PCG64([127, ws, bs, mode]))
+    x = gen.bf16_bits(rng.standard_normal((T, H), np.float32))
+    ids = gen.topk_uniform(rng, T, E, K)
+    sc = gen.softmax_scales(rng, T, K)
+    table = gen.identity_table(E, ws)
+    sm = rng.uniform(0.5, 2.0, size=(E, H)).astype(np.float32) if smooth else None
+    res = gen.bf16_bits(rng.standard_normal((T, H), np.float32))
+    sh = gen.bf16_bits(rng.standard_normal((T, H), np.float32))
+    g = gen.bf16_bits(rng.uniform(0.5, 1.5, size=H).astype(np.float32))
+    p0 = gen.bf16_bits(rng.standard_normal((T * K, H), np.float32))
+    p1 = gen.bf16_bits(rng.standard_normal((T * K, H), np.float32))
+
+    pair = TP.EmulatedTPPair(ws=ws, bs=bs, hidden=H, top_k=K, quant_mode=mode,
+                             scales_len=0 if sm is None else sm.size)
+    half = lambda a, t: a[t * Th:(t + 1) * Th]
+    local = [dict(x=dev_bf16(half(x, t)), expert_ids=dev(half(ids, t)), expert_scales=dev(half(sc, t)))
+             for t in (0, 1)]
+    for r in pair.ranks:
+        for v in r.d.values():
+            if v is not None:
+                poison_(v)
+    full = pair.dispatch(local, dev(table), smooth=None if sm is None else dev(sm), prune_threshold=prune)
+    pair.ranks[0].partial.copy_(dev_bf16(p0))
+    pair.ranks[1].partial.copy_(dev_bf16(p1))
+    inputs = [dict(residual=dev_bf16(half(res, t)), gamma=dev_bf16(g), shared_x=dev_bf16(half(sh, t)))
+              for t in (0, 1)]
+    outs = pair.combine(full, inputs, 1e-6, peer_by_address=by_address)
+    one = B.combine_add_rmsnorm_tp2(dev_bf16(p0), dev_bf16(p1), pair.ranks[0].d["expand_idx"], dev(sc),
+                                    dev_bf16(res), dev_bf16(g), 1e-6, shared_x=dev_bf16(sh), sources=S)
+    torch.cuda.synchronize()
+    assert all(r.device_errors() == 0 for r in pair.ranks)
+
+    bal_o, bm_o, e1 = orc.update_expert(ids, table, ws, expert_scales=sc, prune_threshold=prune)
+    assert e1 == 0
+    od = orc.dispatch_tp(x, bal_o, E, mode, ws, bs, mask=bm_o, smooth=sm)
+    n = od["n"]
+    for r in pair.ranks:
+        np.testing.assert_array_equal(host(r.d["expand_idx"]), od["expand_idx"])
+        np.testing.assert_array_equal(host(r.d["offsets"]), od["offsets"])
+        np.testing.assert_array_equal(_bytes(host(r.d["expand_x"]), 0, n), _bytes(od["expand_x"], 0, n))
+        if od["dyn_scales"] is not None:
+            np.testing.assert_array_equal(_bytes(host(r.d["dyn_scales"]), 0, n), _bytes(od["dyn_scales"], 0, n))
+        np.testing.assert_array_equal(host(r.tp_counts), od["tp_counts"])
+    oc = orc.combine_add_rmsnorm_tp(p0, p1, od["expand_idx"], sc, res, g, 1e-6, shared_x=sh)
+    for t, o in enumerate(outs):
+        np.testing.assert_array_equal(host(o["y"]), half(host(one["y"]), t))
+        assert_close_bf16(host(o["y"]), half(oc["y_f64"], t), what=f"y of GPU {t}")
+        assert_close_bf16(host(o["x_out"]), half(oc["x_f64"], t), what=f"x_out of GPU {t}")
