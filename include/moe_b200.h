@@ -305,7 +305,11 @@ MOE_API moe_status moe_combine_add_rmsnorm(const moe_combine_params *p, const vo
  * TP-major), so the scatter half and the AllToAllV back are the gather
  * through expand_idx.
  *   expand_x0, expand_x1 [expand_rows, H] bf16 device, 16-byte aligned: the
- *                        two TP ranks' partial outputs
+ *                        two TP ranks' partial outputs; either may be the
+ *                        other GPU's buffer as mapped on this one
+ *                        (moe_ipc_import), read with plain loads over
+ *                        NVLink, so a TP pair on two GPUs combines each
+ *                        GPU's own tokens with this call
  * Other arguments and errors as moe_combine_add_rmsnorm.
  */
 MOE_API moe_status moe_combine_add_rmsnorm_tp2(const moe_combine_params *p, const void *expand_x0,
