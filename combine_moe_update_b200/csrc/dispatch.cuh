@@ -938,7 +938,6 @@ __host__ __device__ inline int smooth_smem_floats(int hidden) {
 template <int MODE, int NT, bool FUSED, bool EP = false, bool GROUPS = false>
 __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_kernel(DispatchArgs a) {
     static_assert(!(FUSED && EP), "an EP scatter follows an earlier route call");
-    static_assert(!(GROUPS && EP), "an EP scatter takes one block per token");
     constexpr int NW = NT / 32;
     extern __shared__ __align__(128) float s_smooth[];  // the current copy's smooth row, then zeros
     __shared__ float s_red[2][NW];
@@ -1051,7 +1050,8 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
             if (t < K) {
                 const int r = a.expand_idx[i * K + t];
                 s_row[t] = r;
-                if constexpr (EP) ep_record(a, i * K + t, a.ids[i * K + t], r);
+                if constexpr (EP)
+                    if (p == 0) ep_record(a, i * K + t, a.ids[i * K + t], r);  // once per token
             }
             __syncthreads();
         }
@@ -1064,8 +1064,15 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
     }
     // A block with no copy still waits for the route kernel, so that this
     // grid ends after it: the next call reads the rows and counts it wrote.
-    if constexpr (!FUSED && !EP)
-        if (ns <= p) pdl_wait();
+    // With EP the token's first block records its copies' global rows (all
+    // -1 then: no copy of the token was sent) for the combine.
+    if constexpr (!FUSED) {
+        if (ns <= p) {
+            pdl_wait();
+            if constexpr (EP)
+                if (p == 0 && t < K) ep_record(a, i * K + t, a.ids[i * K + t], a.expand_idx[i * K + t]);
+        }
+    }
 }
 
 }  // namespace moe

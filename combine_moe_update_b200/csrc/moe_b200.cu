@@ -277,13 +277,11 @@ struct TokenSmoothLaunch {
         auto kernel = moe::dispatch_token_smooth_kernel<MODE, NT, FUSED, EP>;
         const size_t smem = (size_t)moe::smooth_smem_floats<NT>(a.hidden) * sizeof(float);
         if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
-        if constexpr (!EP) {
-            const int P = copy_groups(a, kernel, smem);
-            if (P > 1) {
-                auto grouped = moe::dispatch_token_smooth_kernel<MODE, NT, FUSED, false, true>;
-                if (!ensure_smem(grouped, smem)) return cudaErrorInvalidValue;
-                return launch(grouped, dim3(a.bs, P), NT, smem, s, a);
-            }
+        const int P = copy_groups(a, kernel, smem);
+        if (P > 1) {
+            auto grouped = moe::dispatch_token_smooth_kernel<MODE, NT, FUSED, EP, true>;
+            if (!ensure_smem(grouped, smem)) return cudaErrorInvalidValue;
+            return launch(grouped, dim3(a.bs, P), NT, smem, s, a);
         }
         return launch(kernel, a.bs, NT, smem, s, a);
     }

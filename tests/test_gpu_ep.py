@@ -70,6 +70,23 @@ def _inputs(seed, G, bs, H, E, K, ws, smooth):
 ])
 @pytest.mark.parametrize("fused", [True, False], ids=["fused", "two_step"])
 def test_emulated_group_equals_one_gpu_dispatch(B, EP, G, bs, H, E, K, ws, mode, smooth, fused):
+    _check_group(B, EP, G, bs, H, E, K, ws, mode, smooth, fused)
+
+
+@pytest.mark.parametrize("G,bs,H,E,K,ws,mode,smooth", [
+    (2, 256, 2048, 32, 8, 8, 2, True),   # smooth scales, two copy groups per token
+    (2, 40, 1024, 16, 8, 4, 2, True),    # four copy groups per token
+    (2, 64, 1024, 16, 6, 4, 0, False),   # one quantization per token
+])
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "two_step"])
+def test_emulated_group_with_pruned_tokens(B, EP, G, bs, H, E, K, ws, mode, smooth, fused):
+    """A pruning threshold above many tokens' largest routing weight: tokens
+    with no sent copy (and copy groups with none) must still record their
+    copies' global rows as -1, so the combine sums nothing for them."""
+    _check_group(B, EP, G, bs, H, E, K, ws, mode, smooth, fused, prune=0.3, min_unsent_tokens=1)
+
+
+def _check_group(B, EP, G, bs, H, E, K, ws, mode, smooth, fused, prune=0.0, min_unsent_tokens=0):
     inp = _inputs(G * 1000 + mode, G, bs, H, E, K, ws, smooth or mode == 1)
     grp = EP.EmulatedGroup(G, fused=fused, bs=bs, hidden=H, top_k=K, num_instances=E, ep_world_size=ws,
                            quant_mode=mode)
@@ -81,14 +98,17 @@ def test_emulated_group_equals_one_gpu_dispatch(B, EP, G, bs, H, E, K, ws, mode,
     table = dev(inp["table"])
     sl = lambda a, g: np.ascontiguousarray(a[g * bs:(g + 1) * bs])
     grp.dispatch([dict(expert_ids=dev(sl(inp["ids"], g)), table=table, x=dev_bf16(sl(inp["x"], g)),
-                       expert_scales=dev(sl(inp["scales"], g)), smooth=sm) for g in range(G)])
+                       expert_scales=dev(sl(inp["scales"], g)), smooth=sm, prune_threshold=prune)
+                  for g in range(G)])
     torch.cuda.synchronize()
     for r in grp.ranks:
         assert r.device_errors() == 0
 
     # the oracle: all G * bs tokens on one device
-    bal, bm, _ = orc.update_expert(inp["ids"], inp["table"], ws, expert_scales=inp["scales"])
+    bal, bm, _ = orc.update_expert(inp["ids"], inp["table"], ws, expert_scales=inp["scales"],
+                                   prune_threshold=prune)
     od = orc.dispatch(inp["x"], bal, E, mode, mask=bm, smooth=inp["smooth"])
+    assert ((od["expand_idx"] < 0).all(axis=1)).sum() >= min_unsent_tokens
     off, El = od["offsets"], E // G
     for q, r in enumerate(grp.ranks):
         b, e_ = int(off[q * El]), int(off[(q + 1) * El])
