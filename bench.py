@@ -106,6 +106,9 @@ KERNEL_SOURCES = {
     "dispatch_token_kernel": ("dispatch.cuh", "common.cuh"),
     "gmm_kernel": ("grouped_matmul.cuh", "common.cuh"),
     "gmm_mx_kernel": ("grouped_matmul.cuh", "common.cuh"),
+    # the EP instantiations (rows stored to / read from their owners), one-GPU group
+    "dispatch_token_smooth_kernel_ep": ("dispatch.cuh", "common.cuh"),
+    "combine_token_kernel_ep": ("combine.cuh", "common.cuh"),
 }
 
 
@@ -734,10 +737,11 @@ def graph_time(body, sets, steps):
     return tot / reps
 
 
-def ep_kernel_roofline(kernel, alg_bytes, t_ms, peak, peak_kind):
+def ep_kernel_roofline(kernel, alg_bytes, t_ms, peak, peak_kind, traffic_key=None, workload=None):
     ach = alg_bytes / (t_ms * 1e-3) / 1e9
     return {"bound": "hbm", "kernel": kernel, "achieved": round(ach, 1), "peak": peak, "peak_kind": peak_kind,
-            "unit": "GB/s", "frac": round(ach / peak, 4), "launch_us": round(t_ms * 1e3, 2), "traffic": None,
+            "unit": "GB/s", "frac": round(ach / peak, 4), "launch_us": round(t_ms * 1e3, 2),
+            "traffic": stored_traffic(traffic_key, workload) if traffic_key else None,
             "algorithmic_bytes": alg_bytes,
             "timing": "launches back to back over input sets larger than twice L2, CUDA events at the graph's ends; "
                       "the dispatch's bytes include the route's outputs (about 0.1 %)"}
@@ -845,11 +849,12 @@ def run_b200_ep(args, rank, world, local_rank):
                    "exchange": "fused into dispatch and combine" if fused else "push and pull",
                    "rows_received_rank0": recv,
                    "l2": "not flushed: each step's exchange and gathers touch more than L2 across the group"},
-        "roofline": ep_kernel_roofline("combine_token_kernel (EP)", alg["combine"], t_epc, peak, peak_kind)
-        if t_epc else None,
+        "roofline": ep_kernel_roofline("combine_token_kernel (EP)", alg["combine"], t_epc, peak, peak_kind,
+                                       "combine_token_kernel_ep", args.workload) if t_epc else None,
         "roofline_other": ep_kernel_roofline("dispatch_token_smooth_kernel (EP)" if w.smooth is not None
                                              else "dispatch_token_kernel (EP)", alg["dispatch"], t_epd, peak,
-                                             peak_kind) if t_epd else None,
+                                             peak_kind, "dispatch_token_smooth_kernel_ep" if w.smooth is not None
+                                             else None, args.workload) if t_epd else None,
         "step_roofline": {"bound": "hbm", "kernel": ("whole step (update, route, plan, EP dispatch, EP combine)"
                                                      if fused else
                                                      "whole step (update, dispatch, plan, push, pull, combine)"),
