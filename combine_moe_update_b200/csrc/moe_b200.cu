@@ -382,30 +382,43 @@ cudaError_t launch_combine_tp2(const moe::CombineArgs &a, int top_k, cudaStream_
 }
 
 // The combine that gathers its rows from the GPUs that own them (one block per token).
-template <int KMAX, bool SHARED, int NT>
+template <int KMAX, bool SHARED, int NT, int SPLIT>
 cudaError_t launch_combine_ep_nt(const moe::CombineArgs &a, cudaStream_t s) {
-    auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, true, 1, true>;
-    constexpr int smem = moe::cb_smem_bytes(KMAX, NT, true, 1);
+    auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, true, SPLIT, true>;
+    constexpr int smem = moe::cb_smem_bytes(KMAX, NT, true, SPLIT);
     if (!ensure_smem(kernel, smem)) return cudaErrorInvalidValue;
-    return launch(kernel, a.bs, NT, smem, s, a);
+    return launch_in_clusters(kernel, a.bs * SPLIT, NT, smem, s, SPLIT, a);
 }
 
-template <int KMAX, bool SHARED>
+template <int KMAX, bool SHARED, int SPLIT>
 cudaError_t launch_combine_ep_tok(const moe::CombineArgs &a, cudaStream_t s) {
-    switch (moe::cb_threads(a.hidden >> 3, 4)) {
-        case 64: return launch_combine_ep_nt<KMAX, SHARED, 64>(a, s);
-        case 128: return launch_combine_ep_nt<KMAX, SHARED, 128>(a, s);
-        case 192: return launch_combine_ep_nt<KMAX, SHARED, 192>(a, s);
-        case 224: return launch_combine_ep_nt<KMAX, SHARED, 224>(a, s);
-        default: return launch_combine_ep_nt<KMAX, SHARED, 256>(a, s);
+    constexpr int VECS = SPLIT == 1 ? 4 : 2;
+    switch (moe::cb_threads((a.hidden >> 3) / SPLIT, VECS)) {
+        case 64: return launch_combine_ep_nt<KMAX, SHARED, 64, SPLIT>(a, s);
+        case 128: return launch_combine_ep_nt<KMAX, SHARED, 128, SPLIT>(a, s);
+        case 192: return launch_combine_ep_nt<KMAX, SHARED, 192, SPLIT>(a, s);
+        case 224: return launch_combine_ep_nt<KMAX, SHARED, 224, SPLIT>(a, s);
+        default: return launch_combine_ep_nt<KMAX, SHARED, 256, SPLIT>(a, s);
     }
 }
 
-cudaError_t launch_combine_ep(const moe::CombineArgs &a, int top_k, cudaStream_t s) {
+// The EP combine splits rows over clusters by the same rule as the one-GPU
+// combine (launch_combine_split): the peers' rows are plain loads, and the
+// sums of squares meet in this GPU's distributed shared memory.
+template <int KMAX>
+cudaError_t launch_combine_ep_k(const moe::CombineArgs &a, cudaStream_t s) {
+    const int sms = device_sms();
+    const int split = a.bs < sms && (a.hidden >> 3) % 4 == 0 ? 4 : a.bs < 2 * sms ? 2 : 1;
     const bool sh = a.shared_x != nullptr;
-    if (top_k <= 4) return sh ? launch_combine_ep_tok<4, true>(a, s) : launch_combine_ep_tok<4, false>(a, s);
-    if (top_k <= 8) return sh ? launch_combine_ep_tok<8, true>(a, s) : launch_combine_ep_tok<8, false>(a, s);
-    return sh ? launch_combine_ep_tok<16, true>(a, s) : launch_combine_ep_tok<16, false>(a, s);
+    if (split == 4) return sh ? launch_combine_ep_tok<KMAX, true, 4>(a, s) : launch_combine_ep_tok<KMAX, false, 4>(a, s);
+    if (split == 2) return sh ? launch_combine_ep_tok<KMAX, true, 2>(a, s) : launch_combine_ep_tok<KMAX, false, 2>(a, s);
+    return sh ? launch_combine_ep_tok<KMAX, true, 1>(a, s) : launch_combine_ep_tok<KMAX, false, 1>(a, s);
+}
+
+cudaError_t launch_combine_ep(const moe::CombineArgs &a, int top_k, cudaStream_t s) {
+    if (top_k <= 4) return launch_combine_ep_k<4>(a, s);
+    if (top_k <= 8) return launch_combine_ep_k<8>(a, s);
+    return launch_combine_ep_k<16>(a, s);
 }
 
 template <bool NORM>
