@@ -381,7 +381,7 @@ cudaError_t launch_combine_tp2(const moe::CombineArgs &a, int top_k, cudaStream_
     return sh ? launch_combine_tp2_tok<16, true>(a, s) : launch_combine_tp2_tok<16, false>(a, s);
 }
 
-// The combine that gathers its rows from the GPUs that own them (one block per token).
+// The combine that gathers its rows from the GPUs that own them.
 template <int KMAX, bool SHARED, int NT, int SPLIT>
 cudaError_t launch_combine_ep_nt(const moe::CombineArgs &a, cudaStream_t s) {
     auto kernel = moe::combine_token_kernel<KMAX, SHARED, NT, true, SPLIT, true>;
