@@ -811,8 +811,12 @@ template <int MODE, int NT, bool FUSED, bool EP = false>
 __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
     static_assert(!(FUSED && EP), "an EP scatter follows an earlier route call");
     __shared__ float s_red[NT / 32];
-    __shared__ int s_row[16], s_inst[EP ? 16 : 1];
+    __shared__ int s_row[16];
     __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
+    // EP: copy k's destination in its owner's receive buffer (row -1: none),
+    // resolved once per token rather than by every thread at every copy
+    __shared__ uint8_t *s_dx[EP ? 16 : 1], *s_dsc[EP ? 16 : 1];
+    __shared__ int s_drow[EP ? 16 : 1];
     const int i = blockIdx.x, t = threadIdx.x;
     const int H = a.hidden, V = H >> 3, K = a.top_k;
     if constexpr (FUSED) {
@@ -883,8 +887,13 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
             const int r = a.expand_idx[i * K + t];
             s_row[t] = r;
             if constexpr (EP) {
-                s_inst[t] = a.ids[i * K + t];
-                ep_record(a, i * K + t, s_inst[t], r);
+                const int e = a.ids[i * K + t];
+                ep_record(a, i * K + t, e, r);
+                RowDst d{nullptr, nullptr, -1};
+                const bool ok = r >= 0 && copy_dst<true>(a, e, r, d);  // r >= 0: e is in range
+                s_dx[t] = d.x;
+                s_dsc[t] = d.sc;
+                s_drow[t] = ok ? d.row : -1;
             }
         }
         __syncthreads();
@@ -893,7 +902,14 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         const int row = FUSED ? rs.row[k] : s_row[k];
         if (row < 0) continue;
         RowDst d;
-        if (!copy_dst<EP>(a, EP ? s_inst[k] : 0, row, d)) continue;
+        if constexpr (EP) {
+            d.x = s_dx[k];
+            d.sc = s_dsc[k];
+            d.row = s_drow[k];
+            if (d.row < 0) continue;
+        } else {
+            copy_dst<false>(a, 0, row, d);
+        }
         if constexpr (MODE == 0) {
             uint16_t *dst = reinterpret_cast<uint16_t *>(d.x) + (size_t)d.row * H;
 #pragma unroll
@@ -944,6 +960,10 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_key[16], s_pos[16], s_row[16], s_ns;
     __shared__ RouteSmemT<FUSED ? kMaxInstances : 1> rs;
+    // EP: copy k's destination in its owner's receive buffer (row -1: none),
+    // resolved once per token rather than by every thread at every copy
+    __shared__ uint8_t *s_dx[EP ? 16 : 1], *s_dsc[EP ? 16 : 1];
+    __shared__ int s_drow[EP ? 16 : 1];
     const int i = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int P = GROUPS ? (int)gridDim.y : 1, p = GROUPS ? (int)blockIdx.y : 0;  // copy group p of the token's P
     const int H = a.hidden, V = H >> 3, K = a.top_k;
@@ -1050,8 +1070,15 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
             if (t < K) {
                 const int r = a.expand_idx[i * K + t];
                 s_row[t] = r;
-                if constexpr (EP)
-                    if (p == 0) ep_record(a, i * K + t, a.ids[i * K + t], r);  // once per token
+                if constexpr (EP) {
+                    const int e = a.ids[i * K + t];
+                    if (p == 0) ep_record(a, i * K + t, e, r);  // once per token
+                    RowDst d{nullptr, nullptr, -1};
+                    const bool ok = r >= 0 && copy_dst<true>(a, e, r, d);  // r >= 0: e is in range
+                    s_dx[t] = d.x;
+                    s_dsc[t] = d.sc;
+                    s_drow[t] = ok ? d.row : -1;
+                }
             }
             __syncthreads();
         }
@@ -1059,8 +1086,17 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         for (int q = 0; q < kDpVecs; ++q)
             if (swap) qv[q] = make_uint2(qv[q].y, qv[q].x);
         RowDst d;
-        if (copy_dst<EP>(a, s_key[c], FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], d))
-            write_row<MODE, NT>(a, d, V, qv, seg, row_scale);
+        bool ok;
+        if constexpr (EP) {
+            const int k = s_pos[c];
+            d.x = s_dx[k];
+            d.sc = s_dsc[k];
+            d.row = s_drow[k];
+            ok = d.row >= 0;
+        } else {
+            ok = copy_dst<false>(a, s_key[c], FUSED ? rs.row[s_pos[c]] : s_row[s_pos[c]], d);
+        }
+        if (ok) write_row<MODE, NT>(a, d, V, qv, seg, row_scale);
     }
     // A block with no copy still waits for the route kernel, so that this
     // grid ends after it: the next call reads the rows and counts it wrote.
