@@ -44,6 +44,9 @@ struct CombineArgs {
     const uint16_t *expand_x1;
 };
 
+// The most GPUs in an EP group (the header's MOE_EP_MAX_GPUS).
+constexpr int kCbMaxGpus = 64;
+
 // K 16 with the norm keeps the pre-norm row in shared memory (XS) and runs
 // four blocks per SM; otherwise four blocks up to 224 threads, three beyond.
 __host__ __device__ constexpr bool cb_xs(int kmax, bool norm) { return norm && kmax == 16; }
@@ -88,6 +91,11 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
     __shared__ int s_row[16];
     __shared__ float s_w[16];
     __shared__ const uint16_t *s_src[EP ? 16 : 1];
+    // EP: the group's row bases and output buffers, staged once per block so
+    // the owner search reads shared memory instead of a chain of dependent
+    // global loads
+    __shared__ int s_gbase[EP ? kCbMaxGpus + 1 : 1];
+    __shared__ const uint16_t *s_peer[EP ? kCbMaxGpus : 1];
     __shared__ int s_nk;
     __shared__ float s_red[NW];
     __shared__ float s_part;
@@ -102,13 +110,24 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
         if constexpr (SHARED) prefetch_l2(a.shared_x + off, bytes);
     }
     pdl_wait();  // expand_idx and the expert rows come from earlier kernels
+    int row0 = -1;
+    float w0 = 0.0f;
+    if (t < K) {  // issued before the EP tables' loads, so they are in flight together
+        row0 = a.expand_idx[i * K + t];
+        w0 = a.scales[i * K + t];
+    }
+    if constexpr (EP) {
+        for (int q = t; q <= a.gpus; q += NT) {
+            s_gbase[q] = a.gbase[q];
+            if (q < a.gpus) s_peer[q] = a.peer_rows[q];
+        }
+        __syncthreads();
+    }
     if (t < 32) {  // warp 0: the kept copies, compacted in k order (a pruned copy adds nothing)
-        int row = -1;
-        float w = 0.0f;
+        int row = row0;
+        const float w = w0;
         const uint16_t *src = nullptr;
         if (t < K) {
-            row = a.expand_idx[i * K + t];
-            w = a.scales[i * K + t];
             if (row < -1 || row >= a.expand_rows) {
                 raise_error(a.err, kDevBadId);
                 row = -1;
@@ -118,14 +137,14 @@ __global__ void __launch_bounds__(NT, cb_min_blocks(KMAX, NT, NORM)) combine_tok
                     int lo = 0, hi = a.gpus - 1;
                     while (lo < hi) {
                         const int mid = (lo + hi + 1) >> 1;
-                        if (a.gbase[mid] <= row) lo = mid; else hi = mid - 1;
+                        if (s_gbase[mid] <= row) lo = mid; else hi = mid - 1;
                     }
-                    const int prow = row - a.gbase[lo];
-                    if (prow >= a.recv_rows || row >= a.gbase[a.gpus]) {
+                    const int prow = row - s_gbase[lo];
+                    if (prow >= a.recv_rows || row >= s_gbase[a.gpus]) {
                         raise_error(a.err, kDevBadId);
                         row = -1;
                     } else {
-                        src = a.peer_rows[lo] + (size_t)prow * H;
+                        src = s_peer[lo] + (size_t)prow * H;
                     }
                 }
             }

@@ -913,6 +913,7 @@ namespace {
 
 bool valid_ep(const moe_ep_params &p) {
     if (p.bs < 1 || p.bs > MOE_MAX_BS || p.top_k < 1 || p.top_k > MOE_MAX_TOP_K) return false;
+    static_assert(moe::kCbMaxGpus == MOE_EP_MAX_GPUS, "the combine stages every GPU's row base");
     if (p.gpus < 1 || p.gpus > MOE_EP_MAX_GPUS || p.rank < 0 || p.rank >= p.gpus) return false;
     if (p.num_instances < 1 || p.num_instances > MOE_MAX_EXPERTS || p.num_instances % p.gpus != 0) return false;
     if (p.row_bytes < 16 || p.row_bytes % 16 != 0 || p.row_bytes > 2 * MOE_MAX_HIDDEN) return false;
