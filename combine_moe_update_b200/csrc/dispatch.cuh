@@ -825,8 +825,10 @@ __global__ void __launch_bounds__(NT) dispatch_token_kernel(DispatchArgs a) {
         // read before the wait.  The x loads issued right after it stay in
         // flight while the block routes its copies.
         block_route_clear<NT>(rs, a.num_instances);
+        if (t == 0) prefetch_l2(a.x + (size_t)i * H, (uint32_t)H * 2u);  // the token row, while the predecessor drains
         pdl_wait();
     } else if constexpr (EP) {
+        if (t == 0) prefetch_l2(a.x + (size_t)i * H, (uint32_t)H * 2u);
         pdl_wait();
     }
 
@@ -980,10 +982,14 @@ __global__ void __launch_bounds__(NT, NT <= 224 ? 4 : 3) dispatch_token_smooth_k
         // The call's first kernel: x, the ids and the scales may all come
         // from the kernel before it, so nothing is read before the wait.
         block_route_clear<NT>(rs, a.num_instances);
-        if (t == 0) mbar_init(&s_bar, 1);
+        if (t == 0) {
+            mbar_init(&s_bar, 1);
+            prefetch_l2(a.x + (size_t)i * H, (uint32_t)H * 2u);  // the token row, while the predecessor drains
+        }
         __syncthreads();
         pdl_wait();
     } else if constexpr (EP) {
+        if (t == 0) prefetch_l2(a.x + (size_t)i * H, (uint32_t)H * 2u);
         pdl_wait();  // the call's first kernel (routed by an earlier call)
     }
     // FUSED: after the wait.  Otherwise the call's route kernel runs first
